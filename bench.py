@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the vision-to-language projector on B200.
+
+One step = one whole pass of the bridge (placeholder index, geometry, LayerNorm,
+GEMM1 with the merge-gather prologue, GEMM2 with the scatter epilogue, newline /
+separator rows) over one batch of the chosen workload, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). Timing: W untimed warm-up steps; then K steps, each
+bracketed by CUDA events on the launching stream, with a 256 MiB write between steps
+to flush L2 (outside the events); barrier + synchronize on both sides of the timed
+region; max over ranks. Multi-GPU (torchrun): every rank projects its own replica
+batch (weak scaling); there is no collective on the data path.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (rank 0
+only), on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "projected image tokens/s on 1 B200; % of dense BF16 tensor peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "moonvit"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["vision_language_projector_b200/csrc/gemm_sm100.cuh", "vision_language_projector_b200/csrc/ptx.cuh",
+                  "vision_language_projector_b200/csrc/kernels_aux.cuh", "vision_language_projector_b200/csrc/vlproj.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def workload_geometry(wl, seed):
+    import vision_language_projector_b200 as vp
+    hw = W.grid_hw(wl, seed)
+    crop = W.spatial_crop(wl)
+    cfg = vp.make_config(wl.k, wl.C, wl.N1, wl.N2, has_ln=wl.has_ln,
+                         tile_tag=vp.TILE_2D if wl.tiled else vp.TILE_NONE)
+    rows = vp.image_rows(cfg, hw, crop, wl.n_images)      # the library's own closed form
+    return hw, crop, rows
+
+
+def merged_tokens(wl, hw) -> int:
+    k = wl.k
+    return int(sum(((int(h) + k - 1) // k) * ((int(w) + k - 1) // k) for h, w in hw))
+
+
+def flops_per_token(wl) -> int:
+    return 2 * (wl.K1 * wl.N1 + wl.N1 * wl.N2)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling of one GPU during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, enabled: bool = True):
+        self.proc = None
+        self.gpu = gpu_index
+        if not enabled:
+            return
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, hw, crop, w, seed, budget_s: float, start_image: int = 0, max_images=None):
+    """Time the fp64 oracle on whole images, in order from start_image, until budget_s is
+    spent (at least one image). Returns (tokens, seconds, images)."""
+    from oracle import projector as O
+    params = O.params_f64(w)
+    per = wl.views_per_image
+    tokens, elapsed, n = 0, 0.0, 0
+    img = start_image
+    while True:
+        views = list(range(img * per, (img + 1) * per))
+        fe = W.features(wl, hw, seed, views=views, threads=1)
+        offs = np.concatenate([[0], np.cumsum([int(hw[v, 0]) * int(hw[v, 1]) for v in views])])
+        feats = [(fe[offs[i]:offs[i + 1]].astype(np.float64) if wl.feat_fp32 else
+                  O.bf16_bits_to_f64(fe[offs[i]:offs[i + 1]])) for i in range(len(views))]
+        vhw = [(int(hw[v, 0]), int(hw[v, 1])) for v in views]
+        c = None if crop is None else (int(crop[img, 0]), int(crop[img, 1]))
+        t0 = time.perf_counter()
+        O.project_image(feats, vhw, wl.k, params, c, wl.ln_eps)
+        elapsed += time.perf_counter() - t0
+        tokens += sum(((h + wl.k - 1) // wl.k) * ((ww + wl.k - 1) // wl.k) for h, ww in vhw)
+        n += 1
+        img = (img + 1) % wl.n_images
+        if elapsed >= budget_s or (max_images is not None and n >= max_images):
+            break
+    return tokens, elapsed, n
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return int(max(i.get("num_threads", 1) for i in info))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    hw = W.grid_hw(wl, args.seed)
+    crop = W.spatial_crop(wl)
+    w = W.weights(wl, args.seed)
+    # one step = the oracle on whole images of the workload, about a few seconds each
+    budget = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    img = 0
+    for _ in range(args.warmup):
+        _, _, n = oracle_sample(wl, hw, crop, w, args.seed, budget, img, max_images=1)
+        img = (img + n) % wl.n_images
+    tok, sec = 0, 0.0
+    for _ in range(args.steps):
+        t, s, n = oracle_sample(wl, hw, crop, w, args.seed, budget, img)
+        tok += t
+        sec += s
+        img = (img + n) % wl.n_images
+    value = tok / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * sec / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample": "whole images of the workload per step, fp64 numpy oracle"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{tok} merged tokens over {args.steps} steps of whole images"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import vision_language_projector_b200 as vp
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    wl = W.WORKLOADS[args.workload]
+    seed = args.seed + rank
+    hw, crop, rows = workload_geometry(wl, seed)
+    M = merged_tokens(wl, hw)
+    wts = W.weights(wl, seed)
+    feats_h = W.features(wl, hw, seed, threads=min(16, os.cpu_count() or 1))
+    ids_h = W.input_ids(wl, rows, seed)
+    prefill_h = W.prefill_embeds(wl, ids_h, W.embed_table(wl, seed))
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+    def f32(a):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+    proj = vp.Projector(wl.k, wl.C, wl.N1, wl.N2, bf(wts["W1"]), bf(wts["W2"]), f32(wts["b1"]), f32(wts["b2"]),
+                        has_ln=wl.has_ln, ln_gamma=f32(wts["gamma"]), ln_beta=f32(wts["beta"]), ln_eps=wl.ln_eps,
+                        feat_dtype=vp.FEAT_F32 if wl.feat_fp32 else vp.FEAT_BF16,
+                        tile_tag=vp.TILE_2D if wl.tiled else vp.TILE_NONE)
+    feats = f32(feats_h) if wl.feat_fp32 else bf(feats_h)
+    ids = torch.from_numpy(ids_h).cuda()
+    prefill = bf(prefill_h)
+    out = prefill.clone()
+    newline = bf(wts["newline"]) if wl.tiled else None
+    sep = bf(wts["sep"]) if wl.tiled else None
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        proj.forward(feats, hw, crop, ids, W.IMAGE_TOKEN_ID, out, newline, sep, stream=stream, n_images=wl.n_images)
+
+    proj.profile(True)
+    for _ in range(max(3, args.warmup)):
+        step()
+    st = proj.status()
+    if st != vp.OK:
+        raise SystemExit(f"warm-up failed: {vp.strerror(st)}")
+
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local, not args.no_clocks)
+    launches0 = proj.launch_count()
+    step_ms, stage_acc = [], {}
+    for _ in range(args.steps):
+        flush.zero_()                      # L2 flush between steps, outside the events
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+        for k_, v in proj.stage_ms().items():
+            stage_acc.setdefault(k_, []).append(v)
+    launches = proj.launch_count() - launches0
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    st = proj.status()
+    if st != vp.OK:
+        raise SystemExit(f"timed steps failed: {vp.strerror(st)}")
+
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    tokens_per_step = M
+    value = world * tokens_per_step * args.steps / (total_ms / 1000.0)
+    ms_per_step = total_ms / args.steps
+    fl_tok = flops_per_token(wl)
+    tflops = value * fl_tok / 1e12 / world
+
+    # ---- roofline of the dominant kernel (largest average stage time)
+    peaks, peak_src = load_peaks()
+    avg = {k_: statistics.mean(v) for k_, v in stage_acc.items()}
+    dom = max(avg, key=avg.get)
+    sustained = total_ms > 2000.0
+    peak_tf = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
+    if dom in ("gemm1", "gemm2"):
+        fl = 2.0 * M * (wl.K1 * wl.N1 if dom == "gemm1" else wl.N1 * wl.N2)
+        achieved = fl / (avg[dom] / 1000.0) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved / peak_tf,
+                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'}",
+                "traffic": traffic_from_profiles(args.workload, dom)}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
+                "frac": None, "peak_source": peak_src, "traffic": None}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        feats_p = (torch.from_numpy(feats_h) if wl.feat_fp32 else torch.from_numpy(feats_h.view(np.int16))).pin_memory()
+        ids_p = torch.from_numpy(ids_h).pin_memory()
+        pre_p = torch.from_numpy(prefill_h.view(np.int16)).pin_memory()
+        res_p = torch.empty_like(pre_p).pin_memory()
+        feats_d = torch.empty(feats_p.shape, dtype=feats_p.dtype, device="cuda")
+        ids_d = torch.empty_like(ids)
+        out_d = torch.empty(pre_p.shape, dtype=torch.int16, device="cuda")
+
+        def e2e_step():
+            feats_d.copy_(feats_p, non_blocking=True)
+            ids_d.copy_(ids_p, non_blocking=True)
+            out_d.copy_(pre_p, non_blocking=True)
+            f = feats_d if wl.feat_fp32 else feats_d.view(torch.bfloat16)
+            proj.forward(f, hw, crop, ids_d, W.IMAGE_TOKEN_ID, out_d.view(torch.bfloat16), newline, sep,
+                         stream=stream, n_images=wl.n_images)
+            res_p.copy_(out_d, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_ms = 0.0
+        for _ in range(args.e2e_steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+            b.synchronize()
+            e_ms += a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        st = proj.status()
+        if st != vp.OK:
+            raise SystemExit(f"e2e steps failed: {vp.strerror(st)}")
+        e2e = {"value": world * tokens_per_step * args.e2e_steps / (e_ms / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": int(feats_p.numel() * feats_p.element_size() + ids_p.numel() * 8 +
+                                         pre_p.numel() * 2),
+               "d2h_bytes_per_step": int(res_p.numel() * 2), "steps": args.e2e_steps}
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok, sec, n = oracle_sample(wl, hw, crop, wts, seed, args.cpu_seconds)
+        cpu = {"value": tok / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{n} whole image(s) of the workload, {tok} merged tokens, fp64 numpy, {sec:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "images": wl.n_images, "merged_tokens": M,
+                       "assembled_rows": int(sum(rows)), "K1": wl.K1, "N1": wl.N1, "N2": wl.N2, "k": wl.k,
+                       "layernorm": wl.has_ln, "tiling": "2D" if wl.tiled else "none",
+                       "sequences": f"{wl.B}x{wl.S}", "l2": "flushed between steps (256 MiB write)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "tflops_per_gpu": tflops,
+            "pct_of_dense_bf16_peak": 100.0 * tflops / peaks.get("bf16_tflops"),
+            "pct_of_datasheet_2250_tflops": 100.0 * tflops / 2250.0,
+            "stage_ms": avg,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    proj.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

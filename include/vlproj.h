@@ -1,0 +1,181 @@
+/*
+ * vlproj - vision-to-language projector for NVIDIA B200 (sm_100a).
+ *
+ * The bridge between a vision tower and a language model's embedding
+ * sequence, as described on the pages studied for this library:
+ *
+ *   1. space-to-depth: each k x k neighbourhood of a view's patch grid becomes
+ *      one token of k*k*C features, grid zero-padded at the high end to a
+ *      multiple of k, features ordered channel-outermost c*k*k + dy*k + dx
+ *      ("port DeepSeek-VL2", Projector (downsample_mlp_gelu) steps 1-2;
+ *      "La voie visuelle", section "Le pixel-unshuffle 3x3");
+ *   2. optional pre-merge LayerNorm over each patch's C features (the MoonViT
+ *      PatchMerger: "DeepSeek-V4-Flash-Vision-BF16", first section);
+ *   3. Linear -> GELU -> Linear, weights stored (out, in)
+ *      ("port DeepSeek-VL2", Projector step 3 and Safetensors weight keys);
+ *   4. for tile tag "2D": global view rows each closed by a learned newline,
+ *      one view separator, then the local tiles laid side by side, rows closed
+ *      by a newline ("port DeepSeek-VL2", Tile-sequence assembly);
+ *   5. the assembled rows overwrite the embedding rows that hold the image
+ *      placeholder id, in order ("port DeepSeek-VL2", end of Tile-sequence
+ *      assembly; image_token_index 100015).
+ *
+ * Number formats: bf16 operands, fp32 accumulation, bf16 hidden activation
+ * and bf16 output rows. Everything below runs on the GPU; there is no CPU path.
+ *
+ * Conventions
+ *   - Every call returns a vlproj status code (>= 0 success, < 0 error) unless
+ *     stated otherwise. Errors found on the host return before any launch and
+ *     leave every buffer untouched.
+ *   - Device pointers are raw CUDA device addresses; host pointers are plain
+ *     CPU memory. The library never takes ownership of a caller's buffer.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Work is enqueued asynchronously; the caller keeps every
+ *     borrowed device buffer alive until that stream's work completes.
+ *   - A handle is bound to the device that was current at vlproj_create and
+ *     is not thread-safe: one thread at a time per handle.
+ */
+#ifndef VLPROJ_H
+#define VLPROJ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define VLPROJ_OK                 0
+#define VLPROJ_ERR_INVALID_ARG   (-1) /* bad pointer, size, shape or layout */
+#define VLPROJ_ERR_UNSUPPORTED   (-2) /* projector variant the library does not build (the
+                                         pages ask for a loud error on these: tile tag "1D",
+                                         token pooling, another projector type) */
+#define VLPROJ_ERR_CUDA          (-3) /* a CUDA runtime/driver call failed */
+#define VLPROJ_ERR_TOKEN_COUNT   (-4) /* device found: placeholder count != assembled rows;
+                                         nothing was written to out_embeds */
+#define VLPROJ_ERR_TIMEOUT       (-5) /* device found: a bounded wait inside a kernel ran out */
+
+/* ---- configuration ----------------------------------------------------- */
+enum { VLPROJ_FEAT_BF16 = 0, VLPROJ_FEAT_F32 = 1 };
+enum { VLPROJ_TILE_NONE = 0, VLPROJ_TILE_2D = 1, VLPROJ_TILE_1D = 2 /* rejected */ };
+enum { VLPROJ_GLOBAL_HEAD = 0, VLPROJ_GLOBAL_TAIL = 1 };
+enum { VLPROJ_ORDER_CHANNEL_OUTER = 0,   /* W1 input index c*k*k + dy*k + dx (the pages' order) */
+       VLPROJ_ORDER_POSITION_OUTER = 1 }; /* W1 input index (dy*k + dx)*C + c */
+
+typedef struct vlproj_config {
+    int32_t k;              /* merge factor: 1, 2 or 3 */
+    int32_t C;              /* vision feature width; multiple of 64 */
+    int32_t N1;             /* MLP hidden width; multiple of 64 */
+    int32_t N2;             /* output embedding width (n_embed); multiple of 32 */
+    int32_t depth;          /* number of Linear layers; must be 2 */
+    int32_t has_ln;         /* 1: pre-merge LayerNorm over C, biased variance */
+    float   ln_eps;         /* LayerNorm epsilon (1e-5 when <= 0) */
+    int32_t feat_dtype;     /* VLPROJ_FEAT_BF16 or VLPROJ_FEAT_F32 features */
+    int32_t k_order;        /* column order of W1 as passed (see enum) */
+    int32_t tile_tag;       /* VLPROJ_TILE_NONE or VLPROJ_TILE_2D */
+    int32_t global_view_pos;/* VLPROJ_GLOBAL_HEAD or VLPROJ_GLOBAL_TAIL (2D tiling) */
+    int32_t token_pooling;  /* must be 0 */
+    /* Parameters, all DEVICE pointers, read once by vlproj_create (which copies
+     * them into storage the handle owns and synchronises, so the caller may free
+     * its buffers when create returns). */
+    const void*  W1;        /* bf16 [N1][k*k*C], stored (out, in) */
+    const float* b1;        /* fp32 [N1], or NULL for zeros */
+    const void*  W2;        /* bf16 [N2][N1], stored (out, in) */
+    const float* b2;        /* fp32 [N2], or NULL for zeros */
+    const float* ln_gamma;  /* fp32 [C] when has_ln, else ignored */
+    const float* ln_beta;   /* fp32 [C] when has_ln, else ignored */
+} vlproj_config;
+
+typedef struct vlproj_handle vlproj_handle;
+
+/* Create a projector on the current device. Validates cfg (VLPROJ_ERR_UNSUPPORTED
+ * for depth != 2, tile tag "1D", token pooling, k outside 1..3; INVALID_ARG for
+ * widths that break the alignment rules above or NULL weights), allocates the
+ * owned weight copies and permutes W1's columns into the kernel's gather order
+ * (an exact permutation of bf16 values). On success *out holds the handle. */
+int vlproj_create(const vlproj_config* cfg, vlproj_handle** out);
+
+/* Run the whole bridge for one batch, asynchronously on `stream`.
+ *   features     DEVICE, packed channel-last patch features of every view, views
+ *                back to back: view v holds grid_hw[v][0]*grid_hw[v][1] rows of C
+ *                values (bf16 or fp32 per cfg), rows row-major over (h, w).
+ *                For 2D tiling the views of an image are [global, local tiles
+ *                row-major]; all views of one image share one grid.
+ *   grid_hw      HOST, int32 [n_views][2] = (h, w) per view; n_views = n_images
+ *                untiled, sum(1 + tw*th) when tiled.
+ *   spatial_crop HOST, int32 [n_images][2] = (tw, th) per image (width count
+ *                first), or NULL when cfg.tile_tag == VLPROJ_TILE_NONE.
+ *   n_images     number of images (0 = text only: the call only checks that no
+ *                placeholder is present).
+ *   input_ids    DEVICE, int64 [n_ids], all sequences flattened (B*S).
+ *   image_token_id  the placeholder id (100015 in the DeepSeek-VL family).
+ *   newline, sep DEVICE, bf16 [N2] each when tiled, else ignored (may be NULL).
+ *   out_embeds   DEVICE, bf16 [n_ids][N2], in/out: only placeholder rows are
+ *                written; every other row is left as it was.
+ * Image i's rows go to the placeholders in order: the j-th placeholder over the
+ * flattened ids receives assembled row j. The placeholder count is checked on the
+ * device against the closed-form row count; on mismatch nothing is written and
+ * VLPROJ_ERR_TOKEN_COUNT is latched (see vlproj_status). */
+int vlproj_forward(vlproj_handle* h,
+                   const void* features,
+                   const int32_t* grid_hw,
+                   const int32_t* spatial_crop,
+                   int32_t n_images,
+                   const int64_t* input_ids, int64_t n_ids,
+                   int64_t image_token_id,
+                   const void* newline, const void* sep,
+                   void* out_embeds,
+                   void* stream);
+
+/* Stage output for inspection: the bf16 hidden activation H = GELU(A W1^T + b1)
+ * of every merged token, views in order, tokens row-major inside a view.
+ * hidden is DEVICE bf16 [M][N1], M = sum over views of ceil(h/k)*ceil(w/k). */
+int vlproj_hidden(vlproj_handle* h, const void* features, const int32_t* grid_hw,
+                  int32_t n_views, void* hidden, void* stream);
+
+/* Synchronise `stream`, then return the first device-found error latched since the
+ * last call (VLPROJ_OK if none) and clear it. */
+int vlproj_status(vlproj_handle* h, void* stream);
+
+/* Free the handle and everything it owns (synchronises its device first). NULL is a no-op. */
+void vlproj_destroy(vlproj_handle* h);
+
+/* Host only, no device work: closed-form placeholder count of each image
+ * (untiled: ceil(h/k)*ceil(w/k); 2D: h'(w'+1) + 1 + (th h')(tw w'+1), from
+ * "port DeepSeek-VL2", Processor step 7). Writes rows_out[n_images] when not
+ * NULL and returns the total (>= 0) or an error code (< 0). */
+int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
+                          const int32_t* spatial_crop, int32_t n_images, int64_t* rows_out);
+
+/* Bound (nanoseconds) on every wait inside this handle's kernels; 0 restores the
+ * default (2 s). A wait that runs out ends its kernel early with
+ * VLPROJ_ERR_TIMEOUT latched; tests use a tiny bound to exercise that path. */
+int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns);
+
+/* ---- tracing ------------------------------------------------------------
+ * Stage timing with CUDA events recorded on the launching stream around each
+ * kernel of vlproj_forward. Stages, in order:
+ *   0 placeholder index, 1 geometry, 2 LayerNorm/convert, 3 GEMM1 (merge + MLP
+ *   first layer + GELU), 4 GEMM2 (second layer + scatter), 5 newline/separator rows.
+ * Off by default; enabling adds seven event records per forward. */
+#define VLPROJ_NUM_STAGES 6
+int vlproj_profile_enable(vlproj_handle* h, int enable);
+
+/* Synchronise the stream of the most recent profiled forward and write the elapsed
+ * milliseconds of each stage into ms[0 .. min(n, VLPROJ_NUM_STAGES)); a stage that did
+ * not run reads 0. Returns the number of values written, or an error code. */
+int vlproj_profile_read(vlproj_handle* h, float* ms, int n);
+
+/* Number of kernels this handle has launched since it was created (all entry points). */
+int64_t vlproj_launch_count(vlproj_handle* h);
+
+/* Human-readable name of a status code (static string). */
+const char* vlproj_strerror(int code);
+
+/* Library version string, e.g. "vlproj 0.1 sm_100a". */
+const char* vlproj_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VLPROJ_H */

@@ -130,16 +130,18 @@ def fold(a: np.ndarray, hp: int, wp: int, k: int, C: int) -> np.ndarray:
     return blocks.reshape(hp * k, wp * k, C)
 
 
+def hidden(a: np.ndarray, W1: np.ndarray, b1: np.ndarray, quantise_hidden: bool = True) -> np.ndarray:
+    """First Linear and GELU: GELU(a W1^T + b1), W1 stored (out, in) and used as-is
+    ("port DeepSeek-VL2", Projector step 3; Safetensors weight keys: Linear weights
+    are consumed as stored). Rounded to bf16 (Q2) unless disabled."""
+    g = gelu(a @ W1.T + b1)
+    return round_bf16(g) if quantise_hidden else g
+
+
 def mlp(a: np.ndarray, W1: np.ndarray, b1: np.ndarray, W2: np.ndarray, b2: np.ndarray,
         quantise_hidden: bool = True) -> np.ndarray:
-    """Linear -> GELU -> Linear with weights stored (out, in) and used as-is
-    ("port DeepSeek-VL2", Projector step 3 and the note that Linear weights are
-    consumed as stored). The GELU output is rounded to bf16 (Q2) unless disabled."""
-    h = a @ W1.T + b1
-    g = gelu(h)
-    if quantise_hidden:
-        g = round_bf16(g)
-    return g @ W2.T + b2
+    """Linear -> GELU -> Linear ("port DeepSeek-VL2", Projector step 3)."""
+    return hidden(a, W1, b1, quantise_hidden) @ W2.T + b2
 
 
 def merge_view(feat: np.ndarray, h: int, w: int, k: int, ln: Optional[tuple]) -> np.ndarray:
@@ -194,7 +196,7 @@ def scatter(embeds: np.ndarray, ids: np.ndarray, image_token_id: int, rows: np.n
 # ----------------------------------------------------------------- whole path
 def project_image(feats: Sequence[np.ndarray], hw: Sequence[tuple], k: int, params: dict,
                   crop: Optional[tuple], ln_eps: float = 1e-5,
-                  quantise: bool = True) -> np.ndarray:
+                  quantise: bool = True, global_view_pos: str = "head") -> np.ndarray:
     """Assembled rows of one image. ``feats[v]`` is view v's (h*w, C) features as fp64.
     ``params`` holds fp64 W1, b1, W2, b2 and optionally gamma, beta, newline, sep."""
     ln = None
@@ -215,12 +217,13 @@ def project_image(feats: Sequence[np.ndarray], hw: Sequence[tuple], k: int, para
         return outs[0]
     tw, th = crop
     hp, wp = merged_side(hw[0][0], k), merged_side(hw[0][1], k)
-    return assemble_2d(np.stack(outs), hp, wp, tw, th, params["newline"], params["sep"])
+    return assemble_2d(np.stack(outs), hp, wp, tw, th, params["newline"], params["sep"], global_view_pos)
 
 
 def forward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[np.ndarray],
             k: int, params: dict, ids: np.ndarray, image_token_id: int, embeds: np.ndarray,
-            ln_eps: float = 1e-5, feat_is_bf16_bits: bool = True, quantise: bool = True) -> np.ndarray:
+            ln_eps: float = 1e-5, feat_is_bf16_bits: bool = True, quantise: bool = True,
+            global_view_pos: str = "head") -> np.ndarray:
     """The whole bridge: per image, merge + MLP (+ assembly), then scatter into ``embeds``
     (fp64 array (n_ids, D)). Returns the new fp64 embedding buffer."""
     grid_hw = np.asarray(grid_hw)
@@ -238,7 +241,7 @@ def forward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[np
     for views, crop in groups:
         feats = [f64[offs[v]:offs[v + 1]] for v in views]
         hw = [(int(grid_hw[v, 0]), int(grid_hw[v, 1])) for v in views]
-        rows.append(project_image(feats, hw, k, params, crop, ln_eps, quantise))
+        rows.append(project_image(feats, hw, k, params, crop, ln_eps, quantise, global_view_pos))
     all_rows = np.concatenate(rows, axis=0) if rows else np.zeros((0, embeds.shape[1]))
     return scatter(embeds, ids, image_token_id, all_rows)
 

@@ -1,0 +1,118 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on a B200.
+
+Small cases compare every row and span several output tiles with ragged tails in
+M and N; the five full-size workloads run in the benchmark's launch configuration
+and compare every row of sampled images plus every text row.
+"""
+import numpy as np
+import pytest
+import torch
+
+import vision_language_projector_b200 as vp
+import workloads as W
+from oracle import projector as O
+
+from gpu_harness import (DeviceInputs, check, custom, dev_bf16, feats_f64, make_case, make_projector,
+                         oracle_params, run, view_groups, TOL_ABS, TOL_REL)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # k=3, LayerNorm, odd grids, M = 199 (2 tiles, ragged), N1 = 320 (ragged 2nd tile), N2 = 96 < 128
+    "ragged_k3_ln": (custom("ragged_k3_ln", 100, 3, 128, 320, 96, 4, 2, 160, has_ln=True),
+                     [[25, 31], [9, 9], [3, 2], [30, 27]], "head", vp.ORDER_CHANNEL_OUTER),
+    # k=1: no merge, 24x24 -> 576 tokens per image (the SigLIP 384/16 count)
+    "k1_siglip": (custom("k1_siglip", 101, 1, 64, 128, 64, 2, 2, 700), [[24, 24], [24, 24]], "head",
+                  vp.ORDER_CHANNEL_OUTER),
+    # 2D tiling, odd 5x5 grids (pad to 6), 2x2 local tiles, global view first / last
+    "tiled_head_odd": (custom("tiled_head_odd", 102, 2, 64, 192, 128, 3, 3, 80, tiled=True, tw=2, th=2),
+                       [[5, 5]] * 15, "head", vp.ORDER_CHANNEL_OUTER),
+    "tiled_tail_odd": (custom("tiled_tail_odd", 103, 2, 64, 192, 128, 3, 3, 80, tiled=True, tw=2, th=2),
+                       [[5, 5]] * 15, "tail", vp.ORDER_CHANNEL_OUTER),
+    # fp32 features without LayerNorm (converted to bf16 on the device)
+    "fp32_noln": (custom("fp32_noln", 104, 2, 64, 256, 128, 2, 1, 200, feat_fp32=True), [[16, 12], [7, 9]],
+                  "head", vp.ORDER_CHANNEL_OUTER),
+    # W1 handed over in position-outer column order
+    "position_outer": (custom("position_outer", 105, 2, 128, 256, 256, 3, 3, 300, has_ln=True),
+                       [[20, 14], [13, 13], [2, 30]], "head", vp.ORDER_POSITION_OUTER),
+    # a single 1x1 grid (one merged token, three pad neighbours)
+    "one_patch": (custom("one_patch", 106, 2, 64, 64, 32, 1, 1, 10), [[1, 1]], "head", vp.ORDER_CHANNEL_OUTER),
+    # many images, 8 sequences; M = 1408 (11 full tiles), N2 = 512 (two 256 tiles)
+    "many_images": (custom("many_images", 107, 2, 64, 256, 512, 32, 8, 256), [[12, 16]] * 32, "head",
+                    vp.ORDER_CHANNEL_OUTER),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_case_all_rows(name):
+    wl, hw, gvp, order = SMALL[name]
+    case = make_case(wl, np.array(hw, np.int32), gvp=gvp, k_order=order)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    out = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    check(case, out, dev)
+    # a second call on the same handle gives the same bits
+    out2 = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["ragged_k3_ln", "tiled_head_odd", "fp32_noln"])
+def test_hidden_stage(name):
+    """Stage parity of H = bf16(GELU(A W1^T + b1)) for every merged token."""
+    wl, hw, gvp, order = SMALL[name]
+    case = make_case(wl, np.array(hw, np.int32), gvp=gvp, k_order=order)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    M = sum(O.tokens_untiled(h, w, wl.k) for h, w in case.hw)
+    H = torch.empty((M, wl.N1), dtype=torch.bfloat16, device="cuda")
+    proj.hidden(dev.feats, case.hw, H)
+    assert proj.status() == vp.OK
+    got = H.double().cpu().numpy()
+    params = oracle_params(case)
+    ln = (params["gamma"], params["beta"], wl.ln_eps) if wl.has_ln else None
+    r = 0
+    for v in range(len(case.hw)):
+        h, w = int(case.hw[v, 0]), int(case.hw[v, 1])
+        a = O.merge_view(feats_f64(case, v), h, w, wl.k, ln)
+        want = O.hidden(a, params["W1"], params["b1"])
+        g = got[r:r + len(want)]
+        assert (np.abs(g - want) <= TOL_ABS + TOL_REL * np.abs(want)).all(), f"view {v}"
+        r += len(want)
+
+
+# image subsets compared against the oracle at full size (all text rows always checked)
+SAMPLES = {"tiny": None, "moonvit": "extremes", "dsvit": [0, 7], "vl2": [0, 17, 31], "stress": [0, 131, 255]}
+
+
+@pytest.mark.parametrize("name", list(SAMPLES))
+def test_workload_full_size(name):
+    wl = W.WORKLOADS[name]
+    case = make_case(wl)
+    images = SAMPLES[name]
+    if images == "extremes":
+        rows = np.array(case.rows)
+        images = sorted({int(rows.argmin()), int(rows.argmax()), 5})
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    out = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    stats = check(case, out, dev, images)
+    print(name, stats)
+
+
+def test_gemm_ragged_edges_are_exact_zero_pad():
+    """An image whose odd grid needs padding must give the same rows as the same image
+    with the pad written out as explicit zero patches (pad rows exactly 0)."""
+    wl = custom("pad_equiv", 108, 3, 64, 128, 64, 1, 1, 64)
+    case = make_case(wl, np.array([[7, 8]], np.int32))
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    out = run(case, proj, dev)
+    padded = np.zeros((9 * 9, wl.C), np.uint16)
+    padded.reshape(9, 9, wl.C)[:7, :8] = case.feats.reshape(7, 8, wl.C)
+    out2 = dev.prefill.clone()
+    proj.forward(dev_bf16(padded), np.array([[9, 9]], np.int32), None, dev.ids, W.IMAGE_TOKEN_ID, out2)
+    assert proj.status() == vp.OK
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))

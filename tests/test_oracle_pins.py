@@ -160,7 +160,7 @@ def test_param_count_pins_moonvit_projector_shape():
 
 
 # ------------------------------------------------------------------ assembly
-def _labels_assembled(hp, wp, tw, th):
+def _labels_assembled(hp, wp, tw, th, gvp="head"):
     """Run the oracle's assembly on label 'vectors' (object arrays of names)."""
     n_views = 1 + tw * th
     views = np.empty((n_views, hp * wp, 1), dtype=object)
@@ -170,12 +170,12 @@ def _labels_assembled(hp, wp, tw, th):
                 views[v, i * wp + j, 0] = f"G{i}{j}" if v == 0 else f"L{v-1}_{i}{j}"
     nl = np.array(["NL"], dtype=object)
     sep = np.array(["SEP"], dtype=object)
-    return list(O.assemble_2d(views, hp, wp, tw, th, nl, sep)[:, 0])
+    return list(O.assemble_2d(views, hp, wp, tw, th, nl, sep, gvp)[:, 0])
 
 
 @pytest.mark.parametrize("case", _golden("assembly_hand.json")["cases"], ids=lambda c: str(c["rows"][:3]))
 def test_assembly_hand_examples(case):
-    got = _labels_assembled(case["hp"], case["wp"], case["tw"], case["th"])
+    got = _labels_assembled(case["hp"], case["wp"], case["tw"], case["th"], case.get("global_view_pos", "head"))
     assert got == case["rows"]
     assert len(got) == O.tokens_tiled(case["hp"], case["wp"], case["tw"], case["th"])
 

@@ -1,0 +1,214 @@
+"""Python binding of ``libvlproj.so``, the B200 vision-to-language projector.
+
+Argument marshalling only: every step of the projector runs in the library's
+CUDA kernels. Tensors are torch tensors (device memory and streams are the only
+things torch provides here); their raw pointers are handed to the C ABI declared
+in ``include/vlproj.h``. Importing this module without the built library raises
+immediately; there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvlproj.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TOKEN_COUNT, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+FEAT_BF16, FEAT_F32 = 0, 1
+TILE_NONE, TILE_2D, TILE_1D = 0, 1, 2
+GLOBAL_HEAD, GLOBAL_TAIL = 0, 1
+ORDER_CHANNEL_OUTER, ORDER_POSITION_OUTER = 0, 1
+
+EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status", "vlproj_destroy",
+            "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
+            "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count")
+NUM_STAGES = 6
+STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows")
+
+
+class VlprojError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+
+
+class Config(ctypes.Structure):
+    """Mirror of ``vlproj_config``."""
+    _fields_ = [
+        ("k", ctypes.c_int32), ("C", ctypes.c_int32), ("N1", ctypes.c_int32), ("N2", ctypes.c_int32),
+        ("depth", ctypes.c_int32), ("has_ln", ctypes.c_int32), ("ln_eps", ctypes.c_float),
+        ("feat_dtype", ctypes.c_int32), ("k_order", ctypes.c_int32), ("tile_tag", ctypes.c_int32),
+        ("global_view_pos", ctypes.c_int32), ("token_pooling", ctypes.c_int32),
+        ("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
+        ("ln_gamma", ctypes.c_void_p), ("ln_beta", ctypes.c_void_p),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m vision_language_projector_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, U64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64
+    lib.vlproj_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(P)]
+    lib.vlproj_create.restype = ctypes.c_int
+    lib.vlproj_forward.argtypes = [P, P, P, P, I32, P, I64, I64, P, P, P, P]
+    lib.vlproj_forward.restype = ctypes.c_int
+    lib.vlproj_hidden.argtypes = [P, P, P, I32, P, P]
+    lib.vlproj_hidden.restype = ctypes.c_int
+    lib.vlproj_status.argtypes = [P, P]
+    lib.vlproj_status.restype = ctypes.c_int
+    lib.vlproj_destroy.argtypes = [P]
+    lib.vlproj_destroy.restype = None
+    lib.vlproj_image_rows.argtypes = [ctypes.POINTER(Config), P, P, I32, P]
+    lib.vlproj_image_rows.restype = I64
+    lib.vlproj_set_wait_limit.argtypes = [P, U64]
+    lib.vlproj_set_wait_limit.restype = ctypes.c_int
+    lib.vlproj_strerror.argtypes = [ctypes.c_int]
+    lib.vlproj_strerror.restype = ctypes.c_char_p
+    lib.vlproj_version.argtypes = []
+    lib.vlproj_version.restype = ctypes.c_char_p
+    lib.vlproj_profile_enable.argtypes = [P, ctypes.c_int]
+    lib.vlproj_profile_enable.restype = ctypes.c_int
+    lib.vlproj_profile_read.argtypes = [P, P, ctypes.c_int]
+    lib.vlproj_profile_read.restype = ctypes.c_int
+    lib.vlproj_launch_count.argtypes = [P]
+    lib.vlproj_launch_count.restype = I64
+    return lib
+
+
+_lib = _load()
+
+
+def strerror(code: int) -> str:
+    return _lib.vlproj_strerror(int(code)).decode()
+
+
+def version() -> str:
+    return _lib.vlproj_version().decode()
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _host_i32(a) -> Optional[np.ndarray]:
+    if a is None:
+        return None
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def make_config(k: int, C: int, N1: int, N2: int, *, has_ln: bool = False, ln_eps: float = 1e-5,
+                feat_dtype: int = FEAT_BF16, tile_tag: int = TILE_NONE, global_view_pos: int = GLOBAL_HEAD,
+                k_order: int = ORDER_CHANNEL_OUTER, depth: int = 2, token_pooling: int = 0,
+                W1=None, b1=None, W2=None, b2=None, ln_gamma=None, ln_beta=None) -> Config:
+    return Config(k, C, N1, N2, depth, int(has_ln), ln_eps, feat_dtype, k_order, tile_tag, global_view_pos,
+                  token_pooling, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(ln_gamma), _ptr(ln_beta))
+
+
+def image_rows(cfg: Config, grid_hw, spatial_crop=None, n_images: Optional[int] = None) -> np.ndarray:
+    """Closed-form placeholder count of every image (host only, no GPU needed)."""
+    g = _host_i32(grid_hw)
+    c = _host_i32(spatial_crop)
+    if n_images is None:
+        n_images = len(c) if c is not None else (0 if g is None else len(g))
+    out = np.zeros(max(n_images, 1), np.int64)
+    r = _lib.vlproj_image_rows(ctypes.byref(cfg), _ptr(g), _ptr(c), n_images, out.ctypes.data)
+    if r < 0:
+        raise VlprojError(int(r), "vlproj_image_rows")
+    return out[:n_images]
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class Projector:
+    """Owns a ``vlproj_handle``. Weight tensors must be CUDA tensors on the current device:
+    W1 bf16 (N1, k*k*C), W2 bf16 (N2, N1), biases / LayerNorm parameters fp32."""
+
+    def __init__(self, k: int, C: int, N1: int, N2: int, W1, W2, b1=None, b2=None, *, has_ln: bool = False,
+                 ln_gamma=None, ln_beta=None, ln_eps: float = 1e-5, feat_dtype: int = FEAT_BF16,
+                 tile_tag: int = TILE_NONE, global_view_pos: int = GLOBAL_HEAD, k_order: int = ORDER_CHANNEL_OUTER,
+                 depth: int = 2, token_pooling: int = 0):
+        self.cfg = make_config(k, C, N1, N2, has_ln=has_ln, ln_eps=ln_eps, feat_dtype=feat_dtype,
+                               tile_tag=tile_tag, global_view_pos=global_view_pos, k_order=k_order, depth=depth,
+                               token_pooling=token_pooling, W1=W1, b1=b1, W2=W2, b2=b2, ln_gamma=ln_gamma,
+                               ln_beta=ln_beta)
+        h = ctypes.c_void_p()
+        rc = _lib.vlproj_create(ctypes.byref(self.cfg), ctypes.byref(h))
+        if rc != OK:
+            raise VlprojError(rc, "vlproj_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.vlproj_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def forward(self, features, grid_hw, spatial_crop, input_ids, image_token_id: int, out_embeds,
+                newline=None, sep=None, stream=None, n_images: Optional[int] = None, check: bool = True) -> int:
+        """Enqueue the bridge; raise on a host-detected error. Returns the status code."""
+        g = _host_i32(grid_hw)
+        c = _host_i32(spatial_crop)
+        if n_images is None:
+            n_images = len(c) if c is not None else (0 if g is None else len(g))
+        n_ids = 0 if input_ids is None else int(input_ids.numel())
+        rc = _lib.vlproj_forward(self._h, _ptr(features), _ptr(g), _ptr(c), n_images, _ptr(input_ids), n_ids,
+                                 int(image_token_id), _ptr(newline), _ptr(sep), _ptr(out_embeds),
+                                 _stream_ptr(stream))
+        if check and rc != OK:
+            raise VlprojError(rc, "vlproj_forward")
+        return rc
+
+    def hidden(self, features, grid_hw, hidden, stream=None) -> None:
+        g = _host_i32(grid_hw)
+        rc = _lib.vlproj_hidden(self._h, _ptr(features), _ptr(g), 0 if g is None else len(g), _ptr(hidden),
+                                _stream_ptr(stream))
+        if rc != OK:
+            raise VlprojError(rc, "vlproj_hidden")
+
+    def status(self, stream=None) -> int:
+        """Synchronise the stream and return (and clear) the latched device status."""
+        return _lib.vlproj_status(self._h, _stream_ptr(stream))
+
+    def profile(self, enable: bool = True) -> None:
+        rc = _lib.vlproj_profile_enable(self._h, int(enable))
+        if rc != OK:
+            raise VlprojError(rc, "vlproj_profile_enable")
+
+    def stage_ms(self) -> dict:
+        """Per-stage device milliseconds of the most recent profiled forward (synchronises)."""
+        buf = (ctypes.c_float * NUM_STAGES)()
+        rc = _lib.vlproj_profile_read(self._h, ctypes.cast(buf, ctypes.c_void_p), NUM_STAGES)
+        if rc < 0:
+            raise VlprojError(rc, "vlproj_profile_read")
+        return {name: float(buf[i]) for i, name in enumerate(STAGES)}
+
+    def launch_count(self) -> int:
+        return int(_lib.vlproj_launch_count(self._h))
+
+    def set_wait_limit(self, ns: int) -> None:
+        rc = _lib.vlproj_set_wait_limit(self._h, int(ns))
+        if rc != OK:
+            raise VlprojError(rc, "vlproj_set_wait_limit")

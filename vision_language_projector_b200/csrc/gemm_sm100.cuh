@@ -1,0 +1,345 @@
+// Projector GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM), sm_100a.
+//
+//   GEMM1 (kGather = true,  kEpi = EPI_GELU):
+//       H[m, n]  = bf16( GELU( sum_q A[m, q] W1p[n, q] + b1[n] ) )
+//       A is never materialised: row m of A is the k x k neighbourhood of merged
+//       token m, gathered straight from the patch features into the swizzled
+//       shared-memory operand tile (high-end pad rows are zero-filled by the copy).
+//   GEMM2 (kGather = false, kEpi = EPI_SCATTER):
+//       out[dest[m], n] = bf16( sum_q H[m, q] W2[n, q] + b2[n] )
+//       the epilogue writes each row straight into its placeholder row.
+//
+// One persistent CTA per SM walks output tiles of BM x BN (N fastest, so the
+// CTAs working at the same time share the A tile through L2). Roles, by warp:
+//   warp 0      TMA producer (B always; A too when it is a dense matrix)
+//   warp 1      TMEM allocator and the single MMA-issuing thread
+//   warps 2-3   A gather producers (GEMM1 only): 64 threads, cp.async 16 B each
+//   warps 4-7   epilogue: TMEM -> registers -> bias (+GELU) -> bf16 -> global
+// Shared memory holds a STAGES-deep ring of (A, B) K-blocks of 64 bf16 (128 B
+// rows, 128-byte swizzle); TMEM holds two BM x BN fp32 accumulators so the
+// epilogue of one tile overlaps the MMAs of the next.
+//
+// Every wait is bounded (GemmParams::wait_ns). When one runs out, the kernel
+// latches VLPROJ_ERR_TIMEOUT, every role unwinds, outstanding copies and MMAs
+// are drained under a separate 1 s bound, TMEM is freed, and the kernel returns.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace vlp {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                  // 64 bf16 = one 128-byte swizzle row
+constexpr int GEMM_THREADS = 256;
+constexpr int GATHER_THREADS = 64;
+constexpr int EPI_GELU = 0;
+constexpr int EPI_SCATTER = 1;
+constexpr uint64_t DRAIN_NS = 1000000000ull;
+constexpr int ERR_TIMEOUT = -5;
+
+template <int BN>
+struct GemmLayout {
+    static constexpr int STAGES = BN == 256 ? 4 : 6;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+    // full_tma[S], full_gather[S], empty[S], tmem_full[2], tmem_empty[2], drain
+    static constexpr int NUM_BARS = 3 * STAGES + 5;
+    static constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
+    static constexpr int BYTES = MISC_OFFSET + 16;
+    static constexpr int SMEM_ALLOC = BYTES + 1024;      // room to align the base to 1024 B
+    static constexpr uint32_t TMEM_COLS = 2 * BN;        // two accumulators
+};
+
+struct GemmParams {
+    int M;                          // rows (merged tokens)
+    int N;                          // output columns
+    int K;                          // reduction length, multiple of BK
+    const float* bias;              // [N] fp32
+    // A gather (GEMM1)
+    const __nv_bfloat16* gsrc;      // bf16 patch features [P][C]
+    const int2* gmeta;              // per row: {top-left patch index, (w << 16) | valid mask}
+    int C;                          // channels per patch; C % BK == 0
+    int k;                          // merge factor
+    // output
+    __nv_bfloat16* out;             // GEMM1: H [M][N]; GEMM2: embeddings [out_rows][N]
+    const int32_t* rowdest;         // GEMM2: destination row of each m
+    int64_t out_rows;               // GEMM2: rows of the embedding buffer (bounds guard)
+    const int* fwd_status;          // GEMM2: nonzero = count check failed, write nothing
+    int* err;                       // latched error word
+    uint64_t wait_ns;               // bound on every wait
+};
+
+__device__ __forceinline__ void latch_error(int* err, int code) { atomicCAS(err, 0, code); }
+
+__device__ __forceinline__ float gelu_erf(float x) {
+    return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int BN, bool kGather, int kEpi>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    vlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmParams p) {
+    using L = GemmLayout<BN>;
+    constexpr int S = L::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
+    uint64_t* full_tma = bars;
+    uint64_t* full_gat = bars + S;
+    uint64_t* empty = bars + 2 * S;
+    uint64_t* tmem_full = bars + 3 * S;
+    uint64_t* tmem_empty = bars + 3 * S + 2;
+    uint64_t* drain = bars + 3 * S + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFFSET);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFFSET + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_tma[s], 1);
+            mbar_init(&full_gat[s], GATHER_THREADS);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tmem_full[a], 1);
+            mbar_init(&tmem_empty[a], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmB);
+        if (!kGather) tma_prefetch_desc(&tmA);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int m_tiles = (p.M + BM - 1) / BM;
+    const int n_tiles = (p.N + BN - 1) / BN;
+    const int num_tiles = m_tiles * n_tiles;
+    const int kblocks = p.K / BK;
+    const uint64_t lim = p.wait_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag)) { ok = false; break; }
+                    uint8_t* sa = smem + stage * L::STAGE_BYTES;
+                    uint8_t* sb = sa + L::A_BYTES;
+                    mbar_arrive_expect_tx(&full_tma[stage], (kGather ? 0 : L::A_BYTES) + L::B_BYTES);
+                    if (!kGather) tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, m_blk * BM);
+                    tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, n_blk * BN);
+                    ++issued;
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                latch_error(p.err, ERR_TIMEOUT);
+            }
+            // Drain: the (at most S) most recent loads may still be landing if the MMA
+            // side stopped early; in a normal run these phases are already complete.
+            int st = stage;
+            uint32_t ph = phase;
+            const int outstanding = issued < S ? issued : S;
+            for (int i = 0; i < outstanding; ++i) {
+                if (st == 0) { st = S - 1; ph ^= 1; } else { --st; }
+                volatile int never = 0;
+                mbar_wait_bounded(&full_tma[st], ph, DRAIN_NS, &never);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!mbar_wait_bounded(&tmem_empty[acc], acc_phase ^ 1, lim, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&full_tma[stage], phase, lim, abort_flag)) { ok = false; break; }
+                    if (kGather) {
+                        if (!mbar_wait_bounded(&full_gat[stage], phase, lim, abort_flag)) { ok = false; break; }
+                        fence_proxy_async_smem();
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
+                    const uint32_t sb = sa + L::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        tc_mma_f16(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
+                                   (kb | kk) != 0);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(&tmem_full[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                latch_error(p.err, ERR_TIMEOUT);
+            }
+            // all MMAs issued by this thread are complete once `drain` flips
+            tc_commit(drain);
+            volatile int never = 0;
+            mbar_wait_bounded(drain, 0, DRAIN_NS, &never);
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------ A gather producers (GEMM1)
+        if (kGather) {
+            const int gt = threadIdx.x - 64;          // 0..63
+            const int chunk = gt & 7;                 // 16-byte chunk of the 128-byte row
+            const int rsub = gt >> 3;                 // rows rsub, rsub+8, ..., rsub+120
+            const uint32_t swz = static_cast<uint32_t>((chunk ^ rsub) * 16);
+            const int cblocks = p.C / BK;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m_blk = tile / n_tiles;
+                int base[16];
+                uint32_t wm[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int m = m_blk * BM + rsub + 8 * q;
+                    if (m < p.M) {
+                        const int2 g = __ldg(&p.gmeta[m]);
+                        base[q] = g.x;
+                        wm[q] = static_cast<uint32_t>(g.y);
+                    } else {
+                        base[q] = 0;
+                        wm[q] = 0;
+                    }
+                }
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    const int pos = kb / cblocks;                  // (dy, dx) position index
+                    const int c0 = (kb - pos * cblocks) * BK + chunk * 8;
+                    const int dy = pos / p.k, dx = pos - dy * p.k;
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag)) { ok = false; break; }
+                    const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int r = rsub + 8 * q;
+                        const int w = static_cast<int>(wm[q] >> 16);
+                        const bool valid = (wm[q] >> pos) & 1u;
+                        const int64_t prow = static_cast<int64_t>(base[q]) + dy * w + dx;
+                        const __nv_bfloat16* src = valid ? p.gsrc + prow * p.C + c0 : p.gsrc;
+                        cp_async_16(sa + r * 128 + swz, src, valid ? 16u : 0u);
+                    }
+                    cp_async_arrive_noinc(&full_gat[stage]);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                latch_error(p.err, ERR_TIMEOUT);
+            }
+            cp_async_wait_all();
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 4..7)
+        const int ew = warp & 3;                      // TMEM lanes 32*ew .. 32*ew+31
+        const int row = ew * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        int status_ok = 1;
+        if (kEpi == EPI_SCATTER) status_ok = (*p.fwd_status == 0);
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
+            // one lane waits, the warp follows it, so tcgen05.ld below is never divergent
+            int got = 0;
+            if (lane == 0) got = mbar_wait_bounded(&tmem_full[acc], acc_phase, lim, abort_flag) ? 1 : 0;
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (!got) { ok = false; break; }
+            tc_fence_after();
+            const int m = m_blk * BM + row;
+            bool row_ok = m < p.M;
+            __nv_bfloat16* dst_row = nullptr;
+            if (kEpi == EPI_SCATTER) {
+                int64_t d = row_ok ? static_cast<int64_t>(__ldg(&p.rowdest[m])) : -1;
+                row_ok = row_ok && status_ok && d >= 0 && d < p.out_rows;
+                if (row_ok) dst_row = p.out + d * p.N;
+            } else {
+                if (row_ok) dst_row = p.out + static_cast<int64_t>(m) * p.N;
+            }
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n0 = n_blk * BN + c * 32;
+                if (n0 >= p.N) break;                  // uniform across the warp
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(t_row + c * 32, v);
+                tmem_ld_wait();
+                const float bl = __ldg(&p.bias[n0 + lane]);
+                uint32_t packed[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    float x0 = __uint_as_float(v[j]) + __shfl_sync(0xffffffffu, bl, j);
+                    float x1 = __uint_as_float(v[j + 1]) + __shfl_sync(0xffffffffu, bl, j + 1);
+                    if (kEpi == EPI_GELU) {
+                        x0 = gelu_erf(x0);
+                        x1 = gelu_erf(x1);
+                    }
+                    packed[j / 2] = pack_bf16x2(x0, x1);
+                }
+                if (row_ok) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst_row + n0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            latch_error(p.err, ERR_TIMEOUT);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, L::TMEM_COLS);
+    }
+}
+
+}  // namespace vlp

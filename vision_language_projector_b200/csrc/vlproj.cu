@@ -1,0 +1,596 @@
+// C-ABI host library of the vision-to-language projector (declared in vlproj.h).
+//
+// vlproj_forward enqueues, on the caller's stream and without any host sync:
+//   1. placeholder index   count + compact (ids == image_token_id), count check
+//   2. geometry            per merged token: gather metadata and destination row
+//   3. LayerNorm/convert   only with a pre-merge LayerNorm or fp32 features
+//   4. GEMM1               gather + tcgen05 MMA + bias + GELU -> H (bf16)
+//   5. GEMM2               tcgen05 MMA + bias -> bf16 rows scattered into out_embeds
+//   6. special rows        newline / separator rows (2D tiling only)
+// Host work per call: argument checks, the closed-form row counts, one small
+// descriptor upload, and tensor-map encoding for H (cached while it is unchanged).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/vlproj.h"
+#include "gemm_sm100.cuh"
+#include "kernels_aux.cuh"
+
+using vlp::GemmLayout;
+using vlp::GemmParams;
+using vlp::ImageDesc;
+using vlp::ViewDesc;
+
+namespace {
+
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+#define VLP_CUDA(call)                                                                        \
+    do {                                                                                      \
+        cudaError_t e_ = (call);                                                              \
+        if (e_ != cudaSuccess) {                                                              \
+            std::fprintf(stderr, "vlproj: %s failed: %s (%s:%d)\n", #call, cudaGetErrorString(e_), \
+                         __FILE__, __LINE__);                                                 \
+            return VLPROJ_ERR_CUDA;                                                           \
+        }                                                                                     \
+    } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2D bf16 row-major matrix [rows][cols], box = box_rows x 64 columns, 128-byte swizzle,
+// out-of-range elements read as zero.
+int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = get_encode_fn();
+    if (!fn) return VLPROJ_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(vlp::BK), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
+template <typename T>
+struct DevBuf {
+    T* ptr = nullptr;
+    size_t cap = 0;   // elements
+    int ensure(size_t n) {
+        if (n <= cap) return VLPROJ_OK;
+        if (ptr) cudaFree(ptr);
+        ptr = nullptr;
+        cap = 0;
+        size_t want = std::max<size_t>(n, 1) + n / 4;
+        if (cudaMalloc(&ptr, want * sizeof(T)) != cudaSuccess) return VLPROJ_ERR_CUDA;
+        cap = want;
+        return VLPROJ_OK;
+    }
+    void release() {
+        if (ptr) cudaFree(ptr);
+        ptr = nullptr;
+        cap = 0;
+    }
+};
+
+struct Plan {
+    std::vector<ViewDesc> views;
+    std::vector<ImageDesc> images;
+    int64_t M = 0;          // merged tokens
+    int64_t R = 0;          // assembled rows
+    int64_t P = 0;          // patches
+    int max_special = 0;    // most special rows of one image
+};
+
+int validate_config(const vlproj_config* c) {
+    if (!c) return VLPROJ_ERR_INVALID_ARG;
+    if (c->depth != 2 || c->tile_tag == VLPROJ_TILE_1D || c->token_pooling != 0) return VLPROJ_ERR_UNSUPPORTED;
+    if (c->k < 1 || c->k > 3) return VLPROJ_ERR_UNSUPPORTED;
+    if (c->tile_tag != VLPROJ_TILE_NONE && c->tile_tag != VLPROJ_TILE_2D) return VLPROJ_ERR_UNSUPPORTED;
+    if (c->global_view_pos != VLPROJ_GLOBAL_HEAD && c->global_view_pos != VLPROJ_GLOBAL_TAIL)
+        return VLPROJ_ERR_INVALID_ARG;
+    if (c->feat_dtype != VLPROJ_FEAT_BF16 && c->feat_dtype != VLPROJ_FEAT_F32) return VLPROJ_ERR_INVALID_ARG;
+    if (c->k_order != VLPROJ_ORDER_CHANNEL_OUTER && c->k_order != VLPROJ_ORDER_POSITION_OUTER)
+        return VLPROJ_ERR_INVALID_ARG;
+    if (c->C <= 0 || c->C % 64 != 0 || c->N1 <= 0 || c->N1 % 64 != 0 || c->N2 <= 0 || c->N2 % 32 != 0)
+        return VLPROJ_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(c->k) * c->k * c->C > (1 << 20) || c->N1 > (1 << 20) || c->N2 > (1 << 20))
+        return VLPROJ_ERR_INVALID_ARG;
+    return VLPROJ_OK;
+}
+
+// Closed-form geometry of one batch. Returns an error for inconsistent shapes.
+int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int32_t* crop, int32_t n_images,
+               bool tiled_override_none, Plan* out) {
+    Plan& pl = *out;
+    pl = Plan();
+    if (n_images < 0) return VLPROJ_ERR_INVALID_ARG;
+    if (n_images > 0 && !grid_hw) return VLPROJ_ERR_INVALID_ARG;
+    const bool tiled = !tiled_override_none && c.tile_tag == VLPROJ_TILE_2D;
+    if (tiled && n_images > 0 && !crop) return VLPROJ_ERR_INVALID_ARG;
+    const int k = c.k;
+    int64_t v = 0;
+    for (int32_t img = 0; img < n_images; ++img) {
+        const int tw = tiled ? crop[2 * img] : 0;
+        const int th = tiled ? crop[2 * img + 1] : 0;
+        if (tiled && (tw < 1 || th < 1 || static_cast<int64_t>(tw) * th > 4096)) return VLPROJ_ERR_INVALID_ARG;
+        const int nv = tiled ? 1 + tw * th : 1;
+        const int h0 = grid_hw[2 * v], w0 = grid_hw[2 * v + 1];
+        if (h0 < 1 || w0 < 1 || h0 > 65535 || w0 > 65535) return VLPROJ_ERR_INVALID_ARG;
+        const int hp = (h0 + k - 1) / k, wp = (w0 + k - 1) / k;
+        int64_t rows;
+        if (tiled) rows = static_cast<int64_t>(hp) * (wp + 1) + 1 + static_cast<int64_t>(th) * hp * (static_cast<int64_t>(tw) * wp + 1);
+        else rows = static_cast<int64_t>(hp) * wp;
+        for (int t = 0; t < nv; ++t, ++v) {
+            const int h = grid_hw[2 * v], w = grid_hw[2 * v + 1];
+            if (h != h0 || w != w0) return VLPROJ_ERR_INVALID_ARG;   // views of one image share a grid
+            ViewDesc d{};
+            d.patch_start = pl.P;
+            d.tok_start = static_cast<int32_t>(pl.M);
+            d.h = h; d.w = w; d.hp = hp; d.wp = wp;
+            d.row_base = static_cast<int32_t>(pl.R);
+            d.view_in_image = t;
+            d.tw = tw; d.th = th;
+            d.tail = tiled && c.global_view_pos == VLPROJ_GLOBAL_TAIL;
+            pl.views.push_back(d);
+            pl.P += static_cast<int64_t>(h) * w;
+            pl.M += static_cast<int64_t>(hp) * wp;
+            if (pl.P >= (int64_t(1) << 31) || pl.M >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
+        }
+        if (tiled) {
+            ImageDesc im{};
+            im.row_base = static_cast<int32_t>(pl.R);
+            im.hp = hp; im.wp = wp; im.tw = tw; im.th = th;
+            im.tail = c.global_view_pos == VLPROJ_GLOBAL_TAIL;
+            pl.images.push_back(im);
+            pl.max_special = std::max(pl.max_special, hp + th * hp + 1);
+        }
+        pl.R += rows;
+        if (pl.R >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
+    }
+    return VLPROJ_OK;
+}
+
+template <int BN, bool G, int E>
+int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int num_sms, cudaStream_t s) {
+    using L = GemmLayout<BN>;
+    VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_gemm_kernel<BN, G, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  L::SMEM_ALLOC));
+    const int tiles = ((p.M + vlp::BM - 1) / vlp::BM) * ((p.N + BN - 1) / BN);
+    const int grid = std::min(tiles, num_sms);
+    if (grid <= 0) return VLPROJ_OK;
+    vlp::vlp_gemm_kernel<BN, G, E><<<grid, vlp::GEMM_THREADS, L::SMEM_ALLOC, s>>>(ta, tb, p);
+    VLP_CUDA(cudaGetLastError());
+    return VLPROJ_OK;
+}
+
+template <bool G, int E>
+int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int num_sms,
+                   cudaStream_t s) {
+    if (bn == 256) return launch_gemm<256, G, E>(ta, tb, p, num_sms, s);
+    return launch_gemm<128, G, E>(ta, tb, p, num_sms, s);
+}
+
+int pick_bn(int N) { return N >= 256 ? 256 : 128; }
+
+}  // namespace
+
+struct vlproj_handle {
+    vlproj_config cfg{};
+    int device = 0;
+    int num_sms = 148;
+    int K1 = 0;
+    uint64_t wait_ns = kDefaultWaitNs;
+    __nv_bfloat16* W1p = nullptr;
+    __nv_bfloat16* W2 = nullptr;
+    float* b1 = nullptr;
+    float* b2 = nullptr;
+    float* gamma = nullptr;
+    float* beta = nullptr;
+    CUtensorMap tmW1{}, tmW2{};
+    // scratch, grown on demand
+    DevBuf<__nv_bfloat16> H, Xn;
+    DevBuf<int32_t> pos, rowdest, counts;
+    DevBuf<int2> gmeta;
+    DevBuf<ViewDesc> dviews;
+    DevBuf<ImageDesc> dimages;
+    int* status = nullptr;       // [0] latched error, [1] per-forward count check
+    // pinned staging for the per-call descriptors, guarded by an event
+    uint8_t* staging = nullptr;
+    size_t staging_cap = 0;
+    cudaEvent_t staging_done = nullptr;
+    // geometry key of the descriptors now on the device (skip re-upload when unchanged)
+    std::vector<int32_t> uploaded_key;
+    // tracing
+    bool profiling = false;
+    bool profiled_valid = false;
+    cudaEvent_t ev[VLPROJ_NUM_STAGES + 1] = {};
+    bool stage_ran[VLPROJ_NUM_STAGES] = {};
+    int64_t launches = 0;
+    // cached tensor map of H
+    CUtensorMap tmH{};
+    const void* tmH_ptr = nullptr;
+    int64_t tmH_rows = -1;
+};
+
+namespace {
+
+// Record the boundary before stage `stage` (stage == VLPROJ_NUM_STAGES closes the last).
+void mark(vlproj_handle* h, int stage, cudaStream_t s) {
+    if (h->profiling) cudaEventRecord(h->ev[stage], s);
+}
+
+std::vector<int32_t> plan_key(const int32_t* grid_hw, int64_t n_views, const int32_t* crop, int32_t n_images,
+                              int32_t mode) {
+    std::vector<int32_t> key;
+    key.reserve(static_cast<size_t>(2 * n_views + 2 * n_images + 2));
+    key.push_back(mode);
+    key.push_back(n_images);
+    for (int64_t i = 0; i < 2 * n_views; ++i) key.push_back(grid_hw[i]);
+    if (crop)
+        for (int64_t i = 0; i < 2 * n_images; ++i) key.push_back(crop[i]);
+    return key;
+}
+
+int upload(vlproj_handle* h, const Plan& pl, std::vector<int32_t>&& key, cudaStream_t s) {
+    if (key == h->uploaded_key) return VLPROJ_OK;
+    h->uploaded_key.clear();
+    const size_t vb = pl.views.size() * sizeof(ViewDesc);
+    const size_t ib = pl.images.size() * sizeof(ImageDesc);
+    const size_t need = vb + ib + 64;
+    VLP_CUDA(cudaEventSynchronize(h->staging_done));   // the previous upload has left the staging area
+    if (need > h->staging_cap) {
+        if (h->staging) cudaFreeHost(h->staging);
+        h->staging = nullptr;
+        h->staging_cap = 0;
+        VLP_CUDA(cudaMallocHost(&h->staging, need * 2));
+        h->staging_cap = need * 2;
+    }
+    if (h->dviews.ensure(std::max<size_t>(pl.views.size(), 1))) return VLPROJ_ERR_CUDA;
+    if (h->dimages.ensure(std::max<size_t>(pl.images.size(), 1))) return VLPROJ_ERR_CUDA;
+    if (vb) std::memcpy(h->staging, pl.views.data(), vb);
+    if (ib) std::memcpy(h->staging + vb, pl.images.data(), ib);
+    if (vb) VLP_CUDA(cudaMemcpyAsync(h->dviews.ptr, h->staging, vb, cudaMemcpyHostToDevice, s));
+    if (ib) VLP_CUDA(cudaMemcpyAsync(h->dimages.ptr, h->staging + vb, ib, cudaMemcpyHostToDevice, s));
+    VLP_CUDA(cudaEventRecord(h->staging_done, s));
+    h->uploaded_key = std::move(key);
+    return VLPROJ_OK;
+}
+
+// Steps 2-4: geometry (+ destinations when pos is given), LayerNorm/convert, GEMM1 into `hidden`.
+int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, const int32_t* pos,
+                    __nv_bfloat16* hidden, cudaStream_t s) {
+    const vlproj_config& c = h->cfg;
+    const int M = static_cast<int>(pl.M);
+    if (M == 0) return VLPROJ_OK;
+    if (h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
+    if (pos && h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
+    mark(h, 1, s);
+    h->stage_ran[1] = true;
+    ++h->launches;
+    vlp::vlp_geometry_kernel<<<(M + 255) / 256, 256, 0, s>>>(h->dviews.ptr, static_cast<int>(pl.views.size()), M,
+                                                             c.k, pos, pl.R, h->gmeta.ptr,
+                                                             pos ? h->rowdest.ptr : nullptr);
+    VLP_CUDA(cudaGetLastError());
+
+    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(features);
+    mark(h, 2, s);
+    if (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) {
+        h->stage_ran[2] = true;
+        ++h->launches;
+        if (h->Xn.ensure(static_cast<size_t>(pl.P) * c.C)) return VLPROJ_ERR_CUDA;
+        const unsigned blocks = static_cast<unsigned>((pl.P + 7) / 8);
+        const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
+        if (c.feat_dtype == VLPROJ_FEAT_F32)
+            vlp::vlp_layernorm_kernel<true><<<blocks, 256, 0, s>>>(features, pl.P, c.C, h->gamma, h->beta, eps,
+                                                                   c.has_ln, h->Xn.ptr);
+        else
+            vlp::vlp_layernorm_kernel<false><<<blocks, 256, 0, s>>>(features, pl.P, c.C, h->gamma, h->beta, eps,
+                                                                    c.has_ln, h->Xn.ptr);
+        VLP_CUDA(cudaGetLastError());
+        src = h->Xn.ptr;
+    }
+
+    GemmParams p{};
+    p.M = M;
+    p.N = c.N1;
+    p.K = h->K1;
+    p.bias = h->b1;
+    p.gsrc = src;
+    p.gmeta = h->gmeta.ptr;
+    p.C = c.C;
+    p.k = c.k;
+    p.out = hidden;
+    p.err = h->status;
+    p.wait_ns = h->wait_ns;
+    CUtensorMap unused{};
+    std::memset(&unused, 0, sizeof(unused));
+    mark(h, 3, s);
+    h->stage_ran[3] = true;
+    ++h->launches;
+    return launch_gemm_bn<true, vlp::EPI_GELU>(pick_bn(c.N1), unused, h->tmW1, p, h->num_sms, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vlproj_strerror(int code) {
+    switch (code) {
+        case VLPROJ_OK: return "ok";
+        case VLPROJ_ERR_INVALID_ARG: return "invalid argument";
+        case VLPROJ_ERR_UNSUPPORTED: return "unsupported projector configuration";
+        case VLPROJ_ERR_CUDA: return "CUDA error";
+        case VLPROJ_ERR_TOKEN_COUNT: return "placeholder count does not match the image rows";
+        case VLPROJ_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+        default: return "unknown status";
+    }
+}
+
+const char* vlproj_version(void) { return "vlproj 0.1 sm_100a"; }
+
+int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw, const int32_t* spatial_crop,
+                          int32_t n_images, int64_t* rows_out) {
+    int rc = validate_config(cfg);
+    if (rc) return rc;
+    Plan pl;
+    rc = build_plan(*cfg, grid_hw, spatial_crop, n_images, false, &pl);
+    if (rc) return rc;
+    if (rows_out) {
+        // rows of image i = (row_base of the next image) - (its own)
+        std::vector<int64_t> base;
+        if (cfg->tile_tag == VLPROJ_TILE_2D) {
+            for (auto& im : pl.images) base.push_back(im.row_base);
+        } else {
+            for (auto& v : pl.views) base.push_back(v.row_base);
+        }
+        base.push_back(pl.R);
+        for (int32_t i = 0; i < n_images; ++i) rows_out[i] = base[i + 1] - base[i];
+    }
+    return pl.R;
+}
+
+int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
+    if (!out) return VLPROJ_ERR_INVALID_ARG;
+    *out = nullptr;
+    int rc = validate_config(cfg);
+    if (rc) return rc;
+    if (!cfg->W1 || !cfg->W2 || (cfg->has_ln && (!cfg->ln_gamma || !cfg->ln_beta))) return VLPROJ_ERR_INVALID_ARG;
+    if (!get_encode_fn()) return VLPROJ_ERR_CUDA;
+
+    vlproj_handle* h = new vlproj_handle();
+    h->cfg = *cfg;
+    h->K1 = cfg->k * cfg->k * cfg->C;
+    auto fail = [&](int code) {
+        vlproj_destroy(h);
+        return code;
+    };
+    if (cudaGetDevice(&h->device) != cudaSuccess) return fail(VLPROJ_ERR_CUDA);
+    if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess)
+        return fail(VLPROJ_ERR_CUDA);
+    const size_t n1 = static_cast<size_t>(cfg->N1), n2 = static_cast<size_t>(cfg->N2), C = static_cast<size_t>(cfg->C);
+    if (cudaMalloc(&h->W1p, n1 * h->K1 * 2) || cudaMalloc(&h->W2, n2 * n1 * 2) || cudaMalloc(&h->b1, n1 * 4) ||
+        cudaMalloc(&h->b2, n2 * 4) || cudaMalloc(&h->gamma, C * 4) || cudaMalloc(&h->beta, C * 4) ||
+        cudaMalloc(&h->status, 2 * sizeof(int)) || cudaEventCreateWithFlags(&h->staging_done, cudaEventDisableTiming))
+        return fail(VLPROJ_ERR_CUDA);
+    cudaStream_t s = nullptr;
+    vlp::vlp_permute_w1_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(cfg->W1), h->W1p,
+                                                    cfg->N1, cfg->C, cfg->k * cfg->k,
+                                                    cfg->k_order == VLPROJ_ORDER_POSITION_OUTER);
+    if (cudaGetLastError() != cudaSuccess) return fail(VLPROJ_ERR_CUDA);
+    ++h->launches;
+    if (cudaMemcpy(h->W2, cfg->W2, n2 * n1 * 2, cudaMemcpyDeviceToDevice)) return fail(VLPROJ_ERR_CUDA);
+    if (cfg->b1 ? cudaMemcpy(h->b1, cfg->b1, n1 * 4, cudaMemcpyDeviceToDevice) : cudaMemset(h->b1, 0, n1 * 4))
+        return fail(VLPROJ_ERR_CUDA);
+    if (cfg->b2 ? cudaMemcpy(h->b2, cfg->b2, n2 * 4, cudaMemcpyDeviceToDevice) : cudaMemset(h->b2, 0, n2 * 4))
+        return fail(VLPROJ_ERR_CUDA);
+    if (cfg->has_ln) {
+        if (cudaMemcpy(h->gamma, cfg->ln_gamma, C * 4, cudaMemcpyDeviceToDevice) ||
+            cudaMemcpy(h->beta, cfg->ln_beta, C * 4, cudaMemcpyDeviceToDevice))
+            return fail(VLPROJ_ERR_CUDA);
+    } else if (cudaMemset(h->gamma, 0, C * 4) || cudaMemset(h->beta, 0, C * 4)) {
+        return fail(VLPROJ_ERR_CUDA);
+    }
+    if (cudaMemset(h->status, 0, 2 * sizeof(int))) return fail(VLPROJ_ERR_CUDA);
+    if (cudaEventRecord(h->staging_done, s) || cudaDeviceSynchronize()) return fail(VLPROJ_ERR_CUDA);
+    if (encode_bf16_2d(&h->tmW1, h->W1p, n1, h->K1, pick_bn(cfg->N1)) ||
+        encode_bf16_2d(&h->tmW2, h->W2, n2, n1, pick_bn(cfg->N2)))
+        return fail(VLPROJ_ERR_CUDA);
+    *out = h;
+    return VLPROJ_OK;
+}
+
+void vlproj_destroy(vlproj_handle* h) {
+    if (!h) return;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    cudaSetDevice(h->device);
+    cudaDeviceSynchronize();
+    cudaFree(h->W1p);
+    cudaFree(h->W2);
+    cudaFree(h->b1);
+    cudaFree(h->b2);
+    cudaFree(h->gamma);
+    cudaFree(h->beta);
+    cudaFree(h->status);
+    h->H.release();
+    h->Xn.release();
+    h->pos.release();
+    h->rowdest.release();
+    h->counts.release();
+    h->gmeta.release();
+    h->dviews.release();
+    h->dimages.release();
+    if (h->staging) cudaFreeHost(h->staging);
+    if (h->staging_done) cudaEventDestroy(h->staging_done);
+    for (auto& e : h->ev)
+        if (e) cudaEventDestroy(e);
+    cudaSetDevice(cur);
+    delete h;
+}
+
+int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns) {
+    if (!h) return VLPROJ_ERR_INVALID_ARG;
+    h->wait_ns = ns ? ns : kDefaultWaitNs;
+    return VLPROJ_OK;
+}
+
+int vlproj_status(vlproj_handle* h, void* stream) {
+    if (!h) return VLPROJ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    VLP_CUDA(cudaStreamSynchronize(s));
+    int st = 0;
+    VLP_CUDA(cudaMemcpy(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost));
+    VLP_CUDA(cudaMemset(h->status, 0, sizeof(int)));
+    return st;
+}
+
+int vlproj_hidden(vlproj_handle* h, const void* features, const int32_t* grid_hw, int32_t n_views, void* hidden,
+                  void* stream) {
+    if (!h || n_views < 0 || (n_views > 0 && (!features || !grid_hw || !hidden))) return VLPROJ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(features) % 16 || reinterpret_cast<uintptr_t>(hidden) % 16)
+        return VLPROJ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Plan pl;
+    int rc = build_plan(h->cfg, grid_hw, nullptr, n_views, true, &pl);
+    if (rc) return rc;
+    if (pl.M == 0) return VLPROJ_OK;
+    rc = upload(h, pl, plan_key(grid_hw, n_views, nullptr, n_views, 1), s);
+    if (rc) return rc;
+    return run_merge_gemm1(h, pl, features, nullptr, static_cast<__nv_bfloat16*>(hidden), s);
+}
+
+int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_hw, const int32_t* spatial_crop,
+                   int32_t n_images, const int64_t* input_ids, int64_t n_ids, int64_t image_token_id,
+                   const void* newline, const void* sep, void* out_embeds, void* stream) {
+    if (!h) return VLPROJ_ERR_INVALID_ARG;
+    const vlproj_config& c = h->cfg;
+    if (n_ids < 0 || n_ids >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
+    if (n_ids > 0 && (!input_ids || !out_embeds)) return VLPROJ_ERR_INVALID_ARG;
+    if (n_images > 0 && !features) return VLPROJ_ERR_INVALID_ARG;
+    const bool tiled = c.tile_tag == VLPROJ_TILE_2D;
+    if (tiled && n_images > 0 && (!newline || !sep)) return VLPROJ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(out_embeds) % 16 || reinterpret_cast<uintptr_t>(features) % 16 ||
+        (tiled && (reinterpret_cast<uintptr_t>(newline) % 16 || reinterpret_cast<uintptr_t>(sep) % 16)))
+        return VLPROJ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Plan pl;
+    int rc = build_plan(c, grid_hw, spatial_crop, n_images, false, &pl);
+    if (rc) return rc;
+
+    // 1. placeholder index
+    const int nblocks = static_cast<int>((n_ids + vlp::SCAN_CHUNK - 1) / vlp::SCAN_CHUNK);
+    if (h->counts.ensure(std::max(nblocks, 1)) || h->pos.ensure(std::max<int64_t>(pl.R, 1)))
+        return VLPROJ_ERR_CUDA;
+    rc = upload(h, pl, plan_key(grid_hw, static_cast<int64_t>(pl.views.size()), tiled ? spatial_crop : nullptr,
+                                n_images, tiled ? 2 : 0),
+                s);
+    if (rc) return rc;
+    h->profiled_valid = false;
+    for (bool& r : h->stage_ran) r = false;
+    mark(h, 0, s);
+    h->stage_ran[0] = true;
+    h->launches += nblocks > 0 ? 2 : 1;
+    if (nblocks > 0) {
+        vlp::vlp_count_kernel<<<nblocks, vlp::SCAN_THREADS, 0, s>>>(input_ids, n_ids, image_token_id, h->counts.ptr);
+        VLP_CUDA(cudaGetLastError());
+    }
+    vlp::vlp_compact_kernel<<<std::max(nblocks, 1), vlp::SCAN_THREADS, 0, s>>>(
+        input_ids, n_ids, image_token_id, h->counts.ptr, nblocks, h->pos.ptr, pl.R, h->status + 1, h->status);
+    VLP_CUDA(cudaGetLastError());
+    if (pl.M == 0) {
+        for (int st = 1; st <= VLPROJ_NUM_STAGES; ++st) mark(h, st, s);
+        h->profiled_valid = h->profiling;
+        return VLPROJ_OK;
+    }
+
+    // 2-4. geometry, LayerNorm, GEMM1 -> H
+    if (h->H.ensure(static_cast<size_t>(pl.M) * c.N1)) return VLPROJ_ERR_CUDA;
+    rc = run_merge_gemm1(h, pl, features, h->pos.ptr, h->H.ptr, s);
+    if (rc) return rc;
+
+    // 5. GEMM2 + scatter
+    if (h->tmH_ptr != h->H.ptr || h->tmH_rows != pl.M) {
+        if (encode_bf16_2d(&h->tmH, h->H.ptr, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
+        h->tmH_ptr = h->H.ptr;
+        h->tmH_rows = pl.M;
+    }
+    GemmParams p{};
+    p.M = static_cast<int>(pl.M);
+    p.N = c.N2;
+    p.K = c.N1;
+    p.bias = h->b2;
+    p.out = static_cast<__nv_bfloat16*>(out_embeds);
+    p.rowdest = h->rowdest.ptr;
+    p.out_rows = n_ids;
+    p.fwd_status = h->status + 1;
+    p.err = h->status;
+    p.wait_ns = h->wait_ns;
+    mark(h, 4, s);
+    h->stage_ran[4] = true;
+    ++h->launches;
+    rc = launch_gemm_bn<false, vlp::EPI_SCATTER>(pick_bn(c.N2), h->tmH, h->tmW2, p, h->num_sms, s);
+    if (rc) return rc;
+
+    // 6. newline / separator rows
+    mark(h, 5, s);
+    if (tiled && !pl.images.empty()) {
+        h->stage_ran[5] = true;
+        ++h->launches;
+        dim3 grid(pl.max_special, static_cast<unsigned>(pl.images.size()));
+        vlp::vlp_special_rows_kernel<<<grid, 128, 0, s>>>(h->dimages.ptr, h->pos.ptr, pl.R,
+                                                          static_cast<const __nv_bfloat16*>(newline),
+                                                          static_cast<const __nv_bfloat16*>(sep),
+                                                          static_cast<__nv_bfloat16*>(out_embeds), n_ids, c.N2,
+                                                          h->status + 1);
+        VLP_CUDA(cudaGetLastError());
+    }
+    mark(h, VLPROJ_NUM_STAGES, s);
+    h->profiled_valid = h->profiling;
+    return VLPROJ_OK;
+}
+
+int vlproj_profile_enable(vlproj_handle* h, int enable) {
+    if (!h) return VLPROJ_ERR_INVALID_ARG;
+    if (enable && !h->ev[0]) {
+        for (auto& e : h->ev) VLP_CUDA(cudaEventCreate(&e));
+    }
+    h->profiling = enable != 0;
+    h->profiled_valid = false;
+    return VLPROJ_OK;
+}
+
+int vlproj_profile_read(vlproj_handle* h, float* ms, int n) {
+    if (!h || !ms || n < 0) return VLPROJ_ERR_INVALID_ARG;
+    if (!h->profiled_valid) return VLPROJ_ERR_INVALID_ARG;
+    VLP_CUDA(cudaEventSynchronize(h->ev[VLPROJ_NUM_STAGES]));
+    const int m = std::min(n, VLPROJ_NUM_STAGES);
+    for (int i = 0; i < m; ++i) {
+        float t = 0.f;
+        if (h->stage_ran[i]) VLP_CUDA(cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]));
+        ms[i] = t;
+    }
+    return m;
+}
+
+int64_t vlproj_launch_count(vlproj_handle* h) { return h ? h->launches : VLPROJ_ERR_INVALID_ARG; }
+
+}  // extern "C"
