@@ -147,6 +147,18 @@ void vlproj_destroy(vlproj_handle* h);
 int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
                           const int32_t* spatial_crop, int32_t n_images, int64_t* rows_out);
 
+/* How GEMM1 fetches each merged token's k x k neighbourhood from the features:
+ *   VLPROJ_GATHER_AUTO    (default) IM2COL when every view of the batch has the same
+ *                         grid, CPASYNC otherwise (measured faster for mixed grids);
+ *   VLPROJ_GATHER_IM2COL  TMA im2col loads, the merge seen as a k x k, stride-k
+ *                         convolution window walk with hardware zero fill of the
+ *                         high-end pad; one map for a batch of same-shape views, else
+ *                         one map per view with each view's rows padded to 32;
+ *   VLPROJ_GATHER_CPASYNC 16-byte cp.async copies per row (zero-filled pad).
+ * All give the same bits. */
+enum { VLPROJ_GATHER_IM2COL = 0, VLPROJ_GATHER_CPASYNC = 1, VLPROJ_GATHER_AUTO = 2 };
+int vlproj_set_gather_mode(vlproj_handle* h, int mode);
+
 /* Bound (nanoseconds) on every wait inside this handle's kernels; 0 restores the
  * default (2 s). A wait that runs out ends its kernel early with
  * VLPROJ_ERR_TIMEOUT latched; tests use a tiny bound to exercise that path. */

@@ -43,11 +43,14 @@ SMALL = {
 }
 
 
+@pytest.mark.parametrize("gather", [vp.GATHER_AUTO, vp.GATHER_IM2COL, vp.GATHER_CPASYNC],
+                         ids=["auto", "im2col", "cpasync"])
 @pytest.mark.parametrize("name", list(SMALL))
-def test_small_case_all_rows(name):
+def test_small_case_all_rows(name, gather):
     wl, hw, gvp, order = SMALL[name]
     case = make_case(wl, np.array(hw, np.int32), gvp=gvp, k_order=order)
     proj = make_projector(case)
+    proj.set_gather_mode(gather)
     dev = DeviceInputs(case)
     out = run(case, proj, dev)
     assert proj.status() == vp.OK
@@ -58,12 +61,14 @@ def test_small_case_all_rows(name):
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("name", ["ragged_k3_ln", "tiled_head_odd", "fp32_noln"])
-def test_hidden_stage(name):
+@pytest.mark.parametrize("gather", [vp.GATHER_IM2COL, vp.GATHER_CPASYNC], ids=["im2col", "cpasync"])
+@pytest.mark.parametrize("name", ["ragged_k3_ln", "tiled_head_odd", "fp32_noln", "many_images"])
+def test_hidden_stage(name, gather):
     """Stage parity of H = bf16(GELU(A W1^T + b1)) for every merged token."""
     wl, hw, gvp, order = SMALL[name]
     case = make_case(wl, np.array(hw, np.int32), gvp=gvp, k_order=order)
     proj = make_projector(case)
+    proj.set_gather_mode(gather)
     dev = DeviceInputs(case)
     M = sum(O.tokens_untiled(h, w, wl.k) for h, w in case.hw)
     H = torch.empty((M, wl.N1), dtype=torch.bfloat16, device="cuda")
@@ -116,3 +121,17 @@ def test_gemm_ragged_edges_are_exact_zero_pad():
     proj.forward(dev_bf16(padded), np.array([[9, 9]], np.int32), None, dev.ids, W.IMAGE_TOKEN_ID, out2)
     assert proj.status() == vp.OK
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+def test_gather_modes_agree_bit_for_bit():
+    """im2col and cp.async fetch the same operand bytes, so the outputs are identical."""
+    wl = W.WORKLOADS["moonvit"]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    proj.set_gather_mode(vp.GATHER_IM2COL)
+    out_a = run(case, proj, dev)
+    proj.set_gather_mode(vp.GATHER_CPASYNC)
+    out_b = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))

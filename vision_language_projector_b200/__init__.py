@@ -25,7 +25,8 @@ ORDER_CHANNEL_OUTER, ORDER_POSITION_OUTER = 0, 1
 
 EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status", "vlproj_destroy",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
-            "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count")
+            "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode")
+GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO = 0, 1, 2
 NUM_STAGES = 6
 STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows")
 
@@ -77,6 +78,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_profile_read.restype = ctypes.c_int
     lib.vlproj_launch_count.argtypes = [P]
     lib.vlproj_launch_count.restype = I64
+    lib.vlproj_set_gather_mode.argtypes = [P, ctypes.c_int]
+    lib.vlproj_set_gather_mode.restype = ctypes.c_int
     return lib
 
 
@@ -207,6 +210,11 @@ class Projector:
 
     def launch_count(self) -> int:
         return int(_lib.vlproj_launch_count(self._h))
+
+    def set_gather_mode(self, mode: int) -> None:
+        rc = _lib.vlproj_set_gather_mode(self._h, int(mode))
+        if rc != OK:
+            raise VlprojError(rc, "vlproj_set_gather_mode")
 
     def set_wait_limit(self, ns: int) -> None:
         rc = _lib.vlproj_set_wait_limit(self._h, int(ns))

@@ -1,19 +1,24 @@
 // Projector GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM), sm_100a.
 //
-//   GEMM1 (kGather = true,  kEpi = EPI_GELU):
+//   GEMM1 (A from the patch features, EPI_GELU):
 //       H[m, n]  = bf16( GELU( sum_q A[m, q] W1p[n, q] + b1[n] ) )
 //       A is never materialised: row m of A is the k x k neighbourhood of merged
-//       token m, gathered straight from the patch features into the swizzled
-//       shared-memory operand tile (high-end pad rows are zero-filled by the copy).
-//   GEMM2 (kGather = false, kEpi = EPI_SCATTER):
+//       token m. The space-to-depth is a k x k convolution of stride k, so the A
+//       tile is fetched with TMA im2col loads straight from the channel-last
+//       features: for K-block (dy, dx, c0) one load walks the tile's tokens (base
+//       positions (k*j, k*i) of each view, wrapping rows and views) and copies
+//       channels c0..c0+63 of patch (k*i + dy, k*j + dx); patches past the grid
+//       (the high-end pad) read as zero. A_CPASYNC is the same gather done with
+//       16-byte cp.async copies (zero-filled pad), used when no im2col map fits.
+//   GEMM2 (A_TILE, EPI_SCATTER):
 //       out[dest[m], n] = bf16( sum_q H[m, q] W2[n, q] + b2[n] )
 //       the epilogue writes each row straight into its placeholder row.
 //
 // One persistent CTA per SM walks output tiles of BM x BN (N fastest, so the
 // CTAs working at the same time share the A tile through L2). Roles, by warp:
-//   warp 0      TMA producer (B always; A too when it is a dense matrix)
+//   warp 0      TMA producer (B; A in the TMA modes)
 //   warp 1      TMEM allocator and the single MMA-issuing thread
-//   warps 2-3   A gather producers (GEMM1 only): 64 threads, cp.async 16 B each
+//   warps 2-3   A gather producers in A_CPASYNC mode (64 threads)
 //   warps 4-7   epilogue: TMEM -> registers -> bias (+GELU) -> bf16 -> global
 // Shared memory holds a STAGES-deep ring of (A, B) K-blocks of 64 bf16 (128 B
 // rows, 128-byte swizzle); TMEM holds two BM x BN fp32 accumulators so the
@@ -36,6 +41,9 @@ constexpr int GEMM_THREADS = 256;
 constexpr int GATHER_THREADS = 64;
 constexpr int EPI_GELU = 0;
 constexpr int EPI_SCATTER = 1;
+constexpr int A_TILE = 0;               // dense row-major A, tiled TMA
+constexpr int A_IM2COL = 1;             // merge-gather by TMA im2col
+constexpr int A_CPASYNC = 2;            // merge-gather by cp.async
 constexpr uint64_t DRAIN_NS = 1000000000ull;
 constexpr int ERR_TIMEOUT = -5;
 
@@ -55,20 +63,25 @@ struct GemmLayout {
 };
 
 struct GemmParams {
-    int M;                          // rows (merged tokens)
+    int M;                          // rows (merged tokens, each view's run padded in im2col varlen mode)
     int N;                          // output columns
     int K;                          // reduction length, multiple of BK
     const float* bias;              // [N] fp32
-    // A gather (GEMM1)
-    const __nv_bfloat16* gsrc;      // bf16 patch features [P][C]
-    const int2* gmeta;              // per row: {top-left patch index, (w << 16) | valid mask}
     int C;                          // channels per patch; C % BK == 0
     int k;                          // merge factor
+    // A_IM2COL
+    const CUtensorMap* gmaps;       // per-view im2col maps in global memory, or null (one map: tmA)
+    int n_gmaps;
+    const int4* chunks;             // per chunk of `chunk` rows: {map, w0, h0, n0} of its first token
+    int chunk;                      // rows per im2col load: 128 (one map) or 32 (per-view maps)
+    // A_CPASYNC
+    const __nv_bfloat16* gsrc;      // bf16 patch features [P][C]
+    const int2* gmeta;              // per row: {top-left patch index, (w << 16) | valid mask}
     // output
-    __nv_bfloat16* out;             // GEMM1: H [M][N]; GEMM2: embeddings [out_rows][N]
-    const int32_t* rowdest;         // GEMM2: destination row of each m
-    int64_t out_rows;               // GEMM2: rows of the embedding buffer (bounds guard)
-    const int* fwd_status;          // GEMM2: nonzero = count check failed, write nothing
+    __nv_bfloat16* out;             // GEMM1: H; GEMM2: embeddings [out_rows][N]
+    const int32_t* rowdest;         // destination row of each m (-1 = no write), or null = row m
+    int64_t out_rows;               // rows of `out` (bounds guard)
+    const int* fwd_status;          // nonzero = count check failed, write nothing (null = ignore)
     int* err;                       // latched error word
     uint64_t wait_ns;               // bound on every wait
 };
@@ -84,12 +97,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int BN, bool kGather, int kEpi>
+template <int BN, int kAMode, int kEpi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     vlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const GemmParams p) {
     using L = GemmLayout<BN>;
     constexpr int S = L::STAGES;
+    constexpr bool kGatherThreads = kAMode == A_CPASYNC;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
@@ -121,7 +135,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmB);
-        if (!kGather) tma_prefetch_desc(&tmA);
+        if (kAMode == A_TILE || (kAMode == A_IM2COL && p.gmaps == nullptr)) tma_prefetch_desc(&tmA);
+        if (kAMode == A_IM2COL && p.gmaps != nullptr)
+            for (int i = 0; i < p.n_gmaps; ++i) tensormap_acquire(p.gmaps + i);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, L::TMEM_COLS);
@@ -136,6 +152,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int n_tiles = (p.N + BN - 1) / BN;
     const int num_tiles = m_tiles * n_tiles;
     const int kblocks = p.K / BK;
+    const int cblocks = p.C / BK;
     const uint64_t lim = p.wait_ns;
 
     if (warp == 0) {
@@ -145,14 +162,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
+            const int nch = (kAMode == A_IM2COL) ? BM / p.chunk : 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
+                int4 ch[4] = {};
+                if (kAMode == A_IM2COL)
+                    for (int q = 0; q < nch; ++q) ch[q] = __ldg(&p.chunks[m_blk * nch + q]);
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag)) { ok = false; break; }
                     uint8_t* sa = smem + stage * L::STAGE_BYTES;
                     uint8_t* sb = sa + L::A_BYTES;
-                    mbar_arrive_expect_tx(&full_tma[stage], (kGather ? 0 : L::A_BYTES) + L::B_BYTES);
-                    if (!kGather) tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, m_blk * BM);
+                    mbar_arrive_expect_tx(&full_tma[stage], (kAMode == A_CPASYNC ? 0 : L::A_BYTES) + L::B_BYTES);
+                    if (kAMode == A_TILE) {
+                        tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, m_blk * BM);
+                    } else if (kAMode == A_IM2COL) {
+                        const int pos = kb / cblocks;                  // (dy, dx) position index
+                        const int c0 = (kb - pos * cblocks) * BK;
+                        const int dy = pos / p.k, dx = pos - dy * p.k;
+                        for (int q = 0; q < nch; ++q) {
+                            const CUtensorMap* mp = p.gmaps ? p.gmaps + ch[q].x : &tmA;
+                            tma_load_im2col_4d(sa + q * p.chunk * 128, mp, &full_tma[stage], c0, ch[q].y, ch[q].z,
+                                               ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
+                        }
+                    }
                     tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, n_blk * BN);
                     ++issued;
                     if (++stage == S) { stage = 0; phase ^= 1; }
@@ -188,7 +220,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full_tma[stage], phase, lim, abort_flag)) { ok = false; break; }
-                    if (kGather) {
+                    if (kGatherThreads) {
                         if (!mbar_wait_bounded(&full_gat[stage], phase, lim, abort_flag)) { ok = false; break; }
                         fence_proxy_async_smem();
                     }
@@ -217,13 +249,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_wait_bounded(drain, 0, DRAIN_NS, &never);
         }
     } else if (warp < 4) {
-        // ------------------------------------------------ A gather producers (GEMM1)
-        if (kGather) {
+        // ------------------------------------------------ A gather producers (A_CPASYNC)
+        if (kGatherThreads) {
             const int gt = threadIdx.x - 64;          // 0..63
             const int chunk = gt & 7;                 // 16-byte chunk of the 128-byte row
             const int rsub = gt >> 3;                 // rows rsub, rsub+8, ..., rsub+120
             const uint32_t swz = static_cast<uint32_t>((chunk ^ rsub) * 16);
-            const int cblocks = p.C / BK;
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -244,7 +275,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                 }
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    const int pos = kb / cblocks;                  // (dy, dx) position index
+                    const int pos = kb / cblocks;
                     const int c0 = (kb - pos * cblocks) * BK + chunk * 8;
                     const int dy = pos / p.k, dx = pos - dy * p.k;
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag)) { ok = false; break; }
@@ -275,8 +306,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        int status_ok = 1;
-        if (kEpi == EPI_SCATTER) status_ok = (*p.fwd_status == 0);
+        const int status_ok = p.fwd_status ? (*p.fwd_status == 0) : 1;
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
             // one lane waits, the warp follows it, so tcgen05.ld below is never divergent
@@ -286,15 +316,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (!got) { ok = false; break; }
             tc_fence_after();
             const int m = m_blk * BM + row;
-            bool row_ok = m < p.M;
-            __nv_bfloat16* dst_row = nullptr;
-            if (kEpi == EPI_SCATTER) {
-                int64_t d = row_ok ? static_cast<int64_t>(__ldg(&p.rowdest[m])) : -1;
-                row_ok = row_ok && status_ok && d >= 0 && d < p.out_rows;
-                if (row_ok) dst_row = p.out + d * p.N;
-            } else {
-                if (row_ok) dst_row = p.out + static_cast<int64_t>(m) * p.N;
-            }
+            bool row_ok = m < p.M && status_ok;
+            int64_t d = m;
+            if (row_ok && p.rowdest) d = __ldg(&p.rowdest[m]);
+            row_ok = row_ok && d >= 0 && d < p.out_rows;
+            __nv_bfloat16* dst_row = row_ok ? p.out + d * p.N : nullptr;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {

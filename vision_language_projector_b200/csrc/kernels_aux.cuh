@@ -98,14 +98,14 @@ __global__ void __launch_bounds__(SCAN_THREADS) vlp_compact_kernel(const int64_t
 // ---------------------------------------------------------------- geometry
 struct ViewDesc {
     int64_t patch_start;   // first patch row of the view in the packed features
-    int32_t tok_start;     // first merged token (GEMM row) of the view
+    int32_t tok_start;     // first GEMM row of the view (runs padded to the im2col chunk when varlen)
+    int32_t tok_real;      // merged tokens of all earlier views (no padding)
     int32_t h, w;          // patch grid
     int32_t hp, wp;        // merged grid: ceil(h/k), ceil(w/k)
     int32_t row_base;      // first assembled row of the view's image (over all images)
     int32_t view_in_image; // 0 = global view (or the only view), t+1 = local tile t
     int32_t tw, th;        // image tiling (0 when untiled)
     int32_t tail;          // 2D tiling with the global view after the local tiles
-    int32_t pad_;
 };
 
 // Assembled row (inside the image) of merged token (i, j) of a view.
@@ -121,28 +121,62 @@ __device__ __forceinline__ int64_t assembled_row(const ViewDesc& V, int i, int j
     return l0 + (static_cast<int64_t>(ty) * V.hp + i) * local_cols + static_cast<int64_t>(tx) * V.wp + j;
 }
 
-__global__ void __launch_bounds__(256) vlp_geometry_kernel(const ViewDesc* __restrict__ views, int n_views, int M,
-                                                           int k, const int32_t* __restrict__ pos, int64_t R,
-                                                           int2* __restrict__ gmeta, int32_t* __restrict__ rowdest) {
-    const int m = blockIdx.x * blockDim.x + threadIdx.x;
-    if (m >= M) return;
+__device__ __forceinline__ int find_view(const ViewDesc* views, int n_views, int m) {
     int lo = 0, hi = n_views - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (views[mid].tok_start <= m) lo = mid; else hi = mid - 1;
     }
-    const ViewDesc V = views[lo];
+    return lo;
+}
+
+constexpr int DEST_NONE = 0;      // no destination table
+constexpr int DEST_EMBED = 1;     // rowdest[m] = embedding row of the placeholder that takes token m
+constexpr int DEST_COMPACT = 2;   // rowdest[m] = merged-token index (views in order, no padding)
+
+// One thread per GEMM row m (and per im2col chunk): gather metadata for the cp.async
+// path, the destination of the row, and the im2col coordinates of each chunk's
+// first token. Rows in a view's padding get no destination and zero gather masks.
+__global__ void __launch_bounds__(256) vlp_geometry_kernel(const ViewDesc* __restrict__ views, int n_views, int M,
+                                                           int k, const int32_t* __restrict__ pos, int64_t R,
+                                                           int dest_mode, int2* __restrict__ gmeta,
+                                                           int32_t* __restrict__ rowdest, int4* __restrict__ chunks,
+                                                           int n_chunks, int chunk, int uniform) {
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m < n_chunks) {
+        const int first = m * chunk;
+        int4 e;
+        if (first >= M) {
+            // past the last GEMM row: any in-range start will do, these rows are never stored
+            e = make_int4(0, 0, 0, 0);
+        } else {
+            const int v = find_view(views, n_views, first);
+            const ViewDesc& V = views[v];
+            const int t = first - V.tok_start;
+            const int i = t / V.wp, j = t - (t / V.wp) * V.wp;
+            e = uniform ? make_int4(0, k * j, k * i, v) : make_int4(v, k * j, k * i, 0);
+        }
+        if (chunks != nullptr) chunks[m] = e;
+    }
+    if (m >= M) return;
+    const ViewDesc V = views[find_view(views, n_views, m)];
     const int t = m - V.tok_start;
-    const int i = t / V.wp, j = t - i * V.wp;
-    const int64_t base = V.patch_start + static_cast<int64_t>(k * i) * V.w + k * j;
-    uint32_t mask = 0;
-    for (int dy = 0; dy < k; ++dy)
-        for (int dx = 0; dx < k; ++dx)
-            if (k * i + dy < V.h && k * j + dx < V.w) mask |= 1u << (dy * k + dx);
-    gmeta[m] = make_int2(static_cast<int>(base), static_cast<int>((static_cast<uint32_t>(V.w) << 16) | mask));
-    if (rowdest != nullptr) {
+    const bool real = t < V.hp * V.wp;
+    const int i = real ? t / V.wp : 0, j = real ? t - i * V.wp : 0;
+    if (gmeta != nullptr) {
+        const int64_t base = V.patch_start + static_cast<int64_t>(k * i) * V.w + k * j;
+        uint32_t mask = 0;
+        if (real)
+            for (int dy = 0; dy < k; ++dy)
+                for (int dx = 0; dx < k; ++dx)
+                    if (k * i + dy < V.h && k * j + dx < V.w) mask |= 1u << (dy * k + dx);
+        gmeta[m] = make_int2(static_cast<int>(base), static_cast<int>((static_cast<uint32_t>(V.w) << 16) | mask));
+    }
+    if (dest_mode == DEST_EMBED) {
         const int64_t g = V.row_base + assembled_row(V, i, j);
-        rowdest[m] = (g >= 0 && g < R) ? pos[g] : -1;
+        rowdest[m] = (real && g >= 0 && g < R) ? pos[g] : -1;
+    } else if (dest_mode == DEST_COMPACT) {
+        rowdest[m] = real ? V.tok_real + t : -1;
     }
 }
 

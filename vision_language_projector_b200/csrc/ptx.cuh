@@ -77,6 +77,28 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_
         : "memory");
 }
 
+// im2col load from a 4D channel-last tensor map (C, W, H, N): walks `pixels per
+// column` base positions starting at (w, h, n) with the map's traversal strides,
+// wrapping along W, then H, then N inside the map's bounding box, and for each base
+// position copies channels [c, c + channels per pixel) of pixel (w + off_w, h + off_h, n)
+// as one row; pixels outside the tensor read as zero. Rows land consecutively at dst.
+__device__ __forceinline__ void tma_load_im2col_4d(void* dst, const void* tmap, uint64_t* bar, int32_t c, int32_t w,
+                                                   int32_t h, int32_t n, uint16_t off_w, uint16_t off_h) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.im2col.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2], {%7, %8};" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c), "r"(w), "r"(h), "r"(n), "h"(off_w),
+        "h"(off_h)
+        : "memory");
+}
+
+// Make generic-proxy writes of a tensor map in global memory (written before this
+// kernel started) visible to the tensor-map proxy before TMA uses it.
+__device__ __forceinline__ void tensormap_acquire(const void* gmap) {
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(gmap))
+                 : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async gather
 // 16-byte global -> shared copy; src_bytes = 0 writes 16 zero bytes (no read).
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {

@@ -1,14 +1,15 @@
 // C-ABI host library of the vision-to-language projector (declared in vlproj.h).
 //
 // vlproj_forward enqueues, on the caller's stream and without any host sync:
-//   1. placeholder index   count + compact (ids == image_token_id), count check
-//   2. geometry            per merged token: gather metadata and destination row
-//   3. LayerNorm/convert   only with a pre-merge LayerNorm or fp32 features
-//   4. GEMM1               gather + tcgen05 MMA + bias + GELU -> H (bf16)
-//   5. GEMM2               tcgen05 MMA + bias -> bf16 rows scattered into out_embeds
-//   6. special rows        newline / separator rows (2D tiling only)
-// Host work per call: argument checks, the closed-form row counts, one small
-// descriptor upload, and tensor-map encoding for H (cached while it is unchanged).
+//   0. placeholder index   count + compact (ids == image_token_id), count check
+//   1. geometry            per GEMM row: destination row; per im2col chunk: the
+//                          coordinates of its first token
+//   2. LayerNorm/convert   only with a pre-merge LayerNorm or fp32 features
+//   3. GEMM1               im2col merge-gather + tcgen05 MMA + bias + GELU -> H (bf16)
+//   4. GEMM2               tcgen05 MMA + bias -> bf16 rows scattered into out_embeds
+//   5. special rows        newline / separator rows (2D tiling only)
+// Host work per call: argument checks, the closed-form row counts, tensor-map
+// encoding, and small descriptor uploads that are skipped while unchanged.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -42,29 +43,60 @@ constexpr uint64_t kDefaultWaitNs = 2000000000ull;
         }                                                                                     \
     } while (0)
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+struct DriverFns {
+    PFN_cuTensorMapEncodeTiled_v12000 tiled = nullptr;
+    PFN_cuTensorMapEncodeIm2col_v12000 im2col = nullptr;
+};
+
+const DriverFns& driver() {
+    static DriverFns fns;
     static std::once_flag once;
     std::call_once(once, [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+            fns.tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeIm2col", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fns.im2col = reinterpret_cast<PFN_cuTensorMapEncodeIm2col_v12000>(p);
     });
-    return fn;
+    return fns;
 }
 
 // 2D bf16 row-major matrix [rows][cols], box = box_rows x 64 columns, 128-byte swizzle,
 // out-of-range elements read as zero.
 int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    auto fn = get_encode_fn();
+    auto fn = driver().tiled;
     if (!fn) return VLPROJ_ERR_CUDA;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
     cuuint32_t box[2] = {static_cast<cuuint32_t>(vlp::BK), box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
+// im2col map of n views of one (h, w) grid of C-channel bf16 patches, packed back to
+// back from `base`: the k x k, stride-k window walk of the merge. Base positions run
+// over 0, k, ..., k*(w'-1) (lower corner 0, upper corner k*w' - w - (k-1), the
+// convolution form of "pad the high end to k*w'"), `pixels` per load, 64 channels each.
+int encode_im2col(CUtensorMap* map, const void* base, int C, int h, int w, int n, int k, int pixels) {
+    auto fn = driver().im2col;
+    if (!fn) return VLPROJ_ERR_CUDA;
+    const int hp = (h + k - 1) / k, wp = (w + k - 1) / k;
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(w), static_cast<cuuint64_t>(h),
+                          static_cast<cuuint64_t>(n)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(w) * C * 2,
+                             static_cast<cuuint64_t>(h) * w * C * 2};
+    int lower[2] = {0, 0};
+    int upper[2] = {k * wp - w - (k - 1), k * hp - h - (k - 1)};
+    cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(k), static_cast<cuuint32_t>(k), 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, lower, upper,
+                    static_cast<cuuint32_t>(vlp::BK), static_cast<cuuint32_t>(pixels), estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
@@ -91,13 +123,61 @@ struct DevBuf {
     }
 };
 
+// Pinned host staging for small per-call uploads: reused only after the previous
+// copy out of it has executed; skipped when the bytes equal the last upload.
+struct Uploader {
+    uint8_t* staging = nullptr;
+    size_t cap = 0;
+    cudaEvent_t done = nullptr;
+    std::vector<uint8_t> last;
+    bool valid = false;
+    int put(void* dst, const void* src, size_t bytes, cudaStream_t s) {
+        if (valid && last.size() == bytes && std::memcmp(last.data(), src, bytes) == 0) {
+            // unchanged: the device copy is (or will be) there; order `s` after it
+            if (done && bytes) VLP_CUDA(cudaStreamWaitEvent(s, done, 0));
+            return VLPROJ_OK;
+        }
+        valid = false;
+        if (bytes == 0) return VLPROJ_OK;
+        if (!done) VLP_CUDA(cudaEventCreateWithFlags(&done, cudaEventDisableTiming));
+        VLP_CUDA(cudaEventSynchronize(done));
+        if (bytes > cap) {
+            if (staging) cudaFreeHost(staging);
+            staging = nullptr;
+            cap = 0;
+            VLP_CUDA(cudaMallocHost(&staging, bytes * 2));
+            cap = bytes * 2;
+        }
+        std::memcpy(staging, src, bytes);
+        VLP_CUDA(cudaMemcpyAsync(dst, staging, bytes, cudaMemcpyHostToDevice, s));
+        VLP_CUDA(cudaEventRecord(done, s));
+        last.assign(static_cast<const uint8_t*>(src), static_cast<const uint8_t*>(src) + bytes);
+        valid = true;
+        return VLPROJ_OK;
+    }
+    void invalidate() { valid = false; }
+    void release() {
+        if (done) cudaEventSynchronize(done);
+        if (staging) cudaFreeHost(staging);
+        if (done) cudaEventDestroy(done);
+        staging = nullptr;
+        done = nullptr;
+        cap = 0;
+        valid = false;
+    }
+};
+
 struct Plan {
     std::vector<ViewDesc> views;
     std::vector<ImageDesc> images;
-    int64_t M = 0;          // merged tokens
+    int64_t M = 0;          // GEMM rows (merged tokens, varlen im2col runs padded to `chunk`)
+    int64_t M_real = 0;     // merged tokens
     int64_t R = 0;          // assembled rows
     int64_t P = 0;          // patches
     int max_special = 0;    // most special rows of one image
+    bool uniform = true;    // every view has the same grid
+    bool im2col = true;     // GEMM1 gathers with TMA im2col (else cp.async)
+    int chunk = 128;        // im2col rows per load
 };
 
 int validate_config(const vlproj_config* c) {
@@ -118,8 +198,11 @@ int validate_config(const vlproj_config* c) {
 }
 
 // Closed-form geometry of one batch. Returns an error for inconsistent shapes.
+// gather_mode (VLPROJ_GATHER_*) resolves to im2col or cp.async here (plan.im2col);
+// with im2col and views of different grids each view's run of GEMM rows is padded to
+// a multiple of 32, so the im2col loads of per-view maps never straddle two views.
 int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int32_t* crop, int32_t n_images,
-               bool tiled_override_none, Plan* out) {
+               bool tiled_override_none, int gather_mode, Plan* out) {
     Plan& pl = *out;
     pl = Plan();
     if (n_images < 0) return VLPROJ_ERR_INVALID_ARG;
@@ -127,33 +210,53 @@ int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int32_t* cr
     const bool tiled = !tiled_override_none && c.tile_tag == VLPROJ_TILE_2D;
     if (tiled && n_images > 0 && !crop) return VLPROJ_ERR_INVALID_ARG;
     const int k = c.k;
-    int64_t v = 0;
+    // first pass: view count, shapes, uniformity
+    int64_t n_views = 0;
     for (int32_t img = 0; img < n_images; ++img) {
         const int tw = tiled ? crop[2 * img] : 0;
         const int th = tiled ? crop[2 * img + 1] : 0;
         if (tiled && (tw < 1 || th < 1 || static_cast<int64_t>(tw) * th > 4096)) return VLPROJ_ERR_INVALID_ARG;
+        n_views += tiled ? 1 + tw * th : 1;
+    }
+    for (int64_t v = 0; v < n_views; ++v) {
+        const int h = grid_hw[2 * v], w = grid_hw[2 * v + 1];
+        if (h < 1 || w < 1 || h > 65535 || w > 65535) return VLPROJ_ERR_INVALID_ARG;
+        if (h != grid_hw[0] || w != grid_hw[1]) pl.uniform = false;
+    }
+    pl.chunk = pl.uniform ? 128 : 32;
+    pl.im2col = gather_mode == VLPROJ_GATHER_IM2COL || (gather_mode == VLPROJ_GATHER_AUTO && pl.uniform);
+    const int pad_to = (pl.im2col && !pl.uniform) ? pl.chunk : 1;
+    int64_t v = 0;
+    for (int32_t img = 0; img < n_images; ++img) {
+        const int tw = tiled ? crop[2 * img] : 0;
+        const int th = tiled ? crop[2 * img + 1] : 0;
         const int nv = tiled ? 1 + tw * th : 1;
         const int h0 = grid_hw[2 * v], w0 = grid_hw[2 * v + 1];
-        if (h0 < 1 || w0 < 1 || h0 > 65535 || w0 > 65535) return VLPROJ_ERR_INVALID_ARG;
         const int hp = (h0 + k - 1) / k, wp = (w0 + k - 1) / k;
         int64_t rows;
-        if (tiled) rows = static_cast<int64_t>(hp) * (wp + 1) + 1 + static_cast<int64_t>(th) * hp * (static_cast<int64_t>(tw) * wp + 1);
-        else rows = static_cast<int64_t>(hp) * wp;
+        if (tiled)
+            rows = static_cast<int64_t>(hp) * (wp + 1) + 1 +
+                   static_cast<int64_t>(th) * hp * (static_cast<int64_t>(tw) * wp + 1);
+        else
+            rows = static_cast<int64_t>(hp) * wp;
         for (int t = 0; t < nv; ++t, ++v) {
             const int h = grid_hw[2 * v], w = grid_hw[2 * v + 1];
             if (h != h0 || w != w0) return VLPROJ_ERR_INVALID_ARG;   // views of one image share a grid
             ViewDesc d{};
             d.patch_start = pl.P;
             d.tok_start = static_cast<int32_t>(pl.M);
+            d.tok_real = static_cast<int32_t>(pl.M_real);
             d.h = h; d.w = w; d.hp = hp; d.wp = wp;
             d.row_base = static_cast<int32_t>(pl.R);
             d.view_in_image = t;
             d.tw = tw; d.th = th;
             d.tail = tiled && c.global_view_pos == VLPROJ_GLOBAL_TAIL;
             pl.views.push_back(d);
+            const int64_t toks = static_cast<int64_t>(hp) * wp;
             pl.P += static_cast<int64_t>(h) * w;
-            pl.M += static_cast<int64_t>(hp) * wp;
-            if (pl.P >= (int64_t(1) << 31) || pl.M >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
+            pl.M_real += toks;
+            pl.M += (toks + pad_to - 1) / pad_to * pad_to;
+            if (pl.P >= (int64_t(1) << 31) || pl.M >= (int64_t(1) << 30)) return VLPROJ_ERR_INVALID_ARG;
         }
         if (tiled) {
             ImageDesc im{};
@@ -169,24 +272,24 @@ int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int32_t* cr
     return VLPROJ_OK;
 }
 
-template <int BN, bool G, int E>
+template <int BN, int A, int E>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int num_sms, cudaStream_t s) {
     using L = GemmLayout<BN>;
-    VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_gemm_kernel<BN, G, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_gemm_kernel<BN, A, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   L::SMEM_ALLOC));
     const int tiles = ((p.M + vlp::BM - 1) / vlp::BM) * ((p.N + BN - 1) / BN);
     const int grid = std::min(tiles, num_sms);
     if (grid <= 0) return VLPROJ_OK;
-    vlp::vlp_gemm_kernel<BN, G, E><<<grid, vlp::GEMM_THREADS, L::SMEM_ALLOC, s>>>(ta, tb, p);
+    vlp::vlp_gemm_kernel<BN, A, E><<<grid, vlp::GEMM_THREADS, L::SMEM_ALLOC, s>>>(ta, tb, p);
     VLP_CUDA(cudaGetLastError());
     return VLPROJ_OK;
 }
 
-template <bool G, int E>
+template <int A, int E>
 int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int num_sms,
                    cudaStream_t s) {
-    if (bn == 256) return launch_gemm<256, G, E>(ta, tb, p, num_sms, s);
-    return launch_gemm<128, G, E>(ta, tb, p, num_sms, s);
+    if (bn == 256) return launch_gemm<256, A, E>(ta, tb, p, num_sms, s);
+    return launch_gemm<128, A, E>(ta, tb, p, num_sms, s);
 }
 
 int pick_bn(int N) { return N >= 256 ? 256 : 128; }
@@ -199,6 +302,7 @@ struct vlproj_handle {
     int num_sms = 148;
     int K1 = 0;
     uint64_t wait_ns = kDefaultWaitNs;
+    int gather_mode = VLPROJ_GATHER_AUTO;
     __nv_bfloat16* W1p = nullptr;
     __nv_bfloat16* W2 = nullptr;
     float* b1 = nullptr;
@@ -210,15 +314,13 @@ struct vlproj_handle {
     DevBuf<__nv_bfloat16> H, Xn;
     DevBuf<int32_t> pos, rowdest, counts;
     DevBuf<int2> gmeta;
+    DevBuf<int4> chunks;
     DevBuf<ViewDesc> dviews;
     DevBuf<ImageDesc> dimages;
+    DevBuf<CUtensorMap> dmaps;
     int* status = nullptr;       // [0] latched error, [1] per-forward count check
-    // pinned staging for the per-call descriptors, guarded by an event
-    uint8_t* staging = nullptr;
-    size_t staging_cap = 0;
-    cudaEvent_t staging_done = nullptr;
-    // geometry key of the descriptors now on the device (skip re-upload when unchanged)
-    std::vector<int32_t> uploaded_key;
+    Uploader up_views, up_images, up_maps;
+    std::vector<CUtensorMap> host_maps;
     // tracing
     bool profiling = false;
     bool profiled_valid = false;
@@ -238,57 +340,39 @@ void mark(vlproj_handle* h, int stage, cudaStream_t s) {
     if (h->profiling) cudaEventRecord(h->ev[stage], s);
 }
 
-std::vector<int32_t> plan_key(const int32_t* grid_hw, int64_t n_views, const int32_t* crop, int32_t n_images,
-                              int32_t mode) {
-    std::vector<int32_t> key;
-    key.reserve(static_cast<size_t>(2 * n_views + 2 * n_images + 2));
-    key.push_back(mode);
-    key.push_back(n_images);
-    for (int64_t i = 0; i < 2 * n_views; ++i) key.push_back(grid_hw[i]);
-    if (crop)
-        for (int64_t i = 0; i < 2 * n_images; ++i) key.push_back(crop[i]);
-    return key;
-}
-
-int upload(vlproj_handle* h, const Plan& pl, std::vector<int32_t>&& key, cudaStream_t s) {
-    if (key == h->uploaded_key) return VLPROJ_OK;
-    h->uploaded_key.clear();
-    const size_t vb = pl.views.size() * sizeof(ViewDesc);
-    const size_t ib = pl.images.size() * sizeof(ImageDesc);
-    const size_t need = vb + ib + 64;
-    VLP_CUDA(cudaEventSynchronize(h->staging_done));   // the previous upload has left the staging area
-    if (need > h->staging_cap) {
-        if (h->staging) cudaFreeHost(h->staging);
-        h->staging = nullptr;
-        h->staging_cap = 0;
-        VLP_CUDA(cudaMallocHost(&h->staging, need * 2));
-        h->staging_cap = need * 2;
-    }
+int upload_plan(vlproj_handle* h, const Plan& pl, cudaStream_t s) {
+    if (h->dviews.ptr == nullptr || h->dviews.cap < pl.views.size()) h->up_views.invalidate();
+    if (h->dimages.ptr == nullptr || h->dimages.cap < pl.images.size()) h->up_images.invalidate();
     if (h->dviews.ensure(std::max<size_t>(pl.views.size(), 1))) return VLPROJ_ERR_CUDA;
     if (h->dimages.ensure(std::max<size_t>(pl.images.size(), 1))) return VLPROJ_ERR_CUDA;
-    if (vb) std::memcpy(h->staging, pl.views.data(), vb);
-    if (ib) std::memcpy(h->staging + vb, pl.images.data(), ib);
-    if (vb) VLP_CUDA(cudaMemcpyAsync(h->dviews.ptr, h->staging, vb, cudaMemcpyHostToDevice, s));
-    if (ib) VLP_CUDA(cudaMemcpyAsync(h->dimages.ptr, h->staging + vb, ib, cudaMemcpyHostToDevice, s));
-    VLP_CUDA(cudaEventRecord(h->staging_done, s));
-    h->uploaded_key = std::move(key);
-    return VLPROJ_OK;
+    int rc = h->up_views.put(h->dviews.ptr, pl.views.data(), pl.views.size() * sizeof(ViewDesc), s);
+    if (rc) return rc;
+    return h->up_images.put(h->dimages.ptr, pl.images.data(), pl.images.size() * sizeof(ImageDesc), s);
 }
 
-// Steps 2-4: geometry (+ destinations when pos is given), LayerNorm/convert, GEMM1 into `hidden`.
-int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, const int32_t* pos,
-                    __nv_bfloat16* hidden, cudaStream_t s) {
+// Steps 1-3: geometry, LayerNorm/convert, GEMM1. GEMM row m goes to
+//   dest_mode DEST_EMBED:   hidden row m (internal H, M rows); pos gives rowdest for GEMM2
+//   dest_mode DEST_COMPACT: hidden row = merged-token index (caller's buffer, M_real rows)
+int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, const int32_t* pos, int dest_mode,
+                    __nv_bfloat16* hidden, int64_t hidden_rows, cudaStream_t s) {
     const vlproj_config& c = h->cfg;
     const int M = static_cast<int>(pl.M);
     if (M == 0) return VLPROJ_OK;
-    if (h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
-    if (pos && h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
+    const bool im2col = pl.im2col;
+    const int nch_tile = vlp::BM / pl.chunk;
+    const int n_chunks = im2col ? ((M + vlp::BM - 1) / vlp::BM) * nch_tile : 0;
+    if (h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
+    if (!im2col && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
+    if (im2col && h->chunks.ensure(std::max(n_chunks, 1))) return VLPROJ_ERR_CUDA;
+
     mark(h, 1, s);
     h->stage_ran[1] = true;
     ++h->launches;
-    vlp::vlp_geometry_kernel<<<(M + 255) / 256, 256, 0, s>>>(h->dviews.ptr, static_cast<int>(pl.views.size()), M,
-                                                             c.k, pos, pl.R, h->gmeta.ptr,
-                                                             pos ? h->rowdest.ptr : nullptr);
+    const int geo_threads = std::max(M, n_chunks);
+    vlp::vlp_geometry_kernel<<<(geo_threads + 255) / 256, 256, 0, s>>>(
+        h->dviews.ptr, static_cast<int>(pl.views.size()), M, c.k, pos, pl.R, dest_mode,
+        im2col ? nullptr : h->gmeta.ptr, h->rowdest.ptr, im2col ? h->chunks.ptr : nullptr, n_chunks, pl.chunk,
+        pl.uniform ? 1 : 0);
     VLP_CUDA(cudaGetLastError());
 
     const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(features);
@@ -314,19 +398,50 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     p.N = c.N1;
     p.K = h->K1;
     p.bias = h->b1;
-    p.gsrc = src;
-    p.gmeta = h->gmeta.ptr;
     p.C = c.C;
     p.k = c.k;
     p.out = hidden;
+    p.rowdest = dest_mode == vlp::DEST_COMPACT ? h->rowdest.ptr : nullptr;
+    p.out_rows = hidden_rows;
+    p.fwd_status = nullptr;
     p.err = h->status;
     p.wait_ns = h->wait_ns;
-    CUtensorMap unused{};
-    std::memset(&unused, 0, sizeof(unused));
+
+    CUtensorMap tmA{};
+    std::memset(&tmA, 0, sizeof(tmA));
+    if (im2col) {
+        p.chunks = h->chunks.ptr;
+        p.chunk = pl.chunk;
+        if (pl.uniform) {
+            const ViewDesc& V = pl.views[0];
+            if (encode_im2col(&tmA, src, c.C, V.h, V.w, static_cast<int>(pl.views.size()), c.k, pl.chunk))
+                return VLPROJ_ERR_CUDA;
+            p.gmaps = nullptr;
+            p.n_gmaps = 0;
+        } else {
+            h->host_maps.resize(pl.views.size());
+            for (size_t v = 0; v < pl.views.size(); ++v) {
+                const ViewDesc& V = pl.views[v];
+                if (encode_im2col(&h->host_maps[v], src + V.patch_start * c.C, c.C, V.h, V.w, 1, c.k, pl.chunk))
+                    return VLPROJ_ERR_CUDA;
+            }
+            if (h->dmaps.ptr == nullptr || h->dmaps.cap < pl.views.size()) h->up_maps.invalidate();
+            if (h->dmaps.ensure(pl.views.size())) return VLPROJ_ERR_CUDA;
+            int rc = h->up_maps.put(h->dmaps.ptr, h->host_maps.data(), pl.views.size() * sizeof(CUtensorMap), s);
+            if (rc) return rc;
+            p.gmaps = h->dmaps.ptr;
+            p.n_gmaps = static_cast<int>(pl.views.size());
+        }
+    } else {
+        p.gsrc = src;
+        p.gmeta = h->gmeta.ptr;
+    }
+
     mark(h, 3, s);
     h->stage_ran[3] = true;
     ++h->launches;
-    return launch_gemm_bn<true, vlp::EPI_GELU>(pick_bn(c.N1), unused, h->tmW1, p, h->num_sms, s);
+    if (im2col) return launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(pick_bn(c.N1), tmA, h->tmW1, p, h->num_sms, s);
+    return launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(pick_bn(c.N1), tmA, h->tmW1, p, h->num_sms, s);
 }
 
 }  // namespace
@@ -345,14 +460,14 @@ const char* vlproj_strerror(int code) {
     }
 }
 
-const char* vlproj_version(void) { return "vlproj 0.1 sm_100a"; }
+const char* vlproj_version(void) { return "vlproj 0.2 sm_100a"; }
 
 int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw, const int32_t* spatial_crop,
                           int32_t n_images, int64_t* rows_out) {
     int rc = validate_config(cfg);
     if (rc) return rc;
     Plan pl;
-    rc = build_plan(*cfg, grid_hw, spatial_crop, n_images, false, &pl);
+    rc = build_plan(*cfg, grid_hw, spatial_crop, n_images, false, VLPROJ_GATHER_CPASYNC, &pl);
     if (rc) return rc;
     if (rows_out) {
         // rows of image i = (row_base of the next image) - (its own)
@@ -374,7 +489,7 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
     int rc = validate_config(cfg);
     if (rc) return rc;
     if (!cfg->W1 || !cfg->W2 || (cfg->has_ln && (!cfg->ln_gamma || !cfg->ln_beta))) return VLPROJ_ERR_INVALID_ARG;
-    if (!get_encode_fn()) return VLPROJ_ERR_CUDA;
+    if (!driver().tiled || !driver().im2col) return VLPROJ_ERR_CUDA;
 
     vlproj_handle* h = new vlproj_handle();
     h->cfg = *cfg;
@@ -389,7 +504,7 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
     const size_t n1 = static_cast<size_t>(cfg->N1), n2 = static_cast<size_t>(cfg->N2), C = static_cast<size_t>(cfg->C);
     if (cudaMalloc(&h->W1p, n1 * h->K1 * 2) || cudaMalloc(&h->W2, n2 * n1 * 2) || cudaMalloc(&h->b1, n1 * 4) ||
         cudaMalloc(&h->b2, n2 * 4) || cudaMalloc(&h->gamma, C * 4) || cudaMalloc(&h->beta, C * 4) ||
-        cudaMalloc(&h->status, 2 * sizeof(int)) || cudaEventCreateWithFlags(&h->staging_done, cudaEventDisableTiming))
+        cudaMalloc(&h->status, 2 * sizeof(int)))
         return fail(VLPROJ_ERR_CUDA);
     cudaStream_t s = nullptr;
     vlp::vlp_permute_w1_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(cfg->W1), h->W1p,
@@ -410,7 +525,7 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
         return fail(VLPROJ_ERR_CUDA);
     }
     if (cudaMemset(h->status, 0, 2 * sizeof(int))) return fail(VLPROJ_ERR_CUDA);
-    if (cudaEventRecord(h->staging_done, s) || cudaDeviceSynchronize()) return fail(VLPROJ_ERR_CUDA);
+    if (cudaDeviceSynchronize()) return fail(VLPROJ_ERR_CUDA);
     if (encode_bf16_2d(&h->tmW1, h->W1p, n1, h->K1, pick_bn(cfg->N1)) ||
         encode_bf16_2d(&h->tmW2, h->W2, n2, n1, pick_bn(cfg->N2)))
         return fail(VLPROJ_ERR_CUDA);
@@ -437,10 +552,13 @@ void vlproj_destroy(vlproj_handle* h) {
     h->rowdest.release();
     h->counts.release();
     h->gmeta.release();
+    h->chunks.release();
     h->dviews.release();
     h->dimages.release();
-    if (h->staging) cudaFreeHost(h->staging);
-    if (h->staging_done) cudaEventDestroy(h->staging_done);
+    h->dmaps.release();
+    h->up_views.release();
+    h->up_images.release();
+    h->up_maps.release();
     for (auto& e : h->ev)
         if (e) cudaEventDestroy(e);
     cudaSetDevice(cur);
@@ -450,6 +568,13 @@ void vlproj_destroy(vlproj_handle* h) {
 int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns) {
     if (!h) return VLPROJ_ERR_INVALID_ARG;
     h->wait_ns = ns ? ns : kDefaultWaitNs;
+    return VLPROJ_OK;
+}
+
+int vlproj_set_gather_mode(vlproj_handle* h, int mode) {
+    if (!h || (mode != VLPROJ_GATHER_IM2COL && mode != VLPROJ_GATHER_CPASYNC && mode != VLPROJ_GATHER_AUTO))
+        return VLPROJ_ERR_INVALID_ARG;
+    h->gather_mode = mode;
     return VLPROJ_OK;
 }
 
@@ -470,12 +595,14 @@ int vlproj_hidden(vlproj_handle* h, const void* features, const int32_t* grid_hw
         return VLPROJ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Plan pl;
-    int rc = build_plan(h->cfg, grid_hw, nullptr, n_views, true, &pl);
+    int rc = build_plan(h->cfg, grid_hw, nullptr, n_views, true, h->gather_mode, &pl);
     if (rc) return rc;
     if (pl.M == 0) return VLPROJ_OK;
-    rc = upload(h, pl, plan_key(grid_hw, n_views, nullptr, n_views, 1), s);
+    h->profiled_valid = false;
+    rc = upload_plan(h, pl, s);
     if (rc) return rc;
-    return run_merge_gemm1(h, pl, features, nullptr, static_cast<__nv_bfloat16*>(hidden), s);
+    return run_merge_gemm1(h, pl, features, nullptr, vlp::DEST_COMPACT, static_cast<__nv_bfloat16*>(hidden),
+                           pl.M_real, s);
 }
 
 int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_hw, const int32_t* spatial_crop,
@@ -493,16 +620,14 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
         return VLPROJ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Plan pl;
-    int rc = build_plan(c, grid_hw, spatial_crop, n_images, false, &pl);
+    int rc = build_plan(c, grid_hw, spatial_crop, n_images, false, h->gather_mode, &pl);
     if (rc) return rc;
 
-    // 1. placeholder index
+    // 0. placeholder index
     const int nblocks = static_cast<int>((n_ids + vlp::SCAN_CHUNK - 1) / vlp::SCAN_CHUNK);
     if (h->counts.ensure(std::max(nblocks, 1)) || h->pos.ensure(std::max<int64_t>(pl.R, 1)))
         return VLPROJ_ERR_CUDA;
-    rc = upload(h, pl, plan_key(grid_hw, static_cast<int64_t>(pl.views.size()), tiled ? spatial_crop : nullptr,
-                                n_images, tiled ? 2 : 0),
-                s);
+    rc = upload_plan(h, pl, s);
     if (rc) return rc;
     h->profiled_valid = false;
     for (bool& r : h->stage_ran) r = false;
@@ -522,12 +647,12 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
         return VLPROJ_OK;
     }
 
-    // 2-4. geometry, LayerNorm, GEMM1 -> H
+    // 1-3. geometry, LayerNorm, GEMM1 -> H
     if (h->H.ensure(static_cast<size_t>(pl.M) * c.N1)) return VLPROJ_ERR_CUDA;
-    rc = run_merge_gemm1(h, pl, features, h->pos.ptr, h->H.ptr, s);
+    rc = run_merge_gemm1(h, pl, features, h->pos.ptr, vlp::DEST_EMBED, h->H.ptr, pl.M, s);
     if (rc) return rc;
 
-    // 5. GEMM2 + scatter
+    // 4. GEMM2 + scatter
     if (h->tmH_ptr != h->H.ptr || h->tmH_rows != pl.M) {
         if (encode_bf16_2d(&h->tmH, h->H.ptr, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
         h->tmH_ptr = h->H.ptr;
@@ -538,6 +663,8 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
     p.N = c.N2;
     p.K = c.N1;
     p.bias = h->b2;
+    p.C = c.C;
+    p.k = c.k;
     p.out = static_cast<__nv_bfloat16*>(out_embeds);
     p.rowdest = h->rowdest.ptr;
     p.out_rows = n_ids;
@@ -547,10 +674,10 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
     mark(h, 4, s);
     h->stage_ran[4] = true;
     ++h->launches;
-    rc = launch_gemm_bn<false, vlp::EPI_SCATTER>(pick_bn(c.N2), h->tmH, h->tmW2, p, h->num_sms, s);
+    rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(pick_bn(c.N2), h->tmH, h->tmW2, p, h->num_sms, s);
     if (rc) return rc;
 
-    // 6. newline / separator rows
+    // 5. newline / separator rows
     mark(h, 5, s);
     if (tiled && !pl.images.empty()) {
         h->stage_ran[5] = true;
