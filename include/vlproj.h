@@ -159,6 +159,12 @@ int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
 enum { VLPROJ_GATHER_IM2COL = 0, VLPROJ_GATHER_CPASYNC = 1, VLPROJ_GATHER_AUTO = 2 };
 int vlproj_set_gather_mode(vlproj_handle* h, int mode);
 
+/* GEMM tile shape. enable = 1 (default): 256 x 256 tiles run on pairs of CTAs
+ * (cta_group::2 MMA; each CTA stages its 128 rows of A and half of B, so B crosses
+ * L2 once per pair) wherever N >= 256 and A arrives by TMA; enable = 0: 128 x 256
+ * tiles on single CTAs. Both give the same bits. */
+int vlproj_set_tile_pairs(vlproj_handle* h, int enable);
+
 /* Bound (nanoseconds) on every wait inside this handle's kernels; 0 restores the
  * default (2 s). A wait that runs out ends its kernel early with
  * VLPROJ_ERR_TIMEOUT latched; tests use a tiny bound to exercise that path. */

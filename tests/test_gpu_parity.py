@@ -43,14 +43,20 @@ SMALL = {
 }
 
 
-@pytest.mark.parametrize("gather", [vp.GATHER_AUTO, vp.GATHER_IM2COL, vp.GATHER_CPASYNC],
-                         ids=["auto", "im2col", "cpasync"])
+# (gather mode, 256 x 256 tiles on CTA pairs)
+MODES = [(vp.GATHER_AUTO, True), (vp.GATHER_AUTO, False), (vp.GATHER_IM2COL, True), (vp.GATHER_IM2COL, False),
+         (vp.GATHER_CPASYNC, True)]
+MODE_IDS = ["auto-pairs", "auto-single", "im2col-pairs", "im2col-single", "cpasync"]
+
+
+@pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
 @pytest.mark.parametrize("name", list(SMALL))
-def test_small_case_all_rows(name, gather):
+def test_small_case_all_rows(name, mode):
     wl, hw, gvp, order = SMALL[name]
     case = make_case(wl, np.array(hw, np.int32), gvp=gvp, k_order=order)
     proj = make_projector(case)
-    proj.set_gather_mode(gather)
+    proj.set_gather_mode(mode[0])
+    proj.set_tile_pairs(mode[1])
     dev = DeviceInputs(case)
     out = run(case, proj, dev)
     assert proj.status() == vp.OK
@@ -61,14 +67,15 @@ def test_small_case_all_rows(name, gather):
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("gather", [vp.GATHER_IM2COL, vp.GATHER_CPASYNC], ids=["im2col", "cpasync"])
+@pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
 @pytest.mark.parametrize("name", ["ragged_k3_ln", "tiled_head_odd", "fp32_noln", "many_images"])
-def test_hidden_stage(name, gather):
+def test_hidden_stage(name, mode):
     """Stage parity of H = bf16(GELU(A W1^T + b1)) for every merged token."""
     wl, hw, gvp, order = SMALL[name]
     case = make_case(wl, np.array(hw, np.int32), gvp=gvp, k_order=order)
     proj = make_projector(case)
-    proj.set_gather_mode(gather)
+    proj.set_gather_mode(mode[0])
+    proj.set_tile_pairs(mode[1])
     dev = DeviceInputs(case)
     M = sum(O.tokens_untiled(h, w, wl.k) for h, w in case.hw)
     H = torch.empty((M, wl.N1), dtype=torch.bfloat16, device="cuda")
@@ -132,6 +139,21 @@ def test_gather_modes_agree_bit_for_bit():
     proj.set_gather_mode(vp.GATHER_IM2COL)
     out_a = run(case, proj, dev)
     proj.set_gather_mode(vp.GATHER_CPASYNC)
+    out_b = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["dsvit", "vl2"])
+def test_tile_pairs_agree_bit_for_bit(name):
+    """256 x 256 tiles on CTA pairs and 128 x 256 tiles on single CTAs accumulate each
+    output over the same K order, so they give identical bits."""
+    wl = W.WORKLOADS[name]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    out_a = run(case, proj, dev)
+    proj.set_tile_pairs(False)
     out_b = run(case, proj, dev)
     assert proj.status() == vp.OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))

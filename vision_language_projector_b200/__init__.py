@@ -25,7 +25,8 @@ ORDER_CHANNEL_OUTER, ORDER_POSITION_OUTER = 0, 1
 
 EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status", "vlproj_destroy",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
-            "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode")
+            "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
+            "vlproj_set_tile_pairs")
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO = 0, 1, 2
 NUM_STAGES = 6
 STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows")
@@ -80,6 +81,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_launch_count.restype = I64
     lib.vlproj_set_gather_mode.argtypes = [P, ctypes.c_int]
     lib.vlproj_set_gather_mode.restype = ctypes.c_int
+    lib.vlproj_set_tile_pairs.argtypes = [P, ctypes.c_int]
+    lib.vlproj_set_tile_pairs.restype = ctypes.c_int
     return lib
 
 
@@ -215,6 +218,11 @@ class Projector:
         rc = _lib.vlproj_set_gather_mode(self._h, int(mode))
         if rc != OK:
             raise VlprojError(rc, "vlproj_set_gather_mode")
+
+    def set_tile_pairs(self, enable: bool) -> None:
+        rc = _lib.vlproj_set_tile_pairs(self._h, int(enable))
+        if rc != OK:
+            raise VlprojError(rc, "vlproj_set_tile_pairs")
 
     def set_wait_limit(self, ns: int) -> None:
         rc = _lib.vlproj_set_wait_limit(self._h, int(ns))

@@ -14,8 +14,9 @@
 //       out[dest[m], n] = bf16( sum_q H[m, q] W2[n, q] + b2[n] )
 //       the epilogue writes each row straight into its placeholder row.
 //
-// One persistent CTA per SM walks output tiles of BM x BN (N fastest, so the
-// CTAs working at the same time share the A tile through L2). Roles, by warp:
+// One persistent CTA per SM walks output tiles of BM x BN in banded order (see
+// tile_coords: the CTAs running together share A tiles and an L2-sized band of B).
+// Roles, by warp:
 //   warp 0      TMA producer (B; A in the TMA modes)
 //   warp 1      TMEM allocator and the single MMA-issuing thread
 //   warps 2-3   A gather producers in A_CPASYNC mode (64 threads)
@@ -47,12 +48,16 @@ constexpr int A_CPASYNC = 2;            // merge-gather by cp.async
 constexpr uint64_t DRAIN_NS = 1000000000ull;
 constexpr int ERR_TIMEOUT = -5;
 
-template <int BN>
+// Shared-memory plan. kCtas = 2 runs one 256-row tile on a CTA pair: each CTA holds
+// its 128 rows of A and half of the BN rows of B per stage, so a stage is 32 KB and
+// six stages fit.
+template <int BN, int kCtas = 1>
 struct GemmLayout {
-    static constexpr int STAGES = BN == 256 ? 4 : 6;
+    static constexpr int B_ROWS = BN / kCtas;
     static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
     static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
     // full_tma[S], full_gather[S], empty[S], tmem_full[2], tmem_empty[2], drain
     static constexpr int NUM_BARS = 3 * STAGES + 5;
@@ -82,11 +87,26 @@ struct GemmParams {
     const int32_t* rowdest;         // destination row of each m (-1 = no write), or null = row m
     int64_t out_rows;               // rows of `out` (bounds guard)
     const int* fwd_status;          // nonzero = count check failed, write nothing (null = ignore)
+    int group_n;                    // N-blocks per raster band (see tile_coords)
     int* err;                       // latched error word
     uint64_t wait_ns;               // bound on every wait
 };
 
 __device__ __forceinline__ void latch_error(int* err, int code) { atomicCAS(err, 0, code); }
+
+// Tile order: bands of `group_n` N-blocks; inside a band the M-block advances slowest
+// and the band's N-blocks fastest, so the CTAs running together share both their A
+// tiles and a band of B that fits in L2 (group_n = n_tiles gives plain N-fastest order).
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int group_n, int& m_blk,
+                                            int& n_blk) {
+    const int band_tiles = m_tiles * group_n;
+    const int band = tile / band_tiles;
+    const int r = tile - band * band_tiles;
+    const int n0 = band * group_n;
+    const int width = min(group_n, n_tiles - n0);
+    m_blk = r / width;
+    n_blk = n0 + (r - m_blk * width);
+}
 
 __device__ __forceinline__ float gelu_erf(float x) {
     return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
@@ -97,13 +117,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int BN, int kAMode, int kEpi>
+template <int BN, int kAMode, int kEpi, int kCtas>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     vlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const GemmParams p) {
-    using L = GemmLayout<BN>;
+    using L = GemmLayout<BN, kCtas>;
     constexpr int S = L::STAGES;
+    constexpr bool kPair = kCtas == 2;
     constexpr bool kGatherThreads = kAMode == A_CPASYNC;
+    static_assert(!(kPair && kGatherThreads), "the cp.async gather runs on single CTAs");
+    static_assert(!kPair || BN == 256, "CTA pairs run 256 x 256 tiles");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
@@ -118,6 +141,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = kPair ? cluster_ctarank() : 0;      // 0 = pair leader
+    const bool leader = rank == 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -127,7 +152,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tmem_full[a], 1);
-            mbar_init(&tmem_empty[a], 4);
+            mbar_init(&tmem_empty[a], 4 * kCtas);               // every epilogue warp of the pair
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -140,52 +165,84 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int i = 0; i < p.n_gmaps; ++i) tensormap_acquire(p.gmaps + i);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, L::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (kPair) {
+            tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, L::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair) cluster_sync();        // barriers of both CTAs initialised before any remote use
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int m_tiles = (p.M + BM - 1) / BM;
+    const int rows_per_tile = BM * kCtas;
+    const int m_tiles = (p.M + rows_per_tile - 1) / rows_per_tile;
     const int n_tiles = (p.N + BN - 1) / BN;
     const int num_tiles = m_tiles * n_tiles;
+    const int group_n = (p.group_n > 0 && p.group_n < n_tiles) ? p.group_n : n_tiles;
     const int kblocks = p.K / BK;
     const int cblocks = p.C / BK;
     const uint64_t lim = p.wait_ns;
+    const int unit = blockIdx.x / kCtas;                      // CTA (or CTA pair) index
+    const int n_units = gridDim.x / kCtas;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (each CTA loads its own halves)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
             const int nch = (kAMode == A_IM2COL) ? BM / p.chunk : 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
+            const uint32_t expect = (kAMode == A_CPASYNC ? 0 : L::A_BYTES * kCtas) + L::B_BYTES * kCtas;
+            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+                int m_blk, n_blk;
+                tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
+                const int a_row_tile = m_blk * kCtas + static_cast<int>(rank);   // this CTA's 128-row slice
                 int4 ch[4] = {};
                 if (kAMode == A_IM2COL)
-                    for (int q = 0; q < nch; ++q) ch[q] = __ldg(&p.chunks[m_blk * nch + q]);
+                    for (int q = 0; q < nch; ++q) ch[q] = __ldg(&p.chunks[a_row_tile * nch + q]);
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag)) { ok = false; break; }
                     uint8_t* sa = smem + stage * L::STAGE_BYTES;
                     uint8_t* sb = sa + L::A_BYTES;
-                    mbar_arrive_expect_tx(&full_tma[stage], (kAMode == A_CPASYNC ? 0 : L::A_BYTES) + L::B_BYTES);
-                    if (kAMode == A_TILE) {
-                        tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, m_blk * BM);
-                    } else if (kAMode == A_IM2COL) {
-                        const int pos = kb / cblocks;                  // (dy, dx) position index
-                        const int c0 = (kb - pos * cblocks) * BK;
-                        const int dy = pos / p.k, dx = pos - dy * p.k;
-                        for (int q = 0; q < nch; ++q) {
-                            const CUtensorMap* mp = p.gmaps ? p.gmaps + ch[q].x : &tmA;
-                            tma_load_im2col_4d(sa + q * p.chunk * 128, mp, &full_tma[stage], c0, ch[q].y, ch[q].z,
-                                               ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
+                    const int b_row = n_blk * BN + static_cast<int>(rank) * L::B_ROWS;
+                    if constexpr (kPair) {
+                        const uint32_t bar = mapa_shared(smem_u32(&full_tma[stage]), 0);
+                        if (leader) mbar_arrive_expect_tx(&full_tma[stage], expect);
+                        if (kAMode == A_TILE) {
+                            tma_load_2d_pair(sa, &tmA, bar, kb * BK, a_row_tile * BM);
+                        } else if (kAMode == A_IM2COL) {
+                            const int pos = kb / cblocks;
+                            const int c0 = (kb - pos * cblocks) * BK;
+                            const int dy = pos / p.k, dx = pos - dy * p.k;
+                            for (int q = 0; q < nch; ++q) {
+                                const CUtensorMap* mp = p.gmaps ? p.gmaps + ch[q].x : &tmA;
+                                tma_load_im2col_4d_pair(sa + q * p.chunk * 128, mp, bar, c0, ch[q].y, ch[q].z,
+                                                        ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
+                            }
                         }
+                        tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
+                    } else {
+                        mbar_arrive_expect_tx(&full_tma[stage], expect);
+                        if (kAMode == A_TILE) {
+                            tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, a_row_tile * BM);
+                        } else if (kAMode == A_IM2COL) {
+                            const int pos = kb / cblocks;                  // (dy, dx) position index
+                            const int c0 = (kb - pos * cblocks) * BK;
+                            const int dy = pos / p.k, dx = pos - dy * p.k;
+                            for (int q = 0; q < nch; ++q) {
+                                const CUtensorMap* mp = p.gmaps ? p.gmaps + ch[q].x : &tmA;
+                                tma_load_im2col_4d(sa + q * p.chunk * 128, mp, &full_tma[stage], c0, ch[q].y, ch[q].z,
+                                                   ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
+                            }
+                        }
+                        tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, b_row);
                     }
-                    tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, n_blk * BN);
                     ++issued;
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
@@ -194,27 +251,35 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 *abort_flag = 1;
                 latch_error(p.err, ERR_TIMEOUT);
             }
-            // Drain: the (at most S) most recent loads may still be landing if the MMA
-            // side stopped early; in a normal run these phases are already complete.
-            int st = stage;
-            uint32_t ph = phase;
-            const int outstanding = issued < S ? issued : S;
-            for (int i = 0; i < outstanding; ++i) {
-                if (st == 0) { st = S - 1; ph ^= 1; } else { --st; }
-                volatile int never = 0;
-                mbar_wait_bounded(&full_tma[st], ph, DRAIN_NS, &never);
+            if (!kPair || leader) {
+                // Drain: the (at most S) most recent loads may still be landing if the MMA
+                // side stopped early; in a normal run these phases are already complete.
+                int st = stage;
+                uint32_t ph = phase;
+                const int outstanding = issued < S ? issued : S;
+                for (int i = 0; i < outstanding; ++i) {
+                    if (st == 0) { st = S - 1; ph ^= 1; } else { --st; }
+                    volatile int never = 0;
+                    mbar_wait_bounded(&full_tma[st], ph, DRAIN_NS, &never);
+                }
+            } else if (!ok) {
+                // The second CTA's loads complete on the leader's barriers, which it cannot
+                // poll: after an early stop give any copy still landing ample time.
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 200000ull) {
+                }
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+        // ------------------------------------------------ MMA issuer (the pair leader's lane 0)
+        if (lane == 0 && leader) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BM * kCtas, BN);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
                 if (!mbar_wait_bounded(&tmem_empty[acc], acc_phase ^ 1, lim, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -229,14 +294,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint32_t sb = sa + L::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        tc_mma_f16(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
-                                   (kb | kk) != 0);
+                        if constexpr (kPair)
+                            tc_mma_f16_pair(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32),
+                                            idesc, (kb | kk) != 0);
+                        else
+                            tc_mma_f16(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
+                                       (kb | kk) != 0);
                     }
-                    tc_commit(&empty[stage]);
+                    if constexpr (kPair) tc_commit_pair(&empty[stage], 0x3);
+                    else tc_commit(&empty[stage]);
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                tc_commit(&tmem_full[acc]);
+                if constexpr (kPair) tc_commit_pair(&tmem_full[acc], 0x3);
+                else tc_commit(&tmem_full[acc]);
                 if (++acc == 2) { acc = 0; acc_phase ^= 1; }
             }
             if (!ok) {
@@ -244,7 +315,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 latch_error(p.err, ERR_TIMEOUT);
             }
             // all MMAs issued by this thread are complete once `drain` flips
-            tc_commit(drain);
+            if constexpr (kPair) tc_commit_pair(drain, 0x1);
+            else tc_commit(drain);
             volatile int never = 0;
             mbar_wait_bounded(drain, 0, DRAIN_NS, &never);
         }
@@ -258,8 +330,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m_blk = tile / n_tiles;
+            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+                int m_blk, n_blk;
+                tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
                 int base[16];
                 uint32_t wm[16];
 #pragma unroll
@@ -300,22 +373,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             cp_async_wait_all();
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 4..7)
+        // ------------------------------------------------ epilogue (warps 4..7 of each CTA)
         const int ew = warp & 3;                      // TMEM lanes 32*ew .. 32*ew+31
         const int row = ew * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
         const int status_ok = p.fwd_status ? (*p.fwd_status == 0) : 1;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-            const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
+        for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+            int m_blk, n_blk;
+            tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
             // one lane waits, the warp follows it, so tcgen05.ld below is never divergent
             int got = 0;
             if (lane == 0) got = mbar_wait_bounded(&tmem_full[acc], acc_phase, lim, abort_flag) ? 1 : 0;
             got = __shfl_sync(0xffffffffu, got, 0);
             if (!got) { ok = false; break; }
             tc_fence_after();
-            const int m = m_blk * BM + row;
+            const int m = (m_blk * kCtas + static_cast<int>(rank)) * BM + row;
             bool row_ok = m < p.M && status_ok;
             int64_t d = m;
             if (row_ok && p.rowdest) d = __ldg(&p.rowdest[m]);
@@ -350,7 +424,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+            if (lane == 0) {
+                if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&tmem_empty[acc]), 0));
+                else mbar_arrive(&tmem_empty[acc]);
+            }
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
         if (!ok) {
@@ -359,12 +436,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     }
 
+    __syncwarp();                     // lanes that skipped a role rejoin their lane 0
     tc_fence_before();
-    __syncthreads();
+    // A pair's CTAs read each other's shared memory (MMA operands, barriers): neither
+    // leaves before the other is done.
+    if constexpr (kPair) cluster_sync();
+    else __syncthreads();
     tc_fence_after();
     if (warp == 1) {
         __syncwarp();
-        tmem_dealloc(tmem_base, L::TMEM_COLS);
+        if constexpr (kPair) tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+        else tmem_dealloc(tmem_base, L::TMEM_COLS);
     }
 }
 

@@ -272,24 +272,64 @@ int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int32_t* cr
     return VLPROJ_OK;
 }
 
-template <int BN, int A, int E>
-int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int num_sms, cudaStream_t s) {
-    using L = GemmLayout<BN>;
-    VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_gemm_kernel<BN, A, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  L::SMEM_ALLOC));
-    const int tiles = ((p.M + vlp::BM - 1) / vlp::BM) * ((p.N + BN - 1) / BN);
-    const int grid = std::min(tiles, num_sms);
-    if (grid <= 0) return VLPROJ_OK;
-    vlp::vlp_gemm_kernel<BN, A, E><<<grid, vlp::GEMM_THREADS, L::SMEM_ALLOC, s>>>(ta, tb, p);
-    VLP_CUDA(cudaGetLastError());
+// N-blocks per raster band: all of them while B fits comfortably in L2 (about 40 MB,
+// a margin under one die's share of the 126 MB), else as many as fit in that budget.
+int raster_group(int N, int K, int BN) {
+    const int n_tiles = (N + BN - 1) / BN;
+    const int64_t per_block = static_cast<int64_t>(BN) * K * 2;
+    const int64_t budget = int64_t(40) << 20;
+    if (per_block * n_tiles <= budget) return n_tiles;
+    return static_cast<int>(std::max<int64_t>(1, budget / per_block));
+}
+
+template <int BN, int A, int E, int CTAS>
+int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, int num_sms, cudaStream_t s) {
+    using L = GemmLayout<BN, CTAS>;
+    auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
+    if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN);
+    VLP_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC));
+    const int tiles = ((p.M + vlp::BM * CTAS - 1) / (vlp::BM * CTAS)) * ((p.N + BN - 1) / BN);
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(vlp::GEMM_THREADS);
+    cfg.dynamicSmemBytes = L::SMEM_ALLOC;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CTAS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    int resident = num_sms / CTAS;               // persistent: one unit per SM (pair of SMs)
+    if constexpr (CTAS > 1) {
+        // pairs must sit in one GPC: ask how many can be resident at once
+        static int cached = -1;
+        if (cached < 0) {
+            cfg.gridDim = dim3(static_cast<unsigned>(2 * resident));
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            cached = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0 ? n : resident;
+        }
+        resident = std::min(resident, cached);
+    }
+    const int units = std::min(tiles, resident);
+    if (units <= 0) return VLPROJ_OK;
+    cfg.gridDim = dim3(static_cast<unsigned>(units * CTAS));
+    cfg.attrs = CTAS > 1 ? attr : nullptr;
+    cfg.numAttrs = CTAS > 1 ? 1 : 0;
+    VLP_CUDA(cudaLaunchKernelEx(&cfg, kernel, ta, tb, p));
     return VLPROJ_OK;
 }
 
+// Tile shape: 256 x 256 tiles on CTA pairs when N allows and the A operand comes by
+// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise.
 template <int A, int E>
-int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int num_sms,
-                   cudaStream_t s) {
-    if (bn == 256) return launch_gemm<256, A, E>(ta, tb, p, num_sms, s);
-    return launch_gemm<128, A, E>(ta, tb, p, num_sms, s);
+int launch_gemm_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb_half,
+                   const GemmParams& p, int num_sms, cudaStream_t s) {
+    if constexpr (A != vlp::A_CPASYNC) {
+        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, p, num_sms, s);
+    }
+    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, p, num_sms, s);
+    return launch_gemm<128, A, E, 1>(ta, tb, p, num_sms, s);
 }
 
 int pick_bn(int N) { return N >= 256 ? 256 : 128; }
@@ -309,7 +349,9 @@ struct vlproj_handle {
     float* b2 = nullptr;
     float* gamma = nullptr;
     float* beta = nullptr;
-    CUtensorMap tmW1{}, tmW2{};
+    CUtensorMap tmW1{}, tmW2{};          // B boxes of BN rows (single-CTA tiles)
+    CUtensorMap tmW1h{}, tmW2h{};        // B boxes of 128 rows (each CTA of a pair loads half)
+    bool pairs = true;                   // run 256 x 256 tiles on CTA pairs where possible
     // scratch, grown on demand
     DevBuf<__nv_bfloat16> H, Xn;
     DevBuf<int32_t> pos, rowdest, counts;
@@ -360,7 +402,8 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     if (M == 0) return VLPROJ_OK;
     const bool im2col = pl.im2col;
     const int nch_tile = vlp::BM / pl.chunk;
-    const int n_chunks = im2col ? ((M + vlp::BM - 1) / vlp::BM) * nch_tile : 0;
+    // chunk entries for every 128-row slice of every (pair) tile, so round to 256 rows
+    const int n_chunks = im2col ? ((M + 2 * vlp::BM - 1) / (2 * vlp::BM)) * 2 * nch_tile : 0;
     if (h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
     if (!im2col && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
     if (im2col && h->chunks.ensure(std::max(n_chunks, 1))) return VLPROJ_ERR_CUDA;
@@ -440,8 +483,11 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     mark(h, 3, s);
     h->stage_ran[3] = true;
     ++h->launches;
-    if (im2col) return launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(pick_bn(c.N1), tmA, h->tmW1, p, h->num_sms, s);
-    return launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(pick_bn(c.N1), tmA, h->tmW1, p, h->num_sms, s);
+    if (im2col)
+        return launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                            h->num_sms, s);
+    return launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(pick_bn(c.N1), false, tmA, h->tmW1, h->tmW1h, p, h->num_sms,
+                                                         s);
 }
 
 }  // namespace
@@ -527,7 +573,8 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
     if (cudaMemset(h->status, 0, 2 * sizeof(int))) return fail(VLPROJ_ERR_CUDA);
     if (cudaDeviceSynchronize()) return fail(VLPROJ_ERR_CUDA);
     if (encode_bf16_2d(&h->tmW1, h->W1p, n1, h->K1, pick_bn(cfg->N1)) ||
-        encode_bf16_2d(&h->tmW2, h->W2, n2, n1, pick_bn(cfg->N2)))
+        encode_bf16_2d(&h->tmW2, h->W2, n2, n1, pick_bn(cfg->N2)) ||
+        encode_bf16_2d(&h->tmW1h, h->W1p, n1, h->K1, 128) || encode_bf16_2d(&h->tmW2h, h->W2, n2, n1, 128))
         return fail(VLPROJ_ERR_CUDA);
     *out = h;
     return VLPROJ_OK;
@@ -568,6 +615,12 @@ void vlproj_destroy(vlproj_handle* h) {
 int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns) {
     if (!h) return VLPROJ_ERR_INVALID_ARG;
     h->wait_ns = ns ? ns : kDefaultWaitNs;
+    return VLPROJ_OK;
+}
+
+int vlproj_set_tile_pairs(vlproj_handle* h, int enable) {
+    if (!h) return VLPROJ_ERR_INVALID_ARG;
+    h->pairs = enable != 0;
     return VLPROJ_OK;
 }
 
@@ -674,7 +727,8 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
     mark(h, 4, s);
     h->stage_ran[4] = true;
     ++h->launches;
-    rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(pick_bn(c.N2), h->tmH, h->tmW2, p, h->num_sms, s);
+    rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(pick_bn(c.N2), h->pairs, h->tmH, h->tmW2, h->tmW2h, p,
+                                                       h->num_sms, s);
     if (rc) return rc;
 
     // 5. newline / separator rows
