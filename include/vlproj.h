@@ -148,15 +148,19 @@ int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
                           const int32_t* spatial_crop, int32_t n_images, int64_t* rows_out);
 
 /* How GEMM1 fetches each merged token's k x k neighbourhood from the features:
- *   VLPROJ_GATHER_AUTO    (default) IM2COL when every view of the batch has the same
- *                         grid, CPASYNC otherwise (measured faster for mixed grids);
+ *   VLPROJ_GATHER_AUTO    (default) BOX when every view has the same grid, k divides
+ *                         it and w' = w/k divides 128; else IM2COL when every view has
+ *                         the same grid; else CPASYNC (measured faster for mixed grids);
+ *   VLPROJ_GATHER_BOX     one 5D tiled TMA box per K-block: the features seen as
+ *                         (c, dx, j, dy, merged row); falls back to IM2COL when the
+ *                         grids are not regular as above;
  *   VLPROJ_GATHER_IM2COL  TMA im2col loads, the merge seen as a k x k, stride-k
  *                         convolution window walk with hardware zero fill of the
  *                         high-end pad; one map for a batch of same-shape views, else
  *                         one map per view with each view's rows padded to 32;
  *   VLPROJ_GATHER_CPASYNC 16-byte cp.async copies per row (zero-filled pad).
  * All give the same bits. */
-enum { VLPROJ_GATHER_IM2COL = 0, VLPROJ_GATHER_CPASYNC = 1, VLPROJ_GATHER_AUTO = 2 };
+enum { VLPROJ_GATHER_IM2COL = 0, VLPROJ_GATHER_CPASYNC = 1, VLPROJ_GATHER_AUTO = 2, VLPROJ_GATHER_BOX = 3 };
 int vlproj_set_gather_mode(vlproj_handle* h, int mode);
 
 /* GEMM tile shape. enable = 1 (default): 256 x 256 tiles run on pairs of CTAs

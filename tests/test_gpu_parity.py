@@ -37,16 +37,19 @@ SMALL = {
                        [[20, 14], [13, 13], [2, 30]], "head", vp.ORDER_POSITION_OUTER),
     # a single 1x1 grid (one merged token, three pad neighbours)
     "one_patch": (custom("one_patch", 106, 2, 64, 64, 32, 1, 1, 10), [[1, 1]], "head", vp.ORDER_CHANNEL_OUTER),
-    # many images, 8 sequences; M = 1408 (11 full tiles), N2 = 512 (two 256 tiles)
+    # many images, 8 sequences; M = 1536 (12 full tiles), N2 = 512 (two 256 tiles); regular grid (w' = 8)
     "many_images": (custom("many_images", 107, 2, 64, 256, 512, 32, 8, 256), [[12, 16]] * 32, "head",
                     vp.ORDER_CHANNEL_OUTER),
+    # regular k = 3 grid with w' = 32: M = 800, a ragged last tile (the 5D box path)
+    "regular_k3": (custom("regular_k3", 109, 3, 128, 256, 256, 5, 5, 256), [[15, 96]] * 5, "head",
+                   vp.ORDER_CHANNEL_OUTER),
 }
 
 
 # (gather mode, 256 x 256 tiles on CTA pairs)
 MODES = [(vp.GATHER_AUTO, True), (vp.GATHER_AUTO, False), (vp.GATHER_IM2COL, True), (vp.GATHER_IM2COL, False),
-         (vp.GATHER_CPASYNC, True)]
-MODE_IDS = ["auto-pairs", "auto-single", "im2col-pairs", "im2col-single", "cpasync"]
+         (vp.GATHER_CPASYNC, True), (vp.GATHER_BOX, True), (vp.GATHER_BOX, False)]
+MODE_IDS = ["auto-pairs", "auto-single", "im2col-pairs", "im2col-single", "cpasync", "box-pairs", "box-single"]
 
 
 @pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
@@ -68,7 +71,7 @@ def test_small_case_all_rows(name, mode):
 
 
 @pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
-@pytest.mark.parametrize("name", ["ragged_k3_ln", "tiled_head_odd", "fp32_noln", "many_images"])
+@pytest.mark.parametrize("name", ["ragged_k3_ln", "tiled_head_odd", "fp32_noln", "many_images", "regular_k3"])
 def test_hidden_stage(name, mode):
     """Stage parity of H = bf16(GELU(A W1^T + b1)) for every merged token."""
     wl, hw, gvp, order = SMALL[name]
@@ -139,6 +142,19 @@ def test_gather_modes_agree_bit_for_bit():
     proj.set_gather_mode(vp.GATHER_IM2COL)
     out_a = run(case, proj, dev)
     proj.set_gather_mode(vp.GATHER_CPASYNC)
+    out_b = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+
+
+def test_box_and_im2col_agree_bit_for_bit():
+    wl = W.WORKLOADS["dsvit"]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    proj.set_gather_mode(vp.GATHER_BOX)
+    out_a = run(case, proj, dev)
+    proj.set_gather_mode(vp.GATHER_IM2COL)
     out_b = run(case, proj, dev)
     assert proj.status() == vp.OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))

@@ -27,7 +27,7 @@ EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
             "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
             "vlproj_set_tile_pairs")
-GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO = 0, 1, 2
+GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX = 0, 1, 2, 3
 NUM_STAGES = 6
 STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows")
 

@@ -8,8 +8,11 @@
 //       features: for K-block (dy, dx, c0) one load walks the tile's tokens (base
 //       positions (k*j, k*i) of each view, wrapping rows and views) and copies
 //       channels c0..c0+63 of patch (k*i + dy, k*j + dx); patches past the grid
-//       (the high-end pad) read as zero. A_CPASYNC is the same gather done with
-//       16-byte cp.async copies (zero-filled pad), used when no im2col map fits.
+//       (the high-end pad) read as zero. When k divides the grid and w' divides
+//       128, the same gather is one 5D tiled box (A_BOX5): the features seen as
+//       (c, dx, j, dy, merged row) with strides (1, C, kC, wC, kwC) and box
+//       (64, 1, w', 1, 128/w') hold a 128-token tile in token order. A_CPASYNC is
+//       the gather done with 16-byte cp.async copies (zero-filled pad).
 //   GEMM2 (A_TILE, EPI_SCATTER):
 //       out[dest[m], n] = bf16( sum_q H[m, q] W2[n, q] + b2[n] )
 //       the epilogue writes each row straight into its placeholder row.
@@ -45,6 +48,7 @@ constexpr int EPI_SCATTER = 1;
 constexpr int A_TILE = 0;               // dense row-major A, tiled TMA
 constexpr int A_IM2COL = 1;             // merge-gather by TMA im2col
 constexpr int A_CPASYNC = 2;            // merge-gather by cp.async
+constexpr int A_BOX5 = 3;               // merge-gather by one 5D tiled TMA box (regular grids)
 constexpr uint64_t DRAIN_NS = 1000000000ull;
 constexpr int ERR_TIMEOUT = -5;
 
@@ -79,6 +83,8 @@ struct GemmParams {
     int n_gmaps;
     const int4* chunks;             // per chunk of `chunk` rows: {map, w0, h0, n0} of its first token
     int chunk;                      // rows per im2col load: 128 (one map) or 32 (per-view maps)
+    // A_BOX5: features seen as (c, dx, j, dy, merged row) with box (64, 1, w', 1, 128 / w')
+    int box_rows;                   // merged rows per 128-row tile (128 / w')
     // A_CPASYNC
     const __nv_bfloat16* gsrc;      // bf16 patch features [P][C]
     const int2* gmeta;              // per row: {top-left patch index, (w << 16) | valid mask}
@@ -160,7 +166,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmB);
-        if (kAMode == A_TILE || (kAMode == A_IM2COL && p.gmaps == nullptr)) tma_prefetch_desc(&tmA);
+        if (kAMode == A_TILE || kAMode == A_BOX5 || (kAMode == A_IM2COL && p.gmaps == nullptr))
+            tma_prefetch_desc(&tmA);
         if (kAMode == A_IM2COL && p.gmaps != nullptr)
             for (int i = 0; i < p.n_gmaps; ++i) tensormap_acquire(p.gmaps + i);
     }
@@ -216,6 +223,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         if (leader) mbar_arrive_expect_tx(&full_tma[stage], expect);
                         if (kAMode == A_TILE) {
                             tma_load_2d_pair(sa, &tmA, bar, kb * BK, a_row_tile * BM);
+                        } else if (kAMode == A_BOX5) {
+                            const int pos = kb / cblocks;
+                            const int c0 = (kb - pos * cblocks) * BK;
+                            const int dy = pos / p.k, dx = pos - dy * p.k;
+                            tma_load_5d_pair(sa, &tmA, bar, c0, dx, 0, dy, a_row_tile * p.box_rows);
                         } else if (kAMode == A_IM2COL) {
                             const int pos = kb / cblocks;
                             const int c0 = (kb - pos * cblocks) * BK;
@@ -231,6 +243,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         mbar_arrive_expect_tx(&full_tma[stage], expect);
                         if (kAMode == A_TILE) {
                             tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, a_row_tile * BM);
+                        } else if (kAMode == A_BOX5) {
+                            const int pos = kb / cblocks;
+                            const int c0 = (kb - pos * cblocks) * BK;
+                            const int dy = pos / p.k, dx = pos - dy * p.k;
+                            tma_load_5d(sa, &tmA, &full_tma[stage], c0, dx, 0, dy, a_row_tile * p.box_rows);
                         } else if (kAMode == A_IM2COL) {
                             const int pos = kb / cblocks;                  // (dy, dx) position index
                             const int c0 = (kb - pos * cblocks) * BK;

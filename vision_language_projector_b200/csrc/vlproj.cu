@@ -102,6 +102,28 @@ int encode_im2col(CUtensorMap* map, const void* base, int C, int h, int w, int n
     return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
 }
 
+// 5D tiled map of n views of one (h, w) grid with k | h, k | w and w' | 128: dims
+// (C, k, w', k, h' * n) with strides (C, k*C, w*C, k*w*C) elements, box
+// (64, 1, w', 1, 128 / w'): one box is 128 merged tokens, row-major, at filter tap
+// (dy, dx) = (coordinate 3, coordinate 1).
+int encode_box5(CUtensorMap* map, const void* base, int C, int h, int w, int n, int k) {
+    auto fn = driver().tiled;
+    if (!fn) return VLPROJ_ERR_CUDA;
+    const int hp = h / k, wp = w / k;
+    cuuint64_t dims[5] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(wp),
+                          static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(hp) * n};
+    const cuuint64_t e = 2;
+    cuuint64_t strides[4] = {static_cast<cuuint64_t>(C) * e, static_cast<cuuint64_t>(k) * C * e,
+                             static_cast<cuuint64_t>(w) * C * e, static_cast<cuuint64_t>(k) * w * C * e};
+    cuuint32_t box[5] = {static_cast<cuuint32_t>(vlp::BK), 1, static_cast<cuuint32_t>(wp), 1,
+                         static_cast<cuuint32_t>(vlp::BM / wp)};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
 template <typename T>
 struct DevBuf {
     T* ptr = nullptr;
@@ -177,6 +199,7 @@ struct Plan {
     int max_special = 0;    // most special rows of one image
     bool uniform = true;    // every view has the same grid
     bool im2col = true;     // GEMM1 gathers with TMA im2col (else cp.async)
+    bool box5 = false;      // ... or with one 5D tiled box per K-block (regular grids)
     int chunk = 128;        // im2col rows per load
 };
 
@@ -225,6 +248,15 @@ int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int32_t* cr
     }
     pl.chunk = pl.uniform ? 128 : 32;
     pl.im2col = gather_mode == VLPROJ_GATHER_IM2COL || (gather_mode == VLPROJ_GATHER_AUTO && pl.uniform);
+    if (pl.uniform && n_views > 0 && (gather_mode == VLPROJ_GATHER_BOX || gather_mode == VLPROJ_GATHER_AUTO)) {
+        const int h = grid_hw[0], w = grid_hw[1];
+        if (h % k == 0 && w % k == 0 && w / k <= vlp::BM && vlp::BM % (w / k) == 0) {
+            pl.box5 = true;
+            pl.im2col = false;
+        } else if (gather_mode == VLPROJ_GATHER_BOX) {
+            pl.im2col = true;             // not regular: the im2col walk does the same job
+        }
+    }
     const int pad_to = (pl.im2col && !pl.uniform) ? pl.chunk : 1;
     int64_t v = 0;
     for (int32_t img = 0; img < n_images; ++img) {
@@ -404,8 +436,9 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     const int nch_tile = vlp::BM / pl.chunk;
     // chunk entries for every 128-row slice of every (pair) tile, so round to 256 rows
     const int n_chunks = im2col ? ((M + 2 * vlp::BM - 1) / (2 * vlp::BM)) * 2 * nch_tile : 0;
+    const bool cpasync = !im2col && !pl.box5;
     if (h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
-    if (!im2col && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
+    if (cpasync && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
     if (im2col && h->chunks.ensure(std::max(n_chunks, 1))) return VLPROJ_ERR_CUDA;
 
     mark(h, 1, s);
@@ -414,7 +447,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     const int geo_threads = std::max(M, n_chunks);
     vlp::vlp_geometry_kernel<<<(geo_threads + 255) / 256, 256, 0, s>>>(
         h->dviews.ptr, static_cast<int>(pl.views.size()), M, c.k, pos, pl.R, dest_mode,
-        im2col ? nullptr : h->gmeta.ptr, h->rowdest.ptr, im2col ? h->chunks.ptr : nullptr, n_chunks, pl.chunk,
+        cpasync ? h->gmeta.ptr : nullptr, h->rowdest.ptr, im2col ? h->chunks.ptr : nullptr, n_chunks, pl.chunk,
         pl.uniform ? 1 : 0);
     VLP_CUDA(cudaGetLastError());
 
@@ -452,7 +485,11 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
 
     CUtensorMap tmA{};
     std::memset(&tmA, 0, sizeof(tmA));
-    if (im2col) {
+    if (pl.box5) {
+        const ViewDesc& V = pl.views[0];
+        if (encode_box5(&tmA, src, c.C, V.h, V.w, static_cast<int>(pl.views.size()), c.k)) return VLPROJ_ERR_CUDA;
+        p.box_rows = vlp::BM / V.wp;
+    } else if (im2col) {
         p.chunks = h->chunks.ptr;
         p.chunk = pl.chunk;
         if (pl.uniform) {
@@ -483,6 +520,9 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     mark(h, 3, s);
     h->stage_ran[3] = true;
     ++h->launches;
+    if (pl.box5)
+        return launch_gemm_bn<vlp::A_BOX5, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                          h->num_sms, s);
     if (im2col)
         return launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
                                                             h->num_sms, s);
@@ -625,7 +665,8 @@ int vlproj_set_tile_pairs(vlproj_handle* h, int enable) {
 }
 
 int vlproj_set_gather_mode(vlproj_handle* h, int mode) {
-    if (!h || (mode != VLPROJ_GATHER_IM2COL && mode != VLPROJ_GATHER_CPASYNC && mode != VLPROJ_GATHER_AUTO))
+    if (!h || (mode != VLPROJ_GATHER_IM2COL && mode != VLPROJ_GATHER_CPASYNC && mode != VLPROJ_GATHER_AUTO &&
+               mode != VLPROJ_GATHER_BOX))
         return VLPROJ_ERR_INVALID_ARG;
     h->gather_mode = mode;
     return VLPROJ_OK;
