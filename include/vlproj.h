@@ -148,9 +148,14 @@ int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
                           const int32_t* spatial_crop, int32_t n_images, int64_t* rows_out);
 
 /* How GEMM1 fetches each merged token's k x k neighbourhood from the features:
- *   VLPROJ_GATHER_AUTO    (default) BOX when every view has the same grid, k divides
- *                         it and w' = w/k divides 128; else IM2COL when every view has
- *                         the same grid; else CPASYNC (measured faster for mixed grids);
+ *   VLPROJ_GATHER_AUTO    (default) with a pre-merge LayerNorm or fp32 features, the
+ *                         LayerNorm / convert pass writes its bf16 output directly in
+ *                         merged-token order and GEMM1 reads it as a plain matrix;
+ *                         otherwise BOX when every view has the same grid, k divides it
+ *                         and w' = w/k divides 128; else IM2COL when every view has the
+ *                         same grid; else CPASYNC (measured faster for mixed grids).
+ *                         The modes below apply the LayerNorm pass in patch order and
+ *                         gather from its output;
  *   VLPROJ_GATHER_BOX     one 5D tiled TMA box per K-block: the features seen as
  *                         (c, dx, j, dy, merged row); falls back to IM2COL when the
  *                         grids are not regular as above;

@@ -173,3 +173,17 @@ def test_tile_pairs_agree_bit_for_bit(name):
     out_b = run(case, proj, dev)
     assert proj.status() == vp.OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+
+
+def test_merged_layernorm_path_agrees_bit_for_bit():
+    """With a LayerNorm, AUTO writes the normalised features straight in merged-token
+    order; the patch-order LayerNorm + gather path reads the same values."""
+    wl = W.WORKLOADS["moonvit"]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    out_a = run(case, proj, dev)                     # AUTO
+    proj.set_gather_mode(vp.GATHER_CPASYNC)
+    out_b = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))

@@ -200,6 +200,7 @@ struct Plan {
     bool uniform = true;    // every view has the same grid
     bool im2col = true;     // GEMM1 gathers with TMA im2col (else cp.async)
     bool box5 = false;      // ... or with one 5D tiled box per K-block (regular grids)
+    bool merged_ln = false; // ... or reads A written in token order by the LayerNorm pass
     int chunk = 128;        // im2col rows per load
 };
 
@@ -247,7 +248,14 @@ int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int32_t* cr
         if (h != grid_hw[0] || w != grid_hw[1]) pl.uniform = false;
     }
     pl.chunk = pl.uniform ? 128 : 32;
-    pl.im2col = gather_mode == VLPROJ_GATHER_IM2COL || (gather_mode == VLPROJ_GATHER_AUTO && pl.uniform);
+    if (gather_mode == VLPROJ_GATHER_AUTO && (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32)) {
+        // a LayerNorm / convert pass writes a bf16 copy anyway: write it as A itself
+        pl.merged_ln = true;
+        pl.im2col = false;
+        gather_mode = VLPROJ_GATHER_CPASYNC;   // no padding, no chunk table
+    }
+    pl.im2col = !pl.merged_ln &&
+                (gather_mode == VLPROJ_GATHER_IM2COL || (gather_mode == VLPROJ_GATHER_AUTO && pl.uniform));
     if (pl.uniform && n_views > 0 && (gather_mode == VLPROJ_GATHER_BOX || gather_mode == VLPROJ_GATHER_AUTO)) {
         const int h = grid_hw[0], w = grid_hw[1];
         if (h % k == 0 && w % k == 0 && w / k <= vlp::BM && vlp::BM % (w / k) == 0) {
@@ -385,7 +393,7 @@ struct vlproj_handle {
     CUtensorMap tmW1h{}, tmW2h{};        // B boxes of 128 rows (each CTA of a pair loads half)
     bool pairs = true;                   // run 256 x 256 tiles on CTA pairs where possible
     // scratch, grown on demand
-    DevBuf<__nv_bfloat16> H, Xn;
+    DevBuf<__nv_bfloat16> H, Xn, A;
     DevBuf<int32_t> pos, rowdest, counts;
     DevBuf<int2> gmeta;
     DevBuf<int4> chunks;
@@ -436,7 +444,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     const int nch_tile = vlp::BM / pl.chunk;
     // chunk entries for every 128-row slice of every (pair) tile, so round to 256 rows
     const int n_chunks = im2col ? ((M + 2 * vlp::BM - 1) / (2 * vlp::BM)) * 2 * nch_tile : 0;
-    const bool cpasync = !im2col && !pl.box5;
+    const bool cpasync = !im2col && !pl.box5;   // (also the merged-LayerNorm path: it needs gmeta)
     if (h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
     if (cpasync && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
     if (im2col && h->chunks.ensure(std::max(n_chunks, 1))) return VLPROJ_ERR_CUDA;
@@ -453,7 +461,21 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
 
     const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(features);
     mark(h, 2, s);
-    if (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) {
+    if (pl.merged_ln) {
+        h->stage_ran[2] = true;
+        ++h->launches;
+        if (h->A.ensure(static_cast<size_t>(M) * h->K1)) return VLPROJ_ERR_CUDA;
+        const int64_t items = static_cast<int64_t>(M) * c.k * c.k;
+        const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+        const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
+        if (c.feat_dtype == VLPROJ_FEAT_F32)
+            vlp::vlp_ln_merge_kernel<true><<<blocks, 256, 0, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma,
+                                                                  h->beta, eps, c.has_ln, h->A.ptr);
+        else
+            vlp::vlp_ln_merge_kernel<false><<<blocks, 256, 0, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma,
+                                                                   h->beta, eps, c.has_ln, h->A.ptr);
+        VLP_CUDA(cudaGetLastError());
+    } else if (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) {
         h->stage_ran[2] = true;
         ++h->launches;
         if (h->Xn.ensure(static_cast<size_t>(pl.P) * c.C)) return VLPROJ_ERR_CUDA;
@@ -485,7 +507,10 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
 
     CUtensorMap tmA{};
     std::memset(&tmA, 0, sizeof(tmA));
-    if (pl.box5) {
+    if (pl.merged_ln) {
+        if (encode_bf16_2d(&tmA, h->A.ptr, static_cast<uint64_t>(M), static_cast<uint64_t>(h->K1), vlp::BM))
+            return VLPROJ_ERR_CUDA;
+    } else if (pl.box5) {
         const ViewDesc& V = pl.views[0];
         if (encode_box5(&tmA, src, c.C, V.h, V.w, static_cast<int>(pl.views.size()), c.k)) return VLPROJ_ERR_CUDA;
         p.box_rows = vlp::BM / V.wp;
@@ -520,6 +545,9 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     mark(h, 3, s);
     h->stage_ran[3] = true;
     ++h->launches;
+    if (pl.merged_ln)
+        return launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                          h->num_sms, s);
     if (pl.box5)
         return launch_gemm_bn<vlp::A_BOX5, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
                                                           h->num_sms, s);
@@ -635,6 +663,7 @@ void vlproj_destroy(vlproj_handle* h) {
     cudaFree(h->status);
     h->H.release();
     h->Xn.release();
+    h->A.release();
     h->pos.release();
     h->rowdest.release();
     h->counts.release();
