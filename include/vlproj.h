@@ -196,6 +196,28 @@ int vlproj_profile_read(vlproj_handle* h, float* ms, int n);
 /* Number of kernels this handle has launched since it was created (all entry points). */
 int64_t vlproj_launch_count(vlproj_handle* h);
 
+/* ---- placeholder index without allocation ------------------------------
+ * The pages have no counterpart to this entry point; it serves callers of this
+ * library that must not allocate device memory when they call it: code where an
+ * allocation would synchronise the device or break a latency budget, or code with
+ * no allocator of its own to hand (a plain C caller that only borrows buffers).
+ *
+ * Writes positions[j] = flat index of the j-th element of input_ids equal to
+ * image_token_id (in order, for j < max_positions) and *count = how many there are,
+ * asynchronously on `stream`: the same step as the placeholder index of
+ * vlproj_forward, needing no handle. input_ids: DEVICE int64 [n_ids]; positions:
+ * DEVICE int32 [max_positions]; count: DEVICE int64 [1].
+ * It calls no allocator: its only scratch (one int32 per 4096 ids) is a fixed array
+ * in the library's device memory, VLPROJ_NOALLOC_MAX_IDS / 4096 entries (64 KB),
+ * held by every GPU that loads the library until the process exits. n_ids beyond
+ * VLPROJ_NOALLOC_MAX_IDS returns VLPROJ_ERR_INVALID_ARG before any launch.
+ * The first call on each device looks up that device's copy of the array (with the
+ * device current) and should come before any stream capture. All calls share the
+ * array: calls that overlap on the same GPU race on it. */
+#define VLPROJ_NOALLOC_MAX_IDS (64 * 1024 * 1024)
+int vlproj_placeholder_index_noalloc(const int64_t* input_ids, int64_t n_ids, int64_t image_token_id,
+                                     int32_t* positions, int64_t max_positions, int64_t* count, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* vlproj_strerror(int code);
 

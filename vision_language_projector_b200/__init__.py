@@ -26,7 +26,8 @@ ORDER_CHANNEL_OUTER, ORDER_POSITION_OUTER = 0, 1
 EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status", "vlproj_destroy",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
             "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
-            "vlproj_set_tile_pairs")
+            "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc")
+NOALLOC_MAX_IDS = 64 * 1024 * 1024
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX = 0, 1, 2, 3
 NUM_STAGES = 6
 STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows")
@@ -83,6 +84,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_set_gather_mode.restype = ctypes.c_int
     lib.vlproj_set_tile_pairs.argtypes = [P, ctypes.c_int]
     lib.vlproj_set_tile_pairs.restype = ctypes.c_int
+    lib.vlproj_placeholder_index_noalloc.argtypes = [P, I64, I64, P, I64, P, P]
+    lib.vlproj_placeholder_index_noalloc.restype = ctypes.c_int
     return lib
 
 
@@ -132,6 +135,16 @@ def image_rows(cfg: Config, grid_hw, spatial_crop=None, n_images: Optional[int] 
     if r < 0:
         raise VlprojError(int(r), "vlproj_image_rows")
     return out[:n_images]
+
+
+def placeholder_index_noalloc(input_ids, image_token_id: int, positions, count, stream=None,
+                              n_ids: Optional[int] = None, max_positions: Optional[int] = None) -> int:
+    """Placeholder positions and count without any allocation (see vlproj.h): for callers
+    that must not allocate device memory at the call. Returns the status code."""
+    n = int(input_ids.numel()) if n_ids is None else int(n_ids)
+    mp = int(positions.numel()) if max_positions is None else int(max_positions)
+    return _lib.vlproj_placeholder_index_noalloc(_ptr(input_ids), n, int(image_token_id), _ptr(positions), mp,
+                                                 _ptr(count), _stream_ptr(stream))
 
 
 def _stream_ptr(stream) -> Optional[int]:
