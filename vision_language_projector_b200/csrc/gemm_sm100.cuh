@@ -368,7 +368,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const int pos = kb / cblocks;
                     const int c0 = (kb - pos * cblocks) * BK + chunk * 8;
                     const int dy = pos / p.k, dx = pos - dy * p.k;
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag)) { ok = false; break; }
+                    // one lane per warp waits, the warp follows it
+                    int got = 0;
+                    if ((threadIdx.x & 31) == 0)
+                        got = mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag) ? 1 : 0;
+                    got = __shfl_sync(0xffffffffu, got, 0);
+                    if (!got) { ok = false; break; }
                     const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
