@@ -348,6 +348,104 @@ __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __restric
     }
 }
 
+// Single-pass form of vlp_ln_merge_kernel for C <= 256 * kVec: each lane keeps its
+// kVec 8-channel vectors of the patch in registers, so the patch is read from memory
+// once. Same statistics (sum, then sum of squared deviations, in fp32) and rounding.
+template <bool kF32In, int kVec>
+__global__ void __launch_bounds__(256) vlp_ln_merge_regs_kernel(const void* __restrict__ x,
+                                                                const int2* __restrict__ gmeta, int M, int k, int C,
+                                                                const float* __restrict__ gamma,
+                                                                const float* __restrict__ beta, float eps, int has_ln,
+                                                                __nv_bfloat16* __restrict__ A) {
+    const int lane = threadIdx.x & 31;
+    const int kk = k * k;
+    const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (item >= static_cast<int64_t>(M) * kk) return;
+    const int m = static_cast<int>(item / kk), p = static_cast<int>(item - static_cast<int64_t>(m) * kk);
+    const int dy = p / k, dx = p - dy * k;
+    const int2 g = gmeta[m];
+    const uint32_t wm = static_cast<uint32_t>(g.y);
+    const int nvec = C / 8;
+    uint4* dst = reinterpret_cast<uint4*>(A + (static_cast<int64_t>(m) * kk + p) * C);
+    if (!((wm >> p) & 1u)) {
+        for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const int64_t row = static_cast<int64_t>(g.x) + dy * static_cast<int>(wm >> 16) + dx;
+    float f[kVec][8];
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+        const int v = lane + 32 * i;
+        if (v < nvec) {
+            if (kF32In) {
+                const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * C) + 2 * v;
+                const float4 a = __ldg(src), b = __ldg(src + 1);
+                f[i][0] = a.x; f[i][1] = a.y; f[i][2] = a.z; f[i][3] = a.w;
+                f[i][4] = b.x; f[i][5] = b.y; f[i][6] = b.z; f[i][7] = b.w;
+            } else {
+                const uint4 u =
+                    __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + row * C) + v);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    f[i][2 * e] = __uint_as_float(w[e] << 16);
+                    f[i][2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[i][e] = 0.f;
+        }
+    }
+    float mean = 0.f, rstd = 1.f;
+    if (has_ln) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < kVec; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s += f[i][e];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        mean = s / static_cast<float>(C);
+        float q = 0.f;
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) {
+            if (lane + 32 * i < nvec) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float d = f[i][e] - mean;
+                    q += d * d;
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+        rstd = rsqrtf(q / static_cast<float>(C) + eps);
+    }
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+        const int v = lane + 32 * i;
+        if (v >= nvec) continue;
+        if (has_ln) {
+            const float4* g4 = reinterpret_cast<const float4*>(gamma) + 2 * v;
+            const float4* b4 = reinterpret_cast<const float4*>(beta) + 2 * v;
+            const float4 g0 = __ldg(g4), g1 = __ldg(g4 + 1), b0 = __ldg(b4), b1 = __ldg(b4 + 1);
+            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[i][e] = (f[i][e] - mean) * rstd * gg[e] + bb[e];
+        }
+        uint4 o;
+        __nv_bfloat162 t0 = __floats2bfloat162_rn(f[i][0], f[i][1]), t1 = __floats2bfloat162_rn(f[i][2], f[i][3]);
+        __nv_bfloat162 t2 = __floats2bfloat162_rn(f[i][4], f[i][5]), t3 = __floats2bfloat162_rn(f[i][6], f[i][7]);
+        o.x = *reinterpret_cast<uint32_t*>(&t0);
+        o.y = *reinterpret_cast<uint32_t*>(&t1);
+        o.z = *reinterpret_cast<uint32_t*>(&t2);
+        o.w = *reinterpret_cast<uint32_t*>(&t3);
+        dst[v] = o;
+    }
+}
+
 // ---------------------------------------------------------------- newline / separator rows
 struct ImageDesc {
     int32_t row_base;       // first assembled row of the image (over all images)

@@ -1,8 +1,10 @@
 // C-ABI host library of the vision-to-language projector (declared in vlproj.h).
 //
-// vlproj_forward enqueues, on the caller's stream and without any host sync:
-//   0. placeholder index   count + compact (ids == image_token_id), count check
-//   1. geometry            per GEMM row: destination row; per im2col chunk: the
+// vlproj_forward enqueues, without any host sync:
+//   0. placeholder index   count + compact (ids == image_token_id), count check, and
+//                          each GEMM row's destination row; on a side stream forked
+//                          from the caller's stream and joined back before step 4
+//   1. geometry            per GEMM row: gather data; per im2col chunk: the
 //                          coordinates of its first token
 //   2. LayerNorm/convert   only with a pre-merge LayerNorm or fp32 features
 //   3. GEMM1               im2col merge-gather + tcgen05 MMA + bias + GELU -> H (bf16)
@@ -403,10 +405,14 @@ struct vlproj_handle {
     int* status = nullptr;       // [0] latched error, [1] per-forward count check
     Uploader up_views, up_images, up_maps;
     std::vector<CUtensorMap> host_maps;
-    // tracing
+    // the placeholder index runs on `side`, forked from / joined to the caller's stream
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    // tracing: start / end event of every stage, recorded on the stream that runs it
     bool profiling = false;
     bool profiled_valid = false;
-    cudaEvent_t ev[VLPROJ_NUM_STAGES + 1] = {};
+    cudaEvent_t ev_begin[VLPROJ_NUM_STAGES] = {};
+    cudaEvent_t ev_end[VLPROJ_NUM_STAGES] = {};
     bool stage_ran[VLPROJ_NUM_STAGES] = {};
     int64_t launches = 0;
     // cached tensor map of H
@@ -417,9 +423,31 @@ struct vlproj_handle {
 
 namespace {
 
-// Record the boundary before stage `stage` (stage == VLPROJ_NUM_STAGES closes the last).
-void mark(vlproj_handle* h, int stage, cudaStream_t s) {
-    if (h->profiling) cudaEventRecord(h->ev[stage], s);
+// Stage timing: begin / end events on the stream that runs the stage.
+void stage_begin(vlproj_handle* h, int stage, cudaStream_t s) {
+    h->stage_ran[stage] = true;
+    if (h->profiling) cudaEventRecord(h->ev_begin[stage], s);
+}
+void stage_end(vlproj_handle* h, int stage, cudaStream_t s) {
+    if (h->profiling) cudaEventRecord(h->ev_end[stage], s);
+}
+
+// LayerNorm-merge launch: the single-pass (registers) form when C fits.
+int launch_ln_merge(const vlproj_config& c, const void* features, const int2* gmeta, int M, const float* gamma,
+                    const float* beta, float eps, __nv_bfloat16* A, cudaStream_t s) {
+    const int64_t items = static_cast<int64_t>(M) * c.k * c.k;
+    const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+    const int nvec = c.C / 8;
+    const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
+#define VLP_LNM(F, V) vlp::vlp_ln_merge_regs_kernel<F, V><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A)
+    if (nvec <= 64) { if (f32) VLP_LNM(true, 2); else VLP_LNM(false, 2); }
+    else if (nvec <= 160) { if (f32) VLP_LNM(true, 5); else VLP_LNM(false, 5); }
+    else if (nvec <= 256) { if (f32) VLP_LNM(true, 8); else VLP_LNM(false, 8); }
+    else if (f32) vlp::vlp_ln_merge_kernel<true><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A);
+    else vlp::vlp_ln_merge_kernel<false><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A);
+#undef VLP_LNM
+    VLP_CUDA(cudaGetLastError());
+    return VLPROJ_OK;
 }
 
 int upload_plan(vlproj_handle* h, const Plan& pl, cudaStream_t s) {
@@ -449,8 +477,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     if (cpasync && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
     if (im2col && h->chunks.ensure(std::max(n_chunks, 1))) return VLPROJ_ERR_CUDA;
 
-    mark(h, 1, s);
-    h->stage_ran[1] = true;
+    stage_begin(h, 1, s);
     ++h->launches;
     const int geo_threads = std::max(M, n_chunks);
     vlp::vlp_geometry_kernel<<<(geo_threads + 255) / 256, 256, 0, s>>>(
@@ -458,25 +485,19 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
         cpasync ? h->gmeta.ptr : nullptr, h->rowdest.ptr, im2col ? h->chunks.ptr : nullptr, n_chunks, pl.chunk,
         pl.uniform ? 1 : 0);
     VLP_CUDA(cudaGetLastError());
+    stage_end(h, 1, s);
 
     const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(features);
-    mark(h, 2, s);
     if (pl.merged_ln) {
-        h->stage_ran[2] = true;
+        stage_begin(h, 2, s);
         ++h->launches;
         if (h->A.ensure(static_cast<size_t>(M) * h->K1)) return VLPROJ_ERR_CUDA;
-        const int64_t items = static_cast<int64_t>(M) * c.k * c.k;
-        const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
         const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
-        if (c.feat_dtype == VLPROJ_FEAT_F32)
-            vlp::vlp_ln_merge_kernel<true><<<blocks, 256, 0, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma,
-                                                                  h->beta, eps, c.has_ln, h->A.ptr);
-        else
-            vlp::vlp_ln_merge_kernel<false><<<blocks, 256, 0, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma,
-                                                                   h->beta, eps, c.has_ln, h->A.ptr);
-        VLP_CUDA(cudaGetLastError());
+        int rc = launch_ln_merge(c, features, h->gmeta.ptr, M, h->gamma, h->beta, eps, h->A.ptr, s);
+        if (rc) return rc;
+        stage_end(h, 2, s);
     } else if (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) {
-        h->stage_ran[2] = true;
+        stage_begin(h, 2, s);
         ++h->launches;
         if (h->Xn.ensure(static_cast<size_t>(pl.P) * c.C)) return VLPROJ_ERR_CUDA;
         const unsigned blocks = static_cast<unsigned>((pl.P + 7) / 8);
@@ -488,6 +509,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
             vlp::vlp_layernorm_kernel<false><<<blocks, 256, 0, s>>>(features, pl.P, c.C, h->gamma, h->beta, eps,
                                                                     c.has_ln, h->Xn.ptr);
         VLP_CUDA(cudaGetLastError());
+        stage_end(h, 2, s);
         src = h->Xn.ptr;
     }
 
@@ -542,20 +564,24 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
         p.gmeta = h->gmeta.ptr;
     }
 
-    mark(h, 3, s);
-    h->stage_ran[3] = true;
+    stage_begin(h, 3, s);
     ++h->launches;
+    int rc;
     if (pl.merged_ln)
-        return launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                        h->num_sms, s);
+    else if (pl.box5)
+        rc = launch_gemm_bn<vlp::A_BOX5, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                        h->num_sms, s);
+    else if (im2col)
+        rc = launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
                                                           h->num_sms, s);
-    if (pl.box5)
-        return launch_gemm_bn<vlp::A_BOX5, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                          h->num_sms, s);
-    if (im2col)
-        return launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                            h->num_sms, s);
-    return launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(pick_bn(c.N1), false, tmA, h->tmW1, h->tmW1h, p, h->num_sms,
-                                                         s);
+    else
+        rc = launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(pick_bn(c.N1), false, tmA, h->tmW1, h->tmW1h, p,
+                                                           h->num_sms, s);
+    if (rc) return rc;
+    stage_end(h, 3, s);
+    return VLPROJ_OK;
 }
 
 }  // namespace
@@ -618,7 +644,9 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
     const size_t n1 = static_cast<size_t>(cfg->N1), n2 = static_cast<size_t>(cfg->N2), C = static_cast<size_t>(cfg->C);
     if (cudaMalloc(&h->W1p, n1 * h->K1 * 2) || cudaMalloc(&h->W2, n2 * n1 * 2) || cudaMalloc(&h->b1, n1 * 4) ||
         cudaMalloc(&h->b2, n2 * 4) || cudaMalloc(&h->gamma, C * 4) || cudaMalloc(&h->beta, C * 4) ||
-        cudaMalloc(&h->status, 2 * sizeof(int)))
+        cudaMalloc(&h->status, 2 * sizeof(int)) || cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) ||
+        cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming) ||
+        cudaEventCreateWithFlags(&h->join, cudaEventDisableTiming))
         return fail(VLPROJ_ERR_CUDA);
     cudaStream_t s = nullptr;
     vlp::vlp_permute_w1_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(cfg->W1), h->W1p,
@@ -675,8 +703,13 @@ void vlproj_destroy(vlproj_handle* h) {
     h->up_views.release();
     h->up_images.release();
     h->up_maps.release();
-    for (auto& e : h->ev)
+    for (auto& e : h->ev_begin)
         if (e) cudaEventDestroy(e);
+    for (auto& e : h->ev_end)
+        if (e) cudaEventDestroy(e);
+    if (h->fork) cudaEventDestroy(h->fork);
+    if (h->join) cudaEventDestroy(h->join);
+    if (h->side) cudaStreamDestroy(h->side);
     cudaSetDevice(cur);
     delete h;
 }
@@ -746,34 +779,51 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
     int rc = build_plan(c, grid_hw, spatial_crop, n_images, false, h->gather_mode, &pl);
     if (rc) return rc;
 
-    // 0. placeholder index
+    // 0. placeholder index (and each GEMM row's destination), on the side stream so it
+    //    overlaps the geometry / LayerNorm / GEMM1 chain on the caller's stream
     const int nblocks = static_cast<int>((n_ids + vlp::SCAN_CHUNK - 1) / vlp::SCAN_CHUNK);
     if (h->counts.ensure(std::max(nblocks, 1)) || h->pos.ensure(std::max<int64_t>(pl.R, 1)))
         return VLPROJ_ERR_CUDA;
+    if (pl.M > 0 && h->rowdest.ensure(pl.M)) return VLPROJ_ERR_CUDA;
+    if (pl.M > 0 && h->H.ensure(static_cast<size_t>(pl.M) * c.N1)) return VLPROJ_ERR_CUDA;
     rc = upload_plan(h, pl, s);
     if (rc) return rc;
     h->profiled_valid = false;
     for (bool& r : h->stage_ran) r = false;
-    mark(h, 0, s);
-    h->stage_ran[0] = true;
+    cudaStream_t si = pl.M > 0 ? h->side : s;
+    if (si != s) {
+        VLP_CUDA(cudaEventRecord(h->fork, s));
+        VLP_CUDA(cudaStreamWaitEvent(si, h->fork, 0));
+    }
+    stage_begin(h, 0, si);
     h->launches += nblocks > 0 ? 2 : 1;
     if (nblocks > 0) {
-        vlp::vlp_count_kernel<<<nblocks, vlp::SCAN_THREADS, 0, s>>>(input_ids, n_ids, image_token_id, h->counts.ptr);
+        vlp::vlp_count_kernel<<<nblocks, vlp::SCAN_THREADS, 0, si>>>(input_ids, n_ids, image_token_id,
+                                                                     h->counts.ptr);
         VLP_CUDA(cudaGetLastError());
     }
-    vlp::vlp_compact_kernel<<<std::max(nblocks, 1), vlp::SCAN_THREADS, 0, s>>>(
+    vlp::vlp_compact_kernel<<<std::max(nblocks, 1), vlp::SCAN_THREADS, 0, si>>>(
         input_ids, n_ids, image_token_id, h->counts.ptr, nblocks, h->pos.ptr, pl.R, h->status + 1, h->status);
     VLP_CUDA(cudaGetLastError());
+    if (pl.M > 0) {
+        ++h->launches;
+        const int M = static_cast<int>(pl.M);
+        vlp::vlp_geometry_kernel<<<(M + 255) / 256, 256, 0, si>>>(h->dviews.ptr, static_cast<int>(pl.views.size()),
+                                                                  M, c.k, h->pos.ptr, pl.R, vlp::DEST_EMBED, nullptr,
+                                                                  h->rowdest.ptr, nullptr, 0, pl.chunk, 0);
+        VLP_CUDA(cudaGetLastError());
+    }
+    stage_end(h, 0, si);
     if (pl.M == 0) {
-        for (int st = 1; st <= VLPROJ_NUM_STAGES; ++st) mark(h, st, s);
         h->profiled_valid = h->profiling;
         return VLPROJ_OK;
     }
+    VLP_CUDA(cudaEventRecord(h->join, si));
 
     // 1-3. geometry, LayerNorm, GEMM1 -> H
-    if (h->H.ensure(static_cast<size_t>(pl.M) * c.N1)) return VLPROJ_ERR_CUDA;
-    rc = run_merge_gemm1(h, pl, features, h->pos.ptr, vlp::DEST_EMBED, h->H.ptr, pl.M, s);
+    rc = run_merge_gemm1(h, pl, features, nullptr, vlp::DEST_NONE, h->H.ptr, pl.M, s);
     if (rc) return rc;
+    VLP_CUDA(cudaStreamWaitEvent(s, h->join, 0));
 
     // 4. GEMM2 + scatter
     if (h->tmH_ptr != h->H.ptr || h->tmH_rows != pl.M) {
@@ -794,17 +844,16 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
     p.fwd_status = h->status + 1;
     p.err = h->status;
     p.wait_ns = h->wait_ns;
-    mark(h, 4, s);
-    h->stage_ran[4] = true;
+    stage_begin(h, 4, s);
     ++h->launches;
     rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(pick_bn(c.N2), h->pairs, h->tmH, h->tmW2, h->tmW2h, p,
                                                        h->num_sms, s);
     if (rc) return rc;
+    stage_end(h, 4, s);
 
     // 5. newline / separator rows
-    mark(h, 5, s);
     if (tiled && !pl.images.empty()) {
-        h->stage_ran[5] = true;
+        stage_begin(h, 5, s);
         ++h->launches;
         dim3 grid(pl.max_special, static_cast<unsigned>(pl.images.size()));
         vlp::vlp_special_rows_kernel<<<grid, 128, 0, s>>>(h->dimages.ptr, h->pos.ptr, pl.R,
@@ -813,16 +862,17 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
                                                           static_cast<__nv_bfloat16*>(out_embeds), n_ids, c.N2,
                                                           h->status + 1);
         VLP_CUDA(cudaGetLastError());
+        stage_end(h, 5, s);
     }
-    mark(h, VLPROJ_NUM_STAGES, s);
     h->profiled_valid = h->profiling;
     return VLPROJ_OK;
 }
 
 int vlproj_profile_enable(vlproj_handle* h, int enable) {
     if (!h) return VLPROJ_ERR_INVALID_ARG;
-    if (enable && !h->ev[0]) {
-        for (auto& e : h->ev) VLP_CUDA(cudaEventCreate(&e));
+    if (enable && !h->ev_begin[0]) {
+        for (auto& e : h->ev_begin) VLP_CUDA(cudaEventCreate(&e));
+        for (auto& e : h->ev_end) VLP_CUDA(cudaEventCreate(&e));
     }
     h->profiling = enable != 0;
     h->profiled_valid = false;
@@ -832,11 +882,13 @@ int vlproj_profile_enable(vlproj_handle* h, int enable) {
 int vlproj_profile_read(vlproj_handle* h, float* ms, int n) {
     if (!h || !ms || n < 0) return VLPROJ_ERR_INVALID_ARG;
     if (!h->profiled_valid) return VLPROJ_ERR_INVALID_ARG;
-    VLP_CUDA(cudaEventSynchronize(h->ev[VLPROJ_NUM_STAGES]));
     const int m = std::min(n, VLPROJ_NUM_STAGES);
     for (int i = 0; i < m; ++i) {
         float t = 0.f;
-        if (h->stage_ran[i]) VLP_CUDA(cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]));
+        if (h->stage_ran[i]) {
+            VLP_CUDA(cudaEventSynchronize(h->ev_end[i]));
+            VLP_CUDA(cudaEventElapsedTime(&t, h->ev_begin[i], h->ev_end[i]));
+        }
         ms[i] = t;
     }
     return m;
