@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -333,25 +333,29 @@ def main():
         roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
                 "frac": None, "peak_source": peak_src, "traffic": None}
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers. Per step: the step's inputs
+    # (features, ids) from pinned host memory to the device, vlproj_forward_ex (projection,
+    # plus the token-embedding lookup of the text rows from the device-resident table and a
+    # compact copy of the assembled rows), and the assembled rows back to pinned host memory.
     e2e = None
     if args.e2e_steps > 0:
+        table = bf(W.embed_table(wl, seed))
+        R = int(sum(rows))
         feats_p = (torch.from_numpy(feats_h) if wl.feat_fp32 else torch.from_numpy(feats_h.view(np.int16))).pin_memory()
         ids_p = torch.from_numpy(ids_h).pin_memory()
-        pre_p = torch.from_numpy(prefill_h.view(np.int16)).pin_memory()
-        res_p = torch.empty_like(pre_p).pin_memory()
+        rows_d = torch.empty((R, wl.N2), dtype=torch.bfloat16, device="cuda")
+        rows_p = torch.empty((R, wl.N2), dtype=torch.int16).pin_memory()
         feats_d = torch.empty(feats_p.shape, dtype=feats_p.dtype, device="cuda")
         ids_d = torch.empty_like(ids)
-        out_d = torch.empty(pre_p.shape, dtype=torch.int16, device="cuda")
+        emb_d = torch.empty_like(out)
 
         def e2e_step():
             feats_d.copy_(feats_p, non_blocking=True)
             ids_d.copy_(ids_p, non_blocking=True)
-            out_d.copy_(pre_p, non_blocking=True)
             f = feats_d if wl.feat_fp32 else feats_d.view(torch.bfloat16)
-            proj.forward(f, hw, crop, ids_d, W.IMAGE_TOKEN_ID, out_d.view(torch.bfloat16), newline, sep,
-                         stream=stream, n_images=wl.n_images)
-            res_p.copy_(out_d, non_blocking=True)
+            proj.forward_ex(f, hw, crop, ids_d, W.IMAGE_TOKEN_ID, emb_d, newline, sep, embed_table=table,
+                            rows_out=rows_d, stream=stream, n_images=wl.n_images)
+            rows_p.copy_(rows_d.view(torch.int16), non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -375,9 +379,10 @@ def main():
         if st != vp.OK:
             raise SystemExit(f"e2e steps failed: {vp.strerror(st)}")
         e2e = {"value": world * tokens_per_step * args.e2e_steps / (e_ms / 1000.0), "unit": UNIT,
-               "h2d_bytes_per_step": int(feats_p.numel() * feats_p.element_size() + ids_p.numel() * 8 +
-                                         pre_p.numel() * 2),
-               "d2h_bytes_per_step": int(res_p.numel() * 2), "steps": args.e2e_steps}
+               "h2d_bytes_per_step": int(feats_p.numel() * feats_p.element_size() + ids_p.numel() * 8),
+               "d2h_bytes_per_step": int(rows_p.numel() * 2), "steps": args.e2e_steps,
+               "path": "vlproj_forward_ex: host features + ids in; token-embedding lookup from the resident "
+                       "table; assembled rows out"}
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None

@@ -127,6 +127,38 @@ int vlproj_forward(vlproj_handle* h,
                    void* out_embeds,
                    void* stream);
 
+/* Extended forward: everything vlproj_forward does, plus two optional outputs.
+ *   embed_table  DEVICE bf16 [vocab][N2], or NULL. When given, every row i of out_embeds
+ *                whose id is not the placeholder is written as embed_table[input_ids[i]]:
+ *                the language model's token-embedding lookup that the assembled rows then
+ *                overwrite at the placeholders ("port DeepSeek-VL2", end of Tile-sequence
+ *                assembly), done in the same call on a side stream while the GEMMs run.
+ *                An id outside [0, vocab) gives a zero row and latches
+ *                VLPROJ_ERR_INVALID_ARG (read with vlproj_status).
+ *   rows_out     DEVICE bf16 [rows_out_cap][N2], or NULL. When given, the R assembled rows
+ *                of the batch (projected rows, newlines and separators, in placeholder
+ *                order) are also written here contiguously; rows_out_cap must be >= R
+ *                (vlproj_image_rows gives R), else VLPROJ_ERR_INVALID_ARG before any
+ *                launch. Nothing is written when the placeholder count check fails.
+ * All other fields mean what the arguments of vlproj_forward mean. */
+typedef struct vlproj_forward_args {
+    const void*    features;
+    const int32_t* grid_hw;
+    const int32_t* spatial_crop;
+    int32_t        n_images;
+    const int64_t* input_ids;
+    int64_t        n_ids;
+    int64_t        image_token_id;
+    const void*    newline;
+    const void*    sep;
+    void*          out_embeds;
+    const void*    embed_table;
+    int64_t        vocab;
+    void*          rows_out;
+    int64_t        rows_out_cap;
+} vlproj_forward_args;
+int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* stream);
+
 /* Stage output for inspection: the bf16 hidden activation H = GELU(A W1^T + b1)
  * of every merged token, views in order, tokens row-major inside a view.
  * hidden is DEVICE bf16 [M][N1], M = sum over views of ceil(h/k)*ceil(w/k). */

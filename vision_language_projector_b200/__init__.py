@@ -26,7 +26,7 @@ ORDER_CHANNEL_OUTER, ORDER_POSITION_OUTER = 0, 1
 EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status", "vlproj_destroy",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
             "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
-            "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc")
+            "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc", "vlproj_forward_ex")
 NOALLOC_MAX_IDS = 64 * 1024 * 1024
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX = 0, 1, 2, 3
 NUM_STAGES = 6
@@ -37,6 +37,17 @@ class VlprojError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
         super().__init__(f"{what}: {strerror(code)} ({code})")
+
+
+class ForwardArgs(ctypes.Structure):
+    """Mirror of ``vlproj_forward_args``."""
+    _fields_ = [
+        ("features", ctypes.c_void_p), ("grid_hw", ctypes.c_void_p), ("spatial_crop", ctypes.c_void_p),
+        ("n_images", ctypes.c_int32), ("input_ids", ctypes.c_void_p), ("n_ids", ctypes.c_int64),
+        ("image_token_id", ctypes.c_int64), ("newline", ctypes.c_void_p), ("sep", ctypes.c_void_p),
+        ("out_embeds", ctypes.c_void_p), ("embed_table", ctypes.c_void_p), ("vocab", ctypes.c_int64),
+        ("rows_out", ctypes.c_void_p), ("rows_out_cap", ctypes.c_int64),
+    ]
 
 
 class Config(ctypes.Structure):
@@ -84,6 +95,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_set_gather_mode.restype = ctypes.c_int
     lib.vlproj_set_tile_pairs.argtypes = [P, ctypes.c_int]
     lib.vlproj_set_tile_pairs.restype = ctypes.c_int
+    lib.vlproj_forward_ex.argtypes = [P, ctypes.POINTER(ForwardArgs), P]
+    lib.vlproj_forward_ex.restype = ctypes.c_int
     lib.vlproj_placeholder_index_noalloc.argtypes = [P, I64, I64, P, I64, P, P]
     lib.vlproj_placeholder_index_noalloc.restype = ctypes.c_int
     return lib
@@ -198,6 +211,25 @@ class Projector:
                                  _stream_ptr(stream))
         if check and rc != OK:
             raise VlprojError(rc, "vlproj_forward")
+        return rc
+
+    def forward_ex(self, features, grid_hw, spatial_crop, input_ids, image_token_id: int, out_embeds,
+                   newline=None, sep=None, embed_table=None, rows_out=None, stream=None,
+                   n_images: Optional[int] = None, check: bool = True) -> int:
+        """vlproj_forward_ex: forward plus the optional token-embedding lookup (embed_table,
+        (vocab, N2) bf16) and a compact copy of the assembled rows (rows_out, (>= R, N2))."""
+        g = _host_i32(grid_hw)
+        c = _host_i32(spatial_crop)
+        if n_images is None:
+            n_images = len(c) if c is not None else (0 if g is None else len(g))
+        a = ForwardArgs(_ptr(features), _ptr(g), _ptr(c), n_images, _ptr(input_ids),
+                        0 if input_ids is None else int(input_ids.numel()), int(image_token_id), _ptr(newline),
+                        _ptr(sep), _ptr(out_embeds), _ptr(embed_table),
+                        0 if embed_table is None else int(embed_table.shape[0]), _ptr(rows_out),
+                        0 if rows_out is None else int(rows_out.shape[0]))
+        rc = _lib.vlproj_forward_ex(self._h, ctypes.byref(a), _stream_ptr(stream))
+        if check and rc != OK:
+            raise VlprojError(rc, "vlproj_forward_ex")
         return rc
 
     def hidden(self, features, grid_hw, hidden, stream=None) -> None:

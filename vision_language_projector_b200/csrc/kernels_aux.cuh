@@ -487,6 +487,45 @@ __global__ void __launch_bounds__(128) vlp_special_rows_kernel(const ImageDesc* 
     for (int v = threadIdx.x; v < N / 8; v += blockDim.x) d4[v] = __ldg(&s4[v]);
 }
 
+// ---------------------------------------------------------------- token-embedding lookup
+// One warp per row: out[r] = table[ids[r]] for every id that is not the placeholder; an
+// id outside [0, vocab) writes a zero row and latches VLPROJ_ERR_INVALID_ARG.
+__global__ void __launch_bounds__(256) vlp_embed_lookup_kernel(const int64_t* __restrict__ ids, int64_t n,
+                                                               int64_t token, const __nv_bfloat16* __restrict__ table,
+                                                               int64_t vocab, __nv_bfloat16* __restrict__ out, int N,
+                                                               int* err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (r >= n) return;
+    const int64_t id = __ldg(&ids[r]);
+    if (id == token) return;
+    uint4* d4 = reinterpret_cast<uint4*>(out + r * N);
+    const int nvec = N / 8;
+    if (id < 0 || id >= vocab) {
+        for (int v = lane; v < nvec; v += 32) d4[v] = make_uint4(0, 0, 0, 0);
+        if (lane == 0) atomicCAS(err, 0, -1);
+        return;
+    }
+    const uint4* s4 = reinterpret_cast<const uint4*>(table + id * N);
+    for (int v = lane; v < nvec; v += 32) d4[v] = __ldg(&s4[v]);
+}
+
+// rows_out[j] = out[pos[j]] for the R assembled rows (nothing when the count check failed).
+__global__ void __launch_bounds__(256) vlp_gather_rows_kernel(const int32_t* __restrict__ pos, int64_t R,
+                                                              const __nv_bfloat16* __restrict__ out, int64_t out_rows,
+                                                              int N, __nv_bfloat16* __restrict__ rows_out,
+                                                              const int* __restrict__ fwd_status) {
+    if (*fwd_status != 0) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (j >= R) return;
+    const int64_t d = pos[j];
+    if (d < 0 || d >= out_rows) return;
+    const uint4* s4 = reinterpret_cast<const uint4*>(out + d * N);
+    uint4* d4 = reinterpret_cast<uint4*>(rows_out + j * N);
+    for (int v = lane; v < N / 8; v += 32) d4[v] = s4[v];
+}
+
 // ---------------------------------------------------------------- W1 column permutation
 // dst[n][p*C + c] = src[n][c*kk + p] for p < kk = k*k (channel-outermost input);
 // with position_outer the columns are copied unchanged.

@@ -407,7 +407,7 @@ struct vlproj_handle {
     std::vector<CUtensorMap> host_maps;
     // the placeholder index runs on `side`, forked from / joined to the caller's stream
     cudaStream_t side = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr;
     // tracing: start / end event of every stage, recorded on the stream that runs it
     bool profiling = false;
     bool profiled_valid = false;
@@ -646,7 +646,8 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
         cudaMalloc(&h->b2, n2 * 4) || cudaMalloc(&h->gamma, C * 4) || cudaMalloc(&h->beta, C * 4) ||
         cudaMalloc(&h->status, 2 * sizeof(int)) || cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) ||
         cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming) ||
-        cudaEventCreateWithFlags(&h->join, cudaEventDisableTiming))
+        cudaEventCreateWithFlags(&h->join, cudaEventDisableTiming) ||
+        cudaEventCreateWithFlags(&h->join2, cudaEventDisableTiming))
         return fail(VLPROJ_ERR_CUDA);
     cudaStream_t s = nullptr;
     vlp::vlp_permute_w1_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(cfg->W1), h->W1p,
@@ -709,6 +710,7 @@ void vlproj_destroy(vlproj_handle* h) {
         if (e) cudaEventDestroy(e);
     if (h->fork) cudaEventDestroy(h->fork);
     if (h->join) cudaEventDestroy(h->join);
+    if (h->join2) cudaEventDestroy(h->join2);
     if (h->side) cudaStreamDestroy(h->side);
     cudaSetDevice(cur);
     delete h;
@@ -764,7 +766,32 @@ int vlproj_hidden(vlproj_handle* h, const void* features, const int32_t* grid_hw
 int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_hw, const int32_t* spatial_crop,
                    int32_t n_images, const int64_t* input_ids, int64_t n_ids, int64_t image_token_id,
                    const void* newline, const void* sep, void* out_embeds, void* stream) {
-    if (!h) return VLPROJ_ERR_INVALID_ARG;
+    vlproj_forward_args a{};
+    a.features = features;
+    a.grid_hw = grid_hw;
+    a.spatial_crop = spatial_crop;
+    a.n_images = n_images;
+    a.input_ids = input_ids;
+    a.n_ids = n_ids;
+    a.image_token_id = image_token_id;
+    a.newline = newline;
+    a.sep = sep;
+    a.out_embeds = out_embeds;
+    return vlproj_forward_ex(h, &a, stream);
+}
+
+int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* stream) {
+    if (!h || !args) return VLPROJ_ERR_INVALID_ARG;
+    const void* features = args->features;
+    const int32_t* grid_hw = args->grid_hw;
+    const int32_t* spatial_crop = args->spatial_crop;
+    const int32_t n_images = args->n_images;
+    const int64_t* input_ids = args->input_ids;
+    const int64_t n_ids = args->n_ids;
+    const int64_t image_token_id = args->image_token_id;
+    const void* newline = args->newline;
+    const void* sep = args->sep;
+    void* out_embeds = args->out_embeds;
     const vlproj_config& c = h->cfg;
     if (n_ids < 0 || n_ids >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
     if (n_ids > 0 && (!input_ids || !out_embeds)) return VLPROJ_ERR_INVALID_ARG;
@@ -774,10 +801,15 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
     if (reinterpret_cast<uintptr_t>(out_embeds) % 16 || reinterpret_cast<uintptr_t>(features) % 16 ||
         (tiled && (reinterpret_cast<uintptr_t>(newline) % 16 || reinterpret_cast<uintptr_t>(sep) % 16)))
         return VLPROJ_ERR_INVALID_ARG;
+    if (args->embed_table && (args->vocab <= 0 || reinterpret_cast<uintptr_t>(args->embed_table) % 16))
+        return VLPROJ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Plan pl;
     int rc = build_plan(c, grid_hw, spatial_crop, n_images, false, h->gather_mode, &pl);
     if (rc) return rc;
+    if (args->rows_out && (args->rows_out_cap < pl.R || reinterpret_cast<uintptr_t>(args->rows_out) % 16))
+        return VLPROJ_ERR_INVALID_ARG;
+    const bool lookup = args->embed_table != nullptr && n_ids > 0;
 
     // 0. placeholder index (and each GEMM row's destination), on the side stream so it
     //    overlaps the geometry / LayerNorm / GEMM1 chain on the caller's stream
@@ -790,7 +822,7 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
     if (rc) return rc;
     h->profiled_valid = false;
     for (bool& r : h->stage_ran) r = false;
-    cudaStream_t si = pl.M > 0 ? h->side : s;
+    cudaStream_t si = (pl.M > 0 || lookup) ? h->side : s;
     if (si != s) {
         VLP_CUDA(cudaEventRecord(h->fork, s));
         VLP_CUDA(cudaStreamWaitEvent(si, h->fork, 0));
@@ -814,11 +846,21 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
         VLP_CUDA(cudaGetLastError());
     }
     stage_end(h, 0, si);
+    if (si != s) VLP_CUDA(cudaEventRecord(h->join, si));
+    if (lookup) {
+        // token-embedding rows: independent of the projector, overlaps the GEMMs
+        ++h->launches;
+        vlp::vlp_embed_lookup_kernel<<<static_cast<unsigned>((n_ids + 7) / 8), 256, 0, si>>>(
+            input_ids, n_ids, image_token_id, static_cast<const __nv_bfloat16*>(args->embed_table), args->vocab,
+            static_cast<__nv_bfloat16*>(out_embeds), c.N2, h->status);
+        VLP_CUDA(cudaGetLastError());
+        VLP_CUDA(cudaEventRecord(h->join2, si));
+    }
     if (pl.M == 0) {
+        if (si != s) VLP_CUDA(cudaStreamWaitEvent(s, lookup ? h->join2 : h->join, 0));
         h->profiled_valid = h->profiling;
         return VLPROJ_OK;
     }
-    VLP_CUDA(cudaEventRecord(h->join, si));
 
     // 1-3. geometry, LayerNorm, GEMM1 -> H
     rc = run_merge_gemm1(h, pl, features, nullptr, vlp::DEST_NONE, h->H.ptr, pl.M, s);
@@ -864,6 +906,14 @@ int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_h
         VLP_CUDA(cudaGetLastError());
         stage_end(h, 5, s);
     }
+    if (args->rows_out && pl.R > 0) {
+        ++h->launches;
+        vlp::vlp_gather_rows_kernel<<<static_cast<unsigned>((pl.R + 7) / 8), 256, 0, s>>>(
+            h->pos.ptr, pl.R, static_cast<const __nv_bfloat16*>(out_embeds), n_ids, c.N2,
+            static_cast<__nv_bfloat16*>(args->rows_out), h->status + 1);
+        VLP_CUDA(cudaGetLastError());
+    }
+    if (lookup) VLP_CUDA(cudaStreamWaitEvent(s, h->join2, 0));
     h->profiled_valid = h->profiling;
     return VLPROJ_OK;
 }
