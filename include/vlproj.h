@@ -206,6 +206,23 @@ int vlproj_set_gather_mode(vlproj_handle* h, int mode);
  * tiles on single CTAs. Both give the same bits. */
 int vlproj_set_tile_pairs(vlproj_handle* h, int enable);
 
+/* Host only, no device work: the processor's tiling choices for the 2D tile scheme
+ * ("port DeepSeek-VL2", Processor steps 1, 2, 6, 7). For each image of one request,
+ * with original size image_wh[i] = (w0, h0) in pixels (width first):
+ *   - cropping applies only when the request has at most 2 images (else grid 1x1);
+ *   - with cropping, the candidate (W, H) in candidates[n_candidates][2] maximising
+ *     effective = min(floor(w0*s)*floor(h0*s), w0*h0), s = min(W/w0, H/h0) (IEEE
+ *     double), ties to the least wasted area W*H - effective, first candidate on a
+ *     full tie;
+ *   - spatial_crop_out[i] = (tw, th) = (W / image_size, H / image_size);
+ *   - rows_out[i] = h'(w'+1) + 1 + (th h')(tw w'+1) placeholders, h' = w' =
+ *     ceil(floor(image_size / patch_size) / downsample).
+ * Returns the number of views, sum of (1 + tw*th), or an error code (< 0). Each view
+ * is one image_size x image_size tile with a floor(image_size/patch_size) square grid. */
+int64_t vlproj_plan_tiles(const int32_t* image_wh, int32_t n_images, const int32_t* candidates, int32_t n_candidates,
+                          int32_t image_size, int32_t patch_size, int32_t downsample, int32_t* spatial_crop_out,
+                          int64_t* rows_out);
+
 /* Bound (nanoseconds) on every wait inside this handle's kernels; 0 restores the
  * default (2 s). A wait that runs out ends its kernel early with
  * VLPROJ_ERR_TIMEOUT latched; tests use a tiny bound to exercise that path. */

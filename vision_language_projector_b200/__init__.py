@@ -26,7 +26,8 @@ ORDER_CHANNEL_OUTER, ORDER_POSITION_OUTER = 0, 1
 EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status", "vlproj_destroy",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
             "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
-            "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc", "vlproj_forward_ex")
+            "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc", "vlproj_forward_ex",
+            "vlproj_plan_tiles")
 NOALLOC_MAX_IDS = 64 * 1024 * 1024
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX = 0, 1, 2, 3
 NUM_STAGES = 6
@@ -95,6 +96,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_set_gather_mode.restype = ctypes.c_int
     lib.vlproj_set_tile_pairs.argtypes = [P, ctypes.c_int]
     lib.vlproj_set_tile_pairs.restype = ctypes.c_int
+    lib.vlproj_plan_tiles.argtypes = [P, I32, P, I32, I32, I32, I32, P, P]
+    lib.vlproj_plan_tiles.restype = I64
     lib.vlproj_forward_ex.argtypes = [P, ctypes.POINTER(ForwardArgs), P]
     lib.vlproj_forward_ex.restype = ctypes.c_int
     lib.vlproj_placeholder_index_noalloc.argtypes = [P, I64, I64, P, I64, P, P]
@@ -158,6 +161,19 @@ def placeholder_index_noalloc(input_ids, image_token_id: int, positions, count, 
     mp = int(positions.numel()) if max_positions is None else int(max_positions)
     return _lib.vlproj_placeholder_index_noalloc(_ptr(input_ids), n, int(image_token_id), _ptr(positions), mp,
                                                  _ptr(count), _stream_ptr(stream))
+
+
+def plan_tiles(image_wh, candidates, image_size: int, patch_size: int, downsample: int):
+    """Processor tiling (host only): ((n, 2) int32 (tw, th), (n,) int64 placeholder counts, views)."""
+    wh = _host_i32(image_wh).reshape(-1, 2)
+    cand = _host_i32(candidates).reshape(-1, 2)
+    crop = np.zeros((max(len(wh), 1), 2), np.int32)
+    rows = np.zeros(max(len(wh), 1), np.int64)
+    v = _lib.vlproj_plan_tiles(wh.ctypes.data, len(wh), cand.ctypes.data, len(cand), image_size, patch_size,
+                               downsample, crop.ctypes.data, rows.ctypes.data)
+    if v < 0:
+        raise VlprojError(int(v), "vlproj_plan_tiles")
+    return crop[:len(wh)], rows[:len(wh)], int(v)
 
 
 def _stream_ptr(stream) -> Optional[int]:

@@ -17,6 +17,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -621,6 +622,49 @@ int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw, cons
         for (int32_t i = 0; i < n_images; ++i) rows_out[i] = base[i + 1] - base[i];
     }
     return pl.R;
+}
+
+int64_t vlproj_plan_tiles(const int32_t* image_wh, int32_t n_images, const int32_t* candidates, int32_t n_candidates,
+                          int32_t image_size, int32_t patch_size, int32_t downsample, int32_t* spatial_crop_out,
+                          int64_t* rows_out) {
+    if (n_images < 0 || (n_images > 0 && (!image_wh || !spatial_crop_out)) || image_size <= 0 || patch_size <= 0 ||
+        downsample <= 0 || patch_size > image_size)
+        return VLPROJ_ERR_INVALID_ARG;
+    const bool crop = n_images <= 2;
+    if (crop && n_images > 0 && (n_candidates <= 0 || !candidates)) return VLPROJ_ERR_INVALID_ARG;
+    const int64_t g = image_size / patch_size;
+    const int64_t hp = (g + downsample - 1) / downsample;
+    int64_t views = 0;
+    for (int32_t i = 0; i < n_images; ++i) {
+        const int64_t w0 = image_wh[2 * i], h0 = image_wh[2 * i + 1];
+        if (w0 <= 0 || h0 <= 0) return VLPROJ_ERR_INVALID_ARG;
+        int64_t W = image_size, H = image_size;
+        if (crop) {
+            int64_t best_eff = -1, best_waste = 0;
+            for (int32_t c = 0; c < n_candidates; ++c) {
+                const int64_t cw = candidates[2 * c], ch = candidates[2 * c + 1];
+                if (cw <= 0 || ch <= 0 || cw % image_size || ch % image_size) return VLPROJ_ERR_INVALID_ARG;
+                const double scale = std::min(static_cast<double>(cw) / static_cast<double>(w0),
+                                              static_cast<double>(ch) / static_cast<double>(h0));
+                const int64_t fw = static_cast<int64_t>(std::floor(static_cast<double>(w0) * scale));
+                const int64_t fh = static_cast<int64_t>(std::floor(static_cast<double>(h0) * scale));
+                const int64_t eff = std::min(fw * fh, w0 * h0);
+                const int64_t waste = cw * ch - eff;
+                if (eff > best_eff || (eff == best_eff && waste < best_waste)) {
+                    best_eff = eff;
+                    best_waste = waste;
+                    W = cw;
+                    H = ch;
+                }
+            }
+        }
+        const int64_t tw = W / image_size, th = H / image_size;
+        spatial_crop_out[2 * i] = static_cast<int32_t>(tw);
+        spatial_crop_out[2 * i + 1] = static_cast<int32_t>(th);
+        if (rows_out) rows_out[i] = hp * (hp + 1) + 1 + (th * hp) * (tw * hp + 1);
+        views += 1 + tw * th;
+    }
+    return views;
 }
 
 int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
