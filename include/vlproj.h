@@ -67,7 +67,9 @@ typedef struct vlproj_config {
     int32_t C;              /* vision feature width; multiple of 64 */
     int32_t N1;             /* MLP hidden width; multiple of 64 */
     int32_t N2;             /* output embedding width (n_embed); multiple of 32 */
-    int32_t depth;          /* number of Linear layers; must be 2 */
+    int32_t depth;          /* number of Linear layers, 2..8: depth > 2 inserts depth-2 pairs
+                               GELU -> Linear(N1 -> N1) between the first and the last
+                               ("port DeepSeek-VL2", Projector step 3) */
     int32_t has_ln;         /* 1: pre-merge LayerNorm over C, biased variance */
     float   ln_eps;         /* LayerNorm epsilon (1e-5 when <= 0) */
     int32_t feat_dtype;     /* VLPROJ_FEAT_BF16 or VLPROJ_FEAT_F32 features */
@@ -84,12 +86,15 @@ typedef struct vlproj_config {
     const float* b2;        /* fp32 [N2], or NULL for zeros */
     const float* ln_gamma;  /* fp32 [C] when has_ln, else ignored */
     const float* ln_beta;   /* fp32 [C] when has_ln, else ignored */
+    /* depth > 2 only: HOST arrays of depth-2 DEVICE pointers, layer order */
+    const void* const*  W_mid;   /* each bf16 [N1][N1], stored (out, in) */
+    const float* const* b_mid;   /* each fp32 [N1]; the array or an entry may be NULL (zeros) */
 } vlproj_config;
 
 typedef struct vlproj_handle vlproj_handle;
 
 /* Create a projector on the current device. Validates cfg (VLPROJ_ERR_UNSUPPORTED
- * for depth != 2, tile tag "1D", token pooling, k outside 1..3; INVALID_ARG for
+ * for depth outside 2..8, tile tag "1D", token pooling, k outside 1..3; INVALID_ARG for
  * widths that break the alignment rules above or NULL weights), allocates the
  * owned weight copies and permutes W1's columns into the kernel's gather order
  * (an exact permutation of bf16 values). On success *out holds the handle. */

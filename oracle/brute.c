@@ -116,3 +116,15 @@ long brute_row_of_newline(int n, int hp, int wp, int tw)
 
 /* Row of the view separator of a tiled image. */
 long brute_row_of_separator(int hp, int wp) { return (long)hp * (wp + 1); }
+
+/* One dense layer of a token: y[n] = b[n] + sum_q W[n][q] x[q] (W stored (out, in)),
+ * then GELU when gelu != 0, then bf16 rounding when quantise != 0. */
+void brute_dense(const double* x, int K, const double* W, const double* b, int N, int gelu, int quantise, double* y)
+{
+    for (int n = 0; n < N; ++n) {
+        double acc = b[n];
+        for (int q = 0; q < K; ++q) acc += W[(long)n * K + q] * x[q];
+        if (gelu) acc = brute_gelu(acc);
+        y[n] = quantise ? brute_round_bf16(acc) : acc;
+    }
+}

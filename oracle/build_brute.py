@@ -33,4 +33,6 @@ def load() -> ctypes.CDLL:
     lib.brute_row_of_token.argtypes, lib.brute_row_of_token.restype = [I, I, I, I, I, I, I], L
     lib.brute_row_of_newline.argtypes, lib.brute_row_of_newline.restype = [I, I, I, I], L
     lib.brute_row_of_separator.argtypes, lib.brute_row_of_separator.restype = [I, I], L
+    lib.brute_dense.argtypes = [P, I, P, P, I, I, I, P]
+    lib.brute_dense.restype = None
     return lib

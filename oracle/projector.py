@@ -83,11 +83,13 @@ def image_rows(grid_hw: np.ndarray, k: int, spatial_crop: Optional[np.ndarray]) 
     return rows
 
 
-def projector_params(C: int, k: int, N1: int, N2: int, has_ln: bool) -> int:
-    """Parameters of [LayerNorm(C)] + Linear(k*k*C -> N1) + Linear(N1 -> N2), with biases
-    ("DeepSeek-V4-Flash-Vision-BF16", first section: 2x2 merge, 4608 -> 4096)."""
+def projector_params(C: int, k: int, N1: int, N2: int, has_ln: bool, depth: int = 2) -> int:
+    """Parameters of [LayerNorm(C)] + Linear(k*k*C -> N1) + (depth-2) x Linear(N1 -> N1)
+    + Linear(N1 -> N2), with biases ("DeepSeek-V4-Flash-Vision-BF16", first section:
+    2x2 merge, 4608 -> 4096; "port DeepSeek-VL2", Projector step 3 for depth > 2)."""
     n = (2 * C if has_ln else 0)
     n += k * k * C * N1 + N1
+    n += (depth - 2) * (N1 * N1 + N1)
     n += N1 * N2 + N2
     return n
 
@@ -139,9 +141,14 @@ def hidden(a: np.ndarray, W1: np.ndarray, b1: np.ndarray, quantise_hidden: bool 
 
 
 def mlp(a: np.ndarray, W1: np.ndarray, b1: np.ndarray, W2: np.ndarray, b2: np.ndarray,
-        quantise_hidden: bool = True) -> np.ndarray:
-    """Linear -> GELU -> Linear ("port DeepSeek-VL2", Projector step 3)."""
-    return hidden(a, W1, b1, quantise_hidden) @ W2.T + b2
+        quantise_hidden: bool = True, mids: Sequence[tuple] = ()) -> np.ndarray:
+    """Linear -> GELU -> [Linear -> GELU] x len(mids) -> Linear ("port DeepSeek-VL2",
+    Projector step 3: with depth > 2 the extra GELU + Linear pairs sit in the middle).
+    Every hidden activation is rounded to bf16 (Q2) unless disabled."""
+    h = hidden(a, W1, b1, quantise_hidden)
+    for Wm, bm in mids:
+        h = hidden(h, Wm, bm, quantise_hidden)
+    return h @ W2.T + b2
 
 
 def merge_view(feat: np.ndarray, h: int, w: int, k: int, ln: Optional[tuple]) -> np.ndarray:
@@ -211,7 +218,8 @@ def project_image(feats: Sequence[np.ndarray], hw: Sequence[tuple], k: int, para
             if ln is not None:
                 x = layernorm(x, *ln)
             a = unshuffle(x.reshape(h, w, -1), k)
-        outs.append(mlp(a, params["W1"], params["b1"], params["W2"], params["b2"], quantise))
+        outs.append(mlp(a, params["W1"], params["b1"], params["W2"], params["b2"], quantise,
+                        params.get("mid") or ()))
     if crop is None:
         assert len(outs) == 1
         return outs[0]
@@ -258,4 +266,5 @@ def params_f64(w: dict) -> dict:
         out[key] = None if w.get(key) is None else np.asarray(w[key], np.float64)
     for key in ("newline", "sep"):
         out[key] = None if w.get(key) is None else bf16_bits_to_f64(w[key])
+    out["mid"] = [(bf16_bits_to_f64(Wm), np.asarray(bm, np.float64)) for Wm, bm in (w.get("mid") or ())]
     return out

@@ -51,10 +51,11 @@ class Case:
 
 
 def make_case(wl: W.Workload, hw: Optional[np.ndarray] = None, seed: int = 0, gvp: str = "head",
-              k_order: int = vp.ORDER_CHANNEL_OUTER) -> Case:
+              k_order: int = vp.ORDER_CHANNEL_OUTER, depth: int = 2) -> Case:
     hw = W.grid_hw(wl, seed) if hw is None else np.asarray(hw, np.int32)
     crop = W.spatial_crop(wl)
     w = W.weights(wl, seed)
+    w["mid"] = W.mid_weights(wl, depth, seed)
     feats = W.features(wl, hw, seed)
     rows = O.image_rows(hw, wl.k, crop)
     ids = W.input_ids(wl, rows, seed)
@@ -75,12 +76,15 @@ def w1_for_gpu(case: Case) -> np.ndarray:
 def make_projector(case: Case) -> vp.Projector:
     wl = case.wl
     w = case.w
+    mids = w.get("mid") or []
+    case._mid_dev = [(dev_bf16(Wm), dev_f32(bm)) for Wm, bm in mids]      # keep alive until create copied them
     return vp.Projector(
         wl.k, wl.C, wl.N1, wl.N2, dev_bf16(w1_for_gpu(case)), dev_bf16(w["W2"]), dev_f32(w["b1"]), dev_f32(w["b2"]),
         has_ln=wl.has_ln, ln_gamma=dev_f32(w["gamma"]), ln_beta=dev_f32(w["beta"]), ln_eps=wl.ln_eps,
         feat_dtype=vp.FEAT_F32 if wl.feat_fp32 else vp.FEAT_BF16,
         tile_tag=vp.TILE_2D if wl.tiled else vp.TILE_NONE,
-        global_view_pos=vp.GLOBAL_TAIL if case.gvp == "tail" else vp.GLOBAL_HEAD, k_order=case.k_order)
+        global_view_pos=vp.GLOBAL_TAIL if case.gvp == "tail" else vp.GLOBAL_HEAD, k_order=case.k_order,
+        depth=2 + len(mids), W_mid=[a for a, _ in case._mid_dev] or None, b_mid=[b for _, b in case._mid_dev] or None)
 
 
 class DeviceInputs:

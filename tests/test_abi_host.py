@@ -96,7 +96,8 @@ def test_image_rows_rejects_bad_shapes():
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(depth=3), vp.ERR_UNSUPPORTED),
+    (dict(depth=1), vp.ERR_UNSUPPORTED),
+    (dict(depth=9), vp.ERR_UNSUPPORTED),
     (dict(tile_tag=vp.TILE_1D), vp.ERR_UNSUPPORTED),
     (dict(token_pooling=1), vp.ERR_UNSUPPORTED),
     (dict(k=4), vp.ERR_UNSUPPORTED),
@@ -113,3 +114,9 @@ def test_create_rejects_before_device_work(kw, code):
     h = ctypes.c_void_p()
     assert vp._lib.vlproj_create(ctypes.byref(cfg), ctypes.byref(h)) == code
     assert not h.value
+
+
+def test_create_rejects_deeper_mlp_without_middle_weights():
+    cfg = vp.make_config(2, 64, 64, 32, depth=3, W1=16, W2=16)     # non-null stand-ins, never dereferenced
+    h = ctypes.c_void_p()
+    assert vp._lib.vlproj_create(ctypes.byref(cfg), ctypes.byref(h)) == vp.ERR_INVALID_ARG

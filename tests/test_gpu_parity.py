@@ -187,3 +187,18 @@ def test_merged_layernorm_path_agrees_bit_for_bit():
     out_b = run(case, proj, dev)
     assert proj.status() == vp.OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+
+
+
+@pytest.mark.parametrize("pairs", [True, False], ids=["pairs", "single"])
+@pytest.mark.parametrize("depth", [3, 4])
+def test_deeper_mlp_all_rows(depth, pairs):
+    """depth > 2: middle GELU + Linear(N1 -> N1) layers chained on the device."""
+    wl = custom(f"depth{depth}", 150 + depth, 2, 128, 256, 256, 3, 3, 300, has_ln=(depth == 3))
+    case = make_case(wl, np.array([[20, 14], [13, 13], [8, 30]], np.int32), depth=depth)
+    proj = make_projector(case)
+    proj.set_tile_pairs(pairs)
+    dev = DeviceInputs(case)
+    out = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    check(case, out, dev)

@@ -301,7 +301,7 @@ def test_pins_catch_a_missing_local_transpose(monkeypatch):
 
 def test_pins_catch_a_dropped_bias(brute, monkeypatch):
     real = O.mlp
-    monkeypatch.setattr(O, "mlp", lambda a, W1, b1, W2, b2, q=True: real(a, W1, 0 * b1, W2, b2, q))
+    monkeypatch.setattr(O, "mlp", lambda a, W1, b1, W2, b2, q=True, mids=(): real(a, W1, 0 * b1, W2, b2, q, mids))
     with pytest.raises(AssertionError):
         test_mlp_matches_c_brute_force(brute, 4, 4, 3, 2, True, True)
 
@@ -377,3 +377,38 @@ def test_generator_places_runs_in_order(name):
         assert m.sum() == sum(rows[b * per_seq:(b + 1) * per_seq])
     if wl.fixed_hw is None:
         assert (hw % 2 == 0).all() and hw.min() >= 16 and hw.max() <= 96
+
+
+
+@pytest.mark.parametrize("depth", [3, 4])
+def test_deeper_mlp_matches_c_brute_force(brute, depth):
+    """depth > 2: extra GELU + Linear(N1 -> N1) pairs in the middle ("port DeepSeek-VL2",
+    Projector step 3), every hidden activation rounded to bf16; checked layer by layer
+    against the scalar C dense layer."""
+    h, w, C, k, N1, N2 = 4, 6, 3, 2, 7, 5
+    feat, p = _tiny_case(h, w, C, k, N1, N2, True, seed=20 + depth)
+    rng = np.random.default_rng(depth)
+    p["mid"] = [(O.round_bf16(0.3 * rng.standard_normal((N1, N1))), 0.1 * rng.standard_normal(N1))
+                for _ in range(depth - 2)]
+    got = O.project_image([feat], [(h, w)], k, p, None, 1e-5, True)
+    fe = np.ascontiguousarray(feat)
+    a = np.zeros(k * k * C)
+    for i in range(O.merged_side(h, k)):
+        for j in range(O.merged_side(w, k)):
+            brute.brute_token_a(_ptr(fe), h, w, C, k, i, j, 1, _ptr(p["gamma"]), _ptr(p["beta"]), 1e-5, 1, _ptr(a))
+            x = np.zeros(N1)
+            brute.brute_dense(_ptr(a), k * k * C, _ptr(np.ascontiguousarray(p["W1"])), _ptr(p["b1"]), N1, 1, 1,
+                              _ptr(x))
+            for Wm, bm in p["mid"]:
+                y = np.zeros(N1)
+                brute.brute_dense(_ptr(x), N1, _ptr(np.ascontiguousarray(Wm)), _ptr(bm), N1, 1, 1, _ptr(y))
+                x = y
+            out = np.zeros(N2)
+            brute.brute_dense(_ptr(x), N1, _ptr(np.ascontiguousarray(p["W2"])), _ptr(p["b2"]), N2, 0, 0, _ptr(out))
+            np.testing.assert_allclose(got[i * O.merged_side(w, k) + j], out, rtol=1e-12, atol=1e-12)
+
+
+def test_param_count_with_depth():
+    g = _golden("params.json")
+    assert O.projector_params(g["C"], g["k"], g["N1"], g["N2"], g["has_ln"], depth=2) == g["params"]
+    assert O.projector_params(64, 2, 128, 32, False, depth=4) == (256 * 128 + 128) + 2 * (128 * 128 + 128) + (128 * 32 + 32)

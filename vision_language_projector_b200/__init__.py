@@ -60,6 +60,7 @@ class Config(ctypes.Structure):
         ("global_view_pos", ctypes.c_int32), ("token_pooling", ctypes.c_int32),
         ("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
         ("ln_gamma", ctypes.c_void_p), ("ln_beta", ctypes.c_void_p),
+        ("W_mid", ctypes.c_void_p), ("b_mid", ctypes.c_void_p),
     ]
 
 
@@ -135,9 +136,17 @@ def _host_i32(a) -> Optional[np.ndarray]:
 def make_config(k: int, C: int, N1: int, N2: int, *, has_ln: bool = False, ln_eps: float = 1e-5,
                 feat_dtype: int = FEAT_BF16, tile_tag: int = TILE_NONE, global_view_pos: int = GLOBAL_HEAD,
                 k_order: int = ORDER_CHANNEL_OUTER, depth: int = 2, token_pooling: int = 0,
-                W1=None, b1=None, W2=None, b2=None, ln_gamma=None, ln_beta=None) -> Config:
-    return Config(k, C, N1, N2, depth, int(has_ln), ln_eps, feat_dtype, k_order, tile_tag, global_view_pos,
-                  token_pooling, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(ln_gamma), _ptr(ln_beta))
+                W1=None, b1=None, W2=None, b2=None, ln_gamma=None, ln_beta=None, W_mid=None, b_mid=None) -> Config:
+    cfg = Config(k, C, N1, N2, depth, int(has_ln), ln_eps, feat_dtype, k_order, tile_tag, global_view_pos,
+                 token_pooling, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(ln_gamma), _ptr(ln_beta), None, None)
+    # host arrays of device pointers for the middle layers; kept alive on the Config
+    if W_mid is not None:
+        cfg._w_mid = (ctypes.c_void_p * len(W_mid))(*[_ptr(t) for t in W_mid])
+        cfg.W_mid = ctypes.cast(cfg._w_mid, ctypes.c_void_p)
+    if b_mid is not None:
+        cfg._b_mid = (ctypes.c_void_p * len(b_mid))(*[_ptr(t) for t in b_mid])
+        cfg.b_mid = ctypes.cast(cfg._b_mid, ctypes.c_void_p)
+    return cfg
 
 
 def image_rows(cfg: Config, grid_hw, spatial_crop=None, n_images: Optional[int] = None) -> np.ndarray:
@@ -192,11 +201,11 @@ class Projector:
     def __init__(self, k: int, C: int, N1: int, N2: int, W1, W2, b1=None, b2=None, *, has_ln: bool = False,
                  ln_gamma=None, ln_beta=None, ln_eps: float = 1e-5, feat_dtype: int = FEAT_BF16,
                  tile_tag: int = TILE_NONE, global_view_pos: int = GLOBAL_HEAD, k_order: int = ORDER_CHANNEL_OUTER,
-                 depth: int = 2, token_pooling: int = 0):
+                 depth: int = 2, token_pooling: int = 0, W_mid=None, b_mid=None):
         self.cfg = make_config(k, C, N1, N2, has_ln=has_ln, ln_eps=ln_eps, feat_dtype=feat_dtype,
                                tile_tag=tile_tag, global_view_pos=global_view_pos, k_order=k_order, depth=depth,
                                token_pooling=token_pooling, W1=W1, b1=b1, W2=W2, b2=b2, ln_gamma=ln_gamma,
-                               ln_beta=ln_beta)
+                               ln_beta=ln_beta, W_mid=W_mid, b_mid=b_mid)
         h = ctypes.c_void_p()
         rc = _lib.vlproj_create(ctypes.byref(self.cfg), ctypes.byref(h))
         if rc != OK:

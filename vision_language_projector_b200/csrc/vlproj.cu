@@ -209,7 +209,8 @@ struct Plan {
 
 int validate_config(const vlproj_config* c) {
     if (!c) return VLPROJ_ERR_INVALID_ARG;
-    if (c->depth != 2 || c->tile_tag == VLPROJ_TILE_1D || c->token_pooling != 0) return VLPROJ_ERR_UNSUPPORTED;
+    if (c->depth < 2 || c->depth > 8 || c->tile_tag == VLPROJ_TILE_1D || c->token_pooling != 0)
+        return VLPROJ_ERR_UNSUPPORTED;
     if (c->k < 1 || c->k > 3) return VLPROJ_ERR_UNSUPPORTED;
     if (c->tile_tag != VLPROJ_TILE_NONE && c->tile_tag != VLPROJ_TILE_2D) return VLPROJ_ERR_UNSUPPORTED;
     if (c->global_view_pos != VLPROJ_GLOBAL_HEAD && c->global_view_pos != VLPROJ_GLOBAL_TAIL)
@@ -396,7 +397,11 @@ struct vlproj_handle {
     CUtensorMap tmW1h{}, tmW2h{};        // B boxes of 128 rows (each CTA of a pair loads half)
     bool pairs = true;                   // run 256 x 256 tiles on CTA pairs where possible
     // scratch, grown on demand
-    DevBuf<__nv_bfloat16> H, Xn, A;
+    DevBuf<__nv_bfloat16> H, H2, Xn, A;       // H2: second hidden buffer (depth > 2)
+    // middle layers (depth > 2): weights, biases, tensor maps (BN-row and 128-row boxes)
+    std::vector<__nv_bfloat16*> Wm;
+    std::vector<float*> bm;
+    std::vector<CUtensorMap> tmWm, tmWmh;
     DevBuf<int32_t> pos, rowdest, counts;
     DevBuf<int2> gmeta;
     DevBuf<int4> chunks;
@@ -673,6 +678,11 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
     int rc = validate_config(cfg);
     if (rc) return rc;
     if (!cfg->W1 || !cfg->W2 || (cfg->has_ln && (!cfg->ln_gamma || !cfg->ln_beta))) return VLPROJ_ERR_INVALID_ARG;
+    if (cfg->depth > 2) {
+        if (!cfg->W_mid) return VLPROJ_ERR_INVALID_ARG;
+        for (int i = 0; i < cfg->depth - 2; ++i)
+            if (!cfg->W_mid[i]) return VLPROJ_ERR_INVALID_ARG;
+    }
     if (!driver().tiled || !driver().im2col) return VLPROJ_ERR_CUDA;
 
     vlproj_handle* h = new vlproj_handle();
@@ -713,6 +723,28 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
     }
     if (cudaMemset(h->status, 0, 2 * sizeof(int))) return fail(VLPROJ_ERR_CUDA);
     if (cudaDeviceSynchronize()) return fail(VLPROJ_ERR_CUDA);
+    for (int i = 0; i < cfg->depth - 2; ++i) {
+        __nv_bfloat16* w = nullptr;
+        float* b = nullptr;
+        if (cudaMalloc(&w, n1 * n1 * 2) || cudaMalloc(&b, n1 * 4)) {
+            if (w) cudaFree(w);
+            return fail(VLPROJ_ERR_CUDA);
+        }
+        h->Wm.push_back(w);
+        h->bm.push_back(b);
+        const float* bsrc = cfg->b_mid ? cfg->b_mid[i] : nullptr;
+        if (cudaMemcpy(w, cfg->W_mid[i], n1 * n1 * 2, cudaMemcpyDeviceToDevice) ||
+            (bsrc ? cudaMemcpy(b, bsrc, n1 * 4, cudaMemcpyDeviceToDevice) : cudaMemset(b, 0, n1 * 4)))
+            return fail(VLPROJ_ERR_CUDA);
+        CUtensorMap full{}, half{};
+        if (encode_bf16_2d(&full, w, n1, n1, pick_bn(cfg->N1)) || encode_bf16_2d(&half, w, n1, n1, 128))
+            return fail(VLPROJ_ERR_CUDA);
+        h->tmWm.push_back(full);
+        h->tmWmh.push_back(half);
+    }
+    if (cudaDeviceSynchronize()) return fail(VLPROJ_ERR_CUDA);
+    h->cfg.W_mid = nullptr;       // the caller's arrays are not kept
+    h->cfg.b_mid = nullptr;
     if (encode_bf16_2d(&h->tmW1, h->W1p, n1, h->K1, pick_bn(cfg->N1)) ||
         encode_bf16_2d(&h->tmW2, h->W2, n2, n1, pick_bn(cfg->N2)) ||
         encode_bf16_2d(&h->tmW1h, h->W1p, n1, h->K1, 128) || encode_bf16_2d(&h->tmW2h, h->W2, n2, n1, 128))
@@ -735,6 +767,9 @@ void vlproj_destroy(vlproj_handle* h) {
     cudaFree(h->beta);
     cudaFree(h->status);
     h->H.release();
+    h->H2.release();
+    for (auto* w : h->Wm) cudaFree(w);
+    for (auto* b : h->bm) cudaFree(b);
     h->Xn.release();
     h->A.release();
     h->pos.release();
@@ -862,6 +897,7 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
         return VLPROJ_ERR_CUDA;
     if (pl.M > 0 && h->rowdest.ensure(pl.M)) return VLPROJ_ERR_CUDA;
     if (pl.M > 0 && h->H.ensure(static_cast<size_t>(pl.M) * c.N1)) return VLPROJ_ERR_CUDA;
+    if (pl.M > 0 && c.depth > 2 && h->H2.ensure(static_cast<size_t>(pl.M) * c.N1)) return VLPROJ_ERR_CUDA;
     rc = upload_plan(h, pl, s);
     if (rc) return rc;
     h->profiled_valid = false;
@@ -909,12 +945,37 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
     // 1-3. geometry, LayerNorm, GEMM1 -> H
     rc = run_merge_gemm1(h, pl, features, nullptr, vlp::DEST_NONE, h->H.ptr, pl.M, s);
     if (rc) return rc;
+    // middle layers (depth > 2): H <- bf16(GELU(H Wm^T + bm)), ping-pong between H and H2
+    bool last_in_h2 = false;
+    for (int layer = 0; layer + 2 < c.depth; ++layer) {
+        DevBuf<__nv_bfloat16>& src = last_in_h2 ? h->H2 : h->H;
+        DevBuf<__nv_bfloat16>& dst = last_in_h2 ? h->H : h->H2;
+        CUtensorMap tin{};
+        if (encode_bf16_2d(&tin, src.ptr, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
+        GemmParams q{};
+        q.M = static_cast<int>(pl.M);
+        q.N = c.N1;
+        q.K = c.N1;
+        q.bias = h->bm[layer];
+        q.C = c.C;
+        q.k = c.k;
+        q.out = dst.ptr;
+        q.out_rows = pl.M;
+        q.err = h->status;
+        q.wait_ns = h->wait_ns;
+        ++h->launches;
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tin, h->tmWm[layer],
+                                                        h->tmWmh[layer], q, h->num_sms, s);
+        if (rc) return rc;
+        last_in_h2 = !last_in_h2;
+    }
     VLP_CUDA(cudaStreamWaitEvent(s, h->join, 0));
 
-    // 4. GEMM2 + scatter
-    if (h->tmH_ptr != h->H.ptr || h->tmH_rows != pl.M) {
-        if (encode_bf16_2d(&h->tmH, h->H.ptr, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
-        h->tmH_ptr = h->H.ptr;
+    // 4. GEMM2 + scatter (from the last hidden activation)
+    const __nv_bfloat16* hlast = last_in_h2 ? h->H2.ptr : h->H.ptr;
+    if (h->tmH_ptr != hlast || h->tmH_rows != pl.M) {
+        if (encode_bf16_2d(&h->tmH, hlast, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
+        h->tmH_ptr = hlast;
         h->tmH_rows = pl.M;
     }
     GemmParams p{};

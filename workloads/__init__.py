@@ -196,6 +196,19 @@ def weights(wl: Workload, seed: int = 0) -> dict:
     return d
 
 
+_T_MID = 13
+
+
+def mid_weights(wl: Workload, depth: int, seed: int = 0) -> list:
+    """(depth - 2) middle layers (W bf16 bits (N1, N1) ~N(0, 0.02), b fp32 ~N(0, 0.02))."""
+    out = []
+    for i in range(depth - 2):
+        r = _rng(wl, _T_MID, i, seed)
+        out.append((_normal_bits(r, (wl.N1, wl.N1), 0.02),
+                    r.standard_normal(wl.N1, dtype=np.float32) * np.float32(0.02)))
+    return out
+
+
 def input_ids(wl: Workload, rows_per_image: Sequence[int], seed: int = 0,
               image_token_id: int = IMAGE_TOKEN_ID) -> np.ndarray:
     """Flattened (B*S,) int64 ids: each sequence holds n_images/B images as placeholder runs.
