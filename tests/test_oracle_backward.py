@@ -1,0 +1,215 @@
+"""Pins of the fp64 backward oracle (oracle/backward.py).
+
+The gradients are checked against central finite differences of the (separately
+pinned) forward oracle: the loss is <d_out, forward(theta)>, so its derivative in
+any parameter entry is the entry of the returned gradient. Finite differences
+share no step with the chain rule written out in the backward, so a dropped term,
+a wrong sign, a transposed operand or a misplaced row fails them.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import backward as B
+from oracle import projector as O
+
+IMG = 7
+
+
+def _case(seed, grid_hw, crop, k, C, N1, N2, has_ln, n_text=9):
+    rng = np.random.default_rng(seed)
+    grid_hw = np.asarray(grid_hw, np.int32)
+    P = int((grid_hw[:, 0] * grid_hw[:, 1]).sum())
+    feats = rng.normal(0.0, 1.0, (P, C)) * rng.uniform(0.5, 2.0, (P, 1)) + rng.normal(0.0, 0.5, (P, 1))
+    K1 = k * k * C
+    params = {
+        "W1": rng.normal(0.0, 0.3, (N1, K1)), "b1": rng.normal(0.0, 0.3, N1),
+        "W2": rng.normal(0.0, 0.3, (N2, N1)), "b2": rng.normal(0.0, 0.3, N2),
+        "gamma": rng.uniform(0.5, 1.5, C) if has_ln else None,
+        "beta": rng.normal(0.0, 0.2, C) if has_ln else None,
+        "newline": rng.normal(0.0, 1.0, N2) if crop is not None else None,
+        "sep": rng.normal(0.0, 1.0, N2) if crop is not None else None,
+        "mid": [],
+    }
+    rows = sum(O.image_rows(grid_hw, k, crop))
+    ids = rng.integers(IMG + 1, IMG + 50, rows + n_text)      # text ids never equal the placeholder
+    slots = np.sort(rng.choice(rows + n_text, rows, replace=False))
+    ids[slots] = IMG
+    d_out = rng.normal(0.0, 1.0, (len(ids), N2))
+    embeds = rng.normal(0.0, 1.0, (len(ids), N2))
+    return dict(features=feats, grid_hw=grid_hw, spatial_crop=crop, k=k, params=params, ids=ids,
+                d_out=d_out, embeds=embeds)
+
+
+CASES = {
+    "untiled_ln_ragged": dict(seed=1, grid_hw=[[3, 5], [4, 4]], crop=None, k=2, C=4, N1=6, N2=5, has_ln=True),
+    "untiled_k3_ln": dict(seed=2, grid_hw=[[4, 5]], crop=None, k=3, C=3, N1=5, N2=4, has_ln=True),
+    "untiled_no_ln": dict(seed=3, grid_hw=[[2, 3], [1, 1]], crop=None, k=2, C=3, N1=4, N2=3, has_ln=False),
+    "tiled_2x1": dict(seed=4, grid_hw=[[3, 3]] * 3, crop=np.array([[2, 1]]), k=2, C=3, N1=4, N2=3, has_ln=True),
+    "tiled_two_images": dict(seed=5, grid_hw=[[2, 2]] * 3 + [[3, 2]] * 3, crop=np.array([[1, 2], [2, 1]]),
+                             k=2, C=2, N1=3, N2=4, has_ln=False),
+}
+
+
+def _loss(c, params=None, features=None, quantise=False, gvp="head"):
+    out = O.forward(c["features"] if features is None else features, c["grid_hw"], c["spatial_crop"], c["k"],
+                    c["params"] if params is None else params, c["ids"], IMG, c["embeds"], 1e-5,
+                    feat_is_bf16_bits=False, quantise=quantise, global_view_pos=gvp)
+    return float((out * c["d_out"]).sum())
+
+
+def _grads(c, quantise=False, gvp="head"):
+    return B.backward(c["features"], c["grid_hw"], c["spatial_crop"], c["k"], c["params"], c["ids"], IMG,
+                      c["d_out"], 1e-5, feat_is_bf16_bits=False, quantise=quantise, gvp=gvp)
+
+
+def _fd(c, name, eps=1e-6, quantise=False, gvp="head"):
+    """Central finite difference of the loss in every entry of parameter `name`."""
+    if name == "features":
+        base = c["features"]
+    else:
+        base = c["params"][name]
+    g = np.zeros_like(base)
+    for idx in np.ndindex(base.shape):
+        vals = []
+        for s in (+1.0, -1.0):
+            t = base.copy()
+            t[idx] += s * eps
+            if name == "features":
+                vals.append(_loss(c, features=t, quantise=quantise, gvp=gvp))
+            else:
+                p = dict(c["params"])
+                p[name] = t
+                vals.append(_loss(c, params=p, quantise=quantise, gvp=gvp))
+        g[idx] = (vals[0] - vals[1]) / (2 * eps)
+    return g
+
+
+def _names(c):
+    names = ["W1", "b1", "W2", "b2", "features"]
+    if c["params"]["gamma"] is not None:
+        names += ["gamma", "beta"]
+    if c["spatial_crop"] is not None:
+        names += ["newline", "sep"]
+    return names
+
+
+def test_gelu_grad_matches_finite_difference():
+    x = np.linspace(-6.0, 6.0, 241)
+    h = 1e-6
+    fd = (O.gelu(x + h) - O.gelu(x - h)) / (2 * h)
+    np.testing.assert_allclose(B.gelu_grad(x), fd, rtol=0, atol=1e-9)
+    # closed forms: GELU'(0) = 1/2, GELU' -> 0 and 1 in the tails
+    assert B.gelu_grad(np.array([0.0]))[0] == 0.5
+    assert abs(B.gelu_grad(np.array([-12.0]))[0]) < 1e-20
+    assert abs(B.gelu_grad(np.array([12.0]))[0] - 1.0) < 1e-20
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_matches_finite_differences(name):
+    spec = CASES[name]
+    c = _case(**spec)
+    g = _grads(c)
+    for key in _names(c):
+        fd = _fd(c, key)
+        scale = max(1.0, float(np.abs(fd).max()))
+        np.testing.assert_allclose(g[key], fd, rtol=0, atol=2e-6 * scale, err_msg=f"{name}: d{key}")
+
+
+def test_backward_tail_global_view_matches_finite_differences():
+    c = _case(**CASES["tiled_2x1"])
+    g = _grads(c, gvp="tail")
+    for key in ("W2", "newline", "sep", "features"):
+        fd = _fd(c, key, gvp="tail")
+        np.testing.assert_allclose(g[key], fd, rtol=0, atol=2e-6 * max(1.0, float(np.abs(fd).max())))
+
+
+def test_quantised_backward_exact_in_the_affine_parameters():
+    """With the bf16 rounding points on, the rows are still affine in W2, b2 and the
+    newline / separator rows (the rounded hidden state does not depend on them), so a
+    finite difference of any step is their exact gradient."""
+    c = _case(**CASES["tiled_two_images"])
+    g = _grads(c, quantise=True)
+    for key in ("W2", "b2", "newline", "sep"):
+        fd = _fd(c, key, eps=0.25, quantise=True)
+        np.testing.assert_allclose(g[key], fd, rtol=0, atol=1e-9 * max(1.0, float(np.abs(fd).max())))
+
+
+def test_quantised_backward_is_close_to_the_exact_one():
+    """Straight-through rounding changes the gradients only by the bf16 rounding of the
+    saved activations (relative 2^-8 per value)."""
+    c = _case(**CASES["untiled_ln_ragged"])
+    gq = _grads(c, quantise=True)
+    g = _grads(c, quantise=False)
+    for key in _names(c):
+        scale = float(np.abs(g[key]).max())
+        assert float(np.abs(gq[key] - g[key]).max()) <= 3e-2 * scale, key
+
+
+def test_text_rows_carry_no_gradient():
+    c = _case(**CASES["untiled_ln_ragged"])
+    g0 = _grads(c)
+    mask = c["ids"] != IMG
+    c["d_out"][mask] += 100.0
+    g1 = _grads(c)
+    for key in _names(c):
+        np.testing.assert_array_equal(g0[key], g1[key])
+
+
+def test_backward_rejects_count_mismatch():
+    c = _case(**CASES["untiled_no_ln"])
+    ids = c["ids"].copy()
+    ids[np.flatnonzero(ids == IMG)[0]] = 1
+    with pytest.raises(ValueError):
+        B.backward(c["features"], c["grid_hw"], None, 2, c["params"], ids, IMG, c["d_out"], feat_is_bf16_bits=False)
+
+
+# ------------------------------------------------------------------ planted mistakes
+def test_pins_catch_a_wrong_gelu_derivative(monkeypatch):
+    c = _case(**CASES["untiled_no_ln"])
+    monkeypatch.setattr(B, "gelu_grad", lambda p: 0.5 * (1.0 + np.vectorize(math.erf)(p / math.sqrt(2.0))))
+    g = _grads(c)
+    fd = _fd(c, "W1")
+    assert not np.allclose(g["W1"], fd, rtol=0, atol=2e-6 * max(1.0, float(np.abs(fd).max())))
+
+
+def test_pins_catch_a_dropped_layernorm_term(monkeypatch):
+    """LayerNorm's input gradient without the xhat * mean(g * xhat) projection term."""
+    c = _case(**CASES["untiled_k3_ln"])
+    monkeypatch.setattr(B, "layernorm_backward",
+                        lambda d, xh, r, gm: r * (d * gm - (d * gm).mean(axis=1, keepdims=True)))
+    g = _grads(c)
+    fd = _fd(c, "features")
+    assert not np.allclose(g["features"], fd, rtol=0, atol=2e-6 * max(1.0, float(np.abs(fd).max())))
+
+
+def test_pins_catch_an_unflipped_fold(monkeypatch):
+    """The input gradient folded back with the channels of each patch reversed."""
+    c = _case(**CASES["untiled_ln_ragged"])
+    real = O.fold
+    monkeypatch.setattr(O, "fold", lambda a, hp, wp, k, C: real(a[:, ::-1].copy(), hp, wp, k, C))
+    g = _grads(c)
+    fd = _fd(c, "features")
+    assert not np.allclose(g["features"], fd, rtol=0, atol=2e-6 * max(1.0, float(np.abs(fd).max())))
+
+
+def test_pins_catch_a_swapped_view_order(monkeypatch):
+    """Gradient rows read from the wrong view of a tiled image (global and first local
+    swapped) fail the finite differences of W2."""
+    c = _case(**CASES["tiled_2x1"])
+    real = B._image_row_map
+
+    def wrong(hp, wp, crop, n_views, gvp):
+        m = real(hp, wp, crop, n_views, gvp).copy()
+        n = hp * wp
+        tok = m >= 0
+        v = np.where(tok, m // n, -1)
+        swap = np.where(v == 0, 1, np.where(v == 1, 0, v))
+        m[tok] = swap[tok] * n + m[tok] % n
+        return m
+
+    monkeypatch.setattr(B, "_image_row_map", wrong)
+    g = _grads(c)
+    fd = _fd(c, "W2")
+    assert not np.allclose(g["W2"], fd, rtol=0, atol=2e-6 * max(1.0, float(np.abs(fd).max())))
