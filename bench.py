@@ -294,7 +294,8 @@ def main():
         e1.synchronize()
         step_ms.append(e0.elapsed_time(e1))
         for k_, v in proj.stage_ms().items():
-            stage_acc.setdefault(k_, []).append(v)
+            if v > 0.0:                    # stages that ran in this step
+                stage_acc.setdefault(k_, []).append(v)
     launches = proj.launch_count() - launches0
     torch.cuda.synchronize()
     if world > 1:

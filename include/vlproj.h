@@ -164,6 +164,61 @@ typedef struct vlproj_forward_args {
 } vlproj_forward_args;
 int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* stream);
 
+/* ---- backward -----------------------------------------------------------
+ * Gradients of the projector for one batch. The bridge is trained with the vision
+ * tower and the language model frozen, so the projector's parameters are the only
+ * trained ones ("DeepSeek-V4-Flash-Vision-BF16", opening section: a 40,119,040-
+ * parameter projector trained between the frozen tower and backbone, with forward /
+ * backward gates passed in BF16). Given d_out, the gradient of the loss with respect
+ * to the combined embedding buffer that vlproj_forward writes, this returns the
+ * gradients of W1, b1, W2, b2, the LayerNorm gamma / beta, the newline and separator
+ * rows, and of the features, by the chain rule through the forward steps:
+ *   dY[m]  = d_out[placeholder row of merged token m]
+ *   dW2    = dY^T H,  db2 = sum_m dY[m]
+ *   dP     = (dY W2) * GELU'(P),  P = A W1^T + b1 (recomputed from the features)
+ *   dW1    = dP^T A,  db1 = sum_m dP[m]
+ *   dA     = dP W1, folded back through the space-to-depth onto the patches, then
+ *            through the LayerNorm: dgamma, dbeta and d_features
+ *   dnewline / dsep = sums of d_out over the newline / separator rows.
+ * The bf16 rounding points of the forward (A and H) pass gradients unchanged; H and A
+ * are the forward's bf16 values, dP is rounded to bf16 once (fp32 accumulation
+ * throughout). Only depth-2 MLPs (VLPROJ_ERR_UNSUPPORTED otherwise).
+ *
+ *   features, grid_hw, spatial_crop, n_images, input_ids, n_ids, image_token_id:
+ *                 as for vlproj_forward (the same batch the loss was computed on).
+ *   d_out         DEVICE bf16 [n_ids][N2], 16-byte aligned. Rows of text tokens are
+ *                 ignored.
+ *   d_W1 .. d_features  DEVICE fp32 outputs, overwritten (not accumulated), each
+ *                 16-byte aligned, or NULL when not wanted (work that only feeds
+ *                 unwanted outputs is skipped):
+ *                   d_W1 [N1][k*k*C] (columns in the config's k_order), d_b1 [N1],
+ *                   d_W2 [N2][N1], d_b2 [N2], d_gamma [C], d_beta [C] (LayerNorm only),
+ *                   d_newline [N2], d_sep [N2] (2D tiling only), d_features [P][C].
+ * Scratch: about 2 * M * (2*N1 + N2 + k*k*C) bf16 plus M*k*k*C fp32 bytes (M merged
+ * tokens), kept in the handle between calls. Errors as for vlproj_forward; when the
+ * placeholder count check fails every gradient is written as zero and
+ * VLPROJ_ERR_TOKEN_COUNT is latched. */
+typedef struct vlproj_backward_args {
+    const void*    features;
+    const int32_t* grid_hw;
+    const int32_t* spatial_crop;
+    int32_t        n_images;
+    const int64_t* input_ids;
+    int64_t        n_ids;
+    int64_t        image_token_id;
+    const void*    d_out;
+    float*         d_W1;
+    float*         d_b1;
+    float*         d_W2;
+    float*         d_b2;
+    float*         d_gamma;
+    float*         d_beta;
+    float*         d_newline;
+    float*         d_sep;
+    float*         d_features;
+} vlproj_backward_args;
+int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* args, void* stream);
+
 /* Stage output for inspection: the bf16 hidden activation H = GELU(A W1^T + b1)
  * of every merged token, views in order, tokens row-major inside a view.
  * hidden is DEVICE bf16 [M][N1], M = sum over views of ceil(h/k)*ceil(w/k). */
@@ -235,14 +290,19 @@ int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns);
 
 /* ---- tracing ------------------------------------------------------------
  * Stage timing with CUDA events recorded on the launching stream around each
- * kernel of vlproj_forward. Stages, in order:
- *   0 placeholder index, 1 geometry, 2 LayerNorm/convert, 3 GEMM1 (merge + MLP
- *   first layer + GELU), 4 GEMM2 (second layer + scatter), 5 newline/separator rows.
- * Off by default; enabling adds seven event records per forward. */
-#define VLPROJ_NUM_STAGES 6
+ * kernel of vlproj_forward / vlproj_backward. Stages, in order:
+ *   forward   0 placeholder index, 1 geometry, 2 LayerNorm/convert, 3 GEMM1 (merge +
+ *             MLP first layer + GELU), 4 GEMM2 (second layer + scatter),
+ *             5 newline/separator rows;
+ *   backward  6 placeholder index + geometry, 7 LayerNorm-merge (A), 8 GEMM1
+ *             recompute (GELU' and H^T), 9 dY gather, 10 dH GEMM (dP), 11 dW2 GEMM,
+ *             12 A^T + dW1 GEMM, 13 dA GEMM, 14 bias sums + LayerNorm backward +
+ *             newline/separator gradients.
+ * Off by default; enabling adds two event records per stage that runs. */
+#define VLPROJ_NUM_STAGES 15
 int vlproj_profile_enable(vlproj_handle* h, int enable);
 
-/* Synchronise the stream of the most recent profiled forward and write the elapsed
+/* Synchronise the stream of the most recent profiled call and write the elapsed
  * milliseconds of each stage into ms[0 .. min(n, VLPROJ_NUM_STAGES)); a stage that did
  * not run reads 0. Returns the number of values written, or an error code. */
 int vlproj_profile_read(vlproj_handle* h, float* ms, int n);

@@ -51,7 +51,20 @@ def _image_row_map(hp: int, wp: int, crop: Optional[tuple], n_views: int, gvp: s
 
 def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[np.ndarray], k: int, params: dict,
              ids: np.ndarray, image_token_id: int, d_out: np.ndarray, ln_eps: float = 1e-5,
-             feat_is_bf16_bits: bool = True, quantise: bool = True, gvp: str = "head") -> dict:
+             feat_is_bf16_bits: bool = True, quantise: bool = True, gvp: str = "head",
+             skip_zero_rows: bool = False, magnitudes: bool = False) -> dict:
+    """Gradients for the loss <d_out, forward(...)>; ``d_out`` is (n_ids, N2) or anything
+    indexable by an array of row numbers. With ``skip_zero_rows`` the MLP is evaluated
+    only for merged tokens whose output gradient row is nonzero: the others contribute
+    exactly zero to every gradient (dY = 0 gives dP = 0, dA = 0 and a zero LayerNorm
+    input gradient).
+
+    With ``magnitudes`` the result also holds, under "mag", the same chain evaluated on
+    absolute values: for every gradient entry the sum of the absolute values of the
+    terms it is made of (|dY|^T |H| for dW2, |dP|^T |A| for dW1, and so on through the
+    LayerNorm backward). A relative perturbation of at most e in each term moves the
+    entry by at most e times this sum, which is how the GPU parity tests bound the
+    effect of bf16 rounding."""
     grid_hw = np.asarray(grid_hw)
     x_all = O.bf16_bits_to_f64(features) if feat_is_bf16_bits else np.asarray(features, np.float64)
     W1, b1, W2, b2 = params["W1"], params["b1"], params["W2"], params["b2"]
@@ -67,6 +80,7 @@ def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[n
         g["newline"] = np.zeros(W2.shape[0])
         g["sep"] = np.zeros(W2.shape[0])
 
+    mag = {key: np.zeros_like(v) for key, v in g.items()} if magnitudes else None
     pos = O.placeholder_positions(ids, image_token_id)
     offs = np.concatenate([[0], np.cumsum(grid_hw[:, 0].astype(np.int64) * grid_hw[:, 1])])
     if spatial_crop is None:
@@ -90,6 +104,9 @@ def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[n
         if crop is not None:
             g["newline"] += d_rows[row_map == -1].sum(axis=0)
             g["sep"] += d_rows[row_map == -2].sum(axis=0)
+            if magnitudes:
+                mag["newline"] += np.abs(d_rows[row_map == -1]).sum(axis=0)
+                mag["sep"] += np.abs(d_rows[row_map == -2]).sum(axis=0)
         tok_rows = np.full(len(views) * hp * wp, -1, np.int64)
         tok_rows[row_map[row_map >= 0]] = np.flatnonzero(row_map >= 0)
         for vi, v in enumerate(views):
@@ -106,18 +123,21 @@ def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[n
             if quantise:
                 src = O.round_bf16(src)
             a = O.unshuffle(src.reshape(h0, w0, C), k)
+            dy = d_rows[tok_rows[vi * hp * wp:(vi + 1) * hp * wp]]
+            sel = np.flatnonzero(np.any(dy != 0, axis=1)) if skip_zero_rows else np.arange(hp * wp)
+            a, dy = a[sel], dy[sel]
             p = a @ W1.T + b1
             hid = O.gelu(p)
             if quantise:
                 hid = O.round_bf16(hid)
             # gradients
-            dy = d_rows[tok_rows[vi * hp * wp:(vi + 1) * hp * wp]]
             g["b2"] += dy.sum(axis=0)
             g["W2"] += dy.T @ hid
             dp = (dy @ W2) * gelu_grad(p)
             g["b1"] += dp.sum(axis=0)
             g["W1"] += dp.T @ a
-            da = dp @ W1
+            da = np.zeros((hp * wp, W1.shape[1]))
+            da[sel] = dp @ W1
             dsrc = O.fold(da, hp, wp, k, C)[:h0, :w0].reshape(h0 * w0, C)
             if has_ln:
                 g["gamma"] += (dsrc * xhat).sum(axis=0)
@@ -126,4 +146,27 @@ def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[n
             else:
                 dx = dsrc
             g["features"][offs[v]:offs[v + 1]] = dx
+            if magnitudes:
+                # |dP| plus the absolute sum of its dot product, scaled far below bf16
+                # precision: a cancelling dY . W2 still gets the room of its fp32 rounding
+                m_dp = np.abs(dp) + 2.0 ** -16 * (np.abs(dy) @ np.abs(W2)) * np.abs(gelu_grad(p))
+                mag["b2"] += np.abs(dy).sum(axis=0)
+                mag["W2"] += np.abs(dy).T @ np.abs(hid)
+                mag["b1"] += m_dp.sum(axis=0)
+                mag["W1"] += m_dp.T @ np.abs(a)
+                m_da = np.zeros((hp * wp, W1.shape[1]))
+                m_da[sel] = m_dp @ np.abs(W1)
+                m_src = O.fold(m_da, hp, wp, k, C)[:h0, :w0].reshape(h0 * w0, C)
+                if has_ln:
+                    ax = np.abs(xhat)
+                    mag["gamma"] += (m_src * ax).sum(axis=0)
+                    mag["beta"] += m_src.sum(axis=0)
+                    m_g = m_src * np.abs(gamma)
+                    m_dx = rstd * (m_g + m_g.mean(axis=1, keepdims=True)
+                                   + ax * (m_g * ax).mean(axis=1, keepdims=True))
+                else:
+                    m_dx = m_src
+                mag["features"][offs[v]:offs[v + 1]] = m_dx
+    if magnitudes:
+        g["mag"] = mag
     return g

@@ -1,0 +1,238 @@
+"""GPU parity of vlproj_backward with the fp64 backward oracle (oracle/backward.py).
+
+Tolerance, per gradient entry:  |gpu - oracle| <= e * mag,  where mag is the oracle's
+absolute-value chain (for dW1[n, q] the sum over tokens of |dP[m, n]| |A[m, q]|, and
+so on, see oracle/backward.py), so each term of an entry may be off by a relative e:
+  * bf16 keeps 8 significant bits: rounding moves a value by at most 2^-8 of it, and a
+    value that the GPU's fp32 arithmetic puts on the other side of a rounding boundary
+    than the fp64 oracle does lands one ulp away, at most 2^-7 of it;
+  * dW2 terms hold H (one such boundary): e = 2^-7;
+  * dW1 terms hold dP, rounded twice (GELU'(P), then dP: (1 + 2^-8)^2 - 1 < 2^-7 + 2^-15),
+    and A (one boundary, 2^-7): e = 2^-6; db1, dA, the LayerNorm gradients and
+    d_features carry dP's rounding only, and take the same e;
+  * db2 and the newline / separator rows are fp32 sums of exact bf16 values: e = 2^-8.
+An entry whose terms are all zero must come out exactly zero.
+"""
+import numpy as np
+import pytest
+import torch
+
+import vision_language_projector_b200 as vp
+import workloads as W
+from oracle import backward as B
+from oracle import projector as O
+from gpu_harness import DeviceInputs, custom, dev_bf16, make_case, make_projector, w1_for_gpu
+
+pytestmark = pytest.mark.gpu
+
+EPS_DP = 2.0 ** -6
+EPS = {"W2": 2.0 ** -7, "b2": 2.0 ** -8, "newline": 2.0 ** -8, "sep": 2.0 ** -8}
+
+
+def grad_shapes(case):
+    wl = case.wl
+    P = int((case.hw[:, 0].astype(np.int64) * case.hw[:, 1]).sum())
+    shapes = {"W1": (wl.N1, wl.K1), "b1": (wl.N1,), "W2": (wl.N2, wl.N1), "b2": (wl.N2,), "features": (P, wl.C)}
+    if wl.has_ln:
+        shapes.update(gamma=(wl.C,), beta=(wl.C,))
+    if wl.tiled:
+        shapes.update(newline=(wl.N2,), sep=(wl.N2,))
+    return shapes
+
+
+def run_backward(case, proj, dev, d_out, names=None, check=True):
+    """Gradients from the GPU as fp64 numpy arrays; outputs start as NaN so that an
+    element the library fails to write shows up."""
+    shapes = grad_shapes(case)
+    names = list(shapes) if names is None else names
+    grads = {n: torch.full(shapes[n], float("nan"), dtype=torch.float32, device="cuda") for n in names}
+    rc = proj.backward(dev.feats, case.hw, case.crop, dev.ids, W.IMAGE_TOKEN_ID, d_out, grads,
+                       n_images=case.wl.n_images, check=check)
+    torch.cuda.synchronize()
+    return rc, {n: t.double().cpu().numpy() for n, t in grads.items()}
+
+
+def oracle_grads(case, d_out, skip_zero_rows=False):
+    g = B.backward(case.feats, case.hw, case.crop, case.wl.k, O.params_f64(case.w), case.ids, W.IMAGE_TOKEN_ID,
+                   d_out, case.wl.ln_eps, feat_is_bf16_bits=not case.wl.feat_fp32, quantise=True, gvp=case.gvp,
+                   skip_zero_rows=skip_zero_rows, magnitudes=True)
+    if case.k_order == vp.ORDER_POSITION_OUTER:
+        kk, C = case.wl.k * case.wl.k, case.wl.C
+        for d in (g, g["mag"]):
+            d["W1"] = d["W1"].reshape(-1, C, kk).transpose(0, 2, 1).reshape(d["W1"].shape[0], -1)
+    return g
+
+
+def assert_grads_close(got, want, label=""):
+    stats = {}
+    for n, gv in got.items():
+        wv, mag = want[n], want["mag"][n]
+        assert gv.shape == wv.shape, n
+        assert np.isfinite(gv).all(), f"{label} d{n}: unwritten or non-finite elements"
+        err = np.abs(gv - wv)
+        bound = EPS.get(n, EPS_DP) * mag
+        assert np.all(err[mag == 0] == 0), f"{label} d{n}: nonzero where every term is zero"
+        live = mag > 0
+        ratio = float((err[live] / bound[live]).max()) if live.any() else 0.0
+        stats[n] = ratio
+        assert ratio <= 1.0, f"{label} d{n}: max err / bound = {ratio:.3f}"
+    return stats
+
+
+def dev_dout(case, seed=0):
+    bits = W.grad_out(case.wl, len(case.ids), seed)
+    return bits, dev_bf16(bits), O.bf16_bits_to_f64(bits)
+
+
+SMALL = {
+    "tiny": lambda: W.WORKLOADS["tiny"],
+    "ragged_ln_bf16": lambda: custom("ragged_ln_bf16", 40, 2, 128, 256, 160, 3, 1, 900, has_ln=True),
+    "k3_no_ln": lambda: custom("k3_no_ln", 41, 3, 64, 192, 128, 2, 2, 200),
+    "tiled_2x1": lambda: custom("tiled_2x1", 42, 2, 64, 128, 128, 2, 2, 260, tiled=True, tw=2, th=1),
+    "fp32_no_ln": lambda: custom("fp32_no_ln", 43, 2, 64, 128, 96, 2, 1, 300, feat_fp32=True),
+}
+GRIDS = {
+    "ragged_ln_bf16": [[20, 30], [17, 9], [32, 32]],
+    "k3_no_ln": [[10, 11], [7, 3]],
+    "tiled_2x1": [[9, 9]] * 3 + [[7, 5]] * 3,
+    "fp32_no_ln": [[15, 13], [4, 4]],
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_backward_matches_oracle(name):
+    wl = SMALL[name]()
+    case = make_case(wl, GRIDS.get(name))
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    _, d_dev, d_f64 = dev_dout(case)
+    rc, got = run_backward(case, proj, dev, d_dev)
+    assert rc == vp.OK and proj.status() == vp.OK
+    assert_grads_close(got, oracle_grads(case, d_f64), name)
+
+
+@pytest.mark.parametrize("gvp", ["head", "tail"])
+def test_backward_tiled_global_view_position(gvp):
+    wl = SMALL["tiled_2x1"]()
+    case = make_case(wl, GRIDS["tiled_2x1"], gvp=gvp)
+    proj = make_projector(case)
+    _, d_dev, d_f64 = dev_dout(case, seed=3)
+    _, got = run_backward(case, proj, DeviceInputs(case), d_dev)
+    assert_grads_close(got, oracle_grads(case, d_f64), gvp)
+
+
+def test_backward_position_outer_weights():
+    wl = SMALL["ragged_ln_bf16"]()
+    case = make_case(wl, GRIDS["ragged_ln_bf16"], k_order=vp.ORDER_POSITION_OUTER)
+    proj = make_projector(case)
+    _, d_dev, d_f64 = dev_dout(case, seed=5)
+    _, got = run_backward(case, proj, DeviceInputs(case), d_dev)
+    assert_grads_close(got, oracle_grads(case, d_f64), "position-outer")
+
+
+def test_backward_is_deterministic_and_tile_shape_independent():
+    wl = SMALL["ragged_ln_bf16"]()
+    case = make_case(wl, GRIDS["ragged_ln_bf16"])
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    _, d_dev, _ = dev_dout(case)
+    _, a = run_backward(case, proj, dev, d_dev)
+    _, b = run_backward(case, proj, dev, d_dev)
+    proj.set_tile_pairs(False)
+    _, c = run_backward(case, proj, dev, d_dev)
+    for n in a:
+        np.testing.assert_array_equal(a[n], b[n], err_msg=n)
+        np.testing.assert_array_equal(a[n], c[n], err_msg=n)
+
+
+@pytest.mark.parametrize("name", ["tiled_2x1", "ragged_ln_bf16"])
+def test_backward_subset_of_outputs_matches_full_run(name):
+    wl = SMALL[name]()
+    case = make_case(wl, GRIDS[name])
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    _, d_dev, _ = dev_dout(case)
+    _, full = run_backward(case, proj, dev, d_dev)
+    for names in (["W2"], ["b1", "newline"], ["features"], ["gamma", "beta"], ["W1", "sep"], ["b2"], ["gamma"]):
+        names = [n for n in names if n in full]
+        if not names:
+            continue
+        _, part = run_backward(case, proj, dev, d_dev, names)
+        for n in names:
+            np.testing.assert_array_equal(part[n], full[n], err_msg=str(names))
+
+
+def test_backward_count_mismatch_gives_zero_gradients():
+    wl = SMALL["ragged_ln_bf16"]()
+    case = make_case(wl, GRIDS["ragged_ln_bf16"])
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    ids = dev.ids.clone()
+    ids[int(np.flatnonzero(case.ids == W.IMAGE_TOKEN_ID)[0])] = 5
+    dev.ids = ids
+    _, d_dev, _ = dev_dout(case)
+    rc, got = run_backward(case, proj, dev, d_dev)
+    assert rc == vp.OK
+    assert proj.status() == vp.ERR_TOKEN_COUNT
+    for n, v in got.items():
+        assert not np.any(v), n
+
+
+def test_backward_without_images_zeroes_outputs():
+    wl = SMALL["tiled_2x1"]()
+    case = make_case(wl, GRIDS["tiled_2x1"])
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    text = torch.randint(0, 1000, (64,), dtype=torch.int64, device="cuda")
+    d = torch.ones((64, wl.N2), dtype=torch.bfloat16, device="cuda")
+    grads = {n: torch.full(s, float("nan"), device="cuda") for n, s in grad_shapes(case).items() if n != "features"}
+    proj.backward(None, None, None, text, W.IMAGE_TOKEN_ID, d, grads, n_images=0)
+    assert proj.status() == vp.OK
+    for n, t in grads.items():
+        assert not bool(t.any()), n
+
+
+def test_backward_rejects_deeper_mlp_and_bad_alignment():
+    wl = SMALL["tiny"]()
+    case = make_case(wl, depth=3)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    _, d_dev, _ = dev_dout(case)
+    rc, _ = run_backward(case, proj, dev, d_dev, ["b2"], check=False)
+    assert rc == vp.ERR_UNSUPPORTED
+    case2 = make_case(wl)
+    proj2 = make_projector(case2)
+    g = torch.zeros(wl.N2 + 1, device="cuda")
+    rc = proj2.backward(dev.feats, case2.hw, None, dev.ids, W.IMAGE_TOKEN_ID, d_dev, {"b2": g[1:]}, check=False)
+    assert rc == vp.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["moonvit", "vl2", "dsvit"])
+def test_backward_full_size_sparse_gradient(name):
+    """Full-size workload, d_out nonzero on 24 placeholder rows and 8 text rows: the
+    oracle evaluates only the tokens with a nonzero output gradient (the others add
+    exactly zero), the GPU runs the whole batch."""
+    wl = W.WORKLOADS[name]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    rng = np.random.default_rng(7)
+    ph = np.flatnonzero(case.ids == W.IMAGE_TOKEN_ID)
+    tx = np.flatnonzero(case.ids != W.IMAGE_TOKEN_ID)
+    rows = np.sort(np.concatenate([rng.choice(ph, 24, replace=False), rng.choice(tx, 8, replace=False)]))
+    vals = W.grad_out_rows(wl, len(rows))
+    d_dev = torch.zeros((len(case.ids), wl.N2), dtype=torch.bfloat16, device="cuda")
+    d_dev[torch.from_numpy(rows).cuda()] = dev_bf16(vals)
+
+    class Sparse:
+        def __getitem__(self, idx):
+            idx = np.asarray(idx)
+            out = np.zeros((len(idx), wl.N2))
+            hit = np.searchsorted(rows, idx)
+            ok = (hit < len(rows)) & (rows[np.minimum(hit, len(rows) - 1)] == idx)
+            out[ok] = O.bf16_bits_to_f64(vals[hit[ok]])
+            return out
+
+    rc, got = run_backward(case, proj, dev, d_dev)
+    assert rc == vp.OK and proj.status() == vp.OK
+    assert_grads_close(got, oracle_grads(case, Sparse(), skip_zero_rows=True), name)

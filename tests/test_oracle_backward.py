@@ -157,6 +157,80 @@ def test_text_rows_carry_no_gradient():
         np.testing.assert_array_equal(g0[key], g1[key])
 
 
+@pytest.mark.parametrize("name", ["untiled_ln_ragged", "tiled_two_images"])
+def test_skipping_zero_gradient_rows_changes_nothing(name):
+    """Tokens whose output gradient is zero contribute nothing, so evaluating only the
+    others gives the same gradients."""
+    c = _case(**CASES[name])
+    rng = np.random.default_rng(11)
+    keep = rng.random(len(c["ids"])) < 0.3
+    c["d_out"][~keep] = 0.0
+    full = _grads(c)
+    part = B.backward(c["features"], c["grid_hw"], c["spatial_crop"], c["k"], c["params"], c["ids"], IMG,
+                      c["d_out"], 1e-5, feat_is_bf16_bits=False, quantise=False, skip_zero_rows=True)
+    for key in _names(c):
+        np.testing.assert_allclose(part[key], full[key], rtol=0, atol=1e-12 * max(1.0, float(np.abs(full[key]).max())))
+
+
+def _bf16(x):
+    import torch
+    return torch.from_numpy(np.asarray(x, np.float32)).bfloat16().float().numpy().astype(np.float64)
+
+
+def _emulated_rounding_grads(c):
+    """dW1, db1, d_features, dgamma, dbeta under the GPU's rounding model: fp32 products
+    and sums, GELU'(P) rounded to bf16, dP rounded to bf16 (A and H as the oracle's)."""
+    f32 = lambda t: np.asarray(t, np.float32)
+    prm, k = c["params"], c["k"]
+    W1, b1, W2 = prm["W1"], prm["b1"], prm["W2"]
+    gamma, beta = prm["gamma"], prm["beta"]
+    x_all, hw = c["features"], c["grid_hw"]
+    pos = O.placeholder_positions(c["ids"], IMG)
+    offs = np.concatenate([[0], np.cumsum(hw[:, 0].astype(np.int64) * hw[:, 1])])
+    out = {"W1": np.zeros_like(W1), "b1": np.zeros_like(b1), "features": np.zeros_like(x_all),
+           "gamma": np.zeros_like(gamma), "beta": np.zeros_like(beta)}
+    base = 0
+    for v in range(len(hw)):
+        h0, w0 = int(hw[v, 0]), int(hw[v, 1])
+        hp, wp = O.merged_side(h0, k), O.merged_side(w0, k)
+        x = x_all[offs[v]:offs[v + 1]]
+        mu = x.mean(axis=1, keepdims=True)
+        rstd = 1.0 / np.sqrt(((x - mu) ** 2).mean(axis=1, keepdims=True) + 1e-5)
+        xhat = (x - mu) * rstd
+        a = O.unshuffle(O.round_bf16(xhat * gamma + beta).reshape(h0, w0, -1), k)
+        dy = c["d_out"][pos[base:base + hp * wp]]
+        base += hp * wp
+        p = (f32(a) @ f32(W1).T + f32(b1)).astype(np.float64)
+        dp = _bf16((f32(dy) @ f32(W2)).astype(np.float64) * _bf16(B.gelu_grad(p)))
+        out["W1"] += (f32(dp).T @ f32(a)).astype(np.float64)
+        out["b1"] += f32(dp).sum(axis=0)
+        da = (f32(dp) @ f32(W1)).astype(np.float64)
+        dsrc = O.fold(da, hp, wp, k, x.shape[1])[:h0, :w0].reshape(h0 * w0, -1)
+        out["gamma"] += (dsrc * xhat).sum(axis=0)
+        out["beta"] += dsrc.sum(axis=0)
+        out["features"][offs[v]:offs[v + 1]] = B.layernorm_backward(dsrc, xhat, rstd, gamma)
+    return out
+
+
+def test_magnitudes_bound_the_gradients_and_the_rounding_model():
+    """The absolute-value chain is at least |gradient| everywhere, and the GPU's rounding
+    model (bf16 GELU'(P) and dP) stays within 2^-7 of it."""
+    c = _case(**CASES["untiled_ln_ragged"])
+    c["params"]["W1"] = _bf16(c["params"]["W1"])
+    c["params"]["W2"] = _bf16(c["params"]["W2"])
+    c["d_out"] = _bf16(c["d_out"])
+    g = B.backward(c["features"], c["grid_hw"], None, c["k"], c["params"], c["ids"], IMG, c["d_out"], 1e-5,
+                   feat_is_bf16_bits=False, quantise=True, magnitudes=True)
+    mag = g["mag"]
+    for key in _names(c):
+        assert np.all(mag[key] >= np.abs(g[key]) * (1 - 1e-12)), key
+    emu = _emulated_rounding_grads(c)
+    for key, val in emu.items():
+        err = np.abs(val - g[key])
+        assert np.all(err <= 2.0 ** -7 * mag[key]), key
+        assert np.any(err > 2.0 ** -12 * mag[key]), key      # the model does round
+
+
 def test_backward_rejects_count_mismatch():
     c = _case(**CASES["untiled_no_ln"])
     ids = c["ids"].copy()

@@ -27,11 +27,13 @@ EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
             "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
             "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc", "vlproj_forward_ex",
-            "vlproj_plan_tiles")
+            "vlproj_plan_tiles", "vlproj_backward")
 NOALLOC_MAX_IDS = 64 * 1024 * 1024
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX = 0, 1, 2, 3
-NUM_STAGES = 6
-STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows")
+NUM_STAGES = 15
+STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows",
+          "bwd_index", "bwd_merge", "bwd_gemm1", "bwd_dy", "bwd_dh", "bwd_dw2", "bwd_dw1", "bwd_da", "bwd_tail")
+GRAD_NAMES = ("W1", "b1", "W2", "b2", "gamma", "beta", "newline", "sep", "features")
 
 
 class VlprojError(RuntimeError):
@@ -49,6 +51,16 @@ class ForwardArgs(ctypes.Structure):
         ("out_embeds", ctypes.c_void_p), ("embed_table", ctypes.c_void_p), ("vocab", ctypes.c_int64),
         ("rows_out", ctypes.c_void_p), ("rows_out_cap", ctypes.c_int64),
     ]
+
+
+class BackwardArgs(ctypes.Structure):
+    """Mirror of ``vlproj_backward_args``."""
+    _fields_ = [
+        ("features", ctypes.c_void_p), ("grid_hw", ctypes.c_void_p), ("spatial_crop", ctypes.c_void_p),
+        ("n_images", ctypes.c_int32), ("input_ids", ctypes.c_void_p), ("n_ids", ctypes.c_int64),
+        ("image_token_id", ctypes.c_int64), ("d_out", ctypes.c_void_p),
+    ] + [("d_" + n, ctypes.c_void_p) for n in ("W1", "b1", "W2", "b2", "gamma", "beta", "newline", "sep",
+                                                  "features")]
 
 
 class Config(ctypes.Structure):
@@ -101,6 +113,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_plan_tiles.restype = I64
     lib.vlproj_forward_ex.argtypes = [P, ctypes.POINTER(ForwardArgs), P]
     lib.vlproj_forward_ex.restype = ctypes.c_int
+    lib.vlproj_backward.argtypes = [P, ctypes.POINTER(BackwardArgs), P]
+    lib.vlproj_backward.restype = ctypes.c_int
     lib.vlproj_placeholder_index_noalloc.argtypes = [P, I64, I64, P, I64, P, P]
     lib.vlproj_placeholder_index_noalloc.restype = ctypes.c_int
     return lib
@@ -257,6 +271,26 @@ class Projector:
             raise VlprojError(rc, "vlproj_forward_ex")
         return rc
 
+    def backward(self, features, grid_hw, spatial_crop, input_ids, image_token_id: int, d_out, grads: dict,
+                 stream=None, n_images: Optional[int] = None, check: bool = True) -> int:
+        """vlproj_backward: fp32 gradients into the tensors of ``grads`` (keys from
+        GRAD_NAMES; a missing key is not computed) for the loss gradient ``d_out``
+        ((n_ids, N2) bf16) of the batch given by the other arguments."""
+        unknown = set(grads) - set(GRAD_NAMES)
+        if unknown:
+            raise ValueError(f"unknown gradient names {sorted(unknown)}")
+        g = _host_i32(grid_hw)
+        c = _host_i32(spatial_crop)
+        if n_images is None:
+            n_images = len(c) if c is not None else (0 if g is None else len(g))
+        a = BackwardArgs(_ptr(features), _ptr(g), _ptr(c), n_images, _ptr(input_ids),
+                         0 if input_ids is None else int(input_ids.numel()), int(image_token_id), _ptr(d_out),
+                         *[_ptr(grads.get(n)) for n in GRAD_NAMES])
+        rc = _lib.vlproj_backward(self._h, ctypes.byref(a), _stream_ptr(stream))
+        if check and rc != OK:
+            raise VlprojError(rc, "vlproj_backward")
+        return rc
+
     def hidden(self, features, grid_hw, hidden, stream=None) -> None:
         g = _host_i32(grid_hw)
         rc = _lib.vlproj_hidden(self._h, _ptr(features), _ptr(g), 0 if g is None else len(g), _ptr(hidden),
@@ -274,7 +308,7 @@ class Projector:
             raise VlprojError(rc, "vlproj_profile_enable")
 
     def stage_ms(self) -> dict:
-        """Per-stage device milliseconds of the most recent profiled forward (synchronises)."""
+        """Per-stage device milliseconds of the most recent profiled call (synchronises)."""
         buf = (ctypes.c_float * NUM_STAGES)()
         rc = _lib.vlproj_profile_read(self._h, ctypes.cast(buf, ctypes.c_void_p), NUM_STAGES)
         if rc < 0:

@@ -16,6 +16,11 @@
 //   GEMM2 (A_TILE, EPI_SCATTER):
 //       out[dest[m], n] = bf16( sum_q H[m, q] W2[n, q] + b2[n] )
 //       the epilogue writes each row straight into its placeholder row.
+//   Backward epilogues (A_TILE, no scatter):
+//       EPI_BWD_H   P = acc + b1: G = bf16(GELU'(P)) row-major and H^T = bf16(GELU(P))
+//                   transposed, so H^T can be a K-major operand of the W2 gradient
+//       EPI_DGELU   dP = bf16(acc * G), row-major and transposed (dP^T)
+//       EPI_F32     acc as fp32, row-major (weight and input gradients)
 //
 // One persistent CTA per SM walks output tiles of BM x BN in banded order (see
 // tile_coords: the CTAs running together share A tiles and an L2-sized band of B).
@@ -45,6 +50,9 @@ constexpr int GEMM_THREADS = 256;
 constexpr int GATHER_THREADS = 64;
 constexpr int EPI_GELU = 0;
 constexpr int EPI_SCATTER = 1;
+constexpr int EPI_BWD_H = 2;
+constexpr int EPI_DGELU = 3;
+constexpr int EPI_F32 = 4;
 constexpr int A_TILE = 0;               // dense row-major A, tiled TMA
 constexpr int A_IM2COL = 1;             // merge-gather by TMA im2col
 constexpr int A_CPASYNC = 2;            // merge-gather by cp.async
@@ -93,6 +101,11 @@ struct GemmParams {
     const int32_t* rowdest;         // destination row of each m (-1 = no write), or null = row m
     int64_t out_rows;               // rows of `out` (bounds guard)
     const int* fwd_status;          // nonzero = count check failed, write nothing (null = ignore)
+    // backward epilogues
+    __nv_bfloat16* out_t;           // EPI_BWD_H: H^T, EPI_DGELU: dP^T, [N][ldt] bf16
+    int64_t ldt;                    // row stride of out_t in elements (a multiple of 8)
+    const __nv_bfloat16* aux;       // EPI_DGELU: G = GELU'(P) [M][N] bf16
+    float* outf;                    // EPI_F32: [M][N] fp32
     int group_n;                    // N-blocks per raster band (see tile_coords)
     int* err;                       // latched error word
     uint64_t wait_ns;               // bound on every wait
@@ -118,9 +131,33 @@ __device__ __forceinline__ float gelu_erf(float x) {
     return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
 }
 
+// d/dx of 0.5 x (1 + erf(x / sqrt 2)): Phi(x) + x phi(x).
+__device__ __forceinline__ float gelu_erf_grad(float x) {
+    return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) + x * 0.39894228040143268f * expf(-0.5f * x * x);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The warp's 32 rows (lane = row m) x 32 columns (x[j] = column n0 + j) stored
+// transposed: out_t[(n0 + j) * ldt + m]. Lanes 2i and 2i+1 trade one value per column
+// pair, so each lane writes two consecutive rows of one column as a 4-byte store and
+// every store instruction covers two 64-byte runs. `ok`: the pair's even row is in range.
+__device__ __forceinline__ void store_transposed(const float (&x)[32], __nv_bfloat16* out_t, int64_t ldt, int n0,
+                                                 int m, int lane, bool ok) {
+    const bool odd = (lane & 1) != 0;
+    const int64_t m_even = m & ~1;
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+        const float give = odd ? x[j] : x[j + 1];
+        const float got = __shfl_xor_sync(0xffffffffu, give, 1);
+        const float lo = odd ? got : x[j];          // row m_even
+        const float hi = odd ? x[j + 1] : got;      // row m_even + 1
+        const int64_t col = n0 + j + (odd ? 1 : 0);
+        if (ok) *reinterpret_cast<uint32_t*>(out_t + col * ldt + m_even) = pack_bf16x2(lo, hi);
+    }
 }
 
 template <int BN, int kAMode, int kEpi, int kCtas>
@@ -416,7 +453,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             int64_t d = m;
             if (row_ok && p.rowdest) d = __ldg(&p.rowdest[m]);
             row_ok = row_ok && d >= 0 && d < p.out_rows;
-            __nv_bfloat16* dst_row = row_ok ? p.out + d * p.N : nullptr;
+            __nv_bfloat16* dst_row = (row_ok && p.out) ? p.out + d * p.N : nullptr;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
@@ -425,23 +462,71 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(t_row + c * 32, v);
                 tmem_ld_wait();
-                const float bl = __ldg(&p.bias[n0 + lane]);
-                uint32_t packed[16];
+                if constexpr (kEpi == EPI_F32) {
+                    if (row_ok) {
+                        float4* d4 = reinterpret_cast<float4*>(p.outf + static_cast<int64_t>(m) * p.N + n0);
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    float x0 = __uint_as_float(v[j]) + __shfl_sync(0xffffffffu, bl, j);
-                    float x1 = __uint_as_float(v[j + 1]) + __shfl_sync(0xffffffffu, bl, j + 1);
-                    if (kEpi == EPI_GELU) {
-                        x0 = gelu_erf(x0);
-                        x1 = gelu_erf(x1);
+                        for (int j = 0; j < 8; ++j)
+                            d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
                     }
-                    packed[j / 2] = pack_bf16x2(x0, x1);
-                }
-                if (row_ok) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst_row + n0);
+                } else if constexpr (kEpi == EPI_BWD_H || kEpi == EPI_DGELU) {
+                    float x[32];
+                    uint32_t packed[16];
+                    if constexpr (kEpi == EPI_BWD_H) {
+                        const float bl = __ldg(&p.bias[n0 + lane]);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                        for (int j = 0; j < 32; j += 2) {
+                            const float p0 = __uint_as_float(v[j]) + __shfl_sync(0xffffffffu, bl, j);
+                            const float p1 = __uint_as_float(v[j + 1]) + __shfl_sync(0xffffffffu, bl, j + 1);
+                            packed[j / 2] = pack_bf16x2(gelu_erf_grad(p0), gelu_erf_grad(p1));
+                            x[j] = gelu_erf(p0);
+                            x[j + 1] = gelu_erf(p1);
+                        }
+                    } else {
+                        uint4 g4[4] = {};
+                        if (row_ok) {
+                            const uint4* src = reinterpret_cast<const uint4*>(p.aux + static_cast<int64_t>(m) * p.N + n0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) g4[j] = __ldg(src + j);
+                        }
+                        const uint32_t* gw = reinterpret_cast<const uint32_t*>(g4);
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            x[j] = __uint_as_float(v[j]) * __uint_as_float(gw[j / 2] << 16);
+                            x[j + 1] = __uint_as_float(v[j + 1]) * __uint_as_float(gw[j / 2] & 0xFFFF0000u);
+                            packed[j / 2] = pack_bf16x2(x[j], x[j + 1]);
+                            // the transposed copy holds the same bf16 values as the row-major one
+                            x[j] = __uint_as_float(packed[j / 2] << 16);
+                            x[j + 1] = __uint_as_float(packed[j / 2] & 0xFFFF0000u);
+                        }
+                    }
+                    if (row_ok) {
+                        uint4* d4 = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(m) * p.N + n0);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                    }
+                    store_transposed(x, p.out_t, p.ldt, n0, m, lane, (m & ~1) < p.M);
+                } else {
+                    const float bl = __ldg(&p.bias[n0 + lane]);
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float x0 = __uint_as_float(v[j]) + __shfl_sync(0xffffffffu, bl, j);
+                        float x1 = __uint_as_float(v[j + 1]) + __shfl_sync(0xffffffffu, bl, j + 1);
+                        if (kEpi == EPI_GELU) {
+                            x0 = gelu_erf(x0);
+                            x1 = gelu_erf(x1);
+                        }
+                        packed[j / 2] = pack_bf16x2(x0, x1);
+                    }
+                    if (row_ok) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst_row + n0);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                    }
                 }
             }
             tc_fence_before();

@@ -1,0 +1,470 @@
+// Host-side pieces shared by the library's translation units: driver entry points,
+// tensor-map encoders, device scratch buffers, the batch plan (closed-form geometry),
+// GEMM launchers, and the handle behind the opaque vlproj_handle.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/vlproj.h"
+#include "gemm_sm100.cuh"
+#include "kernels_aux.cuh"
+
+#define VLP_CUDA(call)                                                                        \
+    do {                                                                                      \
+        cudaError_t e_ = (call);                                                              \
+        if (e_ != cudaSuccess) {                                                              \
+            std::fprintf(stderr, "vlproj: %s failed: %s (%s:%d)\n", #call, cudaGetErrorString(e_), \
+                         __FILE__, __LINE__);                                                 \
+            return VLPROJ_ERR_CUDA;                                                           \
+        }                                                                                     \
+    } while (0)
+
+namespace vlp_host {
+
+using vlp::GemmLayout;
+using vlp::GemmParams;
+using vlp::ImageDesc;
+using vlp::ViewDesc;
+
+
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+struct DriverFns {
+    PFN_cuTensorMapEncodeTiled_v12000 tiled = nullptr;
+    PFN_cuTensorMapEncodeIm2col_v12000 im2col = nullptr;
+};
+
+inline const DriverFns& driver() {
+    static DriverFns fns;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fns.tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeIm2col", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fns.im2col = reinterpret_cast<PFN_cuTensorMapEncodeIm2col_v12000>(p);
+    });
+    return fns;
+}
+
+// 2D bf16 row-major matrix [rows][cols] with row stride ld elements (0 = cols, a
+// multiple of 8), box = box_rows x 64 columns, 128-byte swizzle, out-of-range elements
+// read as zero.
+inline int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                          uint64_t ld = 0) {
+    auto fn = driver().tiled;
+    if (!fn) return VLPROJ_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {(ld ? ld : cols) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(vlp::BK), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
+// im2col map of n views of one (h, w) grid of C-channel bf16 patches, packed back to
+// back from `base`: the k x k, stride-k window walk of the merge. Base positions run
+// over 0, k, ..., k*(w'-1) (lower corner 0, upper corner k*w' - w - (k-1), the
+// convolution form of "pad the high end to k*w'"), `pixels` per load, 64 channels each.
+inline int encode_im2col(CUtensorMap* map, const void* base, int C, int h, int w, int n, int k, int pixels) {
+    auto fn = driver().im2col;
+    if (!fn) return VLPROJ_ERR_CUDA;
+    const int hp = (h + k - 1) / k, wp = (w + k - 1) / k;
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(w), static_cast<cuuint64_t>(h),
+                          static_cast<cuuint64_t>(n)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(w) * C * 2,
+                             static_cast<cuuint64_t>(h) * w * C * 2};
+    int lower[2] = {0, 0};
+    int upper[2] = {k * wp - w - (k - 1), k * hp - h - (k - 1)};
+    cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(k), static_cast<cuuint32_t>(k), 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, lower, upper,
+                    static_cast<cuuint32_t>(vlp::BK), static_cast<cuuint32_t>(pixels), estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
+// 5D tiled map of n views of one (h, w) grid with k | h, k | w and w' | 128: dims
+// (C, k, w', k, h' * n) with strides (C, k*C, w*C, k*w*C) elements, box
+// (64, 1, w', 1, 128 / w'): one box is 128 merged tokens, row-major, at filter tap
+// (dy, dx) = (coordinate 3, coordinate 1).
+inline int encode_box5(CUtensorMap* map, const void* base, int C, int h, int w, int n, int k) {
+    auto fn = driver().tiled;
+    if (!fn) return VLPROJ_ERR_CUDA;
+    const int hp = h / k, wp = w / k;
+    cuuint64_t dims[5] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(wp),
+                          static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(hp) * n};
+    const cuuint64_t e = 2;
+    cuuint64_t strides[4] = {static_cast<cuuint64_t>(C) * e, static_cast<cuuint64_t>(k) * C * e,
+                             static_cast<cuuint64_t>(w) * C * e, static_cast<cuuint64_t>(k) * w * C * e};
+    cuuint32_t box[5] = {static_cast<cuuint32_t>(vlp::BK), 1, static_cast<cuuint32_t>(wp), 1,
+                         static_cast<cuuint32_t>(vlp::BM / wp)};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
+template <typename T>
+struct DevBuf {
+    T* ptr = nullptr;
+    size_t cap = 0;   // elements
+    int ensure(size_t n) {
+        if (n <= cap) return VLPROJ_OK;
+        if (ptr) cudaFree(ptr);
+        ptr = nullptr;
+        cap = 0;
+        size_t want = std::max<size_t>(n, 1) + n / 4;
+        if (cudaMalloc(&ptr, want * sizeof(T)) != cudaSuccess) return VLPROJ_ERR_CUDA;
+        cap = want;
+        return VLPROJ_OK;
+    }
+    void release() {
+        if (ptr) cudaFree(ptr);
+        ptr = nullptr;
+        cap = 0;
+    }
+};
+
+// Pinned host staging for small per-call uploads: reused only after the previous
+// copy out of it has executed; skipped when the bytes equal the last upload.
+struct Uploader {
+    uint8_t* staging = nullptr;
+    size_t cap = 0;
+    cudaEvent_t done = nullptr;
+    std::vector<uint8_t> last;
+    bool valid = false;
+    int put(void* dst, const void* src, size_t bytes, cudaStream_t s) {
+        if (valid && last.size() == bytes && std::memcmp(last.data(), src, bytes) == 0) {
+            // unchanged: the device copy is (or will be) there; order `s` after it
+            if (done && bytes) VLP_CUDA(cudaStreamWaitEvent(s, done, 0));
+            return VLPROJ_OK;
+        }
+        valid = false;
+        if (bytes == 0) return VLPROJ_OK;
+        if (!done) VLP_CUDA(cudaEventCreateWithFlags(&done, cudaEventDisableTiming));
+        VLP_CUDA(cudaEventSynchronize(done));
+        if (bytes > cap) {
+            if (staging) cudaFreeHost(staging);
+            staging = nullptr;
+            cap = 0;
+            VLP_CUDA(cudaMallocHost(&staging, bytes * 2));
+            cap = bytes * 2;
+        }
+        std::memcpy(staging, src, bytes);
+        VLP_CUDA(cudaMemcpyAsync(dst, staging, bytes, cudaMemcpyHostToDevice, s));
+        VLP_CUDA(cudaEventRecord(done, s));
+        last.assign(static_cast<const uint8_t*>(src), static_cast<const uint8_t*>(src) + bytes);
+        valid = true;
+        return VLPROJ_OK;
+    }
+    void invalidate() { valid = false; }
+    void release() {
+        if (done) cudaEventSynchronize(done);
+        if (staging) cudaFreeHost(staging);
+        if (done) cudaEventDestroy(done);
+        staging = nullptr;
+        done = nullptr;
+        cap = 0;
+        valid = false;
+    }
+};
+
+struct Plan {
+    std::vector<ViewDesc> views;
+    std::vector<ImageDesc> images;
+    int64_t M = 0;          // GEMM rows (merged tokens, varlen im2col runs padded to `chunk`)
+    int64_t M_real = 0;     // merged tokens
+    int64_t R = 0;          // assembled rows
+    int64_t P = 0;          // patches
+    int max_special = 0;    // most special rows of one image
+    bool uniform = true;    // every view has the same grid
+    bool im2col = true;     // GEMM1 gathers with TMA im2col (else cp.async)
+    bool box5 = false;      // ... or with one 5D tiled box per K-block (regular grids)
+    bool merged_ln = false; // ... or reads A written in token order by the LayerNorm pass
+    int chunk = 128;        // im2col rows per load
+};
+
+inline int validate_config(const vlproj_config* c) {
+    if (!c) return VLPROJ_ERR_INVALID_ARG;
+    if (c->depth < 2 || c->depth > 8 || c->tile_tag == VLPROJ_TILE_1D || c->token_pooling != 0)
+        return VLPROJ_ERR_UNSUPPORTED;
+    if (c->k < 1 || c->k > 3) return VLPROJ_ERR_UNSUPPORTED;
+    if (c->tile_tag != VLPROJ_TILE_NONE && c->tile_tag != VLPROJ_TILE_2D) return VLPROJ_ERR_UNSUPPORTED;
+    if (c->global_view_pos != VLPROJ_GLOBAL_HEAD && c->global_view_pos != VLPROJ_GLOBAL_TAIL)
+        return VLPROJ_ERR_INVALID_ARG;
+    if (c->feat_dtype != VLPROJ_FEAT_BF16 && c->feat_dtype != VLPROJ_FEAT_F32) return VLPROJ_ERR_INVALID_ARG;
+    if (c->k_order != VLPROJ_ORDER_CHANNEL_OUTER && c->k_order != VLPROJ_ORDER_POSITION_OUTER)
+        return VLPROJ_ERR_INVALID_ARG;
+    if (c->C <= 0 || c->C % 64 != 0 || c->N1 <= 0 || c->N1 % 64 != 0 || c->N2 <= 0 || c->N2 % 32 != 0)
+        return VLPROJ_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(c->k) * c->k * c->C > (1 << 20) || c->N1 > (1 << 20) || c->N2 > (1 << 20))
+        return VLPROJ_ERR_INVALID_ARG;
+    return VLPROJ_OK;
+}
+
+// Closed-form geometry of one batch. Returns an error for inconsistent shapes.
+// gather_mode (VLPROJ_GATHER_*) resolves to im2col or cp.async here (plan.im2col);
+// with im2col and views of different grids each view's run of GEMM rows is padded to
+// a multiple of 32, so the im2col loads of per-view maps never straddle two views.
+inline int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int32_t* crop, int32_t n_images,
+               bool tiled_override_none, int gather_mode, Plan* out) {
+    Plan& pl = *out;
+    pl = Plan();
+    if (n_images < 0) return VLPROJ_ERR_INVALID_ARG;
+    if (n_images > 0 && !grid_hw) return VLPROJ_ERR_INVALID_ARG;
+    const bool tiled = !tiled_override_none && c.tile_tag == VLPROJ_TILE_2D;
+    if (tiled && n_images > 0 && !crop) return VLPROJ_ERR_INVALID_ARG;
+    const int k = c.k;
+    // first pass: view count, shapes, uniformity
+    int64_t n_views = 0;
+    for (int32_t img = 0; img < n_images; ++img) {
+        const int tw = tiled ? crop[2 * img] : 0;
+        const int th = tiled ? crop[2 * img + 1] : 0;
+        if (tiled && (tw < 1 || th < 1 || static_cast<int64_t>(tw) * th > 4096)) return VLPROJ_ERR_INVALID_ARG;
+        n_views += tiled ? 1 + tw * th : 1;
+    }
+    for (int64_t v = 0; v < n_views; ++v) {
+        const int h = grid_hw[2 * v], w = grid_hw[2 * v + 1];
+        if (h < 1 || w < 1 || h > 65535 || w > 65535) return VLPROJ_ERR_INVALID_ARG;
+        if (h != grid_hw[0] || w != grid_hw[1]) pl.uniform = false;
+    }
+    pl.chunk = pl.uniform ? 128 : 32;
+    if (gather_mode == VLPROJ_GATHER_AUTO && (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32)) {
+        // a LayerNorm / convert pass writes a bf16 copy anyway: write it as A itself
+        pl.merged_ln = true;
+        pl.im2col = false;
+        gather_mode = VLPROJ_GATHER_CPASYNC;   // no padding, no chunk table
+    }
+    pl.im2col = !pl.merged_ln &&
+                (gather_mode == VLPROJ_GATHER_IM2COL || (gather_mode == VLPROJ_GATHER_AUTO && pl.uniform));
+    if (pl.uniform && n_views > 0 && (gather_mode == VLPROJ_GATHER_BOX || gather_mode == VLPROJ_GATHER_AUTO)) {
+        const int h = grid_hw[0], w = grid_hw[1];
+        if (h % k == 0 && w % k == 0 && w / k <= vlp::BM && vlp::BM % (w / k) == 0) {
+            pl.box5 = true;
+            pl.im2col = false;
+        } else if (gather_mode == VLPROJ_GATHER_BOX) {
+            pl.im2col = true;             // not regular: the im2col walk does the same job
+        }
+    }
+    const int pad_to = (pl.im2col && !pl.uniform) ? pl.chunk : 1;
+    int64_t v = 0;
+    for (int32_t img = 0; img < n_images; ++img) {
+        const int tw = tiled ? crop[2 * img] : 0;
+        const int th = tiled ? crop[2 * img + 1] : 0;
+        const int nv = tiled ? 1 + tw * th : 1;
+        const int h0 = grid_hw[2 * v], w0 = grid_hw[2 * v + 1];
+        const int hp = (h0 + k - 1) / k, wp = (w0 + k - 1) / k;
+        int64_t rows;
+        if (tiled)
+            rows = static_cast<int64_t>(hp) * (wp + 1) + 1 +
+                   static_cast<int64_t>(th) * hp * (static_cast<int64_t>(tw) * wp + 1);
+        else
+            rows = static_cast<int64_t>(hp) * wp;
+        for (int t = 0; t < nv; ++t, ++v) {
+            const int h = grid_hw[2 * v], w = grid_hw[2 * v + 1];
+            if (h != h0 || w != w0) return VLPROJ_ERR_INVALID_ARG;   // views of one image share a grid
+            ViewDesc d{};
+            d.patch_start = pl.P;
+            d.tok_start = static_cast<int32_t>(pl.M);
+            d.tok_real = static_cast<int32_t>(pl.M_real);
+            d.h = h; d.w = w; d.hp = hp; d.wp = wp;
+            d.row_base = static_cast<int32_t>(pl.R);
+            d.view_in_image = t;
+            d.tw = tw; d.th = th;
+            d.tail = tiled && c.global_view_pos == VLPROJ_GLOBAL_TAIL;
+            pl.views.push_back(d);
+            const int64_t toks = static_cast<int64_t>(hp) * wp;
+            pl.P += static_cast<int64_t>(h) * w;
+            pl.M_real += toks;
+            pl.M += (toks + pad_to - 1) / pad_to * pad_to;
+            if (pl.P >= (int64_t(1) << 31) || pl.M >= (int64_t(1) << 30)) return VLPROJ_ERR_INVALID_ARG;
+        }
+        if (tiled) {
+            ImageDesc im{};
+            im.row_base = static_cast<int32_t>(pl.R);
+            im.hp = hp; im.wp = wp; im.tw = tw; im.th = th;
+            im.tail = c.global_view_pos == VLPROJ_GLOBAL_TAIL;
+            pl.images.push_back(im);
+            pl.max_special = std::max(pl.max_special, hp + th * hp + 1);
+        }
+        pl.R += rows;
+        if (pl.R >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
+    }
+    return VLPROJ_OK;
+}
+
+// N-blocks per raster band: all of them while B fits comfortably in L2 (about 40 MB,
+// a margin under one die's share of the 126 MB), else as many as fit in that budget.
+inline int raster_group(int N, int K, int BN) {
+    const int n_tiles = (N + BN - 1) / BN;
+    const int64_t per_block = static_cast<int64_t>(BN) * K * 2;
+    const int64_t budget = int64_t(40) << 20;
+    if (per_block * n_tiles <= budget) return n_tiles;
+    return static_cast<int>(std::max<int64_t>(1, budget / per_block));
+}
+
+template <int BN, int A, int E, int CTAS>
+int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, int num_sms, cudaStream_t s) {
+    using L = GemmLayout<BN, CTAS>;
+    auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
+    if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN);
+    VLP_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC));
+    const int tiles = ((p.M + vlp::BM * CTAS - 1) / (vlp::BM * CTAS)) * ((p.N + BN - 1) / BN);
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(vlp::GEMM_THREADS);
+    cfg.dynamicSmemBytes = L::SMEM_ALLOC;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CTAS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    int resident = num_sms / CTAS;               // persistent: one unit per SM (pair of SMs)
+    if constexpr (CTAS > 1) {
+        // pairs must sit in one GPC: ask how many can be resident at once
+        static int cached = -1;
+        if (cached < 0) {
+            cfg.gridDim = dim3(static_cast<unsigned>(2 * resident));
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            cached = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0 ? n : resident;
+        }
+        resident = std::min(resident, cached);
+    }
+    const int units = std::min(tiles, resident);
+    if (units <= 0) return VLPROJ_OK;
+    cfg.gridDim = dim3(static_cast<unsigned>(units * CTAS));
+    cfg.attrs = CTAS > 1 ? attr : nullptr;
+    cfg.numAttrs = CTAS > 1 ? 1 : 0;
+    VLP_CUDA(cudaLaunchKernelEx(&cfg, kernel, ta, tb, p));
+    return VLPROJ_OK;
+}
+
+// Tile shape: 256 x 256 tiles on CTA pairs when N allows and the A operand comes by
+// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise.
+template <int A, int E>
+int launch_gemm_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb_half,
+                   const GemmParams& p, int num_sms, cudaStream_t s) {
+    if constexpr (A != vlp::A_CPASYNC) {
+        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, p, num_sms, s);
+    }
+    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, p, num_sms, s);
+    return launch_gemm<128, A, E, 1>(ta, tb, p, num_sms, s);
+}
+
+inline int pick_bn(int N) { return N >= 256 ? 256 : 128; }
+
+}  // namespace vlp_host
+
+// The state behind the opaque handle: copies of the weights, their tensor maps, and
+// scratch buffers that grow on demand and are kept between calls.
+struct vlproj_handle {
+    vlproj_config cfg{};
+    int device = 0;
+    int num_sms = 148;
+    int K1 = 0;
+    uint64_t wait_ns = vlp_host::kDefaultWaitNs;
+    int gather_mode = VLPROJ_GATHER_AUTO;
+    __nv_bfloat16* W1p = nullptr;
+    __nv_bfloat16* W2 = nullptr;
+    float* b1 = nullptr;
+    float* b2 = nullptr;
+    float* gamma = nullptr;
+    float* beta = nullptr;
+    CUtensorMap tmW1{}, tmW2{};          // B boxes of BN rows (single-CTA tiles)
+    CUtensorMap tmW1h{}, tmW2h{};        // B boxes of 128 rows (each CTA of a pair loads half)
+    bool pairs = true;                   // run 256 x 256 tiles on CTA pairs where possible
+    // scratch, grown on demand
+    vlp_host::DevBuf<__nv_bfloat16> H, H2, Xn, A;       // H2: second hidden buffer (depth > 2)
+    // middle layers (depth > 2): weights, biases, tensor maps (BN-row and 128-row boxes)
+    std::vector<__nv_bfloat16*> Wm;
+    std::vector<float*> bm;
+    std::vector<CUtensorMap> tmWm, tmWmh;
+    vlp_host::DevBuf<int32_t> pos, rowdest, counts;
+    vlp_host::DevBuf<int2> gmeta;
+    vlp_host::DevBuf<int4> chunks;
+    vlp_host::DevBuf<vlp::ViewDesc> dviews;
+    vlp_host::DevBuf<vlp::ImageDesc> dimages;
+    vlp_host::DevBuf<CUtensorMap> dmaps;
+    int* status = nullptr;       // [0] latched error, [1] per-forward count check
+    vlp_host::Uploader up_views, up_images, up_maps;
+    std::vector<CUtensorMap> host_maps;
+    // the placeholder index runs on `side`, forked from / joined to the caller's stream
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr;
+    // tracing: start / end event of every stage, recorded on the stream that runs it
+    bool profiling = false;
+    bool profiled_valid = false;
+    cudaEvent_t ev_begin[VLPROJ_NUM_STAGES] = {};
+    cudaEvent_t ev_end[VLPROJ_NUM_STAGES] = {};
+    bool stage_ran[VLPROJ_NUM_STAGES] = {};
+    int64_t launches = 0;
+    // cached tensor map of H
+    CUtensorMap tmH{};
+    const void* tmH_ptr = nullptr;
+    int64_t tmH_rows = -1;
+    // backward: transposed weights (made on the first backward call) and scratch
+    __nv_bfloat16* W2t = nullptr;        // [N1][N2]
+    __nv_bfloat16* W1pt = nullptr;       // [K1][N1], rows in position-outer order
+    CUtensorMap tmW2t{}, tmW2th{}, tmW1pt{}, tmW1pth{};
+    vlp_host::DevBuf<__nv_bfloat16> G, Ht, dY, dYt, dP, dPt, At;
+    vlp_host::DevBuf<float> dA, part, part_sp;
+};
+
+namespace vlp_host {
+
+// Stage timing: begin / end events on the stream that runs the stage.
+inline void stage_begin(vlproj_handle* h, int stage, cudaStream_t s) {
+    h->stage_ran[stage] = true;
+    if (h->profiling) cudaEventRecord(h->ev_begin[stage], s);
+}
+inline void stage_end(vlproj_handle* h, int stage, cudaStream_t s) {
+    if (h->profiling) cudaEventRecord(h->ev_end[stage], s);
+}
+
+// LayerNorm-merge launch: the single-pass (registers) form when C fits.
+inline int launch_ln_merge(const vlproj_config& c, const void* features, const int2* gmeta, int M, const float* gamma,
+                    const float* beta, float eps, __nv_bfloat16* A, cudaStream_t s) {
+    const int64_t items = static_cast<int64_t>(M) * c.k * c.k;
+    const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+    const int nvec = c.C / 8;
+    const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
+#define VLP_LNM(F, V) vlp::vlp_ln_merge_regs_kernel<F, V><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A)
+    if (nvec <= 64) { if (f32) VLP_LNM(true, 2); else VLP_LNM(false, 2); }
+    else if (nvec <= 160) { if (f32) VLP_LNM(true, 5); else VLP_LNM(false, 5); }
+    else if (nvec <= 256) { if (f32) VLP_LNM(true, 8); else VLP_LNM(false, 8); }
+    else if (f32) vlp::vlp_ln_merge_kernel<true><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A);
+    else vlp::vlp_ln_merge_kernel<false><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A);
+#undef VLP_LNM
+    VLP_CUDA(cudaGetLastError());
+    return VLPROJ_OK;
+}
+
+inline int upload_plan(vlproj_handle* h, const Plan& pl, cudaStream_t s) {
+    if (h->dviews.ptr == nullptr || h->dviews.cap < pl.views.size()) h->up_views.invalidate();
+    if (h->dimages.ptr == nullptr || h->dimages.cap < pl.images.size()) h->up_images.invalidate();
+    if (h->dviews.ensure(std::max<size_t>(pl.views.size(), 1))) return VLPROJ_ERR_CUDA;
+    if (h->dimages.ensure(std::max<size_t>(pl.images.size(), 1))) return VLPROJ_ERR_CUDA;
+    int rc = h->up_views.put(h->dviews.ptr, pl.views.data(), pl.views.size() * sizeof(ViewDesc), s);
+    if (rc) return rc;
+    return h->up_images.put(h->dimages.ptr, pl.images.data(), pl.images.size() * sizeof(ImageDesc), s);
+}
+
+}  // namespace vlp_host

@@ -36,7 +36,7 @@ __device__ __forceinline__ int block_sum_256(int v, int* red) {
 }
 
 // counts[b] = number of placeholders in ids[b*SCAN_CHUNK, (b+1)*SCAN_CHUNK)
-__global__ void __launch_bounds__(SCAN_THREADS) vlp_count_kernel(const int64_t* __restrict__ ids, int64_t n,
+static __global__ void __launch_bounds__(SCAN_THREADS) vlp_count_kernel(const int64_t* __restrict__ ids, int64_t n,
                                                                  int64_t token, int32_t* __restrict__ counts) {
     __shared__ int red[SCAN_THREADS / 32];
     const int64_t start = static_cast<int64_t>(blockIdx.x) * SCAN_CHUNK;
@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) vlp_count_kernel(const int64_t* 
 // Writes pos[j] = flat index of the j-th placeholder (j < R), in order. Each block
 // finds its starting rank from the counts of the blocks before it, then ranks its
 // own placeholders with warp ballots. Block 0 records whether the total equals R.
-__global__ void __launch_bounds__(SCAN_THREADS) vlp_compact_kernel(const int64_t* __restrict__ ids, int64_t n,
+static __global__ void __launch_bounds__(SCAN_THREADS) vlp_compact_kernel(const int64_t* __restrict__ ids, int64_t n,
                                                                    int64_t token, const int32_t* __restrict__ counts,
                                                                    int nblocks, int32_t* __restrict__ pos, int64_t R,
                                                                    int* fwd_status, int* err) {
@@ -138,7 +138,7 @@ constexpr int DEST_COMPACT = 2;   // rowdest[m] = merged-token index (views in o
 // One thread per GEMM row m (and per im2col chunk): gather metadata for the cp.async
 // path, the destination of the row, and the im2col coordinates of each chunk's
 // first token. Rows in a view's padding get no destination and zero gather masks.
-__global__ void __launch_bounds__(256) vlp_geometry_kernel(const ViewDesc* __restrict__ views, int n_views, int M,
+static __global__ void __launch_bounds__(256) vlp_geometry_kernel(const ViewDesc* __restrict__ views, int n_views, int M,
                                                            int k, const int32_t* __restrict__ pos, int64_t R,
                                                            int dest_mode, int2* __restrict__ gmeta,
                                                            int32_t* __restrict__ rowdest, int4* __restrict__ chunks,
@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(256) vlp_geometry_kernel(const ViewDesc* __res
 // One warp per patch row: y = bf16(((x - mean) * rstd) * gamma + beta) (biased
 // variance, fp32 statistics) or, without LayerNorm, y = bf16(x). C % 8 == 0.
 template <bool kF32In>
-__global__ void __launch_bounds__(256) vlp_layernorm_kernel(const void* __restrict__ x, int64_t P, int C,
+static __global__ void __launch_bounds__(256) vlp_layernorm_kernel(const void* __restrict__ x, int64_t P, int C,
                                                             const float* __restrict__ gamma,
                                                             const float* __restrict__ beta, float eps, int has_ln,
                                                             __nv_bfloat16* __restrict__ y) {
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(256) vlp_layernorm_kernel(const void* __restri
 // statistics and rounding are those of vlp_layernorm_kernel, so A holds exactly the
 // values the gathering paths read from its output.
 template <bool kF32In>
-__global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __restrict__ x, const int2* __restrict__ gmeta,
+static __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __restrict__ x, const int2* __restrict__ gmeta,
                                                            int M, int k, int C, const float* __restrict__ gamma,
                                                            const float* __restrict__ beta, float eps, int has_ln,
                                                            __nv_bfloat16* __restrict__ A) {
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __restric
 // kVec 8-channel vectors of the patch in registers, so the patch is read from memory
 // once. Same statistics (sum, then sum of squared deviations, in fp32) and rounding.
 template <bool kF32In, int kVec>
-__global__ void __launch_bounds__(256) vlp_ln_merge_regs_kernel(const void* __restrict__ x,
+static __global__ void __launch_bounds__(256) vlp_ln_merge_regs_kernel(const void* __restrict__ x,
                                                                 const int2* __restrict__ gmeta, int M, int k, int C,
                                                                 const float* __restrict__ gamma,
                                                                 const float* __restrict__ beta, float eps, int has_ln,
@@ -453,11 +453,24 @@ struct ImageDesc {
     int32_t tail;           // global view after the local tiles
 };
 
-// blockIdx.y = image, blockIdx.x = special row n of that image:
+// Row, inside its image, of special row n of a 2D-tiled image:
 //   n <  hp            newline closing global row n
 //   n <  hp + th*hp    newline closing local canvas row n - hp
 //   n == hp + th*hp    the view separator
-__global__ void __launch_bounds__(128) vlp_special_rows_kernel(const ImageDesc* __restrict__ imgs,
+__device__ __forceinline__ int64_t special_row(const ImageDesc& I, int n) {
+    const int n_nl = I.hp + I.th * I.hp;
+    const int64_t global_rows = static_cast<int64_t>(I.hp) * (I.wp + 1);
+    const int64_t local_cols = static_cast<int64_t>(I.tw) * I.wp + 1;
+    const int64_t local_rows = static_cast<int64_t>(I.th) * I.hp * local_cols;
+    const int64_t g0 = I.tail ? local_rows + 1 : 0;
+    const int64_t l0 = I.tail ? 0 : global_rows + 1;
+    if (n < I.hp) return g0 + static_cast<int64_t>(n) * (I.wp + 1) + I.wp;
+    if (n < n_nl) return l0 + static_cast<int64_t>(n - I.hp) * local_cols + local_cols - 1;
+    return I.tail ? local_rows : global_rows;
+}
+
+// blockIdx.y = image, blockIdx.x = special row n of that image (see special_row).
+static __global__ void __launch_bounds__(128) vlp_special_rows_kernel(const ImageDesc* __restrict__ imgs,
                                                                const int32_t* __restrict__ pos, int64_t R,
                                                                const __nv_bfloat16* __restrict__ newline,
                                                                const __nv_bfloat16* __restrict__ sep,
@@ -468,17 +481,8 @@ __global__ void __launch_bounds__(128) vlp_special_rows_kernel(const ImageDesc* 
     const int n = blockIdx.x;
     const int n_nl = I.hp + I.th * I.hp;
     if (n > n_nl) return;
-    const int64_t global_rows = static_cast<int64_t>(I.hp) * (I.wp + 1);
-    const int64_t local_cols = static_cast<int64_t>(I.tw) * I.wp + 1;
-    const int64_t local_rows = static_cast<int64_t>(I.th) * I.hp * local_cols;
-    const int64_t g0 = I.tail ? local_rows + 1 : 0;
-    const int64_t l0 = I.tail ? 0 : global_rows + 1;
-    int64_t r;
-    const __nv_bfloat16* src = newline;
-    if (n < I.hp) r = g0 + static_cast<int64_t>(n) * (I.wp + 1) + I.wp;
-    else if (n < n_nl) r = l0 + static_cast<int64_t>(n - I.hp) * local_cols + local_cols - 1;
-    else { r = I.tail ? local_rows : global_rows; src = sep; }
-    const int64_t g = I.row_base + r;
+    const __nv_bfloat16* src = n < n_nl ? newline : sep;
+    const int64_t g = I.row_base + special_row(I, n);
     if (g < 0 || g >= R) return;
     const int64_t d = pos[g];
     if (d < 0 || d >= out_rows) return;
@@ -490,7 +494,7 @@ __global__ void __launch_bounds__(128) vlp_special_rows_kernel(const ImageDesc* 
 // ---------------------------------------------------------------- token-embedding lookup
 // One warp per row: out[r] = table[ids[r]] for every id that is not the placeholder; an
 // id outside [0, vocab) writes a zero row and latches VLPROJ_ERR_INVALID_ARG.
-__global__ void __launch_bounds__(256) vlp_embed_lookup_kernel(const int64_t* __restrict__ ids, int64_t n,
+static __global__ void __launch_bounds__(256) vlp_embed_lookup_kernel(const int64_t* __restrict__ ids, int64_t n,
                                                                int64_t token, const __nv_bfloat16* __restrict__ table,
                                                                int64_t vocab, __nv_bfloat16* __restrict__ out, int N,
                                                                int* err) {
@@ -511,7 +515,7 @@ __global__ void __launch_bounds__(256) vlp_embed_lookup_kernel(const int64_t* __
 }
 
 // rows_out[j] = out[pos[j]] for the R assembled rows (nothing when the count check failed).
-__global__ void __launch_bounds__(256) vlp_gather_rows_kernel(const int32_t* __restrict__ pos, int64_t R,
+static __global__ void __launch_bounds__(256) vlp_gather_rows_kernel(const int32_t* __restrict__ pos, int64_t R,
                                                               const __nv_bfloat16* __restrict__ out, int64_t out_rows,
                                                               int N, __nv_bfloat16* __restrict__ rows_out,
                                                               const int* __restrict__ fwd_status) {
@@ -529,7 +533,7 @@ __global__ void __launch_bounds__(256) vlp_gather_rows_kernel(const int32_t* __r
 // ---------------------------------------------------------------- W1 column permutation
 // dst[n][p*C + c] = src[n][c*kk + p] for p < kk = k*k (channel-outermost input);
 // with position_outer the columns are copied unchanged.
-__global__ void vlp_permute_w1_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+static __global__ void vlp_permute_w1_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
                                       int64_t N1, int C, int kk, int position_outer) {
     const int64_t K1 = static_cast<int64_t>(C) * kk;
     const int64_t total = N1 * K1;

@@ -1,0 +1,350 @@
+// vlproj_backward (declared in vlproj.h): gradients of the projector for one batch.
+//
+// Enqueued on the caller's stream without host syncs (stage numbers as in vlproj.h):
+//    6  placeholder index + geometry  placeholder positions, the count check, each merged
+//                                     token's destination row and gather data
+//    7  LayerNorm-merge               A [M][k*k*C] bf16, position-outer: the forward's
+//                                     bf16 A operand
+//    8  GEMM1 recompute               P = A W1p^T + b1 -> G = GELU'(P) [M][N1] and
+//                                     H^T = GELU(P)^T [N1][M] (bf16)
+//    9  dY gather                     dY [M][N2] and dY^T [N2][M] from d_out's
+//                                     placeholder rows (zeros if the count check failed)
+//   10  dH GEMM                       dP = (dY W2) * G -> dP [M][N1] and dP^T [N1][M]
+//   11  dW2 GEMM                      dW2 = dY^T H, K = M
+//   12  A^T + dW1 GEMM                A^T with rows in the caller's column order, then
+//                                     dW1 = dP^T A, K = M
+//   13  dA GEMM                       dA = dP W1p [M][k*k*C] fp32
+//   14  tails                         LayerNorm backward -> d_features and gamma / beta
+//                                     partials, column sums -> dgamma, dbeta; newline /
+//                                     separator gradients (db2, db1: row sums of dY^T and
+//                                     dP^T, beside stages 11 and 12)
+// Every contraction runs on the tcgen05 GEMM kernel with a K-major A and B from tensor
+// maps: the weight gradients take the transposed copies (K = M contiguous), which the
+// producing epilogues and the gather kernel write directly. W2^T and W1p^T are made
+// once, on the first call. Stages 11-12 and the bias sums run on the handle's side
+// stream, forked after stage 9 and joined before the call returns.
+#include "host.cuh"
+#include "kernels_bwd.cuh"
+
+using namespace vlp_host;
+
+namespace {
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Tensor maps for a B operand: box of BN rows (single CTAs) and of 128 rows (pairs).
+int encode_b(CUtensorMap* full, CUtensorMap* half, const void* base, uint64_t rows, uint64_t cols, int bn,
+             uint64_t ld = 0) {
+    if (encode_bf16_2d(full, base, rows, cols, static_cast<uint32_t>(bn), ld)) return VLPROJ_ERR_CUDA;
+    return encode_bf16_2d(half, base, rows, cols, 128, ld);
+}
+
+GemmParams gemm_params(const vlproj_handle* h, int64_t M, int N, int64_t K) {
+    GemmParams p{};
+    p.M = static_cast<int>(M);
+    p.N = N;
+    p.K = static_cast<int>(round_up(K, vlp::BK));
+    p.C = h->cfg.C;
+    p.k = h->cfg.k;
+    p.out_rows = M;
+    p.err = h->status;
+    p.wait_ns = h->wait_ns;
+    return p;
+}
+
+void transpose_launch(const __nv_bfloat16* src, int64_t ld_src, int64_t src_rows, const int32_t* rowsel,
+                      const int* zero_if, int64_t M, int Q, __nv_bfloat16* dst, __nv_bfloat16* dst_t, int64_t ldt,
+                      int C, int kk, int chan_outer, cudaStream_t s) {
+    dim3 grid(static_cast<unsigned>((Q + vlp::TR_TILE - 1) / vlp::TR_TILE),
+              static_cast<unsigned>((M + vlp::TR_TILE - 1) / vlp::TR_TILE));
+    vlp::vlp_gather_transpose_kernel<<<grid, 256, 0, s>>>(src, ld_src, src_rows, rowsel, zero_if,
+                                                          static_cast<int>(M), Q, dst, dst_t, ldt, C, kk, chan_outer);
+}
+
+// W2^T [N1][N2] and W1p^T [K1][N1] with their tensor maps, made once per handle.
+int ensure_transposed_weights(vlproj_handle* h, cudaStream_t s) {
+    if (h->W2t && h->W1pt) return VLPROJ_OK;
+    const vlproj_config& c = h->cfg;
+    const size_t n1 = static_cast<size_t>(c.N1), n2 = static_cast<size_t>(c.N2), k1 = static_cast<size_t>(h->K1);
+    if (!h->W2t) VLP_CUDA(cudaMalloc(&h->W2t, n1 * n2 * 2));
+    if (!h->W1pt) VLP_CUDA(cudaMalloc(&h->W1pt, k1 * n1 * 2));
+    h->launches += 2;
+    transpose_launch(h->W2, c.N1, c.N2, nullptr, nullptr, c.N2, c.N1, nullptr, h->W2t, c.N2, c.C, 1, 0, s);
+    transpose_launch(h->W1p, h->K1, c.N1, nullptr, nullptr, c.N1, h->K1, nullptr, h->W1pt, c.N1, c.C, 1, 0, s);
+    VLP_CUDA(cudaGetLastError());
+    if (encode_b(&h->tmW2t, &h->tmW2th, h->W2t, n1, n2, pick_bn(c.N1)) ||
+        encode_b(&h->tmW1pt, &h->tmW1pth, h->W1pt, k1, n1, pick_bn(h->K1)))
+        return VLPROJ_ERR_CUDA;
+    return VLPROJ_OK;
+}
+
+int zero_outputs(const vlproj_backward_args* a, const vlproj_config& c, int K1, int64_t P, cudaStream_t s) {
+    const size_t n1 = c.N1, n2 = c.N2, C = c.C;
+    if (a->d_W1) VLP_CUDA(cudaMemsetAsync(a->d_W1, 0, n1 * K1 * 4, s));
+    if (a->d_b1) VLP_CUDA(cudaMemsetAsync(a->d_b1, 0, n1 * 4, s));
+    if (a->d_W2) VLP_CUDA(cudaMemsetAsync(a->d_W2, 0, n2 * n1 * 4, s));
+    if (a->d_b2) VLP_CUDA(cudaMemsetAsync(a->d_b2, 0, n2 * 4, s));
+    if (a->d_gamma) VLP_CUDA(cudaMemsetAsync(a->d_gamma, 0, C * 4, s));
+    if (a->d_beta) VLP_CUDA(cudaMemsetAsync(a->d_beta, 0, C * 4, s));
+    if (a->d_newline) VLP_CUDA(cudaMemsetAsync(a->d_newline, 0, n2 * 4, s));
+    if (a->d_sep) VLP_CUDA(cudaMemsetAsync(a->d_sep, 0, n2 * 4, s));
+    if (a->d_features && P > 0) VLP_CUDA(cudaMemsetAsync(a->d_features, 0, static_cast<size_t>(P) * C * 4, s));
+    return VLPROJ_OK;
+}
+
+bool misaligned(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 != 0; }
+
+}  // namespace
+
+extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, void* stream) {
+    if (!h || !a) return VLPROJ_ERR_INVALID_ARG;
+    const vlproj_config& c = h->cfg;
+    if (c.depth != 2) return VLPROJ_ERR_UNSUPPORTED;
+    if (c.has_ln && static_cast<size_t>(c.C) * 2 * vlp::LNB_WARPS * 4 > 227 * 1024) return VLPROJ_ERR_UNSUPPORTED;
+    const int64_t n_ids = a->n_ids;
+    if (n_ids < 0 || n_ids >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
+    if (n_ids > 0 && (!a->input_ids || !a->d_out)) return VLPROJ_ERR_INVALID_ARG;
+    if (a->n_images > 0 && !a->features) return VLPROJ_ERR_INVALID_ARG;
+    for (const void* p : {a->features, a->d_out, static_cast<const void*>(a->d_W1), static_cast<const void*>(a->d_b1),
+                          static_cast<const void*>(a->d_W2), static_cast<const void*>(a->d_b2),
+                          static_cast<const void*>(a->d_gamma), static_cast<const void*>(a->d_beta),
+                          static_cast<const void*>(a->d_newline), static_cast<const void*>(a->d_sep),
+                          static_cast<const void*>(a->d_features)})
+        if (misaligned(p)) return VLPROJ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Plan pl;
+    int rc = build_plan(c, a->grid_hw, a->spatial_crop, a->n_images, false, VLPROJ_GATHER_CPASYNC, &pl);
+    if (rc) return rc;
+    const bool tiled = c.tile_tag == VLPROJ_TILE_2D;
+    const int kk = c.k * c.k;
+    const int K1 = h->K1;
+    const int64_t M = pl.M;          // no padding in this plan: M merged tokens
+    const int64_t ldt = round_up(std::max<int64_t>(M, 1), 8);
+
+    // scratch
+    const int nblocks = static_cast<int>((n_ids + vlp::SCAN_CHUNK - 1) / vlp::SCAN_CHUNK);
+    if (h->counts.ensure(std::max(nblocks, 1)) || h->pos.ensure(std::max<int64_t>(pl.R, 1))) return VLPROJ_ERR_CUDA;
+    const bool want_l1 = a->d_W1 || a->d_b1 || a->d_features || a->d_gamma || a->d_beta;
+    const bool want_da = a->d_features || (c.has_ln && (a->d_gamma || a->d_beta));
+    if (M > 0) {
+        if (h->rowdest.ensure(M) || h->gmeta.ensure(M) || h->A.ensure(static_cast<size_t>(M) * K1) ||
+            h->G.ensure(static_cast<size_t>(M) * c.N1) || h->Ht.ensure(static_cast<size_t>(c.N1) * ldt) ||
+            h->dY.ensure(static_cast<size_t>(M) * c.N2) || h->dYt.ensure(static_cast<size_t>(c.N2) * ldt) ||
+            h->dP.ensure(static_cast<size_t>(M) * c.N1) || h->dPt.ensure(static_cast<size_t>(c.N1) * ldt))
+            return VLPROJ_ERR_CUDA;
+        if (a->d_W1 && h->At.ensure(static_cast<size_t>(K1) * ldt)) return VLPROJ_ERR_CUDA;
+        if (want_da && h->dA.ensure(static_cast<size_t>(M) * K1)) return VLPROJ_ERR_CUDA;
+        rc = ensure_transposed_weights(h, s);
+        if (rc) return rc;
+    }
+    rc = upload_plan(h, pl, s);
+    if (rc) return rc;
+    h->profiled_valid = false;
+    for (bool& r : h->stage_ran) r = false;
+
+    // 6. placeholder index, count check, destinations and gather data
+    stage_begin(h, 6, s);
+    h->launches += nblocks > 0 ? 2 : 1;
+    if (nblocks > 0) {
+        vlp::vlp_count_kernel<<<nblocks, vlp::SCAN_THREADS, 0, s>>>(a->input_ids, n_ids, a->image_token_id,
+                                                                    h->counts.ptr);
+        VLP_CUDA(cudaGetLastError());
+    }
+    vlp::vlp_compact_kernel<<<std::max(nblocks, 1), vlp::SCAN_THREADS, 0, s>>>(
+        a->input_ids, n_ids, a->image_token_id, h->counts.ptr, nblocks, h->pos.ptr, pl.R, h->status + 1, h->status);
+    VLP_CUDA(cudaGetLastError());
+    if (M == 0) {
+        stage_end(h, 6, s);
+        rc = zero_outputs(a, c, K1, pl.P, s);
+        if (rc) return rc;
+        h->profiled_valid = h->profiling;
+        return VLPROJ_OK;
+    }
+    ++h->launches;
+    vlp::vlp_geometry_kernel<<<static_cast<unsigned>((M + 255) / 256), 256, 0, s>>>(
+        h->dviews.ptr, static_cast<int>(pl.views.size()), static_cast<int>(M), c.k, h->pos.ptr, pl.R,
+        vlp::DEST_EMBED, h->gmeta.ptr, h->rowdest.ptr, nullptr, 0, pl.chunk, 0);
+    VLP_CUDA(cudaGetLastError());
+    stage_end(h, 6, s);
+
+    const bool want_gemm1 = want_l1 || a->d_W2;     // G feeds dP, H^T feeds dW2
+    const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
+    CUtensorMap tmA{}, tmB{}, tmBh{};
+    GemmParams p{};
+
+    if (want_gemm1) {
+        // 7. A, exactly as the forward pass rounds it
+        stage_begin(h, 7, s);
+        ++h->launches;
+        rc = launch_ln_merge(c, a->features, h->gmeta.ptr, static_cast<int>(M), h->gamma, h->beta, eps, h->A.ptr, s);
+        if (rc) return rc;
+        stage_end(h, 7, s);
+
+        // 8. GEMM1 recompute: G = GELU'(P), H^T
+        if (encode_bf16_2d(&tmA, h->A.ptr, M, K1, vlp::BM)) return VLPROJ_ERR_CUDA;
+        p = gemm_params(h, M, c.N1, K1);
+        p.bias = h->b1;
+        p.out = h->G.ptr;
+        p.out_t = h->Ht.ptr;
+        p.ldt = ldt;
+        stage_begin(h, 8, s);
+        ++h->launches;
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                         h->num_sms, s);
+        if (rc) return rc;
+        stage_end(h, 8, s);
+    }
+
+    // 9. dY and dY^T from the placeholder rows of d_out
+    stage_begin(h, 9, s);
+    ++h->launches;
+    transpose_launch(static_cast<const __nv_bfloat16*>(a->d_out), c.N2, n_ids, h->rowdest.ptr, h->status + 1, M,
+                     c.N2, h->dY.ptr, h->dYt.ptr, ldt, c.C, 1, 0, s);
+    VLP_CUDA(cudaGetLastError());
+    stage_end(h, 9, s);
+
+    // The weight gradients run on the side stream, beside the dP / dA chain on the
+    // caller's stream: A^T and dW2 need only stages 7-9, dW1 waits for dP. Each persistent
+    // GEMM takes the SMs the other leaves free, which fills their last, partial waves.
+    cudaStream_t ss = h->side;
+    VLP_CUDA(cudaEventRecord(h->fork, s));
+    VLP_CUDA(cudaStreamWaitEvent(ss, h->fork, 0));
+
+    // 10. dP = (dY W2) * G, row-major and transposed (caller's stream)
+    if (want_l1) {
+        if (encode_bf16_2d(&tmA, h->dY.ptr, M, c.N2, vlp::BM)) return VLPROJ_ERR_CUDA;
+        p = gemm_params(h, M, c.N1, c.N2);
+        p.aux = h->G.ptr;
+        p.out = h->dP.ptr;
+        p.out_t = h->dPt.ptr;
+        p.ldt = ldt;
+        stage_begin(h, 10, s);
+        ++h->launches;
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW2t, h->tmW2th, p,
+                                                         h->num_sms, s);
+        if (rc) return rc;
+        stage_end(h, 10, s);
+        VLP_CUDA(cudaEventRecord(h->join2, s));
+    }
+
+    // 12a. A^T in the caller's column order (side stream)
+    if (a->d_W1) {
+        stage_begin(h, 12, ss);
+        ++h->launches;
+        transpose_launch(h->A.ptr, K1, M, nullptr, nullptr, M, K1, nullptr, h->At.ptr, ldt, c.C, kk,
+                         c.k_order == VLPROJ_ORDER_CHANNEL_OUTER ? 1 : 0, ss);
+        VLP_CUDA(cudaGetLastError());
+    }
+
+    // 11. dW2 = dY^T H and db2 (side stream)
+    CUtensorMap tmA2{}, tmB2{}, tmB2h{};
+    if (a->d_W2) {
+        if (encode_bf16_2d(&tmA2, h->dYt.ptr, c.N2, M, vlp::BM, ldt) ||
+            encode_b(&tmB2, &tmB2h, h->Ht.ptr, c.N1, M, pick_bn(c.N1), ldt))
+            return VLPROJ_ERR_CUDA;
+        GemmParams q = gemm_params(h, c.N2, c.N1, M);
+        q.outf = a->d_W2;
+        stage_begin(h, 11, ss);
+        ++h->launches;
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(c.N1), h->pairs, tmA2, tmB2, tmB2h, q, h->num_sms,
+                                                       ss);
+        if (rc) return rc;
+        stage_end(h, 11, ss);
+    }
+    if (a->d_b2) {
+        ++h->launches;
+        vlp::vlp_rowsum_kernel<<<(c.N2 + 7) / 8, 256, 0, ss>>>(h->dYt.ptr, ldt, c.N2, M, a->d_b2);
+        VLP_CUDA(cudaGetLastError());
+    }
+
+    // 12b. dW1 = dP^T A and db1 (side stream, after dP)
+    if (want_l1) VLP_CUDA(cudaStreamWaitEvent(ss, h->join2, 0));
+    if (a->d_W1) {
+        if (encode_bf16_2d(&tmA2, h->dPt.ptr, c.N1, M, vlp::BM, ldt) ||
+            encode_b(&tmB2, &tmB2h, h->At.ptr, K1, M, pick_bn(K1), ldt))
+            return VLPROJ_ERR_CUDA;
+        GemmParams q = gemm_params(h, c.N1, K1, M);
+        q.outf = a->d_W1;
+        ++h->launches;
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(K1), h->pairs, tmA2, tmB2, tmB2h, q, h->num_sms,
+                                                       ss);
+        if (rc) return rc;
+        stage_end(h, 12, ss);
+    }
+    if (a->d_b1) {
+        ++h->launches;
+        vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, ss>>>(h->dPt.ptr, ldt, c.N1, M, a->d_b1);
+        VLP_CUDA(cudaGetLastError());
+    }
+    VLP_CUDA(cudaEventRecord(h->join, ss));
+
+    // 13. dA = dP W1p (fp32, position-outer columns; caller's stream)
+    if (want_da) {
+        if (encode_bf16_2d(&tmA, h->dP.ptr, M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
+        p = gemm_params(h, M, K1, c.N1);
+        p.outf = h->dA.ptr;
+        stage_begin(h, 13, s);
+        ++h->launches;
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth, p,
+                                                       h->num_sms, s);
+        if (rc) return rc;
+        stage_end(h, 13, s);
+    }
+
+    // 14. LayerNorm backward, newline / separator gradients (caller's stream)
+    stage_begin(h, 14, s);
+    if (want_da) {
+        const int64_t items = M * kk;
+        const int nb = static_cast<int>(std::min<int64_t>((items + vlp::LNB_WARPS - 1) / vlp::LNB_WARPS,
+                                                          4 * static_cast<int64_t>(h->num_sms)));
+        const bool ln_sums = c.has_ln && (a->d_gamma || a->d_beta);
+        const size_t smem = c.has_ln ? static_cast<size_t>(c.C) * 2 * vlp::LNB_WARPS * 4 : 0;
+        if (ln_sums && h->part.ensure(static_cast<size_t>(nb) * 2 * c.C)) return VLPROJ_ERR_CUDA;
+        float* partial = ln_sums ? h->part.ptr : nullptr;
+        ++h->launches;
+        if (c.feat_dtype == VLPROJ_FEAT_F32) {
+            VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_ln_backward_kernel<true>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+            vlp::vlp_ln_backward_kernel<true><<<nb, 256, smem, s>>>(a->features, h->gmeta.ptr, static_cast<int>(M),
+                                                                    c.k, c.C, h->gamma, eps, c.has_ln, h->dA.ptr,
+                                                                    a->d_features, partial);
+        } else {
+            VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_ln_backward_kernel<false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+            vlp::vlp_ln_backward_kernel<false><<<nb, 256, smem, s>>>(a->features, h->gmeta.ptr, static_cast<int>(M),
+                                                                     c.k, c.C, h->gamma, eps, c.has_ln, h->dA.ptr,
+                                                                     a->d_features, partial);
+        }
+        VLP_CUDA(cudaGetLastError());
+        if (ln_sums) {
+            ++h->launches;
+            vlp::vlp_colsum_kernel<<<(2 * c.C + vlp::CS_COLS - 1) / vlp::CS_COLS, vlp::CS_COLS * vlp::CS_GROUPS, 0, s>>>(
+                partial, nb, c.C, a->d_gamma, a->d_beta);
+            VLP_CUDA(cudaGetLastError());
+        }
+    }
+    if (!c.has_ln) {
+        if (a->d_gamma) VLP_CUDA(cudaMemsetAsync(a->d_gamma, 0, static_cast<size_t>(c.C) * 4, s));
+        if (a->d_beta) VLP_CUDA(cudaMemsetAsync(a->d_beta, 0, static_cast<size_t>(c.C) * 4, s));
+    }
+    if (a->d_newline || a->d_sep) {
+        if (tiled && !pl.images.empty()) {
+            const int n_img = static_cast<int>(pl.images.size());
+            if (h->part_sp.ensure(static_cast<size_t>(n_img) * 2 * c.N2)) return VLPROJ_ERR_CUDA;
+            h->launches += 2;
+            vlp::vlp_special_grad_kernel<<<dim3((c.N2 + 255) / 256, n_img), 256, 0, s>>>(
+                h->dimages.ptr, h->pos.ptr, pl.R, static_cast<const __nv_bfloat16*>(a->d_out), n_ids, c.N2,
+                h->status + 1, h->part_sp.ptr);
+            vlp::vlp_colsum_kernel<<<(2 * c.N2 + vlp::CS_COLS - 1) / vlp::CS_COLS, vlp::CS_COLS * vlp::CS_GROUPS, 0,
+                                     s>>>(h->part_sp.ptr, n_img, c.N2, a->d_newline, a->d_sep);
+            VLP_CUDA(cudaGetLastError());
+        } else {
+            if (a->d_newline) VLP_CUDA(cudaMemsetAsync(a->d_newline, 0, static_cast<size_t>(c.N2) * 4, s));
+            if (a->d_sep) VLP_CUDA(cudaMemsetAsync(a->d_sep, 0, static_cast<size_t>(c.N2) * 4, s));
+        }
+    }
+    stage_end(h, 14, s);
+    VLP_CUDA(cudaStreamWaitEvent(s, h->join, 0));
+    h->profiled_valid = h->profiling;
+    return VLPROJ_OK;
+}

@@ -209,6 +209,19 @@ def mid_weights(wl: Workload, depth: int, seed: int = 0) -> list:
     return out
 
 
+_T_DOUT = 14
+
+
+def grad_out(wl: Workload, n_ids: int, seed: int = 0) -> np.ndarray:
+    """(n_ids, N2) bf16 bits ~N(0, 1): a loss gradient with respect to the embedding buffer."""
+    return _normal_bits(_rng(wl, _T_DOUT, 0, seed), (n_ids, wl.N2))
+
+
+def grad_out_rows(wl: Workload, n_rows: int, seed: int = 0) -> np.ndarray:
+    """(n_rows, N2) bf16 bits ~N(0, 1): the nonzero rows of a sparse loss gradient."""
+    return _normal_bits(_rng(wl, _T_DOUT, 1, seed), (n_rows, wl.N2))
+
+
 def input_ids(wl: Workload, rows_per_image: Sequence[int], seed: int = 0,
               image_token_id: int = IMAGE_TOKEN_ID) -> np.ndarray:
     """Flattened (B*S,) int64 ids: each sequence holds n_images/B images as placeholder runs.
