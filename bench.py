@@ -3,7 +3,9 @@
 
 One step = one whole pass of the bridge (placeholder index, geometry, LayerNorm,
 GEMM1 with the merge-gather prologue, GEMM2 with the scatter epilogue, newline /
-separator rows) over one batch of the chosen workload, through the C ABI.
+separator rows) over one batch of the chosen workload, through the C ABI. The line
+also carries the projector backward (vlproj_backward, every gradient) timed the same
+way on the same batch under "backward".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -19,13 +21,10 @@ only), on a bounded sample of the same workload per step.
 from __future__ import annotations
 
 import argparse
-import csv
 import hashlib
-import io
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -40,19 +39,21 @@ METRIC = "projected image tokens/s on 1 B200; % of dense BF16 tensor peak"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "moonvit"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["vision_language_projector_b200/csrc/gemm_sm100.cuh", "vision_language_projector_b200/csrc/ptx.cuh",
-                  "vision_language_projector_b200/csrc/kernels_aux.cuh", "vision_language_projector_b200/csrc/vlproj.cu"]
+CSRC = os.path.join(ROOT, "vision_language_projector_b200", "csrc")
+KERNEL_SOURCES = sorted(os.path.join("vision_language_projector_b200", "csrc", f) for f in os.listdir(CSRC)
+                        if f.endswith((".cu", ".cuh")))
 
 
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--backward-steps", type=int, default=5, help="timed vlproj_backward steps (0 = skip)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -111,41 +112,64 @@ def flops_per_token(wl) -> int:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling of one GPU during the timed region."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and throttle reasons of one GPU, polled through NVML every 5 ms on a
+    background thread for as long as the timed region lasts (read-only queries)."""
+    PERIOD_S = 0.005
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int, enabled: bool = True):
-        self.proc = None
-        self.gpu = gpu_index
+    def __init__(self, device: int, enabled: bool = True):
+        import threading
+        self.samples = []
+        self.thread = None
+        self.smax = None
         if not enabled:
             return
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            prop = torch.cuda.get_device_properties(device)
+            bus = f"{prop.pci_domain_id:08x}:{prop.pci_bus_id:02x}:{prop.pci_device_id:02x}.0"
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except pynvml.NVMLError:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device)
+            self.nvml = pynvml
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            return
+        self.stop_flag = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        n = self.nvml
+        while not self.stop_flag.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = n.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((sm, mask, pw))
+            except Exception:
+                pass
+            self.stop_flag.wait(self.PERIOD_S)
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
-        if not rows:
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        if not self.samples:
             return None
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows)}
+        n = self.nvml
+        reasons = sorted({name for _, mask, _ in self.samples for name, const in self.REASONS
+                          if mask & getattr(n, const)})
+        return {"sm_mhz": statistics.median(sm for sm, _, _ in self.samples), "sm_max_mhz": self.smax,
+                "power_w_median": statistics.median(pw for _, _, pw in self.samples), "reasons": reasons,
+                "samples": len(self.samples), "source": "NVML, 5 ms polling during the timed region"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -385,6 +409,62 @@ def main():
                "path": "vlproj_forward_ex: host features + ids in; token-embedding lookup from the resident "
                        "table; assembled rows out"}
 
+    # ---- backward: every gradient of the projector for the same batch, timed like the forward
+    bwd = None
+    if args.backward_steps > 0:
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(1000 + seed)
+        d_out = torch.randn((ids.numel(), wl.N2), device="cuda", generator=gen).to(torch.bfloat16)
+        P = int(feats.shape[0])
+        shapes = {"W1": (wl.N1, wl.K1), "b1": (wl.N1,), "W2": (wl.N2, wl.N1), "b2": (wl.N2,), "features": (P, wl.C)}
+        if wl.has_ln:
+            shapes.update(gamma=(wl.C,), beta=(wl.C,))
+        if wl.tiled:
+            shapes.update(newline=(wl.N2,), sep=(wl.N2,))
+        grads = {n: torch.empty(sh, dtype=torch.float32, device="cuda") for n, sh in shapes.items()}
+
+        def bstep():
+            proj.backward(feats, hw, crop, ids, W.IMAGE_TOKEN_ID, d_out, grads, stream=stream, n_images=wl.n_images)
+
+        for _ in range(3):
+            bstep()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        b_ms, b_stage = [], {}
+        for _ in range(args.backward_steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            bstep()
+            b.record(stream)
+            b.synchronize()
+            b_ms.append(a.elapsed_time(b))
+            for k_, v in proj.stage_ms().items():
+                if v > 0.0:
+                    b_stage.setdefault(k_, []).append(v)
+        bt = float(sum(b_ms))
+        if world > 1:
+            t = torch.tensor([bt], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            bt = float(t.item())
+        st = proj.status()
+        if st != vp.OK:
+            raise SystemExit(f"backward steps failed: {vp.strerror(st)}")
+        b_step = bt / args.backward_steps
+        b_flops = 2.0 * M * (3 * wl.K1 * wl.N1 + 2 * wl.N1 * wl.N2)
+        b_tf = b_flops / (b_step / 1000.0) / 1e12
+        b_peak = peaks.get("bf16_tflops_sustained" if bt > 2000.0 else "bf16_tflops")
+        bwd = {"ms_per_step": b_step, "tflops_per_gpu": b_tf, "peak": b_peak,
+               "frac_of_peak": b_tf / b_peak,
+               "peak_source": f"{peak_src} bf16 {'sustained' if bt > 2000.0 else 'burst'}",
+               "flops_per_step": b_flops, "steps": args.backward_steps, "gradients": sorted(shapes),
+               "stage_ms": {k_: statistics.mean(v) for k_, v in b_stage.items()},
+               "what": "vlproj_backward: GEMM1 recompute, dP, dW2, dW1, dA, LayerNorm backward, bias and "
+                       "newline/separator sums; d_out ~N(0,1) bf16 on every id"}
+        del grads, d_out
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -409,6 +489,7 @@ def main():
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "backward": bwd,
             "gpu_launches": int(launches),
             "clocks": clk,
         }

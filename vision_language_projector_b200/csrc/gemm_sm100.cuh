@@ -21,6 +21,9 @@
 //                   transposed, so H^T can be a K-major operand of the W2 gradient
 //       EPI_DGELU   dP = bf16(acc * G), row-major and transposed (dP^T)
 //       EPI_F32     acc as fp32, row-major (weight and input gradients)
+//       EPI_FOLD_F32  acc as fp32, folded back onto the patches: column p*C + c of
+//                   merged token m goes to channel c of the patch at position p of its
+//                   k x k neighbourhood (gmeta), so dA never goes to memory
 //
 // One persistent CTA per SM walks output tiles of BM x BN in banded order (see
 // tile_coords: the CTAs running together share A tiles and an L2-sized band of B).
@@ -53,6 +56,7 @@ constexpr int EPI_SCATTER = 1;
 constexpr int EPI_BWD_H = 2;
 constexpr int EPI_DGELU = 3;
 constexpr int EPI_F32 = 4;
+constexpr int EPI_FOLD_F32 = 5;
 constexpr int A_TILE = 0;               // dense row-major A, tiled TMA
 constexpr int A_IM2COL = 1;             // merge-gather by TMA im2col
 constexpr int A_CPASYNC = 2;            // merge-gather by cp.async
@@ -105,7 +109,7 @@ struct GemmParams {
     __nv_bfloat16* out_t;           // EPI_BWD_H: H^T, EPI_DGELU: dP^T, [N][ldt] bf16
     int64_t ldt;                    // row stride of out_t in elements (a multiple of 8)
     const __nv_bfloat16* aux;       // EPI_DGELU: G = GELU'(P) [M][N] bf16
-    float* outf;                    // EPI_F32: [M][N] fp32
+    float* outf;                    // EPI_F32: [M][N] fp32; EPI_FOLD_F32: [patches][C] fp32
     int group_n;                    // N-blocks per raster band (see tile_coords)
     int* err;                       // latched error word
     uint64_t wait_ns;               // bound on every wait
@@ -454,6 +458,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (row_ok && p.rowdest) d = __ldg(&p.rowdest[m]);
             row_ok = row_ok && d >= 0 && d < p.out_rows;
             __nv_bfloat16* dst_row = (row_ok && p.out) ? p.out + d * p.N : nullptr;
+            int2 fold = make_int2(0, 0);
+            if constexpr (kEpi == EPI_FOLD_F32) {
+                if (row_ok) fold = __ldg(&p.gmeta[m]);
+            }
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
@@ -462,9 +470,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(t_row + c * 32, v);
                 tmem_ld_wait();
-                if constexpr (kEpi == EPI_F32) {
-                    if (row_ok) {
-                        float4* d4 = reinterpret_cast<float4*>(p.outf + static_cast<int64_t>(m) * p.N + n0);
+                if constexpr (kEpi == EPI_F32 || kEpi == EPI_FOLD_F32) {
+                    float* dst = nullptr;
+                    if constexpr (kEpi == EPI_F32) {
+                        if (row_ok) dst = p.outf + static_cast<int64_t>(m) * p.N + n0;
+                    } else if (row_ok) {
+                        // a 32-column chunk lies inside one position: C is a multiple of 64
+                        const int pos = n0 / p.C, c0 = n0 - pos * p.C;
+                        const uint32_t wm = static_cast<uint32_t>(fold.y);
+                        if ((wm >> pos) & 1u) {
+                            const int dy = pos / p.k, dx = pos - dy * p.k;
+                            const int64_t prow = static_cast<int64_t>(fold.x) + dy * static_cast<int>(wm >> 16) + dx;
+                            dst = p.outf + prow * p.C + c0;
+                        }
+                    }
+                    if (dst) {
+                        float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
                             d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),

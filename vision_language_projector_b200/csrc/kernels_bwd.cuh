@@ -4,6 +4,8 @@
 //                      (dY and dY^T from the output gradient, A^T, transposed weights)
 //   row sums           bias gradients from the transposed gradient matrices
 //   LayerNorm backward input gradient per patch, gamma / beta partial sums per block
+//                      (without a LayerNorm the dA GEMM's epilogue writes the input
+//                      gradient itself)
 //   column sums        gamma / beta (and newline / separator) gradients from partials
 //   special-row grads  per-image newline / separator sums (2D tiling)
 // Every reduction runs in a fixed order over a fixed grid, so repeated calls give the
@@ -129,21 +131,23 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Backward of the pre-merge LayerNorm (or of the plain copy without one), one warp per
-// (merged token m, position p) item as in the merge pass; the item's patch is row
-// gmeta[m].x + dy * w + dx of the features, and items in the pad are skipped.
+// Backward of the pre-merge LayerNorm, one warp per (merged token m, position p) item as
+// in the merge pass; the item's patch is row gmeta[m].x + dy * w + dx of the features,
+// and items in the pad are skipped.
 //   dsrc = dA[m][p*C .. p*C + C)            fp32, position-outer columns
 //   xhat = (x - mean) * rstd                the forward pass's fp32 statistics
 //   dx   = rstd * (g - mean(g) - xhat * mean(g * xhat)),  g = dsrc * gamma
-// dfeat [P][C] fp32 (null = not wanted) receives dx (dsrc without LayerNorm). With
-// LayerNorm each warp adds dsrc * xhat and dsrc into its own shared-memory slice (channel
-// 8v + e kept at e * C/8 + v, so the lanes of a warp hit adjacent banks), and
-// each block writes the sum of its slices, in warp order, to partial[block][0 | 1][C].
-// Items are dealt round-robin over a fixed grid. Dynamic shared memory: 8 * 2 * C floats.
-template <bool kF32In>
-static __global__ void __launch_bounds__(256) vlp_ln_backward_kernel(const void* __restrict__ x,
+// Each lane holds its kVec 8-channel vectors of x and dsrc in registers, so both are
+// read once. dfeat [P][C] fp32 (null = not wanted) receives dx. Each warp adds
+// dsrc * xhat and dsrc into its own shared-memory slice (channel 8v + e kept at
+// e * C/8 + v, so the lanes of a warp hit adjacent banks), and each block writes the sum
+// of its slices, in warp order, to partial[block][0 | 1][C] (null = not wanted). Items
+// are dealt round-robin over a fixed grid. C <= 256 * kVec. Dynamic shared memory:
+// 8 * 2 * C floats.
+template <bool kF32In, int kVec>
+__global__ void __launch_bounds__(256) vlp_ln_backward_kernel(const void* __restrict__ x,
                                                               const int2* __restrict__ gmeta, int M, int k, int C,
-                                                              const float* __restrict__ gamma, float eps, int has_ln,
+                                                              const float* __restrict__ gamma, float eps,
                                                               const float* __restrict__ dA, float* __restrict__ dfeat,
                                                               float* __restrict__ partial) {
     extern __shared__ float lnb_acc[];
@@ -152,8 +156,7 @@ static __global__ void __launch_bounds__(256) vlp_ln_backward_kernel(const void*
     const int nvec = C / 8;
     const float invC = 1.0f / static_cast<float>(C);
     float* my = lnb_acc + warp * 2 * C;
-    if (has_ln)
-        for (int i = lane; i < 2 * C; i += 32) my[i] = 0.f;
+    for (int i = lane; i < 2 * C; i += 32) my[i] = 0.f;
     const int64_t items = static_cast<int64_t>(M) * kk;
     for (int64_t item = static_cast<int64_t>(blockIdx.x) * LNB_WARPS + warp; item < items;
          item += static_cast<int64_t>(gridDim.x) * LNB_WARPS) {
@@ -164,67 +167,67 @@ static __global__ void __launch_bounds__(256) vlp_ln_backward_kernel(const void*
         const int dy = pp / k, dx = pp - dy * k;
         const int64_t row = static_cast<int64_t>(g.x) + dy * static_cast<int>(wm >> 16) + dx;
         const float* d = dA + (static_cast<int64_t>(m) * kk + pp) * C;
-        float* out = dfeat ? dfeat + row * C : nullptr;
-        if (!has_ln) {
-            if (out)
-                for (int v = lane; v < nvec; v += 32) {
-                    reinterpret_cast<float4*>(out)[2 * v] = __ldg(reinterpret_cast<const float4*>(d) + 2 * v);
-                    reinterpret_cast<float4*>(out)[2 * v + 1] = __ldg(reinterpret_cast<const float4*>(d) + 2 * v + 1);
-                }
-            continue;
-        }
-        float f[8], dd[8];
+        float f[kVec][8], dd[kVec][8];
         float s = 0.f;
-        for (int v = lane; v < nvec; v += 32) {
-            load8_feat<kF32In>(x, row, C, v, f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s += f[e];
+        for (int i = 0; i < kVec; ++i) {
+            const int v = lane + 32 * i;
+            if (v < nvec) {
+                load8_feat<kF32In>(x, row, C, v, f[i]);
+                load8_f32(d, v, dd[i]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[i][e] = dd[i][e] = 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s += f[i][e];
         }
         const float mean = warp_sum(s) * invC;
         float q = 0.f;
-        for (int v = lane; v < nvec; v += 32) {
-            load8_feat<kF32In>(x, row, C, v, f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float t = f[e] - mean;
-                q += t * t;
+        for (int i = 0; i < kVec; ++i) {
+            if (lane + 32 * i < nvec) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float t = f[i][e] - mean;
+                    q += t * t;
+                }
             }
         }
         const float rstd = rsqrtf(warp_sum(q) * invC + eps);
         float sg = 0.f, sgx = 0.f;
-        for (int v = lane; v < nvec; v += 32) {
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) {
+            const int v = lane + 32 * i;
+            if (v >= nvec) continue;
             float gm[8];
-            load8_feat<kF32In>(x, row, C, v, f);
-            load8_f32(d, v, dd);
             load8_f32(gamma, v, gm);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float xh = (f[e] - mean) * rstd;
-                const float gg = dd[e] * gm[e];
-                sg += gg;
-                sgx += gg * xh;
-                my[e * nvec + v] += dd[e] * xh;         // channel 8v + e, lanes on adjacent banks
-                my[C + e * nvec + v] += dd[e];
+                const float xh = (f[i][e] - mean) * rstd;
+                my[e * nvec + v] += dd[i][e] * xh;
+                my[C + e * nvec + v] += dd[i][e];
+                f[i][e] = xh;                       // x is not needed again
+                dd[i][e] *= gm[e];                  // g = dsrc * gamma
+                sg += dd[i][e];
+                sgx += dd[i][e] * xh;
             }
         }
+        if (dfeat == nullptr) continue;
         const float mg = warp_sum(sg) * invC, mgx = warp_sum(sgx) * invC;
-        if (out) {
-            for (int v = lane; v < nvec; v += 32) {
-                float gm[8], r[8];
-                load8_feat<kF32In>(x, row, C, v, f);
-                load8_f32(d, v, dd);
-                load8_f32(gamma, v, gm);
+        float* out = dfeat + row * C;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float xh = (f[e] - mean) * rstd;
-                    r[e] = rstd * (dd[e] * gm[e] - mg - xh * mgx);
-                }
-                reinterpret_cast<float4*>(out)[2 * v] = make_float4(r[0], r[1], r[2], r[3]);
-                reinterpret_cast<float4*>(out)[2 * v + 1] = make_float4(r[4], r[5], r[6], r[7]);
-            }
+        for (int i = 0; i < kVec; ++i) {
+            const int v = lane + 32 * i;
+            if (v >= nvec) continue;
+            float r[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[e] = rstd * (dd[i][e] - mg - f[i][e] * mgx);
+            reinterpret_cast<float4*>(out)[2 * v] = make_float4(r[0], r[1], r[2], r[3]);
+            reinterpret_cast<float4*>(out)[2 * v + 1] = make_float4(r[4], r[5], r[6], r[7]);
         }
     }
-    if (!has_ln || partial == nullptr) return;      // uniform over the block
+    if (partial == nullptr) return;      // uniform over the block
     __syncthreads();
     for (int i = threadIdx.x; i < 2 * C; i += blockDim.x) {
         const int part = i >= C ? 1 : 0, c = i - part * C;

@@ -13,7 +13,8 @@
 //   11  dW2 GEMM                      dW2 = dY^T H, K = M
 //   12  A^T + dW1 GEMM                A^T with rows in the caller's column order, then
 //                                     dW1 = dP^T A, K = M
-//   13  dA GEMM                       dA = dP W1p [M][k*k*C] fp32
+//   13  dA GEMM                       dA = dP W1p [M][k*k*C] fp32 (without a LayerNorm
+//                                     folded straight onto the patches: d_features)
 //   14  tails                         LayerNorm backward -> d_features and gamma / beta
 //                                     partials, column sums -> dgamma, dbeta; newline /
 //                                     separator gradients (db2, db1: row sums of dY^T and
@@ -21,8 +22,9 @@
 // Every contraction runs on the tcgen05 GEMM kernel with a K-major A and B from tensor
 // maps: the weight gradients take the transposed copies (K = M contiguous), which the
 // producing epilogues and the gather kernel write directly. W2^T and W1p^T are made
-// once, on the first call. Stages 11-12 and the bias sums run on the handle's side
-// stream, forked after stage 9 and joined before the call returns.
+// once, on the first call. For batches up to about 2^28 hidden activations, stages
+// 11-12 and the bias sums run on the handle's side stream, forked after stage 9 and
+// joined before the call returns.
 #include "host.cuh"
 #include "kernels_bwd.cuh"
 
@@ -100,7 +102,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     if (!h || !a) return VLPROJ_ERR_INVALID_ARG;
     const vlproj_config& c = h->cfg;
     if (c.depth != 2) return VLPROJ_ERR_UNSUPPORTED;
-    if (c.has_ln && static_cast<size_t>(c.C) * 2 * vlp::LNB_WARPS * 4 > 227 * 1024) return VLPROJ_ERR_UNSUPPORTED;
+    if (c.has_ln && c.C > 256 * 8) return VLPROJ_ERR_UNSUPPORTED;     // LayerNorm backward keeps C in registers
     const int64_t n_ids = a->n_ids;
     if (n_ids < 0 || n_ids >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
     if (n_ids > 0 && (!a->input_ids || !a->d_out)) return VLPROJ_ERR_INVALID_ARG;
@@ -119,13 +121,15 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     const int kk = c.k * c.k;
     const int K1 = h->K1;
     const int64_t M = pl.M;          // no padding in this plan: M merged tokens
-    const int64_t ldt = round_up(std::max<int64_t>(M, 1), 8);
+    // row stride of the transposed copies: whole 128-byte lines, so every TMA box row
+    // of the weight-gradient GEMMs starts on a line
+    const int64_t ldt = round_up(std::max<int64_t>(M, 1), 64);
 
     // scratch
     const int nblocks = static_cast<int>((n_ids + vlp::SCAN_CHUNK - 1) / vlp::SCAN_CHUNK);
     if (h->counts.ensure(std::max(nblocks, 1)) || h->pos.ensure(std::max<int64_t>(pl.R, 1))) return VLPROJ_ERR_CUDA;
     const bool want_l1 = a->d_W1 || a->d_b1 || a->d_features || a->d_gamma || a->d_beta;
-    const bool want_da = a->d_features || (c.has_ln && (a->d_gamma || a->d_beta));
+    const bool want_da = a->d_features || (c.has_ln && (a->d_gamma || a->d_beta));   // the dA GEMM
     if (M > 0) {
         if (h->rowdest.ensure(M) || h->gmeta.ensure(M) || h->A.ensure(static_cast<size_t>(M) * K1) ||
             h->G.ensure(static_cast<size_t>(M) * c.N1) || h->Ht.ensure(static_cast<size_t>(c.N1) * ldt) ||
@@ -133,7 +137,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             h->dP.ensure(static_cast<size_t>(M) * c.N1) || h->dPt.ensure(static_cast<size_t>(c.N1) * ldt))
             return VLPROJ_ERR_CUDA;
         if (a->d_W1 && h->At.ensure(static_cast<size_t>(K1) * ldt)) return VLPROJ_ERR_CUDA;
-        if (want_da && h->dA.ensure(static_cast<size_t>(M) * K1)) return VLPROJ_ERR_CUDA;
+        if (want_da && c.has_ln && h->dA.ensure(static_cast<size_t>(M) * K1)) return VLPROJ_ERR_CUDA;
         rc = ensure_transposed_weights(h, s);
         if (rc) return rc;
     }
@@ -169,7 +173,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
 
     const bool want_gemm1 = want_l1 || a->d_W2;     // G feeds dP, H^T feeds dW2
     const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
-    CUtensorMap tmA{}, tmB{}, tmBh{};
+    CUtensorMap tmA{};
     GemmParams p{};
 
     if (want_gemm1) {
@@ -203,10 +207,14 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     VLP_CUDA(cudaGetLastError());
     stage_end(h, 9, s);
 
-    // The weight gradients run on the side stream, beside the dP / dA chain on the
-    // caller's stream: A^T and dW2 need only stages 7-9, dW1 waits for dP. Each persistent
-    // GEMM takes the SMs the other leaves free, which fills their last, partial waves.
-    cudaStream_t ss = h->side;
+    // Up to about 2^28 hidden activations (M * N1) the weight gradients run on the side
+    // stream, beside the dP / dA chain on the caller's stream: dW2 and A^T need only
+    // stages 7-9, dW1 waits for dP, and each persistent GEMM takes the SMs the other
+    // leaves free, which fills their partial last waves (measured 1.4-2% faster on the
+    // MoonViT, DeepSeek-ViT and VL2 batches). Larger batches run in sequence: there the
+    // two GEMM streams contend for L2 and power (measured 8% slower on 262,144 tokens).
+    const bool overlap = M * c.N1 <= (int64_t(1) << 28);
+    cudaStream_t ss = overlap ? h->side : s;
     VLP_CUDA(cudaEventRecord(h->fork, s));
     VLP_CUDA(cudaStreamWaitEvent(ss, h->fork, 0));
 
@@ -227,15 +235,6 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         VLP_CUDA(cudaEventRecord(h->join2, s));
     }
 
-    // 12a. A^T in the caller's column order (side stream)
-    if (a->d_W1) {
-        stage_begin(h, 12, ss);
-        ++h->launches;
-        transpose_launch(h->A.ptr, K1, M, nullptr, nullptr, M, K1, nullptr, h->At.ptr, ldt, c.C, kk,
-                         c.k_order == VLPROJ_ORDER_CHANNEL_OUTER ? 1 : 0, ss);
-        VLP_CUDA(cudaGetLastError());
-    }
-
     // 11. dW2 = dY^T H and db2 (side stream)
     CUtensorMap tmA2{}, tmB2{}, tmB2h{};
     if (a->d_W2) {
@@ -254,6 +253,15 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     if (a->d_b2) {
         ++h->launches;
         vlp::vlp_rowsum_kernel<<<(c.N2 + 7) / 8, 256, 0, ss>>>(h->dYt.ptr, ldt, c.N2, M, a->d_b2);
+        VLP_CUDA(cudaGetLastError());
+    }
+
+    // 12a. A^T in the caller's column order (side stream)
+    if (a->d_W1) {
+        stage_begin(h, 12, ss);
+        ++h->launches;
+        transpose_launch(h->A.ptr, K1, M, nullptr, nullptr, M, K1, nullptr, h->At.ptr, ldt, c.C, kk,
+                         c.k_order == VLPROJ_ORDER_CHANNEL_OUTER ? 1 : 0, ss);
         VLP_CUDA(cudaGetLastError());
     }
 
@@ -278,43 +286,53 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     }
     VLP_CUDA(cudaEventRecord(h->join, ss));
 
-    // 13. dA = dP W1p (fp32, position-outer columns; caller's stream)
+    // 13. dA = dP W1p (caller's stream): fp32, position-outer columns, for the LayerNorm
+    //     backward; without a LayerNorm the epilogue folds it onto the patches as the
+    //     feature gradient itself
     if (want_da) {
         if (encode_bf16_2d(&tmA, h->dP.ptr, M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
         p = gemm_params(h, M, K1, c.N1);
-        p.outf = h->dA.ptr;
         stage_begin(h, 13, s);
         ++h->launches;
-        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth, p,
-                                                       h->num_sms, s);
+        if (c.has_ln) {
+            p.outf = h->dA.ptr;
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth, p,
+                                                           h->num_sms, s);
+        } else {
+            p.outf = a->d_features;
+            p.gmeta = h->gmeta.ptr;
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_FOLD_F32>(pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth,
+                                                                p, h->num_sms, s);
+        }
         if (rc) return rc;
         stage_end(h, 13, s);
     }
 
     // 14. LayerNorm backward, newline / separator gradients (caller's stream)
     stage_begin(h, 14, s);
-    if (want_da) {
+    if (want_da && c.has_ln) {
         const int64_t items = M * kk;
         const int nb = static_cast<int>(std::min<int64_t>((items + vlp::LNB_WARPS - 1) / vlp::LNB_WARPS,
                                                           4 * static_cast<int64_t>(h->num_sms)));
-        const bool ln_sums = c.has_ln && (a->d_gamma || a->d_beta);
-        const size_t smem = c.has_ln ? static_cast<size_t>(c.C) * 2 * vlp::LNB_WARPS * 4 : 0;
+        const bool ln_sums = a->d_gamma || a->d_beta;
+        const size_t smem = static_cast<size_t>(c.C) * 2 * vlp::LNB_WARPS * 4;
         if (ln_sums && h->part.ensure(static_cast<size_t>(nb) * 2 * c.C)) return VLPROJ_ERR_CUDA;
         float* partial = ln_sums ? h->part.ptr : nullptr;
         ++h->launches;
-        if (c.feat_dtype == VLPROJ_FEAT_F32) {
-            VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_ln_backward_kernel<true>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
-            vlp::vlp_ln_backward_kernel<true><<<nb, 256, smem, s>>>(a->features, h->gmeta.ptr, static_cast<int>(M),
-                                                                    c.k, c.C, h->gamma, eps, c.has_ln, h->dA.ptr,
-                                                                    a->d_features, partial);
-        } else {
-            VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_ln_backward_kernel<false>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
-            vlp::vlp_ln_backward_kernel<false><<<nb, 256, smem, s>>>(a->features, h->gmeta.ptr, static_cast<int>(M),
-                                                                     c.k, c.C, h->gamma, eps, c.has_ln, h->dA.ptr,
-                                                                     a->d_features, partial);
-        }
+        const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
+        const int nvec = c.C / 8;
+#define VLP_LNB(F, V)                                                                                         \
+    do {                                                                                                      \
+        VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_ln_backward_kernel<F, V>,                                       \
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));  \
+        vlp::vlp_ln_backward_kernel<F, V><<<nb, 256, smem, s>>>(a->features, h->gmeta.ptr, static_cast<int>(M), \
+                                                               c.k, c.C, h->gamma, eps, h->dA.ptr,              \
+                                                               a->d_features, partial);                        \
+    } while (0)
+        if (nvec <= 64) { if (f32) VLP_LNB(true, 2); else VLP_LNB(false, 2); }
+        else if (nvec <= 160) { if (f32) VLP_LNB(true, 5); else VLP_LNB(false, 5); }
+        else { if (f32) VLP_LNB(true, 8); else VLP_LNB(false, 8); }
+#undef VLP_LNB
         VLP_CUDA(cudaGetLastError());
         if (ln_sums) {
             ++h->launches;
