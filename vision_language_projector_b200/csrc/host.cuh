@@ -309,14 +309,17 @@ inline int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int3
     return VLPROJ_OK;
 }
 
-// N-blocks per raster band: all of them while B fits comfortably in L2 (about 40 MB,
-// a margin under one die's share of the 126 MB), else as many as fit in that budget.
+// N-blocks per raster band: all of them while B fits in about half of the 126 MB L2
+// (64 MB), else the fewest bands under that budget, of equal width, so that no band is
+// a narrow remainder whose tiles share little of A.
 inline int raster_group(int N, int K, int BN) {
     const int n_tiles = (N + BN - 1) / BN;
     const int64_t per_block = static_cast<int64_t>(BN) * K * 2;
-    const int64_t budget = int64_t(40) << 20;
-    if (per_block * n_tiles <= budget) return n_tiles;
-    return static_cast<int>(std::max<int64_t>(1, budget / per_block));
+    const int64_t budget = int64_t(64) << 20;
+    const int max_group = static_cast<int>(std::max<int64_t>(1, budget / per_block));
+    if (n_tiles <= max_group) return n_tiles;
+    const int bands = (n_tiles + max_group - 1) / max_group;
+    return (n_tiles + bands - 1) / bands;
 }
 
 template <int BN, int A, int E, int CTAS>
