@@ -20,6 +20,8 @@
 //       EPI_BWD_H   P = acc + b1: G = bf16(GELU'(P)) row-major and H^T = bf16(GELU(P))
 //                   transposed, so H^T can be a K-major operand of the W2 gradient
 //       EPI_DGELU   dP = bf16(acc * G), row-major and transposed (dP^T)
+//   bf16 outputs with plain rows (GEMM1's H, the backward's G, H^T, dP, dP^T) leave the
+//   epilogue as 32 x 32 blocks through shared memory and TMA tile stores.
 //       EPI_F32     acc as fp32, row-major (weight and input gradients)
 //       EPI_FOLD_F32  acc as fp32, folded back onto the patches: column p*C + c of
 //                   merged token m goes to channel c of the patch at position p of its
@@ -67,14 +69,23 @@ constexpr int ERR_TIMEOUT = -5;
 // Shared-memory plan. kCtas = 2 runs one 256-row tile on a CTA pair: each CTA holds
 // its 128 rows of A and half of the BN rows of B per stage, so a stage is 32 KB and
 // six stages fit.
-template <int BN, int kCtas = 1>
+// Epilogues that send bf16 tiles out by TMA store stage them here: per epilogue warp two
+// 32 x 32 bf16 blocks (two chunks of one output in flight, or one chunk of an output and
+// of its transpose).
+constexpr int EPI_WARP_BYTES = 2 * 32 * 32 * 2;
+__host__ __device__ constexpr int epi_stage_bytes(int epi) {
+    return (epi == EPI_GELU || epi == EPI_BWD_H || epi == EPI_DGELU) ? 4 * EPI_WARP_BYTES : 0;
+}
+
+template <int BN, int kCtas = 1, int kEpiBytes = 0>
 struct GemmLayout {
     static constexpr int B_ROWS = BN / kCtas;
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
-    static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+    static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;
+    static constexpr int BAR_OFFSET = EPI_OFFSET + kEpiBytes;
     // full_tma[S], full_gather[S], empty[S], tmem_full[2], tmem_empty[2], drain
     static constexpr int NUM_BARS = 3 * STAGES + 5;
     static constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
@@ -105,9 +116,8 @@ struct GemmParams {
     const int32_t* rowdest;         // destination row of each m (-1 = no write), or null = row m
     int64_t out_rows;               // rows of `out` (bounds guard)
     const int* fwd_status;          // nonzero = count check failed, write nothing (null = ignore)
-    // backward epilogues
-    __nv_bfloat16* out_t;           // EPI_BWD_H: H^T, EPI_DGELU: dP^T, [N][ldt] bf16
-    int64_t ldt;                    // row stride of out_t in elements (a multiple of 8)
+    int tma_store;                  // EPI_GELU: rows are stored by TMA through tmC (identity rows)
+    // backward epilogues (outputs through tmC, and tmCt for the transposed copy)
     const __nv_bfloat16* aux;       // EPI_DGELU: G = GELU'(P) [M][N] bf16
     float* outf;                    // EPI_F32: [M][N] fp32; EPI_FOLD_F32: [patches][C] fp32
     int group_n;                    // N-blocks per raster band (see tile_coords)
@@ -145,30 +155,37 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// The warp's 32 rows (lane = row m) x 32 columns (x[j] = column n0 + j) stored
-// transposed: out_t[(n0 + j) * ldt + m]. Lanes 2i and 2i+1 trade one value per column
-// pair, so each lane writes two consecutive rows of one column as a 4-byte store and
-// every store instruction covers two 64-byte runs. `ok`: the pair's even row is in range.
-__device__ __forceinline__ void store_transposed(const float (&x)[32], __nv_bfloat16* out_t, int64_t ldt, int n0,
-                                                 int m, int lane, bool ok) {
+// The warp's 32 rows (lane = row m) x 32 columns (x[j] = column n0 + j) written
+// transposed into a 32 x 32 bf16 block in shared memory, row j = column n0 + j, element
+// m = lane. Lanes 2i and 2i+1 trade one value per column pair, so each lane writes two
+// consecutive m of one column as one 4-byte word, and the 32 words an instruction writes
+// fall in 32 different banks.
+__device__ __forceinline__ void write_transposed_block(const float (&x)[32], uint32_t* words, int lane) {
     const bool odd = (lane & 1) != 0;
-    const int64_t m_even = m & ~1;
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
         const float give = odd ? x[j] : x[j + 1];
         const float got = __shfl_xor_sync(0xffffffffu, give, 1);
-        const float lo = odd ? got : x[j];          // row m_even
-        const float hi = odd ? x[j + 1] : got;      // row m_even + 1
-        const int64_t col = n0 + j + (odd ? 1 : 0);
-        if (ok) *reinterpret_cast<uint32_t*>(out_t + col * ldt + m_even) = pack_bf16x2(lo, hi);
+        const float lo = odd ? got : x[j];          // element m_even
+        const float hi = odd ? x[j + 1] : got;      // element m_even + 1
+        words[(j + (odd ? 1 : 0)) * 16 + (lane >> 1)] = pack_bf16x2(lo, hi);
     }
+}
+
+// Row-major 32 x 32 bf16 block in shared memory: the lane's row, 16 packed words.
+__device__ __forceinline__ void write_row_block(const uint32_t (&packed)[16], uint8_t* block, int lane) {
+    uint4* r4 = reinterpret_cast<uint4*>(block + lane * 64);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        r4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
 }
 
 template <int BN, int kAMode, int kEpi, int kCtas>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     vlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmCt,
                     const GemmParams p) {
-    using L = GemmLayout<BN, kCtas>;
+    using L = GemmLayout<BN, kCtas, epi_stage_bytes(kEpi)>;
     constexpr int S = L::STAGES;
     constexpr bool kPair = kCtas == 2;
     constexpr bool kGatherThreads = kAMode == A_CPASYNC;
@@ -438,7 +455,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     } else {
         // ------------------------------------------------ epilogue (warps 4..7 of each CTA)
         const int ew = warp & 3;                      // TMEM lanes 32*ew .. 32*ew+31
-        const int row = ew * 32 + lane;
+        uint8_t* ebuf = smem + L::EPI_OFFSET + ew * EPI_WARP_BYTES;   // this warp's staging blocks
+        int ehalf = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
@@ -452,7 +470,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             got = __shfl_sync(0xffffffffu, got, 0);
             if (!got) { ok = false; break; }
             tc_fence_after();
-            const int m = (m_blk * kCtas + static_cast<int>(rank)) * BM + row;
+            const int m_row0 = (m_blk * kCtas + static_cast<int>(rank)) * BM + ew * 32;
+            const int m = m_row0 + lane;
             bool row_ok = m < p.M && status_ok;
             int64_t d = m;
             if (row_ok && p.rowdest) d = __ldg(&p.rowdest[m]);
@@ -522,13 +541,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                             x[j + 1] = __uint_as_float(packed[j / 2] & 0xFFFF0000u);
                         }
                     }
-                    if (row_ok) {
-                        uint4* d4 = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(m) * p.N + n0);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                    // both copies leave through shared memory and TMA stores (rows and
+                    // columns past the tensors are not written)
+                    if (lane == 0) bulk_wait_read<0>();      // the previous chunk's stores have read both blocks
+                    __syncwarp();
+                    write_row_block(packed, ebuf, lane);
+                    write_transposed_block(x, reinterpret_cast<uint32_t*>(ebuf + EPI_WARP_BYTES / 2), lane);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && m_row0 < p.M) {        // a block wholly past M is not stored
+                        tma_store_2d(&tmC, ebuf, n0, m_row0);
+                        tma_store_2d(&tmCt, ebuf + EPI_WARP_BYTES / 2, m_row0, n0);
+                        bulk_commit_group();
                     }
-                    store_transposed(x, p.out_t, p.ldt, n0, m, lane, (m & ~1) < p.M);
                 } else {
                     const float bl = __ldg(&p.bias[n0 + lane]);
                     uint32_t packed[16];
@@ -542,7 +567,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         }
                         packed[j / 2] = pack_bf16x2(x0, x1);
                     }
-                    if (row_ok) {
+                    if (kEpi == EPI_GELU && p.tma_store) {
+                        // rows leave through a shared-memory block and one TMA store (full
+                        // lines, instead of 32 rows touched per store instruction)
+                        uint8_t* blk = ebuf + ehalf * (EPI_WARP_BYTES / 2);
+                        if (lane == 0) bulk_wait_read<1>();  // the store from this block two chunks ago is done
+                        __syncwarp();
+                        write_row_block(packed, blk, lane);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0 && m_row0 < p.M) {
+                            tma_store_2d(&tmC, blk, n0, m_row0);
+                            bulk_commit_group();
+                        }
+                        ehalf ^= 1;
+                    } else if (row_ok) {
                         uint4* d4 = reinterpret_cast<uint4*>(dst_row + n0);
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
@@ -561,6 +600,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (!ok) {
             *abort_flag = 1;
             latch_error(p.err, ERR_TIMEOUT);
+        }
+        if constexpr (epi_stage_bytes(kEpi) > 0) {
+            if (lane == 0) bulk_wait_all();          // every TMA store of this warp has landed
+            __syncwarp();
         }
     }
 

@@ -76,6 +76,22 @@ inline int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uin
     return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
 }
 
+// Output map of a bf16 matrix [rows][cols] with row stride ld elements (0 = cols, a
+// multiple of 8) for the TMA-store epilogues: 32 x 32 boxes, no swizzle; boxes reaching
+// past the matrix are clipped.
+inline int encode_bf16_store(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld = 0) {
+    auto fn = driver().tiled;
+    if (!fn) return VLPROJ_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {(ld ? ld : cols) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
 // im2col map of n views of one (h, w) grid of C-channel bf16 patches, packed back to
 // back from `base`: the k x k, stride-k window walk of the merge. Base positions run
 // over 0, k, ..., k*(w'-1) (lower corner 0, upper corner k*w' - w - (k-1), the
@@ -323,8 +339,9 @@ inline int raster_group(int N, int K, int BN) {
 }
 
 template <int BN, int A, int E, int CTAS>
-int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, int num_sms, cudaStream_t s) {
-    using L = GemmLayout<BN, CTAS>;
+int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tct,
+                GemmParams p, int num_sms, cudaStream_t s) {
+    using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E)>;
     auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
     if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN);
     VLP_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC));
@@ -356,20 +373,27 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, int 
     cfg.gridDim = dim3(static_cast<unsigned>(units * CTAS));
     cfg.attrs = CTAS > 1 ? attr : nullptr;
     cfg.numAttrs = CTAS > 1 ? 1 : 0;
-    VLP_CUDA(cudaLaunchKernelEx(&cfg, kernel, ta, tb, p));
+    VLP_CUDA(cudaLaunchKernelEx(&cfg, kernel, ta, tb, tc, tct, p));
     return VLPROJ_OK;
 }
 
 // Tile shape: 256 x 256 tiles on CTA pairs when N allows and the A operand comes by
-// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise.
+// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise. tc / tct: output maps
+// of the TMA-store epilogues (unused by the others).
+inline const CUtensorMap& no_map() {
+    static const CUtensorMap zero{};
+    return zero;
+}
+
 template <int A, int E>
 int launch_gemm_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb_half,
-                   const GemmParams& p, int num_sms, cudaStream_t s) {
+                   const GemmParams& p, int num_sms, cudaStream_t s, const CUtensorMap& tc = no_map(),
+                   const CUtensorMap& tct = no_map()) {
     if constexpr (A != vlp::A_CPASYNC) {
-        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, p, num_sms, s);
+        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tct, p, num_sms, s);
     }
-    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, p, num_sms, s);
-    return launch_gemm<128, A, E, 1>(ta, tb, p, num_sms, s);
+    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tct, p, num_sms, s);
+    return launch_gemm<128, A, E, 1>(ta, tb, tc, tct, p, num_sms, s);
 }
 
 inline int pick_bn(int N) { return N >= 256 ? 256 : 128; }

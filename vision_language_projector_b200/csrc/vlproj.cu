@@ -81,6 +81,11 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     p.out = hidden;
     p.rowdest = dest_mode == vlp::DEST_COMPACT ? h->rowdest.ptr : nullptr;
     p.out_rows = hidden_rows;
+    // GEMM row m is hidden row m unless rows are remapped: then rows leave by TMA store
+    CUtensorMap tmC{};
+    p.tma_store = p.rowdest == nullptr ? 1 : 0;
+    if (p.tma_store && encode_bf16_store(&tmC, hidden, static_cast<uint64_t>(hidden_rows), c.N1))
+        return VLPROJ_ERR_CUDA;
     p.fwd_status = nullptr;
     p.err = h->status;
     p.wait_ns = h->wait_ns;
@@ -127,16 +132,16 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     int rc;
     if (pl.merged_ln)
         rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                        h->num_sms, s);
+                                                        h->num_sms, s, tmC);
     else if (pl.box5)
         rc = launch_gemm_bn<vlp::A_BOX5, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                        h->num_sms, s);
+                                                        h->num_sms, s, tmC);
     else if (im2col)
         rc = launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                          h->num_sms, s);
+                                                          h->num_sms, s, tmC);
     else
         rc = launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(pick_bn(c.N1), false, tmA, h->tmW1, h->tmW1h, p,
-                                                           h->num_sms, s);
+                                                           h->num_sms, s, tmC);
     if (rc) return rc;
     stage_end(h, 3, s);
     return VLPROJ_OK;
@@ -521,9 +526,12 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
         q.out_rows = pl.M;
         q.err = h->status;
         q.wait_ns = h->wait_ns;
+        CUtensorMap tout{};
+        q.tma_store = 1;
+        if (encode_bf16_store(&tout, dst.ptr, pl.M, c.N1)) return VLPROJ_ERR_CUDA;
         ++h->launches;
         rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tin, h->tmWm[layer],
-                                                        h->tmWmh[layer], q, h->num_sms, s);
+                                                        h->tmWmh[layer], q, h->num_sms, s, tout);
         if (rc) return rc;
         last_in_h2 = !last_in_h2;
     }

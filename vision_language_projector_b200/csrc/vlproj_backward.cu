@@ -188,13 +188,13 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         if (encode_bf16_2d(&tmA, h->A.ptr, M, K1, vlp::BM)) return VLPROJ_ERR_CUDA;
         p = gemm_params(h, M, c.N1, K1);
         p.bias = h->b1;
-        p.out = h->G.ptr;
-        p.out_t = h->Ht.ptr;
-        p.ldt = ldt;
+        CUtensorMap tmG{}, tmHt{};
+        if (encode_bf16_store(&tmG, h->G.ptr, M, c.N1) || encode_bf16_store(&tmHt, h->Ht.ptr, c.N1, M, ldt))
+            return VLPROJ_ERR_CUDA;
         stage_begin(h, 8, s);
         ++h->launches;
         rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                         h->num_sms, s);
+                                                         h->num_sms, s, tmG, tmHt);
         if (rc) return rc;
         stage_end(h, 8, s);
     }
@@ -223,13 +223,13 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         if (encode_bf16_2d(&tmA, h->dY.ptr, M, c.N2, vlp::BM)) return VLPROJ_ERR_CUDA;
         p = gemm_params(h, M, c.N1, c.N2);
         p.aux = h->G.ptr;
-        p.out = h->dP.ptr;
-        p.out_t = h->dPt.ptr;
-        p.ldt = ldt;
+        CUtensorMap tmP{}, tmPt{};
+        if (encode_bf16_store(&tmP, h->dP.ptr, M, c.N1) || encode_bf16_store(&tmPt, h->dPt.ptr, c.N1, M, ldt))
+            return VLPROJ_ERR_CUDA;
         stage_begin(h, 10, s);
         ++h->launches;
         rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW2t, h->tmW2th, p,
-                                                         h->num_sms, s);
+                                                         h->num_sms, s, tmP, tmPt);
         if (rc) return rc;
         stage_end(h, 10, s);
         VLP_CUDA(cudaEventRecord(h->join2, s));
