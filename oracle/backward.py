@@ -11,8 +11,10 @@ input features, by the chain rule through the forward steps of `projector`:
     rows of an image at its placeholders  <- assembly of per-view rows (+ newline, sep)
     y = h W2^T + b2,  h = bf16(GELU(p)),  p = a W1^T + b1,  a = unshuffle(bf16(LN(x)))
 
-Reading: the bf16 rounding points (a and h) pass gradients through unchanged
-(straight-through), as mixed-precision training treats them. Only depth-2 MLPs.
+Reading: the bf16 rounding points (a and every hidden activation) pass gradients
+through unchanged (straight-through), as mixed-precision training treats them. With
+depth > 2 ("port DeepSeek-VL2", Projector step 3) the middle Linear(N1 -> N1) layers'
+gradients come back under "mid", one [dW, db] pair per layer, in order.
 """
 from __future__ import annotations
 
@@ -80,7 +82,21 @@ def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[n
         g["newline"] = np.zeros(W2.shape[0])
         g["sep"] = np.zeros(W2.shape[0])
 
-    mag = {key: np.zeros_like(v) for key, v in g.items()} if magnitudes else None
+    mids = [(np.asarray(Wm, np.float64), np.asarray(bm, np.float64)) for Wm, bm in (params.get("mid") or ())]
+    layers = [(W1, b1)] + mids + [(W2, b2)]
+    g["mid"] = [[np.zeros_like(Wm), np.zeros_like(bm)] for Wm, bm in mids]
+    mag = {key: (np.zeros_like(v) if key != "mid" else [[np.zeros_like(a), np.zeros_like(b)] for a, b in v])
+           for key, v in g.items()} if magnitudes else None
+
+    def acc(store, li, which, value):
+        """Add to layer li's weight (which = 0) or bias (which = 1) gradient."""
+        if li == 0:
+            store[("W1", "b1")[which]] += value
+        elif li == len(layers) - 1:
+            store[("W2", "b2")[which]] += value
+        else:
+            store["mid"][li - 1][which] += value
+
     pos = O.placeholder_positions(ids, image_token_id)
     offs = np.concatenate([[0], np.cumsum(grid_hw[:, 0].astype(np.int64) * grid_hw[:, 1])])
     if spatial_crop is None:
@@ -126,16 +142,37 @@ def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[n
             dy = d_rows[tok_rows[vi * hp * wp:(vi + 1) * hp * wp]]
             sel = np.flatnonzero(np.any(dy != 0, axis=1)) if skip_zero_rows else np.arange(hp * wp)
             a, dy = a[sel], dy[sel]
-            p = a @ W1.T + b1
-            hid = O.gelu(p)
-            if quantise:
-                hid = O.round_bf16(hid)
-            # gradients
-            g["b2"] += dy.sum(axis=0)
-            g["W2"] += dy.T @ hid
-            dp = (dy @ W2) * gelu_grad(p)
-            g["b1"] += dp.sum(axis=0)
-            g["W1"] += dp.T @ a
+            # forward through Linear -> GELU -> [Linear -> GELU] x len(mids) -> Linear,
+            # keeping each layer's input and pre-activation
+            xs, ps = [a], []
+            for W, b in layers[:-1]:
+                p = xs[-1] @ W.T + b
+                hid = O.gelu(p)
+                ps.append(p)
+                xs.append(O.round_bf16(hid) if quantise else hid)
+            # backward, top layer first: dW_l = dP_l^T x_l, db_l = sum dP_l,
+            # dP_(l-1) = (dP_l W_l) * GELU'(P_(l-1)); the first layer's input gradient is dA
+            dp = dy
+            m_dp = np.abs(dy)
+            for li in range(len(layers) - 1, -1, -1):
+                W = layers[li][0]
+                acc(g, li, 0, dp.T @ xs[li])
+                acc(g, li, 1, dp.sum(axis=0))
+                if magnitudes:
+                    acc(mag, li, 0, m_dp.T @ np.abs(xs[li]))
+                    acc(mag, li, 1, m_dp.sum(axis=0))
+                if li == 0:
+                    break
+                gp_ = gelu_grad(ps[li - 1])
+                nxt = (dp @ W) * gp_
+                if magnitudes:
+                    if li == len(layers) - 1:
+                        # dY is exact: |dP| plus its dot product's room for fp32 rounding
+                        m_dp = np.abs(nxt) + 2.0 ** -16 * (np.abs(dp) @ np.abs(W)) * np.abs(gp_)
+                    else:
+                        # dP above was rounded: its error reaches here through the whole sum
+                        m_dp = np.abs(nxt) + (m_dp @ np.abs(W)) * np.abs(gp_)
+                dp = nxt
             da = np.zeros((hp * wp, W1.shape[1]))
             da[sel] = dp @ W1
             dsrc = O.fold(da, hp, wp, k, C)[:h0, :w0].reshape(h0 * w0, C)
@@ -147,13 +184,6 @@ def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[n
                 dx = dsrc
             g["features"][offs[v]:offs[v + 1]] = dx
             if magnitudes:
-                # |dP| plus the absolute sum of its dot product, scaled far below bf16
-                # precision: a cancelling dY . W2 still gets the room of its fp32 rounding
-                m_dp = np.abs(dp) + 2.0 ** -16 * (np.abs(dy) @ np.abs(W2)) * np.abs(gelu_grad(p))
-                mag["b2"] += np.abs(dy).sum(axis=0)
-                mag["W2"] += np.abs(dy).T @ np.abs(hid)
-                mag["b1"] += m_dp.sum(axis=0)
-                mag["W1"] += m_dp.T @ np.abs(a)
                 m_da = np.zeros((hp * wp, W1.shape[1]))
                 m_da[sel] = m_dp @ np.abs(W1)
                 m_src = O.fold(m_da, hp, wp, k, C)[:h0, :w0].reshape(h0 * w0, C)

@@ -17,7 +17,7 @@ from oracle import projector as O
 IMG = 7
 
 
-def _case(seed, grid_hw, crop, k, C, N1, N2, has_ln, n_text=9):
+def _case(seed, grid_hw, crop, k, C, N1, N2, has_ln, n_text=9, depth=2):
     rng = np.random.default_rng(seed)
     grid_hw = np.asarray(grid_hw, np.int32)
     P = int((grid_hw[:, 0] * grid_hw[:, 1]).sum())
@@ -30,7 +30,7 @@ def _case(seed, grid_hw, crop, k, C, N1, N2, has_ln, n_text=9):
         "beta": rng.normal(0.0, 0.2, C) if has_ln else None,
         "newline": rng.normal(0.0, 1.0, N2) if crop is not None else None,
         "sep": rng.normal(0.0, 1.0, N2) if crop is not None else None,
-        "mid": [],
+        "mid": [(rng.normal(0.0, 0.3, (N1, N1)), rng.normal(0.0, 0.3, N1)) for _ in range(depth - 2)],
     }
     rows = sum(O.image_rows(grid_hw, k, crop))
     ids = rng.integers(IMG + 1, IMG + 50, rows + n_text)      # text ids never equal the placeholder
@@ -65,7 +65,10 @@ def _grads(c, quantise=False, gvp="head"):
 
 
 def _fd(c, name, eps=1e-6, quantise=False, gvp="head"):
-    """Central finite difference of the loss in every entry of parameter `name`."""
+    """Central finite difference of the loss in every entry of parameter `name`
+    (("mid", i, 0 | 1) names a middle layer's weight or bias)."""
+    if isinstance(name, tuple):
+        return _fd_mid(c, name[1], name[2], eps)
     if name == "features":
         base = c["features"]
     else:
@@ -82,6 +85,23 @@ def _fd(c, name, eps=1e-6, quantise=False, gvp="head"):
                 p = dict(c["params"])
                 p[name] = t
                 vals.append(_loss(c, params=p, quantise=quantise, gvp=gvp))
+        g[idx] = (vals[0] - vals[1]) / (2 * eps)
+    return g
+
+
+def _fd_mid(c, i, which, eps):
+    base = c["params"]["mid"][i][which]
+    g = np.zeros_like(base)
+    for idx in np.ndindex(base.shape):
+        vals = []
+        for sgn in (+1.0, -1.0):
+            t = base.copy()
+            t[idx] += sgn * eps
+            mids = [list(m) for m in c["params"]["mid"]]
+            mids[i][which] = t
+            p = dict(c["params"])
+            p["mid"] = [tuple(m) for m in mids]
+            vals.append(_loss(c, params=p))
         g[idx] = (vals[0] - vals[1]) / (2 * eps)
     return g
 
@@ -115,6 +135,30 @@ def test_backward_matches_finite_differences(name):
         fd = _fd(c, key)
         scale = max(1.0, float(np.abs(fd).max()))
         np.testing.assert_allclose(g[key], fd, rtol=0, atol=2e-6 * scale, err_msg=f"{name}: d{key}")
+
+
+@pytest.mark.parametrize("name,depth", [("untiled_ln_ragged", 3), ("tiled_2x1", 4), ("untiled_k3_ln", 3)])
+def test_deeper_mlp_backward_matches_finite_differences(name, depth):
+    c = _case(**CASES[name], depth=depth)
+    g = _grads(c)
+    assert len(g["mid"]) == depth - 2
+    keys = _names(c) + [("mid", i, w) for i in range(depth - 2) for w in (0, 1)]
+    for key in keys:
+        fd = _fd(c, key)
+        got = g["mid"][key[1]][key[2]] if isinstance(key, tuple) else g[key]
+        np.testing.assert_allclose(got, fd, rtol=0, atol=2e-6 * max(1.0, float(np.abs(fd).max())),
+                                   err_msg=f"{name} depth {depth}: d{key}")
+
+
+def test_deeper_mlp_magnitudes_bound_the_gradients():
+    c = _case(**CASES["tiled_2x1"], depth=4)
+    g = B.backward(c["features"], c["grid_hw"], c["spatial_crop"], c["k"], c["params"], c["ids"], IMG, c["d_out"],
+                   1e-5, feat_is_bf16_bits=False, quantise=True, magnitudes=True)
+    for key in _names(c):
+        assert np.all(g["mag"][key] >= np.abs(g[key]) * (1 - 1e-12)), key
+    for i in range(2):
+        for w in (0, 1):
+            assert np.all(g["mag"]["mid"][i][w] >= np.abs(g["mid"][i][w]) * (1 - 1e-12))
 
 
 def test_backward_tail_global_view_matches_finite_differences():
