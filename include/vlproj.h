@@ -180,9 +180,13 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
  *   dA     = dP W1, folded back through the space-to-depth onto the patches, then
  *            through the LayerNorm: dgamma, dbeta and d_features
  *   dnewline / dsep = sums of d_out over the newline / separator rows.
- * The bf16 rounding points of the forward (A and H) pass gradients unchanged; H and A
- * are the forward's bf16 values, dP is rounded to bf16 once (fp32 accumulation
- * throughout). Only depth-2 MLPs (VLPROJ_ERR_UNSUPPORTED otherwise).
+ * With depth > 2 ("port DeepSeek-VL2", Projector step 3) the chain runs through the
+ * middle GELU + Linear(N1 -> N1) layers the same way: dW_mid[i] = dP_(i+2)^T H_(i+1),
+ * db_mid[i] = sum_m dP_(i+2)[m], dP_(i+1) = (dP_(i+2) W_mid[i]) * GELU'(P_(i+1)), where
+ * layer 1 is the first Linear and layer `depth` the last.
+ * The bf16 rounding points of the forward (A and every hidden activation) pass
+ * gradients unchanged; A and the hidden activations are the forward's bf16 values,
+ * each dP is rounded to bf16 once (fp32 accumulation throughout).
  *
  *   features, grid_hw, spatial_crop, n_images, input_ids, n_ids, image_token_id:
  *                 as for vlproj_forward (the same batch the loss was computed on).
@@ -194,8 +198,11 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
  *                   d_W1 [N1][k*k*C] (columns in the config's k_order), d_b1 [N1],
  *                   d_W2 [N2][N1], d_b2 [N2], d_gamma [C], d_beta [C] (LayerNorm only),
  *                   d_newline [N2], d_sep [N2] (2D tiling only), d_features [P][C].
- * Scratch: about 2 * M * (2*N1 + N2 + k*k*C) bf16 plus M*k*k*C fp32 bytes (M merged
- * tokens), kept in the handle between calls. Errors as for vlproj_forward; when the
+ *   d_W_mid, d_b_mid  depth > 2: HOST arrays of depth - 2 DEVICE fp32 pointers
+ *                 (d_W_mid[i] [N1][N1], d_b_mid[i] [N1]), or NULL; an entry may be NULL.
+ *                 Ignored for depth 2.
+ * Scratch: about 2 * M * (2*N1*(depth - 1) + N1*(depth - 2) + 2*N1 + 2*N2 + 2*k*k*C)
+ * bytes, plus M*k*k*C fp32 with a LayerNorm (M merged tokens), kept in the handle. Errors as for vlproj_forward; when the
  * placeholder count check fails every gradient is written as zero and
  * VLPROJ_ERR_TOKEN_COUNT is latched. */
 typedef struct vlproj_backward_args {
@@ -216,6 +223,8 @@ typedef struct vlproj_backward_args {
     float*         d_newline;
     float*         d_sep;
     float*         d_features;
+    float* const*  d_W_mid;
+    float* const*  d_b_mid;
 } vlproj_backward_args;
 int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* args, void* stream);
 

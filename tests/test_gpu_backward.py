@@ -192,19 +192,80 @@ def test_backward_without_images_zeroes_outputs():
         assert not bool(t.any()), n
 
 
-def test_backward_rejects_deeper_mlp_and_bad_alignment():
+def test_backward_rejects_bad_alignment():
     wl = SMALL["tiny"]()
-    case = make_case(wl, depth=3)
+    case = make_case(wl)
     proj = make_projector(case)
     dev = DeviceInputs(case)
     _, d_dev, _ = dev_dout(case)
-    rc, _ = run_backward(case, proj, dev, d_dev, ["b2"], check=False)
-    assert rc == vp.ERR_UNSUPPORTED
-    case2 = make_case(wl)
-    proj2 = make_projector(case2)
     g = torch.zeros(wl.N2 + 1, device="cuda")
-    rc = proj2.backward(dev.feats, case2.hw, None, dev.ids, W.IMAGE_TOKEN_ID, d_dev, {"b2": g[1:]}, check=False)
+    rc = proj.backward(dev.feats, case.hw, None, dev.ids, W.IMAGE_TOKEN_ID, d_dev, {"b2": g[1:]}, check=False)
     assert rc == vp.ERR_INVALID_ARG
+
+
+def run_backward_mid(case, proj, dev, d_out, depth, want=("W1", "b1", "W2", "b2", "features"), mid=True):
+    """Like run_backward, plus the middle layers' gradients (lists under "W_mid" / "b_mid")."""
+    shapes = grad_shapes(case)
+    wl = case.wl
+    grads = {n: torch.full(shapes[n], float("nan"), dtype=torch.float32, device="cuda") for n in want if n in shapes}
+    if mid:
+        grads["W_mid"] = [torch.full((wl.N1, wl.N1), float("nan"), device="cuda") for _ in range(depth - 2)]
+        grads["b_mid"] = [torch.full((wl.N1,), float("nan"), device="cuda") for _ in range(depth - 2)]
+    proj.backward(dev.feats, case.hw, case.crop, dev.ids, W.IMAGE_TOKEN_ID, d_out, grads, n_images=wl.n_images)
+    torch.cuda.synchronize()
+    out = {n: t.double().cpu().numpy() for n, t in grads.items() if n not in ("W_mid", "b_mid")}
+    if mid:
+        out["mid"] = [[w.double().cpu().numpy(), b.double().cpu().numpy()]
+                      for w, b in zip(grads["W_mid"], grads["b_mid"])]
+    return out
+
+
+def assert_frobenius_close(got, want, label, tol=1e-2):
+    num = float(np.linalg.norm(got - want))
+    den = float(np.linalg.norm(want))
+    assert num <= tol * den + 1e-30, f"{label}: relative Frobenius error {num / max(den, 1e-30):.2e}"
+
+
+@pytest.mark.parametrize("name,depth", [("ragged_ln_bf16", 3), ("tiled_2x1", 4)])
+def test_backward_deeper_mlp_matches_oracle(name, depth):
+    """depth > 2: every gradient, the middle layers' included, within the elementwise
+    magnitude bound (which below the top layer carries the rounded dP of the layer
+    above through the whole sum) and within 1 % relative Frobenius error."""
+    wl = SMALL[name]()
+    case = make_case(wl, GRIDS[name], depth=depth)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    _, d_dev, d_f64 = dev_dout(case)
+    want_names = tuple(grad_shapes(case))
+    got = run_backward_mid(case, proj, dev, d_dev, depth, want_names)
+    assert proj.status() == vp.OK
+    want = oracle_grads(case, d_f64)
+    flat_got = {n: v for n, v in got.items() if n != "mid"}
+    assert_grads_close(flat_got, want, f"{name} depth {depth}")
+    for n, v in flat_got.items():
+        assert_frobenius_close(v, want[n], f"d{n}")
+    for i, (gw, gb) in enumerate(got["mid"]):
+        for which, gv in ((0, gw), (1, gb)):
+            wv, mag = want["mid"][i][which], want["mag"]["mid"][i][which]
+            assert np.isfinite(gv).all()
+            assert np.all(np.abs(gv - wv) <= EPS_DP * mag), f"mid {i} {which}"
+            assert_frobenius_close(gv, wv, f"mid {i} {'W' if which == 0 else 'b'}")
+
+
+def test_backward_deeper_mlp_partial_chain():
+    """Asking only for a middle layer's gradients stops the dP chain there; the values
+    equal those of the full run."""
+    wl = SMALL["ragged_ln_bf16"]()
+    case = make_case(wl, GRIDS["ragged_ln_bf16"], depth=4)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    _, d_dev, _ = dev_dout(case)
+    full = run_backward_mid(case, proj, dev, d_dev, 4, tuple(grad_shapes(case)))
+    part = run_backward_mid(case, proj, dev, d_dev, 4, ("W2",))
+    np.testing.assert_array_equal(part["W2"], full["W2"])
+    for i in range(2):
+        for which in (0, 1):
+            np.testing.assert_array_equal(part["mid"][i][which], full["mid"][i][which])
 
 
 @pytest.mark.parametrize("name", ["moonvit", "vl2", "dsvit"])

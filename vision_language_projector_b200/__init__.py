@@ -60,7 +60,8 @@ class BackwardArgs(ctypes.Structure):
         ("n_images", ctypes.c_int32), ("input_ids", ctypes.c_void_p), ("n_ids", ctypes.c_int64),
         ("image_token_id", ctypes.c_int64), ("d_out", ctypes.c_void_p),
     ] + [("d_" + n, ctypes.c_void_p) for n in ("W1", "b1", "W2", "b2", "gamma", "beta", "newline", "sep",
-                                                  "features")]
+                                                  "features")] + [("d_W_mid", ctypes.c_void_p),
+                                                                  ("d_b_mid", ctypes.c_void_p)]
 
 
 class Config(ctypes.Structure):
@@ -274,18 +275,25 @@ class Projector:
     def backward(self, features, grid_hw, spatial_crop, input_ids, image_token_id: int, d_out, grads: dict,
                  stream=None, n_images: Optional[int] = None, check: bool = True) -> int:
         """vlproj_backward: fp32 gradients into the tensors of ``grads`` (keys from
-        GRAD_NAMES; a missing key is not computed) for the loss gradient ``d_out``
+        GRAD_NAMES, plus "W_mid" / "b_mid": lists of depth - 2 tensors or None for the
+        middle layers; a missing key is not computed) for the loss gradient ``d_out``
         ((n_ids, N2) bf16) of the batch given by the other arguments."""
-        unknown = set(grads) - set(GRAD_NAMES)
+        unknown = set(grads) - set(GRAD_NAMES) - {"W_mid", "b_mid"}
         if unknown:
             raise ValueError(f"unknown gradient names {sorted(unknown)}")
+        mids = {}
+        for key in ("W_mid", "b_mid"):
+            if grads.get(key) is not None:
+                arr = (ctypes.c_void_p * len(grads[key]))(*[_ptr(t) for t in grads[key]])
+                mids[key] = arr
         g = _host_i32(grid_hw)
         c = _host_i32(spatial_crop)
         if n_images is None:
             n_images = len(c) if c is not None else (0 if g is None else len(g))
         a = BackwardArgs(_ptr(features), _ptr(g), _ptr(c), n_images, _ptr(input_ids),
                          0 if input_ids is None else int(input_ids.numel()), int(image_token_id), _ptr(d_out),
-                         *[_ptr(grads.get(n)) for n in GRAD_NAMES])
+                         *[_ptr(grads.get(n)) for n in GRAD_NAMES],
+                         *[ctypes.cast(mids[k], ctypes.c_void_p) if k in mids else None for k in ("W_mid", "b_mid")])
         rc = _lib.vlproj_backward(self._h, ctypes.byref(a), _stream_ptr(stream))
         if check and rc != OK:
             raise VlprojError(rc, "vlproj_backward")

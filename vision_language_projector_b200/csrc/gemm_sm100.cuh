@@ -69,13 +69,14 @@ constexpr int ERR_TIMEOUT = -5;
 // Shared-memory plan. kCtas = 2 runs one 256-row tile on a CTA pair: each CTA holds
 // its 128 rows of A and half of the BN rows of B per stage, so a stage is 32 KB and
 // six stages fit.
-// Epilogues that send bf16 tiles out by TMA store stage them here: per epilogue warp two
-// 32 x 32 bf16 blocks (two chunks of one output in flight, or one chunk of an output and
-// of its transpose).
-constexpr int EPI_WARP_BYTES = 2 * 32 * 32 * 2;
-__host__ __device__ constexpr int epi_stage_bytes(int epi) {
-    return (epi == EPI_GELU || epi == EPI_BWD_H || epi == EPI_DGELU) ? 4 * EPI_WARP_BYTES : 0;
+// Epilogues that send bf16 tiles out by TMA store stage them here, per epilogue warp in
+// 32 x 32 bf16 blocks: GELU two (two chunks in flight), DGELU two (a chunk of dP and of
+// dP^T), BWD_H three (G, H^T and, for a following layer, H).
+constexpr int EPI_BLOCK_BYTES = 32 * 32 * 2;
+__host__ __device__ constexpr int epi_blocks(int epi) {
+    return epi == EPI_BWD_H ? 3 : (epi == EPI_GELU || epi == EPI_DGELU) ? 2 : 0;
 }
+__host__ __device__ constexpr int epi_stage_bytes(int epi) { return 4 * epi_blocks(epi) * EPI_BLOCK_BYTES; }
 
 template <int BN, int kCtas = 1, int kEpiBytes = 0>
 struct GemmLayout {
@@ -117,6 +118,7 @@ struct GemmParams {
     int64_t out_rows;               // rows of `out` (bounds guard)
     const int* fwd_status;          // nonzero = count check failed, write nothing (null = ignore)
     int tma_store;                  // EPI_GELU: rows are stored by TMA through tmC (identity rows)
+    int store_h;                    // EPI_BWD_H: also store H row-major through tmC2
     // backward epilogues (outputs through tmC, and tmCt for the transposed copy)
     const __nv_bfloat16* aux;       // EPI_DGELU: G = GELU'(P) [M][N] bf16
     float* outf;                    // EPI_F32: [M][N] fp32; EPI_FOLD_F32: [patches][C] fp32
@@ -184,7 +186,7 @@ template <int BN, int kAMode, int kEpi, int kCtas>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     vlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmCt,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmC2, const GemmParams p) {
     using L = GemmLayout<BN, kCtas, epi_stage_bytes(kEpi)>;
     constexpr int S = L::STAGES;
     constexpr bool kPair = kCtas == 2;
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     } else {
         // ------------------------------------------------ epilogue (warps 4..7 of each CTA)
         const int ew = warp & 3;                      // TMEM lanes 32*ew .. 32*ew+31
-        uint8_t* ebuf = smem + L::EPI_OFFSET + ew * EPI_WARP_BYTES;   // this warp's staging blocks
+        uint8_t* ebuf = smem + L::EPI_OFFSET + ew * epi_blocks(kEpi) * EPI_BLOCK_BYTES;   // this warp's blocks
         int ehalf = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -543,15 +545,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                     // both copies leave through shared memory and TMA stores (rows and
                     // columns past the tensors are not written)
-                    if (lane == 0) bulk_wait_read<0>();      // the previous chunk's stores have read both blocks
+                    if (lane == 0) bulk_wait_read<0>();      // the previous chunk's stores have read the blocks
                     __syncwarp();
                     write_row_block(packed, ebuf, lane);
-                    write_transposed_block(x, reinterpret_cast<uint32_t*>(ebuf + EPI_WARP_BYTES / 2), lane);
+                    write_transposed_block(x, reinterpret_cast<uint32_t*>(ebuf + EPI_BLOCK_BYTES), lane);
+                    bool with_h = false;
+                    if constexpr (kEpi == EPI_BWD_H) {
+                        with_h = p.store_h != 0;
+                        if (with_h) {                        // H itself, the next layer's input
+                            uint32_t hp[16];
+#pragma unroll
+                            for (int j = 0; j < 32; j += 2) hp[j / 2] = pack_bf16x2(x[j], x[j + 1]);
+                            write_row_block(hp, ebuf + 2 * EPI_BLOCK_BYTES, lane);
+                        }
+                    }
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0 && m_row0 < p.M) {        // a block wholly past M is not stored
                         tma_store_2d(&tmC, ebuf, n0, m_row0);
-                        tma_store_2d(&tmCt, ebuf + EPI_WARP_BYTES / 2, m_row0, n0);
+                        tma_store_2d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0, n0);
+                        if (with_h) tma_store_2d(&tmC2, ebuf + 2 * EPI_BLOCK_BYTES, n0, m_row0);
                         bulk_commit_group();
                     }
                 } else {
@@ -570,7 +583,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     if (kEpi == EPI_GELU && p.tma_store) {
                         // rows leave through a shared-memory block and one TMA store (full
                         // lines, instead of 32 rows touched per store instruction)
-                        uint8_t* blk = ebuf + ehalf * (EPI_WARP_BYTES / 2);
+                        uint8_t* blk = ebuf + ehalf * EPI_BLOCK_BYTES;
                         if (lane == 0) bulk_wait_read<1>();  // the store from this block two chunks ago is done
                         __syncwarp();
                         write_row_block(packed, blk, lane);

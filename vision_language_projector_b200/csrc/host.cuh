@@ -340,7 +340,7 @@ inline int raster_group(int N, int K, int BN) {
 
 template <int BN, int A, int E, int CTAS>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tct,
-                GemmParams p, int num_sms, cudaStream_t s) {
+                const CUtensorMap& tc2, GemmParams p, int num_sms, cudaStream_t s) {
     using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E)>;
     auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
     if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN);
@@ -373,13 +373,13 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
     cfg.gridDim = dim3(static_cast<unsigned>(units * CTAS));
     cfg.attrs = CTAS > 1 ? attr : nullptr;
     cfg.numAttrs = CTAS > 1 ? 1 : 0;
-    VLP_CUDA(cudaLaunchKernelEx(&cfg, kernel, ta, tb, tc, tct, p));
+    VLP_CUDA(cudaLaunchKernelEx(&cfg, kernel, ta, tb, tc, tct, tc2, p));
     return VLPROJ_OK;
 }
 
 // Tile shape: 256 x 256 tiles on CTA pairs when N allows and the A operand comes by
-// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise. tc / tct: output maps
-// of the TMA-store epilogues (unused by the others).
+// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise. tc / tct / tc2: output
+// maps of the TMA-store epilogues (unused by the others).
 inline const CUtensorMap& no_map() {
     static const CUtensorMap zero{};
     return zero;
@@ -388,12 +388,12 @@ inline const CUtensorMap& no_map() {
 template <int A, int E>
 int launch_gemm_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb_half,
                    const GemmParams& p, int num_sms, cudaStream_t s, const CUtensorMap& tc = no_map(),
-                   const CUtensorMap& tct = no_map()) {
+                   const CUtensorMap& tct = no_map(), const CUtensorMap& tc2 = no_map()) {
     if constexpr (A != vlp::A_CPASYNC) {
-        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tct, p, num_sms, s);
+        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tct, tc2, p, num_sms, s);
     }
-    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tct, p, num_sms, s);
-    return launch_gemm<128, A, E, 1>(ta, tb, tc, tct, p, num_sms, s);
+    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tct, tc2, p, num_sms, s);
+    return launch_gemm<128, A, E, 1>(ta, tb, tc, tct, tc2, p, num_sms, s);
 }
 
 inline int pick_bn(int N) { return N >= 256 ? 256 : 128; }
@@ -451,7 +451,11 @@ struct vlproj_handle {
     __nv_bfloat16* W2t = nullptr;        // [N1][N2]
     __nv_bfloat16* W1pt = nullptr;       // [K1][N1], rows in position-outer order
     CUtensorMap tmW2t{}, tmW2th{}, tmW1pt{}, tmW1pth{};
-    vlp_host::DevBuf<__nv_bfloat16> G, Ht, dY, dYt, dP, dPt, At;
+    std::vector<__nv_bfloat16*> Wmt;     // middle layers transposed, [N1][N1] each
+    std::vector<CUtensorMap> tmWmt, tmWmth;
+    // G, H^T: one [M][N1] / [N1][ldt] slab per hidden layer; Hr: H row-major for the
+    // hidden layers that feed another one; dP, dP^T: two slabs, layer by layer
+    vlp_host::DevBuf<__nv_bfloat16> G, Ht, Hr, dY, dYt, dP, dPt, At;
     vlp_host::DevBuf<float> dA, part, part_sp;
 };
 

@@ -327,7 +327,8 @@ void vlproj_destroy(vlproj_handle* h) {
     h->H2.release();
     cudaFree(h->W2t);
     cudaFree(h->W1pt);
-    for (auto* b : {&h->G, &h->Ht, &h->dY, &h->dYt, &h->dP, &h->dPt, &h->At}) b->release();
+    for (auto* w : h->Wmt) cudaFree(w);
+    for (auto* b : {&h->G, &h->Ht, &h->Hr, &h->dY, &h->dYt, &h->dP, &h->dPt, &h->At}) b->release();
     h->dA.release();
     h->part.release();
     h->part_sp.release();

@@ -6,10 +6,13 @@
 //    7  LayerNorm-merge               A [M][k*k*C] bf16, position-outer: the forward's
 //                                     bf16 A operand
 //    8  GEMM1 recompute               P = A W1p^T + b1 -> G = GELU'(P) [M][N1] and
-//                                     H^T = GELU(P)^T [N1][M] (bf16)
+//                                     H^T = GELU(P)^T [N1][M] (bf16), for every hidden
+//                                     layer (H itself too where a middle layer reads it)
 //    9  dY gather                     dY [M][N2] and dY^T [N2][M] from d_out's
 //                                     placeholder rows (zeros if the count check failed)
-//   10  dH GEMM                       dP = (dY W2) * G -> dP [M][N1] and dP^T [N1][M]
+//   10  dH GEMMs                      dP = (dY W2) * G -> dP [M][N1] and dP^T [N1][M], and
+//                                     with depth > 2 down through the middle layers, with
+//                                     their weight gradients dW_mid = dP^T H (K = M)
 //   11  dW2 GEMM                      dW2 = dY^T H, K = M
 //   12  A^T + dW1 GEMM                A^T with rows in the caller's column order, then
 //                                     dW1 = dP^T A, K = M
@@ -63,20 +66,35 @@ void transpose_launch(const __nv_bfloat16* src, int64_t ld_src, int64_t src_rows
                                                           static_cast<int>(M), Q, dst, dst_t, ldt, C, kk, chan_outer);
 }
 
-// W2^T [N1][N2] and W1p^T [K1][N1] with their tensor maps, made once per handle.
+// W2^T [N1][N2], W1p^T [K1][N1] and each middle layer's W^T [N1][N1], with their tensor
+// maps, made once per handle.
 int ensure_transposed_weights(vlproj_handle* h, cudaStream_t s) {
-    if (h->W2t && h->W1pt) return VLPROJ_OK;
     const vlproj_config& c = h->cfg;
     const size_t n1 = static_cast<size_t>(c.N1), n2 = static_cast<size_t>(c.N2), k1 = static_cast<size_t>(h->K1);
-    if (!h->W2t) VLP_CUDA(cudaMalloc(&h->W2t, n1 * n2 * 2));
-    if (!h->W1pt) VLP_CUDA(cudaMalloc(&h->W1pt, k1 * n1 * 2));
-    h->launches += 2;
-    transpose_launch(h->W2, c.N1, c.N2, nullptr, nullptr, c.N2, c.N1, nullptr, h->W2t, c.N2, c.C, 1, 0, s);
-    transpose_launch(h->W1p, h->K1, c.N1, nullptr, nullptr, c.N1, h->K1, nullptr, h->W1pt, c.N1, c.C, 1, 0, s);
-    VLP_CUDA(cudaGetLastError());
-    if (encode_b(&h->tmW2t, &h->tmW2th, h->W2t, n1, n2, pick_bn(c.N1)) ||
-        encode_b(&h->tmW1pt, &h->tmW1pth, h->W1pt, k1, n1, pick_bn(h->K1)))
-        return VLPROJ_ERR_CUDA;
+    if (!h->W2t || !h->W1pt) {
+        if (!h->W2t) VLP_CUDA(cudaMalloc(&h->W2t, n1 * n2 * 2));
+        if (!h->W1pt) VLP_CUDA(cudaMalloc(&h->W1pt, k1 * n1 * 2));
+        h->launches += 2;
+        transpose_launch(h->W2, c.N1, c.N2, nullptr, nullptr, c.N2, c.N1, nullptr, h->W2t, c.N2, c.C, 1, 0, s);
+        transpose_launch(h->W1p, h->K1, c.N1, nullptr, nullptr, c.N1, h->K1, nullptr, h->W1pt, c.N1, c.C, 1, 0, s);
+        VLP_CUDA(cudaGetLastError());
+        if (encode_b(&h->tmW2t, &h->tmW2th, h->W2t, n1, n2, pick_bn(c.N1)) ||
+            encode_b(&h->tmW1pt, &h->tmW1pth, h->W1pt, k1, n1, pick_bn(h->K1)))
+            return VLPROJ_ERR_CUDA;
+    }
+    while (h->Wmt.size() < h->Wm.size()) {
+        const size_t i = h->Wmt.size();
+        __nv_bfloat16* w = nullptr;
+        VLP_CUDA(cudaMalloc(&w, n1 * n1 * 2));
+        h->Wmt.push_back(w);
+        ++h->launches;
+        transpose_launch(h->Wm[i], c.N1, c.N1, nullptr, nullptr, c.N1, c.N1, nullptr, w, c.N1, c.C, 1, 0, s);
+        VLP_CUDA(cudaGetLastError());
+        CUtensorMap full{}, half{};
+        if (encode_b(&full, &half, w, n1, n1, pick_bn(c.N1))) return VLPROJ_ERR_CUDA;
+        h->tmWmt.push_back(full);
+        h->tmWmth.push_back(half);
+    }
     return VLPROJ_OK;
 }
 
@@ -91,6 +109,10 @@ int zero_outputs(const vlproj_backward_args* a, const vlproj_config& c, int K1, 
     if (a->d_newline) VLP_CUDA(cudaMemsetAsync(a->d_newline, 0, n2 * 4, s));
     if (a->d_sep) VLP_CUDA(cudaMemsetAsync(a->d_sep, 0, n2 * 4, s));
     if (a->d_features && P > 0) VLP_CUDA(cudaMemsetAsync(a->d_features, 0, static_cast<size_t>(P) * C * 4, s));
+    for (int i = 0; i + 2 < c.depth; ++i) {
+        if (a->d_W_mid && a->d_W_mid[i]) VLP_CUDA(cudaMemsetAsync(a->d_W_mid[i], 0, n1 * n1 * 4, s));
+        if (a->d_b_mid && a->d_b_mid[i]) VLP_CUDA(cudaMemsetAsync(a->d_b_mid[i], 0, n1 * 4, s));
+    }
     return VLPROJ_OK;
 }
 
@@ -101,8 +123,11 @@ bool misaligned(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 != 0
 extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, void* stream) {
     if (!h || !a) return VLPROJ_ERR_INVALID_ARG;
     const vlproj_config& c = h->cfg;
-    if (c.depth != 2) return VLPROJ_ERR_UNSUPPORTED;
     if (c.has_ln && c.C > 256 * 8) return VLPROJ_ERR_UNSUPPORTED;     // LayerNorm backward keeps C in registers
+    const int depth = c.depth;       // Linear layers; hidden layers 1 .. depth - 1
+    const int n_mid = depth - 2;
+    auto mid_w = [&](int i) -> float* { return a->d_W_mid ? a->d_W_mid[i] : nullptr; };
+    auto mid_b = [&](int i) -> float* { return a->d_b_mid ? a->d_b_mid[i] : nullptr; };
     const int64_t n_ids = a->n_ids;
     if (n_ids < 0 || n_ids >= (int64_t(1) << 31)) return VLPROJ_ERR_INVALID_ARG;
     if (n_ids > 0 && (!a->input_ids || !a->d_out)) return VLPROJ_ERR_INVALID_ARG;
@@ -113,6 +138,8 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
                           static_cast<const void*>(a->d_newline), static_cast<const void*>(a->d_sep),
                           static_cast<const void*>(a->d_features)})
         if (misaligned(p)) return VLPROJ_ERR_INVALID_ARG;
+    for (int i = 0; i < n_mid; ++i)
+        if (misaligned(mid_w(i)) || misaligned(mid_b(i))) return VLPROJ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Plan pl;
     int rc = build_plan(c, a->grid_hw, a->spatial_crop, a->n_images, false, VLPROJ_GATHER_CPASYNC, &pl);
@@ -124,23 +151,34 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     // row stride of the transposed copies: whole 128-byte lines, so every TMA box row
     // of the weight-gradient GEMMs starts on a line
     const int64_t ldt = round_up(std::max<int64_t>(M, 1), 64);
+    const size_t hslab = static_cast<size_t>(M) * c.N1, tslab = static_cast<size_t>(c.N1) * ldt;
+
+    // which dP are needed: Linear l's gradients need dP_l; dP_l needs every dP above it
+    const bool want_l1 = a->d_W1 || a->d_b1 || a->d_features || a->d_gamma || a->d_beta;
+    const bool want_da = a->d_features || (c.has_ln && (a->d_gamma || a->d_beta));   // the dA GEMM
+    int l_min = depth;               // lowest Linear whose dP is needed (dP_depth = dY)
+    for (int i = n_mid - 1; i >= 0; --i)
+        if (mid_w(i) || mid_b(i)) l_min = i + 2;
+    if (want_l1) l_min = 1;
+    const bool want_recompute = l_min < depth || a->d_W2;     // G feeds dP, H^T feeds the weight gradients
 
     // scratch
     const int nblocks = static_cast<int>((n_ids + vlp::SCAN_CHUNK - 1) / vlp::SCAN_CHUNK);
     if (h->counts.ensure(std::max(nblocks, 1)) || h->pos.ensure(std::max<int64_t>(pl.R, 1))) return VLPROJ_ERR_CUDA;
-    const bool want_l1 = a->d_W1 || a->d_b1 || a->d_features || a->d_gamma || a->d_beta;
-    const bool want_da = a->d_features || (c.has_ln && (a->d_gamma || a->d_beta));   // the dA GEMM
     if (M > 0) {
         if (h->rowdest.ensure(M) || h->gmeta.ensure(M) || h->A.ensure(static_cast<size_t>(M) * K1) ||
-            h->G.ensure(static_cast<size_t>(M) * c.N1) || h->Ht.ensure(static_cast<size_t>(c.N1) * ldt) ||
+            h->G.ensure(hslab * (depth - 1)) || h->Ht.ensure(tslab * (depth - 1)) ||
+            (depth > 2 && h->Hr.ensure(hslab * (depth - 2))) ||
             h->dY.ensure(static_cast<size_t>(M) * c.N2) || h->dYt.ensure(static_cast<size_t>(c.N2) * ldt) ||
-            h->dP.ensure(static_cast<size_t>(M) * c.N1) || h->dPt.ensure(static_cast<size_t>(c.N1) * ldt))
+            h->dP.ensure(hslab * 2) || h->dPt.ensure(tslab * 2))
             return VLPROJ_ERR_CUDA;
         if (a->d_W1 && h->At.ensure(static_cast<size_t>(K1) * ldt)) return VLPROJ_ERR_CUDA;
         if (want_da && c.has_ln && h->dA.ensure(static_cast<size_t>(M) * K1)) return VLPROJ_ERR_CUDA;
         rc = ensure_transposed_weights(h, s);
         if (rc) return rc;
     }
+    __nv_bfloat16* const G = h->G.ptr;
+    __nv_bfloat16* const Ht = h->Ht.ptr;
     rc = upload_plan(h, pl, s);
     if (rc) return rc;
     h->profiled_valid = false;
@@ -171,12 +209,11 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     VLP_CUDA(cudaGetLastError());
     stage_end(h, 6, s);
 
-    const bool want_gemm1 = want_l1 || a->d_W2;     // G feeds dP, H^T feeds dW2
     const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
     CUtensorMap tmA{};
     GemmParams p{};
 
-    if (want_gemm1) {
+    if (want_recompute) {
         // 7. A, exactly as the forward pass rounds it
         stage_begin(h, 7, s);
         ++h->launches;
@@ -184,18 +221,31 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         if (rc) return rc;
         stage_end(h, 7, s);
 
-        // 8. GEMM1 recompute: G = GELU'(P), H^T
-        if (encode_bf16_2d(&tmA, h->A.ptr, M, K1, vlp::BM)) return VLPROJ_ERR_CUDA;
-        p = gemm_params(h, M, c.N1, K1);
-        p.bias = h->b1;
-        CUtensorMap tmG{}, tmHt{};
-        if (encode_bf16_store(&tmG, h->G.ptr, M, c.N1) || encode_bf16_store(&tmHt, h->Ht.ptr, c.N1, M, ldt))
-            return VLPROJ_ERR_CUDA;
+        // 8. every hidden layer recomputed: G_l = GELU'(P_l), H_l^T, and H_l itself when a
+        //    middle layer reads it
         stage_begin(h, 8, s);
-        ++h->launches;
-        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                         h->num_sms, s, tmG, tmHt);
-        if (rc) return rc;
+        for (int l = 1; l <= depth - 1; ++l) {
+            const bool first = l == 1;
+            const __nv_bfloat16* x = first ? h->A.ptr : h->Hr.ptr + (l - 2) * hslab;
+            const int K = first ? K1 : c.N1;
+            if (encode_bf16_2d(&tmA, x, M, K, vlp::BM)) return VLPROJ_ERR_CUDA;
+            p = gemm_params(h, M, c.N1, K);
+            p.bias = first ? h->b1 : h->bm[l - 2];
+            CUtensorMap tmG{}, tmHt{}, tmHr{};
+            if (encode_bf16_store(&tmG, G + (l - 1) * hslab, M, c.N1) ||
+                encode_bf16_store(&tmHt, Ht + (l - 1) * tslab, c.N1, M, ldt))
+                return VLPROJ_ERR_CUDA;
+            if (l < depth - 1) {
+                p.store_h = 1;
+                if (encode_bf16_store(&tmHr, h->Hr.ptr + (l - 1) * hslab, M, c.N1)) return VLPROJ_ERR_CUDA;
+            }
+            ++h->launches;
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(pick_bn(c.N1), h->pairs, tmA,
+                                                             first ? h->tmW1 : h->tmWm[l - 2],
+                                                             first ? h->tmW1h : h->tmWmh[l - 2], p, h->num_sms, s,
+                                                             tmG, tmHt, tmHr);
+            if (rc) return rc;
+        }
         stage_end(h, 8, s);
     }
 
@@ -207,39 +257,23 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     VLP_CUDA(cudaGetLastError());
     stage_end(h, 9, s);
 
-    // Up to about 2^28 hidden activations (M * N1) the weight gradients run on the side
-    // stream, beside the dP / dA chain on the caller's stream: dW2 and A^T need only
-    // stages 7-9, dW1 waits for dP, and each persistent GEMM takes the SMs the other
-    // leaves free, which fills their partial last waves (measured 1.4-2% faster on the
-    // MoonViT, DeepSeek-ViT and VL2 batches). Larger batches run in sequence: there the
-    // two GEMM streams contend for L2 and power (measured 8% slower on 262,144 tokens).
+    // Up to about 2^28 hidden activations (M * N1) the top and first layers' weight
+    // gradients run on the side stream, beside the dP chain on the caller's stream: the
+    // top one and A^T need only stages 7-9, dW1 waits for dP_1, and each persistent GEMM
+    // takes the SMs the other leaves free, which fills their partial last waves (measured
+    // 1.4-2 % faster on the MoonViT, DeepSeek-ViT and VL2 batches). Larger batches run in
+    // sequence: there the two GEMM streams contend for L2 and power (measured 8 % slower
+    // on 262,144 tokens).
     const bool overlap = M * c.N1 <= (int64_t(1) << 28);
     cudaStream_t ss = overlap ? h->side : s;
     VLP_CUDA(cudaEventRecord(h->fork, s));
     VLP_CUDA(cudaStreamWaitEvent(ss, h->fork, 0));
 
-    // 10. dP = (dY W2) * G, row-major and transposed (caller's stream)
-    if (want_l1) {
-        if (encode_bf16_2d(&tmA, h->dY.ptr, M, c.N2, vlp::BM)) return VLPROJ_ERR_CUDA;
-        p = gemm_params(h, M, c.N1, c.N2);
-        p.aux = h->G.ptr;
-        CUtensorMap tmP{}, tmPt{};
-        if (encode_bf16_store(&tmP, h->dP.ptr, M, c.N1) || encode_bf16_store(&tmPt, h->dPt.ptr, c.N1, M, ldt))
-            return VLPROJ_ERR_CUDA;
-        stage_begin(h, 10, s);
-        ++h->launches;
-        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW2t, h->tmW2th, p,
-                                                         h->num_sms, s, tmP, tmPt);
-        if (rc) return rc;
-        stage_end(h, 10, s);
-        VLP_CUDA(cudaEventRecord(h->join2, s));
-    }
-
-    // 11. dW2 = dY^T H and db2 (side stream)
+    // 11. top layer: dW2 = dY^T H_(depth-1) and db2 (side stream)
     CUtensorMap tmA2{}, tmB2{}, tmB2h{};
     if (a->d_W2) {
         if (encode_bf16_2d(&tmA2, h->dYt.ptr, c.N2, M, vlp::BM, ldt) ||
-            encode_b(&tmB2, &tmB2h, h->Ht.ptr, c.N1, M, pick_bn(c.N1), ldt))
+            encode_b(&tmB2, &tmB2h, Ht + (depth - 2) * tslab, c.N1, M, pick_bn(c.N1), ldt))
             return VLPROJ_ERR_CUDA;
         GemmParams q = gemm_params(h, c.N2, c.N1, M);
         q.outf = a->d_W2;
@@ -256,6 +290,60 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         VLP_CUDA(cudaGetLastError());
     }
 
+    // 10. the dP chain (caller's stream): dP_l = (dP_(l+1) W_(l+1)) * G_l from the top
+    //     down to the lowest layer asked for, with the middle layers' weight gradients
+    //     dW_mid = dP^T H and db_mid on the way; dP ping-pongs between two slabs
+    int cur = 0;                       // slab holding the latest dP
+    if (l_min < depth) {
+        stage_begin(h, 10, s);
+        for (int l = depth - 1; l >= l_min; --l) {
+            // dP_l from dP_(l+1) (dY for the top) through Linear l+1
+            const bool top = l == depth - 1;
+            const int nxt = top ? 0 : cur ^ 1;
+            if (encode_bf16_2d(&tmA, top ? h->dY.ptr : h->dP.ptr + cur * hslab, M, top ? c.N2 : c.N1, vlp::BM))
+                return VLPROJ_ERR_CUDA;
+            p = gemm_params(h, M, c.N1, top ? c.N2 : c.N1);
+            p.aux = G + (l - 1) * hslab;
+            CUtensorMap tmP{}, tmPt{};
+            if (encode_bf16_store(&tmP, h->dP.ptr + nxt * hslab, M, c.N1) ||
+                encode_bf16_store(&tmPt, h->dPt.ptr + nxt * tslab, c.N1, M, ldt))
+                return VLPROJ_ERR_CUDA;
+            ++h->launches;
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(pick_bn(c.N1), h->pairs, tmA,
+                                                             top ? h->tmW2t : h->tmWmt[l - 1],
+                                                             top ? h->tmW2th : h->tmWmth[l - 1], p, h->num_sms, s,
+                                                             tmP, tmPt);
+            if (rc) return rc;
+            cur = nxt;
+            if (l < 2) continue;
+            // Linear l (middle layer l - 2): dW = dP_l^T H_(l-1), db = sum dP_l
+            const int i = l - 2;
+            if (mid_w(i)) {
+                CUtensorMap ta{}, tb{}, tbh{};
+                if (encode_bf16_2d(&ta, h->dPt.ptr + cur * tslab, c.N1, M, vlp::BM, ldt) ||
+                    encode_b(&tb, &tbh, Ht + (l - 2) * tslab, c.N1, M, pick_bn(c.N1), ldt))
+                    return VLPROJ_ERR_CUDA;
+                GemmParams q = gemm_params(h, c.N1, c.N1, M);
+                q.outf = mid_w(i);
+                ++h->launches;
+                rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(c.N1), h->pairs, ta, tb, tbh, q, h->num_sms,
+                                                               s);
+                if (rc) return rc;
+            }
+            if (mid_b(i)) {
+                ++h->launches;
+                vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, s>>>(h->dPt.ptr + cur * tslab, ldt, c.N1, M,
+                                                                      mid_b(i));
+                VLP_CUDA(cudaGetLastError());
+            }
+        }
+        stage_end(h, 10, s);
+        VLP_CUDA(cudaEventRecord(h->join2, s));
+    }
+    // dP_1, when the chain reached it (l_min == 1)
+    const __nv_bfloat16* dP1 = h->dP.ptr + cur * hslab;
+    const __nv_bfloat16* dP1t = h->dPt.ptr + cur * tslab;
+
     // 12a. A^T in the caller's column order (side stream)
     if (a->d_W1) {
         stage_begin(h, 12, ss);
@@ -265,10 +353,10 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         VLP_CUDA(cudaGetLastError());
     }
 
-    // 12b. dW1 = dP^T A and db1 (side stream, after dP)
+    // 12b. dW1 = dP_1^T A and db1 (side stream, after dP_1)
     if (want_l1) VLP_CUDA(cudaStreamWaitEvent(ss, h->join2, 0));
     if (a->d_W1) {
-        if (encode_bf16_2d(&tmA2, h->dPt.ptr, c.N1, M, vlp::BM, ldt) ||
+        if (encode_bf16_2d(&tmA2, dP1t, c.N1, M, vlp::BM, ldt) ||
             encode_b(&tmB2, &tmB2h, h->At.ptr, K1, M, pick_bn(K1), ldt))
             return VLPROJ_ERR_CUDA;
         GemmParams q = gemm_params(h, c.N1, K1, M);
@@ -281,7 +369,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     }
     if (a->d_b1) {
         ++h->launches;
-        vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, ss>>>(h->dPt.ptr, ldt, c.N1, M, a->d_b1);
+        vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, ss>>>(dP1t, ldt, c.N1, M, a->d_b1);
         VLP_CUDA(cudaGetLastError());
     }
     VLP_CUDA(cudaEventRecord(h->join, ss));
@@ -290,7 +378,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     //     backward; without a LayerNorm the epilogue folds it onto the patches as the
     //     feature gradient itself
     if (want_da) {
-        if (encode_bf16_2d(&tmA, h->dP.ptr, M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
+        if (encode_bf16_2d(&tmA, dP1, M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
         p = gemm_params(h, M, K1, c.N1);
         stage_begin(h, 13, s);
         ++h->launches;
