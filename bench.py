@@ -371,29 +371,18 @@ def main():
                 "frac": None if achieved is None else achieved / peaks.get("hbm_gbs"),
                 "peak_source": f"{peak_src} HBM copy", "traffic": None, "algorithmic_bytes": b}
 
-    # ---- end to end through the public API with host buffers. Per step: the step's inputs
-    # (features, ids) from pinned host memory to the device, vlproj_forward_ex (projection,
-    # plus the token-embedding lookup of the text rows from the device-resident table and a
-    # compact copy of the assembled rows), and the assembled rows back to pinned host memory.
+    # ---- end to end through the public API with host buffers: vlproj_project_host takes the
+    # step's features from pinned host memory and returns the assembled rows of every image to
+    # pinned host memory, its copies pipelined against the projection; the step ends when the
+    # last rows have landed in host memory.
     e2e = None
     if args.e2e_steps > 0:
-        table = bf(W.embed_table(wl, seed))
         R = int(sum(rows))
         feats_p = (torch.from_numpy(feats_h) if wl.feat_fp32 else torch.from_numpy(feats_h.view(np.int16))).pin_memory()
-        ids_p = torch.from_numpy(ids_h).pin_memory()
-        rows_d = torch.empty((R, wl.N2), dtype=torch.bfloat16, device="cuda")
         rows_p = torch.empty((R, wl.N2), dtype=torch.int16).pin_memory()
-        feats_d = torch.empty(feats_p.shape, dtype=feats_p.dtype, device="cuda")
-        ids_d = torch.empty_like(ids)
-        emb_d = torch.empty_like(out)
 
         def e2e_step():
-            feats_d.copy_(feats_p, non_blocking=True)
-            ids_d.copy_(ids_p, non_blocking=True)
-            f = feats_d if wl.feat_fp32 else feats_d.view(torch.bfloat16)
-            proj.forward_ex(f, hw, crop, ids_d, W.IMAGE_TOKEN_ID, emb_d, newline, sep, embed_table=table,
-                            rows_out=rows_d, stream=stream, n_images=wl.n_images)
-            rows_p.copy_(rows_d.view(torch.int16), non_blocking=True)
+            proj.project_host(feats_p, hw, crop, rows_p, newline, sep, stream=stream, n_images=wl.n_images)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -417,10 +406,10 @@ def main():
         if st != vp.OK:
             raise SystemExit(f"e2e steps failed: {vp.strerror(st)}")
         e2e = {"value": world * tokens_per_step * args.e2e_steps / (e_ms / 1000.0), "unit": UNIT,
-               "h2d_bytes_per_step": int(feats_p.numel() * feats_p.element_size() + ids_p.numel() * 8),
+               "h2d_bytes_per_step": int(feats_p.numel() * feats_p.element_size()),
                "d2h_bytes_per_step": int(rows_p.numel() * 2), "steps": args.e2e_steps,
-               "path": "vlproj_forward_ex: host features + ids in; token-embedding lookup from the resident "
-                       "table; assembled rows out"}
+               "path": "vlproj_project_host: pinned host features in, every image's assembled rows out to "
+                       "pinned host memory, copies pipelined against the projection in image chunks"}
 
     # ---- backward: every gradient of the projector for the same batch, timed like the forward
     bwd = None

@@ -164,6 +164,39 @@ typedef struct vlproj_forward_args {
 } vlproj_forward_args;
 int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* stream);
 
+/* ---- host memory in, host memory out -----------------------------------
+ * The projected rows of a batch whose features are in host memory, written to host
+ * memory: the same rows as vlproj_forward_ex's rows_out (every image's assembled rows,
+ * newlines and separators included, images in order; "port DeepSeek-VL2",
+ * Tile-sequence assembly), without the embedding buffer. The batch is cut into
+ * `chunks` runs of whole images of about equal token count (0 = automatic); chunk j's
+ * features are copied to the device while chunk j-1 is projected and chunk j-2's rows
+ * are copied back, on copy streams of the handle, so PCIe traffic in both directions
+ * overlaps the GEMMs. Work is enqueued behind `stream`; the call returns without
+ * waiting, and `stream` completes only after the last rows have reached rows_out.
+ *   features   HOST, as for vlproj_forward (packed views, feat_dtype); page-locked
+ *              memory (cudaHostAlloc / cudaHostRegister) for the copies to overlap.
+ *   grid_hw, spatial_crop, n_images, newline, sep: as for vlproj_forward.
+ *   rows_out   HOST bf16 [rows_out_cap][N2], rows_out_cap >= R (vlproj_image_rows),
+ *              page-locked for the copies to overlap.
+ *   chunks     pipeline depth in image runs; 0 picks about one run per 16 MiB of
+ *              features, 2 to 16; never more runs than images.
+ * Both host buffers must stay valid and untouched until `stream` has completed.
+ * Errors: VLPROJ_ERR_INVALID_ARG for inconsistent shapes, a small rows_out_cap or a
+ * NULL buffer, before any work is enqueued. */
+typedef struct vlproj_host_args {
+    const void*    features;
+    const int32_t* grid_hw;
+    const int32_t* spatial_crop;
+    int32_t        n_images;
+    const void*    newline;
+    const void*    sep;
+    void*          rows_out;
+    int64_t        rows_out_cap;
+    int32_t        chunks;
+} vlproj_host_args;
+int vlproj_project_host(vlproj_handle* h, const vlproj_host_args* args, void* stream);
+
 /* ---- backward -----------------------------------------------------------
  * Gradients of the projector for one batch. The bridge is trained with the vision
  * tower and the language model frozen, so the projector's parameters are the only

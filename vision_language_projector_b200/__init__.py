@@ -27,7 +27,7 @@ EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
             "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
             "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc", "vlproj_forward_ex",
-            "vlproj_plan_tiles", "vlproj_backward")
+            "vlproj_plan_tiles", "vlproj_backward", "vlproj_project_host")
 NOALLOC_MAX_IDS = 64 * 1024 * 1024
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX = 0, 1, 2, 3
 NUM_STAGES = 15
@@ -62,6 +62,15 @@ class BackwardArgs(ctypes.Structure):
     ] + [("d_" + n, ctypes.c_void_p) for n in ("W1", "b1", "W2", "b2", "gamma", "beta", "newline", "sep",
                                                   "features")] + [("d_W_mid", ctypes.c_void_p),
                                                                   ("d_b_mid", ctypes.c_void_p)]
+
+
+class HostArgs(ctypes.Structure):
+    """Mirror of ``vlproj_host_args``."""
+    _fields_ = [
+        ("features", ctypes.c_void_p), ("grid_hw", ctypes.c_void_p), ("spatial_crop", ctypes.c_void_p),
+        ("n_images", ctypes.c_int32), ("newline", ctypes.c_void_p), ("sep", ctypes.c_void_p),
+        ("rows_out", ctypes.c_void_p), ("rows_out_cap", ctypes.c_int64), ("chunks", ctypes.c_int32),
+    ]
 
 
 class Config(ctypes.Structure):
@@ -114,6 +123,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_plan_tiles.restype = I64
     lib.vlproj_forward_ex.argtypes = [P, ctypes.POINTER(ForwardArgs), P]
     lib.vlproj_forward_ex.restype = ctypes.c_int
+    lib.vlproj_project_host.argtypes = [P, ctypes.POINTER(HostArgs), P]
+    lib.vlproj_project_host.restype = ctypes.c_int
     lib.vlproj_backward.argtypes = [P, ctypes.POINTER(BackwardArgs), P]
     lib.vlproj_backward.restype = ctypes.c_int
     lib.vlproj_placeholder_index_noalloc.argtypes = [P, I64, I64, P, I64, P, P]
@@ -297,6 +308,23 @@ class Projector:
         rc = _lib.vlproj_backward(self._h, ctypes.byref(a), _stream_ptr(stream))
         if check and rc != OK:
             raise VlprojError(rc, "vlproj_backward")
+        return rc
+
+    def project_host(self, features, grid_hw, spatial_crop, rows_out, newline=None, sep=None, chunks: int = 0,
+                     stream=None, n_images: Optional[int] = None, check: bool = True) -> int:
+        """vlproj_project_host: features in HOST memory (page-locked for overlap), the
+        assembled rows of every image written to ``rows_out`` (HOST, (>= R, N2) bf16),
+        copies pipelined against the projection. Completes with ``stream``."""
+        g = _host_i32(grid_hw)
+        c = _host_i32(spatial_crop)
+        if n_images is None:
+            n_images = len(c) if c is not None else (0 if g is None else len(g))
+        self._host_keep = (g, c)           # the host tables must outlive the enqueue only
+        a = HostArgs(_ptr(features), _ptr(g), _ptr(c), n_images, _ptr(newline), _ptr(sep), _ptr(rows_out),
+                     0 if rows_out is None else int(rows_out.shape[0]), int(chunks))
+        rc = _lib.vlproj_project_host(self._h, ctypes.byref(a), _stream_ptr(stream))
+        if check and rc != OK:
+            raise VlprojError(rc, "vlproj_project_host")
         return rc
 
     def hidden(self, features, grid_hw, hidden, stream=None) -> None:

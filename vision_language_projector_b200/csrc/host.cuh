@@ -457,6 +457,11 @@ struct vlproj_handle {
     // hidden layers that feed another one; dP, dP^T: two slabs, layer by layer
     vlp_host::DevBuf<__nv_bfloat16> G, Ht, Hr, dY, dYt, dP, dPt, At;
     vlp_host::DevBuf<float> dA, part, part_sp;
+    // host-memory entry point: copy streams, per-slot events and double-buffered staging
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};
+    vlp_host::DevBuf<uint8_t> stage_feat[2];
+    vlp_host::DevBuf<__nv_bfloat16> stage_rows[2];
 };
 
 namespace vlp_host {
@@ -497,5 +502,11 @@ inline int upload_plan(vlproj_handle* h, const Plan& pl, cudaStream_t s) {
     if (rc) return rc;
     return h->up_images.put(h->dimages.ptr, pl.images.data(), pl.images.size() * sizeof(ImageDesc), s);
 }
+
+// Defined in vlproj.cu: the forward's geometry + LayerNorm/convert + GEMM1 steps, and
+// its middle layers (depth > 2).
+int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, const int32_t* pos, int dest_mode,
+                    __nv_bfloat16* hidden, int64_t hidden_rows, cudaStream_t s, const vlp::ViewDesc* dviews);
+int run_middle_layers(vlproj_handle* h, const Plan& pl, cudaStream_t s, const __nv_bfloat16** hlast);
 
 }  // namespace vlp_host

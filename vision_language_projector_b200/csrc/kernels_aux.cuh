@@ -134,6 +134,7 @@ __device__ __forceinline__ int find_view(const ViewDesc* views, int n_views, int
 constexpr int DEST_NONE = 0;      // no destination table
 constexpr int DEST_EMBED = 1;     // rowdest[m] = embedding row of the placeholder that takes token m
 constexpr int DEST_COMPACT = 2;   // rowdest[m] = merged-token index (views in order, no padding)
+constexpr int DEST_ROW = 3;       // rowdest[m] = assembled row of token m (the rows of the batch in order)
 
 // One thread per GEMM row m (and per im2col chunk): gather metadata for the cp.async
 // path, the destination of the row, and the im2col coordinates of each chunk's
@@ -178,6 +179,9 @@ static __global__ void __launch_bounds__(256) vlp_geometry_kernel(const ViewDesc
         rowdest[m] = (real && g >= 0 && g < R) ? pos[g] : -1;
     } else if (dest_mode == DEST_COMPACT) {
         rowdest[m] = real ? V.tok_real + t : -1;
+    } else if (dest_mode == DEST_ROW) {
+        const int64_t g = V.row_base + assembled_row(V, i, j);
+        rowdest[m] = (real && g >= 0 && g < R) ? static_cast<int32_t>(g) : -1;
     }
 }
 
@@ -469,14 +473,16 @@ __device__ __forceinline__ int64_t special_row(const ImageDesc& I, int n) {
     return I.tail ? local_rows : global_rows;
 }
 
-// blockIdx.y = image, blockIdx.x = special row n of that image (see special_row).
+// blockIdx.y = image, blockIdx.x = special row n of that image (see special_row). The row
+// goes to out[pos[g]] for assembled row g, or to out[g] when pos is null (rows in
+// assembled order); fwd_status null = no count check.
 static __global__ void __launch_bounds__(128) vlp_special_rows_kernel(const ImageDesc* __restrict__ imgs,
                                                                const int32_t* __restrict__ pos, int64_t R,
                                                                const __nv_bfloat16* __restrict__ newline,
                                                                const __nv_bfloat16* __restrict__ sep,
                                                                __nv_bfloat16* __restrict__ out, int64_t out_rows,
                                                                int N, const int* __restrict__ fwd_status) {
-    if (*fwd_status != 0) return;
+    if (fwd_status != nullptr && *fwd_status != 0) return;
     const ImageDesc I = imgs[blockIdx.y];
     const int n = blockIdx.x;
     const int n_nl = I.hp + I.th * I.hp;
@@ -484,7 +490,7 @@ static __global__ void __launch_bounds__(128) vlp_special_rows_kernel(const Imag
     const __nv_bfloat16* src = n < n_nl ? newline : sep;
     const int64_t g = I.row_base + special_row(I, n);
     if (g < 0 || g >= R) return;
-    const int64_t d = pos[g];
+    const int64_t d = pos != nullptr ? pos[g] : g;
     if (d < 0 || d >= out_rows) return;
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(out + d * N);

@@ -16,13 +16,16 @@
 
 using namespace vlp_host;
 
-namespace {
+namespace vlp_host {
 
 // Steps 1-3: geometry, LayerNorm/convert, GEMM1. GEMM row m goes to
 //   dest_mode DEST_EMBED:   hidden row m (internal H, M rows); pos gives rowdest for GEMM2
+//   dest_mode DEST_ROW:     hidden row m; rowdest[m] = the token's assembled row
 //   dest_mode DEST_COMPACT: hidden row = merged-token index (caller's buffer, M_real rows)
+// dviews: the plan's view table on the device (null = the handle's).
 int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, const int32_t* pos, int dest_mode,
-                    __nv_bfloat16* hidden, int64_t hidden_rows, cudaStream_t s) {
+                    __nv_bfloat16* hidden, int64_t hidden_rows, cudaStream_t s, const ViewDesc* dviews) {
+    if (!dviews) dviews = h->dviews.ptr;
     const vlproj_config& c = h->cfg;
     const int M = static_cast<int>(pl.M);
     if (M == 0) return VLPROJ_OK;
@@ -39,7 +42,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     ++h->launches;
     const int geo_threads = std::max(M, n_chunks);
     vlp::vlp_geometry_kernel<<<(geo_threads + 255) / 256, 256, 0, s>>>(
-        h->dviews.ptr, static_cast<int>(pl.views.size()), M, c.k, pos, pl.R, dest_mode,
+        dviews, static_cast<int>(pl.views.size()), M, c.k, pos, pl.R, dest_mode,
         cpasync ? h->gmeta.ptr : nullptr, h->rowdest.ptr, im2col ? h->chunks.ptr : nullptr, n_chunks, pl.chunk,
         pl.uniform ? 1 : 0);
     VLP_CUDA(cudaGetLastError());
@@ -147,7 +150,41 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     return VLPROJ_OK;
 }
 
-}  // namespace
+// Middle layers (depth > 2): H <- bf16(GELU(H Wm^T + bm)), ping-pong between H and H2.
+// *hlast: the buffer holding the last hidden activation.
+int run_middle_layers(vlproj_handle* h, const Plan& pl, cudaStream_t s, const __nv_bfloat16** hlast) {
+    const vlproj_config& c = h->cfg;
+    bool last_in_h2 = false;
+    for (int layer = 0; layer + 2 < c.depth; ++layer) {
+        DevBuf<__nv_bfloat16>& src = last_in_h2 ? h->H2 : h->H;
+        DevBuf<__nv_bfloat16>& dst = last_in_h2 ? h->H : h->H2;
+        CUtensorMap tin{};
+        if (encode_bf16_2d(&tin, src.ptr, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
+        GemmParams q{};
+        q.M = static_cast<int>(pl.M);
+        q.N = c.N1;
+        q.K = c.N1;
+        q.bias = h->bm[layer];
+        q.C = c.C;
+        q.k = c.k;
+        q.out = dst.ptr;
+        q.out_rows = pl.M;
+        q.err = h->status;
+        q.wait_ns = h->wait_ns;
+        CUtensorMap tout{};
+        q.tma_store = 1;
+        if (encode_bf16_store(&tout, dst.ptr, pl.M, c.N1)) return VLPROJ_ERR_CUDA;
+        ++h->launches;
+        int rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tin, h->tmWm[layer],
+                                                            h->tmWmh[layer], q, h->num_sms, s, tout);
+        if (rc) return rc;
+        last_in_h2 = !last_in_h2;
+    }
+    *hlast = last_in_h2 ? h->H2.ptr : h->H.ptr;
+    return VLPROJ_OK;
+}
+
+}  // namespace vlp_host
 
 extern "C" {
 
@@ -332,6 +369,15 @@ void vlproj_destroy(vlproj_handle* h) {
     h->dA.release();
     h->part.release();
     h->part_sp.release();
+    for (int i = 0; i < 2; ++i) {
+        h->stage_feat[i].release();
+        h->stage_rows[i].release();
+        if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+        if (h->ev_done[i]) cudaEventDestroy(h->ev_done[i]);
+        if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+    }
+    if (h->copy_in) cudaStreamDestroy(h->copy_in);
+    if (h->copy_out) cudaStreamDestroy(h->copy_out);
     for (auto* w : h->Wm) cudaFree(w);
     for (auto* b : h->bm) cudaFree(b);
     h->Xn.release();
@@ -403,7 +449,7 @@ int vlproj_hidden(vlproj_handle* h, const void* features, const int32_t* grid_hw
     rc = upload_plan(h, pl, s);
     if (rc) return rc;
     return run_merge_gemm1(h, pl, features, nullptr, vlp::DEST_COMPACT, static_cast<__nv_bfloat16*>(hidden),
-                           pl.M_real, s);
+                           pl.M_real, s, nullptr);
 }
 
 int vlproj_forward(vlproj_handle* h, const void* features, const int32_t* grid_hw, const int32_t* spatial_crop,
@@ -507,39 +553,15 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
     }
 
     // 1-3. geometry, LayerNorm, GEMM1 -> H
-    rc = run_merge_gemm1(h, pl, features, nullptr, vlp::DEST_NONE, h->H.ptr, pl.M, s);
+    rc = run_merge_gemm1(h, pl, features, nullptr, vlp::DEST_NONE, h->H.ptr, pl.M, s, nullptr);
     if (rc) return rc;
-    // middle layers (depth > 2): H <- bf16(GELU(H Wm^T + bm)), ping-pong between H and H2
-    bool last_in_h2 = false;
-    for (int layer = 0; layer + 2 < c.depth; ++layer) {
-        DevBuf<__nv_bfloat16>& src = last_in_h2 ? h->H2 : h->H;
-        DevBuf<__nv_bfloat16>& dst = last_in_h2 ? h->H : h->H2;
-        CUtensorMap tin{};
-        if (encode_bf16_2d(&tin, src.ptr, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
-        GemmParams q{};
-        q.M = static_cast<int>(pl.M);
-        q.N = c.N1;
-        q.K = c.N1;
-        q.bias = h->bm[layer];
-        q.C = c.C;
-        q.k = c.k;
-        q.out = dst.ptr;
-        q.out_rows = pl.M;
-        q.err = h->status;
-        q.wait_ns = h->wait_ns;
-        CUtensorMap tout{};
-        q.tma_store = 1;
-        if (encode_bf16_store(&tout, dst.ptr, pl.M, c.N1)) return VLPROJ_ERR_CUDA;
-        ++h->launches;
-        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tin, h->tmWm[layer],
-                                                        h->tmWmh[layer], q, h->num_sms, s, tout);
-        if (rc) return rc;
-        last_in_h2 = !last_in_h2;
-    }
+    // middle layers (depth > 2)
+    const __nv_bfloat16* hlast = nullptr;
+    rc = run_middle_layers(h, pl, s, &hlast);
+    if (rc) return rc;
     VLP_CUDA(cudaStreamWaitEvent(s, h->join, 0));
 
     // 4. GEMM2 + scatter (from the last hidden activation)
-    const __nv_bfloat16* hlast = last_in_h2 ? h->H2.ptr : h->H.ptr;
     if (h->tmH_ptr != hlast || h->tmH_rows != pl.M) {
         if (encode_bf16_2d(&h->tmH, hlast, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
         h->tmH_ptr = hlast;
