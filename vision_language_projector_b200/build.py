@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libvlproj.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("vlproj.cu", "vlproj_backward.cu", "vlproj_host.cu", "vlproj_noalloc.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "gemm_sm100.cuh", "kernels_aux.cuh", "kernels_bwd.cuh", "host.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "gemm_sm100.cuh", "kernels_aux.cuh", "kernels_bwd.cuh", "host.cuh", "gelu_poly.cuh")] + [
     os.path.join(ROOT, "include", "vlproj.h")]
 
 
