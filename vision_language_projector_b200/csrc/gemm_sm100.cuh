@@ -161,6 +161,20 @@ __device__ __forceinline__ void gelu_grad2(float p0, float p1, float& g0, float&
     f2_unpack(f2_fma(d, f2_splat(1.0f), f2_splat(0.5f)), g0, g1);
 }
 
+// The 32 bias values of a chunk, the same for every lane: eight broadcast 16-byte loads
+// (bias is 16-byte aligned and n0 a multiple of 32) instead of one load and 32 shuffles.
+__device__ __forceinline__ void load_bias32(const float* bias, int n0, float (&b)[32]) {
+    const float4* b4 = reinterpret_cast<const float4*>(bias + n0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 t = __ldg(b4 + q);
+        b[4 * q] = t.x;
+        b[4 * q + 1] = t.y;
+        b[4 * q + 2] = t.z;
+        b[4 * q + 3] = t.w;
+    }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -525,11 +539,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     float x[32];
                     uint32_t packed[16];
                     if constexpr (kEpi == EPI_BWD_H) {
-                        const float bl = __ldg(&p.bias[n0 + lane]);
+                        float bb[32];
+                        load_bias32(p.bias, n0, bb);
 #pragma unroll
                         for (int j = 0; j < 32; j += 2) {
-                            const float p0 = __uint_as_float(v[j]) + __shfl_sync(0xffffffffu, bl, j);
-                            const float p1 = __uint_as_float(v[j + 1]) + __shfl_sync(0xffffffffu, bl, j + 1);
+                            const float p0 = __uint_as_float(v[j]) + bb[j];
+                            const float p1 = __uint_as_float(v[j + 1]) + bb[j + 1];
                             float g0, g1;
                             gelu_grad2(p0, p1, g0, g1);
                             packed[j / 2] = pack_bf16x2(g0, g1);
@@ -580,12 +595,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         bulk_commit_group();
                     }
                 } else {
-                    const float bl = __ldg(&p.bias[n0 + lane]);
+                    float bb[32];
+                    load_bias32(p.bias, n0, bb);
                     uint32_t packed[16];
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
-                        float x0 = __uint_as_float(v[j]) + __shfl_sync(0xffffffffu, bl, j);
-                        float x1 = __uint_as_float(v[j + 1]) + __shfl_sync(0xffffffffu, bl, j + 1);
+                        float x0 = __uint_as_float(v[j]) + bb[j];
+                        float x1 = __uint_as_float(v[j + 1]) + bb[j + 1];
                         if (kEpi == EPI_GELU) gelu2(x0, x1);
                         packed[j / 2] = pack_bf16x2(x0, x1);
                     }
