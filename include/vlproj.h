@@ -219,7 +219,8 @@ int vlproj_project_host(vlproj_handle* h, const vlproj_host_args* args, void* st
  * layer 1 is the first Linear and layer `depth` the last.
  * The bf16 rounding points of the forward (A and every hidden activation) pass
  * gradients unchanged; A and the hidden activations are the forward's bf16 values,
- * each dP is rounded to bf16 once (fp32 accumulation throughout).
+ * each dP is rounded to bf16 once, and with a LayerNorm so is dA (fp32 accumulation
+ * throughout).
  *
  *   features, grid_hw, spatial_crop, n_images, input_ids, n_ids, image_token_id:
  *                 as for vlproj_forward (the same batch the loss was computed on).
@@ -234,8 +235,8 @@ int vlproj_project_host(vlproj_handle* h, const vlproj_host_args* args, void* st
  *   d_W_mid, d_b_mid  depth > 2: HOST arrays of depth - 2 DEVICE fp32 pointers
  *                 (d_W_mid[i] [N1][N1], d_b_mid[i] [N1]), or NULL; an entry may be NULL.
  *                 Ignored for depth 2.
- * Scratch: about 2 * M * (2*N1*(depth - 1) + N1*(depth - 2) + 2*N1 + 2*N2 + 2*k*k*C)
- * bytes, plus M*k*k*C fp32 with a LayerNorm (M merged tokens), kept in the handle. Errors as for vlproj_forward; when the
+ * Scratch: about 2 * M * (2*N1*(depth - 1) + N1*(depth - 2) + 2*N1 + 2*N2 + 3*k*k*C)
+ * bytes (M merged tokens), kept in the handle. Errors as for vlproj_forward; when the
  * placeholder count check fails every gradient is written as zero and
  * VLPROJ_ERR_TOKEN_COUNT is latched. */
 typedef struct vlproj_backward_args {

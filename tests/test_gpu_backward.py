@@ -8,8 +8,9 @@ so on, see oracle/backward.py), so each term of an entry may be off by a relativ
     than the fp64 oracle does lands one ulp away, at most 2^-7 of it;
   * dW2 terms hold H (one such boundary): e = 2^-7;
   * dW1 terms hold dP, rounded twice (GELU'(P), then dP: (1 + 2^-8)^2 - 1 < 2^-7 + 2^-15),
-    and A (one boundary, 2^-7): e = 2^-6; db1, dA, the LayerNorm gradients and
-    d_features carry dP's rounding only, and take the same e;
+    and A (one boundary, 2^-7): e = 2^-6; db1 carries dP's rounding only; with a
+    LayerNorm, dA is rounded to bf16 too (2^-8 more), so d_features, dgamma and dbeta
+    carry under 2^-7 + 2^-8 + 2^-15: all take the same e;
   * db2 and the newline / separator rows are fp32 sums of exact bf16 values: e = 2^-8.
 An entry whose terms are all zero must come out exactly zero.
 """

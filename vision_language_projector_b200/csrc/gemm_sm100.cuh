@@ -23,6 +23,7 @@
 //   bf16 outputs with plain rows (GEMM1's H, the backward's G, H^T, dP, dP^T) leave the
 //   epilogue as 32 x 32 blocks through shared memory and TMA tile stores.
 //       EPI_F32     acc as fp32, row-major (weight and input gradients)
+//       EPI_BF16    acc as bf16 through TMA stores (the LayerNorm backward's dA)
 //       EPI_FOLD_F32  acc as fp32, folded back onto the patches: column p*C + c of
 //                   merged token m goes to channel c of the patch at position p of its
 //                   k x k neighbourhood (gmeta), so dA never goes to memory
@@ -60,6 +61,7 @@ constexpr int EPI_BWD_H = 2;
 constexpr int EPI_DGELU = 3;
 constexpr int EPI_F32 = 4;
 constexpr int EPI_FOLD_F32 = 5;
+constexpr int EPI_BF16 = 6;
 constexpr int A_TILE = 0;               // dense row-major A, tiled TMA
 constexpr int A_IM2COL = 1;             // merge-gather by TMA im2col
 constexpr int A_CPASYNC = 2;            // merge-gather by cp.async
@@ -75,7 +77,7 @@ constexpr int ERR_TIMEOUT = -5;
 // dP^T), BWD_H three (G, H^T and, for a following layer, H).
 constexpr int EPI_BLOCK_BYTES = 32 * 32 * 2;
 __host__ __device__ constexpr int epi_blocks(int epi) {
-    return epi == EPI_BWD_H ? 3 : (epi == EPI_GELU || epi == EPI_DGELU) ? 2 : 0;
+    return epi == EPI_BWD_H ? 3 : (epi == EPI_GELU || epi == EPI_DGELU || epi == EPI_BF16) ? 2 : 0;
 }
 __host__ __device__ constexpr int epi_stage_bytes(int epi) { return 4 * epi_blocks(epi) * EPI_BLOCK_BYTES; }
 
@@ -596,7 +598,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                 } else {
                     float bb[32];
-                    load_bias32(p.bias, n0, bb);
+                    if constexpr (kEpi == EPI_BF16) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) bb[j] = 0.0f;
+                    } else {
+                        load_bias32(p.bias, n0, bb);
+                    }
                     uint32_t packed[16];
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
@@ -605,7 +612,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         if (kEpi == EPI_GELU) gelu2(x0, x1);
                         packed[j / 2] = pack_bf16x2(x0, x1);
                     }
-                    if (kEpi == EPI_GELU && p.tma_store) {
+                    if ((kEpi == EPI_GELU || kEpi == EPI_BF16) && p.tma_store) {
                         // rows leave through a shared-memory block and one TMA store (full
                         // lines, instead of 32 rows touched per store instruction)
                         uint8_t* blk = ebuf + ehalf * EPI_BLOCK_BYTES;

@@ -456,7 +456,8 @@ struct vlproj_handle {
     // G, H^T: one [M][N1] / [N1][ldt] slab per hidden layer; Hr: H row-major for the
     // hidden layers that feed another one; dP, dP^T: two slabs, layer by layer
     vlp_host::DevBuf<__nv_bfloat16> G, Ht, Hr, dY, dYt, dP, dPt, At;
-    vlp_host::DevBuf<float> dA, part, part_sp;
+    vlp_host::DevBuf<__nv_bfloat16> dA;
+    vlp_host::DevBuf<float> part, part_sp;
     // host-memory entry point: copy streams, per-slot events and double-buffered staging
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
     cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};

@@ -134,7 +134,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Backward of the pre-merge LayerNorm, one warp per (merged token m, position p) item as
 // in the merge pass; the item's patch is row gmeta[m].x + dy * w + dx of the features,
 // and items in the pad are skipped.
-//   dsrc = dA[m][p*C .. p*C + C)            fp32, position-outer columns
+//   dsrc = dA[m][p*C .. p*C + C)            bf16, position-outer columns
 //   xhat = (x - mean) * rstd                the forward pass's fp32 statistics
 //   dx   = rstd * (g - mean(g) - xhat * mean(g * xhat)),  g = dsrc * gamma
 // Each lane holds its kVec 8-channel vectors of x and dsrc in registers, so both are
@@ -148,7 +148,8 @@ template <bool kF32In, int kVec>
 __global__ void __launch_bounds__(256) vlp_ln_backward_kernel(const void* __restrict__ x,
                                                               const int2* __restrict__ gmeta, int M, int k, int C,
                                                               const float* __restrict__ gamma, float eps,
-                                                              const float* __restrict__ dA, float* __restrict__ dfeat,
+                                                              const __nv_bfloat16* __restrict__ dA,
+                                                              float* __restrict__ dfeat,
                                                               float* __restrict__ partial) {
     extern __shared__ float lnb_acc[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(256) vlp_ln_backward_kernel(const void* __rest
         if (!((wm >> pp) & 1u)) continue;
         const int dy = pp / k, dx = pp - dy * k;
         const int64_t row = static_cast<int64_t>(g.x) + dy * static_cast<int>(wm >> 16) + dx;
-        const float* d = dA + (static_cast<int64_t>(m) * kk + pp) * C;
+        const int64_t drow = static_cast<int64_t>(m) * kk + pp;     // dA row of C values
         float f[kVec][8], dd[kVec][8];
         float s = 0.f;
 #pragma unroll
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(256) vlp_ln_backward_kernel(const void* __rest
             const int v = lane + 32 * i;
             if (v < nvec) {
                 load8_feat<kF32In>(x, row, C, v, f[i]);
-                load8_f32(d, v, dd[i]);
+                load8_feat<false>(dA, drow, C, v, dd[i]);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) f[i][e] = dd[i][e] = 0.f;

@@ -16,8 +16,8 @@
 //   11  dW2 GEMM                      dW2 = dY^T H, K = M
 //   12  A^T + dW1 GEMM                A^T with rows in the caller's column order, then
 //                                     dW1 = dP^T A, K = M
-//   13  dA GEMM                       dA = dP W1p [M][k*k*C] fp32 (without a LayerNorm
-//                                     folded straight onto the patches: d_features)
+//   13  dA GEMM                       dA = dP W1p [M][k*k*C] bf16 (without a LayerNorm
+//                                     folded straight onto the patches in fp32: d_features)
 //   14  tails                         LayerNorm backward -> d_features and gamma / beta
 //                                     partials, column sums -> dgamma, dbeta; newline /
 //                                     separator gradients (db2, db1: row sums of dY^T and
@@ -374,18 +374,20 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     }
     VLP_CUDA(cudaEventRecord(h->join, ss));
 
-    // 13. dA = dP W1p (caller's stream): fp32, position-outer columns, for the LayerNorm
-    //     backward; without a LayerNorm the epilogue folds it onto the patches as the
-    //     feature gradient itself
+    // 13. dA = dP W1p (caller's stream): bf16, position-outer columns, for the LayerNorm
+    //     backward; without a LayerNorm the epilogue folds it (fp32) onto the patches as
+    //     the feature gradient itself
     if (want_da) {
         if (encode_bf16_2d(&tmA, dP1, M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
         p = gemm_params(h, M, K1, c.N1);
         stage_begin(h, 13, s);
         ++h->launches;
         if (c.has_ln) {
-            p.outf = h->dA.ptr;
-            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth, p,
-                                                           h->num_sms, s);
+            CUtensorMap tmD{};
+            if (encode_bf16_store(&tmD, h->dA.ptr, M, K1)) return VLPROJ_ERR_CUDA;
+            p.tma_store = 1;
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BF16>(pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth, p,
+                                                            h->num_sms, s, tmD);
         } else {
             p.outf = a->d_features;
             p.gmeta = h->gmeta.ptr;
