@@ -345,6 +345,12 @@ int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns);
 #define VLPROJ_NUM_STAGES 15
 int vlproj_profile_enable(vlproj_handle* h, int enable);
 
+/* Which stages record events while profiling is on: bit i = stage i (default: all).
+ * Each timed stage adds two event records to the stream, which separate its kernel
+ * from its neighbours; timing only the stages of interest keeps that cost off the
+ * others. Stages outside the mask read 0 in vlproj_profile_read. */
+int vlproj_profile_stages(vlproj_handle* h, uint32_t mask);
+
 /* Synchronise the stream of the most recent profiled call and write the elapsed
  * milliseconds of each stage into ms[0 .. min(n, VLPROJ_NUM_STAGES)); a stage that did
  * not run reads 0. Returns the number of values written, or an error code. */

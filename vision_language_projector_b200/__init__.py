@@ -27,7 +27,7 @@ EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status",
             "vlproj_image_rows", "vlproj_set_wait_limit", "vlproj_strerror", "vlproj_version",
             "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
             "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc", "vlproj_forward_ex",
-            "vlproj_plan_tiles", "vlproj_backward", "vlproj_project_host")
+            "vlproj_plan_tiles", "vlproj_backward", "vlproj_project_host", "vlproj_profile_stages")
 NOALLOC_MAX_IDS = 64 * 1024 * 1024
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX = 0, 1, 2, 3
 NUM_STAGES = 15
@@ -111,6 +111,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_version.restype = ctypes.c_char_p
     lib.vlproj_profile_enable.argtypes = [P, ctypes.c_int]
     lib.vlproj_profile_enable.restype = ctypes.c_int
+    lib.vlproj_profile_stages.argtypes = [P, ctypes.c_uint32]
+    lib.vlproj_profile_stages.restype = ctypes.c_int
     lib.vlproj_profile_read.argtypes = [P, P, ctypes.c_int]
     lib.vlproj_profile_read.restype = ctypes.c_int
     lib.vlproj_launch_count.argtypes = [P]
@@ -342,6 +344,13 @@ class Projector:
         rc = _lib.vlproj_profile_enable(self._h, int(enable))
         if rc != OK:
             raise VlprojError(rc, "vlproj_profile_enable")
+
+    def profile_stages(self, names=None) -> None:
+        """Time only the named stages (STAGES names; None = all) while profiling."""
+        mask = 0xFFFFFFFF if names is None else sum(1 << STAGES.index(n) for n in names)
+        rc = _lib.vlproj_profile_stages(self._h, mask)
+        if rc != OK:
+            raise VlprojError(rc, "vlproj_profile_stages")
 
     def stage_ms(self) -> dict:
         """Per-stage device milliseconds of the most recent profiled call (synchronises)."""

@@ -438,6 +438,7 @@ struct vlproj_handle {
     cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr;
     // tracing: start / end event of every stage, recorded on the stream that runs it
     bool profiling = false;
+    uint32_t profile_mask = ~0u;         // stages that record events while profiling
     bool profiled_valid = false;
     cudaEvent_t ev_begin[VLPROJ_NUM_STAGES] = {};
     cudaEvent_t ev_end[VLPROJ_NUM_STAGES] = {};
@@ -469,11 +470,11 @@ namespace vlp_host {
 
 // Stage timing: begin / end events on the stream that runs the stage.
 inline void stage_begin(vlproj_handle* h, int stage, cudaStream_t s) {
-    h->stage_ran[stage] = true;
-    if (h->profiling) cudaEventRecord(h->ev_begin[stage], s);
+    h->stage_ran[stage] = ((h->profile_mask >> stage) & 1u) != 0;
+    if (h->profiling && ((h->profile_mask >> stage) & 1u)) cudaEventRecord(h->ev_begin[stage], s);
 }
 inline void stage_end(vlproj_handle* h, int stage, cudaStream_t s) {
-    if (h->profiling) cudaEventRecord(h->ev_end[stage], s);
+    if (h->profiling && ((h->profile_mask >> stage) & 1u)) cudaEventRecord(h->ev_end[stage], s);
 }
 
 // LayerNorm-merge launch: the single-pass (registers) form when C fits.

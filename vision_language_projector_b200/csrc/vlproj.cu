@@ -623,6 +623,13 @@ int vlproj_profile_enable(vlproj_handle* h, int enable) {
     return VLPROJ_OK;
 }
 
+int vlproj_profile_stages(vlproj_handle* h, uint32_t mask) {
+    if (!h) return VLPROJ_ERR_INVALID_ARG;
+    h->profile_mask = mask;
+    h->profiled_valid = false;
+    return VLPROJ_OK;
+}
+
 int vlproj_profile_read(vlproj_handle* h, float* ms, int n) {
     if (!h || !ms || n < 0) return VLPROJ_ERR_INVALID_ARG;
     if (!h->profiled_valid) return VLPROJ_ERR_INVALID_ARG;
