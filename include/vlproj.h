@@ -18,7 +18,10 @@
  *      by a newline ("port DeepSeek-VL2", Tile-sequence assembly);
  *   5. the assembled rows overwrite the embedding rows that hold the image
  *      placeholder id, in order ("port DeepSeek-VL2", end of Tile-sequence
- *      assembly; image_token_index 100015).
+ *      assembly; image_token_index 100015);
+ *   6. the gradients of the projector's parameters and of the features, for
+ *      training the projector between a frozen tower and a frozen language model
+ *      ("DeepSeek-V4-Flash-Vision-BF16", opening section): vlproj_backward.
  *
  * Number formats: bf16 operands, fp32 accumulation, bf16 hidden activation
  * and bf16 output rows. Everything below runs on the GPU; there is no CPU path.
@@ -33,7 +36,9 @@
  *     stream). Work is enqueued asynchronously; the caller keeps every
  *     borrowed device buffer alive until that stream's work completes.
  *   - A handle is bound to the device that was current at vlproj_create and
- *     is not thread-safe: one thread at a time per handle.
+ *     is not thread-safe: one thread at a time per handle. Its calls share the
+ *     handle's scratch buffers, so successive calls go on one stream (or on
+ *     streams the caller orders); calls on different handles are independent.
  */
 #ifndef VLPROJ_H
 #define VLPROJ_H
