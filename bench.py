@@ -440,8 +440,14 @@ def main():
             shapes.update(newline=(wl.N2,), sep=(wl.N2,))
         grads = {n: torch.empty(sh, dtype=torch.float32, device="cuda") for n, sh in shapes.items()}
 
+        from vision_language_projector_b200.shard import allreduce_gradients
+        weight_grads = {n: t for n, t in grads.items() if n != "features"}
+
         def bstep():
             proj.backward(feats, hw, crop, ids, W.IMAGE_TOKEN_ID, d_out, grads, stream=stream, n_images=wl.n_images)
+            if world > 1:
+                # data-parallel training step: the ranks' weight gradients summed (one NCCL all-reduce)
+                allreduce_gradients(weight_grads)
 
         for _ in range(3):
             bstep()
@@ -479,7 +485,8 @@ def main():
                "flops_per_step": b_flops, "steps": args.backward_steps, "gradients": sorted(shapes),
                "stage_ms": {k_: statistics.mean(v) for k_, v in b_stage.items()},
                "what": "vlproj_backward: GEMM1 recompute, dP, dW2, dW1, dA, LayerNorm backward, bias and "
-                       "newline/separator sums; d_out ~N(0,1) bf16 on every id"}
+                       "newline/separator sums; d_out ~N(0,1) bf16 on every id"
+                       + ("; plus the all-reduce of the weight gradients over the ranks" if world > 1 else "")}
         del grads, d_out
 
     # ---- CPU oracle baseline (rank 0, one GPU only)

@@ -1,6 +1,8 @@
 """Multi-rank host logic on CPU: two gloo ranks split a batch by sequence, each
-projects its shard with the oracle, and the gathered shards equal the whole batch.
-No GPU and no data-path collective: the all_gather only collects results to check."""
+projects its shard with the oracle, and the gathered shards equal the whole batch
+(no data-path collective: the all_gather only collects results to check). For
+data-parallel training, each rank's backward of its shard, summed over ranks by
+allreduce_gradients, equals the backward of the whole batch."""
 import os
 import socket
 
@@ -12,7 +14,8 @@ import torch.multiprocessing as mp
 
 import workloads as W
 from oracle import projector as O
-from vision_language_projector_b200.shard import plan_shard, sequence_block
+from oracle import backward as B
+from vision_language_projector_b200.shard import allreduce_gradients, plan_shard, sequence_block
 
 
 def _free_port():
@@ -85,3 +88,50 @@ def test_two_gloo_ranks_reassemble_the_batch():
         covered[a:b] = True
     assert covered.all()
     np.testing.assert_array_equal(got, whole)
+
+
+def _grad_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl, hw, crop, rows, ids, feats, w, emb = _case()
+        per_seq = wl.n_images // wl.B
+        image_seq = [i // per_seq for i in range(wl.n_images)]
+        sh = plan_shard(image_seq, [wl.views_per_image] * wl.n_images, hw, wl.B, wl.S, world, rank)
+        d_out = O.bf16_bits_to_f64(W.grad_out(wl, len(ids)))
+        params = O.params_f64(w)
+        params["mid"] = [(np.ones((wl.N1, wl.N1)) * 0.01, np.zeros(wl.N1))]       # depth 3
+        g = B.backward(feats[sh.patches], hw[sh.views], crop[sh.images], wl.k, params, ids[sh.ids],
+                       W.IMAGE_TOKEN_ID, d_out[sh.ids])
+        mine = {k: torch.from_numpy(g[k]) for k in ("W1", "b1", "W2", "b2", "gamma", "beta", "newline", "sep")}
+        mine["W_mid"] = [torch.from_numpy(g["mid"][0][0])]
+        mine["b_mid"] = [torch.from_numpy(g["mid"][0][1])]
+        allreduce_gradients(mine)
+        if rank == 0:
+            out.put({k: ([t.numpy().tolist() for t in v] if isinstance(v, list) else v.numpy().tolist())
+                     for k, v in mine.items()})
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_sum_to_the_batch_gradient():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_grad_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    wl, hw, crop, rows, ids, feats, w, emb = _case()
+    params = O.params_f64(w)
+    params["mid"] = [(np.ones((wl.N1, wl.N1)) * 0.01, np.zeros(wl.N1))]
+    want = B.backward(feats, hw, crop, wl.k, params, ids, W.IMAGE_TOKEN_ID,
+                      O.bf16_bits_to_f64(W.grad_out(wl, len(ids))))
+    for k in ("W1", "b1", "W2", "b2", "gamma", "beta", "newline", "sep"):
+        np.testing.assert_allclose(np.array(got[k]), want[k], rtol=1e-12, atol=1e-12, err_msg=k)
+    np.testing.assert_allclose(np.array(got["W_mid"][0]), want["mid"][0][0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(np.array(got["b_mid"][0]), want["mid"][0][1], rtol=1e-12, atol=1e-12)

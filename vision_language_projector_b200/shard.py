@@ -1,9 +1,15 @@
-"""Partition one batch across ranks by sequence (host logic, no device work).
+"""Partition one batch across ranks by sequence (host logic, no device work), and the
+one exchange that data-parallel training of the projector has.
 
 Images are independent units and every image's placeholder run lies inside one
 sequence, so a batch splits into contiguous blocks of sequences with no exchange:
 rank r projects the images whose runs lie in its sequences into its slice of the
 embedding buffer. ``plan_shard`` returns the slices of every input a rank needs.
+
+Training the projector on such shards, each rank's ``Projector.backward`` gives the
+gradients of its sequences' share of the loss; the batch gradient of every parameter
+is their sum over ranks (the loss is a sum over rows). ``allreduce_gradients`` adds
+them in place across the process group (NCCL on GPUs) in one flat buffer.
 """
 from __future__ import annotations
 
@@ -48,3 +54,27 @@ def plan_shard(image_seq: Sequence[int], views_per_image: Sequence[int], grid_hw
     pcum = np.concatenate([[0], np.cumsum(grid_hw[:, 0] * grid_hw[:, 1])])
     return Shard(rank, s, slice(s.start * seq_len, s.stop * seq_len), slice(i0, i1), slice(v0, v1),
                  slice(int(pcum[v0]), int(pcum[v1])))
+
+
+def allreduce_gradients(grads: dict, group=None) -> None:
+    """Sum every gradient tensor of ``grads`` over the ranks of ``group`` in place.
+
+    Values may be tensors or lists of tensors (the middle layers' "W_mid" / "b_mid"),
+    all of one dtype and device; keys are visited in sorted order on every rank. The
+    tensors are packed into one buffer, so the exchange is a single all-reduce."""
+    import torch
+    import torch.distributed as dist
+
+    tensors = []
+    for key in sorted(grads):
+        v = grads[key]
+        tensors.extend(v if isinstance(v, (list, tuple)) else [v])
+    if not tensors:
+        return
+    flat = torch.cat([t.reshape(-1) for t in tensors])
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    offset = 0
+    for t in tensors:
+        n = t.numel()
+        t.copy_(flat[offset:offset + n].view_as(t))
+        offset += n
