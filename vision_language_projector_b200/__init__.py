@@ -321,7 +321,6 @@ class Projector:
         c = _host_i32(spatial_crop)
         if n_images is None:
             n_images = len(c) if c is not None else (0 if g is None else len(g))
-        self._host_keep = (g, c)           # the host tables must outlive the enqueue only
         a = HostArgs(_ptr(features), _ptr(g), _ptr(c), n_images, _ptr(newline), _ptr(sep), _ptr(rows_out),
                      0 if rows_out is None else int(rows_out.shape[0]), int(chunks))
         rc = _lib.vlproj_project_host(self._h, ctypes.byref(a), _stream_ptr(stream))
