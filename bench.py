@@ -41,7 +41,7 @@ DEFAULT_WORKLOAD = "moonvit"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the sources that decide the GEMMs' DRAM traffic (kernel, its PTX, its launch and raster)
 KERNEL_SOURCES = [os.path.join("vision_language_projector_b200", "csrc", f)
-                  for f in ("gemm_sm100.cuh", "gelu_poly.cuh", "ptx.cuh", "host.cuh")]
+                  for f in ("gemm_sm100.cuh", "gelu_poly.cuh", "ptx.cuh", "host.cuh", "kernels_aux.cuh")]
 
 
 def parse_args():
@@ -380,7 +380,8 @@ def main():
         achieved = None if b is None else b / (avg[dom] / 1000.0) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
                 "frac": None if achieved is None else achieved / peaks.get("hbm_gbs"),
-                "peak_source": f"{peak_src} HBM copy", "traffic": None, "algorithmic_bytes": b}
+                "peak_source": f"{peak_src} HBM copy", "traffic": traffic_from_profiles(args.workload, dom),
+                "algorithmic_bytes": b}
 
     # ---- end to end through the public API with host buffers: vlproj_project_host takes the
     # step's features from pinned host memory and returns the assembled rows of every image to

@@ -431,6 +431,7 @@ struct vlproj_handle {
     vlp_host::DevBuf<vlp::ImageDesc> dimages;
     vlp_host::DevBuf<CUtensorMap> dmaps;
     int* status = nullptr;       // [0] latched error, [1] per-forward count check
+    int lnp_per_sm = 0;          // resident blocks per SM of the LayerNorm-merge kernel (0: not queried)
     vlp_host::Uploader up_views, up_images, up_maps;
     std::vector<CUtensorMap> host_maps;
     // the placeholder index runs on `side`, forked from / joined to the caller's stream
@@ -477,20 +478,57 @@ inline void stage_end(vlproj_handle* h, int stage, cudaStream_t s) {
     if (h->profiling && ((h->profile_mask >> stage) & 1u)) cudaEventRecord(h->ev_end[stage], s);
 }
 
-// LayerNorm-merge launch: the single-pass (registers) form when C fits.
-inline int launch_ln_merge(const vlproj_config& c, const void* features, const int2* gmeta, int M, const float* gamma,
-                    const float* beta, float eps, __nv_bfloat16* A, cudaStream_t s) {
+// LayerNorm-merge launch: the pipelined form when C fits (C <= 2048), a grid of the
+// blocks that fit on the SMs at once, each warp with a ring of about 9 KB of patch rows
+// (2 to 16 rows; MoonViT's 2304-byte rows: 4 per warp, 2 blocks per SM, measured
+// faster than 3 rows at 3 blocks, 5 rows at 2 and 8 rows at 1); the two-pass form
+// beyond. The kernel's shared-memory attribute and
+// occupancy are set up on the handle's first launch (the configuration fixes both).
+template <bool F32, int V>
+inline int launch_ln_merge_pipe(vlproj_handle* h, const void* features, int M, float eps, __nv_bfloat16* A,
+                                cudaStream_t s) {
+    const vlproj_config& c = h->cfg;
     const int64_t items = static_cast<int64_t>(M) * c.k * c.k;
-    const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+    const size_t row_bytes = static_cast<size_t>(c.C) * (F32 ? 4 : 2);
+    const int stages = static_cast<int>(std::min<size_t>(vlp::LNP_MAX_STAGES,
+                                                         std::max<size_t>(2, (9u << 10) / row_bytes)));
+    const size_t smem = vlp::LNP_BAR_BYTES + (c.has_ln ? 8 * static_cast<size_t>(c.C) : 0) +
+                        static_cast<size_t>(vlp::LNP_WARPS) * stages * row_bytes;
+    auto kern = vlp::vlp_ln_merge_pipe_kernel<F32, V>;
+    if (h->lnp_per_sm == 0) {
+        VLP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+        VLP_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->lnp_per_sm, kern, vlp::LNP_WARPS * 32, smem));
+        h->lnp_per_sm = std::max(h->lnp_per_sm, 1);
+    }
+    const int64_t want = (items + vlp::LNP_WARPS - 1) / vlp::LNP_WARPS;
+    const unsigned blocks =
+        static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(h->num_sms) * h->lnp_per_sm)));
+    kern<<<blocks, vlp::LNP_WARPS * 32, smem, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma, h->beta, eps,
+                                                  c.has_ln, A, stages, h->wait_ns, h->status);
+    VLP_CUDA(cudaGetLastError());
+    return VLPROJ_OK;
+}
+
+inline int launch_ln_merge(vlproj_handle* h, const void* features, int M, float eps, __nv_bfloat16* A,
+                           cudaStream_t s) {
+    const vlproj_config& c = h->cfg;
+    const int64_t items = static_cast<int64_t>(M) * c.k * c.k;
+    if (items == 0) return VLPROJ_OK;
     const int nvec = c.C / 8;
     const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
-#define VLP_LNM(F, V) vlp::vlp_ln_merge_regs_kernel<F, V><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A)
-    if (nvec <= 64) { if (f32) VLP_LNM(true, 2); else VLP_LNM(false, 2); }
-    else if (nvec <= 160) { if (f32) VLP_LNM(true, 5); else VLP_LNM(false, 5); }
-    else if (nvec <= 256) { if (f32) VLP_LNM(true, 8); else VLP_LNM(false, 8); }
-    else if (f32) vlp::vlp_ln_merge_kernel<true><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A);
-    else vlp::vlp_ln_merge_kernel<false><<<blocks, 256, 0, s>>>(features, gmeta, M, c.k, c.C, gamma, beta, eps, c.has_ln, A);
-#undef VLP_LNM
+    if (nvec <= 64) return f32 ? launch_ln_merge_pipe<true, 2>(h, features, M, eps, A, s)
+                               : launch_ln_merge_pipe<false, 2>(h, features, M, eps, A, s);
+    if (nvec <= 160) return f32 ? launch_ln_merge_pipe<true, 5>(h, features, M, eps, A, s)
+                                : launch_ln_merge_pipe<false, 5>(h, features, M, eps, A, s);
+    if (nvec <= 256) return f32 ? launch_ln_merge_pipe<true, 8>(h, features, M, eps, A, s)
+                                : launch_ln_merge_pipe<false, 8>(h, features, M, eps, A, s);
+    const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+    if (f32)
+        vlp::vlp_ln_merge_kernel<true><<<blocks, 256, 0, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma, h->beta,
+                                                              eps, c.has_ln, A);
+    else
+        vlp::vlp_ln_merge_kernel<false><<<blocks, 256, 0, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma,
+                                                               h->beta, eps, c.has_ln, A);
     VLP_CUDA(cudaGetLastError());
     return VLPROJ_OK;
 }

@@ -13,6 +13,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace vlp {
 
 constexpr int ERR_TOKEN_COUNT = -4;
@@ -186,8 +188,146 @@ static __global__ void __launch_bounds__(256) vlp_geometry_kernel(const ViewDesc
 }
 
 // ---------------------------------------------------------------- LayerNorm / convert
-// One warp per patch row: y = bf16(((x - mean) * rstd) * gamma + beta) (biased
-// variance, fp32 statistics) or, without LayerNorm, y = bf16(x). C % 8 == 0.
+// y = bf16(((x - mean) * rstd) * gamma + beta) per patch row, biased variance, fp32
+// statistics, or y = bf16(x) without a LayerNorm; C % 8 == 0. One warp per row; lane l
+// owns the 8-channel vectors v = l, l + 32, ... and works on channel pairs (2e, 2e+1)
+// held as packed fp32x2, two channels per add / mul / fma instruction.
+//
+// Every kernel below reduces in the same order, so they produce the same bits: a
+// lane accumulates its vectors in increasing v into an (even, odd) pair of sums,
+// adds the pair, and the warp combines lanes by an xor tree; the sum of squared
+// deviations from the mean likewise.
+
+// The 8 channels of vector v of a row as 4 packed pairs.
+template <bool kF32In>
+__device__ __forceinline__ void ln_load_pairs(const void* __restrict__ x, int64_t row, int C, int v,
+                                              uint64_t (&q)[4]) {
+    if (kF32In) {
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * C) + 2 * v;
+        const float4 a = __ldg(src), b = __ldg(src + 1);
+        q[0] = f2_pack(a.x, a.y);
+        q[1] = f2_pack(a.z, a.w);
+        q[2] = f2_pack(b.x, b.y);
+        q[3] = f2_pack(b.z, b.w);
+    } else {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + row * C) + v);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) q[e] = f2_pack(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+    }
+}
+
+// Same from a row staged in shared memory.
+template <bool kF32In>
+__device__ __forceinline__ void ln_smem_pairs(const uint8_t* st, int v, uint64_t (&q)[4]) {
+    if (kF32In) {
+        const float4 a = reinterpret_cast<const float4*>(st)[2 * v];
+        const float4 b = reinterpret_cast<const float4*>(st)[2 * v + 1];
+        q[0] = f2_pack(a.x, a.y);
+        q[1] = f2_pack(a.z, a.w);
+        q[2] = f2_pack(b.x, b.y);
+        q[3] = f2_pack(b.z, b.w);
+    } else {
+        const uint4 u = reinterpret_cast<const uint4*>(st)[v];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) q[e] = f2_pack(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+    }
+}
+
+// Sum of the pair accumulator's halves, then across the warp.
+__device__ __forceinline__ float ln_warp_total(uint64_t acc) {
+    float a, b;
+    f2_unpack(acc, a, b);
+    float t = a + b;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    return t;
+}
+
+// bf16 of 8 channels: d = x - mean (packed), y = (d * rstd) * gamma + beta, with
+// gamma / beta of the 8 channels in g0, g1 / b0, b1.
+__device__ __forceinline__ uint4 ln_out_pairs(const uint64_t (&d)[4], uint64_t rstd2, float4 g0, float4 g1, float4 b0,
+                                              float4 b1) {
+    const uint64_t gg[4] = {f2_pack(g0.x, g0.y), f2_pack(g0.z, g0.w), f2_pack(g1.x, g1.y), f2_pack(g1.z, g1.w)};
+    const uint64_t bb[4] = {f2_pack(b0.x, b0.y), f2_pack(b0.z, b0.w), f2_pack(b1.x, b1.y), f2_pack(b1.z, b1.w)};
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float lo, hi;
+        f2_unpack(f2_fma(f2_mul(d[e], rstd2), gg[e], bb[e]), lo, hi);
+        __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+        w[e] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// bf16 of 8 channels without a LayerNorm.
+__device__ __forceinline__ uint4 ln_convert_pairs(const uint64_t (&x)[4]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float lo, hi;
+        f2_unpack(x[e], lo, hi);
+        __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+        w[e] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Statistics of the row `row` read vector by vector from memory: mean, 1/sqrt(var + eps).
+template <bool kF32In>
+__device__ __forceinline__ void ln_row_stats(const void* __restrict__ x, int64_t row, int C, int lane, float eps,
+                                             float& mean, float& rstd) {
+    const int nvec = C / 8;
+    uint64_t acc = 0;
+    for (int v = lane; v < nvec; v += 32) {
+        uint64_t q[4];
+        ln_load_pairs<kF32In>(x, row, C, v, q);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc = f2_add(acc, q[e]);
+    }
+    const float inv_c = 1.0f / static_cast<float>(C);
+    mean = ln_warp_total(acc) * inv_c;
+    const uint64_t nm = f2_splat(-mean);
+    acc = 0;
+    for (int v = lane; v < nvec; v += 32) {
+        uint64_t q[4];
+        ln_load_pairs<kF32In>(x, row, C, v, q);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint64_t d = f2_add(q[e], nm);
+            acc = f2_fma(d, d, acc);
+        }
+    }
+    rstd = rsqrtf(ln_warp_total(acc) * inv_c + eps);
+}
+
+// Normalise row `row` of x into dst (bf16, C channels), re-reading x vector by vector.
+template <bool kF32In>
+__device__ __forceinline__ void ln_row_write(const void* __restrict__ x, int64_t row, int C, int lane,
+                                             const float* __restrict__ gamma, const float* __restrict__ beta,
+                                             float eps, int has_ln, uint4* __restrict__ dst) {
+    const int nvec = C / 8;
+    float mean = 0.f, rstd = 1.f;
+    if (has_ln) ln_row_stats<kF32In>(x, row, C, lane, eps, mean, rstd);
+    const uint64_t nm = f2_splat(-mean), r2 = f2_splat(rstd);
+    for (int v = lane; v < nvec; v += 32) {
+        uint64_t q[4];
+        ln_load_pairs<kF32In>(x, row, C, v, q);
+        if (has_ln) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) q[e] = f2_add(q[e], nm);
+            const float4* g4 = reinterpret_cast<const float4*>(gamma) + 2 * v;
+            const float4* b4 = reinterpret_cast<const float4*>(beta) + 2 * v;
+            dst[v] = ln_out_pairs(q, r2, __ldg(g4), __ldg(g4 + 1), __ldg(b4), __ldg(b4 + 1));
+        } else {
+            dst[v] = ln_convert_pairs(q);
+        }
+    }
+}
+
+// Patch order: row p of the features -> row p of y.
 template <bool kF32In>
 static __global__ void __launch_bounds__(256) vlp_layernorm_kernel(const void* __restrict__ x, int64_t P, int C,
                                                             const float* __restrict__ gamma,
@@ -196,78 +336,26 @@ static __global__ void __launch_bounds__(256) vlp_layernorm_kernel(const void* _
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (row >= P) return;
-    const int nvec = C / 8;
-    auto load8 = [&](int v, float (&f)[8]) {
-        if (kF32In) {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * C) + 2 * v;
-            const float4 a = __ldg(src), b = __ldg(src + 1);
-            f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-        } else {
-            const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + row * C) + v);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                f[2 * e] = __uint_as_float(w[e] << 16);
-                f[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-            }
-        }
-    };
-    float mean = 0.f, rstd = 1.f;
-    if (has_ln) {
-        float s = 0.f;
-        for (int v = lane; v < nvec; v += 32) {
-            float f[8];
-            load8(v, f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) s += f[e];
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        mean = s / static_cast<float>(C);
-        float q = 0.f;
-        for (int v = lane; v < nvec; v += 32) {
-            float f[8];
-            load8(v, f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float d = f[e] - mean;
-                q += d * d;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-        rstd = rsqrtf(q / static_cast<float>(C) + eps);
-    }
-    for (int v = lane; v < nvec; v += 32) {
-        float f[8];
-        load8(v, f);
-        if (has_ln) {
-            const float4* g4 = reinterpret_cast<const float4*>(gamma) + 2 * v;
-            const float4* b4 = reinterpret_cast<const float4*>(beta) + 2 * v;
-            const float4 g0 = __ldg(g4), g1 = __ldg(g4 + 1), b0 = __ldg(b4), b1 = __ldg(b4 + 1);
-            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = (f[e] - mean) * rstd * gg[e] + bb[e];
-        }
-        uint4 o;
-        __nv_bfloat162 t0 = __floats2bfloat162_rn(f[0], f[1]), t1 = __floats2bfloat162_rn(f[2], f[3]);
-        __nv_bfloat162 t2 = __floats2bfloat162_rn(f[4], f[5]), t3 = __floats2bfloat162_rn(f[6], f[7]);
-        o.x = *reinterpret_cast<uint32_t*>(&t0);
-        o.y = *reinterpret_cast<uint32_t*>(&t1);
-        o.z = *reinterpret_cast<uint32_t*>(&t2);
-        o.w = *reinterpret_cast<uint32_t*>(&t3);
-        reinterpret_cast<uint4*>(y + row * C)[v] = o;
-    }
+    ln_row_write<kF32In>(x, row, C, lane, gamma, beta, eps, has_ln, reinterpret_cast<uint4*>(y + row * C));
 }
 
 // ---------------------------------------------------------------- LayerNorm + merge
-// One warp per (merged token m, position p = dy*k + dx): the patch at (k*i+dy, k*j+dx)
-// of m's view (from gmeta), LayerNorm'd (when has_ln) and rounded to bf16, lands at
-// A[m][p*C : (p+1)*C]; positions in the high-end pad are written as zeros. Each
-// patch is read once, and A is GEMM1's operand in the kernel's K order. The
-// statistics and rounding are those of vlp_layernorm_kernel, so A holds exactly the
-// values the gathering paths read from its output.
+// Item (merged token m, position p = dy*k + dx): the patch at (k*i+dy, k*j+dx) of m's
+// view (from gmeta), LayerNorm'd (when has_ln) and rounded to bf16, lands at
+// A[m][p*C : (p+1)*C]; positions in the high-end pad are written as zeros. Each patch
+// is read from memory once and A is GEMM1's operand in the kernel's K order. Values
+// equal vlp_layernorm_kernel's output bit for bit, so A holds exactly what the
+// gathering paths read.
+
+// Source row of item (m, p), or -1 for a zero pad.
+__device__ __forceinline__ int64_t merge_source_row(const int2* __restrict__ gmeta, int m, int p, int k) {
+    const int2 g = __ldg(gmeta + m);
+    const uint32_t wm = static_cast<uint32_t>(g.y);
+    if (!((wm >> p) & 1u)) return -1;
+    return static_cast<int64_t>(g.x) + (p / k) * static_cast<int>(wm >> 16) + (p % k);
+}
+
+// Any C: one warp per item, the row re-read from memory for each pass.
 template <bool kF32In>
 static __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __restrict__ x, const int2* __restrict__ gmeta,
                                                            int M, int k, int C, const float* __restrict__ gamma,
@@ -278,175 +366,162 @@ static __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __
     const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (item >= static_cast<int64_t>(M) * kk) return;
     const int m = static_cast<int>(item / kk), p = static_cast<int>(item - static_cast<int64_t>(m) * kk);
-    const int dy = p / k, dx = p - dy * k;
-    const int2 g = gmeta[m];
-    const uint32_t wm = static_cast<uint32_t>(g.y);
-    const int nvec = C / 8;
-    uint4* dst = reinterpret_cast<uint4*>(A + (static_cast<int64_t>(m) * kk + p) * C);
-    if (!((wm >> p) & 1u)) {
-        for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+    uint4* dst = reinterpret_cast<uint4*>(A + item * C);
+    const int64_t row = merge_source_row(gmeta, m, p, k);
+    if (row < 0) {
+        for (int v = lane; v < C / 8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
         return;
     }
-    const int64_t row = static_cast<int64_t>(g.x) + dy * static_cast<int>(wm >> 16) + dx;
-    auto load8 = [&](int v, float (&f)[8]) {
-        if (kF32In) {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * C) + 2 * v;
-            const float4 a = __ldg(src), b = __ldg(src + 1);
-            f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-        } else {
-            const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + row * C) + v);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                f[2 * e] = __uint_as_float(w[e] << 16);
-                f[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-            }
-        }
-    };
-    float mean = 0.f, rstd = 1.f;
-    if (has_ln) {
-        float s = 0.f;
-        for (int v = lane; v < nvec; v += 32) {
-            float f[8];
-            load8(v, f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) s += f[e];
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        mean = s / static_cast<float>(C);
-        float q = 0.f;
-        for (int v = lane; v < nvec; v += 32) {
-            float f[8];
-            load8(v, f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float d = f[e] - mean;
-                q += d * d;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-        rstd = rsqrtf(q / static_cast<float>(C) + eps);
-    }
-    for (int v = lane; v < nvec; v += 32) {
-        float f[8];
-        load8(v, f);
-        if (has_ln) {
-            const float4* g4 = reinterpret_cast<const float4*>(gamma) + 2 * v;
-            const float4* b4 = reinterpret_cast<const float4*>(beta) + 2 * v;
-            const float4 g0 = __ldg(g4), g1 = __ldg(g4 + 1), b0 = __ldg(b4), b1 = __ldg(b4 + 1);
-            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = (f[e] - mean) * rstd * gg[e] + bb[e];
-        }
-        uint4 o;
-        __nv_bfloat162 t0 = __floats2bfloat162_rn(f[0], f[1]), t1 = __floats2bfloat162_rn(f[2], f[3]);
-        __nv_bfloat162 t2 = __floats2bfloat162_rn(f[4], f[5]), t3 = __floats2bfloat162_rn(f[6], f[7]);
-        o.x = *reinterpret_cast<uint32_t*>(&t0);
-        o.y = *reinterpret_cast<uint32_t*>(&t1);
-        o.z = *reinterpret_cast<uint32_t*>(&t2);
-        o.w = *reinterpret_cast<uint32_t*>(&t3);
-        dst[v] = o;
-    }
+    ln_row_write<kF32In>(x, row, C, lane, gamma, beta, eps, has_ln, dst);
 }
 
-// Single-pass form of vlp_ln_merge_kernel for C <= 256 * kVec: each lane keeps its
-// kVec 8-channel vectors of the patch in registers, so the patch is read from memory
-// once. Same statistics (sum, then sum of squared deviations, in fp32) and rounding.
+// Pipelined form for C <= 256 * kVec. Items are dealt to warps with a stride of the
+// grid's warp count; each warp keeps up to `stages` of its next patch rows in flight in
+// a shared-memory ring of its own, fetched by 1D bulk copies that complete on one
+// mbarrier per slot, so a grid of resident blocks keeps the memory system busy while
+// the warps normalise. A row is read from its slot once into registers (kVec vectors of
+// 4 packed pairs per lane). gamma / beta are staged once per block in shared memory as
+// four arrays of float4 (channels 8v..8v+3 and 8v+4..8v+7 of each), so that a warp's
+// reads of one of them are consecutive. A wait that runs out latches
+// VLPROJ_ERR_TIMEOUT in *err, waits (bounded) for the warp's copies still in flight
+// and ends the warp. Shared memory: LNP_BAR_BYTES, then 8 C bytes of gamma / beta
+// when has_ln, then the rings.
+constexpr int LNP_WARPS = 8;
+constexpr int LNP_MAX_STAGES = 16;
+constexpr int LNP_BAR_BYTES = LNP_WARPS * LNP_MAX_STAGES * 8;
+
 template <bool kF32In, int kVec>
-static __global__ void __launch_bounds__(256) vlp_ln_merge_regs_kernel(const void* __restrict__ x,
-                                                                const int2* __restrict__ gmeta, int M, int k, int C,
-                                                                const float* __restrict__ gamma,
-                                                                const float* __restrict__ beta, float eps, int has_ln,
-                                                                __nv_bfloat16* __restrict__ A) {
-    const int lane = threadIdx.x & 31;
+static __global__ void __launch_bounds__(LNP_WARPS * 32, kVec > 5 ? 2 : 3) vlp_ln_merge_pipe_kernel(
+    const void* __restrict__ x, const int2* __restrict__ gmeta, int M, int k, int C, const float* __restrict__ gamma,
+    const float* __restrict__ beta, float eps, int has_ln, __nv_bfloat16* __restrict__ A, int stages,
+    uint64_t wait_ns, int* err) {
+    extern __shared__ __align__(128) uint8_t lnp_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int kk = k * k;
-    const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (item >= static_cast<int64_t>(M) * kk) return;
-    const int m = static_cast<int>(item / kk), p = static_cast<int>(item - static_cast<int64_t>(m) * kk);
-    const int dy = p / k, dx = p - dy * k;
-    const int2 g = gmeta[m];
-    const uint32_t wm = static_cast<uint32_t>(g.y);
     const int nvec = C / 8;
-    uint4* dst = reinterpret_cast<uint4*>(A + (static_cast<int64_t>(m) * kk + p) * C);
-    if (!((wm >> p) & 1u)) {
-        for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
-        return;
-    }
-    const int64_t row = static_cast<int64_t>(g.x) + dy * static_cast<int>(wm >> 16) + dx;
-    float f[kVec][8];
-#pragma unroll
-    for (int i = 0; i < kVec; ++i) {
-        const int v = lane + 32 * i;
-        if (v < nvec) {
-            if (kF32In) {
-                const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * C) + 2 * v;
-                const float4 a = __ldg(src), b = __ldg(src + 1);
-                f[i][0] = a.x; f[i][1] = a.y; f[i][2] = a.z; f[i][3] = a.w;
-                f[i][4] = b.x; f[i][5] = b.y; f[i][6] = b.z; f[i][7] = b.w;
-            } else {
-                const uint4 u =
-                    __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + row * C) + v);
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    f[i][2 * e] = __uint_as_float(w[e] << 16);
-                    f[i][2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-                }
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[i][e] = 0.f;
+    const int64_t total = static_cast<int64_t>(M) * kk;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * LNP_WARPS;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * LNP_WARPS + warp;
+    float4* gb = reinterpret_cast<float4*>(lnp_smem + LNP_BAR_BYTES);     // [4][nvec]
+    if (has_ln) {
+        for (int v = threadIdx.x; v < nvec; v += LNP_WARPS * 32) {
+            const float4* g4 = reinterpret_cast<const float4*>(gamma) + 2 * v;
+            const float4* b4 = reinterpret_cast<const float4*>(beta) + 2 * v;
+            gb[v] = __ldg(g4);
+            gb[nvec + v] = __ldg(g4 + 1);
+            gb[2 * nvec + v] = __ldg(b4);
+            gb[3 * nvec + v] = __ldg(b4 + 1);
         }
     }
-    float mean = 0.f, rstd = 1.f;
-    if (has_ln) {
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < kVec; ++i)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) s += f[i][e];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        mean = s / static_cast<float>(C);
-        float q = 0.f;
+    __syncthreads();
+    if (gw >= total) return;
+    const int n_items = static_cast<int>((total - gw + nwarps - 1) / nwarps);
+    const uint32_t row_bytes = static_cast<uint32_t>(C) * (kF32In ? 4u : 2u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(lnp_smem) + warp * LNP_MAX_STAGES;
+    uint8_t* ring = lnp_smem + LNP_BAR_BYTES + (has_ln ? 8 * C : 0) + static_cast<size_t>(warp) * stages * row_bytes;
+    const uint8_t* xb = static_cast<const uint8_t*>(x);
+    if (lane == 0) {
+        for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // Lane l holds the source row of the warp's item (32 b + l), -1 for a zero pad.
+    int64_t batch_row = -1;
+    uint32_t loaded = 0, phase = 0;     // per slot: a copy was issued / parity to wait for
+    int si = 0;                         // slot of the next issue (j mod stages)
+    auto issue = [&](int j) {           // warp-uniform, called for j = 0, 1, 2, ... in order
+        const int s = si;
+        si = si + 1 == stages ? 0 : si + 1;
+        if (j >= n_items) {
+            loaded &= ~(1u << s);
+            return;
+        }
+        if ((j & 31) == 0) {
+            batch_row = -1;
+            if (j + lane < n_items) {
+                const int64_t it = gw + static_cast<int64_t>(j + lane) * nwarps;
+                const int m = static_cast<int>(it / kk);
+                batch_row = merge_source_row(gmeta, m, static_cast<int>(it - static_cast<int64_t>(m) * kk), k);
+            }
+        }
+        const int64_t r = __shfl_sync(0xffffffffu, batch_row, j & 31);
+        if (r >= 0) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars[s], row_bytes);
+                bulk_load_1d(ring + static_cast<size_t>(s) * row_bytes, xb + r * row_bytes, row_bytes, &bars[s]);
+            }
+            loaded |= 1u << s;
+        } else {
+            loaded &= ~(1u << s);
+        }
+    };
+    for (int j = 0; j < stages; ++j) issue(j);
+
+    const uint64_t zero2 = 0;
+    const float inv_c = 1.0f / static_cast<float>(C);
+    const int64_t dst_step = nwarps * C / 8;            // uint4 between a warp's items
+    uint4* dst = reinterpret_cast<uint4*>(A + gw * C);
+    for (int j = 0, s = 0; j < n_items; ++j, s = s + 1 == stages ? 0 : s + 1, dst += dst_step) {
+        if (!((loaded >> s) & 1u)) {            // neighbour outside the grid: zeros
+            issue(j + stages);
+            for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+            continue;
+        }
+        if (!mbar_wait_limit(&bars[s], (phase >> s) & 1u, wait_ns)) {
+            if (lane == 0) atomicCAS(err, 0, -5);
+            for (int t = 0; t < stages; ++t)        // drain the copies still landing
+                if (((loaded >> t) & 1u) && t != s) mbar_wait_limit(&bars[t], (phase >> t) & 1u, wait_ns);
+            mbar_wait_limit(&bars[s], (phase >> s) & 1u, wait_ns);
+            return;
+        }
+        phase ^= 1u << s;
+        const uint8_t* st = ring + static_cast<size_t>(s) * row_bytes;
+        uint64_t q[kVec][4];
 #pragma unroll
         for (int i = 0; i < kVec; ++i) {
             if (lane + 32 * i < nvec) {
+                ln_smem_pairs<kF32In>(st, lane + 32 * i, q[i]);
+            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float d = f[i][e] - mean;
-                    q += d * d;
-                }
+                for (int e = 0; e < 4; ++e) q[i][e] = zero2;
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-        rstd = rsqrtf(q / static_cast<float>(C) + eps);
-    }
-#pragma unroll
-    for (int i = 0; i < kVec; ++i) {
-        const int v = lane + 32 * i;
-        if (v >= nvec) continue;
+        // the slot's bytes are in registers: order those reads before the next copy into it
+        fence_proxy_async_smem();
+        __syncwarp();
+        issue(j + stages);
+
+        float rstd = 1.f;
         if (has_ln) {
-            const float4* g4 = reinterpret_cast<const float4*>(gamma) + 2 * v;
-            const float4* b4 = reinterpret_cast<const float4*>(beta) + 2 * v;
-            const float4 g0 = __ldg(g4), g1 = __ldg(g4 + 1), b0 = __ldg(b4), b1 = __ldg(b4 + 1);
-            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            uint64_t acc = 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[i][e] = (f[i][e] - mean) * rstd * gg[e] + bb[e];
+            for (int i = 0; i < kVec; ++i)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc = f2_add(acc, q[i][e]);
+            const float mean = ln_warp_total(acc) * inv_c;
+            const uint64_t nm = f2_splat(-mean);
+            acc = 0;
+#pragma unroll
+            for (int i = 0; i < kVec; ++i) {
+                if (lane + 32 * i < nvec) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        q[i][e] = f2_add(q[i][e], nm);          // keep d = x - mean
+                        acc = f2_fma(q[i][e], q[i][e], acc);
+                    }
+                }
+            }
+            rstd = rsqrtf(ln_warp_total(acc) * inv_c + eps);
         }
-        uint4 o;
-        __nv_bfloat162 t0 = __floats2bfloat162_rn(f[i][0], f[i][1]), t1 = __floats2bfloat162_rn(f[i][2], f[i][3]);
-        __nv_bfloat162 t2 = __floats2bfloat162_rn(f[i][4], f[i][5]), t3 = __floats2bfloat162_rn(f[i][6], f[i][7]);
-        o.x = *reinterpret_cast<uint32_t*>(&t0);
-        o.y = *reinterpret_cast<uint32_t*>(&t1);
-        o.z = *reinterpret_cast<uint32_t*>(&t2);
-        o.w = *reinterpret_cast<uint32_t*>(&t3);
-        dst[v] = o;
+        const uint64_t r2 = f2_splat(rstd);
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) {
+            const int v = lane + 32 * i;
+            if (v >= nvec) continue;
+            dst[v] = has_ln ? ln_out_pairs(q[i], r2, gb[v], gb[nvec + v], gb[2 * nvec + v], gb[3 * nvec + v])
+                            : ln_convert_pairs(q[i]);
+        }
     }
 }
 

@@ -54,7 +54,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
         ++h->launches;
         if (h->A.ensure(static_cast<size_t>(M) * h->K1)) return VLPROJ_ERR_CUDA;
         const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
-        int rc = launch_ln_merge(c, features, h->gmeta.ptr, M, h->gamma, h->beta, eps, h->A.ptr, s);
+        int rc = launch_ln_merge(h, features, M, eps, h->A.ptr, s);
         if (rc) return rc;
         stage_end(h, 2, s);
     } else if (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) {
