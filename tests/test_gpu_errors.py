@@ -106,3 +106,19 @@ def test_bounded_wait_timeout_then_recovery():
     out = run(case, proj, dev)
     assert proj.status() == vp.OK
     check(case, out, dev)
+
+
+def test_wait_bound_runs_out_in_layernorm_merge():
+    """The same with a LayerNorm: the LayerNorm-merge kernel's ring waits run out too; it
+    latches VLPROJ_ERR_TIMEOUT, lets the copies already issued land, and returns."""
+    wl = custom("timeout_ln", 113, 2, 1152, 256, 128, 4, 2, 800, has_ln=True)
+    case = make_case(wl, np.array([[24, 24]] * 4, np.int32))
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    proj.set_wait_limit(1)
+    run(case, proj, dev)
+    assert proj.status() == vp.ERR_TIMEOUT
+    proj.set_wait_limit(0)
+    out = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    check(case, out, dev)

@@ -383,12 +383,13 @@ static __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __
 // 4 packed pairs per lane). gamma / beta are staged once per block in shared memory as
 // four arrays of float4 (channels 8v..8v+3 and 8v+4..8v+7 of each), so that a warp's
 // reads of one of them are consecutive. A wait that runs out latches
-// VLPROJ_ERR_TIMEOUT in *err, waits (bounded) for the warp's copies still in flight
-// and ends the warp. Shared memory: LNP_BAR_BYTES, then 8 C bytes of gamma / beta
-// when has_ln, then the rings.
+// VLPROJ_ERR_TIMEOUT in *err, waits for the warp's copies still in flight (bounded by
+// LNP_DRAIN_NS, not by the wait bound) and ends the warp. Shared memory: LNP_BAR_BYTES,
+// then 8 C bytes of gamma / beta when has_ln, then the rings.
 constexpr int LNP_WARPS = 8;
 constexpr int LNP_MAX_STAGES = 16;
 constexpr int LNP_BAR_BYTES = LNP_WARPS * LNP_MAX_STAGES * 8;
+constexpr uint64_t LNP_DRAIN_NS = 1000000000ull;
 
 template <bool kF32In, int kVec>
 static __global__ void __launch_bounds__(LNP_WARPS * 32, kVec > 5 ? 2 : 3) vlp_ln_merge_pipe_kernel(
@@ -470,9 +471,10 @@ static __global__ void __launch_bounds__(LNP_WARPS * 32, kVec > 5 ? 2 : 3) vlp_l
         }
         if (!mbar_wait_limit(&bars[s], (phase >> s) & 1u, wait_ns)) {
             if (lane == 0) atomicCAS(err, 0, -5);
-            for (int t = 0; t < stages; ++t)        // drain the copies still landing
-                if (((loaded >> t) & 1u) && t != s) mbar_wait_limit(&bars[t], (phase >> t) & 1u, wait_ns);
-            mbar_wait_limit(&bars[s], (phase >> s) & 1u, wait_ns);
+            // drain: no copy may still be landing in the ring when the warp ends, so these
+            // waits have their own, longer bound (copies of a few KB land in microseconds)
+            for (int t = 0; t < stages; ++t)
+                if ((loaded >> t) & 1u) mbar_wait_limit(&bars[t], (phase >> t) & 1u, LNP_DRAIN_NS);
             return;
         }
         phase ^= 1u << s;
