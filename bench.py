@@ -211,9 +211,17 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+def workload_config(args, wl, M: int, R: int) -> dict:
+    """The workload keys of `config`, the same on both arms."""
+    return {"workload": args.workload, "images": wl.n_images, "merged_tokens": M, "assembled_rows": R,
+            "K1": wl.K1, "N1": wl.N1, "N2": wl.N2, "k": wl.k, "layernorm": wl.has_ln,
+            "tiling": "2D" if wl.tiled else "none", "sequences": f"{wl.B}x{wl.S}"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
+    from oracle import projector as O
     wl = W.WORKLOADS[args.workload]
     hw = W.grid_hw(wl, args.seed)
     crop = W.spatial_crop(wl)
@@ -231,11 +239,14 @@ def run_reference(args, rank, world):
         sec += s
         img = (img + n) % wl.n_images
     value = tok / sec
+    M = sum(O.tokens_untiled(int(h_), int(w_), wl.k) for h_, w_ in hw)
+    R = int(sum(O.image_rows(hw, wl.k, crop)))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * sec / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "sample": "whole images of the workload per step, fp64 numpy oracle"},
+        "config": dict(workload_config(args, wl, M, R),
+                       sample="whole images of the workload per step, fp64 numpy oracle on the host cores"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": f"{tok} merged tokens over {args.steps} steps of whole images"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -504,11 +515,8 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "images": wl.n_images, "merged_tokens": M,
-                       "assembled_rows": int(sum(rows)), "K1": wl.K1, "N1": wl.N1, "N2": wl.N2, "k": wl.k,
-                       "layernorm": wl.has_ln, "tiling": "2D" if wl.tiled else "none",
-                       "sequences": f"{wl.B}x{wl.S}", "l2": "flushed between steps (256 MiB write)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "config": dict(workload_config(args, wl, M, int(sum(rows))), l2="flushed between steps (256 MiB write)",
+                           parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
             "tflops_per_gpu": tflops,
             "pct_of_dense_bf16_peak": 100.0 * tflops / peaks.get("bf16_tflops"),
             "pct_of_datasheet_2250_tflops": 100.0 * tflops / 2250.0,
