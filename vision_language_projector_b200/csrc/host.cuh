@@ -485,8 +485,8 @@ inline void stage_end(vlproj_handle* h, int stage, cudaStream_t s) {
 // beyond. The kernel's shared-memory attribute and
 // occupancy are set up on the handle's first launch (the configuration fixes both).
 template <bool F32, int V>
-inline int launch_ln_merge_pipe(vlproj_handle* h, const void* features, int M, float eps, __nv_bfloat16* A,
-                                cudaStream_t s) {
+inline int launch_ln_merge_pipe(vlproj_handle* h, const void* features, const ViewDesc* views, int n_views, int M,
+                                float eps, __nv_bfloat16* A, cudaStream_t s) {
     const vlproj_config& c = h->cfg;
     const int64_t items = static_cast<int64_t>(M) * c.k * c.k;
     const size_t row_bytes = static_cast<size_t>(c.C) * (F32 ? 4 : 2);
@@ -503,31 +503,32 @@ inline int launch_ln_merge_pipe(vlproj_handle* h, const void* features, int M, f
     const int64_t want = (items + vlp::LNP_WARPS - 1) / vlp::LNP_WARPS;
     const unsigned blocks =
         static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(h->num_sms) * h->lnp_per_sm)));
-    kern<<<blocks, vlp::LNP_WARPS * 32, smem, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma, h->beta, eps,
+    kern<<<blocks, vlp::LNP_WARPS * 32, smem, s>>>(features, views, n_views, M, c.k, c.C, h->gamma, h->beta, eps,
                                                   c.has_ln, A, stages, h->wait_ns, h->status);
     VLP_CUDA(cudaGetLastError());
     return VLPROJ_OK;
 }
 
-inline int launch_ln_merge(vlproj_handle* h, const void* features, int M, float eps, __nv_bfloat16* A,
-                           cudaStream_t s) {
+// Source rows come from the view table `views` (n_views entries, on the device).
+inline int launch_ln_merge(vlproj_handle* h, const void* features, const ViewDesc* views, int n_views, int M,
+                           float eps, __nv_bfloat16* A, cudaStream_t s) {
     const vlproj_config& c = h->cfg;
     const int64_t items = static_cast<int64_t>(M) * c.k * c.k;
     if (items == 0) return VLPROJ_OK;
     const int nvec = c.C / 8;
     const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
-    if (nvec <= 64) return f32 ? launch_ln_merge_pipe<true, 2>(h, features, M, eps, A, s)
-                               : launch_ln_merge_pipe<false, 2>(h, features, M, eps, A, s);
-    if (nvec <= 160) return f32 ? launch_ln_merge_pipe<true, 5>(h, features, M, eps, A, s)
-                                : launch_ln_merge_pipe<false, 5>(h, features, M, eps, A, s);
-    if (nvec <= 256) return f32 ? launch_ln_merge_pipe<true, 8>(h, features, M, eps, A, s)
-                                : launch_ln_merge_pipe<false, 8>(h, features, M, eps, A, s);
+    if (nvec <= 64) return f32 ? launch_ln_merge_pipe<true, 2>(h, features, views, n_views, M, eps, A, s)
+                               : launch_ln_merge_pipe<false, 2>(h, features, views, n_views, M, eps, A, s);
+    if (nvec <= 160) return f32 ? launch_ln_merge_pipe<true, 5>(h, features, views, n_views, M, eps, A, s)
+                                : launch_ln_merge_pipe<false, 5>(h, features, views, n_views, M, eps, A, s);
+    if (nvec <= 256) return f32 ? launch_ln_merge_pipe<true, 8>(h, features, views, n_views, M, eps, A, s)
+                                : launch_ln_merge_pipe<false, 8>(h, features, views, n_views, M, eps, A, s);
     const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
     if (f32)
-        vlp::vlp_ln_merge_kernel<true><<<blocks, 256, 0, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma, h->beta,
-                                                              eps, c.has_ln, A);
+        vlp::vlp_ln_merge_kernel<true><<<blocks, 256, 0, s>>>(features, views, n_views, M, c.k, c.C, h->gamma,
+                                                              h->beta, eps, c.has_ln, A);
     else
-        vlp::vlp_ln_merge_kernel<false><<<blocks, 256, 0, s>>>(features, h->gmeta.ptr, M, c.k, c.C, h->gamma,
+        vlp::vlp_ln_merge_kernel<false><<<blocks, 256, 0, s>>>(features, views, n_views, M, c.k, c.C, h->gamma,
                                                                h->beta, eps, c.has_ln, A);
     VLP_CUDA(cudaGetLastError());
     return VLPROJ_OK;

@@ -341,7 +341,7 @@ static __global__ void __launch_bounds__(256) vlp_layernorm_kernel(const void* _
 
 // ---------------------------------------------------------------- LayerNorm + merge
 // Item (merged token m, position p = dy*k + dx): the patch at (k*i+dy, k*j+dx) of m's
-// view (from gmeta), LayerNorm'd (when has_ln) and rounded to bf16, lands at
+// view (found in the view table), LayerNorm'd (when has_ln) and rounded to bf16, lands at
 // A[m][p*C : (p+1)*C]; positions in the high-end pad are written as zeros. Each patch
 // is read from memory once and A is GEMM1's operand in the kernel's K order. Values
 // equal vlp_layernorm_kernel's output bit for bit, so A holds exactly what the
@@ -355,9 +355,24 @@ __device__ __forceinline__ int64_t merge_source_row(const int2* __restrict__ gme
     return static_cast<int64_t>(g.x) + (p / k) * static_cast<int>(wm >> 16) + (p % k);
 }
 
+// The same from the view table (no gather metadata needed): token m of its view is
+// merged-grid cell (i, j), tap p = dy * k + dx is patch (k i + dy, k j + dx) if that lies
+// inside the view's grid.
+__device__ __forceinline__ int64_t merge_source_row(const ViewDesc* __restrict__ views, int n_views, int m, int p,
+                                                    int k) {
+    const ViewDesc& V = views[find_view(views, n_views, m)];
+    const int t = m - V.tok_start;
+    if (t >= V.hp * V.wp) return -1;
+    const int i = t / V.wp, j = t - (t / V.wp) * V.wp;
+    const int y = k * i + p / k, x = k * j + p % k;
+    if (y >= V.h || x >= V.w) return -1;
+    return V.patch_start + static_cast<int64_t>(y) * V.w + x;
+}
+
 // Any C: one warp per item, the row re-read from memory for each pass.
 template <bool kF32In>
-static __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __restrict__ x, const int2* __restrict__ gmeta,
+static __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __restrict__ x,
+                                                           const ViewDesc* __restrict__ views, int n_views,
                                                            int M, int k, int C, const float* __restrict__ gamma,
                                                            const float* __restrict__ beta, float eps, int has_ln,
                                                            __nv_bfloat16* __restrict__ A) {
@@ -367,7 +382,7 @@ static __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __
     if (item >= static_cast<int64_t>(M) * kk) return;
     const int m = static_cast<int>(item / kk), p = static_cast<int>(item - static_cast<int64_t>(m) * kk);
     uint4* dst = reinterpret_cast<uint4*>(A + item * C);
-    const int64_t row = merge_source_row(gmeta, m, p, k);
+    const int64_t row = merge_source_row(views, n_views, m, p, k);
     if (row < 0) {
         for (int v = lane; v < C / 8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
         return;
@@ -393,8 +408,9 @@ constexpr uint64_t LNP_DRAIN_NS = 1000000000ull;
 
 template <bool kF32In, int kVec>
 static __global__ void __launch_bounds__(LNP_WARPS * 32, kVec > 5 ? 2 : 3) vlp_ln_merge_pipe_kernel(
-    const void* __restrict__ x, const int2* __restrict__ gmeta, int M, int k, int C, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, int has_ln, __nv_bfloat16* __restrict__ A, int stages,
+    const void* __restrict__ x, const ViewDesc* __restrict__ views, int n_views, int M, int k, int C,
+    const float* __restrict__ gamma, const float* __restrict__ beta, float eps, int has_ln,
+    __nv_bfloat16* __restrict__ A, int stages,
     uint64_t wait_ns, int* err) {
     extern __shared__ __align__(128) uint8_t lnp_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -443,7 +459,8 @@ static __global__ void __launch_bounds__(LNP_WARPS * 32, kVec > 5 ? 2 : 3) vlp_l
             if (j + lane < n_items) {
                 const int64_t it = gw + static_cast<int64_t>(j + lane) * nwarps;
                 const int m = static_cast<int>(it / kk);
-                batch_row = merge_source_row(gmeta, m, static_cast<int>(it - static_cast<int64_t>(m) * kk), k);
+                batch_row =
+                    merge_source_row(views, n_views, m, static_cast<int>(it - static_cast<int64_t>(m) * kk), k);
             }
         }
         const int64_t r = __shfl_sync(0xffffffffu, batch_row, j & 31);

@@ -33,20 +33,26 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     const int nch_tile = vlp::BM / pl.chunk;
     // chunk entries for every 128-row slice of every (pair) tile, so round to 256 rows
     const int n_chunks = im2col ? ((M + 2 * vlp::BM - 1) / (2 * vlp::BM)) * 2 * nch_tile : 0;
-    const bool cpasync = !im2col && !pl.box5;   // (also the merged-LayerNorm path: it needs gmeta)
+    // gather metadata only for GEMM1's cp.async gather (the merged-LayerNorm pass finds its
+    // source rows in the view table, the box and im2col modes need none)
+    const bool cpasync = !im2col && !pl.box5 && !pl.merged_ln;
     if (h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
     if (cpasync && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
     if (im2col && h->chunks.ensure(std::max(n_chunks, 1))) return VLPROJ_ERR_CUDA;
 
-    stage_begin(h, 1, s);
-    ++h->launches;
-    const int geo_threads = std::max(M, n_chunks);
-    vlp::vlp_geometry_kernel<<<(geo_threads + 255) / 256, 256, 0, s>>>(
-        dviews, static_cast<int>(pl.views.size()), M, c.k, pos, pl.R, dest_mode,
-        cpasync ? h->gmeta.ptr : nullptr, h->rowdest.ptr, im2col ? h->chunks.ptr : nullptr, n_chunks, pl.chunk,
-        pl.uniform ? 1 : 0);
-    VLP_CUDA(cudaGetLastError());
-    stage_end(h, 1, s);
+    // the geometry pass only when something below reads its output (a forward with the
+    // merged LayerNorm or the box gather and no row table skips it)
+    if (cpasync || im2col || dest_mode != vlp::DEST_NONE) {
+        stage_begin(h, 1, s);
+        ++h->launches;
+        const int geo_threads = std::max(M, n_chunks);
+        vlp::vlp_geometry_kernel<<<(geo_threads + 255) / 256, 256, 0, s>>>(
+            dviews, static_cast<int>(pl.views.size()), M, c.k, pos, pl.R, dest_mode,
+            cpasync ? h->gmeta.ptr : nullptr, h->rowdest.ptr, im2col ? h->chunks.ptr : nullptr, n_chunks, pl.chunk,
+            pl.uniform ? 1 : 0);
+        VLP_CUDA(cudaGetLastError());
+        stage_end(h, 1, s);
+    }
 
     const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(features);
     if (pl.merged_ln) {
@@ -54,7 +60,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
         ++h->launches;
         if (h->A.ensure(static_cast<size_t>(M) * h->K1)) return VLPROJ_ERR_CUDA;
         const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
-        int rc = launch_ln_merge(h, features, M, eps, h->A.ptr, s);
+        int rc = launch_ln_merge(h, features, dviews, static_cast<int>(pl.views.size()), M, eps, h->A.ptr, s);
         if (rc) return rc;
         stage_end(h, 2, s);
     } else if (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) {

@@ -217,7 +217,8 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         // 7. A, exactly as the forward pass rounds it
         stage_begin(h, 7, s);
         ++h->launches;
-        rc = launch_ln_merge(h, a->features, static_cast<int>(M), eps, h->A.ptr, s);
+        rc = launch_ln_merge(h, a->features, h->dviews.ptr, static_cast<int>(pl.views.size()), static_cast<int>(M), eps,
+                             h->A.ptr, s);
         if (rc) return rc;
         stage_end(h, 7, s);
 
