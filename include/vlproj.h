@@ -339,8 +339,10 @@ int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns);
 /* ---- tracing ------------------------------------------------------------
  * Stage timing with CUDA events recorded on the launching stream around each
  * kernel of vlproj_forward / vlproj_backward. Stages, in order:
- *   forward   0 placeholder index, 1 geometry, 2 LayerNorm/convert, 3 GEMM1 (merge +
- *             MLP first layer + GELU), 4 GEMM2 (second layer + scatter),
+ *   forward   0 placeholder index (and GEMM2's row map), 1 geometry (gather data; not
+ *             launched when GEMM1 reads none and no row table is wanted, e.g. with the
+ *             merged LayerNorm or the 5D box gather), 2 LayerNorm/convert, 3 GEMM1
+ *             (merge + MLP first layer + GELU), 4 GEMM2 (second layer + scatter),
  *             5 newline/separator rows;
  *   backward  6 placeholder index + geometry, 7 LayerNorm-merge (A), 8 GEMM1
  *             recompute (GELU' and H^T), 9 dY gather, 10 dH GEMM (dP), 11 dW2 GEMM,
