@@ -155,6 +155,53 @@ def _ptr(t) -> Optional[int]:
     return t.data_ptr()
 
 
+def _arg_error(name: str, why: str) -> "VlprojError":
+    return VlprojError(ERR_INVALID_ARG, f"{name}: {why}")
+
+
+def _dev(t, name: str, itemsize: int, numel: int = 0) -> Optional[int]:
+    """Device pointer of ``t`` after the checks only the binding can make (the C ABI gets
+    bare pointers): a contiguous CUDA tensor whose elements are ``itemsize`` bytes, with at
+    least ``numel`` of them. None and integer addresses pass through unchecked."""
+    if t is None or isinstance(t, int):
+        return t
+    if isinstance(t, np.ndarray) or not hasattr(t, "is_cuda"):
+        raise _arg_error(name, f"a CUDA tensor is required, got {type(t).__name__}")
+    if not t.is_cuda:
+        raise _arg_error(name, f"a CUDA tensor is required, got one on {t.device}")
+    if not t.is_contiguous():
+        raise _arg_error(name, "the tensor must be contiguous")
+    if t.element_size() != itemsize:
+        raise _arg_error(name, f"{t.dtype} has {t.element_size()}-byte elements, {itemsize} expected")
+    if t.numel() < numel:
+        raise _arg_error(name, f"{t.numel()} elements, at least {numel} needed")
+    return t.data_ptr()
+
+
+def _host(t, name: str, itemsize: int, numel: int = 0) -> Optional[int]:
+    """Host address of ``t`` (a CPU tensor, page-locked for overlapped copies, or a numpy
+    array) after the same checks."""
+    if t is None or isinstance(t, int):
+        return t
+    if isinstance(t, np.ndarray):
+        if not t.flags["C_CONTIGUOUS"]:
+            raise _arg_error(name, "the array must be C-contiguous")
+        size, n, addr = t.itemsize, t.size, t.ctypes.data
+    elif hasattr(t, "is_cuda"):
+        if t.is_cuda:
+            raise _arg_error(name, "host memory is required, got a CUDA tensor")
+        if not t.is_contiguous():
+            raise _arg_error(name, "the tensor must be contiguous")
+        size, n, addr = t.element_size(), t.numel(), t.data_ptr()
+    else:
+        raise _arg_error(name, f"a host tensor or array is required, got {type(t).__name__}")
+    if size != itemsize:
+        raise _arg_error(name, f"{size}-byte elements, {itemsize} expected")
+    if n < numel:
+        raise _arg_error(name, f"{n} elements, at least {numel} needed")
+    return addr
+
+
 def _host_i32(a) -> Optional[np.ndarray]:
     if a is None:
         return None
@@ -251,6 +298,40 @@ class Projector:
         except Exception:
             pass
 
+    # ---- argument checks the C ABI cannot make (it receives bare pointers)
+    def _feat_size(self) -> int:
+        return 4 if self.cfg.feat_dtype == FEAT_F32 else 2
+
+    def _views(self, g, c, n_images: int) -> int:
+        """grid_hw rows the library reads for n_images images; host arrays that are too
+        short are rejected here (the library cannot see their length)."""
+        if g is None or n_images <= 0:
+            return 0
+        nv = n_images
+        if self.cfg.tile_tag == TILE_2D and c is not None:
+            c2 = c.reshape(-1, 2)
+            if len(c2) < n_images:
+                raise _arg_error("spatial_crop", f"{len(c2)} rows for {n_images} images")
+            nv = int(sum(1 + max(int(c2[i, 0]), 0) * max(int(c2[i, 1]), 0) for i in range(n_images)))
+        rows = len(g.reshape(-1, 2))
+        if rows < nv:
+            raise _arg_error("grid_hw", f"{rows} rows, {nv} views")
+        return nv
+
+    def _extent(self, g, nv: int):
+        """(patches, merged tokens) of the first nv views."""
+        if g is None or nv <= 0:
+            return 0, 0
+        hw = np.maximum(g.reshape(-1, 2)[:nv].astype(np.int64), 0)
+        k = self.cfg.k
+        return int((hw[:, 0] * hw[:, 1]).sum()), int((((hw[:, 0] + k - 1) // k) * ((hw[:, 1] + k - 1) // k)).sum())
+
+    @staticmethod
+    def _fail(e: "VlprojError", check: bool) -> int:
+        if check:
+            raise e
+        return e.code
+
     def forward(self, features, grid_hw, spatial_crop, input_ids, image_token_id: int, out_embeds,
                 newline=None, sep=None, stream=None, n_images: Optional[int] = None, check: bool = True) -> int:
         """Enqueue the bridge; raise on a host-detected error. Returns the status code."""
@@ -259,9 +340,17 @@ class Projector:
         if n_images is None:
             n_images = len(c) if c is not None else (0 if g is None else len(g))
         n_ids = 0 if input_ids is None else int(input_ids.numel())
-        rc = _lib.vlproj_forward(self._h, _ptr(features), _ptr(g), _ptr(c), n_images, _ptr(input_ids), n_ids,
-                                 int(image_token_id), _ptr(newline), _ptr(sep), _ptr(out_embeds),
-                                 _stream_ptr(stream))
+        N2 = self.cfg.N2
+        try:
+            P, _ = self._extent(g, self._views(g, c, n_images))
+            pf = _dev(features, "features", self._feat_size(), P * self.cfg.C)
+            pi = _dev(input_ids, "input_ids", 8)
+            pn, ps = _dev(newline, "newline", 2, N2), _dev(sep, "sep", 2, N2)
+            po = _dev(out_embeds, "out_embeds", 2, n_ids * N2)
+        except VlprojError as e:
+            return self._fail(e, check)
+        rc = _lib.vlproj_forward(self._h, pf, _ptr(g), _ptr(c), n_images, pi, n_ids, int(image_token_id), pn, ps,
+                                 po, _stream_ptr(stream))
         if check and rc != OK:
             raise VlprojError(rc, "vlproj_forward")
         return rc
@@ -275,11 +364,20 @@ class Projector:
         c = _host_i32(spatial_crop)
         if n_images is None:
             n_images = len(c) if c is not None else (0 if g is None else len(g))
-        a = ForwardArgs(_ptr(features), _ptr(g), _ptr(c), n_images, _ptr(input_ids),
-                        0 if input_ids is None else int(input_ids.numel()), int(image_token_id), _ptr(newline),
-                        _ptr(sep), _ptr(out_embeds), _ptr(embed_table),
-                        0 if embed_table is None else int(embed_table.shape[0]), _ptr(rows_out),
-                        0 if rows_out is None else int(rows_out.shape[0]))
+        n_ids = 0 if input_ids is None else int(input_ids.numel())
+        vocab = 0 if embed_table is None else int(embed_table.shape[0])
+        n_rows = 0 if rows_out is None else int(rows_out.shape[0])
+        N2 = self.cfg.N2
+        try:
+            P, _ = self._extent(g, self._views(g, c, n_images))
+            a = ForwardArgs(_dev(features, "features", self._feat_size(), P * self.cfg.C), _ptr(g), _ptr(c),
+                            n_images, _dev(input_ids, "input_ids", 8), n_ids, int(image_token_id),
+                            _dev(newline, "newline", 2, N2), _dev(sep, "sep", 2, N2),
+                            _dev(out_embeds, "out_embeds", 2, n_ids * N2),
+                            _dev(embed_table, "embed_table", 2, vocab * N2), vocab,
+                            _dev(rows_out, "rows_out", 2, n_rows * N2), n_rows)
+        except VlprojError as e:
+            return self._fail(e, check)
         rc = _lib.vlproj_forward_ex(self._h, ctypes.byref(a), _stream_ptr(stream))
         if check and rc != OK:
             raise VlprojError(rc, "vlproj_forward_ex")
@@ -294,19 +392,33 @@ class Projector:
         unknown = set(grads) - set(GRAD_NAMES) - {"W_mid", "b_mid"}
         if unknown:
             raise ValueError(f"unknown gradient names {sorted(unknown)}")
-        mids = {}
-        for key in ("W_mid", "b_mid"):
-            if grads.get(key) is not None:
-                arr = (ctypes.c_void_p * len(grads[key]))(*[_ptr(t) for t in grads[key]])
-                mids[key] = arr
         g = _host_i32(grid_hw)
         c = _host_i32(spatial_crop)
         if n_images is None:
             n_images = len(c) if c is not None else (0 if g is None else len(g))
-        a = BackwardArgs(_ptr(features), _ptr(g), _ptr(c), n_images, _ptr(input_ids),
-                         0 if input_ids is None else int(input_ids.numel()), int(image_token_id), _ptr(d_out),
-                         *[_ptr(grads.get(n)) for n in GRAD_NAMES],
-                         *[ctypes.cast(mids[k], ctypes.c_void_p) if k in mids else None for k in ("W_mid", "b_mid")])
+        n_ids = 0 if input_ids is None else int(input_ids.numel())
+        cfg = self.cfg
+        K1 = cfg.k * cfg.k * cfg.C
+        try:
+            P, _ = self._extent(g, self._views(g, c, n_images))
+            need = {"W1": cfg.N1 * K1, "b1": cfg.N1, "W2": cfg.N2 * cfg.N1, "b2": cfg.N2, "gamma": cfg.C,
+                    "beta": cfg.C, "newline": cfg.N2, "sep": cfg.N2, "features": P * cfg.C}
+            grad_ptrs = [_dev(grads.get(n), f"grads[{n!r}]", 4, need[n]) for n in GRAD_NAMES]
+            mids = {}
+            for key, numel in (("W_mid", cfg.N1 * cfg.N1), ("b_mid", cfg.N1)):
+                if grads.get(key) is not None:
+                    if len(grads[key]) != cfg.depth - 2:
+                        raise _arg_error(f"grads[{key!r}]", f"{len(grads[key])} tensors, depth - 2 = "
+                                                            f"{cfg.depth - 2} expected")
+                    mids[key] = (ctypes.c_void_p * len(grads[key]))(
+                        *[_dev(t, f"grads[{key!r}][{i}]", 4, numel) for i, t in enumerate(grads[key])])
+            a = BackwardArgs(_dev(features, "features", self._feat_size(), P * cfg.C), _ptr(g), _ptr(c), n_images,
+                             _dev(input_ids, "input_ids", 8), n_ids, int(image_token_id),
+                             _dev(d_out, "d_out", 2, n_ids * cfg.N2), *grad_ptrs,
+                             *[ctypes.cast(mids[k], ctypes.c_void_p) if k in mids else None
+                               for k in ("W_mid", "b_mid")])
+        except VlprojError as e:
+            return self._fail(e, check)
         rc = _lib.vlproj_backward(self._h, ctypes.byref(a), _stream_ptr(stream))
         if check and rc != OK:
             raise VlprojError(rc, "vlproj_backward")
@@ -321,8 +433,15 @@ class Projector:
         c = _host_i32(spatial_crop)
         if n_images is None:
             n_images = len(c) if c is not None else (0 if g is None else len(g))
-        a = HostArgs(_ptr(features), _ptr(g), _ptr(c), n_images, _ptr(newline), _ptr(sep), _ptr(rows_out),
-                     0 if rows_out is None else int(rows_out.shape[0]), int(chunks))
+        n_rows = 0 if rows_out is None else int(rows_out.shape[0])
+        N2 = self.cfg.N2
+        try:
+            P, _ = self._extent(g, self._views(g, c, n_images))
+            a = HostArgs(_host(features, "features", self._feat_size(), P * self.cfg.C), _ptr(g), _ptr(c), n_images,
+                         _dev(newline, "newline", 2, N2), _dev(sep, "sep", 2, N2),
+                         _host(rows_out, "rows_out", 2, n_rows * N2), n_rows, int(chunks))
+        except VlprojError as e:
+            return self._fail(e, check)
         rc = _lib.vlproj_project_host(self._h, ctypes.byref(a), _stream_ptr(stream))
         if check and rc != OK:
             raise VlprojError(rc, "vlproj_project_host")
@@ -330,8 +449,10 @@ class Projector:
 
     def hidden(self, features, grid_hw, hidden, stream=None) -> None:
         g = _host_i32(grid_hw)
-        rc = _lib.vlproj_hidden(self._h, _ptr(features), _ptr(g), 0 if g is None else len(g), _ptr(hidden),
-                                _stream_ptr(stream))
+        nv = 0 if g is None else len(g.reshape(-1, 2))
+        P, M = self._extent(g, nv)
+        rc = _lib.vlproj_hidden(self._h, _dev(features, "features", self._feat_size(), P * self.cfg.C), _ptr(g), nv,
+                                _dev(hidden, "hidden", 2, M * self.cfg.N1), _stream_ptr(stream))
         if rc != OK:
             raise VlprojError(rc, "vlproj_hidden")
 
