@@ -278,6 +278,12 @@ def main():
     seed = args.seed + rank
     hw, crop, rows = workload_geometry(wl, seed)
     M = merged_tokens(wl, hw)
+    # every rank has its own seeded batch, so the job's token count is the sum over ranks
+    M_all = M
+    if world > 1:
+        t = torch.tensor([float(M)], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        M_all = int(round(t.item()))
     wts = W.weights(wl, seed)
     feats_h = W.features(wl, hw, seed, threads=min(16, os.cpu_count() or 1))
     ids_h = W.input_ids(wl, rows, seed)
@@ -359,8 +365,7 @@ def main():
         t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-    tokens_per_step = M
-    value = world * tokens_per_step * args.steps / (total_ms / 1000.0)
+    value = M_all * args.steps / (total_ms / 1000.0)
     ms_per_step = total_ms / args.steps
     fl_tok = flops_per_token(wl)
     tflops = value * fl_tok / 1e12 / world
@@ -432,9 +437,13 @@ def main():
         st = proj.status()
         if st != vp.OK:
             raise SystemExit(f"e2e steps failed: {vp.strerror(st)}")
-        e2e = {"value": world * tokens_per_step * args.e2e_steps / (e_ms / 1000.0), "unit": UNIT,
-               "h2d_bytes_per_step": int(feats_p.numel() * feats_p.element_size()),
-               "d2h_bytes_per_step": int(rows_p.numel() * 2), "steps": args.e2e_steps,
+        io = [float(feats_p.numel() * feats_p.element_size()), float(rows_p.numel() * 2)]
+        if world > 1:
+            t = torch.tensor(io, dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.SUM)
+            io = t.tolist()
+        e2e = {"value": M_all * args.e2e_steps / (e_ms / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": int(io[0]), "d2h_bytes_per_step": int(io[1]), "steps": args.e2e_steps,
                "path": "vlproj_project_host: pinned host features in, every image's assembled rows out to "
                        "pinned host memory, copies pipelined against the projection in image chunks"}
 
@@ -490,8 +499,8 @@ def main():
         if st != vp.OK:
             raise SystemExit(f"backward steps failed: {vp.strerror(st)}")
         b_step = bt / args.backward_steps
-        b_flops = 2.0 * M * (3 * wl.K1 * wl.N1 + 2 * wl.N1 * wl.N2)
-        b_tf = b_flops / (b_step / 1000.0) / 1e12
+        b_flops = 2.0 * M_all * (3 * wl.K1 * wl.N1 + 2 * wl.N1 * wl.N2)       # whole job, per step
+        b_tf = b_flops / world / (b_step / 1000.0) / 1e12
         b_peak = peaks.get("bf16_tflops_sustained" if bt > 2000.0 else "bf16_tflops")
         bwd = {"ms_per_step": b_step, "tflops_per_gpu": b_tf, "peak": b_peak,
                "frac_of_peak": b_tf / b_peak,
