@@ -275,17 +275,18 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
     wl = W.WORKLOADS[args.workload]
-    seed = args.seed + rank
+    # data-parallel replicas: every rank holds the same weights and a batch of the same
+    # shapes (geometry, placeholder layout), with feature values of its own
+    seed = args.seed
     hw, crop, rows = workload_geometry(wl, seed)
     M = merged_tokens(wl, hw)
-    # every rank has its own seeded batch, so the job's token count is the sum over ranks
-    M_all = M
+    M_all = M                              # the job's tokens: the sum over the ranks
     if world > 1:
         t = torch.tensor([float(M)], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.SUM)
         M_all = int(round(t.item()))
     wts = W.weights(wl, seed)
-    feats_h = W.features(wl, hw, seed, threads=min(16, os.cpu_count() or 1))
+    feats_h = W.features(wl, hw, seed + rank, threads=min(16, os.cpu_count() or 1))
     ids_h = W.input_ids(wl, rows, seed)
     prefill_h = W.prefill_embeds(wl, ids_h, W.embed_table(wl, seed))
 
@@ -453,7 +454,7 @@ def main():
         proj.profile(True)
         proj.profile_stages(None)
         gen = torch.Generator(device="cuda")
-        gen.manual_seed(1000 + seed)
+        gen.manual_seed(1000 + seed + rank)
         d_out = torch.randn((ids.numel(), wl.N2), device="cuda", generator=gen).to(torch.bfloat16)
         P = int(feats.shape[0])
         shapes = {"W1": (wl.N1, wl.K1), "b1": (wl.N1,), "W2": (wl.N2, wl.N1), "b2": (wl.N2,), "features": (P, wl.C)}
