@@ -37,7 +37,7 @@ import workloads as W  # noqa: E402
 
 METRIC = "projected image tokens/s on 1 B200; % of dense BF16 tensor peak"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "moonvit"
+DEFAULT_WORKLOAD = "stress"         # the largest single-GPU workload (262,144 tokens, 38.5 TFLOP per step)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the sources that decide the GEMMs' DRAM traffic (kernel, its PTX, its launch and raster)
 KERNEL_SOURCES = [os.path.join("vision_language_projector_b200", "csrc", f)
@@ -68,6 +68,22 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return FALLBACK_PEAKS, "fallback"
+
+
+def peak_clock_mhz(peaks: dict, sustained: bool):
+    """SM clock (MHz) under which the bf16 peak was measured, when the peaks file says."""
+    for key in (("bf16_sustained_sm_mhz", "sustained_sm_mhz") if sustained else ("bf16_sm_mhz", "burst_sm_mhz")) + (
+            "sm_mhz_median_under_load", "sm_mhz_median", "sm_mhz"):
+        v = peaks.get(key)
+        if isinstance(v, (int, float)) and v > 0:
+            return float(v)
+    clocks = peaks.get("clocks")
+    if isinstance(clocks, dict):
+        for key in ("sm_mhz_median_under_load", "median_sm_mhz", "sm_mhz_median", "sm_mhz"):
+            v = clocks.get(key)
+            if isinstance(v, (int, float)) and v > 0:
+                return float(v)
+    return None
 
 
 def kernel_source_hash() -> str:
@@ -402,6 +418,31 @@ def main():
                 "peak_source": f"{peak_src} HBM copy", "traffic": traffic_from_profiles(args.workload, dom),
                 "algorithmic_bytes": b}
 
+    # bytes per step: what the path must move (features in, image rows out, ids read) beside
+    # what this implementation moves on top (the hidden activations written by GEMM1 and read
+    # by GEMM2, per hidden layer; with a LayerNorm, the merged bf16 A written and read back)
+    n_ids_step = int(ids_h.shape[0])
+    R_step = int(sum(rows))
+    P_step = int(sum(int(h) * int(w_) for h, w_ in hw))
+    feat_b = 4 if wl.feat_fp32 else 2
+    traffic_model = {
+        "algorithmic_bytes": P_step * wl.C * feat_b + R_step * wl.N2 * 2 + 8 * n_ids_step,
+        "hidden_round_trip_bytes": 2 * M * wl.N1 * 2,
+        "merged_a_round_trip_bytes": 2 * M * wl.K1 * 2 if wl.has_ln or wl.feat_fp32 else 0,
+        "weights_bytes": 2 * (wl.N1 * wl.K1 + wl.N2 * wl.N1),
+        "note": "per step and GPU; the hidden and merged-A round trips are implementation costs, not algorithmic",
+    }
+    # clock-normalised view of the dominant kernel: its FLOP per SM cycle at the median SM
+    # clock seen in the timed region, against the same figure for the peak
+    if clk and clk.get("sm_mhz") and roof.get("achieved"):
+        mhz = float(clk["sm_mhz"])
+        roof["sm_mhz"] = mhz
+        roof["time_x_mhz"] = avg[dom] * mhz          # ms x MHz = thousands of SM cycles per launch
+        pk_mhz = peak_clock_mhz(peaks, "sustained" in roof.get("peak_source", ""))
+        if pk_mhz:
+            roof["peak_sm_mhz"] = pk_mhz
+            roof["frac_clock_normalised"] = roof["frac"] * pk_mhz / mhz
+
     # ---- end to end through the public API with host buffers: vlproj_project_host takes the
     # step's features from pinned host memory and returns the assembled rows of every image to
     # pinned host memory, its copies pipelined against the projection; the step ends when the
@@ -534,6 +575,7 @@ def main():
             "stage_ms_note": "per stage, every stage timed, median over the warm-up steps; the timed steps time the dominant "
                              "kernel only",
             "roofline": roof,
+            "traffic_model": traffic_model,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "backward": bwd,

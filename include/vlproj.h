@@ -377,9 +377,10 @@ int64_t vlproj_launch_count(vlproj_handle* h);
  * asynchronously on `stream`: the same step as the placeholder index of
  * vlproj_forward, needing no handle. input_ids: DEVICE int64 [n_ids]; positions:
  * DEVICE int32 [max_positions]; count: DEVICE int64 [1].
- * It calls no allocator: its only scratch (one int32 per 4096 ids) is a fixed array
- * in the library's device memory, VLPROJ_NOALLOC_MAX_IDS / 4096 entries (64 KB),
- * held by every GPU that loads the library until the process exits. n_ids beyond
+ * It calls no allocator: its only scratch (one int32 per 4096 ids, then their total)
+ * is a fixed array in the library's device memory, VLPROJ_NOALLOC_MAX_IDS / 4096 + 1
+ * entries (about 64 KB), held by every GPU that loads the library until the process
+ * exits. The work is linear in n_ids (count, one prefix-sum pass, compact). n_ids beyond
  * VLPROJ_NOALLOC_MAX_IDS returns VLPROJ_ERR_INVALID_ARG before any launch.
  * The first call on each device looks up that device's copy of the array (with the
  * device current) and should come before any stream capture. All calls share the

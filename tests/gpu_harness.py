@@ -170,3 +170,97 @@ def check(case: Case, out: torch.Tensor, dev: DeviceInputs, images: Optional[Seq
         if sm.any():
             np.testing.assert_array_equal(got[sm], want[sm])      # newline / separator rows exact
     return {"worst_err_over_bound": worst, "max_abs_err": max_abs}
+
+
+def token_rows_in_image(case: Case, img: int) -> np.ndarray:
+    """(views, h'*w') table: the assembled row, inside image img, of every merged token of
+    each of its views. Built by running the oracle's own assembly on token labels."""
+    views = view_groups(case)[img]
+    v0 = views[0]
+    hp, wp = O.merged_side(case.hw[v0, 0], case.wl.k), O.merged_side(case.hw[v0, 1], case.wl.k)
+    if case.crop is None:
+        return np.arange(hp * wp, dtype=np.int64)[None, :]
+    tw, th = int(case.crop[img, 0]), int(case.crop[img, 1])
+    n_tok = hp * wp
+    labels = (np.arange(len(views) * n_tok, dtype=np.float64) + 1.0).reshape(len(views), n_tok, 1)
+    col = O.assemble_2d(labels, hp, wp, tw, th, np.zeros(1), np.full(1, -1.0), case.gvp)[:, 0]
+    table = np.full(len(views) * n_tok, -1, np.int64)
+    rows = np.flatnonzero(col > 0)
+    table[col[rows].astype(np.int64) - 1] = rows
+    assert (table >= 0).all()
+    return table.reshape(len(views), n_tok)
+
+
+def token_a(case: Case, view: int, i: int, j: int) -> np.ndarray:
+    """The merged operand of token (i, j) of `view`: the oracle's merge applied to the
+    token's own k x k window of patches (cut at the grid's high end, where the merge pads
+    with zeros). The LayerNorm is per patch, so the window gives the same values as the
+    whole view."""
+    k = case.wl.k
+    h, w = int(case.hw[view, 0]), int(case.hw[view, 1])
+    if not hasattr(case, "_patch0"):
+        case._patch0 = np.concatenate([[0], np.cumsum(case.hw[:, 0].astype(np.int64) * case.hw[:, 1])])
+    raw = case.feats[case._patch0[view]:case._patch0[view + 1]].reshape(h, w, -1)
+    win = raw[k * i:min(h, k * i + k), k * j:min(w, k * j + k)]
+    hs, ws = win.shape[0], win.shape[1]
+    win = win.astype(np.float64) if case.wl.feat_fp32 else O.bf16_bits_to_f64(win)
+    p = oracle_params(case) if not hasattr(case, "_params") else case._params
+    ln = (p["gamma"], p["beta"], case.wl.ln_eps) if case.wl.has_ln else None
+    a = O.merge_view(win.reshape(hs * ws, -1), hs, ws, k, ln)
+    assert a.shape[0] == 1
+    return a[0]
+
+
+def sample_tokens(case: Case, per_image: int = 4, block: int = 128, seed: int = 0) -> list:
+    """Seeded (view, token) picks: one token in every `block` consecutive merged tokens
+    (views in order, so every GEMM M-tile holds one) plus `per_image` more in every image."""
+    rng = np.random.default_rng(seed)
+    k = case.wl.k
+    n_tok = np.array([O.tokens_untiled(int(h), int(w), k) for h, w in case.hw], np.int64)
+    start = np.concatenate([[0], np.cumsum(n_tok)])
+    M = int(start[-1])
+    picks = set()
+    for b0 in range(0, M, block):
+        m = int(rng.integers(b0, min(M, b0 + block)))
+        v = int(np.searchsorted(start, m, side="right") - 1)
+        picks.add((v, m - int(start[v])))
+    for views in view_groups(case):
+        tot = int(sum(n_tok[v] for v in views))
+        for m in rng.choice(tot, size=min(per_image, tot), replace=False):
+            m = int(m)
+            for v in views:
+                if m < n_tok[v]:
+                    picks.add((v, m))
+                    break
+                m -= int(n_tok[v])
+    return sorted(picks)
+
+
+def check_tokens(case: Case, out: torch.Tensor, picks: Sequence[tuple]) -> dict:
+    """Compare the placeholder row of every picked (view, token) with the oracle's row
+    of that token: its merged operand from token_a, then the oracle's MLP. The row is
+    located independently of the CUDA path: the image's assembled order from
+    token_rows_in_image, and the oracle's placeholder positions."""
+    params = oracle_params(case)
+    case._params = params
+    k = case.wl.k
+    pos = O.placeholder_positions(case.ids, W.IMAGE_TOKEN_ID)
+    base = np.concatenate([[0], np.cumsum(case.rows)])
+    per = case.wl.views_per_image
+    tables = {}
+    A, dest = [], []
+    for v, t in picks:
+        img = v // per
+        if img not in tables:
+            tables[img] = token_rows_in_image(case, img)
+        wp = O.merged_side(case.hw[v, 1], k)
+        A.append(token_a(case, v, t // wp, t % wp))
+        dest.append(int(pos[base[img] + tables[img][v - img * per, t]]))
+    want = O.mlp(np.stack(A), params["W1"], params["b1"], params["W2"], params["b2"], True, params.get("mid") or ())
+    got = out.index_select(0, torch.tensor(dest, dtype=torch.int64, device=out.device)).double().cpu().numpy()
+    err = np.abs(got - want)
+    ratio = err / (TOL_ABS + TOL_REL * np.abs(want))
+    bad = np.argwhere(ratio > 1.0)
+    assert bad.size == 0, (f"{len(np.unique(bad[:, 0]))} of {len(picks)} sampled tokens out of tolerance, first "
+                           f"(view, token) {picks[int(bad[0, 0])]}: max err/bound {ratio.max():.3f}")
+    return {"tokens": len(picks), "worst_err_over_bound": float(ratio.max()), "max_abs_err": float(err.max())}

@@ -81,3 +81,41 @@ def test_fp32_features_need_four_byte_elements():
     p = _proj(feat_dtype=vp.FEAT_F32)
     _raises(lambda: p.project_host(torch.zeros(31, C, dtype=torch.bfloat16), HW, None,
                                    torch.zeros(10, N2, dtype=torch.int16)), "features")
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor on this CPU-only machine: only what the binding's
+    checks look at. Every check below fails before the library is called."""
+
+    is_cuda = True
+    device = "cuda:0"
+    dtype = "fake"
+
+    def __init__(self, numel: int, itemsize: int, contiguous: bool = True):
+        self._n, self._size, self._contig = numel, itemsize, contiguous
+
+    def numel(self):
+        return self._n
+
+    def element_size(self):
+        return self._size
+
+    def is_contiguous(self):
+        return self._contig
+
+    def data_ptr(self):
+        return 0x1000
+
+
+def test_noalloc_index_checks_its_tensors():
+    ids, pos, cnt = _FakeCuda(100, 8), _FakeCuda(100, 4), _FakeCuda(1, 8)
+    f = vp.placeholder_index_noalloc
+    _raises(lambda: f(_FakeCuda(100, 4), 7, pos, cnt), "input_ids")                 # int32 ids
+    _raises(lambda: f(ids, 7, _FakeCuda(100, 8), cnt), "positions")                 # int64 positions
+    _raises(lambda: f(ids, 7, pos, _FakeCuda(1, 4)), "count")                       # int32 count
+    _raises(lambda: f(ids, 7, pos, _FakeCuda(0, 8)), "count")                       # no room for the count
+    _raises(lambda: f(ids, 7, pos, cnt, n_ids=101), "input_ids")                    # more ids than the tensor
+    _raises(lambda: f(ids, 7, pos, cnt, max_positions=101), "positions")            # more room than the tensor
+    _raises(lambda: f(_FakeCuda(100, 8, contiguous=False), 7, pos, cnt), "input_ids")
+    _raises(lambda: f(torch.zeros(100, dtype=torch.int64), 7, pos, cnt), "input_ids")   # host memory
+    _raises(lambda: f(ids, 7, pos, cnt, n_ids=-1), "n_ids")

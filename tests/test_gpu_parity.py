@@ -2,7 +2,8 @@
 
 Small cases compare every row and span several output tiles with ragged tails in
 M and N; the five full-size workloads run in the benchmark's launch configuration
-and compare every row of sampled images plus every text row.
+and compare every row of sampled images, every text row, and a seeded token in every
+128-row M-block plus four in every image.
 """
 import numpy as np
 import pytest
@@ -12,8 +13,8 @@ import vision_language_projector_b200 as vp
 import workloads as W
 from oracle import projector as O
 
-from gpu_harness import (DeviceInputs, check, custom, dev_bf16, feats_f64, make_case, make_projector,
-                         oracle_params, run, view_groups, TOL_ABS, TOL_REL)
+from gpu_harness import (DeviceInputs, check, check_tokens, custom, dev_bf16, feats_f64, make_case, make_projector,
+                         oracle_params, run, sample_tokens, view_groups, TOL_ABS, TOL_REL)
 
 pytestmark = pytest.mark.gpu
 
@@ -123,7 +124,10 @@ def test_workload_full_size(name):
     out = run(case, proj, dev)
     assert proj.status() == vp.OK
     stats = check(case, out, dev, images)
-    print(name, stats)
+    # on top of the whole images: a seeded token in every 128-row M-block (so every GEMM
+    # tile, persistent-loop position and view is value-checked) and 4 more in every image
+    tok = check_tokens(case, out, sample_tokens(case, per_image=4, block=128, seed=1))
+    print(name, stats, tok)
 
 
 def test_gemm_ragged_edges_are_exact_zero_pad():

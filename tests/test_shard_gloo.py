@@ -106,7 +106,10 @@ def _grad_worker(rank, world, port, out):
         mine = {k: torch.from_numpy(g[k]) for k in ("W1", "b1", "W2", "b2", "gamma", "beta", "newline", "sep")}
         mine["W_mid"] = [torch.from_numpy(g["mid"][0][0])]
         mine["b_mid"] = [torch.from_numpy(g["mid"][0][1])]
+        # the shard's own feature gradient: a different size on every rank, not summed
+        mine["features"] = torch.from_numpy(g["features"]).clone()
         allreduce_gradients(mine)
+        assert torch.equal(mine.pop("features"), torch.from_numpy(g["features"]))
         if rank == 0:
             out.put({k: ([t.numpy().tolist() for t in v] if isinstance(v, list) else v.numpy().tolist())
                      for k, v in mine.items()})

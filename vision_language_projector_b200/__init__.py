@@ -240,11 +240,20 @@ def image_rows(cfg: Config, grid_hw, spatial_crop=None, n_images: Optional[int] 
 def placeholder_index_noalloc(input_ids, image_token_id: int, positions, count, stream=None,
                               n_ids: Optional[int] = None, max_positions: Optional[int] = None) -> int:
     """Placeholder positions and count without any allocation (see vlproj.h): for callers
-    that must not allocate device memory at the call. Returns the status code."""
-    n = int(input_ids.numel()) if n_ids is None else int(n_ids)
-    mp = int(positions.numel()) if max_positions is None else int(max_positions)
-    return _lib.vlproj_placeholder_index_noalloc(_ptr(input_ids), n, int(image_token_id), _ptr(positions), mp,
-                                                 _ptr(count), _stream_ptr(stream))
+    that must not allocate device memory at the call. Returns the status code.
+
+    Tensors are checked like every other entry point's (CUDA, contiguous, element size,
+    enough elements for ``n_ids`` / ``max_positions``); integer addresses pass through
+    unchecked, for callers that manage raw device memory themselves."""
+    n = (0 if isinstance(input_ids, int) else int(input_ids.numel())) if n_ids is None else int(n_ids)
+    mp = (0 if isinstance(positions, int) else int(positions.numel())) if max_positions is None else int(max_positions)
+    if n < 0 or mp < 0:
+        raise _arg_error("n_ids" if n < 0 else "max_positions", "must not be negative")
+    # over the library's limit: the C ABI rejects it before touching any buffer
+    pi = _ptr(input_ids) if n > NOALLOC_MAX_IDS else _dev(input_ids, "input_ids", 8, n)
+    pp = _dev(positions, "positions", 4, mp)
+    pc = _dev(count, "count", 8, 1)
+    return _lib.vlproj_placeholder_index_noalloc(pi, n, int(image_token_id), pp, mp, pc, _stream_ptr(stream))
 
 
 def plan_tiles(image_wh, candidates, image_size: int, patch_size: int, downsample: int):

@@ -52,28 +52,67 @@ static __global__ void __launch_bounds__(SCAN_THREADS) vlp_count_kernel(const in
     if (threadIdx.x == 0) counts[blockIdx.x] = c;
 }
 
-// Writes pos[j] = flat index of the j-th placeholder (j < R), in order. Each block
-// finds its starting rank from the counts of the blocks before it, then ranks its
-// own placeholders with warp ballots. Block 0 records whether the total equals R.
+// One block of SCAN_TOTAL_THREADS turns the per-block counts into exclusive prefix sums
+// in place and appends the total: counts[b] <- counts[0] + ... + counts[b-1] for b <
+// nblocks, counts[nblocks] <- the sum of all (counts holds nblocks + 1 entries). Thread t
+// owns the contiguous segment [t*seg, (t+1)*seg) with seg = ceil(nblocks / threads); the
+// segment sums are scanned across the block (warp shuffles, then the warp totals), so the
+// work is O(nblocks) however many blocks there are. The sum is below 2^31 (n < 2^31).
+constexpr int SCAN_TOTAL_THREADS = 1024;
+static __global__ void __launch_bounds__(SCAN_TOTAL_THREADS) vlp_scan_counts_kernel(int32_t* __restrict__ counts,
+                                                                                     int nblocks) {
+    __shared__ int warp_tot[SCAN_TOTAL_THREADS / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int seg = (nblocks + SCAN_TOTAL_THREADS - 1) / SCAN_TOTAL_THREADS;
+    const int b0 = min(nblocks, static_cast<int>(threadIdx.x) * seg), b1 = min(nblocks, b0 + seg);
+    int own = 0;
+    for (int b = b0; b < b1; ++b) own += counts[b];
+    // inclusive scan of the segment sums inside the warp
+    int inc = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < SCAN_TOTAL_THREADS / 32; ++w) {
+        const int t = warp_tot[w];
+        before += (w < warp) ? t : 0;
+        total += t;
+    }
+    int run = before + inc - own;          // exclusive prefix of this thread's segment
+    for (int b = b0; b < b1; ++b) {
+        const int c = counts[b];
+        counts[b] = run;
+        run += c;
+    }
+    if (threadIdx.x == 0) counts[nblocks] = total;
+}
+
+// Writes pos[j] = flat index of the j-th placeholder (j < R), in order. `prefix` holds
+// the exclusive prefix sums of the per-block counts and their total at prefix[nblocks]
+// (vlp_scan_counts_kernel; with nblocks == 0 only prefix[0] = 0 is read). Each block
+// starts at its own prefix and ranks its placeholders with warp ballots. Block 0 writes
+// the total to *count_out (when given) and, when fwd_status is given, whether the total
+// equals R (latching VLPROJ_ERR_TOKEN_COUNT in *err when it does not).
 static __global__ void __launch_bounds__(SCAN_THREADS) vlp_compact_kernel(const int64_t* __restrict__ ids, int64_t n,
-                                                                   int64_t token, const int32_t* __restrict__ counts,
+                                                                   int64_t token, const int32_t* __restrict__ prefix,
                                                                    int nblocks, int32_t* __restrict__ pos, int64_t R,
-                                                                   int* fwd_status, int* err) {
-    __shared__ int red[SCAN_THREADS / 32];
+                                                                   int* fwd_status, int* err, int64_t* count_out) {
     __shared__ int warp_cnt[SCAN_THREADS / 32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int pre = 0, tot = 0;
-    for (int b = threadIdx.x; b < nblocks; b += SCAN_THREADS) {
-        const int c = counts[b];
-        tot += c;
-        if (b < static_cast<int>(blockIdx.x)) pre += c;
-    }
-    pre = block_sum_256(pre, red);
-    tot = block_sum_256(tot, red);
+    const int pre = nblocks > 0 ? prefix[blockIdx.x] : 0;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
-        const int st = (static_cast<int64_t>(tot) == R) ? 0 : ERR_TOKEN_COUNT;
-        *fwd_status = st;
-        if (st != 0) atomicCAS(err, 0, st);
+        const int tot = nblocks > 0 ? prefix[nblocks] : 0;
+        if (count_out != nullptr) *count_out = tot;
+        if (fwd_status != nullptr) {
+            const int st = (static_cast<int64_t>(tot) == R) ? 0 : ERR_TOKEN_COUNT;
+            *fwd_status = st;
+            if (st != 0 && err != nullptr) atomicCAS(err, 0, st);
+        }
     }
     const int64_t start = static_cast<int64_t>(blockIdx.x) * SCAN_CHUNK;
     int64_t run = pre;
@@ -96,6 +135,28 @@ static __global__ void __launch_bounds__(SCAN_THREADS) vlp_compact_kernel(const 
         run += all;
         __syncthreads();
     }
+}
+
+// Blocks of SCAN_CHUNK ids the index step uses for n ids; its count buffer holds one
+// more entry than that (the total).
+inline int scan_blocks(int64_t n) { return static_cast<int>((n + SCAN_CHUNK - 1) / SCAN_CHUNK); }
+
+// The whole placeholder-index step on `s`: count per block, prefix sums, compact.
+// `counts` holds scan_blocks(n) + 1 entries; pos, R, fwd_status, err, count_out as in
+// vlp_compact_kernel. Adds the number of kernels launched to *launches. n < 2^31.
+inline cudaError_t enqueue_placeholder_index(const int64_t* ids, int64_t n, int64_t token, int32_t* counts,
+                                             int32_t* pos, int64_t R, int* fwd_status, int* err, int64_t* count_out,
+                                             cudaStream_t s, int64_t* launches) {
+    const int nblocks = scan_blocks(n);
+    if (nblocks > 0) {
+        vlp_count_kernel<<<nblocks, SCAN_THREADS, 0, s>>>(ids, n, token, counts);
+        vlp_scan_counts_kernel<<<1, SCAN_TOTAL_THREADS, 0, s>>>(counts, nblocks);
+        *launches += 2;
+    }
+    vlp_compact_kernel<<<nblocks > 0 ? nblocks : 1, SCAN_THREADS, 0, s>>>(ids, n, token, counts, nblocks, pos, R,
+                                                                         fwd_status, err, count_out);
+    *launches += 1;
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- geometry

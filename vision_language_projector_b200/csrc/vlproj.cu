@@ -508,9 +508,8 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
 
     // 0. placeholder index (and each GEMM row's destination), on the side stream so it
     //    overlaps the geometry / LayerNorm / GEMM1 chain on the caller's stream
-    const int nblocks = static_cast<int>((n_ids + vlp::SCAN_CHUNK - 1) / vlp::SCAN_CHUNK);
-    if (h->counts.ensure(std::max(nblocks, 1)) || h->pos.ensure(std::max<int64_t>(pl.R, 1)))
-        return VLPROJ_ERR_CUDA;
+    const int nblocks = vlp::scan_blocks(n_ids);
+    if (h->counts.ensure(nblocks + 1) || h->pos.ensure(std::max<int64_t>(pl.R, 1))) return VLPROJ_ERR_CUDA;
     if (pl.M > 0 && h->rowdest.ensure(pl.M)) return VLPROJ_ERR_CUDA;
     if (pl.M > 0 && h->H.ensure(static_cast<size_t>(pl.M) * c.N1)) return VLPROJ_ERR_CUDA;
     if (pl.M > 0 && c.depth > 2 && h->H2.ensure(static_cast<size_t>(pl.M) * c.N1)) return VLPROJ_ERR_CUDA;
@@ -523,23 +522,22 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
         VLP_CUDA(cudaEventRecord(h->fork, s));
         VLP_CUDA(cudaStreamWaitEvent(si, h->fork, 0));
     }
+    // a launch error on the side stream still leaves the caller's stream ordered after it
+    auto fail_side = [&](int code) {
+        if (si != s && cudaEventRecord(h->join, si) == cudaSuccess) cudaStreamWaitEvent(s, h->join, 0);
+        return code;
+    };
     stage_begin(h, 0, si);
-    h->launches += nblocks > 0 ? 2 : 1;
-    if (nblocks > 0) {
-        vlp::vlp_count_kernel<<<nblocks, vlp::SCAN_THREADS, 0, si>>>(input_ids, n_ids, image_token_id,
-                                                                     h->counts.ptr);
-        VLP_CUDA(cudaGetLastError());
-    }
-    vlp::vlp_compact_kernel<<<std::max(nblocks, 1), vlp::SCAN_THREADS, 0, si>>>(
-        input_ids, n_ids, image_token_id, h->counts.ptr, nblocks, h->pos.ptr, pl.R, h->status + 1, h->status);
-    VLP_CUDA(cudaGetLastError());
+    if (vlp::enqueue_placeholder_index(input_ids, n_ids, image_token_id, h->counts.ptr, h->pos.ptr, pl.R,
+                                       h->status + 1, h->status, nullptr, si, &h->launches) != cudaSuccess)
+        return fail_side(VLPROJ_ERR_CUDA);
     if (pl.M > 0) {
         ++h->launches;
         const int M = static_cast<int>(pl.M);
         vlp::vlp_geometry_kernel<<<(M + 255) / 256, 256, 0, si>>>(h->dviews.ptr, static_cast<int>(pl.views.size()),
                                                                   M, c.k, h->pos.ptr, pl.R, vlp::DEST_EMBED, nullptr,
                                                                   h->rowdest.ptr, nullptr, 0, pl.chunk, 0);
-        VLP_CUDA(cudaGetLastError());
+        if (cudaGetLastError() != cudaSuccess) return fail_side(VLPROJ_ERR_CUDA);
     }
     stage_end(h, 0, si);
     if (si != s) VLP_CUDA(cudaEventRecord(h->join, si));
@@ -549,7 +547,7 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
         vlp::vlp_embed_lookup_kernel<<<static_cast<unsigned>((n_ids + 7) / 8), 256, 0, si>>>(
             input_ids, n_ids, image_token_id, static_cast<const __nv_bfloat16*>(args->embed_table), args->vocab,
             static_cast<__nv_bfloat16*>(out_embeds), c.N2, h->status);
-        VLP_CUDA(cudaGetLastError());
+        if (cudaGetLastError() != cudaSuccess) return fail_side(VLPROJ_ERR_CUDA);
         VLP_CUDA(cudaEventRecord(h->join2, si));
     }
     if (pl.M == 0) {
@@ -558,18 +556,27 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
         return VLPROJ_OK;
     }
 
+    // An error past this point still orders the caller's stream after the side stream's
+    // work (the index and lookup kernels write pos and out_embeds), as a success does.
+    auto fail_joined = [&](int code) {
+        if (si != s) {
+            cudaStreamWaitEvent(s, h->join, 0);
+            if (lookup) cudaStreamWaitEvent(s, h->join2, 0);
+        }
+        return code;
+    };
     // 1-3. geometry, LayerNorm, GEMM1 -> H
     rc = run_merge_gemm1(h, pl, features, nullptr, vlp::DEST_NONE, h->H.ptr, pl.M, s, nullptr);
-    if (rc) return rc;
+    if (rc) return fail_joined(rc);
     // middle layers (depth > 2)
     const __nv_bfloat16* hlast = nullptr;
     rc = run_middle_layers(h, pl, s, &hlast);
-    if (rc) return rc;
-    VLP_CUDA(cudaStreamWaitEvent(s, h->join, 0));
+    if (rc) return fail_joined(rc);
+    if (cudaStreamWaitEvent(s, h->join, 0) != cudaSuccess) return fail_joined(VLPROJ_ERR_CUDA);
 
     // 4. GEMM2 + scatter (from the last hidden activation)
     if (h->tmH_ptr != hlast || h->tmH_rows != pl.M) {
-        if (encode_bf16_2d(&h->tmH, hlast, pl.M, c.N1, vlp::BM)) return VLPROJ_ERR_CUDA;
+        if (encode_bf16_2d(&h->tmH, hlast, pl.M, c.N1, vlp::BM)) return fail_joined(VLPROJ_ERR_CUDA);
         h->tmH_ptr = hlast;
         h->tmH_rows = pl.M;
     }
@@ -590,7 +597,7 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
     ++h->launches;
     rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(pick_bn(c.N2), h->pairs, h->tmH, h->tmW2, h->tmW2h, p,
                                                        h->num_sms, s);
-    if (rc) return rc;
+    if (rc) return fail_joined(rc);
     stage_end(h, 4, s);
 
     // 5. newline / separator rows
@@ -603,7 +610,7 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
                                                           static_cast<const __nv_bfloat16*>(sep),
                                                           static_cast<__nv_bfloat16*>(out_embeds), n_ids, c.N2,
                                                           h->status + 1);
-        VLP_CUDA(cudaGetLastError());
+        if (cudaGetLastError() != cudaSuccess) return fail_joined(VLPROJ_ERR_CUDA);
         stage_end(h, 5, s);
     }
     if (args->rows_out && pl.R > 0) {
@@ -611,7 +618,7 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
         vlp::vlp_gather_rows_kernel<<<static_cast<unsigned>((pl.R + 7) / 8), 256, 0, s>>>(
             h->pos.ptr, pl.R, static_cast<const __nv_bfloat16*>(out_embeds), n_ids, c.N2,
             static_cast<__nv_bfloat16*>(args->rows_out), h->status + 1);
-        VLP_CUDA(cudaGetLastError());
+        if (cudaGetLastError() != cudaSuccess) return fail_joined(VLPROJ_ERR_CUDA);
     }
     if (lookup) VLP_CUDA(cudaStreamWaitEvent(s, h->join2, 0));
     h->profiled_valid = h->profiling;

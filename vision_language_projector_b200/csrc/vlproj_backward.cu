@@ -163,8 +163,8 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     const bool want_recompute = l_min < depth || a->d_W2;     // G feeds dP, H^T feeds the weight gradients
 
     // scratch
-    const int nblocks = static_cast<int>((n_ids + vlp::SCAN_CHUNK - 1) / vlp::SCAN_CHUNK);
-    if (h->counts.ensure(std::max(nblocks, 1)) || h->pos.ensure(std::max<int64_t>(pl.R, 1))) return VLPROJ_ERR_CUDA;
+    const int nblocks = vlp::scan_blocks(n_ids);
+    if (h->counts.ensure(nblocks + 1) || h->pos.ensure(std::max<int64_t>(pl.R, 1))) return VLPROJ_ERR_CUDA;
     if (M > 0) {
         if (h->rowdest.ensure(M) || h->gmeta.ensure(M) || h->A.ensure(static_cast<size_t>(M) * K1) ||
             h->G.ensure(hslab * (depth - 1)) || h->Ht.ensure(tslab * (depth - 1)) ||
@@ -186,15 +186,8 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
 
     // 6. placeholder index, count check, destinations and gather data
     stage_begin(h, 6, s);
-    h->launches += nblocks > 0 ? 2 : 1;
-    if (nblocks > 0) {
-        vlp::vlp_count_kernel<<<nblocks, vlp::SCAN_THREADS, 0, s>>>(a->input_ids, n_ids, a->image_token_id,
-                                                                    h->counts.ptr);
-        VLP_CUDA(cudaGetLastError());
-    }
-    vlp::vlp_compact_kernel<<<std::max(nblocks, 1), vlp::SCAN_THREADS, 0, s>>>(
-        a->input_ids, n_ids, a->image_token_id, h->counts.ptr, nblocks, h->pos.ptr, pl.R, h->status + 1, h->status);
-    VLP_CUDA(cudaGetLastError());
+    VLP_CUDA(vlp::enqueue_placeholder_index(a->input_ids, n_ids, a->image_token_id, h->counts.ptr, h->pos.ptr, pl.R,
+                                            h->status + 1, h->status, nullptr, s, &h->launches));
     if (M == 0) {
         stage_end(h, 6, s);
         rc = zero_outputs(a, c, K1, pl.P, s);

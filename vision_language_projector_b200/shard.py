@@ -57,16 +57,23 @@ def plan_shard(image_seq: Sequence[int], views_per_image: Sequence[int], grid_hw
 
 
 def allreduce_gradients(grads: dict, group=None) -> None:
-    """Sum every gradient tensor of ``grads`` over the ranks of ``group`` in place.
+    """Sum every parameter gradient of ``grads`` over the ranks of ``group`` in place.
 
     Values may be tensors or lists of tensors (the middle layers' "W_mid" / "b_mid"),
     all of one dtype and device; keys are visited in sorted order on every rank. The
-    tensors are packed into one buffer, so the exchange is a single all-reduce."""
+    tensors are packed into one buffer, so the exchange is a single all-reduce.
+
+    The "features" entry (the gradient with respect to this rank's own feature rows)
+    is left as it is: it belongs to the rank's shard of the batch, its size differs
+    from rank to rank, and summing it across ranks would mix different patches. So
+    ``Projector.backward``'s whole ``grads`` dict can be passed unchanged."""
     import torch
     import torch.distributed as dist
 
     tensors = []
     for key in sorted(grads):
+        if key == "features":
+            continue
         v = grads[key]
         tensors.extend(v if isinstance(v, (list, tuple)) else [v])
     if not tensors:
