@@ -409,7 +409,8 @@ def main():
         n_special = R - M
         algo = {"index": 16 * n_ids + 4 * R,                      # ids read by count and compact, pos written
                 "geometry": 12 * M,                              # pos read, rowdest + gather data written
-                "layernorm": P * wl.C * feat_b + M * wl.K1 * 2,  # features in, merged bf16 A out
+                # features in; out: the merged bf16 A (fp32 features) or 8 B of statistics per patch
+                "layernorm": P * wl.C * feat_b + (M * wl.K1 * 2 if wl.feat_fp32 else 8 * M * wl.k * wl.k),
                 "special_rows": 4 * n_special * wl.N2}           # learned row read, placeholder row written
         b = algo.get(dom)
         achieved = None if b is None else b / (avg[dom] / 1000.0) / 1e9
@@ -428,7 +429,8 @@ def main():
     traffic_model = {
         "algorithmic_bytes": P_step * wl.C * feat_b + R_step * wl.N2 * 2 + 8 * n_ids_step,
         "hidden_round_trip_bytes": 2 * M * wl.N1 * 2,
-        "merged_a_round_trip_bytes": 2 * M * wl.K1 * 2 if wl.has_ln or wl.feat_fp32 else 0,
+        "merged_a_round_trip_bytes": 2 * M * wl.K1 * 2 if wl.feat_fp32 else 0,
+        "layernorm_statistics_bytes": 2 * 8 * M * wl.k * wl.k if wl.has_ln and not wl.feat_fp32 else 0,
         "weights_bytes": 2 * (wl.N1 * wl.K1 + wl.N2 * wl.N1),
         "note": "per step and GPU; the hidden and merged-A round trips are implementation costs, not algorithmic",
     }

@@ -288,14 +288,20 @@ int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
                           const int32_t* spatial_crop, int32_t n_images, int64_t* rows_out);
 
 /* How GEMM1 fetches each merged token's k x k neighbourhood from the features:
- *   VLPROJ_GATHER_AUTO    (default) with a pre-merge LayerNorm or fp32 features, the
- *                         LayerNorm / convert pass writes its bf16 output directly in
- *                         merged-token order and GEMM1 reads it as a plain matrix;
- *                         otherwise BOX when every view has the same grid, k divides it
- *                         and w' = w/k divides 128; else IM2COL when every view has the
- *                         same grid; else CPASYNC (measured faster for mixed grids).
- *                         The modes below apply the LayerNorm pass in patch order and
- *                         gather from its output;
+ *   VLPROJ_GATHER_AUTO    (default) with bf16 features and a pre-merge LayerNorm,
+ *                         THREADS: only per-patch statistics (8 bytes per patch) go
+ *                         through memory, the normalised merged operand never does;
+ *                         with fp32 features the convert (and LayerNorm) pass writes its
+ *                         bf16 output directly in merged-token order and GEMM1 reads it
+ *                         as a plain matrix; otherwise BOX when every view has the same
+ *                         grid, k divides it and w' = w/k divides 128; else IM2COL when
+ *                         every view has the same grid; else CPASYNC (measured faster
+ *                         for mixed grids). BOX, IM2COL and CPASYNC apply a LayerNorm
+ *                         pass in patch order and gather from its output;
+ *   VLPROJ_GATHER_THREADS four extra warps per CTA gather each row by 16-byte cp.async
+ *                         (zero-filled pad), on CTA pairs too, and with a LayerNorm
+ *                         normalise the stage in shared memory from the statistics pass
+ *                         before the tensor cores read it;
  *   VLPROJ_GATHER_BOX     one 5D tiled TMA box per K-block: the features seen as
  *                         (c, dx, j, dy, merged row); falls back to IM2COL when the
  *                         grids are not regular as above;
@@ -305,7 +311,13 @@ int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
  *                         one map per view with each view's rows padded to 32;
  *   VLPROJ_GATHER_CPASYNC 16-byte cp.async copies per row (zero-filled pad).
  * All give the same bits. */
-enum { VLPROJ_GATHER_IM2COL = 0, VLPROJ_GATHER_CPASYNC = 1, VLPROJ_GATHER_AUTO = 2, VLPROJ_GATHER_BOX = 3 };
+enum {
+    VLPROJ_GATHER_IM2COL = 0,
+    VLPROJ_GATHER_CPASYNC = 1,
+    VLPROJ_GATHER_AUTO = 2,
+    VLPROJ_GATHER_BOX = 3,
+    VLPROJ_GATHER_THREADS = 4
+};
 int vlproj_set_gather_mode(vlproj_handle* h, int mode);
 
 /* GEMM tile shape. enable = 1 (default): 256 x 256 tiles run on pairs of CTAs

@@ -200,3 +200,98 @@ def backward(features: np.ndarray, grid_hw: np.ndarray, spatial_crop: Optional[n
     if magnitudes:
         g["mag"] = mag
     return g
+
+
+def backward_image_sampled(feats, hw, k: int, params: dict, crop: Optional[tuple], d_rows: np.ndarray,
+                           units: np.ndarray, tokens: dict, ln_eps: float = 1e-5, gvp: str = "head") -> dict:
+    """The share of one image in selected gradient entries, for a dense ``d_out``
+    (depth 2, bf16 quantisation as in `backward`). Every entry is a sum over the image's
+    merged tokens, so the batch value is the sum of the images' shares.
+
+    ``feats[v]`` / ``hw[v]``: the image's views as in `projector.project_image`;
+    ``d_rows``: d_out at the image's placeholder rows, in assembled order; ``units``: the
+    hidden units j whose columns are sampled; ``tokens``: {view index in the image:
+    merged-token indices} whose patches' feature gradients are wanted.
+
+    Returns, each with its magnitude chain under "mag" (as in `backward`):
+      "W2_cols" (N2, |units|) = dW2[:, units];  "b1_sel" = db1[units];
+      "W1_rows" (|units|, K1) = dW1[units, :];  "b2" = db2 (all of it);
+      "newline", "sep" (tiled images); "features": {(view, patch row): gradient row}.
+    By linearity the hidden units are independent: column j of P = A W1^T + b1 needs only
+    row j of W1, and dW2[:, j], db1[j], dW1[j, :] need only that column. The feature
+    gradient of a token's patches needs that token's whole row of dP (all units); each
+    patch belongs to exactly one token, so its gradient row is complete."""
+    W1, b1, W2, b2 = params["W1"], params["b1"], params["W2"], params["b2"]
+    gamma, beta = params.get("gamma"), params.get("beta")
+    has_ln = gamma is not None
+    C = np.asarray(feats[0]).shape[1]
+    units = np.asarray(units, np.int64)
+    h0, w0 = hw[0]
+    hp, wp = O.merged_side(h0, k), O.merged_side(w0, k)
+    row_map = _image_row_map(hp, wp, crop, len(feats), gvp)
+    tok_rows = np.full(len(feats) * hp * wp, -1, np.int64)
+    tok_rows[row_map[row_map >= 0]] = np.flatnonzero(row_map >= 0)
+    out = {"W2_cols": np.zeros((W2.shape[0], len(units))), "b1_sel": np.zeros(len(units)),
+           "W1_rows": np.zeros((len(units), W1.shape[1])), "b2": np.zeros(W2.shape[0]), "features": {}}
+    mag = {"W2_cols": np.zeros_like(out["W2_cols"]), "b1_sel": np.zeros(len(units)),
+           "W1_rows": np.zeros_like(out["W1_rows"]), "b2": np.zeros(W2.shape[0]), "features": {}}
+    if crop is not None:
+        out["newline"] = d_rows[row_map == -1].sum(axis=0)
+        out["sep"] = d_rows[row_map == -2].sum(axis=0)
+        mag["newline"] = np.abs(d_rows[row_map == -1]).sum(axis=0)
+        mag["sep"] = np.abs(d_rows[row_map == -2]).sum(axis=0)
+    for vi, x in enumerate(feats):
+        x = np.asarray(x, np.float64)
+        h, w = hw[vi]
+        if has_ln:
+            mu = x.mean(axis=1, keepdims=True)
+            rstd = 1.0 / np.sqrt(((x - mu) ** 2).mean(axis=1, keepdims=True) + ln_eps)
+            xhat = (x - mu) * rstd
+            src = xhat * gamma + beta
+        else:
+            src = x
+        a = O.unshuffle(O.round_bf16(src).reshape(h, w, C), k)
+        dy = d_rows[tok_rows[vi * hp * wp:(vi + 1) * hp * wp]]
+        out["b2"] += dy.sum(axis=0)
+        mag["b2"] += np.abs(dy).sum(axis=0)
+        # the sampled hidden units, every token
+        p = a @ W1[units].T + b1[units]
+        hid = O.round_bf16(O.gelu(p))
+        gp_ = gelu_grad(p)
+        dp = (dy @ W2[:, units]) * gp_
+        m_dp = np.abs(dp) + 2.0 ** -16 * (np.abs(dy) @ np.abs(W2[:, units])) * np.abs(gp_)
+        out["W2_cols"] += dy.T @ hid
+        mag["W2_cols"] += np.abs(dy).T @ np.abs(hid)
+        out["b1_sel"] += dp.sum(axis=0)
+        mag["b1_sel"] += m_dp.sum(axis=0)
+        out["W1_rows"] += dp.T @ a
+        mag["W1_rows"] += m_dp.T @ np.abs(a)
+        # the sampled tokens, every hidden unit: their patches' feature gradients
+        for t in np.asarray(tokens.get(vi, ()), np.int64):
+            pt = a[t] @ W1.T + b1
+            gt = gelu_grad(pt)
+            dpt = (dy[t] @ W2) * gt
+            m_dpt = np.abs(dpt) + 2.0 ** -16 * (np.abs(dy[t]) @ np.abs(W2)) * np.abs(gt)
+            da, m_da = dpt @ W1, m_dpt @ np.abs(W1)
+            i, j = int(t) // wp, int(t) % wp
+            for dyy in range(k):
+                for dxx in range(k):
+                    r, s = k * i + dyy, k * j + dxx
+                    if r >= h or s >= w:
+                        continue
+                    cols = np.arange(C) * k * k + dyy * k + dxx          # channel-outer merge order
+                    dsrc, m_src = da[cols], m_da[cols]
+                    prow = r * w + s
+                    if has_ln:
+                        gg = dsrc * gamma
+                        xr = xhat[prow]
+                        dx = rstd[prow, 0] * (gg - gg.mean() - xr * (gg * xr).mean())
+                        mg = m_src * np.abs(gamma)
+                        ax = np.abs(xr)
+                        m_dx = rstd[prow, 0] * (mg + mg.mean() + ax * (mg * ax).mean())
+                    else:
+                        dx, m_dx = dsrc, m_src
+                    out["features"][(vi, prow)] = dx
+                    mag["features"][(vi, prow)] = m_dx
+    out["mag"] = mag
+    return out

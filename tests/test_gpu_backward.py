@@ -298,3 +298,88 @@ def test_backward_full_size_sparse_gradient(name):
     rc, got = run_backward(case, proj, dev, d_dev)
     assert rc == vp.OK and proj.status() == vp.OK
     assert_grads_close(got, oracle_grads(case, Sparse(), skip_zero_rows=True), name)
+
+
+@pytest.mark.parametrize("name", ["stress", "dsvit", "vl2", "moonvit"])
+def test_backward_full_size_dense_gradient(name):
+    """Full-size workload with d_out ~N(0, 1) on every id. Checked against the oracle's
+    per-image shares of sampled entries (oracle/backward.py, backward_image_sampled):
+    dW2 columns, db1 and dW1 rows of five hidden units (the first, the last and three
+    seeded), all of db2 (and the newline / separator gradients when tiled), and the
+    feature gradient of every patch of one seeded token per image. Every sampled entry
+    is a sum over all merged tokens of the batch."""
+    from concurrent.futures import ThreadPoolExecutor
+    wl = W.WORKLOADS[name]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    n_ids = len(case.ids)
+    bits = W.grad_out_blocks(wl, n_ids, seed=2)
+    d_dev = dev_bf16(bits)
+    shapes = grad_shapes(case)
+    names = ["W1", "b1", "W2", "b2", "features"] + (["newline", "sep"] if wl.tiled else [])
+    grads = {n: torch.full(shapes[n], float("nan"), dtype=torch.float32, device="cuda") for n in names}
+    rc = proj.backward(dev.feats, case.hw, case.crop, dev.ids, W.IMAGE_TOKEN_ID, d_dev, grads, n_images=wl.n_images)
+    assert rc == vp.OK and proj.status() == vp.OK
+    del d_dev
+
+    rng = np.random.default_rng(11)
+    units = np.unique(np.concatenate([[0, wl.N1 - 1], rng.choice(wl.N1, 3, replace=False)]))
+    per = wl.views_per_image
+    hw = case.hw
+    offs = np.concatenate([[0], np.cumsum(hw[:, 0].astype(np.int64) * hw[:, 1])])
+    pos = O.placeholder_positions(case.ids, W.IMAGE_TOKEN_ID)
+    rbase = np.concatenate([[0], np.cumsum(case.rows)])
+    params = O.params_f64(case.w)
+    picks = []
+    for img in range(wl.n_images):
+        vi = int(rng.integers(per))
+        v = img * per + vi
+        picks.append((vi, int(rng.integers(O.tokens_untiled(int(hw[v, 0]), int(hw[v, 1]), wl.k)))))
+
+    def share(img):
+        views = list(range(img * per, (img + 1) * per))
+        feats = [O.bf16_bits_to_f64(case.feats[offs[v]:offs[v + 1]]) for v in views]
+        vhw = [(int(hw[v, 0]), int(hw[v, 1])) for v in views]
+        crop = None if case.crop is None else (int(case.crop[img, 0]), int(case.crop[img, 1]))
+        d_rows = O.bf16_bits_to_f64(bits[pos[rbase[img]:rbase[img + 1]]])
+        vi, t = picks[img]
+        return B.backward_image_sampled(feats, vhw, wl.k, params, crop, d_rows, units, {vi: [t]}, wl.ln_eps, case.gvp)
+
+    with ThreadPoolExecutor(8) as ex:
+        parts = list(ex.map(share, range(wl.n_images)))
+    want, mag = {}, {}
+    for key in ("W2_cols", "b1_sel", "W1_rows", "b2") + (("newline", "sep") if wl.tiled else ()):
+        want[key] = sum(pt[key] for pt in parts)
+        mag[key] = sum(pt["mag"][key] for pt in parts)
+    got = {"W2_cols": grads["W2"][:, torch.from_numpy(units).cuda()], "b1_sel": grads["b1"][torch.from_numpy(units).cuda()],
+           "W1_rows": grads["W1"][torch.from_numpy(units).cuda()], "b2": grads["b2"]}
+    if wl.tiled:
+        got.update(newline=grads["newline"], sep=grads["sep"])
+    eps = {"W2_cols": EPS["W2"], "b2": EPS["b2"], "newline": EPS["newline"], "sep": EPS["sep"]}
+    worst = {}
+    for key, g in got.items():
+        g = g.double().cpu().numpy()
+        assert np.isfinite(g).all(), key
+        bound = eps.get(key, EPS_DP) * mag[key]
+        err = np.abs(g - want[key])
+        assert np.all(err[mag[key] == 0] == 0), key
+        live = mag[key] > 0
+        worst[key] = float((err[live] / bound[live]).max())
+        assert worst[key] <= 1.0, f"{name} {key}: max err / bound {worst[key]:.3f}"
+    # feature gradients of the sampled tokens' patches
+    rows, want_f, mag_f = [], [], []
+    for img, pt in enumerate(parts):
+        for (vi, prow), g in pt["features"].items():
+            rows.append(int(offs[img * per + vi]) + prow)
+            want_f.append(g)
+            mag_f.append(pt["mag"]["features"][(vi, prow)])
+    gf = grads["features"][torch.tensor(rows, device="cuda")].double().cpu().numpy()
+    want_f, mag_f = np.stack(want_f), np.stack(mag_f)
+    assert np.isfinite(gf).all()
+    err = np.abs(gf - want_f)
+    assert np.all(err[mag_f == 0] == 0)
+    live = mag_f > 0
+    worst["features"] = float((err[live] / (EPS_DP * mag_f[live])).max())
+    assert worst["features"] <= 1.0, f"{name} features: max err / bound {worst['features']:.3f}"
+    print(name, worst)

@@ -49,8 +49,10 @@ SMALL = {
 
 # (gather mode, 256 x 256 tiles on CTA pairs)
 MODES = [(vp.GATHER_AUTO, True), (vp.GATHER_AUTO, False), (vp.GATHER_IM2COL, True), (vp.GATHER_IM2COL, False),
-         (vp.GATHER_CPASYNC, True), (vp.GATHER_BOX, True), (vp.GATHER_BOX, False)]
-MODE_IDS = ["auto-pairs", "auto-single", "im2col-pairs", "im2col-single", "cpasync", "box-pairs", "box-single"]
+         (vp.GATHER_CPASYNC, True), (vp.GATHER_BOX, True), (vp.GATHER_BOX, False), (vp.GATHER_THREADS, True),
+         (vp.GATHER_THREADS, False)]
+MODE_IDS = ["auto-pairs", "auto-single", "im2col-pairs", "im2col-single", "cpasync", "box-pairs", "box-single",
+            "threads-pairs", "threads-single"]
 
 
 @pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
@@ -174,6 +176,21 @@ def test_box_and_im2col_agree_bit_for_bit():
 
 
 @pytest.mark.parametrize("name", ["dsvit", "vl2"])
+def test_thread_gather_agrees_bit_for_bit(name):
+    """The thread gather (cp.async by four extra warps, CTA pairs) fetches the same operand
+    bytes as the TMA box / im2col modes AUTO picks for these grids."""
+    wl = W.WORKLOADS[name]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    out_a = run(case, proj, dev)
+    proj.set_gather_mode(vp.GATHER_THREADS)
+    out_b = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["dsvit", "vl2"])
 def test_tile_pairs_agree_bit_for_bit(name):
     """256 x 256 tiles on CTA pairs and 128 x 256 tiles on single CTAs accumulate each
     output over the same K order, so they give identical bits."""
@@ -188,9 +205,10 @@ def test_tile_pairs_agree_bit_for_bit(name):
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
 
 
-def test_merged_layernorm_path_agrees_bit_for_bit():
-    """With a LayerNorm, AUTO writes the normalised features straight in merged-token
-    order; the patch-order LayerNorm + gather path reads the same values."""
+def test_fused_layernorm_path_agrees_bit_for_bit():
+    """With a LayerNorm and bf16 features, AUTO normalises the gathered patches inside
+    GEMM1 from per-patch statistics; the patch-order LayerNorm pass + cp.async gather
+    path reads the same values, so the outputs are identical."""
     wl = W.WORKLOADS["moonvit"]
     case = make_case(wl)
     proj = make_projector(case)

@@ -331,3 +331,72 @@ def test_pins_catch_a_swapped_view_order(monkeypatch):
     g = _grads(c)
     fd = _fd(c, "W2")
     assert not np.allclose(g["W2"], fd, rtol=0, atol=2e-6 * max(1.0, float(np.abs(fd).max())))
+
+
+def _sampled_sum(c, units, tokens_of, gvp="head"):
+    """backward_image_sampled summed over the images of case c (quantised, as the GPU)."""
+    grid_hw, crop, k = c["grid_hw"], c["spatial_crop"], c["k"]
+    offs = np.concatenate([[0], np.cumsum(grid_hw[:, 0].astype(np.int64) * grid_hw[:, 1])])
+    pos = O.placeholder_positions(c["ids"], IMG)
+    rows = O.image_rows(grid_hw, k, crop)
+    per = [1] * len(grid_hw) if crop is None else [1 + int(a) * int(b) for a, b in crop]
+    total, v0, r0 = None, 0, 0
+    for img, n in enumerate(per):
+        views = list(range(v0, v0 + n))
+        feats = [c["features"][offs[v]:offs[v + 1]] for v in views]
+        hw = [(int(grid_hw[v, 0]), int(grid_hw[v, 1])) for v in views]
+        cr = None if crop is None else (int(crop[img, 0]), int(crop[img, 1]))
+        d_rows = c["d_out"][pos[r0:r0 + rows[img]]]
+        part = B.backward_image_sampled(feats, hw, k, c["params"], cr, d_rows, units, tokens_of(img, views), 1e-5,
+                                        gvp)
+        part["features"] = {(views[vi], prow): g for (vi, prow), g in part["features"].items()}
+        part["mag"]["features"] = {(views[vi], prow): g for (vi, prow), g in part["mag"]["features"].items()}
+        if total is None:
+            total = part
+        else:
+            for d, s in ((total, part), (total["mag"], part["mag"])):
+                for key, val in s.items():
+                    if key == "mag":
+                        continue
+                    if key == "features":
+                        d[key].update(val)
+                    else:
+                        d[key] = d[key] + val
+        v0, r0 = v0 + n, r0 + rows[img]
+    return total, offs
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("gvp", ["head", "tail"])
+def test_sampled_backward_equals_the_whole_backward(name, gvp):
+    """The per-image, per-unit restriction used for full-size checks gives exactly the
+    entries of the whole backward (depth 2, quantised) and of its magnitude chain."""
+    c = _case(**CASES[name])
+    if c["spatial_crop"] is None and gvp == "tail":
+        pytest.skip("untiled")
+    full = B.backward(c["features"], c["grid_hw"], c["spatial_crop"], c["k"], c["params"], c["ids"], IMG,
+                      c["d_out"], 1e-5, feat_is_bf16_bits=False, quantise=True, gvp=gvp, magnitudes=True)
+    N1 = c["params"]["W1"].shape[0]
+    units = np.array([0, N1 - 1, N1 // 2])
+    k = c["k"]
+
+    def tokens_of(img, views):
+        out = {}
+        for vi, v in enumerate(views):
+            n = O.tokens_untiled(int(c["grid_hw"][v, 0]), int(c["grid_hw"][v, 1]), k)
+            out[vi] = np.arange(n)                           # every token: every patch is checked
+        return out
+
+    got, offs = _sampled_sum(c, units, tokens_of, gvp)
+    for src, ref in ((got, full), (got["mag"], full["mag"])):
+        np.testing.assert_allclose(src["W2_cols"], ref["W2"][:, units], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(src["b1_sel"], ref["b1"][units], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(src["W1_rows"], ref["W1"][units], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(src["b2"], ref["b2"], rtol=1e-12, atol=1e-13)
+        if c["spatial_crop"] is not None:
+            np.testing.assert_allclose(src["newline"], ref["newline"], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(src["sep"], ref["sep"], rtol=1e-12, atol=1e-13)
+        P = int(offs[-1])
+        assert len(src["features"]) == P                     # every patch covered once
+        for (v, prow), g in src["features"].items():
+            np.testing.assert_allclose(g, ref["features"][offs[v] + prow], rtol=1e-11, atol=1e-13)

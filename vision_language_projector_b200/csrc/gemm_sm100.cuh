@@ -55,6 +55,8 @@ constexpr int BM = 128;
 constexpr int BK = 64;                  // 64 bf16 = one 128-byte swizzle row
 constexpr int GEMM_THREADS = 256;
 constexpr int GATHER_THREADS = 64;
+constexpr int GEMM_THREADS_TG = 384;    // thread-gather modes: warps 8-11 fetch (and normalise) A
+constexpr int TG_THREADS = 128;
 constexpr int EPI_GELU = 0;
 constexpr int EPI_SCATTER = 1;
 constexpr int EPI_BWD_H = 2;
@@ -66,6 +68,8 @@ constexpr int A_TILE = 0;               // dense row-major A, tiled TMA
 constexpr int A_IM2COL = 1;             // merge-gather by TMA im2col
 constexpr int A_CPASYNC = 2;            // merge-gather by cp.async
 constexpr int A_BOX5 = 3;               // merge-gather by one 5D tiled TMA box (regular grids)
+constexpr int A_TGATHER = 4;            // merge-gather by 128 threads' cp.async, CTA pairs allowed
+constexpr int A_TGATHER_LN = 5;         // ... then the pre-merge LayerNorm applied in shared memory
 constexpr uint64_t DRAIN_NS = 1000000000ull;
 constexpr int ERR_TIMEOUT = -5;
 
@@ -74,29 +78,42 @@ constexpr int ERR_TIMEOUT = -5;
 // six stages fit.
 // Epilogues that send bf16 tiles out by TMA store stage them here, per epilogue warp in
 // 32 x 32 bf16 blocks: GELU two (two chunks in flight), DGELU two (a chunk of dP and of
-// dP^T), BWD_H three (G, H^T and, for a following layer, H).
+// dP^T), BWD_H three (G, H^T and, for a following layer, H). SCATTER stages 32 rows x 64
+// columns (the two blocks side by side) so that its stores write whole row segments.
 constexpr int EPI_BLOCK_BYTES = 32 * 32 * 2;
 __host__ __device__ constexpr int epi_blocks(int epi) {
-    return epi == EPI_BWD_H ? 3 : (epi == EPI_GELU || epi == EPI_DGELU || epi == EPI_BF16) ? 2 : 0;
+    return epi == EPI_BWD_H ? 3 : (epi == EPI_GELU || epi == EPI_DGELU || epi == EPI_BF16 || epi == EPI_SCATTER) ? 2 : 0;
 }
 __host__ __device__ constexpr int epi_stage_bytes(int epi) { return 4 * epi_blocks(epi) * EPI_BLOCK_BYTES; }
 
-template <int BN, int kCtas = 1, int kEpiBytes = 0>
+// kAuxBytes: bytes per stage beside the operands (the LayerNorm statistics of the stage's
+// 128 rows in A_TGATHER_LN), kept after the ring; such layouts size the ring from the whole
+// 227 KB a CTA may use.
+template <int BN, int kCtas = 1, int kEpiBytes = 0, int kAuxBytes = 0>
 struct GemmLayout {
     static constexpr int B_ROWS = BN / kCtas;
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
-    static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;
+    static constexpr int RING_BUDGET = kAuxBytes ? 232448 - 1024 - 1024 - kEpiBytes : 196608;
+    static constexpr int STAGES_FIT = RING_BUDGET / (STAGE_BYTES + kAuxBytes);
+    static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
+    static constexpr int AUX_OFFSET = STAGES * STAGE_BYTES;
+    static constexpr int AUX_BYTES_PER = kAuxBytes;
+    static constexpr int EPI_OFFSET = AUX_OFFSET + STAGES * kAuxBytes;
     static constexpr int BAR_OFFSET = EPI_OFFSET + kEpiBytes;
-    // full_tma[S], full_gather[S], empty[S], tmem_full[2], tmem_empty[2], drain
-    static constexpr int NUM_BARS = 3 * STAGES + 5;
+    // full_tma[S], full_gather[S], empty[S], full_local[S], tmem_full[2], tmem_empty[2], drain
+    static constexpr int NUM_BARS = 4 * STAGES + 5;
     static constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
     static constexpr int BYTES = MISC_OFFSET + 16;
     static constexpr int SMEM_ALLOC = BYTES + 1024;      // room to align the base to 1024 B
     static constexpr uint32_t TMEM_COLS = 2 * BN;        // two accumulators
 };
+
+// Statistics bytes per stage in A_TGATHER_LN: (mean, rstd) of each of the 128 rows.
+__host__ __device__ constexpr int a_aux_bytes(int amode) { return amode == A_TGATHER_LN ? BM * 8 : 0; }
+__host__ __device__ constexpr bool a_thread_gather(int amode) { return amode == A_TGATHER || amode == A_TGATHER_LN; }
+__host__ __device__ constexpr int gemm_threads(int amode) { return a_thread_gather(amode) ? GEMM_THREADS_TG : GEMM_THREADS; }
 
 struct GemmParams {
     int M;                          // rows (merged tokens, each view's run padded in im2col varlen mode)
@@ -112,9 +129,15 @@ struct GemmParams {
     int chunk;                      // rows per im2col load: 128 (one map) or 32 (per-view maps)
     // A_BOX5: features seen as (c, dx, j, dy, merged row) with box (64, 1, w', 1, 128 / w')
     int box_rows;                   // merged rows per 128-row tile (128 / w')
-    // A_CPASYNC
+    // A_CPASYNC, A_TGATHER, A_TGATHER_LN
     const __nv_bfloat16* gsrc;      // bf16 patch features [P][C]
     const int2* gmeta;              // per row: {top-left patch index, (w << 16) | valid mask}
+    // A_TGATHER_LN: (mean, rstd) of the patch at tap p of row m at ln_stats[p * stats_ld + m],
+    // (0, 0) for a pad position or a row past M; gamma / beta [C] fp32
+    const float2* ln_stats;
+    int64_t stats_ld;               // a multiple of 256 rows
+    const float* ln_gamma;
+    const float* ln_beta;
     // output
     __nv_bfloat16* out;             // GEMM1: H; GEMM2: embeddings [out_rows][N]
     const int32_t* rowdest;         // destination row of each m (-1 = no write), or null = row m
@@ -208,15 +231,17 @@ __device__ __forceinline__ void write_row_block(const uint32_t (&packed)[16], ui
 }
 
 template <int BN, int kAMode, int kEpi, int kCtas>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     vlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmCt,
                     const __grid_constant__ CUtensorMap tmC2, const GemmParams p) {
-    using L = GemmLayout<BN, kCtas, epi_stage_bytes(kEpi)>;
+    using L = GemmLayout<BN, kCtas, epi_stage_bytes(kEpi), a_aux_bytes(kAMode)>;
     constexpr int S = L::STAGES;
     constexpr bool kPair = kCtas == 2;
     constexpr bool kGatherThreads = kAMode == A_CPASYNC;
-    static_assert(!(kPair && kGatherThreads), "the cp.async gather runs on single CTAs");
+    constexpr bool kTG = a_thread_gather(kAMode);          // warps 8-11 fetch A by cp.async
+    constexpr bool kLN = kAMode == A_TGATHER_LN;           // ... and normalise it in place
+    static_assert(!(kPair && kGatherThreads), "the 64-thread cp.async gather runs on single CTAs");
     static_assert(!kPair || BN == 256, "CTA pairs run 256 x 256 tiles");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -224,9 +249,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint64_t* full_tma = bars;
     uint64_t* full_gat = bars + S;
     uint64_t* empty = bars + 2 * S;
-    uint64_t* tmem_full = bars + 3 * S;
-    uint64_t* tmem_empty = bars + 3 * S + 2;
-    uint64_t* drain = bars + 3 * S + 4;
+    uint64_t* full_loc = bars + 3 * S;
+    uint64_t* tmem_full = bars + 4 * S;
+    uint64_t* tmem_empty = bars + 4 * S + 2;
+    uint64_t* drain = bars + 4 * S + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFFSET);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFFSET + 4);
 
@@ -236,10 +262,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const bool leader = rank == 0;
 
     if (threadIdx.x == 0) {
+        // "A ready" arrivals: the 64 gather threads (A_CPASYNC); in the thread-gather modes
+        // one per gather warp of every CTA (A_TGATHER_LN) or one relay thread per CTA
+        const uint32_t gat_count = kGatherThreads ? GATHER_THREADS : kLN ? 4 * kCtas : kTG ? kCtas : 1;
         for (int s = 0; s < S; ++s) {
             mbar_init(&full_tma[s], 1);
-            mbar_init(&full_gat[s], GATHER_THREADS);
+            mbar_init(&full_gat[s], gat_count);
             mbar_init(&empty[s], 1);
+            mbar_init(&full_loc[s], TG_THREADS);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tmem_full[a], 1);
@@ -290,7 +320,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             int issued = 0;
             bool ok = true;
             const int nch = (kAMode == A_IM2COL) ? BM / p.chunk : 0;
-            const uint32_t expect = (kAMode == A_CPASYNC ? 0 : L::A_BYTES * kCtas) + L::B_BYTES * kCtas;
+            const uint32_t expect = (kAMode == A_CPASYNC || kTG ? 0 : L::A_BYTES * kCtas) + L::B_BYTES * kCtas;
             for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
                 int m_blk, n_blk;
                 tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
@@ -387,7 +417,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full_tma[stage], phase, lim, abort_flag)) { ok = false; break; }
-                    if (kGatherThreads) {
+                    if (kGatherThreads || kTG) {
                         if (!mbar_wait_bounded(&full_gat[stage], phase, lim, abort_flag)) { ok = false; break; }
                         fence_proxy_async_smem();
                     }
@@ -423,6 +453,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_wait_bounded(drain, 0, DRAIN_NS, &never);
         }
     } else if (warp < 4) {
+        // ------------------------------------------------ relay (A_TGATHER): once a stage's
+        // cp.async copies of this CTA have landed, make them visible to the tensor cores'
+        // proxy and tell the pair leader's MMA thread
+        if (kTG && !kLN && warp == 2 && lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            const uint32_t gat_leader = kPair ? mapa_shared(smem_u32(&full_gat[0]), 0) : 0u;
+            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&full_loc[stage], phase, lim, abort_flag)) { ok = false; break; }
+                    fence_proxy_async_smem();
+                    if constexpr (kPair) mbar_arrive_cluster(gat_leader + 8u * static_cast<uint32_t>(stage));
+                    else mbar_arrive(&full_gat[stage]);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                latch_error(p.err, ERR_TIMEOUT);
+            }
+        }
         // ------------------------------------------------ A gather producers (A_CPASYNC)
         if (kGatherThreads) {
             const int gt = threadIdx.x - 64;          // 0..63
@@ -471,6 +523,140 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                     cp_async_arrive_noinc(&full_gat[stage]);
                     if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                latch_error(p.err, ERR_TIMEOUT);
+            }
+            cp_async_wait_all();
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------ thread gather (A_TGATHER[_LN], warps 8-11)
+        // Thread t copies 16-byte chunk (t & 7) of rows (t >> 3) + 16 i, i < 8, of every A
+        // stage with cp.async (a zero-filled chunk where the neighbour lies in the pad or the
+        // row is past M), into the 128-byte-swizzled place the tensor cores read. In
+        // A_TGATHER_LN the first 64 threads also copy the stage's (mean, rstd) pairs, and
+        // the warps normalise each stage in place once it has landed, LOOK stages behind the
+        // copies: y = bf16(((x - mean) * rstd) * gamma + beta) with packed fp32 arithmetic
+        // (the same operations, in the same order, as the LayerNorm kernels), exactly 0 at
+        // a pad position. Then every lane fences its shared-memory writes to the async
+        // proxy and lane 0 of each warp arrives on the pair leader's "A ready" barrier.
+        if constexpr (kTG) {
+            constexpr int LOOK = S - 2 > 0 ? S - 2 : 1;
+            const int gt = threadIdx.x - 256;
+            const int chunk = gt & 7;
+            const int rsub = gt >> 3;                                 // rows rsub + 16 i
+            const uint32_t swz = static_cast<uint32_t>((chunk ^ (rsub & 7)) * 16);
+            const uint32_t gat_leader = kPair ? mapa_shared(smem_u32(&full_gat[0]), 0) : 0u;
+            int stage = 0, tstage = 0, tkb = 0;
+            uint32_t phase = 0, tphase = 0;
+            int pending = 0;
+            bool ok = true;
+            // normalise the oldest issued stage in place and hand it to the MMA
+            auto transform_one = [&]() -> bool {
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_loc[tstage], tphase, lim, abort_flag)))
+                    return false;
+                uint8_t* sa = smem + tstage * L::STAGE_BYTES;
+                const float2* st = reinterpret_cast<const float2*>(smem + L::AUX_OFFSET + tstage * L::AUX_BYTES_PER);
+                const int c0 = (tkb - (tkb / cblocks) * cblocks) * BK + chunk * 8;
+                const float4 g0 = __ldg(reinterpret_cast<const float4*>(p.ln_gamma + c0));
+                const float4 g1 = __ldg(reinterpret_cast<const float4*>(p.ln_gamma + c0) + 1);
+                const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.ln_beta + c0));
+                const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.ln_beta + c0) + 1);
+                const uint64_t gg[4] = {f2_pack(g0.x, g0.y), f2_pack(g0.z, g0.w), f2_pack(g1.x, g1.y),
+                                        f2_pack(g1.z, g1.w)};
+                const uint64_t bb[4] = {f2_pack(b0.x, b0.y), f2_pack(b0.z, b0.w), f2_pack(b1.x, b1.y),
+                                        f2_pack(b1.z, b1.w)};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = rsub + 16 * i;
+                    const float2 ms = st[r];
+                    uint4* cell = reinterpret_cast<uint4*>(sa + r * 128 + swz);
+                    uint4 u = *cell;
+                    if (ms.y == 0.0f) {
+                        u = make_uint4(0, 0, 0, 0);               // pad position: exact zero
+                    } else {
+                        const uint64_t nm = f2_splat(-ms.x), r2 = f2_splat(ms.y);
+                        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint64_t d =
+                                f2_add(f2_pack(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)), nm);
+                            float lo, hi;
+                            f2_unpack(f2_fma(f2_mul(d, r2), gg[e], bb[e]), lo, hi);
+                            w[e] = pack_bf16x2(lo, hi);
+                        }
+                        u = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                    *cell = u;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (kPair) mbar_arrive_cluster(gat_leader + 8u * static_cast<uint32_t>(tstage));
+                    else mbar_arrive(&full_gat[tstage]);
+                }
+                if (++tstage == S) { tstage = 0; tphase ^= 1; }
+                if (++tkb == kblocks) tkb = 0;
+                return true;
+            };
+            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+                int m_blk, n_blk;
+                tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
+                const int row0 = (m_blk * kCtas + static_cast<int>(rank)) * BM;      // this CTA's 128 rows
+                int base[8];
+                uint32_t wm[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int m = row0 + rsub + 16 * i;
+                    if (m < p.M) {
+                        const int2 g = __ldg(&p.gmeta[m]);
+                        base[i] = g.x;
+                        wm[i] = static_cast<uint32_t>(g.y);
+                    } else {
+                        base[i] = 0;
+                        wm[i] = 0;
+                    }
+                }
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    const int pos = kb / cblocks;
+                    const int c0 = (kb - pos * cblocks) * BK + chunk * 8;
+                    const int dy = pos / p.k, dx = pos - dy * p.k;
+                    int got = 0;
+                    if (lane == 0) got = mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag) ? 1 : 0;
+                    got = __shfl_sync(0xffffffffu, got, 0);
+                    if (!got) { ok = false; break; }
+                    const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = rsub + 16 * i;
+                        const int w = static_cast<int>(wm[i] >> 16);
+                        const bool valid = (wm[i] >> pos) & 1u;
+                        const int64_t prow = static_cast<int64_t>(base[i]) + dy * w + dx;
+                        const __nv_bfloat16* src = valid ? p.gsrc + prow * p.C + c0 : p.gsrc;
+                        cp_async_16(sa + r * 128 + swz, src, valid ? 16u : 0u);
+                    }
+                    if constexpr (kLN) {
+                        if (gt < 64) {      // the stage's statistics, two rows per thread
+                            const float2* src = p.ln_stats + static_cast<int64_t>(pos) * p.stats_ld + row0 + 2 * gt;
+                            cp_async_16(smem_u32(smem + L::AUX_OFFSET + stage * L::AUX_BYTES_PER) + 16 * gt, src, 16u);
+                        }
+                    }
+                    cp_async_arrive_noinc(&full_loc[stage]);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                    if constexpr (kLN) {
+                        if (++pending > LOOK) {
+                            if (!transform_one()) { ok = false; break; }
+                            --pending;
+                        }
+                    }
+                }
+            }
+            if constexpr (kLN) {
+                while (ok && pending > 0) {
+                    if (!transform_one()) { ok = false; break; }
+                    --pending;
                 }
             }
             if (!ok) {
@@ -595,6 +781,43 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         tma_store_2d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0, n0);
                         if (with_h) tma_store_2d(&tmC2, ebuf + 2 * EPI_BLOCK_BYTES, n0, m_row0);
                         bulk_commit_group();
+                    }
+                } else if constexpr (kEpi == EPI_SCATTER) {
+                    // The warp's 32 rows x 64 columns (two chunks) are staged in shared memory,
+                    // 128 bytes per row with the 16-byte chunk index XOR (row & 7), so both the
+                    // row-wise writes below and the column-wise reads after them touch every
+                    // bank once per 128 bytes. Then each store instruction writes 4 rows x 128
+                    // contiguous bytes: lane l takes 16-byte chunk (l & 7) of row 4 i + (l >> 3),
+                    // sent to that row's placeholder row (lanes share the destinations by shuffle).
+                    float bb[32];
+                    load_bias32(p.bias, n0, bb);
+                    const int half = c & 1;
+                    if (half == 0) __syncwarp();             // the previous block has been read out
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2)
+                        packed[j / 2] = pack_bf16x2(__uint_as_float(v[j]) + bb[j], __uint_as_float(v[j + 1]) + bb[j + 1]);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int q = half * 4 + j;
+                        *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                            make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                    }
+                    if (half == 1 || c + 1 == BN / 32 || n0 + 32 >= p.N) {
+                        __syncwarp();
+                        const int nb = n0 - half * 32;               // first column of the block
+                        const int q = lane & 7;
+                        const bool col_ok = q < 4 * (half + 1);      // a lone last chunk fills q < 4
+                        const int64_t my_dest = row_ok ? d : -1;
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int r = 4 * it + (lane >> 3);
+                            const int64_t dr = __shfl_sync(0xffffffffu, my_dest, r);
+                            if (dr >= 0 && col_ok) {
+                                const uint4 val = *reinterpret_cast<const uint4*>(ebuf + r * 128 + ((q ^ (r & 7)) << 4));
+                                *reinterpret_cast<uint4*>(p.out + dr * p.N + nb + q * 8) = val;
+                            }
+                        }
                     }
                 } else {
                     float bb[32];

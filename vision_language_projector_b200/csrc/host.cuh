@@ -213,6 +213,8 @@ struct Plan {
     bool im2col = true;     // GEMM1 gathers with TMA im2col (else cp.async)
     bool box5 = false;      // ... or with one 5D tiled box per K-block (regular grids)
     bool merged_ln = false; // ... or reads A written in token order by the LayerNorm pass
+    bool tgather = false;   // ... or gathers A by 128 threads' cp.async (CTA pairs allowed)
+    bool tgather_ln = false;// ... and applies the LayerNorm to it in shared memory
     int chunk = 128;        // im2col rows per load
 };
 
@@ -261,13 +263,23 @@ inline int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int3
         if (h != grid_hw[0] || w != grid_hw[1]) pl.uniform = false;
     }
     pl.chunk = pl.uniform ? 128 : 32;
-    if (gather_mode == VLPROJ_GATHER_AUTO && (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32)) {
-        // a LayerNorm / convert pass writes a bf16 copy anyway: write it as A itself
+    const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
+    if (gather_mode == VLPROJ_GATHER_AUTO && f32) {
+        // fp32 features need a conversion pass, which writes a bf16 copy anyway: write it
+        // as A itself, already merged
         pl.merged_ln = true;
         pl.im2col = false;
         gather_mode = VLPROJ_GATHER_CPASYNC;   // no padding, no chunk table
+    } else if ((gather_mode == VLPROJ_GATHER_AUTO && c.has_ln) || gather_mode == VLPROJ_GATHER_THREADS) {
+        // bf16 features with a LayerNorm: GEMM1 gathers the raw patches and normalises them
+        // in shared memory (only the per-patch statistics go through memory); with
+        // GATHER_THREADS and no LayerNorm (or fp32 features, converted first) it only gathers
+        pl.tgather = true;
+        pl.tgather_ln = c.has_ln && !f32;
+        pl.im2col = false;
+        gather_mode = VLPROJ_GATHER_CPASYNC;
     }
-    pl.im2col = !pl.merged_ln &&
+    pl.im2col = !pl.merged_ln && !pl.tgather &&
                 (gather_mode == VLPROJ_GATHER_IM2COL || (gather_mode == VLPROJ_GATHER_AUTO && pl.uniform));
     if (pl.uniform && n_views > 0 && (gather_mode == VLPROJ_GATHER_BOX || gather_mode == VLPROJ_GATHER_AUTO)) {
         const int h = grid_hw[0], w = grid_hw[1];
@@ -341,13 +353,13 @@ inline int raster_group(int N, int K, int BN) {
 template <int BN, int A, int E, int CTAS>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tct,
                 const CUtensorMap& tc2, GemmParams p, int num_sms, cudaStream_t s) {
-    using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E)>;
+    using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E), vlp::a_aux_bytes(A)>;
     auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
     if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN);
     VLP_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC));
     const int tiles = ((p.M + vlp::BM * CTAS - 1) / (vlp::BM * CTAS)) * ((p.N + BN - 1) / BN);
     cudaLaunchConfig_t cfg{};
-    cfg.blockDim = dim3(vlp::GEMM_THREADS);
+    cfg.blockDim = dim3(vlp::gemm_threads(A));
     cfg.dynamicSmemBytes = L::SMEM_ALLOC;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -426,6 +438,7 @@ struct vlproj_handle {
     std::vector<CUtensorMap> tmWm, tmWmh;
     vlp_host::DevBuf<int32_t> pos, rowdest, counts;
     vlp_host::DevBuf<int2> gmeta;
+    vlp_host::DevBuf<float2> lnstats;    // per (tap, GEMM row) LayerNorm statistics (A_TGATHER_LN)
     vlp_host::DevBuf<int4> chunks;
     vlp_host::DevBuf<vlp::ViewDesc> dviews;
     vlp_host::DevBuf<vlp::ImageDesc> dimages;

@@ -451,6 +451,29 @@ static __global__ void __launch_bounds__(256) vlp_ln_merge_kernel(const void* __
     ln_row_write<kF32In>(x, row, C, lane, gamma, beta, eps, has_ln, dst);
 }
 
+// LayerNorm statistics for the GEMM that normalises its A operand in shared memory
+// (A_TGATHER_LN): for GEMM row m < rows and tap p < k*k, stats[p * rows + m] = (mean,
+// rstd) of the patch at tap p of merged token m, computed by ln_row_stats (the same
+// arithmetic, in the same order, as every LayerNorm kernel here, so the normalised values
+// match theirs bit for bit), or (0, 0) where the tap lies in the high-end pad or m >= M.
+// One warp per (p, m); consecutive warps take consecutive m at one tap. Every patch of the
+// batch is read once (twice from the same warp: mean, then variance, the second from L1).
+template <bool kF32In>
+static __global__ void __launch_bounds__(256) vlp_ln_stats_kernel(const void* __restrict__ x,
+                                                           const ViewDesc* __restrict__ views, int n_views, int M,
+                                                           int64_t rows, int k, int C, float eps,
+                                                           float2* __restrict__ stats) {
+    const int lane = threadIdx.x & 31;
+    const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (item >= rows * k * k) return;
+    const int p = static_cast<int>(item / rows);
+    const int m = static_cast<int>(item - static_cast<int64_t>(p) * rows);
+    const int64_t src = m < M ? merge_source_row(views, n_views, m, p, k) : -1;
+    float mean = 0.f, rstd = 0.f;
+    if (src >= 0) ln_row_stats<kF32In>(x, src, C, lane, eps, mean, rstd);
+    if (lane == 0) stats[item] = make_float2(mean, rstd);
+}
+
 // Pipelined form for C <= 256 * kVec. Items are dealt to warps with a stride of the
 // grid's warp count; each warp keeps up to `stages` of its next patch rows in flight in
 // a shared-memory ring of its own, fetched by 1D bulk copies that complete on one

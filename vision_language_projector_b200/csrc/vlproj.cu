@@ -35,7 +35,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     const int n_chunks = im2col ? ((M + 2 * vlp::BM - 1) / (2 * vlp::BM)) * 2 * nch_tile : 0;
     // gather metadata only for GEMM1's cp.async gather (the merged-LayerNorm pass finds its
     // source rows in the view table, the box and im2col modes need none)
-    const bool cpasync = !im2col && !pl.box5 && !pl.merged_ln;
+    const bool cpasync = !im2col && !pl.box5 && !pl.merged_ln;       // includes the thread gather
     if (h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
     if (cpasync && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
     if (im2col && h->chunks.ensure(std::max(n_chunks, 1))) return VLPROJ_ERR_CUDA;
@@ -55,7 +55,20 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     }
 
     const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(features);
-    if (pl.merged_ln) {
+    // A_TGATHER_LN: rows of the statistics table, whole 256-row tiles
+    const int64_t stats_ld = (static_cast<int64_t>(M) + 255) / 256 * 256;
+    if (pl.tgather_ln) {
+        stage_begin(h, 2, s);
+        ++h->launches;
+        const int kk = c.k * c.k;
+        if (h->lnstats.ensure(static_cast<size_t>(stats_ld) * kk)) return VLPROJ_ERR_CUDA;
+        const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
+        const int64_t items = stats_ld * kk;
+        vlp::vlp_ln_stats_kernel<false><<<static_cast<unsigned>((items + 7) / 8), 256, 0, s>>>(
+            features, dviews, static_cast<int>(pl.views.size()), M, stats_ld, c.k, c.C, eps, h->lnstats.ptr);
+        VLP_CUDA(cudaGetLastError());
+        stage_end(h, 2, s);
+    } else if (pl.merged_ln) {
         stage_begin(h, 2, s);
         ++h->launches;
         if (h->A.ensure(static_cast<size_t>(M) * h->K1)) return VLPROJ_ERR_CUDA;
@@ -63,7 +76,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
         int rc = launch_ln_merge(h, features, dviews, static_cast<int>(pl.views.size()), M, eps, h->A.ptr, s);
         if (rc) return rc;
         stage_end(h, 2, s);
-    } else if (c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) {
+    } else if ((c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) && !pl.tgather_ln) {
         stage_begin(h, 2, s);
         ++h->launches;
         if (h->Xn.ensure(static_cast<size_t>(pl.P) * c.C)) return VLPROJ_ERR_CUDA;
@@ -134,12 +147,24 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     } else {
         p.gsrc = src;
         p.gmeta = h->gmeta.ptr;
+        if (pl.tgather_ln) {
+            p.ln_stats = h->lnstats.ptr;
+            p.stats_ld = stats_ld;
+            p.ln_gamma = h->gamma;
+            p.ln_beta = h->beta;
+        }
     }
 
     stage_begin(h, 3, s);
     ++h->launches;
     int rc;
-    if (pl.merged_ln)
+    if (pl.tgather_ln)
+        rc = launch_gemm_bn<vlp::A_TGATHER_LN, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                              h->num_sms, s, tmC);
+    else if (pl.tgather)
+        rc = launch_gemm_bn<vlp::A_TGATHER, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                           h->num_sms, s, tmC);
+    else if (pl.merged_ln)
         rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
                                                         h->num_sms, s, tmC);
     else if (pl.box5)
@@ -392,6 +417,7 @@ void vlproj_destroy(vlproj_handle* h) {
     h->rowdest.release();
     h->counts.release();
     h->gmeta.release();
+    h->lnstats.release();
     h->chunks.release();
     h->dviews.release();
     h->dimages.release();
@@ -425,7 +451,7 @@ int vlproj_set_tile_pairs(vlproj_handle* h, int enable) {
 
 int vlproj_set_gather_mode(vlproj_handle* h, int mode) {
     if (!h || (mode != VLPROJ_GATHER_IM2COL && mode != VLPROJ_GATHER_CPASYNC && mode != VLPROJ_GATHER_AUTO &&
-               mode != VLPROJ_GATHER_BOX))
+               mode != VLPROJ_GATHER_BOX && mode != VLPROJ_GATHER_THREADS))
         return VLPROJ_ERR_INVALID_ARG;
     h->gather_mode = mode;
     return VLPROJ_OK;

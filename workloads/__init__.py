@@ -217,6 +217,20 @@ def grad_out(wl: Workload, n_ids: int, seed: int = 0) -> np.ndarray:
     return _normal_bits(_rng(wl, _T_DOUT, 0, seed), (n_ids, wl.N2))
 
 
+def grad_out_blocks(wl: Workload, n_ids: int, seed: int = 0, threads: int = 8, block: int = 4096) -> np.ndarray:
+    """(n_ids, N2) bf16 bits ~N(0, 1), drawn in blocks of `block` rows from streams of
+    their own (so large batches are generated in parallel): a dense loss gradient."""
+    out = np.empty((n_ids, wl.N2), np.uint16)
+
+    def fill(b):
+        r0, r1 = b * block, min(n_ids, (b + 1) * block)
+        out[r0:r1] = _normal_bits(_rng(wl, _T_DOUT, 16 + b, seed), (r1 - r0, wl.N2))
+
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(fill, range((n_ids + block - 1) // block)))
+    return out
+
+
 def grad_out_rows(wl: Workload, n_rows: int, seed: int = 0) -> np.ndarray:
     """(n_rows, N2) bf16 bits ~N(0, 1): the nonzero rows of a sparse loss gradient."""
     return _normal_bits(_rng(wl, _T_DOUT, 1, seed), (n_rows, wl.N2))
