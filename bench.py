@@ -57,6 +57,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--gather", default="auto", choices=["auto", "box", "im2col", "cpasync", "threads"],
+                    help="GEMM1's merge-gather (vlproj_set_gather_mode); auto = the library's choice")
     return ap.parse_args()
 
 
@@ -316,6 +318,8 @@ def main():
                         has_ln=wl.has_ln, ln_gamma=f32(wts["gamma"]), ln_beta=f32(wts["beta"]), ln_eps=wl.ln_eps,
                         feat_dtype=vp.FEAT_F32 if wl.feat_fp32 else vp.FEAT_BF16,
                         tile_tag=vp.TILE_2D if wl.tiled else vp.TILE_NONE)
+    proj.set_gather_mode({"auto": vp.GATHER_AUTO, "box": vp.GATHER_BOX, "im2col": vp.GATHER_IM2COL,
+                          "cpasync": vp.GATHER_CPASYNC, "threads": vp.GATHER_THREADS}[args.gather])
     feats = f32(feats_h) if wl.feat_fp32 else bf(feats_h)
     ids = torch.from_numpy(ids_h).cuda()
     prefill = bf(prefill_h)
@@ -569,6 +573,7 @@ def main():
             "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(workload_config(args, wl, M, int(sum(rows))), l2="flushed between steps (256 MiB write)",
+                           gather=args.gather,
                            parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
             "tflops_per_gpu": tflops,
             "pct_of_dense_bf16_peak": 100.0 * tflops / peaks.get("bf16_tflops"),

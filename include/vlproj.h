@@ -174,7 +174,9 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
  * memory: the same rows as vlproj_forward_ex's rows_out (every image's assembled rows,
  * newlines and separators included, images in order; "port DeepSeek-VL2",
  * Tile-sequence assembly), without the embedding buffer. The batch is cut into
- * `chunks` runs of whole images of about equal token count (0 = automatic); chunk j's
+ * `chunks` runs of whole images of about equal token count, the first and the last
+ * about half the others when there are three or more, since their copies overlap no
+ * projection (0 = automatic); chunk j's
  * features are copied to the device while chunk j-1 is projected and chunk j-2's rows
  * are copied back, on copy streams of the handle, so PCIe traffic in both directions
  * overlaps the GEMMs. Work is enqueued behind `stream`; the call returns without
@@ -288,20 +290,19 @@ int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
                           const int32_t* spatial_crop, int32_t n_images, int64_t* rows_out);
 
 /* How GEMM1 fetches each merged token's k x k neighbourhood from the features:
- *   VLPROJ_GATHER_AUTO    (default) with bf16 features and a pre-merge LayerNorm,
- *                         THREADS: only per-patch statistics (8 bytes per patch) go
- *                         through memory, the normalised merged operand never does;
- *                         with fp32 features the convert (and LayerNorm) pass writes its
- *                         bf16 output directly in merged-token order and GEMM1 reads it
- *                         as a plain matrix; otherwise BOX when every view has the same
- *                         grid, k divides it and w' = w/k divides 128; else IM2COL when
- *                         every view has the same grid; else CPASYNC (measured faster
- *                         for mixed grids). BOX, IM2COL and CPASYNC apply a LayerNorm
- *                         pass in patch order and gather from its output;
+ *   VLPROJ_GATHER_AUTO    (default) with a pre-merge LayerNorm or fp32 features, the
+ *                         LayerNorm / convert pass writes its bf16 output directly in
+ *                         merged-token order and GEMM1 reads it as a plain matrix;
+ *                         otherwise BOX when every view has the same grid, k divides it
+ *                         and w' = w/k divides 128; else IM2COL when every view has the
+ *                         same grid; else CPASYNC (measured faster for mixed grids).
+ *                         BOX, IM2COL and CPASYNC apply a LayerNorm pass in patch order
+ *                         and gather from its output;
  *   VLPROJ_GATHER_THREADS four extra warps per CTA gather each row by 16-byte cp.async
- *                         (zero-filled pad), on CTA pairs too, and with a LayerNorm
- *                         normalise the stage in shared memory from the statistics pass
- *                         before the tensor cores read it;
+ *                         (zero-filled pad), on CTA pairs too; with a LayerNorm on bf16
+ *                         features they normalise each landed stage in shared memory
+ *                         from per-patch statistics (8 bytes per patch), so no
+ *                         normalised or merged copy of the features exists in memory;
  *   VLPROJ_GATHER_BOX     one 5D tiled TMA box per K-block: the features seen as
  *                         (c, dx, j, dy, merged row); falls back to IM2COL when the
  *                         grids are not regular as above;

@@ -4,10 +4,9 @@ The classes are 2, 5 and 8 packed vectors per lane, and the two-pass form past
 C = 2048, with bf16 and fp32 features. The cases include a ring with more slots than
 the warp has items, and warps that walk more than 32 items (the source-row table is
 reloaded). For each case: the hidden activations against the oracle, the whole
-forward against the oracle, and bit for bit against each other: the default path
-(bf16 features: statistics pass + LayerNorm applied inside GEMM1; fp32 features: the
+forward against the oracle, and bit for bit against each other: the default path (the
 LayerNorm written already merged), the patch-order LayerNorm + cp.async gather path, and
-the thread-gather path.
+the thread gather (bf16 features: statistics pass + LayerNorm applied inside GEMM1).
 """
 import numpy as np
 import pytest
@@ -69,7 +68,7 @@ def test_merged_and_patch_order_layernorm_agree_bit_for_bit(name):
     case = _case(name)
     proj = make_projector(case)
     dev = DeviceInputs(case)
-    out_a = run(case, proj, dev)                     # AUTO: fused (bf16) or written already merged (fp32)
+    out_a = run(case, proj, dev)                     # AUTO: LayerNorm written already merged
     assert proj.status() == vp.OK
     check(case, out_a, dev)
     proj.set_gather_mode(vp.GATHER_CPASYNC)          # patch-order LayerNorm, GEMM1 gathers

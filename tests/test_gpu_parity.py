@@ -205,10 +205,10 @@ def test_tile_pairs_agree_bit_for_bit(name):
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
 
 
-def test_fused_layernorm_path_agrees_bit_for_bit():
-    """With a LayerNorm and bf16 features, AUTO normalises the gathered patches inside
-    GEMM1 from per-patch statistics; the patch-order LayerNorm pass + cp.async gather
-    path reads the same values, so the outputs are identical."""
+def test_layernorm_paths_agree_bit_for_bit():
+    """With a LayerNorm, AUTO writes the normalised features straight in merged-token
+    order; the patch-order LayerNorm + gather path and the thread gather that normalises
+    inside GEMM1 (from per-patch statistics) read the same values."""
     wl = W.WORKLOADS["moonvit"]
     case = make_case(wl)
     proj = make_projector(case)
@@ -216,8 +216,11 @@ def test_fused_layernorm_path_agrees_bit_for_bit():
     out_a = run(case, proj, dev)                     # AUTO
     proj.set_gather_mode(vp.GATHER_CPASYNC)
     out_b = run(case, proj, dev)
+    proj.set_gather_mode(vp.GATHER_THREADS)
+    out_c = run(case, proj, dev)
     assert proj.status() == vp.OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+    assert torch.equal(out_a.view(torch.int16), out_c.view(torch.int16))
 
 
 

@@ -264,16 +264,17 @@ inline int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int3
     }
     pl.chunk = pl.uniform ? 128 : 32;
     const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
-    if (gather_mode == VLPROJ_GATHER_AUTO && f32) {
-        // fp32 features need a conversion pass, which writes a bf16 copy anyway: write it
-        // as A itself, already merged
+    if (gather_mode == VLPROJ_GATHER_AUTO && (c.has_ln || f32)) {
+        // a LayerNorm / convert pass writes a bf16 copy anyway: write it as A itself,
+        // already merged, so GEMM1 reads a plain matrix by TMA tiles (measured faster than
+        // normalising inside GEMM1 behind the thread gather)
         pl.merged_ln = true;
         pl.im2col = false;
         gather_mode = VLPROJ_GATHER_CPASYNC;   // no padding, no chunk table
-    } else if ((gather_mode == VLPROJ_GATHER_AUTO && c.has_ln) || gather_mode == VLPROJ_GATHER_THREADS) {
-        // bf16 features with a LayerNorm: GEMM1 gathers the raw patches and normalises them
-        // in shared memory (only the per-patch statistics go through memory); with
-        // GATHER_THREADS and no LayerNorm (or fp32 features, converted first) it only gathers
+    } else if (gather_mode == VLPROJ_GATHER_THREADS) {
+        // GEMM1 gathers the raw patches itself and, with a LayerNorm on bf16 features,
+        // normalises them in shared memory (only the per-patch statistics go through
+        // memory); with fp32 features a convert / LayerNorm pass runs first
         pl.tgather = true;
         pl.tgather_ln = c.has_ln && !f32;
         pl.im2col = false;

@@ -124,6 +124,10 @@ extern "C" int vlproj_project_host(vlproj_handle* h, const vlproj_host_args* a, 
     const int auto_chunks = static_cast<int>(std::min<size_t>(16, std::max<size_t>(2, (feat_bytes + (8u << 20)) >> 24)));
     const int nc = std::max(1, std::min(n_images, a->chunks > 0 ? a->chunks : auto_chunks));
     const int64_t total_tok = full.M_real;
+    // The first run's copy in and the last run's copy out overlap no projection, so with
+    // three or more runs those two are half the size of the others.
+    std::vector<double> cum(nc + 1, 0.0);
+    for (int j = 0; j < nc; ++j) cum[j + 1] = cum[j] + ((nc >= 3 && (j == 0 || j == nc - 1)) ? 0.5 : 1.0);
     std::vector<Chunk> chunks;
     {
         int img = 0;
@@ -134,7 +138,7 @@ extern "C" int vlproj_project_host(vlproj_handle* h, const vlproj_host_args* a, 
             ch.view0 = img_view0[img];
             ch.patch0 = patch;
             ch.row0 = row;
-            const int64_t target = total_tok * (j + 1) / nc;
+            const int64_t target = static_cast<int64_t>(static_cast<double>(total_tok) * cum[j + 1] / cum[nc]);
             const int left = nc - j - 1;                       // chunks still to fill after this one
             do {
                 done_tok += img_tok[img];
