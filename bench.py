@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--gather", default="auto", choices=["auto", "box", "im2col", "cpasync", "threads"],
+    ap.add_argument("--gather", default="auto", choices=["auto", "box", "im2col", "cpasync", "threads", "fused", "merged"],
                     help="GEMM1's merge-gather (vlproj_set_gather_mode); auto = the library's choice")
     return ap.parse_args()
 
@@ -319,7 +319,8 @@ def main():
                         feat_dtype=vp.FEAT_F32 if wl.feat_fp32 else vp.FEAT_BF16,
                         tile_tag=vp.TILE_2D if wl.tiled else vp.TILE_NONE)
     proj.set_gather_mode({"auto": vp.GATHER_AUTO, "box": vp.GATHER_BOX, "im2col": vp.GATHER_IM2COL,
-                          "cpasync": vp.GATHER_CPASYNC, "threads": vp.GATHER_THREADS}[args.gather])
+                          "cpasync": vp.GATHER_CPASYNC, "threads": vp.GATHER_THREADS, "fused": vp.GATHER_FUSED,
+                          "merged": vp.GATHER_MERGED}[args.gather])
     feats = f32(feats_h) if wl.feat_fp32 else bf(feats_h)
     ids = torch.from_numpy(ids_h).cuda()
     prefill = bf(prefill_h)

@@ -298,6 +298,13 @@ int64_t vlproj_image_rows(const vlproj_config* cfg, const int32_t* grid_hw,
  *                         same grid; else CPASYNC (measured faster for mixed grids).
  *                         BOX, IM2COL and CPASYNC apply a LayerNorm pass in patch order
  *                         and gather from its output;
+ *   VLPROJ_GATHER_FUSED   four producer warps per CTA of GEMM1 write the merged (and
+ *                         LayerNorm'd or converted) operand rows into device memory, in
+ *                         256-row blocks by tap, a little ahead of the TMA tile loads that
+ *                         read them back (each waits for its block's tap to be complete):
+ *                         one kernel, the copy's writes overlapped with the MMAs;
+ *   VLPROJ_GATHER_MERGED  a LayerNorm / convert / merge pass writes the merged operand
+ *                         first, then GEMM1 reads it by TMA tiles;
  *   VLPROJ_GATHER_THREADS four extra warps per CTA gather each row by 16-byte cp.async
  *                         (zero-filled pad), on CTA pairs too; with a LayerNorm on bf16
  *                         features they normalise each landed stage in shared memory
@@ -317,7 +324,9 @@ enum {
     VLPROJ_GATHER_CPASYNC = 1,
     VLPROJ_GATHER_AUTO = 2,
     VLPROJ_GATHER_BOX = 3,
-    VLPROJ_GATHER_THREADS = 4
+    VLPROJ_GATHER_THREADS = 4,
+    VLPROJ_GATHER_FUSED = 5,
+    VLPROJ_GATHER_MERGED = 6
 };
 int vlproj_set_gather_mode(vlproj_handle* h, int mode);
 

@@ -6,7 +6,8 @@ the warp has items, and warps that walk more than 32 items (the source-row table
 reloaded). For each case: the hidden activations against the oracle, the whole
 forward against the oracle, and bit for bit against each other: the default path (the
 LayerNorm written already merged), the patch-order LayerNorm + cp.async gather path, and
-the thread gather (bf16 features: statistics pass + LayerNorm applied inside GEMM1).
+the thread gather (bf16 features: statistics pass + LayerNorm applied inside GEMM1), and
+the fused producer warps (LayerNorm-merge written inside GEMM1 ahead of its TMA loads).
 """
 import numpy as np
 import pytest
@@ -75,9 +76,10 @@ def test_merged_and_patch_order_layernorm_agree_bit_for_bit(name):
     out_b = run(case, proj, dev)
     assert proj.status() == vp.OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
-    for pairs in (True, False):                      # thread gather, CTA pairs and single CTAs
-        proj.set_gather_mode(vp.GATHER_THREADS)
-        proj.set_tile_pairs(pairs)
-        out_c = run(case, proj, dev)
-        assert proj.status() == vp.OK
-        assert torch.equal(out_a.view(torch.int16), out_c.view(torch.int16)), f"pairs={pairs}"
+    for mode in (vp.GATHER_THREADS, vp.GATHER_FUSED):  # thread gather, fused producers
+        for pairs in (True, False):                      # CTA pairs and single CTAs
+            proj.set_gather_mode(mode)
+            proj.set_tile_pairs(pairs)
+            out_c = run(case, proj, dev)
+            assert proj.status() == vp.OK
+            assert torch.equal(out_a.view(torch.int16), out_c.view(torch.int16)), f"mode={mode} pairs={pairs}"

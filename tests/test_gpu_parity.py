@@ -50,9 +50,9 @@ SMALL = {
 # (gather mode, 256 x 256 tiles on CTA pairs)
 MODES = [(vp.GATHER_AUTO, True), (vp.GATHER_AUTO, False), (vp.GATHER_IM2COL, True), (vp.GATHER_IM2COL, False),
          (vp.GATHER_CPASYNC, True), (vp.GATHER_BOX, True), (vp.GATHER_BOX, False), (vp.GATHER_THREADS, True),
-         (vp.GATHER_THREADS, False)]
+         (vp.GATHER_THREADS, False), (vp.GATHER_FUSED, True), (vp.GATHER_FUSED, False), (vp.GATHER_MERGED, True)]
 MODE_IDS = ["auto-pairs", "auto-single", "im2col-pairs", "im2col-single", "cpasync", "box-pairs", "box-single",
-            "threads-pairs", "threads-single"]
+            "threads-pairs", "threads-single", "fused-pairs", "fused-single", "merged-pairs"]
 
 
 @pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
@@ -175,16 +175,17 @@ def test_box_and_im2col_agree_bit_for_bit():
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
 
 
+@pytest.mark.parametrize("mode", ["threads", "fused"])
 @pytest.mark.parametrize("name", ["dsvit", "vl2"])
-def test_thread_gather_agrees_bit_for_bit(name):
-    """The thread gather (cp.async by four extra warps, CTA pairs) fetches the same operand
-    bytes as the TMA box / im2col modes AUTO picks for these grids."""
+def test_thread_gather_and_fused_agree_bit_for_bit(name, mode):
+    """The thread gather (cp.async by four extra warps, CTA pairs) and the fused producer
+    warps fetch the same operand bytes as the TMA box / im2col modes AUTO picks."""
     wl = W.WORKLOADS[name]
     case = make_case(wl)
     proj = make_projector(case)
     dev = DeviceInputs(case)
     out_a = run(case, proj, dev)
-    proj.set_gather_mode(vp.GATHER_THREADS)
+    proj.set_gather_mode(vp.GATHER_THREADS if mode == "threads" else vp.GATHER_FUSED)
     out_b = run(case, proj, dev)
     assert proj.status() == vp.OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
@@ -218,9 +219,12 @@ def test_layernorm_paths_agree_bit_for_bit():
     out_b = run(case, proj, dev)
     proj.set_gather_mode(vp.GATHER_THREADS)
     out_c = run(case, proj, dev)
+    proj.set_gather_mode(vp.GATHER_FUSED)
+    out_d = run(case, proj, dev)
     assert proj.status() == vp.OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
     assert torch.equal(out_a.view(torch.int16), out_c.view(torch.int16))
+    assert torch.equal(out_a.view(torch.int16), out_d.view(torch.int16))
 
 
 

@@ -29,7 +29,7 @@ EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status",
             "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc", "vlproj_forward_ex",
             "vlproj_plan_tiles", "vlproj_backward", "vlproj_project_host", "vlproj_profile_stages")
 NOALLOC_MAX_IDS = 64 * 1024 * 1024
-GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX, GATHER_THREADS = 0, 1, 2, 3, 4
+GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX, GATHER_THREADS, GATHER_FUSED, GATHER_MERGED = 0, 1, 2, 3, 4, 5, 6
 NUM_STAGES = 15
 STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows",
           "bwd_index", "bwd_merge", "bwd_gemm1", "bwd_dy", "bwd_dh", "bwd_dw2", "bwd_dw1", "bwd_da", "bwd_tail")

@@ -47,6 +47,7 @@
 #include <cstdint>
 
 #include "gelu_poly.cuh"
+#include "kernels_aux.cuh"
 #include "ptx.cuh"
 
 namespace vlp {
@@ -70,6 +71,8 @@ constexpr int A_CPASYNC = 2;            // merge-gather by cp.async
 constexpr int A_BOX5 = 3;               // merge-gather by one 5D tiled TMA box (regular grids)
 constexpr int A_TGATHER = 4;            // merge-gather by 128 threads' cp.async, CTA pairs allowed
 constexpr int A_TGATHER_LN = 5;         // ... then the pre-merge LayerNorm applied in shared memory
+constexpr int A_FUSED = 6;              // A produced inside the kernel (merge + LayerNorm / convert) by
+                                        // four producer warps per CTA, read back by TMA tiles
 constexpr uint64_t DRAIN_NS = 1000000000ull;
 constexpr int ERR_TIMEOUT = -5;
 
@@ -113,7 +116,10 @@ struct GemmLayout {
 // Statistics bytes per stage in A_TGATHER_LN: (mean, rstd) of each of the 128 rows.
 __host__ __device__ constexpr int a_aux_bytes(int amode) { return amode == A_TGATHER_LN ? BM * 8 : 0; }
 __host__ __device__ constexpr bool a_thread_gather(int amode) { return amode == A_TGATHER || amode == A_TGATHER_LN; }
-__host__ __device__ constexpr int gemm_threads(int amode) { return a_thread_gather(amode) ? GEMM_THREADS_TG : GEMM_THREADS; }
+__host__ __device__ constexpr int gemm_threads(int amode) {
+    return (a_thread_gather(amode) || amode == A_FUSED) ? GEMM_THREADS_TG : GEMM_THREADS;
+}
+constexpr int FUSED_BLOCK = 256;        // A_FUSED readiness granularity: rows per block (one pair tile)
 
 struct GemmParams {
     int M;                          // rows (merged tokens, each view's run padded in im2col varlen mode)
@@ -138,6 +144,21 @@ struct GemmParams {
     int64_t stats_ld;               // a multiple of 256 rows
     const float* ln_gamma;
     const float* ln_beta;
+    // A_FUSED: the producer warps write A[m][p*C + c] (bf16, row stride K) for every merged
+    // token m < M and tap p: the patch at tap p of token m (found in the view table),
+    // LayerNorm'd when has_ln, rounded to bf16, or zeros in the high-end pad. Items are
+    // taken in (256-row block, tap, row) order from *work; ready[b * k*k + p] counts the
+    // finished items of block b, tap p (256 when done, rows past M included).
+    const ViewDesc* views;
+    int n_views;
+    const void* feat;               // features, bf16 or fp32 (feat_f32)
+    int feat_f32;
+    int has_ln;
+    float ln_eps;
+    __nv_bfloat16* a_out;
+    unsigned long long* work;       // zero at launch
+    uint32_t* ready;                // zero at launch, m_blocks * k*k counters
+    int m_blocks;
     // output
     __nv_bfloat16* out;             // GEMM1: H; GEMM2: embeddings [out_rows][N]
     const int32_t* rowdest;         // destination row of each m (-1 = no write), or null = row m
@@ -241,6 +262,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     constexpr bool kGatherThreads = kAMode == A_CPASYNC;
     constexpr bool kTG = a_thread_gather(kAMode);          // warps 8-11 fetch A by cp.async
     constexpr bool kLN = kAMode == A_TGATHER_LN;           // ... and normalise it in place
+    constexpr bool kFused = kAMode == A_FUSED;             // warps 8-11 produce A, TMA tiles read it
     static_assert(!(kPair && kGatherThreads), "the 64-thread cp.async gather runs on single CTAs");
     static_assert(!kPair || BN == 256, "CTA pairs run 256 x 256 tiles");
     extern __shared__ uint8_t smem_raw[];
@@ -281,7 +303,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmB);
-        if (kAMode == A_TILE || kAMode == A_BOX5 || (kAMode == A_IM2COL && p.gmaps == nullptr))
+        if (kAMode == A_TILE || kFused || kAMode == A_BOX5 || (kAMode == A_IM2COL && p.gmaps == nullptr))
             tma_prefetch_desc(&tmA);
         if (kAMode == A_IM2COL && p.gmaps != nullptr)
             for (int i = 0; i < p.n_gmaps; ++i) tensormap_acquire(p.gmaps + i);
@@ -330,13 +352,31 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                     for (int q = 0; q < nch; ++q) ch[q] = __ldg(&p.chunks[a_row_tile * nch + q]);
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag)) { ok = false; break; }
+                    if constexpr (kFused) {
+                        // the first K-block of a tap: wait until the producer warps (of every
+                        // CTA) have written this block's rows at that tap
+                        if (kb % cblocks == 0) {
+                            const int blk = (m_blk * kCtas * BM) / FUSED_BLOCK;
+                            const uint32_t* flag = p.ready + blk * p.k * p.k + kb / cblocks;
+                            bool got = ld_acquire_gpu(flag) >= static_cast<uint32_t>(FUSED_BLOCK);
+                            if (!got) {
+                                const uint64_t t0 = globaltimer_ns();
+                                while (!(got = ld_acquire_gpu(flag) >= static_cast<uint32_t>(FUSED_BLOCK))) {
+                                    if (*abort_flag || globaltimer_ns() - t0 > lim) break;
+                                    __nanosleep(200);
+                                }
+                            }
+                            if (!got) { ok = false; break; }
+                            fence_proxy_async_global();
+                        }
+                    }
                     uint8_t* sa = smem + stage * L::STAGE_BYTES;
                     uint8_t* sb = sa + L::A_BYTES;
                     const int b_row = n_blk * BN + static_cast<int>(rank) * L::B_ROWS;
                     if constexpr (kPair) {
                         const uint32_t bar = mapa_shared(smem_u32(&full_tma[stage]), 0);
                         if (leader) mbar_arrive_expect_tx(&full_tma[stage], expect);
-                        if (kAMode == A_TILE) {
+                        if (kAMode == A_TILE || kFused) {
                             tma_load_2d_pair(sa, &tmA, bar, kb * BK, a_row_tile * BM);
                         } else if (kAMode == A_BOX5) {
                             const int pos = kb / cblocks;
@@ -356,7 +396,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                         tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
                     } else {
                         mbar_arrive_expect_tx(&full_tma[stage], expect);
-                        if (kAMode == A_TILE) {
+                        if (kAMode == A_TILE || kFused) {
                             tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, a_row_tile * BM);
                         } else if (kAMode == A_BOX5) {
                             const int pos = kb / cblocks;
@@ -531,7 +571,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             }
             cp_async_wait_all();
         }
-    } else if (warp >= 8) {
+    } else if (kTG && warp >= 8) {
         // ------------------------------------------------ thread gather (A_TGATHER[_LN], warps 8-11)
         // Thread t copies 16-byte chunk (t & 7) of rows (t >> 3) + 16 i, i < 8, of every A
         // stage with cp.async (a zero-filled chunk where the neighbour lies in the pad or the
@@ -664,6 +704,67 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                 latch_error(p.err, ERR_TIMEOUT);
             }
             cp_async_wait_all();
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------ A producers (A_FUSED, warps 8-11)
+        // Each warp takes two items at a time from the kernel-wide counter, in (256-row
+        // block, tap, row) order, so the blocks become ready in the order the tiles need
+        // them, whichever CTAs are running. Item (b, p, r) is merged token m = 256 b + r
+        // at tap p: its patch row, LayerNorm'd (or converted), lands at A[m][p*C ...].
+        // Every lane fences its writes to the async proxy (TMA loads will read them), then
+        // lane 0 adds the items to their blocks' counters with release semantics.
+        if constexpr (kFused) {
+            const int kk = p.k * p.k;
+            const uint64_t per_block = static_cast<uint64_t>(FUSED_BLOCK) * kk;
+            const uint64_t total = static_cast<uint64_t>(p.m_blocks) * per_block;
+            const bool fast = !p.feat_f32 && p.C <= 32 * FUSED_VEC * 8;
+            const int K = p.K;
+            while (!*abort_flag) {
+                unsigned long long j0 = 0;
+                if (lane == 0) j0 = atomicAdd(p.work, 2ull);
+                j0 = __shfl_sync(0xffffffffu, j0, 0);
+                if (j0 >= total) break;
+                int64_t src[2] = {-1, -1};
+                uint4* dst[2] = {nullptr, nullptr};
+                uint32_t* cnt[2] = {nullptr, nullptr};
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const uint64_t j = j0 + t;
+                    if (j >= total) continue;
+                    const int b = static_cast<int>(j / per_block);
+                    const int rem = static_cast<int>(j - static_cast<uint64_t>(b) * per_block);
+                    const int pp = rem / FUSED_BLOCK;
+                    const int m = b * FUSED_BLOCK + (rem - pp * FUSED_BLOCK);
+                    cnt[t] = p.ready + b * kk + pp;
+                    if (m >= p.M) continue;                      // rows past M: nothing to write
+                    src[t] = merge_source_row(p.views, p.n_views, m, pp, p.k);
+                    dst[t] = reinterpret_cast<uint4*>(p.a_out + static_cast<int64_t>(m) * K + pp * p.C);
+                }
+                if (fast) {
+                    ln_rows_bf16_x2(static_cast<const __nv_bfloat16*>(p.feat), src[0], src[1], p.C, lane, p.ln_gamma,
+                                    p.ln_beta, p.ln_eps, p.has_ln, dst[0], dst[1]);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        if (dst[t] == nullptr) continue;
+                        if (src[t] < 0) {
+                            for (int v = lane; v < p.C / 8; v += 32) dst[t][v] = make_uint4(0, 0, 0, 0);
+                        } else if (p.feat_f32) {
+                            ln_row_write<true>(p.feat, src[t], p.C, lane, p.ln_gamma, p.ln_beta, p.ln_eps, p.has_ln,
+                                               dst[t]);
+                        } else {
+                            ln_row_write<false>(p.feat, src[t], p.C, lane, p.ln_gamma, p.ln_beta, p.ln_eps, p.has_ln,
+                                                dst[t]);
+                        }
+                    }
+                }
+                fence_proxy_async_global();
+                __syncwarp();
+                if (lane == 0) {
+                    if (cnt[0]) red_release_gpu_add(cnt[0], 1u);
+                    if (cnt[1]) red_release_gpu_add(cnt[1], 1u);
+                }
+            }
         }
     } else {
         // ------------------------------------------------ epilogue (warps 4..7 of each CTA)

@@ -213,6 +213,7 @@ struct Plan {
     bool im2col = true;     // GEMM1 gathers with TMA im2col (else cp.async)
     bool box5 = false;      // ... or with one 5D tiled box per K-block (regular grids)
     bool merged_ln = false; // ... or reads A written in token order by the LayerNorm pass
+    bool fused = false;     // ... or produces A inside GEMM1 (merge + LayerNorm / convert)
     bool tgather = false;   // ... or gathers A by 128 threads' cp.async (CTA pairs allowed)
     bool tgather_ln = false;// ... and applies the LayerNorm to it in shared memory
     int chunk = 128;        // im2col rows per load
@@ -264,13 +265,18 @@ inline int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int3
     }
     pl.chunk = pl.uniform ? 128 : 32;
     const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
-    if (gather_mode == VLPROJ_GATHER_AUTO && (c.has_ln || f32)) {
+    if ((gather_mode == VLPROJ_GATHER_AUTO && (c.has_ln || f32)) || gather_mode == VLPROJ_GATHER_MERGED) {
         // a LayerNorm / convert pass writes a bf16 copy anyway: write it as A itself,
         // already merged, so GEMM1 reads a plain matrix by TMA tiles (measured faster than
         // normalising inside GEMM1 behind the thread gather)
         pl.merged_ln = true;
         pl.im2col = false;
         gather_mode = VLPROJ_GATHER_CPASYNC;   // no padding, no chunk table
+    } else if (gather_mode == VLPROJ_GATHER_FUSED) {
+        // the same copy, written by GEMM1's own producer warps just ahead of its TMA loads
+        pl.fused = true;
+        pl.im2col = false;
+        gather_mode = VLPROJ_GATHER_CPASYNC;
     } else if (gather_mode == VLPROJ_GATHER_THREADS) {
         // GEMM1 gathers the raw patches itself and, with a LayerNorm on bf16 features,
         // normalises them in shared memory (only the per-patch statistics go through
@@ -280,9 +286,10 @@ inline int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int3
         pl.im2col = false;
         gather_mode = VLPROJ_GATHER_CPASYNC;
     }
-    pl.im2col = !pl.merged_ln && !pl.tgather &&
+    pl.im2col = !pl.merged_ln && !pl.tgather && !pl.fused &&
                 (gather_mode == VLPROJ_GATHER_IM2COL || (gather_mode == VLPROJ_GATHER_AUTO && pl.uniform));
-    if (pl.uniform && n_views > 0 && (gather_mode == VLPROJ_GATHER_BOX || gather_mode == VLPROJ_GATHER_AUTO)) {
+    if (pl.uniform && n_views > 0 && !pl.fused && !pl.merged_ln && !pl.tgather &&
+        (gather_mode == VLPROJ_GATHER_BOX || gather_mode == VLPROJ_GATHER_AUTO)) {
         const int h = grid_hw[0], w = grid_hw[1];
         if (h % k == 0 && w % k == 0 && w / k <= vlp::BM && vlp::BM % (w / k) == 0) {
             pl.box5 = true;
@@ -440,6 +447,7 @@ struct vlproj_handle {
     vlp_host::DevBuf<int32_t> pos, rowdest, counts;
     vlp_host::DevBuf<int2> gmeta;
     vlp_host::DevBuf<float2> lnstats;    // per (tap, GEMM row) LayerNorm statistics (A_TGATHER_LN)
+    vlp_host::DevBuf<uint32_t> fwork;    // A_FUSED: item counter (64-bit) and per (block, tap) counters
     vlp_host::DevBuf<int4> chunks;
     vlp_host::DevBuf<vlp::ViewDesc> dviews;
     vlp_host::DevBuf<vlp::ImageDesc> dimages;

@@ -474,6 +474,78 @@ static __global__ void __launch_bounds__(256) vlp_ln_stats_kernel(const void* __
     if (lane == 0) stats[item] = make_float2(mean, rstd);
 }
 
+// One warp writes the merged-operand rows of up to two items (dst0 / dst1, C bf16 each)
+// from the patch rows src0 / src1 of bf16 features x (-1: a pad position, zeros; a null
+// dst: no item): LayerNorm'd when has_ln, else copied. Both rows are loaded into registers
+// before either is computed, so two rows' loads are in flight per warp. The arithmetic is
+// the LayerNorm kernels' (same operations in the same order), so the values match theirs
+// bit for bit. For C <= 32 * FUSED_VEC * 8 channels.
+constexpr int FUSED_VEC = 5;
+__device__ __forceinline__ void ln_rows_bf16_x2(const __nv_bfloat16* __restrict__ x, int64_t src0, int64_t src1,
+                                                int C, int lane, const float* __restrict__ gamma,
+                                                const float* __restrict__ beta, float eps, int has_ln,
+                                                uint4* __restrict__ dst0, uint4* __restrict__ dst1) {
+    const int nvec = C / 8;
+    uint4 u[2][FUSED_VEC];
+    const int64_t src[2] = {src0, src1};
+    uint4* dst[2] = {dst0, dst1};
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int i = 0; i < FUSED_VEC; ++i) {
+            const int v = lane + 32 * i;
+            u[t][i] = (dst[t] != nullptr && src[t] >= 0 && v < nvec)
+                          ? __ldg(reinterpret_cast<const uint4*>(x + src[t] * C) + v)
+                          : make_uint4(0, 0, 0, 0);
+        }
+    const float inv_c = 1.0f / static_cast<float>(C);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        if (dst[t] == nullptr) continue;                        // warp-uniform
+        if (src[t] < 0 || !has_ln) {                            // pad: zeros; no LayerNorm: the bf16 row
+#pragma unroll
+            for (int i = 0; i < FUSED_VEC; ++i)
+                if (lane + 32 * i < nvec) dst[t][lane + 32 * i] = u[t][i];
+            continue;
+        }
+        uint64_t q[FUSED_VEC][4];
+#pragma unroll
+        for (int i = 0; i < FUSED_VEC; ++i) {
+            const uint32_t w[4] = {u[t][i].x, u[t][i].y, u[t][i].z, u[t][i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) q[i][e] = f2_pack(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+        }
+        uint64_t acc = 0;
+#pragma unroll
+        for (int i = 0; i < FUSED_VEC; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc = f2_add(acc, q[i][e]);
+        const float mean = ln_warp_total(acc) * inv_c;
+        const uint64_t nm = f2_splat(-mean);
+        acc = 0;
+#pragma unroll
+        for (int i = 0; i < FUSED_VEC; ++i) {
+            if (lane + 32 * i < nvec) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    q[i][e] = f2_add(q[i][e], nm);
+                    acc = f2_fma(q[i][e], q[i][e], acc);
+                }
+            }
+        }
+        const float rstd = rsqrtf(ln_warp_total(acc) * inv_c + eps);
+        const uint64_t r2 = f2_splat(rstd);
+#pragma unroll
+        for (int i = 0; i < FUSED_VEC; ++i) {
+            const int v = lane + 32 * i;
+            if (v >= nvec) continue;
+            const float4* g4 = reinterpret_cast<const float4*>(gamma) + 2 * v;
+            const float4* b4 = reinterpret_cast<const float4*>(beta) + 2 * v;
+            dst[t][v] = ln_out_pairs(q[i], r2, __ldg(g4), __ldg(g4 + 1), __ldg(b4), __ldg(b4 + 1));
+        }
+    }
+}
+
 // Pipelined form for C <= 256 * kVec. Items are dealt to warps with a stride of the
 // grid's warp count; each warp keeps up to `stages` of its next patch rows in flight in
 // a shared-memory ring of its own, fetched by 1D bulk copies that complete on one

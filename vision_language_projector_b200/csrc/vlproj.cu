@@ -35,7 +35,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     const int n_chunks = im2col ? ((M + 2 * vlp::BM - 1) / (2 * vlp::BM)) * 2 * nch_tile : 0;
     // gather metadata only for GEMM1's cp.async gather (the merged-LayerNorm pass finds its
     // source rows in the view table, the box and im2col modes need none)
-    const bool cpasync = !im2col && !pl.box5 && !pl.merged_ln;       // includes the thread gather
+    const bool cpasync = !im2col && !pl.box5 && !pl.merged_ln && !pl.fused;   // includes the thread gather
     if (h->rowdest.ensure(M)) return VLPROJ_ERR_CUDA;
     if (cpasync && h->gmeta.ensure(M)) return VLPROJ_ERR_CUDA;
     if (im2col && h->chunks.ensure(std::max(n_chunks, 1))) return VLPROJ_ERR_CUDA;
@@ -76,7 +76,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
         int rc = launch_ln_merge(h, features, dviews, static_cast<int>(pl.views.size()), M, eps, h->A.ptr, s);
         if (rc) return rc;
         stage_end(h, 2, s);
-    } else if ((c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) && !pl.tgather_ln) {
+    } else if ((c.has_ln || c.feat_dtype == VLPROJ_FEAT_F32) && !pl.tgather_ln && !pl.fused) {
         stage_begin(h, 2, s);
         ++h->launches;
         if (h->Xn.ensure(static_cast<size_t>(pl.P) * c.C)) return VLPROJ_ERR_CUDA;
@@ -117,6 +117,27 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     if (pl.merged_ln) {
         if (encode_bf16_2d(&tmA, h->A.ptr, static_cast<uint64_t>(M), static_cast<uint64_t>(h->K1), vlp::BM))
             return VLPROJ_ERR_CUDA;
+    } else if (pl.fused) {
+        // A written by GEMM1's producer warps, read back by its TMA tiles; counters zeroed
+        const int kk = c.k * c.k;
+        const int m_blocks = (M + vlp::FUSED_BLOCK - 1) / vlp::FUSED_BLOCK;
+        const size_t words = 2 + static_cast<size_t>(m_blocks) * kk;
+        if (h->A.ensure(static_cast<size_t>(M) * h->K1) || h->fwork.ensure(words)) return VLPROJ_ERR_CUDA;
+        VLP_CUDA(cudaMemsetAsync(h->fwork.ptr, 0, words * sizeof(uint32_t), s));
+        if (encode_bf16_2d(&tmA, h->A.ptr, static_cast<uint64_t>(M), static_cast<uint64_t>(h->K1), vlp::BM))
+            return VLPROJ_ERR_CUDA;
+        p.views = dviews;
+        p.n_views = static_cast<int>(pl.views.size());
+        p.feat = features;
+        p.feat_f32 = c.feat_dtype == VLPROJ_FEAT_F32 ? 1 : 0;
+        p.has_ln = c.has_ln ? 1 : 0;
+        p.ln_eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
+        p.ln_gamma = h->gamma;
+        p.ln_beta = h->beta;
+        p.a_out = h->A.ptr;
+        p.work = reinterpret_cast<unsigned long long*>(h->fwork.ptr);
+        p.ready = h->fwork.ptr + 2;
+        p.m_blocks = m_blocks;
     } else if (pl.box5) {
         const ViewDesc& V = pl.views[0];
         if (encode_box5(&tmA, src, c.C, V.h, V.w, static_cast<int>(pl.views.size()), c.k)) return VLPROJ_ERR_CUDA;
@@ -158,7 +179,10 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     stage_begin(h, 3, s);
     ++h->launches;
     int rc;
-    if (pl.tgather_ln)
+    if (pl.fused)
+        rc = launch_gemm_bn<vlp::A_FUSED, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                         h->num_sms, s, tmC);
+    else if (pl.tgather_ln)
         rc = launch_gemm_bn<vlp::A_TGATHER_LN, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
                                                               h->num_sms, s, tmC);
     else if (pl.tgather)
@@ -418,6 +442,7 @@ void vlproj_destroy(vlproj_handle* h) {
     h->counts.release();
     h->gmeta.release();
     h->lnstats.release();
+    h->fwork.release();
     h->chunks.release();
     h->dviews.release();
     h->dimages.release();
@@ -450,8 +475,7 @@ int vlproj_set_tile_pairs(vlproj_handle* h, int enable) {
 }
 
 int vlproj_set_gather_mode(vlproj_handle* h, int mode) {
-    if (!h || (mode != VLPROJ_GATHER_IM2COL && mode != VLPROJ_GATHER_CPASYNC && mode != VLPROJ_GATHER_AUTO &&
-               mode != VLPROJ_GATHER_BOX && mode != VLPROJ_GATHER_THREADS))
+    if (!h || mode < VLPROJ_GATHER_IM2COL || mode > VLPROJ_GATHER_MERGED)
         return VLPROJ_ERR_INVALID_ARG;
     h->gather_mode = mode;
     return VLPROJ_OK;
