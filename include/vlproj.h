@@ -336,6 +336,14 @@ int vlproj_set_gather_mode(vlproj_handle* h, int mode);
  * tiles on single CTAs. Both give the same bits. */
 int vlproj_set_tile_pairs(vlproj_handle* h, int enable);
 
+/* Raster of the forward GEMMs' persistent tile loop: output tiles are walked in bands
+ * of N-blocks whose slice of the weight operand B fits in `bytes` (0 = the default
+ * 64 MB, about half of the 126 MB L2); inside a band the M-block advances slowest, so
+ * the CTAs running together share their A tiles and the band's B stays in L2. A
+ * larger budget means fewer bands, so A is read from memory fewer times. The result
+ * does not depend on it (each output's K order is fixed). bytes < 0 is rejected. */
+int vlproj_set_raster_budget(vlproj_handle* h, int64_t bytes);
+
 /* Host only, no device work: the processor's tiling choices for the 2D tile scheme
  * ("port DeepSeek-VL2", Processor steps 1, 2, 6, 7). For each image of one request,
  * with original size image_wh[i] = (w0, h0) in pixels (width first):

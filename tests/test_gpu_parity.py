@@ -240,3 +240,18 @@ def test_deeper_mlp_all_rows(depth, pairs):
     out = run(case, proj, dev)
     assert proj.status() == vp.OK
     check(case, out, dev)
+
+
+@pytest.mark.parametrize("budget", [1 << 20, 256 << 20])
+def test_raster_budget_does_not_change_the_bits(budget):
+    """The raster band width (how many N-blocks share the L2 at once) only reorders the
+    output tiles; each output is accumulated over the same K order."""
+    wl = W.WORKLOADS["dsvit"]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    out_a = run(case, proj, dev)
+    proj.set_raster_budget(budget)
+    out_b = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))

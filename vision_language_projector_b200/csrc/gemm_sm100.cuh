@@ -169,7 +169,8 @@ struct GemmParams {
     // backward epilogues (outputs through tmC, and tmCt for the transposed copy)
     const __nv_bfloat16* aux;       // EPI_DGELU: G = GELU'(P) [M][N] bf16
     float* outf;                    // EPI_F32: [M][N] fp32; EPI_FOLD_F32: [patches][C] fp32
-    int group_n;                    // N-blocks per raster band (see tile_coords)
+    int group_n;                    // N-blocks per raster band (see tile_coords); 0 = from l2_budget
+    int64_t l2_budget;              // host only: bytes of B one raster band may hold (0 = 64 MB)
     int* err;                       // latched error word
     uint64_t wait_ns;               // bound on every wait
 };

@@ -348,10 +348,10 @@ inline int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int3
 // N-blocks per raster band: all of them while B fits in about half of the 126 MB L2
 // (64 MB), else the fewest bands under that budget, of equal width, so that no band is
 // a narrow remainder whose tiles share little of A.
-inline int raster_group(int N, int K, int BN) {
+inline int raster_group(int N, int K, int BN, int64_t budget = 0) {
     const int n_tiles = (N + BN - 1) / BN;
     const int64_t per_block = static_cast<int64_t>(BN) * K * 2;
-    const int64_t budget = int64_t(64) << 20;
+    if (budget <= 0) budget = int64_t(64) << 20;
     const int max_group = static_cast<int>(std::max<int64_t>(1, budget / per_block));
     if (n_tiles <= max_group) return n_tiles;
     const int bands = (n_tiles + max_group - 1) / max_group;
@@ -363,7 +363,7 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
                 const CUtensorMap& tc2, GemmParams p, int num_sms, cudaStream_t s) {
     using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E), vlp::a_aux_bytes(A)>;
     auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
-    if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN);
+    if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN, p.l2_budget);
     VLP_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC));
     const int tiles = ((p.M + vlp::BM * CTAS - 1) / (vlp::BM * CTAS)) * ((p.N + BN - 1) / BN);
     cudaLaunchConfig_t cfg{};
@@ -438,6 +438,7 @@ struct vlproj_handle {
     CUtensorMap tmW1{}, tmW2{};          // B boxes of BN rows (single-CTA tiles)
     CUtensorMap tmW1h{}, tmW2h{};        // B boxes of 128 rows (each CTA of a pair loads half)
     bool pairs = true;                   // run 256 x 256 tiles on CTA pairs where possible
+    int64_t l2_budget = 0;               // forward GEMMs: bytes of B per raster band (0 = 64 MB)
     // scratch, grown on demand
     vlp_host::DevBuf<__nv_bfloat16> H, H2, Xn, A;       // H2: second hidden buffer (depth > 2)
     // middle layers (depth > 2): weights, biases, tensor maps (BN-row and 128-row boxes)

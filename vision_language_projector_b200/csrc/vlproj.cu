@@ -111,6 +111,7 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     p.fwd_status = nullptr;
     p.err = h->status;
     p.wait_ns = h->wait_ns;
+    p.l2_budget = h->l2_budget;
 
     CUtensorMap tmA{};
     std::memset(&tmA, 0, sizeof(tmA));
@@ -468,6 +469,12 @@ int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns) {
     return VLPROJ_OK;
 }
 
+int vlproj_set_raster_budget(vlproj_handle* h, int64_t bytes) {
+    if (!h || bytes < 0) return VLPROJ_ERR_INVALID_ARG;
+    h->l2_budget = bytes;
+    return VLPROJ_OK;
+}
+
 int vlproj_set_tile_pairs(vlproj_handle* h, int enable) {
     if (!h) return VLPROJ_ERR_INVALID_ARG;
     h->pairs = enable != 0;
@@ -643,6 +650,7 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
     p.fwd_status = h->status + 1;
     p.err = h->status;
     p.wait_ns = h->wait_ns;
+    p.l2_budget = h->l2_budget;
     stage_begin(h, 4, s);
     ++h->launches;
     rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(pick_bn(c.N2), h->pairs, h->tmH, h->tmW2, h->tmW2h, p,
