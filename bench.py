@@ -39,6 +39,9 @@ METRIC = "projected image tokens/s on 1 B200; % of dense BF16 tensor peak"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "stress"         # the largest single-GPU workload (262,144 tokens, 38.5 TFLOP per step)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# SM clock of the sustained cuBLAS figure when the peaks file gives none (the pool's
+# earlier measurement settled near 1.4 PFLOP/s at about 1.3 GHz under the power cap)
+SUSTAINED_PEAK_MHZ = 1300.0
 # the sources that decide the GEMMs' DRAM traffic (kernel, its PTX, its launch and raster)
 KERNEL_SOURCES = [os.path.join("vision_language_projector_b200", "csrc", f)
                   for f in ("gemm_sm100.cuh", "gelu_poly.cuh", "ptx.cuh", "host.cuh", "kernels_aux.cuh")]
@@ -57,6 +60,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--raster-mb", type=int, default=0,
+                    help="GEMM raster band budget in MB (vlproj_set_raster_budget); 0 = the library default")
     ap.add_argument("--gather", default="auto", choices=["auto", "box", "im2col", "cpasync", "threads", "fused", "merged"],
                     help="GEMM1's merge-gather (vlproj_set_gather_mode); auto = the library's choice")
     return ap.parse_args()
@@ -321,6 +326,7 @@ def main():
     proj.set_gather_mode({"auto": vp.GATHER_AUTO, "box": vp.GATHER_BOX, "im2col": vp.GATHER_IM2COL,
                           "cpasync": vp.GATHER_CPASYNC, "threads": vp.GATHER_THREADS, "fused": vp.GATHER_FUSED,
                           "merged": vp.GATHER_MERGED}[args.gather])
+    proj.set_raster_budget(args.raster_mb << 20)
     feats = f32(feats_h) if wl.feat_fp32 else bf(feats_h)
     ids = torch.from_numpy(ids_h).cuda()
     prefill = bf(prefill_h)
@@ -449,6 +455,14 @@ def main():
         if pk_mhz:
             roof["peak_sm_mhz"] = pk_mhz
             roof["frac_clock_normalised"] = roof["frac"] * pk_mhz / mhz
+        if roof.get("bound") == "tensor":
+            # the sustained peak scaled to this run's median clock: per-clock efficiency
+            # against cuBLAS under the power cap (NVML clocks are 5 ms samples, a guide)
+            s_mhz = peak_clock_mhz(peaks, True) or SUSTAINED_PEAK_MHZ
+            s_tf = peaks.get("bf16_tflops_sustained")
+            if s_tf:
+                roof["per_clock_vs_sustained"] = roof["achieved"] / (s_tf * mhz / s_mhz)
+                roof["per_clock_reference"] = f"bf16 sustained {s_tf} TFLOP/s at {s_mhz:.0f} MHz"
 
     # ---- end to end through the public API with host buffers: vlproj_project_host takes the
     # step's features from pinned host memory and returns the assembled rows of every image to
@@ -574,7 +588,7 @@ def main():
             "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(workload_config(args, wl, M, int(sum(rows))), l2="flushed between steps (256 MiB write)",
-                           gather=args.gather,
+                           gather=args.gather, raster_mb=args.raster_mb,
                            parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
             "tflops_per_gpu": tflops,
             "pct_of_dense_bf16_peak": 100.0 * tflops / peaks.get("bf16_tflops"),

@@ -336,12 +336,15 @@ int vlproj_set_gather_mode(vlproj_handle* h, int mode);
  * tiles on single CTAs. Both give the same bits. */
 int vlproj_set_tile_pairs(vlproj_handle* h, int enable);
 
-/* Raster of the forward GEMMs' persistent tile loop: output tiles are walked in bands
- * of N-blocks whose slice of the weight operand B fits in `bytes` (0 = the default
- * 64 MB, about half of the 126 MB L2); inside a band the M-block advances slowest, so
- * the CTAs running together share their A tiles and the band's B stays in L2. A
- * larger budget means fewer bands, so A is read from memory fewer times. The result
- * does not depend on it (each output's K order is fixed). bytes < 0 is rejected. */
+/* Raster of the GEMMs' persistent tile loop (forward and backward): output tiles are
+ * walked in bands of N-blocks whose slice of the operand B fits in `bytes`; inside a band
+ * the M-block advances slowest, so the CTAs running together share their A tiles and the
+ * band's B stays in L2. A larger budget means fewer bands, so A is read from memory fewer
+ * times. 0 = the default: 64 MB (about half of the 126 MB L2), and where a single
+ * N-block's slice is larger than that (the weight gradients of big batches, K = tokens)
+ * bands of about sqrt(number of CTAs running at once) N-blocks, so a wave reads the
+ * fewest operand panels. The result does not depend on it (each output's K order is
+ * fixed). bytes < 0 is rejected. */
 int vlproj_set_raster_budget(vlproj_handle* h, int64_t bytes);
 
 /* Host only, no device work: the processor's tiling choices for the 2D tile scheme

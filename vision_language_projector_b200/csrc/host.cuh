@@ -348,10 +348,21 @@ inline int build_plan(const vlproj_config& c, const int32_t* grid_hw, const int3
 // N-blocks per raster band: all of them while B fits in about half of the 126 MB L2
 // (64 MB), else the fewest bands under that budget, of equal width, so that no band is
 // a narrow remainder whose tiles share little of A.
-inline int raster_group(int N, int K, int BN, int64_t budget = 0) {
+// When even one N-block's slice of B is larger than the default budget (the weight
+// gradients, where K is the batch's token count), no band stays in L2 and the operands
+// stream from memory in panels: then bands of about sqrt(units) N-blocks make the units
+// running together read the fewest panels (units M-blocks x N-blocks in one wave), instead
+// of one N-block against every M-block. An explicit budget keeps the plain rule.
+inline int raster_group(int N, int K, int BN, int64_t budget = 0, int units = 74) {
     const int n_tiles = (N + BN - 1) / BN;
     const int64_t per_block = static_cast<int64_t>(BN) * K * 2;
-    if (budget <= 0) budget = int64_t(64) << 20;
+    if (budget <= 0) {
+        budget = int64_t(64) << 20;
+        if (per_block > budget) {
+            const int g = static_cast<int>(std::lround(std::sqrt(static_cast<double>(std::max(units, 1)))));
+            return std::max(1, std::min(n_tiles, g));
+        }
+    }
     const int max_group = static_cast<int>(std::max<int64_t>(1, budget / per_block));
     if (n_tiles <= max_group) return n_tiles;
     const int bands = (n_tiles + max_group - 1) / max_group;
@@ -363,7 +374,7 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
                 const CUtensorMap& tc2, GemmParams p, int num_sms, cudaStream_t s) {
     using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E), vlp::a_aux_bytes(A)>;
     auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
-    if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN, p.l2_budget);
+    if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN, p.l2_budget, num_sms / CTAS);
     VLP_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC));
     const int tiles = ((p.M + vlp::BM * CTAS - 1) / (vlp::BM * CTAS)) * ((p.N + BN - 1) / BN);
     cudaLaunchConfig_t cfg{};

@@ -54,6 +54,7 @@ GemmParams gemm_params(const vlproj_handle* h, int64_t M, int N, int64_t K) {
     p.out_rows = M;
     p.err = h->status;
     p.wait_ns = h->wait_ns;
+    p.l2_budget = h->l2_budget;
     return p;
 }
 
