@@ -169,6 +169,12 @@ struct GemmParams {
     // backward epilogues (outputs through tmC, and tmCt for the transposed copy)
     const __nv_bfloat16* aux;       // EPI_DGELU: G = GELU'(P) [M][N] bf16
     float* outf;                    // EPI_F32: [M][N] fp32; EPI_FOLD_F32: [patches][C] fp32
+    // operands / transposed outputs stored blocked by 64 along K (the token axis of the
+    // weight gradients): element (row r, column m) of an R-row matrix at ((m / 64) * R + r)
+    // * 64 + m % 64, so a tile's K-block is one contiguous run (3D tensor maps: (m % 64, r,
+    // m / 64)). ct_kb64: the epilogue's transposed copy (tmCt) is stored so, with the
+    // columns from M up to the next multiple of 64 written as zeros.
+    int a_kb64, b_kb64, ct_kb64;
     int group_n;                    // N-blocks per raster band (see tile_coords); 0 = from l2_budget
     int64_t l2_budget;              // host only: bytes of B one raster band may hold (0 = 64 MB)
     int* err;                       // latched error word
@@ -378,7 +384,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                         const uint32_t bar = mapa_shared(smem_u32(&full_tma[stage]), 0);
                         if (leader) mbar_arrive_expect_tx(&full_tma[stage], expect);
                         if (kAMode == A_TILE || kFused) {
-                            tma_load_2d_pair(sa, &tmA, bar, kb * BK, a_row_tile * BM);
+                            if (p.a_kb64) tma_load_3d_pair(sa, &tmA, bar, 0, a_row_tile * BM, kb);
+                            else tma_load_2d_pair(sa, &tmA, bar, kb * BK, a_row_tile * BM);
                         } else if (kAMode == A_BOX5) {
                             const int pos = kb / cblocks;
                             const int c0 = (kb - pos * cblocks) * BK;
@@ -394,11 +401,13 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                         ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
                             }
                         }
-                        tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
+                        if (p.b_kb64) tma_load_3d_pair(sb, &tmB, bar, 0, b_row, kb);
+                        else tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
                     } else {
                         mbar_arrive_expect_tx(&full_tma[stage], expect);
                         if (kAMode == A_TILE || kFused) {
-                            tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, a_row_tile * BM);
+                            if (p.a_kb64) tma_load_3d(sa, &tmA, &full_tma[stage], 0, a_row_tile * BM, kb);
+                            else tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, a_row_tile * BM);
                         } else if (kAMode == A_BOX5) {
                             const int pos = kb / cblocks;
                             const int c0 = (kb - pos * cblocks) * BK;
@@ -414,7 +423,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                    ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
                             }
                         }
-                        tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, b_row);
+                        if (p.b_kb64) tma_load_3d(sb, &tmB, &full_tma[stage], 0, b_row, kb);
+                        else tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, b_row);
                     }
                     ++issued;
                     if (++stage == S) { stage = 0; phase ^= 1; }
@@ -841,6 +851,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                             x[j] = p0;
                             x[j + 1] = p1;
                             gelu2(x[j], x[j + 1]);
+                            if (m >= p.M) x[j] = x[j + 1] = 0.0f;   // H^T columns past M are zero
                         }
                     } else {
                         uint4 g4[4] = {};
@@ -878,10 +889,14 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0 && m_row0 < p.M) {        // a block wholly past M is not stored
-                        tma_store_2d(&tmC, ebuf, n0, m_row0);
-                        tma_store_2d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0, n0);
-                        if (with_h) tma_store_2d(&tmC2, ebuf + 2 * EPI_BLOCK_BYTES, n0, m_row0);
+                    // a block wholly past M is not stored; a blocked transposed copy is
+                    // stored up to the next multiple of 64 (its zero columns)
+                    const int m_end_t = p.ct_kb64 ? (p.M + 63) / 64 * 64 : p.M;
+                    if (lane == 0 && m_row0 < m_end_t) {
+                        if (m_row0 < p.M) tma_store_2d(&tmC, ebuf, n0, m_row0);
+                        if (p.ct_kb64) tma_store_3d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0 & 63, n0, m_row0 >> 6);
+                        else tma_store_2d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0, n0);
+                        if (with_h && m_row0 < p.M) tma_store_2d(&tmC2, ebuf + 2 * EPI_BLOCK_BYTES, n0, m_row0);
                         bulk_commit_group();
                     }
                 } else if constexpr (kEpi == EPI_SCATTER) {

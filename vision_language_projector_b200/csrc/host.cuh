@@ -92,6 +92,25 @@ inline int encode_bf16_store(CUtensorMap* map, const void* base, uint64_t rows, 
     return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
 }
 
+// Maps of a bf16 matrix of `rows` rows and `cols` (a multiple of 64) columns stored
+// blocked by 64 columns: element (r, m) at ((m / 64) * rows + r) * 64 + m % 64. Seen as
+// 3D (m % 64, r, m / 64): a load box (64, box_rows, 1) is box_rows * 128 contiguous bytes,
+// 128-byte swizzle; a store box (32, 32, 1), no swizzle.
+inline int encode_bf16_kb64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                            bool store = false) {
+    auto fn = driver().tiled;
+    if (!fn || cols % 64) return VLPROJ_ERR_CUDA;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {128, rows * 128};
+    cuuint32_t box[3] = {store ? 32u : 64u, store ? 32u : box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, store ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                    store ? CU_TENSOR_MAP_L2_PROMOTION_NONE : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
 // im2col map of n views of one (h, w) grid of C-channel bf16 patches, packed back to
 // back from `base`: the k x k, stride-k window walk of the merge. Base positions run
 // over 0, k, ..., k*(w'-1) (lower corner 0, upper corner k*w' - w - (k-1), the

@@ -26,13 +26,16 @@ constexpr int LNB_WARPS = 8;
 // reads zeros. Writes, for q < Q:
 //   dst[m * Q + q]           row-major copy (skipped when dst is null)
 //   dst_t[perm(q) * ldt + m] transposed copy (skipped when dst_t is null), where
-//                            perm(q) = c*kk + p for q = p*C + c when chan_outer, else q.
-// Rows M .. ceil(M/8)*8 - 1 of the transposed copy are written as zeros. Grid
-// (ceil(Q/64), ceil(M/64)), 256 threads. Q, ld_src and ldt are multiples of 8.
+//                            perm(q) = c*kk + p for q = p*C + c when chan_outer, else q;
+//                            with kb64 stored blocked by 64 columns instead:
+//                            dst_t[((m / 64) * Q + perm(q)) * 64 + m % 64]
+// Columns M .. ceil(M/8)*8 - 1 of the transposed copy (.. ceil(M/64)*64 - 1 with kb64)
+// are written as zeros. Grid (ceil(Q/64), ceil(M/64)), 256 threads. Q, ld_src and ldt
+// are multiples of 8 (ldt of 64 with kb64).
 static __global__ void __launch_bounds__(256) vlp_gather_transpose_kernel(
     const __nv_bfloat16* __restrict__ src, int64_t ld_src, int64_t src_rows, const int32_t* __restrict__ rowsel,
     const int* __restrict__ zero_if, int M, int Q, __nv_bfloat16* __restrict__ dst, __nv_bfloat16* __restrict__ dst_t,
-    int64_t ldt, int C, int kk, int chan_outer) {
+    int64_t ldt, int C, int kk, int chan_outer, int kb64) {
     __shared__ __align__(16) __nv_bfloat16 tile[TR_TILE][TR_TILE + 8];
     const int q0 = blockIdx.x * TR_TILE;
     const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TR_TILE;
@@ -67,7 +70,7 @@ static __global__ void __launch_bounds__(256) vlp_gather_transpose_kernel(
     for (int h = 0; h < 2; ++h) {
         const int r0 = 16 * mh + 8 * h;
         const int64_t m = m0 + r0;
-        if (m >= M) break;
+        if (m >= M && !kb64) break;        // blocked: the tile's zero tail is written too
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -75,21 +78,23 @@ static __global__ void __launch_bounds__(256) vlp_gather_transpose_kernel(
             const uint32_t hi = __bfloat16_as_ushort(tile[r0 + 2 * e + 1][qq]);
             w[e] = lo | (hi << 16);
         }
-        *reinterpret_cast<uint4*>(dst_t + orow * ldt + m) = make_uint4(w[0], w[1], w[2], w[3]);
+        const int64_t off = kb64 ? ((m >> 6) * Q + orow) * 64 + (m & 63) : orow * ldt + m;
+        *reinterpret_cast<uint4*>(dst_t + off) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
-// out[n] = sum over m < M of T[n * ld + m] (bf16), accumulated in fp32: one warp per
-// row, each lane over every 32nd run of 8 elements, then a butterfly. ld % 8 == 0.
+// out[n] = sum over m < M of T(n, m) (bf16), accumulated in fp32: one warp per row, each
+// lane over every 32nd run of 8 elements, then a butterfly. T(n, m) = T[n * ld + m], or
+// with kb64 T[((m / 64) * N + n) * 64 + m % 64] (blocked by 64 columns). ld % 8 == 0.
 static __global__ void __launch_bounds__(256) vlp_rowsum_kernel(const __nv_bfloat16* __restrict__ T, int64_t ld, int N,
-                                                         int64_t M, float* __restrict__ out) {
+                                                         int64_t M, float* __restrict__ out, int kb64) {
     const int lane = threadIdx.x & 31;
     const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (n >= N) return;
-    const __nv_bfloat16* row = T + static_cast<int64_t>(n) * ld;
     float s = 0.f;
     for (int64_t m = 8 * lane; m < M; m += 256) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + m));
+        const int64_t off = kb64 ? ((m >> 6) * N + n) * 64 + (m & 63) : static_cast<int64_t>(n) * ld + m;
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(T + off));
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {

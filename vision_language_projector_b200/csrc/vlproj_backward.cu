@@ -44,6 +44,13 @@ int encode_b(CUtensorMap* full, CUtensorMap* half, const void* base, uint64_t ro
     return encode_bf16_2d(half, base, rows, cols, 128, ld);
 }
 
+// The same for a B operand stored blocked by 64 columns (the transposed activations and
+// gradients, K = tokens): each K-block of the box's rows is one contiguous run.
+int encode_b_kb64(CUtensorMap* full, CUtensorMap* half, const void* base, uint64_t rows, uint64_t cols, int bn) {
+    if (encode_bf16_kb64(full, base, rows, cols, static_cast<uint32_t>(bn))) return VLPROJ_ERR_CUDA;
+    return encode_bf16_kb64(half, base, rows, cols, 128);
+}
+
 GemmParams gemm_params(const vlproj_handle* h, int64_t M, int N, int64_t K) {
     GemmParams p{};
     p.M = static_cast<int>(M);
@@ -60,11 +67,12 @@ GemmParams gemm_params(const vlproj_handle* h, int64_t M, int N, int64_t K) {
 
 void transpose_launch(const __nv_bfloat16* src, int64_t ld_src, int64_t src_rows, const int32_t* rowsel,
                       const int* zero_if, int64_t M, int Q, __nv_bfloat16* dst, __nv_bfloat16* dst_t, int64_t ldt,
-                      int C, int kk, int chan_outer, cudaStream_t s) {
+                      int C, int kk, int chan_outer, cudaStream_t s, int kb64 = 0) {
     dim3 grid(static_cast<unsigned>((Q + vlp::TR_TILE - 1) / vlp::TR_TILE),
               static_cast<unsigned>((M + vlp::TR_TILE - 1) / vlp::TR_TILE));
     vlp::vlp_gather_transpose_kernel<<<grid, 256, 0, s>>>(src, ld_src, src_rows, rowsel, zero_if,
-                                                          static_cast<int>(M), Q, dst, dst_t, ldt, C, kk, chan_outer);
+                                                          static_cast<int>(M), Q, dst, dst_t, ldt, C, kk, chan_outer,
+                                                          kb64);
 }
 
 // W2^T [N1][N2], W1p^T [K1][N1] and each middle layer's W^T [N1][N1], with their tensor
@@ -228,8 +236,9 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             p.bias = first ? h->b1 : h->bm[l - 2];
             CUtensorMap tmG{}, tmHt{}, tmHr{};
             if (encode_bf16_store(&tmG, G + (l - 1) * hslab, M, c.N1) ||
-                encode_bf16_store(&tmHt, Ht + (l - 1) * tslab, c.N1, M, ldt))
+                encode_bf16_kb64(&tmHt, Ht + (l - 1) * tslab, c.N1, ldt, 0, true))
                 return VLPROJ_ERR_CUDA;
+            p.ct_kb64 = 1;
             if (l < depth - 1) {
                 p.store_h = 1;
                 if (encode_bf16_store(&tmHr, h->Hr.ptr + (l - 1) * hslab, M, c.N1)) return VLPROJ_ERR_CUDA;
@@ -248,7 +257,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     stage_begin(h, 9, s);
     ++h->launches;
     transpose_launch(static_cast<const __nv_bfloat16*>(a->d_out), c.N2, n_ids, h->rowdest.ptr, h->status + 1, M,
-                     c.N2, h->dY.ptr, h->dYt.ptr, ldt, c.C, 1, 0, s);
+                     c.N2, h->dY.ptr, h->dYt.ptr, ldt, c.C, 1, 0, s, 1);
     VLP_CUDA(cudaGetLastError());
     stage_end(h, 9, s);
 
@@ -267,10 +276,11 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     // 11. top layer: dW2 = dY^T H_(depth-1) and db2 (side stream)
     CUtensorMap tmA2{}, tmB2{}, tmB2h{};
     if (a->d_W2) {
-        if (encode_bf16_2d(&tmA2, h->dYt.ptr, c.N2, M, vlp::BM, ldt) ||
-            encode_b(&tmB2, &tmB2h, Ht + (depth - 2) * tslab, c.N1, M, pick_bn(c.N1), ldt))
+        if (encode_bf16_kb64(&tmA2, h->dYt.ptr, c.N2, ldt, vlp::BM) ||
+            encode_b_kb64(&tmB2, &tmB2h, Ht + (depth - 2) * tslab, c.N1, ldt, pick_bn(c.N1)))
             return VLPROJ_ERR_CUDA;
         GemmParams q = gemm_params(h, c.N2, c.N1, M);
+        q.a_kb64 = q.b_kb64 = 1;
         q.outf = a->d_W2;
         stage_begin(h, 11, ss);
         ++h->launches;
@@ -281,7 +291,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     }
     if (a->d_b2) {
         ++h->launches;
-        vlp::vlp_rowsum_kernel<<<(c.N2 + 7) / 8, 256, 0, ss>>>(h->dYt.ptr, ldt, c.N2, M, a->d_b2);
+        vlp::vlp_rowsum_kernel<<<(c.N2 + 7) / 8, 256, 0, ss>>>(h->dYt.ptr, ldt, c.N2, M, a->d_b2, 1);
         VLP_CUDA(cudaGetLastError());
     }
 
@@ -301,8 +311,9 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             p.aux = G + (l - 1) * hslab;
             CUtensorMap tmP{}, tmPt{};
             if (encode_bf16_store(&tmP, h->dP.ptr + nxt * hslab, M, c.N1) ||
-                encode_bf16_store(&tmPt, h->dPt.ptr + nxt * tslab, c.N1, M, ldt))
+                encode_bf16_kb64(&tmPt, h->dPt.ptr + nxt * tslab, c.N1, ldt, 0, true))
                 return VLPROJ_ERR_CUDA;
+            p.ct_kb64 = 1;
             ++h->launches;
             rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(pick_bn(c.N1), h->pairs, tmA,
                                                              top ? h->tmW2t : h->tmWmt[l - 1],
@@ -315,10 +326,11 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             const int i = l - 2;
             if (mid_w(i)) {
                 CUtensorMap ta{}, tb{}, tbh{};
-                if (encode_bf16_2d(&ta, h->dPt.ptr + cur * tslab, c.N1, M, vlp::BM, ldt) ||
-                    encode_b(&tb, &tbh, Ht + (l - 2) * tslab, c.N1, M, pick_bn(c.N1), ldt))
+                if (encode_bf16_kb64(&ta, h->dPt.ptr + cur * tslab, c.N1, ldt, vlp::BM) ||
+                    encode_b_kb64(&tb, &tbh, Ht + (l - 2) * tslab, c.N1, ldt, pick_bn(c.N1)))
                     return VLPROJ_ERR_CUDA;
                 GemmParams q = gemm_params(h, c.N1, c.N1, M);
+                q.a_kb64 = q.b_kb64 = 1;
                 q.outf = mid_w(i);
                 ++h->launches;
                 rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(c.N1), h->pairs, ta, tb, tbh, q, h->num_sms,
@@ -328,7 +340,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             if (mid_b(i)) {
                 ++h->launches;
                 vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, s>>>(h->dPt.ptr + cur * tslab, ldt, c.N1, M,
-                                                                      mid_b(i));
+                                                                      mid_b(i), 1);
                 VLP_CUDA(cudaGetLastError());
             }
         }
@@ -344,17 +356,18 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         stage_begin(h, 12, ss);
         ++h->launches;
         transpose_launch(h->A.ptr, K1, M, nullptr, nullptr, M, K1, nullptr, h->At.ptr, ldt, c.C, kk,
-                         c.k_order == VLPROJ_ORDER_CHANNEL_OUTER ? 1 : 0, ss);
+                         c.k_order == VLPROJ_ORDER_CHANNEL_OUTER ? 1 : 0, ss, 1);
         VLP_CUDA(cudaGetLastError());
     }
 
     // 12b. dW1 = dP_1^T A and db1 (side stream, after dP_1)
     if (want_l1) VLP_CUDA(cudaStreamWaitEvent(ss, h->join2, 0));
     if (a->d_W1) {
-        if (encode_bf16_2d(&tmA2, dP1t, c.N1, M, vlp::BM, ldt) ||
-            encode_b(&tmB2, &tmB2h, h->At.ptr, K1, M, pick_bn(K1), ldt))
+        if (encode_bf16_kb64(&tmA2, dP1t, c.N1, ldt, vlp::BM) ||
+            encode_b_kb64(&tmB2, &tmB2h, h->At.ptr, K1, ldt, pick_bn(K1)))
             return VLPROJ_ERR_CUDA;
         GemmParams q = gemm_params(h, c.N1, K1, M);
+        q.a_kb64 = q.b_kb64 = 1;
         q.outf = a->d_W1;
         ++h->launches;
         rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(K1), h->pairs, tmA2, tmB2, tmB2h, q, h->num_sms,
@@ -364,7 +377,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     }
     if (a->d_b1) {
         ++h->launches;
-        vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, ss>>>(dP1t, ldt, c.N1, M, a->d_b1);
+        vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, ss>>>(dP1t, ldt, c.N1, M, a->d_b1, 1);
         VLP_CUDA(cudaGetLastError());
     }
     VLP_CUDA(cudaEventRecord(h->join, ss));
