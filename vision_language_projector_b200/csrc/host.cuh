@@ -490,7 +490,6 @@ struct vlproj_handle {
     // the placeholder index runs on `side`, forked from / joined to the caller's stream
     cudaStream_t side = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr;
-    cudaEvent_t ev_dy = nullptr;         // backward: dY / dY^T done on the side stream
     // tracing: start / end event of every stage, recorded on the stream that runs it
     bool profiling = false;
     uint32_t profile_mask = ~0u;         // stages that record events while profiling

@@ -458,7 +458,6 @@ void vlproj_destroy(vlproj_handle* h) {
     if (h->fork) cudaEventDestroy(h->fork);
     if (h->join) cudaEventDestroy(h->join);
     if (h->join2) cudaEventDestroy(h->join2);
-    if (h->ev_dy) cudaEventDestroy(h->ev_dy);
     if (h->side) cudaStreamDestroy(h->side);
     cudaSetDevice(cur);
     delete h;

@@ -211,29 +211,6 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     VLP_CUDA(cudaGetLastError());
     stage_end(h, 6, s);
 
-    // 9. dY and dY^T from the placeholder rows of d_out. It needs only the index, so for
-    //    batches whose weight gradients overlap the dP chain (below) it runs on the side
-    //    stream beside stages 7-8, joined back before the first GEMM that reads it.
-    const bool overlap = M * c.N1 <= (int64_t(1) << 28);
-    if (overlap && !h->ev_dy) VLP_CUDA(cudaEventCreateWithFlags(&h->ev_dy, cudaEventDisableTiming));
-    cudaStream_t sdy = overlap ? h->side : s;
-    if (overlap) {
-        VLP_CUDA(cudaEventRecord(h->fork, s));
-        VLP_CUDA(cudaStreamWaitEvent(sdy, h->fork, 0));
-    }
-    stage_begin(h, 9, sdy);
-    ++h->launches;
-    transpose_launch(static_cast<const __nv_bfloat16*>(a->d_out), c.N2, n_ids, h->rowdest.ptr, h->status + 1, M,
-                     c.N2, h->dY.ptr, h->dYt.ptr, ldt, c.C, 1, 0, sdy, 1);
-    VLP_CUDA(cudaGetLastError());
-    stage_end(h, 9, sdy);
-    if (overlap) VLP_CUDA(cudaEventRecord(h->ev_dy, sdy));
-    // an error before the join still orders the caller's stream after the dY gather
-    auto fail_dy = [&](int code) {
-        if (overlap) cudaStreamWaitEvent(s, h->ev_dy, 0);
-        return code;
-    };
-
     const float eps = c.ln_eps > 0.f ? c.ln_eps : 1e-5f;
     CUtensorMap tmA{};
     GemmParams p{};
@@ -244,7 +221,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         ++h->launches;
         rc = launch_ln_merge(h, a->features, h->dviews.ptr, static_cast<int>(pl.views.size()), static_cast<int>(M), eps,
                              h->A.ptr, s);
-        if (rc) return fail_dy(rc);
+        if (rc) return rc;
         stage_end(h, 7, s);
 
         // 8. every hidden layer recomputed: G_l = GELU'(P_l), H_l^T, and H_l itself when a
@@ -254,29 +231,35 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             const bool first = l == 1;
             const __nv_bfloat16* x = first ? h->A.ptr : h->Hr.ptr + (l - 2) * hslab;
             const int K = first ? K1 : c.N1;
-            if (encode_bf16_2d(&tmA, x, M, K, vlp::BM)) return fail_dy(VLPROJ_ERR_CUDA);
+            if (encode_bf16_2d(&tmA, x, M, K, vlp::BM)) return VLPROJ_ERR_CUDA;
             p = gemm_params(h, M, c.N1, K);
             p.bias = first ? h->b1 : h->bm[l - 2];
             CUtensorMap tmG{}, tmHt{}, tmHr{};
             if (encode_bf16_store(&tmG, G + (l - 1) * hslab, M, c.N1) ||
                 encode_bf16_kb64(&tmHt, Ht + (l - 1) * tslab, c.N1, ldt, 0, true))
-                return fail_dy(VLPROJ_ERR_CUDA);
+                return VLPROJ_ERR_CUDA;
             p.ct_kb64 = 1;
             if (l < depth - 1) {
                 p.store_h = 1;
-                if (encode_bf16_store(&tmHr, h->Hr.ptr + (l - 1) * hslab, M, c.N1)) return fail_dy(VLPROJ_ERR_CUDA);
+                if (encode_bf16_store(&tmHr, h->Hr.ptr + (l - 1) * hslab, M, c.N1)) return VLPROJ_ERR_CUDA;
             }
             ++h->launches;
             rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(pick_bn(c.N1), h->pairs, tmA,
                                                              first ? h->tmW1 : h->tmWm[l - 2],
                                                              first ? h->tmW1h : h->tmWmh[l - 2], p, h->num_sms, s,
                                                              tmG, tmHt, tmHr);
-            if (rc) return fail_dy(rc);
+            if (rc) return rc;
         }
         stage_end(h, 8, s);
     }
 
-    if (overlap) VLP_CUDA(cudaStreamWaitEvent(s, h->ev_dy, 0));
+    // 9. dY and dY^T from the placeholder rows of d_out
+    stage_begin(h, 9, s);
+    ++h->launches;
+    transpose_launch(static_cast<const __nv_bfloat16*>(a->d_out), c.N2, n_ids, h->rowdest.ptr, h->status + 1, M,
+                     c.N2, h->dY.ptr, h->dYt.ptr, ldt, c.C, 1, 0, s, 1);
+    VLP_CUDA(cudaGetLastError());
+    stage_end(h, 9, s);
 
     // Up to about 2^28 hidden activations (M * N1) the top and first layers' weight
     // gradients run on the side stream, beside the dP chain on the caller's stream: the
@@ -285,6 +268,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     // 1.4-2 % faster on the MoonViT, DeepSeek-ViT and VL2 batches). Larger batches run in
     // sequence: there the two GEMM streams contend for L2 and power (measured 8 % slower
     // on 262,144 tokens).
+    const bool overlap = M * c.N1 <= (int64_t(1) << 28);
     cudaStream_t ss = overlap ? h->side : s;
     VLP_CUDA(cudaEventRecord(h->fork, s));
     VLP_CUDA(cudaStreamWaitEvent(ss, h->fork, 0));
