@@ -175,7 +175,6 @@ struct GemmParams {
     // m / 64)). ct_kb64: the epilogue's transposed copy (tmCt) is stored so, with the
     // columns from M up to the next multiple of 64 written as zeros.
     int a_kb64, b_kb64, ct_kb64;
-    int b_evict_last;               // B loads carry an L2 evict-last policy (its raster band fits in L2)
     int group_n;                    // N-blocks per raster band (see tile_coords); 0 = from l2_budget
     int64_t l2_budget;              // host only: bytes of B one raster band may hold (0 = 64 MB)
     int* err;                       // latched error word
@@ -351,10 +350,6 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             bool ok = true;
             const int nch = (kAMode == A_IM2COL) ? BM / p.chunk : 0;
             const uint32_t expect = (kAMode == A_CPASYNC || kTG ? 0 : L::A_BYTES * kCtas) + L::B_BYTES * kCtas;
-            // the B band is read again by the next waves of tiles: keep it in L2 ahead of the
-            // A tiles streaming through
-            const uint64_t pol_b = l2_policy_evict_last();
-            const bool hint_b = p.b_evict_last != 0;
             for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
                 int m_blk, n_blk;
                 tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
@@ -406,14 +401,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                         ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
                             }
                         }
-                        if (p.b_kb64) {
-                            if (hint_b) tma_load_3d_pair_hint(sb, &tmB, bar, 0, b_row, kb, pol_b);
-                            else tma_load_3d_pair(sb, &tmB, bar, 0, b_row, kb);
-                        } else if (hint_b) {
-                            tma_load_2d_pair_hint(sb, &tmB, bar, kb * BK, b_row, pol_b);
-                        } else {
-                            tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
-                        }
+                        if (p.b_kb64) tma_load_3d_pair(sb, &tmB, bar, 0, b_row, kb);
+                        else tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
                     } else {
                         mbar_arrive_expect_tx(&full_tma[stage], expect);
                         if (kAMode == A_TILE || kFused) {
@@ -434,14 +423,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                    ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
                             }
                         }
-                        if (p.b_kb64) {
-                            if (hint_b) tma_load_3d_hint(sb, &tmB, &full_tma[stage], 0, b_row, kb, pol_b);
-                            else tma_load_3d(sb, &tmB, &full_tma[stage], 0, b_row, kb);
-                        } else if (hint_b) {
-                            tma_load_2d_hint(sb, &tmB, &full_tma[stage], kb * BK, b_row, pol_b);
-                        } else {
-                            tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, b_row);
-                        }
+                        if (p.b_kb64) tma_load_3d(sb, &tmB, &full_tma[stage], 0, b_row, kb);
+                        else tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, b_row);
                     }
                     ++issued;
                     if (++stage == S) { stage = 0; phase ^= 1; }

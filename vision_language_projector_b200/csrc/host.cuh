@@ -394,13 +394,6 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
     using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E), vlp::a_aux_bytes(A)>;
     auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
     if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN, p.l2_budget, num_sms / CTAS);
-    {
-        // the B band is meant to stay in L2 across waves when it fits the budget: mark its
-        // loads evict-last (not when whole operand panels stream, the weight gradients)
-        const int64_t budget = p.l2_budget > 0 ? p.l2_budget : (int64_t(64) << 20);
-        const int64_t band = static_cast<int64_t>(BN) * p.K * 2 * p.group_n;
-        p.b_evict_last = band <= budget ? 1 : 0;
-    }
     VLP_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC));
     const int tiles = ((p.M + vlp::BM * CTAS - 1) / (vlp::BM * CTAS)) * ((p.N + BN - 1) / BN);
     cudaLaunchConfig_t cfg{};
