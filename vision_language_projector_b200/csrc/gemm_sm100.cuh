@@ -74,6 +74,10 @@ constexpr int A_TGATHER_LN = 5;         // ... then the pre-merge LayerNorm appl
 constexpr int A_FUSED = 6;              // A produced inside the kernel (merge + LayerNorm / convert) by
                                         // four producer warps per CTA, read back by TMA tiles
 constexpr uint64_t DRAIN_NS = 1000000000ull;
+// Naps between the tests of a wait (ns): the epilogue waits a whole tile for its
+// accumulator, the gather warps about one stage for a free slot or landed copies.
+constexpr uint32_t EPI_NAP_NS = 256;
+constexpr uint32_t GATHER_NAP_NS = 64;
 constexpr int ERR_TIMEOUT = -5;
 
 // Shared-memory plan. kCtas = 2 runs one 256-row tile on a CTA pair: each CTA holds
@@ -514,7 +518,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             const uint32_t gat_leader = kPair ? mapa_shared(smem_u32(&full_gat[0]), 0) : 0u;
             for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait_bounded(&full_loc[stage], phase, lim, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait_bounded(&full_loc[stage], phase, lim, abort_flag, GATHER_NAP_NS)) { ok = false; break; }
                     fence_proxy_async_smem();
                     if constexpr (kPair) mbar_arrive_cluster(gat_leader + 8u * static_cast<uint32_t>(stage));
                     else mbar_arrive(&full_gat[stage]);
@@ -559,7 +563,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                     // one lane per warp waits, the warp follows it
                     int got = 0;
                     if ((threadIdx.x & 31) == 0)
-                        got = mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag) ? 1 : 0;
+                        got = mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag, GATHER_NAP_NS) ? 1 : 0;
                     got = __shfl_sync(0xffffffffu, got, 0);
                     if (!got) { ok = false; break; }
                     const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
@@ -606,7 +610,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             bool ok = true;
             // normalise the oldest issued stage in place and hand it to the MMA
             auto transform_one = [&]() -> bool {
-                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_loc[tstage], tphase, lim, abort_flag)))
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_loc[tstage], tphase, lim, abort_flag, GATHER_NAP_NS)))
                     return false;
                 uint8_t* sa = smem + tstage * L::STAGE_BYTES;
                 const float2* st = reinterpret_cast<const float2*>(smem + L::AUX_OFFSET + tstage * L::AUX_BYTES_PER);
@@ -675,7 +679,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                     const int c0 = (kb - pos * cblocks) * BK + chunk * 8;
                     const int dy = pos / p.k, dx = pos - dy * p.k;
                     int got = 0;
-                    if (lane == 0) got = mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag) ? 1 : 0;
+                    if (lane == 0)
+                        got = mbar_wait_bounded(&empty[stage], phase ^ 1, lim, abort_flag, GATHER_NAP_NS) ? 1 : 0;
                     got = __shfl_sync(0xffffffffu, got, 0);
                     if (!got) { ok = false; break; }
                     const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
@@ -791,7 +796,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
             // one lane waits, the warp follows it, so tcgen05.ld below is never divergent
             int got = 0;
-            if (lane == 0) got = mbar_wait_bounded(&tmem_full[acc], acc_phase, lim, abort_flag) ? 1 : 0;
+            if (lane == 0) got = mbar_wait_bounded(&tmem_full[acc], acc_phase, lim, abort_flag, EPI_NAP_NS) ? 1 : 0;
             got = __shfl_sync(0xffffffffu, got, 0);
             if (!got) { ok = false; break; }
             tc_fence_after();

@@ -52,16 +52,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
 
 // Wait for the phase with the given parity to complete, for at most limit_ns.
 // Returns false when the bound ran out or another role has already raised
-// `abort_flag` (then the caller unwinds).
+// `abort_flag` (then the caller unwinds). The abort flag and the clock are checked on
+// every 16th failed test only, and a waiter that is not on the critical path (sleep_ns >
+// 0) naps between tests: a spinning thread takes issue slots from the warps that share
+// its scheduler (the TMA producer, the MMA issuer, the epilogue).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                                  volatile int* abort_flag) {
+                                                  volatile int* abort_flag, uint32_t sleep_ns = 0) {
     const uint32_t hint = limit_ns < 20000 ? static_cast<uint32_t>(limit_ns) : 20000u;
     if (mbar_try_wait(bar, parity, hint)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (true) {
+    for (uint32_t it = 1;; ++it) {
+        if (sleep_ns) __nanosleep(sleep_ns);
         if (mbar_try_wait(bar, parity, hint)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+        if ((it & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > limit_ns) return false;
+        }
     }
 }
 
