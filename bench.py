@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--raster-mb", type=int, default=0,
                     help="GEMM raster band budget in MB (vlproj_set_raster_budget); 0 = the library default")
+    ap.add_argument("--tile-order", choices=("dynamic", "static"), default="dynamic",
+                    help="GEMM tile order (vlproj_set_tile_order): from a counter (default) or fixed per CTA")
     ap.add_argument("--gather", default="auto", choices=["auto", "box", "im2col", "cpasync", "threads", "fused", "merged"],
                     help="GEMM1's merge-gather (vlproj_set_gather_mode); auto = the library's choice")
     return ap.parse_args()
@@ -327,6 +329,7 @@ def main():
                           "cpasync": vp.GATHER_CPASYNC, "threads": vp.GATHER_THREADS, "fused": vp.GATHER_FUSED,
                           "merged": vp.GATHER_MERGED}[args.gather])
     proj.set_raster_budget(args.raster_mb << 20)
+    proj.set_tile_order(args.tile_order == "dynamic")
     feats = f32(feats_h) if wl.feat_fp32 else bf(feats_h)
     ids = torch.from_numpy(ids_h).cuda()
     prefill = bf(prefill_h)
@@ -588,7 +591,7 @@ def main():
             "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(workload_config(args, wl, M, int(sum(rows))), l2="flushed between steps (256 MiB write)",
-                           gather=args.gather, raster_mb=args.raster_mb,
+                           gather=args.gather, raster_mb=args.raster_mb, tile_order=args.tile_order,
                            parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
             "tflops_per_gpu": tflops,
             "pct_of_dense_bf16_peak": 100.0 * tflops / peaks.get("bf16_tflops"),

@@ -242,6 +242,26 @@ def test_deeper_mlp_all_rows(depth, pairs):
     check(case, out, dev)
 
 
+@pytest.mark.parametrize("workload", ["dsvit", "vl2"])
+def test_tile_order_does_not_change_the_bits(workload):
+    """The dynamic tile order (units take the next tile from a counter) and the static
+    one run the same tiles with the same K order. Forty more forwards on the handle take
+    its 64 tile queues round more than once: each GEMM must leave its queue at zero."""
+    wl = W.WORKLOADS[workload]
+    case = make_case(wl)
+    proj = make_projector(case)
+    dev = DeviceInputs(case)
+    out_dyn = run(case, proj, dev)
+    proj.set_tile_order(False)
+    out_static = run(case, proj, dev)
+    proj.set_tile_order(True)
+    for _ in range(40):
+        out_again = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    assert torch.equal(out_dyn.view(torch.int16), out_static.view(torch.int16))
+    assert torch.equal(out_dyn.view(torch.int16), out_again.view(torch.int16))
+
+
 @pytest.mark.parametrize("budget", [1 << 20, 256 << 20])
 def test_raster_budget_does_not_change_the_bits(budget):
     """The raster band width (how many N-blocks share the L2 at once) only reorders the

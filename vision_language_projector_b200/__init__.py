@@ -28,7 +28,7 @@ EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status",
             "vlproj_profile_enable", "vlproj_profile_read", "vlproj_launch_count", "vlproj_set_gather_mode",
             "vlproj_set_tile_pairs", "vlproj_placeholder_index_noalloc", "vlproj_forward_ex",
             "vlproj_plan_tiles", "vlproj_backward", "vlproj_project_host", "vlproj_profile_stages",
-            "vlproj_set_raster_budget")
+            "vlproj_set_raster_budget", "vlproj_set_tile_order")
 NOALLOC_MAX_IDS = 64 * 1024 * 1024
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX, GATHER_THREADS, GATHER_FUSED, GATHER_MERGED = 0, 1, 2, 3, 4, 5, 6
 NUM_STAGES = 15
@@ -124,6 +124,8 @@ def _load() -> ctypes.CDLL:
     lib.vlproj_set_tile_pairs.restype = ctypes.c_int
     lib.vlproj_set_raster_budget.argtypes = [P, I64]
     lib.vlproj_set_raster_budget.restype = ctypes.c_int
+    lib.vlproj_set_tile_order.argtypes = [P, I32]
+    lib.vlproj_set_tile_order.restype = ctypes.c_int
     lib.vlproj_plan_tiles.argtypes = [P, I32, P, I32, I32, I32, I32, P, P]
     lib.vlproj_plan_tiles.restype = I64
     lib.vlproj_forward_ex.argtypes = [P, ctypes.POINTER(ForwardArgs), P]
@@ -509,6 +511,11 @@ class Projector:
         rc = _lib.vlproj_set_raster_budget(self._h, int(nbytes))
         if rc != OK:
             raise VlprojError(rc, "vlproj_set_raster_budget")
+
+    def set_tile_order(self, dynamic: bool) -> None:
+        rc = _lib.vlproj_set_tile_order(self._h, 1 if dynamic else 0)
+        if rc != OK:
+            raise VlprojError(rc, "vlproj_set_tile_order")
 
     def set_wait_limit(self, ns: int) -> None:
         rc = _lib.vlproj_set_wait_limit(self._h, int(ns))

@@ -93,6 +93,10 @@ __host__ __device__ constexpr int epi_blocks(int epi) {
 }
 __host__ __device__ constexpr int epi_stage_bytes(int epi) { return 4 * epi_blocks(epi) * EPI_BLOCK_BYTES; }
 
+// Slots of the ring that hands tile indices from the TMA producer to the other roles
+// (dynamic tile order).
+constexpr int SCHED_SLOTS = 8;
+
 // kAuxBytes: bytes per stage beside the operands (the LayerNorm statistics of the stage's
 // 128 rows in A_TGATHER_LN), kept after the ring; such layouts size the ring from the whole
 // 227 KB a CTA may use.
@@ -109,10 +113,12 @@ struct GemmLayout {
     static constexpr int AUX_BYTES_PER = kAuxBytes;
     static constexpr int EPI_OFFSET = AUX_OFFSET + STAGES * kAuxBytes;
     static constexpr int BAR_OFFSET = EPI_OFFSET + kEpiBytes;
-    // full_tma[S], full_gather[S], empty[S], full_local[S], tmem_full[2], tmem_empty[2], drain
-    static constexpr int NUM_BARS = 4 * STAGES + 5;
+    // full_tma[S], full_gather[S], empty[S], full_local[S], tmem_full[2], tmem_empty[2], drain,
+    // sched_full[SCHED_SLOTS], sched_empty[SCHED_SLOTS]
+    static constexpr int NUM_BARS = 4 * STAGES + 5 + 2 * SCHED_SLOTS;
     static constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
-    static constexpr int BYTES = MISC_OFFSET + 16;
+    static constexpr int RING_OFFSET = MISC_OFFSET + 16;          // tile indices of the dynamic order
+    static constexpr int BYTES = RING_OFFSET + 4 * SCHED_SLOTS;
     static constexpr int SMEM_ALLOC = BYTES + 1024;      // room to align the base to 1024 B
     static constexpr uint32_t TMEM_COLS = 2 * BN;        // two accumulators
 };
@@ -181,11 +187,101 @@ struct GemmParams {
     int a_kb64, b_kb64, ct_kb64;
     int group_n;                    // N-blocks per raster band (see tile_coords); 0 = from l2_budget
     int64_t l2_budget;              // host only: bytes of B one raster band may hold (0 = 64 MB)
+    // Dynamic tile order: [0] the next tile index, [1] units that have finished taking
+    // tiles; both 0 at launch, and the last unit to finish sets them back to 0. nullptr:
+    // static order. Two kernels that may run at the same time never share one.
+    int* tile_queue;
     int* err;                       // latched error word
     uint64_t wait_ns;               // bound on every wait
 };
 
 __device__ __forceinline__ void latch_error(int* err, int code) { atomicCAS(err, 0, code); }
+
+// The sequence of tiles a unit (CTA or CTA pair) runs, -1 at its end.
+// Static order: unit u runs tiles u, u + units, u + 2 units, ... Over hundreds of waves
+// the units drift apart, and tiles that share an A block (or a B panel) no longer run
+// together: each then reads the block from DRAM on its own.
+// Dynamic order: the pair leader's TMA producer takes the next index from a kernel-wide
+// counter as it starts a tile, so tiles start in index order whichever units run ahead.
+// It publishes each index through a ring of SCHED_SLOTS in the shared memory of both CTAs
+// of the pair ("slot written" barriers of each CTA); every other role reads the ring in
+// the same order and frees the slot on the leader's "slot read" barrier.
+struct TileSeq {
+    int next, step, num;          // static order
+    bool dyn;
+    int* ring;                    // this CTA's ring
+    uint64_t* full;               // this CTA's "slot written" barriers
+    uint64_t* empty;              // "slot read" barriers (the leader's count)
+    int slot;
+    uint32_t ph;
+};
+
+__device__ __forceinline__ TileSeq tile_seq(int unit, int n_units, int num_tiles, bool dyn, int* ring, uint64_t* full,
+                                            uint64_t* empty) {
+    TileSeq q;
+    q.next = unit;
+    q.step = n_units;
+    q.num = num_tiles;
+    q.dyn = dyn;
+    q.ring = ring;
+    q.full = full;
+    q.empty = empty;
+    q.slot = 0;
+    q.ph = 0;
+    return q;
+}
+
+// A reader's next tile (one thread per reading warp or role). False: the wait ran out.
+template <bool kPair>
+__device__ __forceinline__ bool seq_take(TileSeq& q, int& tile, uint64_t lim, volatile int* abort_flag,
+                                         uint32_t nap) {
+    if (!q.dyn) {
+        tile = q.next < q.num ? q.next : -1;
+        q.next += q.step;
+        return true;
+    }
+    if (!mbar_wait_bounded<kPair>(&q.full[q.slot], q.ph, lim, abort_flag, nap)) return false;
+    tile = *reinterpret_cast<volatile int*>(q.ring + q.slot);
+    if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&q.empty[q.slot]), 0));
+    else mbar_arrive(&q.empty[q.slot]);
+    if (++q.slot == SCHED_SLOTS) { q.slot = 0; q.ph ^= 1; }
+    return true;
+}
+
+// The writer's next tile (the leader's TMA producer): take it from the counter and
+// publish it to both CTAs' rings.
+template <bool kPair>
+__device__ __forceinline__ bool seq_publish(TileSeq& q, int* counter, int& tile, uint64_t lim,
+                                            volatile int* abort_flag) {
+    if (!q.dyn) {
+        tile = q.next < q.num ? q.next : -1;
+        q.next += q.step;
+        return true;
+    }
+    if (!mbar_wait_bounded<kPair>(&q.empty[q.slot], q.ph ^ 1, lim, abort_flag)) return false;
+    int t = atomicAdd(counter, 1);
+    if (t >= q.num) t = -1;
+    *reinterpret_cast<volatile int*>(q.ring + q.slot) = t;
+    if constexpr (kPair) {
+        st_shared_cluster_u32(mapa_shared(smem_u32(q.ring + q.slot), 1), static_cast<uint32_t>(t));
+        mbar_arrive_cluster(mapa_shared(smem_u32(&q.full[q.slot]), 1));
+    }
+    mbar_arrive(&q.full[q.slot]);
+    if (++q.slot == SCHED_SLOTS) { q.slot = 0; q.ph ^= 1; }
+    tile = t;
+    return true;
+}
+
+// The writer is done taking tiles (normally or not): the last unit to get here sets the
+// queue back to 0 for the next kernel that uses it.
+__device__ __forceinline__ void seq_finish(int* queue, int n_units) {
+    __threadfence();
+    if (atomicAdd(queue + 1, 1) == n_units - 1) {
+        __threadfence();
+        atomicExch(queue, 0);
+        atomicExch(queue + 1, 0);
+    }
+}
 
 // Tile order: bands of `group_n` N-blocks; inside a band the M-block advances slowest
 // and the band's N-blocks fastest, so the CTAs running together share both their A
@@ -286,6 +382,13 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     uint64_t* tmem_full = bars + 4 * S;
     uint64_t* tmem_empty = bars + 4 * S + 2;
     uint64_t* drain = bars + 4 * S + 4;
+    uint64_t* sched_full = bars + 4 * S + 5;
+    uint64_t* sched_empty = sched_full + SCHED_SLOTS;
+    int* ring = reinterpret_cast<int*>(smem + L::RING_OFFSET);
+    // readers of each ring slot: the second CTA's TMA producer, the MMA issuer, the relay
+    // threads, the cp.async gather warps, the thread-gather warps, the epilogue warps
+    constexpr uint32_t sched_readers = (kPair ? 1 : 0) + 1 + ((kTG && !kLN) ? kCtas : 0) + (kGatherThreads ? 2 : 0) +
+                                       (kTG ? 4 * kCtas : 0) + 4 * kCtas;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFFSET);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFFSET + 4);
 
@@ -309,6 +412,10 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             mbar_init(&tmem_empty[a], 4 * kCtas);               // every epilogue warp of the pair
         }
         mbar_init(drain, 1);
+        for (int j = 0; j < SCHED_SLOTS; ++j) {
+            mbar_init(&sched_full[j], 1);
+            mbar_init(&sched_empty[j], sched_readers);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -344,6 +451,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     const uint64_t lim = p.wait_ns;
     const int unit = blockIdx.x / kCtas;                      // CTA (or CTA pair) index
     const int n_units = gridDim.x / kCtas;
+    const bool dyn = p.tile_queue != nullptr;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (each CTA loads its own halves)
@@ -354,7 +462,13 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             bool ok = true;
             const int nch = (kAMode == A_IM2COL) ? BM / p.chunk : 0;
             const uint32_t expect = (kAMode == A_CPASYNC || kTG ? 0 : L::A_BYTES * kCtas) + L::B_BYTES * kCtas;
-            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+            TileSeq seq = tile_seq(unit, n_units, num_tiles, dyn, ring, sched_full, sched_empty);
+            while (ok) {
+                int tile;
+                const bool got = leader ? seq_publish<kPair>(seq, p.tile_queue, tile, lim, abort_flag)
+                                        : seq_take<kPair>(seq, tile, lim, abort_flag, 0);
+                if (!got) { ok = false; break; }
+                if (tile < 0) break;
                 int m_blk, n_blk;
                 tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
                 const int a_row_tile = m_blk * kCtas + static_cast<int>(rank);   // this CTA's 128-row slice
@@ -434,6 +548,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
             }
+            if (dyn && leader) seq_finish(p.tile_queue, n_units);
             if (!ok) {
                 *abort_flag = 1;
                 latch_error(p.err, ERR_TIMEOUT);
@@ -466,7 +581,11 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+            TileSeq seq = tile_seq(unit, n_units, num_tiles, dyn, ring, sched_full, sched_empty);
+            while (ok) {
+                int tile;
+                if (!seq_take<kPair>(seq, tile, lim, abort_flag, 0)) { ok = false; break; }
+                if (tile < 0) break;
                 if (!mbar_wait_bounded(&tmem_empty[acc], acc_phase ^ 1, lim, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -516,7 +635,11 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             uint32_t phase = 0;
             bool ok = true;
             const uint32_t gat_leader = kPair ? mapa_shared(smem_u32(&full_gat[0]), 0) : 0u;
-            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+            TileSeq seq = tile_seq(unit, n_units, num_tiles, dyn, ring, sched_full, sched_empty);
+            while (ok) {
+                int tile;
+                if (!seq_take<kPair>(seq, tile, lim, abort_flag, GATHER_NAP_NS)) { ok = false; break; }
+                if (tile < 0) break;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full_loc[stage], phase, lim, abort_flag, GATHER_NAP_NS)) { ok = false; break; }
                     fence_proxy_async_smem();
@@ -539,7 +662,15 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+            TileSeq seq = tile_seq(unit, n_units, num_tiles, dyn, ring, sched_full, sched_empty);
+            while (ok) {
+                // lane 0 of each of the two warps reads the ring, its warp follows
+                int tile = 0, got = 1;
+                if ((threadIdx.x & 31) == 0) got = seq_take<kPair>(seq, tile, lim, abort_flag, GATHER_NAP_NS) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                tile = __shfl_sync(0xffffffffu, tile, 0);
+                if (!got) { ok = false; break; }
+                if (tile < 0) break;
                 int m_blk, n_blk;
                 tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
                 int base[16];
@@ -656,7 +787,14 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                 if (++tkb == kblocks) tkb = 0;
                 return true;
             };
-            for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+            TileSeq seq = tile_seq(unit, n_units, num_tiles, dyn, ring, sched_full, sched_empty);
+            while (ok) {
+                int tile = 0, got = 1;
+                if (lane == 0) got = seq_take<kPair>(seq, tile, lim, abort_flag, GATHER_NAP_NS) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                tile = __shfl_sync(0xffffffffu, tile, 0);
+                if (!got) { ok = false; break; }
+                if (tile < 0) break;
                 int m_blk, n_blk;
                 tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
                 const int row0 = (m_blk * kCtas + static_cast<int>(rank)) * BM;      // this CTA's 128 rows
@@ -791,11 +929,18 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
         uint32_t acc_phase = 0;
         bool ok = true;
         const int status_ok = p.fwd_status ? (*p.fwd_status == 0) : 1;
-        for (int tile = unit; tile < num_tiles && ok; tile += n_units) {
+        TileSeq seq = tile_seq(unit, n_units, num_tiles, dyn, ring, sched_full, sched_empty);
+        while (ok) {
+            // one lane reads the ring and waits, the warp follows it, so tcgen05.ld below is
+            // never divergent
+            int tile = 0, got = 1;
+            if (lane == 0) got = seq_take<kPair>(seq, tile, lim, abort_flag, EPI_NAP_NS) ? 1 : 0;
+            got = __shfl_sync(0xffffffffu, got, 0);
+            tile = __shfl_sync(0xffffffffu, tile, 0);
+            if (!got) { ok = false; break; }
+            if (tile < 0) break;
             int m_blk, n_blk;
             tile_coords(tile, m_tiles, n_tiles, group_n, m_blk, n_blk);
-            // one lane waits, the warp follows it, so tcgen05.ld below is never divergent
-            int got = 0;
             if (lane == 0) got = mbar_wait_bounded(&tmem_full[acc], acc_phase, lim, abort_flag, EPI_NAP_NS) ? 1 : 0;
             got = __shfl_sync(0xffffffffu, got, 0);
             if (!got) { ok = false; break; }

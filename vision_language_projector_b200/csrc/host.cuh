@@ -36,6 +36,8 @@ using vlp::ViewDesc;
 
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+// Tile queues per handle (dynamic tile order): counter pairs taken in turn by launches.
+constexpr uint32_t kTileQueues = 64;
 
 struct DriverFns {
     PFN_cuTensorMapEncodeTiled_v12000 tiled = nullptr;
@@ -427,25 +429,6 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
     return VLPROJ_OK;
 }
 
-// Tile shape: 256 x 256 tiles on CTA pairs when N allows and the A operand comes by
-// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise. tc / tct / tc2: output
-// maps of the TMA-store epilogues (unused by the others).
-inline const CUtensorMap& no_map() {
-    static const CUtensorMap zero{};
-    return zero;
-}
-
-template <int A, int E>
-int launch_gemm_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb_half,
-                   const GemmParams& p, int num_sms, cudaStream_t s, const CUtensorMap& tc = no_map(),
-                   const CUtensorMap& tct = no_map(), const CUtensorMap& tc2 = no_map()) {
-    if constexpr (A != vlp::A_CPASYNC) {
-        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tct, tc2, p, num_sms, s);
-    }
-    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tct, tc2, p, num_sms, s);
-    return launch_gemm<128, A, E, 1>(ta, tb, tc, tct, tc2, p, num_sms, s);
-}
-
 inline int pick_bn(int N) { return N >= 256 ? 256 : 128; }
 
 }  // namespace vlp_host
@@ -469,6 +452,12 @@ struct vlproj_handle {
     CUtensorMap tmW1h{}, tmW2h{};        // B boxes of 128 rows (each CTA of a pair loads half)
     bool pairs = true;                   // run 256 x 256 tiles on CTA pairs where possible
     int64_t l2_budget = 0;               // forward GEMMs: bytes of B per raster band (0 = 64 MB)
+    // dynamic tile order: kTileQueues counter pairs, taken in turn by successive GEMM
+    // launches (kernels that may overlap, on the caller's and the side stream, are a few
+    // launches apart and so never share one)
+    bool dynamic_tiles = true;
+    int* tqueue = nullptr;
+    uint32_t tq_next = 0;
     // scratch, grown on demand
     vlp_host::DevBuf<__nv_bfloat16> H, H2, Xn, A;       // H2: second hidden buffer (depth > 2)
     // middle layers (depth > 2): weights, biases, tensor maps (BN-row and 128-row boxes)
@@ -521,6 +510,29 @@ struct vlproj_handle {
 };
 
 namespace vlp_host {
+
+// Tile shape: 256 x 256 tiles on CTA pairs when N allows and the A operand comes by
+// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise. tc / tct / tc2: output
+// maps of the TMA-store epilogues (unused by the others). Each launch takes the handle's
+// next tile queue (dynamic tile order) unless the static order is selected.
+inline const CUtensorMap& no_map() {
+    static const CUtensorMap zero{};
+    return zero;
+}
+
+template <int A, int E>
+int launch_gemm_bn(vlproj_handle* h, int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb,
+                   const CUtensorMap& tb_half, GemmParams p, cudaStream_t s, const CUtensorMap& tc = no_map(),
+                   const CUtensorMap& tct = no_map(), const CUtensorMap& tc2 = no_map()) {
+    p.tile_queue = nullptr;
+    if (h->dynamic_tiles && h->tqueue) p.tile_queue = h->tqueue + 2 * (h->tq_next++ % kTileQueues);
+    const int num_sms = h->num_sms;
+    if constexpr (A != vlp::A_CPASYNC) {
+        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tct, tc2, p, num_sms, s);
+    }
+    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tct, tc2, p, num_sms, s);
+    return launch_gemm<128, A, E, 1>(ta, tb, tc, tct, tc2, p, num_sms, s);
+}
 
 // Stage timing: begin / end events on the stream that runs the stage.
 inline void stage_begin(vlproj_handle* h, int stage, cudaStream_t s) {

@@ -38,15 +38,27 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 // Test the phase; while it is incomplete the thread may sleep until it completes or
 // about `suspend_ns` pass (a hint), so waiting threads issue almost nothing.
+// kCluster: acquire at cluster scope, for a phase completed by arrivals (release,
+// cluster scope) from the other CTA of a pair that also wrote this CTA's shared memory.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t suspend_ns = 20000) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
-        : "memory");
+    if constexpr (kCluster)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+            : "memory");
     return ok != 0;
 }
 
@@ -56,14 +68,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
 // every 16th failed test only, and a waiter that is not on the critical path (sleep_ns >
 // 0) naps between tests: a spinning thread takes issue slots from the warps that share
 // its scheduler (the TMA producer, the MMA issuer, the epilogue).
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                   volatile int* abort_flag, uint32_t sleep_ns = 0) {
     const uint32_t hint = limit_ns < 20000 ? static_cast<uint32_t>(limit_ns) : 20000u;
-    if (mbar_try_wait(bar, parity, hint)) return true;
+    if (mbar_try_wait<kCluster>(bar, parity, hint)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (sleep_ns) __nanosleep(sleep_ns);
-        if (mbar_try_wait(bar, parity, hint)) return true;
+        if (mbar_try_wait<kCluster>(bar, parity, hint)) return true;
         if ((it & 15u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns) return false;
@@ -169,6 +182,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 32-bit store to shared memory of a CTA of the cluster (address from mapa_shared).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // Pair forms of the TMA loads: data lands in the issuing CTA's shared memory, the

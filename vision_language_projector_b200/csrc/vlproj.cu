@@ -181,26 +181,26 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     ++h->launches;
     int rc;
     if (pl.fused)
-        rc = launch_gemm_bn<vlp::A_FUSED, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                         h->num_sms, s, tmC);
+        rc = launch_gemm_bn<vlp::A_FUSED, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                         s, tmC);
     else if (pl.tgather_ln)
-        rc = launch_gemm_bn<vlp::A_TGATHER_LN, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                              h->num_sms, s, tmC);
+        rc = launch_gemm_bn<vlp::A_TGATHER_LN, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                              s, tmC);
     else if (pl.tgather)
-        rc = launch_gemm_bn<vlp::A_TGATHER, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                           h->num_sms, s, tmC);
+        rc = launch_gemm_bn<vlp::A_TGATHER, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                           s, tmC);
     else if (pl.merged_ln)
-        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                        h->num_sms, s, tmC);
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                        s, tmC);
     else if (pl.box5)
-        rc = launch_gemm_bn<vlp::A_BOX5, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                        h->num_sms, s, tmC);
+        rc = launch_gemm_bn<vlp::A_BOX5, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                        s, tmC);
     else if (im2col)
-        rc = launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                          h->num_sms, s, tmC);
+        rc = launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
+                                                          s, tmC);
     else
-        rc = launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(pick_bn(c.N1), false, tmA, h->tmW1, h->tmW1h, p,
-                                                           h->num_sms, s, tmC);
+        rc = launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(h, pick_bn(c.N1), false, tmA, h->tmW1, h->tmW1h, p,
+                                                           s, tmC);
     if (rc) return rc;
     stage_end(h, 3, s);
     return VLPROJ_OK;
@@ -231,8 +231,8 @@ int run_middle_layers(vlproj_handle* h, const Plan& pl, cudaStream_t s, const __
         q.tma_store = 1;
         if (encode_bf16_store(&tout, dst.ptr, pl.M, c.N1)) return VLPROJ_ERR_CUDA;
         ++h->launches;
-        int rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(pick_bn(c.N1), h->pairs, tin, h->tmWm[layer],
-                                                            h->tmWmh[layer], q, h->num_sms, s, tout);
+        int rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tin, h->tmWm[layer],
+                                                            h->tmWmh[layer], q, s, tout);
         if (rc) return rc;
         last_in_h2 = !last_in_h2;
     }
@@ -348,7 +348,8 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
     const size_t n1 = static_cast<size_t>(cfg->N1), n2 = static_cast<size_t>(cfg->N2), C = static_cast<size_t>(cfg->C);
     if (cudaMalloc(&h->W1p, n1 * h->K1 * 2) || cudaMalloc(&h->W2, n2 * n1 * 2) || cudaMalloc(&h->b1, n1 * 4) ||
         cudaMalloc(&h->b2, n2 * 4) || cudaMalloc(&h->gamma, C * 4) || cudaMalloc(&h->beta, C * 4) ||
-        cudaMalloc(&h->status, 2 * sizeof(int)) || cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) ||
+        cudaMalloc(&h->status, 2 * sizeof(int)) || cudaMalloc(&h->tqueue, 2 * kTileQueues * sizeof(int)) ||
+        cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) ||
         cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming) ||
         cudaEventCreateWithFlags(&h->join, cudaEventDisableTiming) ||
         cudaEventCreateWithFlags(&h->join2, cudaEventDisableTiming))
@@ -371,7 +372,8 @@ int vlproj_create(const vlproj_config* cfg, vlproj_handle** out) {
     } else if (cudaMemset(h->gamma, 0, C * 4) || cudaMemset(h->beta, 0, C * 4)) {
         return fail(VLPROJ_ERR_CUDA);
     }
-    if (cudaMemset(h->status, 0, 2 * sizeof(int))) return fail(VLPROJ_ERR_CUDA);
+    if (cudaMemset(h->status, 0, 2 * sizeof(int)) || cudaMemset(h->tqueue, 0, 2 * kTileQueues * sizeof(int)))
+        return fail(VLPROJ_ERR_CUDA);
     if (cudaDeviceSynchronize()) return fail(VLPROJ_ERR_CUDA);
     for (int i = 0; i < cfg->depth - 2; ++i) {
         __nv_bfloat16* w = nullptr;
@@ -416,6 +418,7 @@ void vlproj_destroy(vlproj_handle* h) {
     cudaFree(h->gamma);
     cudaFree(h->beta);
     cudaFree(h->status);
+    cudaFree(h->tqueue);
     h->H.release();
     h->H2.release();
     cudaFree(h->W2t);
@@ -472,6 +475,12 @@ int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns) {
 int vlproj_set_raster_budget(vlproj_handle* h, int64_t bytes) {
     if (!h || bytes < 0) return VLPROJ_ERR_INVALID_ARG;
     h->l2_budget = bytes;
+    return VLPROJ_OK;
+}
+
+int vlproj_set_tile_order(vlproj_handle* h, int dynamic) {
+    if (!h) return VLPROJ_ERR_INVALID_ARG;
+    h->dynamic_tiles = dynamic != 0;
     return VLPROJ_OK;
 }
 
@@ -653,8 +662,8 @@ int vlproj_forward_ex(vlproj_handle* h, const vlproj_forward_args* args, void* s
     p.l2_budget = h->l2_budget;
     stage_begin(h, 4, s);
     ++h->launches;
-    rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(pick_bn(c.N2), h->pairs, h->tmH, h->tmW2, h->tmW2h, p,
-                                                       h->num_sms, s);
+    rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(h, pick_bn(c.N2), h->pairs, h->tmH, h->tmW2, h->tmW2h, p,
+                                                       s);
     if (rc) return fail_joined(rc);
     stage_end(h, 4, s);
 

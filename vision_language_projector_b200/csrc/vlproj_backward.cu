@@ -244,9 +244,9 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
                 if (encode_bf16_store(&tmHr, h->Hr.ptr + (l - 1) * hslab, M, c.N1)) return VLPROJ_ERR_CUDA;
             }
             ++h->launches;
-            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(pick_bn(c.N1), h->pairs, tmA,
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(h, pick_bn(c.N1), h->pairs, tmA,
                                                              first ? h->tmW1 : h->tmWm[l - 2],
-                                                             first ? h->tmW1h : h->tmWmh[l - 2], p, h->num_sms, s,
+                                                             first ? h->tmW1h : h->tmWmh[l - 2], p, s,
                                                              tmG, tmHt, tmHr);
             if (rc) return rc;
         }
@@ -284,8 +284,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         q.outf = a->d_W2;
         stage_begin(h, 11, ss);
         ++h->launches;
-        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(c.N1), h->pairs, tmA2, tmB2, tmB2h, q, h->num_sms,
-                                                       ss);
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(h, pick_bn(c.N1), h->pairs, tmA2, tmB2, tmB2h, q, ss);
         if (rc) return rc;
         stage_end(h, 11, ss);
     }
@@ -315,9 +314,9 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
                 return VLPROJ_ERR_CUDA;
             p.ct_kb64 = 1;
             ++h->launches;
-            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(pick_bn(c.N1), h->pairs, tmA,
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(h, pick_bn(c.N1), h->pairs, tmA,
                                                              top ? h->tmW2t : h->tmWmt[l - 1],
-                                                             top ? h->tmW2th : h->tmWmth[l - 1], p, h->num_sms, s,
+                                                             top ? h->tmW2th : h->tmWmth[l - 1], p, s,
                                                              tmP, tmPt);
             if (rc) return rc;
             cur = nxt;
@@ -333,8 +332,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
                 q.a_kb64 = q.b_kb64 = 1;
                 q.outf = mid_w(i);
                 ++h->launches;
-                rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(c.N1), h->pairs, ta, tb, tbh, q, h->num_sms,
-                                                               s);
+                rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(h, pick_bn(c.N1), h->pairs, ta, tb, tbh, q, s);
                 if (rc) return rc;
             }
             if (mid_b(i)) {
@@ -370,8 +368,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         q.a_kb64 = q.b_kb64 = 1;
         q.outf = a->d_W1;
         ++h->launches;
-        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(pick_bn(K1), h->pairs, tmA2, tmB2, tmB2h, q, h->num_sms,
-                                                       ss);
+        rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(h, pick_bn(K1), h->pairs, tmA2, tmB2, tmB2h, q, ss);
         if (rc) return rc;
         stage_end(h, 12, ss);
     }
@@ -394,13 +391,13 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             CUtensorMap tmD{};
             if (encode_bf16_store(&tmD, h->dA.ptr, M, K1)) return VLPROJ_ERR_CUDA;
             p.tma_store = 1;
-            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BF16>(pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth, p,
-                                                            h->num_sms, s, tmD);
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BF16>(h, pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth, p,
+                                                            s, tmD);
         } else {
             p.outf = a->d_features;
             p.gmeta = h->gmeta.ptr;
-            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_FOLD_F32>(pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth,
-                                                                p, h->num_sms, s);
+            rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_FOLD_F32>(h, pick_bn(K1), h->pairs, tmA, h->tmW1pt, h->tmW1pth,
+                                                                p, s);
         }
         if (rc) return rc;
         stage_end(h, 13, s);

@@ -66,8 +66,8 @@ int project_rows(vlproj_handle* h, const Chunk& ch, const void* features, __nv_b
     p.wait_ns = h->wait_ns;
     stage_begin(h, 4, s);
     ++h->launches;
-    rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(pick_bn(c.N2), h->pairs, tmH, h->tmW2, h->tmW2h, p,
-                                                       h->num_sms, s);
+    rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_SCATTER>(h, pick_bn(c.N2), h->pairs, tmH, h->tmW2, h->tmW2h, p,
+                                                       s);
     if (rc) return rc;
     stage_end(h, 4, s);
     if (c.tile_tag == VLPROJ_TILE_2D && !pl.images.empty()) {
