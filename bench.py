@@ -62,8 +62,9 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--raster-mb", type=int, default=0,
                     help="GEMM raster band budget in MB (vlproj_set_raster_budget); 0 = the library default")
-    ap.add_argument("--tile-order", choices=("dynamic", "static"), default="dynamic",
-                    help="GEMM tile order (vlproj_set_tile_order): from a counter (default) or fixed per CTA")
+    ap.add_argument("--tile-order", choices=("auto", "dynamic", "static"), default="auto",
+                    help="GEMM tile order (vlproj_set_tile_order): the library's choice (default), every GEMM "
+                         "from a counter, or fixed per CTA")
     ap.add_argument("--gather", default="auto", choices=["auto", "box", "im2col", "cpasync", "threads", "fused", "merged"],
                     help="GEMM1's merge-gather (vlproj_set_gather_mode); auto = the library's choice")
     return ap.parse_args()
@@ -329,7 +330,8 @@ def main():
                           "cpasync": vp.GATHER_CPASYNC, "threads": vp.GATHER_THREADS, "fused": vp.GATHER_FUSED,
                           "merged": vp.GATHER_MERGED}[args.gather])
     proj.set_raster_budget(args.raster_mb << 20)
-    proj.set_tile_order(args.tile_order == "dynamic")
+    proj.set_tile_order({"static": vp.TILE_ORDER_STATIC, "auto": vp.TILE_ORDER_AUTO,
+                         "dynamic": vp.TILE_ORDER_DYNAMIC}[args.tile_order])
     feats = f32(feats_h) if wl.feat_fp32 else bf(feats_h)
     ids = torch.from_numpy(ids_h).cuda()
     prefill = bf(prefill_h)

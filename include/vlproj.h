@@ -348,15 +348,19 @@ int vlproj_set_tile_pairs(vlproj_handle* h, int enable);
 int vlproj_set_raster_budget(vlproj_handle* h, int64_t bytes);
 
 /* Order in which the GEMMs' persistent CTAs (or CTA pairs) take their output tiles.
- * dynamic != 0 (the default): each takes the next tile of the raster order from a
- * counter in device memory when it starts one, so tiles start in raster order however
- * the CTAs' speeds differ, and the tiles that share an A block or a B panel run at the
- * same time and read it from L2. dynamic = 0: CTA u runs tiles u, u + CTAs, u + 2 CTAs,
- * ... (over hundreds of waves the CTAs drift apart and re-read operands from DRAM). The
- * handle holds 64 counters, zeroed by vlproj_create and left zeroed by every GEMM; calls
- * on one handle must not run concurrently (as for its other scratch). Both orders give
- * the same bits (each output's K order is fixed). */
-int vlproj_set_tile_order(vlproj_handle* h, int dynamic);
+ * VLPROJ_TILE_ORDER_DYNAMIC: each takes the next tile of the raster order from a counter
+ * in device memory when it starts one, so tiles start in raster order however the CTAs'
+ * speeds differ, and the tiles that share an A block or a B panel run at the same time
+ * and read it from L2. VLPROJ_TILE_ORDER_STATIC: CTA u runs tiles u, u + CTAs, u + 2 CTAs,
+ * ... (over hundreds of waves the CTAs drift apart and re-read operands from DRAM).
+ * VLPROJ_TILE_ORDER_AUTO (the default): dynamic for GEMMs whose A operand is gathered
+ * (the merge-gather feeds) and for those with at least 64 waves of tiles, static for the
+ * other plain-matrix GEMMs (measured faster so). The handle holds 64 counters, zeroed by
+ * vlproj_create and left zeroed by every GEMM; calls on one handle must not run
+ * concurrently (as for its other scratch). Every order gives the same bits (each
+ * output's K order is fixed). Other values are rejected with VLPROJ_ERR_INVALID_ARG. */
+enum { VLPROJ_TILE_ORDER_STATIC = 0, VLPROJ_TILE_ORDER_AUTO = 1, VLPROJ_TILE_ORDER_DYNAMIC = 2 };
+int vlproj_set_tile_order(vlproj_handle* h, int order);
 
 /* Host only, no device work: the processor's tiling choices for the 2D tile scheme
  * ("port DeepSeek-VL2", Processor steps 1, 2, 6, 7). For each image of one request,

@@ -120,3 +120,11 @@ def test_create_rejects_deeper_mlp_without_middle_weights():
     cfg = vp.make_config(2, 64, 64, 32, depth=3, W1=16, W2=16)     # non-null stand-ins, never dereferenced
     h = ctypes.c_void_p()
     assert vp._lib.vlproj_create(ctypes.byref(cfg), ctypes.byref(h)) == vp.ERR_INVALID_ARG
+
+
+def test_setters_reject_a_null_handle_and_bad_values():
+    """Host-side argument checks of the tuning setters, no device work."""
+    assert vp._lib.vlproj_set_tile_order(None, vp.TILE_ORDER_AUTO) == vp.ERR_INVALID_ARG
+    assert vp._lib.vlproj_set_raster_budget(None, 0) == vp.ERR_INVALID_ARG
+    assert vp._lib.vlproj_set_tile_pairs(None, 1) == vp.ERR_INVALID_ARG
+    assert (vp.TILE_ORDER_STATIC, vp.TILE_ORDER_AUTO, vp.TILE_ORDER_DYNAMIC) == (0, 1, 2)

@@ -142,12 +142,15 @@ def test_backward_is_deterministic_and_tile_shape_independent():
     proj.set_tile_pairs(False)
     _, c = run_backward(case, proj, dev, d_dev)
     proj.set_tile_pairs(True)
-    proj.set_tile_order(False)       # static tile order: the same tiles, the same K order
+    proj.set_tile_order(vp.TILE_ORDER_DYNAMIC)    # every GEMM from a counter: same tiles, same K order
     _, d = run_backward(case, proj, dev, d_dev)
+    proj.set_tile_order(vp.TILE_ORDER_STATIC)
+    _, e = run_backward(case, proj, dev, d_dev)
     for n in a:
         np.testing.assert_array_equal(a[n], b[n], err_msg=n)
         np.testing.assert_array_equal(a[n], c[n], err_msg=n)
         np.testing.assert_array_equal(a[n], d[n], err_msg=n)
+        np.testing.assert_array_equal(a[n], e[n], err_msg=n)
 
 
 @pytest.mark.parametrize("name", ["tiled_2x1", "ragged_ln_bf16"])

@@ -244,22 +244,25 @@ def test_deeper_mlp_all_rows(depth, pairs):
 
 @pytest.mark.parametrize("workload", ["dsvit", "vl2"])
 def test_tile_order_does_not_change_the_bits(workload):
-    """The dynamic tile order (units take the next tile from a counter) and the static
-    one run the same tiles with the same K order. Forty more forwards on the handle take
-    its 64 tile queues round more than once: each GEMM must leave its queue at zero."""
+    """The dynamic tile order (units take the next tile from a counter), the static one
+    and the automatic choice run the same tiles with the same K order. Forty more
+    forwards in the dynamic order take the handle's 64 tile queues round more than once:
+    each GEMM must leave its queue at zero."""
     wl = W.WORKLOADS[workload]
     case = make_case(wl)
     proj = make_projector(case)
     dev = DeviceInputs(case)
-    out_dyn = run(case, proj, dev)
-    proj.set_tile_order(False)
+    out_auto = run(case, proj, dev)
+    proj.set_tile_order(vp.TILE_ORDER_STATIC)
     out_static = run(case, proj, dev)
-    proj.set_tile_order(True)
+    proj.set_tile_order(vp.TILE_ORDER_DYNAMIC)
+    out_dyn = run(case, proj, dev)
     for _ in range(40):
         out_again = run(case, proj, dev)
     assert proj.status() == vp.OK
-    assert torch.equal(out_dyn.view(torch.int16), out_static.view(torch.int16))
-    assert torch.equal(out_dyn.view(torch.int16), out_again.view(torch.int16))
+    assert torch.equal(out_auto.view(torch.int16), out_static.view(torch.int16))
+    assert torch.equal(out_auto.view(torch.int16), out_dyn.view(torch.int16))
+    assert torch.equal(out_auto.view(torch.int16), out_again.view(torch.int16))
 
 
 @pytest.mark.parametrize("budget", [1 << 20, 256 << 20])

@@ -30,6 +30,7 @@ EXPORTED = ("vlproj_create", "vlproj_forward", "vlproj_hidden", "vlproj_status",
             "vlproj_plan_tiles", "vlproj_backward", "vlproj_project_host", "vlproj_profile_stages",
             "vlproj_set_raster_budget", "vlproj_set_tile_order")
 NOALLOC_MAX_IDS = 64 * 1024 * 1024
+TILE_ORDER_STATIC, TILE_ORDER_AUTO, TILE_ORDER_DYNAMIC = 0, 1, 2
 GATHER_IM2COL, GATHER_CPASYNC, GATHER_AUTO, GATHER_BOX, GATHER_THREADS, GATHER_FUSED, GATHER_MERGED = 0, 1, 2, 3, 4, 5, 6
 NUM_STAGES = 15
 STAGES = ("index", "geometry", "layernorm", "gemm1", "gemm2", "special_rows",
@@ -512,8 +513,9 @@ class Projector:
         if rc != OK:
             raise VlprojError(rc, "vlproj_set_raster_budget")
 
-    def set_tile_order(self, dynamic: bool) -> None:
-        rc = _lib.vlproj_set_tile_order(self._h, 1 if dynamic else 0)
+    def set_tile_order(self, order: int) -> None:
+        """TILE_ORDER_STATIC, TILE_ORDER_AUTO (the default) or TILE_ORDER_DYNAMIC."""
+        rc = _lib.vlproj_set_tile_order(self._h, int(order))
         if rc != OK:
             raise VlprojError(rc, "vlproj_set_tile_order")
 

@@ -38,6 +38,12 @@ using vlp::ViewDesc;
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 // Tile queues per handle (dynamic tile order): counter pairs taken in turn by launches.
 constexpr uint32_t kTileQueues = 64;
+// Automatic tile order: GEMMs whose A is a plain row-major matrix keep the static order
+// below this many waves of tiles (measured 1-3 % slower in the dynamic order at 10-25
+// waves: MoonViT's GEMM1 over the merged copy, VL2's and DS-ViT's GEMM2), the rest take
+// the dynamic one (1-2 % faster for the gathered-A GEMM1s, 11 % for the 277-wave Stress
+// batch under the power cap, where it halves the DRAM reads).
+constexpr int kDynamicMinWaves = 64;
 
 struct DriverFns {
     PFN_cuTensorMapEncodeTiled_v12000 tiled = nullptr;
@@ -455,7 +461,7 @@ struct vlproj_handle {
     // dynamic tile order: kTileQueues counter pairs, taken in turn by successive GEMM
     // launches (kernels that may overlap, on the caller's and the side stream, are a few
     // launches apart and so never share one)
-    bool dynamic_tiles = true;
+    int tile_order = VLPROJ_TILE_ORDER_AUTO;
     int* tqueue = nullptr;
     uint32_t tq_next = 0;
     // scratch, grown on demand
@@ -513,8 +519,8 @@ namespace vlp_host {
 
 // Tile shape: 256 x 256 tiles on CTA pairs when N allows and the A operand comes by
 // TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise. tc / tct / tc2: output
-// maps of the TMA-store epilogues (unused by the others). Each launch takes the handle's
-// next tile queue (dynamic tile order) unless the static order is selected.
+// maps of the TMA-store epilogues (unused by the others). A launch in the dynamic tile
+// order takes the handle's next tile queue.
 inline const CUtensorMap& no_map() {
     static const CUtensorMap zero{};
     return zero;
@@ -524,9 +530,13 @@ template <int A, int E>
 int launch_gemm_bn(vlproj_handle* h, int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb,
                    const CUtensorMap& tb_half, GemmParams p, cudaStream_t s, const CUtensorMap& tc = no_map(),
                    const CUtensorMap& tct = no_map(), const CUtensorMap& tc2 = no_map()) {
-    p.tile_queue = nullptr;
-    if (h->dynamic_tiles && h->tqueue) p.tile_queue = h->tqueue + 2 * (h->tq_next++ % kTileQueues);
     const int num_sms = h->num_sms;
+    const int ctas = (A != vlp::A_CPASYNC && pair && bn == 256) ? 2 : 1;
+    const int64_t tiles = ((static_cast<int64_t>(p.M) + vlp::BM * ctas - 1) / (vlp::BM * ctas)) * ((p.N + bn - 1) / bn);
+    const bool dyn = h->tile_order == VLPROJ_TILE_ORDER_DYNAMIC ||
+                     (h->tile_order == VLPROJ_TILE_ORDER_AUTO &&
+                      (A != vlp::A_TILE || tiles >= static_cast<int64_t>(kDynamicMinWaves) * (num_sms / ctas)));
+    p.tile_queue = (dyn && h->tqueue) ? h->tqueue + 2 * (h->tq_next++ % kTileQueues) : nullptr;
     if constexpr (A != vlp::A_CPASYNC) {
         if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tct, tc2, p, num_sms, s);
     }

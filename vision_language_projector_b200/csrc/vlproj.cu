@@ -478,9 +478,9 @@ int vlproj_set_raster_budget(vlproj_handle* h, int64_t bytes) {
     return VLPROJ_OK;
 }
 
-int vlproj_set_tile_order(vlproj_handle* h, int dynamic) {
-    if (!h) return VLPROJ_ERR_INVALID_ARG;
-    h->dynamic_tiles = dynamic != 0;
+int vlproj_set_tile_order(vlproj_handle* h, int order) {
+    if (!h || order < VLPROJ_TILE_ORDER_STATIC || order > VLPROJ_TILE_ORDER_DYNAMIC) return VLPROJ_ERR_INVALID_ARG;
+    h->tile_order = order;
     return VLPROJ_OK;
 }
 
