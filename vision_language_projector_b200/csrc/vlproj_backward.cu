@@ -407,34 +407,38 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     stage_begin(h, 14, s);
     if (want_da && c.has_ln) {
         const int64_t items = M * kk;
-        const int nb = static_cast<int>(std::min<int64_t>((items + vlp::LNB_WARPS - 1) / vlp::LNB_WARPS,
-                                                          4 * static_cast<int64_t>(h->num_sms)));
         const bool ln_sums = a->d_gamma || a->d_beta;
         const size_t smem = static_cast<size_t>(c.C) * 2 * vlp::LNB_WARPS * 4;
-        if (ln_sums && h->part.ensure(static_cast<size_t>(nb) * 2 * c.C)) return VLPROJ_ERR_CUDA;
-        float* partial = ln_sums ? h->part.ptr : nullptr;
-        ++h->launches;
         const bool f32 = c.feat_dtype == VLPROJ_FEAT_F32;
         const int nvec = c.C / 8;
+        // one wave of blocks: as many as fit on the SMs at once (their shared-memory
+        // accumulators bound it, 3 per SM at C = 1152), so no block starts late with a
+        // full share of the rows
 #define VLP_LNB(F, V)                                                                                         \
     do {                                                                                                      \
-        VLP_CUDA(cudaFuncSetAttribute(vlp::vlp_ln_backward_kernel<F, V>,                                       \
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));  \
-        vlp::vlp_ln_backward_kernel<F, V><<<nb, 256, smem, s>>>(a->features, h->gmeta.ptr, static_cast<int>(M), \
-                                                               c.k, c.C, h->gamma, eps, h->dA.ptr,              \
-                                                               a->d_features, partial);                        \
+        auto kern = vlp::vlp_ln_backward_kernel<F, V>;                                                        \
+        VLP_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))); \
+        int per_sm = 0;                                                                                       \
+        VLP_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem));                   \
+        const int nb = static_cast<int>(std::min<int64_t>((items + vlp::LNB_WARPS - 1) / vlp::LNB_WARPS,      \
+                                                          std::max(per_sm, 1) * static_cast<int64_t>(h->num_sms))); \
+        if (ln_sums && h->part.ensure(static_cast<size_t>(nb) * 2 * c.C)) return VLPROJ_ERR_CUDA;           \
+        float* partial = ln_sums ? h->part.ptr : nullptr;                                                     \
+        ++h->launches;                                                                                        \
+        kern<<<nb, 256, smem, s>>>(a->features, h->gmeta.ptr, static_cast<int>(M), c.k, c.C, h->gamma, eps,   \
+                                   h->dA.ptr, a->d_features, partial);                                        \
+        VLP_CUDA(cudaGetLastError());                                                                         \
+        if (ln_sums) {                                                                                        \
+            ++h->launches;                                                                                    \
+            vlp::vlp_colsum_kernel<<<(2 * c.C + vlp::CS_COLS - 1) / vlp::CS_COLS, vlp::CS_COLS * vlp::CS_GROUPS, 0, \
+                                     s>>>(partial, nb, c.C, a->d_gamma, a->d_beta);                           \
+            VLP_CUDA(cudaGetLastError());                                                                     \
+        }                                                                                                     \
     } while (0)
         if (nvec <= 64) { if (f32) VLP_LNB(true, 2); else VLP_LNB(false, 2); }
         else if (nvec <= 160) { if (f32) VLP_LNB(true, 5); else VLP_LNB(false, 5); }
         else { if (f32) VLP_LNB(true, 8); else VLP_LNB(false, 8); }
 #undef VLP_LNB
-        VLP_CUDA(cudaGetLastError());
-        if (ln_sums) {
-            ++h->launches;
-            vlp::vlp_colsum_kernel<<<(2 * c.C + vlp::CS_COLS - 1) / vlp::CS_COLS, vlp::CS_COLS * vlp::CS_GROUPS, 0, s>>>(
-                partial, nb, c.C, a->d_gamma, a->d_beta);
-            VLP_CUDA(cudaGetLastError());
-        }
     }
     if (!c.has_ln) {
         if (a->d_gamma) VLP_CUDA(cudaMemsetAsync(a->d_gamma, 0, static_cast<size_t>(c.C) * 4, s));
