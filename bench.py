@@ -21,6 +21,7 @@ only), on a bounded sample of the same workload per step.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -53,6 +54,9 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--images", type=int, default=0,
+                    help="run the workload with this many images instead (sequences scaled to match; for "
+                         "profiling captures of a smaller case); 0 = the workload's own count")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -237,6 +241,15 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+def pick_workload(args):
+    """The named workload, or the same shapes with --images images (sequences scaled)."""
+    wl = W.WORKLOADS[args.workload]
+    if args.images and args.images != wl.n_images:
+        seqs = max(1, -(-wl.B * args.images // wl.n_images))
+        wl = dataclasses.replace(wl, n_images=args.images, B=seqs)
+    return wl
+
+
 def workload_config(args, wl, M: int, R: int) -> dict:
     """The workload keys of `config`, the same on both arms."""
     return {"workload": args.workload, "images": wl.n_images, "merged_tokens": M, "assembled_rows": R,
@@ -248,7 +261,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     from oracle import projector as O
-    wl = W.WORKLOADS[args.workload]
+    wl = pick_workload(args)
     hw = W.grid_hw(wl, args.seed)
     crop = W.spatial_crop(wl)
     w = W.weights(wl, args.seed)
@@ -300,7 +313,7 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
-    wl = W.WORKLOADS[args.workload]
+    wl = pick_workload(args)
     # data-parallel replicas: every rank holds the same weights and a batch of the same
     # shapes (geometry, placeholder layout), with feature values of its own
     seed = args.seed
@@ -415,7 +428,7 @@ def main():
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                 "frac": achieved / peak_tf,
                 "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'}",
-                "traffic": traffic_from_profiles(args.workload, dom)}
+                "traffic": (traffic_from_profiles(args.workload, dom) if not args.images else None)}
     else:
         # algorithmic bytes of the memory-bound stages (what a perfect cache would move)
         n_ids = int(ids_h.shape[0])
@@ -432,7 +445,7 @@ def main():
         achieved = None if b is None else b / (avg[dom] / 1000.0) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
                 "frac": None if achieved is None else achieved / peaks.get("hbm_gbs"),
-                "peak_source": f"{peak_src} HBM copy", "traffic": traffic_from_profiles(args.workload, dom),
+                "peak_source": f"{peak_src} HBM copy", "traffic": (traffic_from_profiles(args.workload, dom) if not args.images else None),
                 "algorithmic_bytes": b}
 
     # bytes per step: what the path must move (features in, image rows out, ids read) beside
