@@ -354,8 +354,8 @@ int vlproj_set_raster_budget(vlproj_handle* h, int64_t bytes);
  * and read it from L2. VLPROJ_TILE_ORDER_STATIC: CTA u runs tiles u, u + CTAs, u + 2 CTAs,
  * ... (over hundreds of waves the CTAs drift apart and re-read operands from DRAM).
  * VLPROJ_TILE_ORDER_AUTO (the default): dynamic for GEMMs whose A operand is gathered
- * (the merge-gather feeds) and for those with at least 64 waves of tiles, static for the
- * other plain-matrix GEMMs (measured faster so). The handle holds 64 counters, zeroed by
+ * (the merge-gather feeds) and for those with at least 64 waves' work of 64-K-block
+ * tiles, static for the other plain-matrix GEMMs (measured faster so). The handle holds 64 counters, zeroed by
  * vlproj_create and left zeroed by every GEMM; calls on one handle must not run
  * concurrently (as for its other scratch). Every order gives the same bits (each
  * output's K order is fixed). Other values are rejected with VLPROJ_ERR_INVALID_ARG. */

@@ -39,10 +39,11 @@ constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 // Tile queues per handle (dynamic tile order): counter pairs taken in turn by launches.
 constexpr uint32_t kTileQueues = 64;
 // Automatic tile order: GEMMs whose A is a plain row-major matrix keep the static order
-// below this many waves of tiles (measured 1-3 % slower in the dynamic order at 10-25
-// waves: MoonViT's GEMM1 over the merged copy, VL2's and DS-ViT's GEMM2), the rest take
-// the dynamic one (1-2 % faster for the gathered-A GEMM1s, 11 % for the 277-wave Stress
-// batch under the power cap, where it halves the DRAM reads).
+// below this much work, counted in waves of 64-K-block tiles (measured 1-3 % slower in the
+// dynamic order at 10-25 such waves: MoonViT's GEMM1 over the merged copy, VL2's and
+// DS-ViT's GEMM2, MoonViT's weight gradients); the rest take the dynamic one (1-2 % faster
+// for the gathered-A GEMM1s; on the Stress batch under the power cap, 300-600 such waves,
+// 11 % for the forward, where it halves the DRAM reads, and 6 % for the backward).
 constexpr int kDynamicMinWaves = 64;
 
 struct DriverFns {
@@ -533,9 +534,11 @@ int launch_gemm_bn(vlproj_handle* h, int bn, bool pair, const CUtensorMap& ta, c
     const int num_sms = h->num_sms;
     const int ctas = (A != vlp::A_CPASYNC && pair && bn == 256) ? 2 : 1;
     const int64_t tiles = ((static_cast<int64_t>(p.M) + vlp::BM * ctas - 1) / (vlp::BM * ctas)) * ((p.N + bn - 1) / bn);
+    const int64_t kblocks = (static_cast<int64_t>(p.K) + vlp::BK - 1) / vlp::BK;
     const bool dyn = h->tile_order == VLPROJ_TILE_ORDER_DYNAMIC ||
                      (h->tile_order == VLPROJ_TILE_ORDER_AUTO &&
-                      (A != vlp::A_TILE || tiles >= static_cast<int64_t>(kDynamicMinWaves) * (num_sms / ctas)));
+                      (A != vlp::A_TILE ||
+                       tiles * kblocks >= static_cast<int64_t>(kDynamicMinWaves) * 64 * (num_sms / ctas)));
     p.tile_queue = (dyn && h->tqueue) ? h->tqueue + 2 * (h->tq_next++ % kTileQueues) : nullptr;
     if constexpr (A != vlp::A_CPASYNC) {
         if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tct, tc2, p, num_sms, s);
