@@ -99,11 +99,18 @@ def test_bounded_wait_timeout_then_recovery():
     case = make_case(wl, np.array([[30, 30]] * 4, np.int32))
     proj = make_projector(case)
     dev = DeviceInputs(case)
+    proj.set_tile_order(vp.TILE_ORDER_DYNAMIC)
     proj.set_wait_limit(1)
     run(case, proj, dev)
     assert proj.status() == vp.ERR_TIMEOUT
     proj.set_wait_limit(0)
     out = run(case, proj, dev)
+    assert proj.status() == vp.OK
+    check(case, out, dev)
+    # the timed-out GEMMs' tile counters were set back to zero: 33 more forwards (66
+    # GEMMs) take every one of the handle's 64 counter pairs again
+    for _ in range(33):
+        out = run(case, proj, dev)
     assert proj.status() == vp.OK
     check(case, out, dev)
 
