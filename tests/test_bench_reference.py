@@ -37,3 +37,17 @@ def test_reference_other_ranks_print_nothing():
     r = _run({"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [x for x in r.stdout.splitlines() if x.startswith("{")]
+
+
+def test_images_override_scales_the_sequences():
+    """--images keeps the workload's shapes and scales its sequences with the image count."""
+    import argparse
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    stress = W.WORKLOADS["stress"]
+    wl = bench.pick_workload(argparse.Namespace(workload="stress", images=16))
+    assert (wl.n_images, wl.B, wl.S, wl.k, wl.C, wl.N1) == (16, 1, stress.S, stress.k, stress.C, stress.N1)
+    wl = bench.pick_workload(argparse.Namespace(workload="moonvit", images=4))
+    assert (wl.n_images, wl.B) == (4, 4)
+    assert bench.pick_workload(argparse.Namespace(workload="vl2", images=0)) is W.WORKLOADS["vl2"]
