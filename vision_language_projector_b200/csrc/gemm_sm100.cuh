@@ -185,6 +185,13 @@ struct GemmParams {
     // m / 64)). ct_kb64: the epilogue's transposed copy (tmCt) is stored so, with the
     // columns from M up to the next multiple of 64 written as zeros.
     int a_kb64, b_kb64, ct_kb64;
+    // a_mn / b_mn: the operand is MN-major, read from a row-major [K][M] (or [K][N]) matrix
+    // through a 3D map (m % 64, k, m / 64) in boxes of 64 K-rows x (rows / 64) strips (the
+    // weight gradients, K = tokens, read dY, H and dP where they lie); a_mn = 2: the same
+    // strips by one 2D box (64 columns x 64 K-rows) each, for a matrix whose width is not a
+    // multiple of 64 (columns past it read as zeros). no_ct: the BWD_H and DGELU epilogues
+    // write no transposed copy.
+    int a_mn, b_mn, no_ct;
     int group_n;                    // N-blocks per raster band (see tile_coords); 0 = from l2_budget
     int64_t l2_budget;              // host only: bytes of B one raster band may hold (0 = 64 MB)
     // Dynamic tile order: [0] the next tile index, [1] units that have finished taking
@@ -502,7 +509,13 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                         const uint32_t bar = mapa_shared(smem_u32(&full_tma[stage]), 0);
                         if (leader) mbar_arrive_expect_tx(&full_tma[stage], expect);
                         if (kAMode == A_TILE || kFused) {
-                            if (p.a_kb64) tma_load_3d_pair(sa, &tmA, bar, 0, a_row_tile * BM, kb);
+                            if (p.a_mn == 2) {
+                                for (int q = 0; q < BM / 64; ++q)
+                                    tma_load_2d_pair(sa + q * 8192, &tmA, bar, (a_row_tile * (BM / 64) + q) * 64, kb * BK);
+                            } else if (p.a_mn) {
+                                tma_load_3d_pair(sa, &tmA, bar, 0, kb * BK, a_row_tile * (BM / 64));
+                            }
+                            else if (p.a_kb64) tma_load_3d_pair(sa, &tmA, bar, 0, a_row_tile * BM, kb);
                             else tma_load_2d_pair(sa, &tmA, bar, kb * BK, a_row_tile * BM);
                         } else if (kAMode == A_BOX5) {
                             const int pos = kb / cblocks;
@@ -519,12 +532,20 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                         ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
                             }
                         }
-                        if (p.b_kb64) tma_load_3d_pair(sb, &tmB, bar, 0, b_row, kb);
+                        if (p.b_mn) tma_load_3d_pair(sb, &tmB, bar, 0, kb * BK, b_row / 64);
+                        else if (p.b_kb64) tma_load_3d_pair(sb, &tmB, bar, 0, b_row, kb);
                         else tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
                     } else {
                         mbar_arrive_expect_tx(&full_tma[stage], expect);
                         if (kAMode == A_TILE || kFused) {
-                            if (p.a_kb64) tma_load_3d(sa, &tmA, &full_tma[stage], 0, a_row_tile * BM, kb);
+                            if (p.a_mn == 2) {
+                                for (int q = 0; q < BM / 64; ++q)
+                                    tma_load_2d(sa + q * 8192, &tmA, &full_tma[stage], (a_row_tile * (BM / 64) + q) * 64,
+                                                kb * BK);
+                            } else if (p.a_mn) {
+                                tma_load_3d(sa, &tmA, &full_tma[stage], 0, kb * BK, a_row_tile * (BM / 64));
+                            }
+                            else if (p.a_kb64) tma_load_3d(sa, &tmA, &full_tma[stage], 0, a_row_tile * BM, kb);
                             else tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, a_row_tile * BM);
                         } else if (kAMode == A_BOX5) {
                             const int pos = kb / cblocks;
@@ -541,7 +562,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                    ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
                             }
                         }
-                        if (p.b_kb64) tma_load_3d(sb, &tmB, &full_tma[stage], 0, b_row, kb);
+                        if (p.b_mn) tma_load_3d(sb, &tmB, &full_tma[stage], 0, kb * BK, b_row / 64);
+                        else if (p.b_kb64) tma_load_3d(sb, &tmB, &full_tma[stage], 0, b_row, kb);
                         else tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, b_row);
                     }
                     ++issued;
@@ -575,7 +597,11 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (the pair leader's lane 0)
         if (lane == 0 && leader) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM * kCtas, BN);
+            const uint32_t idesc = idesc_bf16_f32(BM * kCtas, BN) | (p.a_mn ? IDESC_A_MN : 0u) |
+                                   (p.b_mn ? IDESC_B_MN : 0u);
+            // a 16-deep K slice: 32 bytes further along a K-major row, 2 KB (two 8-row
+            // atoms) further down an MN-major strip
+            const uint32_t a_step = p.a_mn ? 2048u : 32u, b_step = p.b_mn ? 2048u : 32u;
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -598,14 +624,17 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
                     const uint32_t sb = sa + L::A_BYTES;
+                    const uint64_t da = p.a_mn ? smem_desc_mn_sw128(sa) : smem_desc_sw128(sa);
+                    const uint64_t db = p.b_mn ? smem_desc_mn_sw128(sb) : smem_desc_sw128(sb);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
+                        // the start address (16-byte units) is the descriptor's low field
+                        const uint64_t dak = da + static_cast<uint64_t>((kk * a_step) >> 4);
+                        const uint64_t dbk = db + static_cast<uint64_t>((kk * b_step) >> 4);
                         if constexpr (kPair)
-                            tc_mma_f16_pair(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32),
-                                            idesc, (kb | kk) != 0);
+                            tc_mma_f16_pair(d_tmem, dak, dbk, idesc, (kb | kk) != 0);
                         else
-                            tc_mma_f16(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
-                                       (kb | kk) != 0);
+                            tc_mma_f16(d_tmem, dak, dbk, idesc, (kb | kk) != 0);
                     }
                     if constexpr (kPair) tc_commit_pair(&empty[stage], 0x3);
                     else tc_commit(&empty[stage]);
@@ -1026,7 +1055,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                     if (lane == 0) bulk_wait_read<0>();      // the previous chunk's stores have read the blocks
                     __syncwarp();
                     write_row_block(packed, ebuf, lane);
-                    write_transposed_block(x, reinterpret_cast<uint32_t*>(ebuf + EPI_BLOCK_BYTES), lane);
+                    const bool with_t = p.no_ct == 0;
+                    if (with_t) write_transposed_block(x, reinterpret_cast<uint32_t*>(ebuf + EPI_BLOCK_BYTES), lane);
                     bool with_h = false;
                     if constexpr (kEpi == EPI_BWD_H) {
                         with_h = p.store_h != 0;
@@ -1041,11 +1071,11 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                     __syncwarp();
                     // a block wholly past M is not stored; a blocked transposed copy is
                     // stored up to the next multiple of 64 (its zero columns)
-                    const int m_end_t = p.ct_kb64 ? (p.M + 63) / 64 * 64 : p.M;
+                    const int m_end_t = (with_t && p.ct_kb64) ? (p.M + 63) / 64 * 64 : p.M;
                     if (lane == 0 && m_row0 < m_end_t) {
                         if (m_row0 < p.M) tma_store_2d(&tmC, ebuf, n0, m_row0);
-                        if (p.ct_kb64) tma_store_3d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0 & 63, n0, m_row0 >> 6);
-                        else tma_store_2d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0, n0);
+                        if (with_t && p.ct_kb64) tma_store_3d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0 & 63, n0, m_row0 >> 6);
+                        else if (with_t) tma_store_2d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0, n0);
                         if (with_h && m_row0 < p.M) tma_store_2d(&tmC2, ebuf + 2 * EPI_BLOCK_BYTES, n0, m_row0);
                         bulk_commit_group();
                     }

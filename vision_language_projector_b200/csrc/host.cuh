@@ -120,6 +120,24 @@ inline int encode_bf16_kb64(CUtensorMap* map, const void* base, uint64_t rows, u
     return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
 }
 
+// Map of a row-major bf16 matrix [rows][cols] (cols a multiple of 64) read as the
+// MN-major operand of a GEMM whose K runs over its rows: seen as 3D (c % 64, r, c / 64),
+// a box (64, 64, strips) holds 64 rows of `strips` 64-column strips, each strip 8 KB
+// contiguous in shared memory with the 128-byte swizzle (the canonical MN-major layout).
+// Rows past `rows` read as zeros.
+inline int encode_bf16_mn(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t strips) {
+    auto fn = driver().tiled;
+    if (!fn || cols % 64) return VLPROJ_ERR_CUDA;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(vlp::BK), strips};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+}
+
 // im2col map of n views of one (h, w) grid of C-channel bf16 patches, packed back to
 // back from `base`: the k x k, stride-k window walk of the merge. Base positions run
 // over 0, k, ..., k*(w'-1) (lower corner 0, upper corner k*w' - w - (k-1), the
@@ -504,9 +522,10 @@ struct vlproj_handle {
     CUtensorMap tmW2t{}, tmW2th{}, tmW1pt{}, tmW1pth{};
     std::vector<__nv_bfloat16*> Wmt;     // middle layers transposed, [N1][N1] each
     std::vector<CUtensorMap> tmWmt, tmWmth;
-    // G, H^T: one [M][N1] / [N1][ldt] slab per hidden layer; Hr: H row-major for the
-    // hidden layers that feed another one; dP, dP^T: two slabs, layer by layer
-    vlp_host::DevBuf<__nv_bfloat16> G, Ht, Hr, dY, dYt, dP, dPt, At;
+    // G, Hr: GELU'(P) and H, one [M][N1] slab each per hidden layer; dP: two slabs, layer
+    // by layer; dY [M][N2]; At: A^T blocked by 64 tokens (dW1's B operand)
+    vlp_host::DevBuf<__nv_bfloat16> G, Hr, dY, dP, At;
+    vlp_host::DevBuf<float> part_cs;     // column-sum partials of the bias gradients
     vlp_host::DevBuf<__nv_bfloat16> dA;
     vlp_host::DevBuf<float> part, part_sp;
     // host-memory entry point: copy streams, per-slot events and double-buffered staging

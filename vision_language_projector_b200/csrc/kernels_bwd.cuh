@@ -107,6 +107,33 @@ static __global__ void __launch_bounds__(256) vlp_rowsum_kernel(const __nv_bfloa
     if (lane == 0) out[n] = s;
 }
 
+// Column sums of a row-major bf16 matrix [M][N] (N even), first pass: partial[b][n] is
+// the sum of column n over rows [b CSR_ROWS, (b + 1) CSR_ROWS), in row order. A thread
+// takes two adjacent columns (one 4-byte load per row), so a warp reads 128 contiguous
+// bytes of each row; vlp_colsum_kernel then adds the row blocks in order (bias gradients:
+// db2 over dY, db1 and the middle layers' db over dP).
+constexpr int CSR_ROWS = 1024;
+constexpr int CSR_THREADS = 128;
+static __global__ void __launch_bounds__(CSR_THREADS) vlp_colsum_rows_kernel(const __nv_bfloat16* __restrict__ X,
+                                                                             int64_t M, int N,
+                                                                             float* __restrict__ partial) {
+    const int n = 2 * (blockIdx.x * CSR_THREADS + threadIdx.x);
+    if (n >= N) return;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * CSR_ROWS;
+    const int64_t m1 = m0 + CSR_ROWS < M ? m0 + CSR_ROWS : M;
+    const uint32_t* col = reinterpret_cast<const uint32_t*>(X + n);
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+    for (int64_t m = m0; m < m1; ++m) {
+        const uint32_t w = __ldg(col + m * (N / 2));
+        s0 += __uint_as_float(w << 16);
+        s1 += __uint_as_float(w & 0xFFFF0000u);
+    }
+    float* row = partial + static_cast<int64_t>(blockIdx.y) * N;
+    row[n] = s0;
+    row[n + 1] = s1;
+}
+
 template <bool kF32In>
 __device__ __forceinline__ void load8_feat(const void* x, int64_t row, int C, int v, float (&f)[8]) {
     if (kF32In) {

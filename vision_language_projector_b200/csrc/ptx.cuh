@@ -418,6 +418,26 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major operand with the 128-byte swizzle:
+// 64-element strips along M (or N), 8 K-rows of 128 bytes each per 1 KB atom. Atoms
+// follow each other along K every 1 KB (stride byte offset) and the strips along M (or
+// N) every 8 KB (leading byte offset): the layout a TMA box (64, 64 rows, strips) of a
+// row-major [K][M] matrix leaves in shared memory. The k-th 16-deep slice of K starts
+// 2 KB further.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFF) >> 4);       // start address, bits 0-13
+    d |= static_cast<uint64_t>(8192 >> 4) << 16;              // leading byte offset, bits 16-29
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;              // stride byte offset, bits 32-45
+    d |= static_cast<uint64_t>(1) << 46;                      // version, bits 46-47
+    d |= static_cast<uint64_t>(2) << 61;                      // layout type, bits 61-63
+    return d;
+}
+
+// Instruction descriptor bits that mark A (bit 15) or B (bit 16) as MN-major.
+constexpr uint32_t IDESC_A_MN = 1u << 15;
+constexpr uint32_t IDESC_B_MN = 1u << 16;
+
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
 // K-major, dense, shape M x N (M = 128 here).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {

@@ -5,14 +5,13 @@
 //                                     token's destination row and gather data
 //    7  LayerNorm-merge               A [M][k*k*C] bf16, position-outer: the forward's
 //                                     bf16 A operand
-//    8  GEMM1 recompute               P = A W1p^T + b1 -> G = GELU'(P) [M][N1] and
-//                                     H^T = GELU(P)^T [N1][M] (bf16), for every hidden
-//                                     layer (H itself too where a middle layer reads it)
-//    9  dY gather                     dY [M][N2] and dY^T [N2][M] from d_out's
-//                                     placeholder rows (zeros if the count check failed)
-//   10  dH GEMMs                      dP = (dY W2) * G -> dP [M][N1] and dP^T [N1][M], and
-//                                     with depth > 2 down through the middle layers, with
-//                                     their weight gradients dW_mid = dP^T H (K = M)
+//    8  GEMM1 recompute               P = A W1p^T + b1 -> G = GELU'(P) and H = GELU(P),
+//                                     [M][N1] bf16 each, for every hidden layer
+//    9  dY gather                     dY [M][N2] from d_out's placeholder rows (zeros if
+//                                     the count check failed)
+//   10  dH GEMMs                      dP = (dY W2) * G -> dP [M][N1], and with depth > 2
+//                                     down through the middle layers, with their weight
+//                                     gradients dW_mid = dP^T H (K = M)
 //   11  dW2 GEMM                      dW2 = dY^T H, K = M
 //   12  A^T + dW1 GEMM                A^T with rows in the caller's column order, then
 //                                     dW1 = dP^T A, K = M
@@ -20,12 +19,13 @@
 //                                     folded straight onto the patches in fp32: d_features)
 //   14  tails                         LayerNorm backward -> d_features and gamma / beta
 //                                     partials, column sums -> dgamma, dbeta; newline /
-//                                     separator gradients (db2, db1: row sums of dY^T and
-//                                     dP^T, beside stages 11 and 12)
-// Every contraction runs on the tcgen05 GEMM kernel with a K-major A and B from tensor
-// maps: the weight gradients take the transposed copies (K = M contiguous), which the
-// producing epilogues and the gather kernel write directly. W2^T and W1p^T are made
-// once, on the first call. For batches up to about 2^28 hidden activations, stages
+//                                     separator gradients (db2, db1: column sums of dY and
+//                                     dP, beside stages 11 and 12)
+// Every contraction runs on the tcgen05 GEMM kernel with operands from tensor maps. The
+// weight gradients (K = M, the tokens) read dY, H and dP where they lie, row-major, as
+// MN-major operands; only A^T is copied, since dW1's columns come back in the caller's
+// channel order. The bias gradients are column sums of dY and dP over the tokens. W2^T
+// and W1p^T are made once, on the first call. For batches up to about 2^28 hidden activations, stages
 // 11-12 and the bias sums run on the handle's side stream, forked after stage 9 and
 // joined before the call returns.
 #include "host.cuh"
@@ -42,6 +42,13 @@ int encode_b(CUtensorMap* full, CUtensorMap* half, const void* base, uint64_t ro
              uint64_t ld = 0) {
     if (encode_bf16_2d(full, base, rows, cols, static_cast<uint32_t>(bn), ld)) return VLPROJ_ERR_CUDA;
     return encode_bf16_2d(half, base, rows, cols, 128, ld);
+}
+
+// A B operand read MN-major from a row-major [K][N] matrix: boxes of BN / 64 strips
+// (single CTAs) and of 2 strips (each CTA of a pair holds 128 of the tile's N).
+int encode_b_mn(CUtensorMap* full, CUtensorMap* half, const void* base, uint64_t rows, uint64_t cols, int bn) {
+    if (encode_bf16_mn(full, base, rows, cols, static_cast<uint32_t>(bn / 64))) return VLPROJ_ERR_CUDA;
+    return encode_bf16_mn(half, base, rows, cols, 2);
 }
 
 // The same for a B operand stored blocked by 64 columns (the transposed activations and
@@ -157,10 +164,12 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     const int kk = c.k * c.k;
     const int K1 = h->K1;
     const int64_t M = pl.M;          // no padding in this plan: M merged tokens
-    // row stride of the transposed copies: whole 128-byte lines, so every TMA box row
-    // of the weight-gradient GEMMs starts on a line
+    // tokens of A^T (blocked by 64 tokens, zeros past M): whole 128-byte lines, so every
+    // TMA box row of the dW1 GEMM starts on a line
     const int64_t ldt = round_up(std::max<int64_t>(M, 1), 64);
-    const size_t hslab = static_cast<size_t>(M) * c.N1, tslab = static_cast<size_t>(c.N1) * ldt;
+    const size_t hslab = static_cast<size_t>(M) * c.N1;
+    // bias gradients: column sums over the tokens, in blocks of CSR_ROWS rows
+    const int64_t nb_cs = (M + vlp::CSR_ROWS - 1) / vlp::CSR_ROWS;
 
     // which dP are needed: Linear l's gradients need dP_l; dP_l needs every dP above it
     const bool want_l1 = a->d_W1 || a->d_b1 || a->d_features || a->d_gamma || a->d_beta;
@@ -169,17 +178,16 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     for (int i = n_mid - 1; i >= 0; --i)
         if (mid_w(i) || mid_b(i)) l_min = i + 2;
     if (want_l1) l_min = 1;
-    const bool want_recompute = l_min < depth || a->d_W2;     // G feeds dP, H^T feeds the weight gradients
+    const bool want_recompute = l_min < depth || a->d_W2;     // G feeds dP, H the weight gradients
 
     // scratch
     const int nblocks = vlp::scan_blocks(n_ids);
     if (h->counts.ensure(nblocks + 1) || h->pos.ensure(std::max<int64_t>(pl.R, 1))) return VLPROJ_ERR_CUDA;
     if (M > 0) {
         if (h->rowdest.ensure(M) || h->gmeta.ensure(M) || h->A.ensure(static_cast<size_t>(M) * K1) ||
-            h->G.ensure(hslab * (depth - 1)) || h->Ht.ensure(tslab * (depth - 1)) ||
-            (depth > 2 && h->Hr.ensure(hslab * (depth - 2))) ||
-            h->dY.ensure(static_cast<size_t>(M) * c.N2) || h->dYt.ensure(static_cast<size_t>(c.N2) * ldt) ||
-            h->dP.ensure(hslab * 2) || h->dPt.ensure(tslab * 2))
+            h->G.ensure(hslab * (depth - 1)) || h->Hr.ensure(hslab * (depth - 1)) ||
+            h->dY.ensure(static_cast<size_t>(M) * c.N2) || h->dP.ensure(hslab * 2) ||
+            h->part_cs.ensure(static_cast<size_t>(nb_cs) * (c.N2 + 2 * c.N1)))
             return VLPROJ_ERR_CUDA;
         if (a->d_W1 && h->At.ensure(static_cast<size_t>(K1) * ldt)) return VLPROJ_ERR_CUDA;
         if (want_da && c.has_ln && h->dA.ensure(static_cast<size_t>(M) * K1)) return VLPROJ_ERR_CUDA;
@@ -187,7 +195,22 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         if (rc) return rc;
     }
     __nv_bfloat16* const G = h->G.ptr;
-    __nv_bfloat16* const Ht = h->Ht.ptr;
+    __nv_bfloat16* const Hr = h->Hr.ptr;
+    // deterministic column sums of a row-major [M][N] bf16 matrix into out[N] (fp32):
+    // row-block partials, then the blocks added in order; each call site has its own
+    // partials region (the side stream's and the caller's sums may overlap in time)
+    auto bias_sums = [&](const __nv_bfloat16* X, int N, float* out, float* part, cudaStream_t st) -> int {
+        h->launches += 2;
+        vlp::vlp_colsum_rows_kernel<<<dim3(static_cast<unsigned>((N / 2 + vlp::CSR_THREADS - 1) / vlp::CSR_THREADS),
+                                           static_cast<unsigned>(nb_cs)),
+                                      vlp::CSR_THREADS, 0, st>>>(X, M, N, part);
+        vlp::vlp_colsum_kernel<<<(N + vlp::CS_COLS - 1) / vlp::CS_COLS, vlp::CS_COLS * vlp::CS_GROUPS, 0, st>>>(
+            part, static_cast<int>(nb_cs), N / 2, out, out + N / 2);
+        return cudaGetLastError() == cudaSuccess ? VLPROJ_OK : VLPROJ_ERR_CUDA;
+    };
+    float* const part_b2 = h->part_cs.ptr;
+    float* const part_b1 = part_b2 + nb_cs * c.N2;
+    float* const part_mid = part_b1 + nb_cs * c.N1;
     rc = upload_plan(h, pl, s);
     if (rc) return rc;
     h->profiled_valid = false;
@@ -224,40 +247,37 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         if (rc) return rc;
         stage_end(h, 7, s);
 
-        // 8. every hidden layer recomputed: G_l = GELU'(P_l), H_l^T, and H_l itself when a
-        //    middle layer reads it
+        // 8. every hidden layer recomputed: G_l = GELU'(P_l) and H_l, both row-major (the
+        //    weight-gradient GEMMs read H_l as an MN-major operand)
         stage_begin(h, 8, s);
         for (int l = 1; l <= depth - 1; ++l) {
             const bool first = l == 1;
-            const __nv_bfloat16* x = first ? h->A.ptr : h->Hr.ptr + (l - 2) * hslab;
+            const __nv_bfloat16* x = first ? h->A.ptr : Hr + (l - 2) * hslab;
             const int K = first ? K1 : c.N1;
             if (encode_bf16_2d(&tmA, x, M, K, vlp::BM)) return VLPROJ_ERR_CUDA;
             p = gemm_params(h, M, c.N1, K);
             p.bias = first ? h->b1 : h->bm[l - 2];
-            CUtensorMap tmG{}, tmHt{}, tmHr{};
+            CUtensorMap tmG{}, tmHr{};
             if (encode_bf16_store(&tmG, G + (l - 1) * hslab, M, c.N1) ||
-                encode_bf16_kb64(&tmHt, Ht + (l - 1) * tslab, c.N1, ldt, 0, true))
+                encode_bf16_store(&tmHr, Hr + (l - 1) * hslab, M, c.N1))
                 return VLPROJ_ERR_CUDA;
-            p.ct_kb64 = 1;
-            if (l < depth - 1) {
-                p.store_h = 1;
-                if (encode_bf16_store(&tmHr, h->Hr.ptr + (l - 1) * hslab, M, c.N1)) return VLPROJ_ERR_CUDA;
-            }
+            p.store_h = 1;
+            p.no_ct = 1;
             ++h->launches;
             rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(h, pick_bn(c.N1), h->pairs, tmA,
                                                              first ? h->tmW1 : h->tmWm[l - 2],
                                                              first ? h->tmW1h : h->tmWmh[l - 2], p, s,
-                                                             tmG, tmHt, tmHr);
+                                                             tmG, no_map(), tmHr);
             if (rc) return rc;
         }
         stage_end(h, 8, s);
     }
 
-    // 9. dY and dY^T from the placeholder rows of d_out
+    // 9. dY from the placeholder rows of d_out
     stage_begin(h, 9, s);
     ++h->launches;
     transpose_launch(static_cast<const __nv_bfloat16*>(a->d_out), c.N2, n_ids, h->rowdest.ptr, h->status + 1, M,
-                     c.N2, h->dY.ptr, h->dYt.ptr, ldt, c.C, 1, 0, s, 1);
+                     c.N2, h->dY.ptr, nullptr, ldt, c.C, 1, 0, s, 1);
     VLP_CUDA(cudaGetLastError());
     stage_end(h, 9, s);
 
@@ -273,14 +293,20 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     VLP_CUDA(cudaEventRecord(h->fork, s));
     VLP_CUDA(cudaStreamWaitEvent(ss, h->fork, 0));
 
-    // 11. top layer: dW2 = dY^T H_(depth-1) and db2 (side stream)
+    // 11. top layer: dW2 = dY^T H_(depth-1) and db2 (side stream); dY and H are read
+    //     where they lie, as MN-major operands
     CUtensorMap tmA2{}, tmB2{}, tmB2h{};
     if (a->d_W2) {
-        if (encode_bf16_kb64(&tmA2, h->dYt.ptr, c.N2, ldt, vlp::BM) ||
-            encode_b_kb64(&tmB2, &tmB2h, Ht + (depth - 2) * tslab, c.N1, ldt, pick_bn(c.N1)))
+        // N2 need only be a multiple of 32: then dY's 64-column strips come by separate 2D
+        // boxes, so the last strip's columns past N2 read as zeros
+        const bool strips = c.N2 % 64 != 0;
+        const int rc_a = strips ? encode_bf16_2d(&tmA2, h->dY.ptr, M, c.N2, 64)
+                                : encode_bf16_mn(&tmA2, h->dY.ptr, M, c.N2, vlp::BM / 64);
+        if (rc_a || encode_b_mn(&tmB2, &tmB2h, Hr + (depth - 2) * hslab, M, c.N1, pick_bn(c.N1)))
             return VLPROJ_ERR_CUDA;
         GemmParams q = gemm_params(h, c.N2, c.N1, M);
-        q.a_kb64 = q.b_kb64 = 1;
+        q.a_mn = strips ? 2 : 1;
+        q.b_mn = 1;
         q.outf = a->d_W2;
         stage_begin(h, 11, ss);
         ++h->launches;
@@ -289,9 +315,8 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         stage_end(h, 11, ss);
     }
     if (a->d_b2) {
-        ++h->launches;
-        vlp::vlp_rowsum_kernel<<<(c.N2 + 7) / 8, 256, 0, ss>>>(h->dYt.ptr, ldt, c.N2, M, a->d_b2, 1);
-        VLP_CUDA(cudaGetLastError());
+        rc = bias_sums(h->dY.ptr, c.N2, a->d_b2, part_b2, ss);
+        if (rc) return rc;
     }
 
     // 10. the dP chain (caller's stream): dP_l = (dP_(l+1) W_(l+1)) * G_l from the top
@@ -308,16 +333,13 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
                 return VLPROJ_ERR_CUDA;
             p = gemm_params(h, M, c.N1, top ? c.N2 : c.N1);
             p.aux = G + (l - 1) * hslab;
-            CUtensorMap tmP{}, tmPt{};
-            if (encode_bf16_store(&tmP, h->dP.ptr + nxt * hslab, M, c.N1) ||
-                encode_bf16_kb64(&tmPt, h->dPt.ptr + nxt * tslab, c.N1, ldt, 0, true))
-                return VLPROJ_ERR_CUDA;
-            p.ct_kb64 = 1;
+            CUtensorMap tmP{};
+            if (encode_bf16_store(&tmP, h->dP.ptr + nxt * hslab, M, c.N1)) return VLPROJ_ERR_CUDA;
+            p.no_ct = 1;
             ++h->launches;
             rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(h, pick_bn(c.N1), h->pairs, tmA,
                                                              top ? h->tmW2t : h->tmWmt[l - 1],
-                                                             top ? h->tmW2th : h->tmWmth[l - 1], p, s,
-                                                             tmP, tmPt);
+                                                             top ? h->tmW2th : h->tmWmth[l - 1], p, s, tmP);
             if (rc) return rc;
             cur = nxt;
             if (l < 2) continue;
@@ -325,21 +347,19 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             const int i = l - 2;
             if (mid_w(i)) {
                 CUtensorMap ta{}, tb{}, tbh{};
-                if (encode_bf16_kb64(&ta, h->dPt.ptr + cur * tslab, c.N1, ldt, vlp::BM) ||
-                    encode_b_kb64(&tb, &tbh, Ht + (l - 2) * tslab, c.N1, ldt, pick_bn(c.N1)))
+                if (encode_bf16_mn(&ta, h->dP.ptr + cur * hslab, M, c.N1, vlp::BM / 64) ||
+                    encode_b_mn(&tb, &tbh, Hr + (l - 2) * hslab, M, c.N1, pick_bn(c.N1)))
                     return VLPROJ_ERR_CUDA;
                 GemmParams q = gemm_params(h, c.N1, c.N1, M);
-                q.a_kb64 = q.b_kb64 = 1;
+                q.a_mn = q.b_mn = 1;
                 q.outf = mid_w(i);
                 ++h->launches;
                 rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(h, pick_bn(c.N1), h->pairs, ta, tb, tbh, q, s);
                 if (rc) return rc;
             }
             if (mid_b(i)) {
-                ++h->launches;
-                vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, s>>>(h->dPt.ptr + cur * tslab, ldt, c.N1, M,
-                                                                      mid_b(i), 1);
-                VLP_CUDA(cudaGetLastError());
+                rc = bias_sums(h->dP.ptr + cur * hslab, c.N1, mid_b(i), part_mid, s);
+                if (rc) return rc;
             }
         }
         stage_end(h, 10, s);
@@ -347,7 +367,6 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     }
     // dP_1, when the chain reached it (l_min == 1)
     const __nv_bfloat16* dP1 = h->dP.ptr + cur * hslab;
-    const __nv_bfloat16* dP1t = h->dPt.ptr + cur * tslab;
 
     // 12a. A^T in the caller's column order (side stream)
     if (a->d_W1) {
@@ -361,11 +380,12 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     // 12b. dW1 = dP_1^T A and db1 (side stream, after dP_1)
     if (want_l1) VLP_CUDA(cudaStreamWaitEvent(ss, h->join2, 0));
     if (a->d_W1) {
-        if (encode_bf16_kb64(&tmA2, dP1t, c.N1, ldt, vlp::BM) ||
+        if (encode_bf16_mn(&tmA2, dP1, M, c.N1, vlp::BM / 64) ||
             encode_b_kb64(&tmB2, &tmB2h, h->At.ptr, K1, ldt, pick_bn(K1)))
             return VLPROJ_ERR_CUDA;
         GemmParams q = gemm_params(h, c.N1, K1, M);
-        q.a_kb64 = q.b_kb64 = 1;
+        q.a_mn = 1;
+        q.b_kb64 = 1;
         q.outf = a->d_W1;
         ++h->launches;
         rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(h, pick_bn(K1), h->pairs, tmA2, tmB2, tmB2h, q, ss);
@@ -373,9 +393,8 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
         stage_end(h, 12, ss);
     }
     if (a->d_b1) {
-        ++h->launches;
-        vlp::vlp_rowsum_kernel<<<(c.N1 + 7) / 8, 256, 0, ss>>>(dP1t, ldt, c.N1, M, a->d_b1, 1);
-        VLP_CUDA(cudaGetLastError());
+        rc = bias_sums(dP1, c.N1, a->d_b1, part_b1, ss);
+        if (rc) return rc;
     }
     VLP_CUDA(cudaEventRecord(h->join, ss));
 
