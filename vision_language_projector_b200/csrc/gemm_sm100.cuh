@@ -84,12 +84,12 @@ constexpr int ERR_TIMEOUT = -5;
 // its 128 rows of A and half of the BN rows of B per stage, so a stage is 32 KB and
 // six stages fit.
 // Epilogues that send bf16 tiles out by TMA store stage them here, per epilogue warp in
-// 32 x 32 bf16 blocks: GELU two (two chunks in flight), DGELU two (a chunk of dP and of
-// dP^T), BWD_H three (G, H^T and, for a following layer, H). SCATTER stages 32 rows x 64
-// columns (the two blocks side by side) so that its stores write whole row segments.
+// 32 x 32 bf16 blocks: GELU two (two chunks in flight), DGELU one (a chunk of dP), BWD_H
+// two (a chunk of G and of H). SCATTER stages 32 rows x 64 columns (the two blocks side
+// by side) so that its stores write whole row segments.
 constexpr int EPI_BLOCK_BYTES = 32 * 32 * 2;
 __host__ __device__ constexpr int epi_blocks(int epi) {
-    return epi == EPI_BWD_H ? 3 : (epi == EPI_GELU || epi == EPI_DGELU || epi == EPI_BF16 || epi == EPI_SCATTER) ? 2 : 0;
+    return epi == EPI_DGELU ? 1 : (epi == EPI_GELU || epi == EPI_BWD_H || epi == EPI_BF16 || epi == EPI_SCATTER) ? 2 : 0;
 }
 __host__ __device__ constexpr int epi_stage_bytes(int epi) { return 4 * epi_blocks(epi) * EPI_BLOCK_BYTES; }
 
@@ -175,23 +175,19 @@ struct GemmParams {
     int64_t out_rows;               // rows of `out` (bounds guard)
     const int* fwd_status;          // nonzero = count check failed, write nothing (null = ignore)
     int tma_store;                  // EPI_GELU: rows are stored by TMA through tmC (identity rows)
-    int store_h;                    // EPI_BWD_H: also store H row-major through tmC2
-    // backward epilogues (outputs through tmC, and tmCt for the transposed copy)
+    // backward epilogues (outputs through tmC, and H through tmC2 in EPI_BWD_H)
     const __nv_bfloat16* aux;       // EPI_DGELU: G = GELU'(P) [M][N] bf16
     float* outf;                    // EPI_F32: [M][N] fp32; EPI_FOLD_F32: [patches][C] fp32
-    // operands / transposed outputs stored blocked by 64 along K (the token axis of the
-    // weight gradients): element (row r, column m) of an R-row matrix at ((m / 64) * R + r)
-    // * 64 + m % 64, so a tile's K-block is one contiguous run (3D tensor maps: (m % 64, r,
-    // m / 64)). ct_kb64: the epilogue's transposed copy (tmCt) is stored so, with the
-    // columns from M up to the next multiple of 64 written as zeros.
-    int a_kb64, b_kb64, ct_kb64;
+    // operands stored blocked by 64 along K (the token axis of the weight gradients):
+    // element (row r, column m) of an R-row matrix at ((m / 64) * R + r) * 64 + m % 64, so
+    // a tile's K-block is one contiguous run (3D tensor maps: (m % 64, r, m / 64)).
+    int a_kb64, b_kb64;
     // a_mn / b_mn: the operand is MN-major, read from a row-major [K][M] (or [K][N]) matrix
     // through a 3D map (m % 64, k, m / 64) in boxes of 64 K-rows x (rows / 64) strips (the
     // weight gradients, K = tokens, read dY, H and dP where they lie); a_mn = 2: the same
     // strips by one 2D box (64 columns x 64 K-rows) each, for a matrix whose width is not a
-    // multiple of 64 (columns past it read as zeros). no_ct: the BWD_H and DGELU epilogues
-    // write no transposed copy.
-    int a_mn, b_mn, no_ct;
+    // multiple of 64 (columns past it read as zeros).
+    int a_mn, b_mn;
     int group_n;                    // N-blocks per raster band (see tile_coords); 0 = from l2_budget
     int64_t l2_budget;              // host only: bytes of B one raster band may hold (0 = 64 MB)
     // Dynamic tile order: [0] the next tile index, [1] units that have finished taking
@@ -340,23 +336,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// The warp's 32 rows (lane = row m) x 32 columns (x[j] = column n0 + j) written
-// transposed into a 32 x 32 bf16 block in shared memory, row j = column n0 + j, element
-// m = lane. Lanes 2i and 2i+1 trade one value per column pair, so each lane writes two
-// consecutive m of one column as one 4-byte word, and the 32 words an instruction writes
-// fall in 32 different banks.
-__device__ __forceinline__ void write_transposed_block(const float (&x)[32], uint32_t* words, int lane) {
-    const bool odd = (lane & 1) != 0;
-#pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-        const float give = odd ? x[j] : x[j + 1];
-        const float got = __shfl_xor_sync(0xffffffffu, give, 1);
-        const float lo = odd ? got : x[j];          // element m_even
-        const float hi = odd ? x[j + 1] : got;      // element m_even + 1
-        words[(j + (odd ? 1 : 0)) * 16 + (lane >> 1)] = pack_bf16x2(lo, hi);
-    }
-}
-
 // Row-major 32 x 32 bf16 block in shared memory: the lane's row, 16 packed words.
 __device__ __forceinline__ void write_row_block(const uint32_t (&packed)[16], uint8_t* block, int lane) {
     uint4* r4 = reinterpret_cast<uint4*>(block + lane * 64);
@@ -368,8 +347,8 @@ __device__ __forceinline__ void write_row_block(const uint32_t (&packed)[16], ui
 template <int BN, int kAMode, int kEpi, int kCtas>
 __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     vlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmCt,
-                    const __grid_constant__ CUtensorMap tmC2, const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
+                    const GemmParams p) {
     using L = GemmLayout<BN, kCtas, epi_stage_bytes(kEpi), a_aux_bytes(kAMode)>;
     constexpr int S = L::STAGES;
     constexpr bool kPair = kCtas == 2;
@@ -1015,22 +994,23 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
                     }
                 } else if constexpr (kEpi == EPI_BWD_H || kEpi == EPI_DGELU) {
-                    float x[32];
+                    // BWD_H: G = GELU'(P) through tmC and H = GELU(P) through tmC2; DGELU: dP =
+                    // (accumulator) * G through tmC. Row-major 32 x 32 blocks through shared
+                    // memory and TMA stores (rows and columns past the tensors are not written).
                     uint32_t packed[16];
+                    uint32_t hp[16];
                     if constexpr (kEpi == EPI_BWD_H) {
                         float bb[32];
                         load_bias32(p.bias, n0, bb);
 #pragma unroll
                         for (int j = 0; j < 32; j += 2) {
-                            const float p0 = __uint_as_float(v[j]) + bb[j];
-                            const float p1 = __uint_as_float(v[j + 1]) + bb[j + 1];
+                            float x0 = __uint_as_float(v[j]) + bb[j];
+                            float x1 = __uint_as_float(v[j + 1]) + bb[j + 1];
                             float g0, g1;
-                            gelu_grad2(p0, p1, g0, g1);
+                            gelu_grad2(x0, x1, g0, g1);
                             packed[j / 2] = pack_bf16x2(g0, g1);
-                            x[j] = p0;
-                            x[j + 1] = p1;
-                            gelu2(x[j], x[j + 1]);
-                            if (m >= p.M) x[j] = x[j + 1] = 0.0f;   // H^T columns past M are zero
+                            gelu2(x0, x1);
+                            hp[j / 2] = pack_bf16x2(x0, x1);
                         }
                     } else {
                         uint4 g4[4] = {};
@@ -1041,42 +1021,19 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                         }
                         const uint32_t* gw = reinterpret_cast<const uint32_t*>(g4);
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            x[j] = __uint_as_float(v[j]) * __uint_as_float(gw[j / 2] << 16);
-                            x[j + 1] = __uint_as_float(v[j + 1]) * __uint_as_float(gw[j / 2] & 0xFFFF0000u);
-                            packed[j / 2] = pack_bf16x2(x[j], x[j + 1]);
-                            // the transposed copy holds the same bf16 values as the row-major one
-                            x[j] = __uint_as_float(packed[j / 2] << 16);
-                            x[j + 1] = __uint_as_float(packed[j / 2] & 0xFFFF0000u);
-                        }
+                        for (int j = 0; j < 32; j += 2)
+                            packed[j / 2] = pack_bf16x2(__uint_as_float(v[j]) * __uint_as_float(gw[j / 2] << 16),
+                                                        __uint_as_float(v[j + 1]) * __uint_as_float(gw[j / 2] & 0xFFFF0000u));
                     }
-                    // both copies leave through shared memory and TMA stores (rows and
-                    // columns past the tensors are not written)
                     if (lane == 0) bulk_wait_read<0>();      // the previous chunk's stores have read the blocks
                     __syncwarp();
                     write_row_block(packed, ebuf, lane);
-                    const bool with_t = p.no_ct == 0;
-                    if (with_t) write_transposed_block(x, reinterpret_cast<uint32_t*>(ebuf + EPI_BLOCK_BYTES), lane);
-                    bool with_h = false;
-                    if constexpr (kEpi == EPI_BWD_H) {
-                        with_h = p.store_h != 0;
-                        if (with_h) {                        // H itself, the next layer's input
-                            uint32_t hp[16];
-#pragma unroll
-                            for (int j = 0; j < 32; j += 2) hp[j / 2] = pack_bf16x2(x[j], x[j + 1]);
-                            write_row_block(hp, ebuf + 2 * EPI_BLOCK_BYTES, lane);
-                        }
-                    }
+                    if constexpr (kEpi == EPI_BWD_H) write_row_block(hp, ebuf + EPI_BLOCK_BYTES, lane);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    // a block wholly past M is not stored; a blocked transposed copy is
-                    // stored up to the next multiple of 64 (its zero columns)
-                    const int m_end_t = (with_t && p.ct_kb64) ? (p.M + 63) / 64 * 64 : p.M;
-                    if (lane == 0 && m_row0 < m_end_t) {
-                        if (m_row0 < p.M) tma_store_2d(&tmC, ebuf, n0, m_row0);
-                        if (with_t && p.ct_kb64) tma_store_3d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0 & 63, n0, m_row0 >> 6);
-                        else if (with_t) tma_store_2d(&tmCt, ebuf + EPI_BLOCK_BYTES, m_row0, n0);
-                        if (with_h && m_row0 < p.M) tma_store_2d(&tmC2, ebuf + 2 * EPI_BLOCK_BYTES, n0, m_row0);
+                    if (lane == 0 && m_row0 < p.M) {         // a block wholly past M is not stored
+                        tma_store_2d(&tmC, ebuf, n0, m_row0);
+                        if constexpr (kEpi == EPI_BWD_H) tma_store_2d(&tmC2, ebuf + EPI_BLOCK_BYTES, n0, m_row0);
                         bulk_commit_group();
                     }
                 } else if constexpr (kEpi == EPI_SCATTER) {

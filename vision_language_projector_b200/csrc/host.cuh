@@ -101,21 +101,19 @@ inline int encode_bf16_store(CUtensorMap* map, const void* base, uint64_t rows, 
     return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
 }
 
-// Maps of a bf16 matrix of `rows` rows and `cols` (a multiple of 64) columns stored
+// Map of a bf16 matrix of `rows` rows and `cols` (a multiple of 64) columns stored
 // blocked by 64 columns: element (r, m) at ((m / 64) * rows + r) * 64 + m % 64. Seen as
 // 3D (m % 64, r, m / 64): a load box (64, box_rows, 1) is box_rows * 128 contiguous bytes,
-// 128-byte swizzle; a store box (32, 32, 1), no swizzle.
-inline int encode_bf16_kb64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
-                            bool store = false) {
+// 128-byte swizzle.
+inline int encode_bf16_kb64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     auto fn = driver().tiled;
     if (!fn || cols % 64) return VLPROJ_ERR_CUDA;
     cuuint64_t dims[3] = {64, rows, cols / 64};
     cuuint64_t strides[2] = {128, rows * 128};
-    cuuint32_t box[3] = {store ? 32u : 64u, store ? 32u : box_rows, 1};
+    cuuint32_t box[3] = {64u, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, store ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
-                    store ? CU_TENSOR_MAP_L2_PROMOTION_NONE : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
 }
@@ -416,8 +414,8 @@ inline int raster_group(int N, int K, int BN, int64_t budget = 0, int units = 74
 }
 
 template <int BN, int A, int E, int CTAS>
-int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tct,
-                const CUtensorMap& tc2, GemmParams p, int num_sms, cudaStream_t s) {
+int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tc2,
+                GemmParams p, int num_sms, cudaStream_t s) {
     using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E), vlp::a_aux_bytes(A)>;
     auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
     if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN, p.l2_budget, num_sms / CTAS);
@@ -450,7 +448,7 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
     cfg.gridDim = dim3(static_cast<unsigned>(units * CTAS));
     cfg.attrs = CTAS > 1 ? attr : nullptr;
     cfg.numAttrs = CTAS > 1 ? 1 : 0;
-    VLP_CUDA(cudaLaunchKernelEx(&cfg, kernel, ta, tb, tc, tct, tc2, p));
+    VLP_CUDA(cudaLaunchKernelEx(&cfg, kernel, ta, tb, tc, tc2, p));
     return VLPROJ_OK;
 }
 
@@ -538,7 +536,7 @@ struct vlproj_handle {
 namespace vlp_host {
 
 // Tile shape: 256 x 256 tiles on CTA pairs when N allows and the A operand comes by
-// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise. tc / tct / tc2: output
+// TMA; 128 x 256 (or x 128 for N < 256) on single CTAs otherwise. tc / tc2: output
 // maps of the TMA-store epilogues (unused by the others). A launch in the dynamic tile
 // order takes the handle's next tile queue.
 inline const CUtensorMap& no_map() {
@@ -549,7 +547,7 @@ inline const CUtensorMap& no_map() {
 template <int A, int E>
 int launch_gemm_bn(vlproj_handle* h, int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb,
                    const CUtensorMap& tb_half, GemmParams p, cudaStream_t s, const CUtensorMap& tc = no_map(),
-                   const CUtensorMap& tct = no_map(), const CUtensorMap& tc2 = no_map()) {
+                   const CUtensorMap& tc2 = no_map()) {
     const int num_sms = h->num_sms;
     const int ctas = (A != vlp::A_CPASYNC && pair && bn == 256) ? 2 : 1;
     const int64_t tiles = ((static_cast<int64_t>(p.M) + vlp::BM * ctas - 1) / (vlp::BM * ctas)) * ((p.N + bn - 1) / bn);
@@ -560,10 +558,10 @@ int launch_gemm_bn(vlproj_handle* h, int bn, bool pair, const CUtensorMap& ta, c
                        tiles * kblocks >= static_cast<int64_t>(kDynamicMinWaves) * 64 * (num_sms / ctas)));
     p.tile_queue = (dyn && h->tqueue) ? h->tqueue + 2 * (h->tq_next++ % kTileQueues) : nullptr;
     if constexpr (A != vlp::A_CPASYNC) {
-        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tct, tc2, p, num_sms, s);
+        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tc2, p, num_sms, s);
     }
-    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tct, tc2, p, num_sms, s);
-    return launch_gemm<128, A, E, 1>(ta, tb, tc, tct, tc2, p, num_sms, s);
+    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tc2, p, num_sms, s);
+    return launch_gemm<128, A, E, 1>(ta, tb, tc, tc2, p, num_sms, s);
 }
 
 // Stage timing: begin / end events on the stream that runs the stage.

@@ -83,30 +83,6 @@ static __global__ void __launch_bounds__(256) vlp_gather_transpose_kernel(
     }
 }
 
-// out[n] = sum over m < M of T(n, m) (bf16), accumulated in fp32: one warp per row, each
-// lane over every 32nd run of 8 elements, then a butterfly. T(n, m) = T[n * ld + m], or
-// with kb64 T[((m / 64) * N + n) * 64 + m % 64] (blocked by 64 columns). ld % 8 == 0.
-static __global__ void __launch_bounds__(256) vlp_rowsum_kernel(const __nv_bfloat16* __restrict__ T, int64_t ld, int N,
-                                                         int64_t M, float* __restrict__ out, int kb64) {
-    const int lane = threadIdx.x & 31;
-    const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (n >= N) return;
-    float s = 0.f;
-    for (int64_t m = 8 * lane; m < M; m += 256) {
-        const int64_t off = kb64 ? ((m >> 6) * N + n) * 64 + (m & 63) : static_cast<int64_t>(n) * ld + m;
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(T + off));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (m + 2 * e < M) s += __uint_as_float(w[e] << 16);
-            if (m + 2 * e + 1 < M) s += __uint_as_float(w[e] & 0xFFFF0000u);
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) out[n] = s;
-}
-
 // Column sums of a row-major bf16 matrix [M][N] (N even), first pass: partial[b][n] is
 // the sum of column n over rows [b CSR_ROWS, (b + 1) CSR_ROWS), in row order. A thread
 // takes two adjacent columns (one 4-byte load per row), so a warp reads 128 contiguous

@@ -261,13 +261,11 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             if (encode_bf16_store(&tmG, G + (l - 1) * hslab, M, c.N1) ||
                 encode_bf16_store(&tmHr, Hr + (l - 1) * hslab, M, c.N1))
                 return VLPROJ_ERR_CUDA;
-            p.store_h = 1;
-            p.no_ct = 1;
             ++h->launches;
             rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_BWD_H>(h, pick_bn(c.N1), h->pairs, tmA,
                                                              first ? h->tmW1 : h->tmWm[l - 2],
                                                              first ? h->tmW1h : h->tmWmh[l - 2], p, s,
-                                                             tmG, no_map(), tmHr);
+                                                             tmG, tmHr);
             if (rc) return rc;
         }
         stage_end(h, 8, s);
@@ -335,7 +333,6 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             p.aux = G + (l - 1) * hslab;
             CUtensorMap tmP{};
             if (encode_bf16_store(&tmP, h->dP.ptr + nxt * hslab, M, c.N1)) return VLPROJ_ERR_CUDA;
-            p.no_ct = 1;
             ++h->launches;
             rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_DGELU>(h, pick_bn(c.N1), h->pairs, tmA,
                                                              top ? h->tmW2t : h->tmWmt[l - 1],
