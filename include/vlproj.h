@@ -394,7 +394,7 @@ int vlproj_set_wait_limit(vlproj_handle* h, uint64_t ns);
  *             5 newline/separator rows;
  *   backward  6 placeholder index + geometry, 7 LayerNorm-merge (A), 8 GEMM1
  *             recompute (GELU' and H^T), 9 dY gather, 10 dH GEMM (dP), 11 dW2 GEMM,
- *             12 A^T + dW1 GEMM, 13 dA GEMM, 14 bias sums + LayerNorm backward +
+ *             12 dW1 GEMM + its column reorder, 13 dA GEMM, 14 bias sums + LayerNorm backward +
  *             newline/separator gradients.
  * Off by default; enabling adds two event records per stage that runs. */
 #define VLPROJ_NUM_STAGES 15

@@ -178,10 +178,6 @@ struct GemmParams {
     // backward epilogues (outputs through tmC, and H through tmC2 in EPI_BWD_H)
     const __nv_bfloat16* aux;       // EPI_DGELU: G = GELU'(P) [M][N] bf16
     float* outf;                    // EPI_F32: [M][N] fp32; EPI_FOLD_F32: [patches][C] fp32
-    // operands stored blocked by 64 along K (the token axis of the weight gradients):
-    // element (row r, column m) of an R-row matrix at ((m / 64) * R + r) * 64 + m % 64, so
-    // a tile's K-block is one contiguous run (3D tensor maps: (m % 64, r, m / 64)).
-    int a_kb64, b_kb64;
     // a_mn / b_mn: the operand is MN-major, read from a row-major [K][M] (or [K][N]) matrix
     // through a 3D map (m % 64, k, m / 64) in boxes of 64 K-rows x (rows / 64) strips (the
     // weight gradients, K = tokens, read dY, H and dP where they lie); a_mn = 2: the same
@@ -493,9 +489,9 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                     tma_load_2d_pair(sa + q * 8192, &tmA, bar, (a_row_tile * (BM / 64) + q) * 64, kb * BK);
                             } else if (p.a_mn) {
                                 tma_load_3d_pair(sa, &tmA, bar, 0, kb * BK, a_row_tile * (BM / 64));
+                            } else {
+                                tma_load_2d_pair(sa, &tmA, bar, kb * BK, a_row_tile * BM);
                             }
-                            else if (p.a_kb64) tma_load_3d_pair(sa, &tmA, bar, 0, a_row_tile * BM, kb);
-                            else tma_load_2d_pair(sa, &tmA, bar, kb * BK, a_row_tile * BM);
                         } else if (kAMode == A_BOX5) {
                             const int pos = kb / cblocks;
                             const int c0 = (kb - pos * cblocks) * BK;
@@ -512,7 +508,6 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                             }
                         }
                         if (p.b_mn) tma_load_3d_pair(sb, &tmB, bar, 0, kb * BK, b_row / 64);
-                        else if (p.b_kb64) tma_load_3d_pair(sb, &tmB, bar, 0, b_row, kb);
                         else tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
                     } else {
                         mbar_arrive_expect_tx(&full_tma[stage], expect);
@@ -523,9 +518,9 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                 kb * BK);
                             } else if (p.a_mn) {
                                 tma_load_3d(sa, &tmA, &full_tma[stage], 0, kb * BK, a_row_tile * (BM / 64));
+                            } else {
+                                tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, a_row_tile * BM);
                             }
-                            else if (p.a_kb64) tma_load_3d(sa, &tmA, &full_tma[stage], 0, a_row_tile * BM, kb);
-                            else tma_load_2d(sa, &tmA, &full_tma[stage], kb * BK, a_row_tile * BM);
                         } else if (kAMode == A_BOX5) {
                             const int pos = kb / cblocks;
                             const int c0 = (kb - pos * cblocks) * BK;
@@ -542,7 +537,6 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                             }
                         }
                         if (p.b_mn) tma_load_3d(sb, &tmB, &full_tma[stage], 0, kb * BK, b_row / 64);
-                        else if (p.b_kb64) tma_load_3d(sb, &tmB, &full_tma[stage], 0, b_row, kb);
                         else tma_load_2d(sb, &tmB, &full_tma[stage], kb * BK, b_row);
                     }
                     ++issued;

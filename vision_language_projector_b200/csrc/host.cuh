@@ -101,23 +101,6 @@ inline int encode_bf16_store(CUtensorMap* map, const void* base, uint64_t rows, 
     return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
 }
 
-// Map of a bf16 matrix of `rows` rows and `cols` (a multiple of 64) columns stored
-// blocked by 64 columns: element (r, m) at ((m / 64) * rows + r) * 64 + m % 64. Seen as
-// 3D (m % 64, r, m / 64): a load box (64, box_rows, 1) is box_rows * 128 contiguous bytes,
-// 128-byte swizzle.
-inline int encode_bf16_kb64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    auto fn = driver().tiled;
-    if (!fn || cols % 64) return VLPROJ_ERR_CUDA;
-    cuuint64_t dims[3] = {64, rows, cols / 64};
-    cuuint64_t strides[2] = {128, rows * 128};
-    cuuint32_t box[3] = {64u, box_rows, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? VLPROJ_OK : VLPROJ_ERR_CUDA;
-}
-
 // Map of a row-major bf16 matrix [rows][cols] (cols a multiple of 64) read as the
 // MN-major operand of a GEMM whose K runs over its rows: seen as 3D (c % 64, r, c / 64),
 // a box (64, 64, strips) holds 64 rows of `strips` 64-column strips, each strip 8 KB
@@ -521,8 +504,9 @@ struct vlproj_handle {
     std::vector<__nv_bfloat16*> Wmt;     // middle layers transposed, [N1][N1] each
     std::vector<CUtensorMap> tmWmt, tmWmth;
     // G, Hr: GELU'(P) and H, one [M][N1] slab each per hidden layer; dP: two slabs, layer
-    // by layer; dY [M][N2]; At: A^T blocked by 64 tokens (dW1's B operand)
-    vlp_host::DevBuf<__nv_bfloat16> G, Hr, dY, dP, At;
+    // by layer; dY [M][N2]; dW1p: dW1 in the kernel's K order before it is reordered
+    vlp_host::DevBuf<__nv_bfloat16> G, Hr, dY, dP;
+    vlp_host::DevBuf<float> dW1p;
     vlp_host::DevBuf<float> part_cs;     // column-sum partials of the bias gradients
     vlp_host::DevBuf<__nv_bfloat16> dA;
     vlp_host::DevBuf<float> part, part_sp;

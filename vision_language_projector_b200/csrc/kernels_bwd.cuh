@@ -1,8 +1,10 @@
 // Memory-bound kernels of the projector backward (sm_100a):
 //   gather-transpose   rows of a bf16 matrix, optionally picked through a row table,
 //                      copied row-major and / or transposed through shared memory
-//                      (dY and dY^T from the output gradient, A^T, transposed weights)
-//   row sums           bias gradients from the transposed gradient matrices
+//                      (dY from the output gradient, the transposed weights)
+//   column sums        bias gradients: row-block partials of dY and dP, then the
+//                      blocks added in order
+//   dW1 reorder        dW1's columns from the kernel's K order to the caller's
 //   LayerNorm backward input gradient per patch, gamma / beta partial sums per block
 //                      (without a LayerNorm the dA GEMM's epilogue writes the input
 //                      gradient itself)
@@ -26,16 +28,13 @@ constexpr int LNB_WARPS = 8;
 // reads zeros. Writes, for q < Q:
 //   dst[m * Q + q]           row-major copy (skipped when dst is null)
 //   dst_t[perm(q) * ldt + m] transposed copy (skipped when dst_t is null), where
-//                            perm(q) = c*kk + p for q = p*C + c when chan_outer, else q;
-//                            with kb64 stored blocked by 64 columns instead:
-//                            dst_t[((m / 64) * Q + perm(q)) * 64 + m % 64]
-// Columns M .. ceil(M/8)*8 - 1 of the transposed copy (.. ceil(M/64)*64 - 1 with kb64)
-// are written as zeros. Grid (ceil(Q/64), ceil(M/64)), 256 threads. Q, ld_src and ldt
-// are multiples of 8 (ldt of 64 with kb64).
+//                            perm(q) = c*kk + p for q = p*C + c when chan_outer, else q
+// Columns M .. ceil(M/8)*8 - 1 of the transposed copy are written as zeros. Grid
+// (ceil(Q/64), ceil(M/64)), 256 threads. Q, ld_src and ldt are multiples of 8.
 static __global__ void __launch_bounds__(256) vlp_gather_transpose_kernel(
     const __nv_bfloat16* __restrict__ src, int64_t ld_src, int64_t src_rows, const int32_t* __restrict__ rowsel,
     const int* __restrict__ zero_if, int M, int Q, __nv_bfloat16* __restrict__ dst, __nv_bfloat16* __restrict__ dst_t,
-    int64_t ldt, int C, int kk, int chan_outer, int kb64) {
+    int64_t ldt, int C, int kk, int chan_outer) {
     __shared__ __align__(16) __nv_bfloat16 tile[TR_TILE][TR_TILE + 8];
     const int q0 = blockIdx.x * TR_TILE;
     const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TR_TILE;
@@ -70,7 +69,7 @@ static __global__ void __launch_bounds__(256) vlp_gather_transpose_kernel(
     for (int h = 0; h < 2; ++h) {
         const int r0 = 16 * mh + 8 * h;
         const int64_t m = m0 + r0;
-        if (m >= M && !kb64) break;        // blocked: the tile's zero tail is written too
+        if (m >= M) break;
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -78,9 +77,26 @@ static __global__ void __launch_bounds__(256) vlp_gather_transpose_kernel(
             const uint32_t hi = __bfloat16_as_ushort(tile[r0 + 2 * e + 1][qq]);
             w[e] = lo | (hi << 16);
         }
-        const int64_t off = kb64 ? ((m >> 6) * Q + orow) * 64 + (m & 63) : orow * ldt + m;
+        const int64_t off = orow * ldt + m;
         *reinterpret_cast<uint4*>(dst_t + off) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+}
+
+// dW1 from the kernel's K order back to the caller's: row n of src holds the columns
+// position-outer (p * C + c), row n of dst channel-outer (c * kk + p). One block per (row,
+// 64 channels): the kk runs of 64 are read coalesced, transposed in shared memory and
+// written as one run of 64 kk values.
+constexpr int UNPERM_MAX_KK = 9;
+static __global__ void __launch_bounds__(64) vlp_unpermute_cols_kernel(const float* __restrict__ src,
+                                                                       float* __restrict__ dst, int C, int kk) {
+    __shared__ float tile[64 * UNPERM_MAX_KK];
+    const int64_t K1 = static_cast<int64_t>(C) * kk;
+    const int64_t row = static_cast<int64_t>(blockIdx.y) * K1;
+    const int c0 = blockIdx.x * 64, t = threadIdx.x;
+    for (int pp = 0; pp < kk; ++pp) tile[t * kk + pp] = src[row + static_cast<int64_t>(pp) * C + c0 + t];
+    __syncthreads();
+    float* out = dst + row + static_cast<int64_t>(c0) * kk;
+    for (int i = t; i < 64 * kk; i += 64) out[i] = tile[i];
 }
 
 // Column sums of a row-major bf16 matrix [M][N] (N even), first pass: partial[b][n] is

@@ -424,7 +424,8 @@ void vlproj_destroy(vlproj_handle* h) {
     cudaFree(h->W2t);
     cudaFree(h->W1pt);
     for (auto* w : h->Wmt) cudaFree(w);
-    for (auto* b : {&h->G, &h->Hr, &h->dY, &h->dP, &h->At}) b->release();
+    for (auto* b : {&h->G, &h->Hr, &h->dY, &h->dP}) b->release();
+    h->dW1p.release();
     h->part_cs.release();
     h->dA.release();
     h->part.release();

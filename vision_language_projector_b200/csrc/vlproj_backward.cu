@@ -13,8 +13,8 @@
 //                                     down through the middle layers, with their weight
 //                                     gradients dW_mid = dP^T H (K = M)
 //   11  dW2 GEMM                      dW2 = dY^T H, K = M
-//   12  A^T + dW1 GEMM                A^T with rows in the caller's column order, then
-//                                     dW1 = dP^T A, K = M
+//   12  dW1 GEMM                      dW1 = dP^T A, K = M, then its columns put back in
+//                                     the caller's channel order
 //   13  dA GEMM                       dA = dP W1p [M][k*k*C] bf16 (without a LayerNorm
 //                                     folded straight onto the patches in fp32: d_features)
 //   14  tails                         LayerNorm backward -> d_features and gamma / beta
@@ -22,12 +22,12 @@
 //                                     separator gradients (db2, db1: column sums of dY and
 //                                     dP, beside stages 11 and 12)
 // Every contraction runs on the tcgen05 GEMM kernel with operands from tensor maps. The
-// weight gradients (K = M, the tokens) read dY, H and dP where they lie, row-major, as
-// MN-major operands; only A^T is copied, since dW1's columns come back in the caller's
-// channel order. The bias gradients are column sums of dY and dP over the tokens. W2^T
-// and W1p^T are made once, on the first call. For batches up to about 2^28 hidden activations, stages
-// 11-12 and the bias sums run on the handle's side stream, forked after stage 9 and
-// joined before the call returns.
+// weight gradients (K = M, the tokens) read dY, H, dP and A where they lie, row-major, as
+// MN-major operands; dW1's columns are then put back in the caller's order. The bias
+// gradients are column sums of dY and dP over the tokens. W2^T and W1p^T are made once,
+// on the first call. For batches up to about 2^28 hidden activations, stages 11-12 and
+// the bias sums run on the handle's side stream, forked after stage 9 and joined before
+// the call returns.
 #include "host.cuh"
 #include "kernels_bwd.cuh"
 
@@ -51,13 +51,6 @@ int encode_b_mn(CUtensorMap* full, CUtensorMap* half, const void* base, uint64_t
     return encode_bf16_mn(half, base, rows, cols, 2);
 }
 
-// The same for a B operand stored blocked by 64 columns (the transposed activations and
-// gradients, K = tokens): each K-block of the box's rows is one contiguous run.
-int encode_b_kb64(CUtensorMap* full, CUtensorMap* half, const void* base, uint64_t rows, uint64_t cols, int bn) {
-    if (encode_bf16_kb64(full, base, rows, cols, static_cast<uint32_t>(bn))) return VLPROJ_ERR_CUDA;
-    return encode_bf16_kb64(half, base, rows, cols, 128);
-}
-
 GemmParams gemm_params(const vlproj_handle* h, int64_t M, int N, int64_t K) {
     GemmParams p{};
     p.M = static_cast<int>(M);
@@ -74,12 +67,11 @@ GemmParams gemm_params(const vlproj_handle* h, int64_t M, int N, int64_t K) {
 
 void transpose_launch(const __nv_bfloat16* src, int64_t ld_src, int64_t src_rows, const int32_t* rowsel,
                       const int* zero_if, int64_t M, int Q, __nv_bfloat16* dst, __nv_bfloat16* dst_t, int64_t ldt,
-                      int C, int kk, int chan_outer, cudaStream_t s, int kb64 = 0) {
+                      int C, int kk, int chan_outer, cudaStream_t s) {
     dim3 grid(static_cast<unsigned>((Q + vlp::TR_TILE - 1) / vlp::TR_TILE),
               static_cast<unsigned>((M + vlp::TR_TILE - 1) / vlp::TR_TILE));
     vlp::vlp_gather_transpose_kernel<<<grid, 256, 0, s>>>(src, ld_src, src_rows, rowsel, zero_if,
-                                                          static_cast<int>(M), Q, dst, dst_t, ldt, C, kk, chan_outer,
-                                                          kb64);
+                                                          static_cast<int>(M), Q, dst, dst_t, ldt, C, kk, chan_outer);
 }
 
 // W2^T [N1][N2], W1p^T [K1][N1] and each middle layer's W^T [N1][N1], with their tensor
@@ -164,9 +156,6 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     const int kk = c.k * c.k;
     const int K1 = h->K1;
     const int64_t M = pl.M;          // no padding in this plan: M merged tokens
-    // tokens of A^T (blocked by 64 tokens, zeros past M): whole 128-byte lines, so every
-    // TMA box row of the dW1 GEMM starts on a line
-    const int64_t ldt = round_up(std::max<int64_t>(M, 1), 64);
     const size_t hslab = static_cast<size_t>(M) * c.N1;
     // bias gradients: column sums over the tokens, in blocks of CSR_ROWS rows
     const int64_t nb_cs = (M + vlp::CSR_ROWS - 1) / vlp::CSR_ROWS;
@@ -189,7 +178,7 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
             h->dY.ensure(static_cast<size_t>(M) * c.N2) || h->dP.ensure(hslab * 2) ||
             h->part_cs.ensure(static_cast<size_t>(nb_cs) * (c.N2 + 2 * c.N1)))
             return VLPROJ_ERR_CUDA;
-        if (a->d_W1 && h->At.ensure(static_cast<size_t>(K1) * ldt)) return VLPROJ_ERR_CUDA;
+        if (a->d_W1 && h->dW1p.ensure(static_cast<size_t>(c.N1) * K1)) return VLPROJ_ERR_CUDA;
         if (want_da && c.has_ln && h->dA.ensure(static_cast<size_t>(M) * K1)) return VLPROJ_ERR_CUDA;
         rc = ensure_transposed_weights(h, s);
         if (rc) return rc;
@@ -275,13 +264,13 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     stage_begin(h, 9, s);
     ++h->launches;
     transpose_launch(static_cast<const __nv_bfloat16*>(a->d_out), c.N2, n_ids, h->rowdest.ptr, h->status + 1, M,
-                     c.N2, h->dY.ptr, nullptr, ldt, c.C, 1, 0, s, 1);
+                     c.N2, h->dY.ptr, nullptr, 0, c.C, 1, 0, s);
     VLP_CUDA(cudaGetLastError());
     stage_end(h, 9, s);
 
     // Up to about 2^28 hidden activations (M * N1) the top and first layers' weight
     // gradients run on the side stream, beside the dP chain on the caller's stream: the
-    // top one and A^T need only stages 7-9, dW1 waits for dP_1, and each persistent GEMM
+    // top one needs only stages 7-9, dW1 waits for dP_1, and each persistent GEMM
     // takes the SMs the other leaves free, which fills their partial last waves (measured
     // 1.4-2 % faster on the MoonViT, DeepSeek-ViT and VL2 batches). Larger batches run in
     // sequence: there the two GEMM streams contend for L2 and power (measured 8 % slower
@@ -365,28 +354,28 @@ extern "C" int vlproj_backward(vlproj_handle* h, const vlproj_backward_args* a, 
     // dP_1, when the chain reached it (l_min == 1)
     const __nv_bfloat16* dP1 = h->dP.ptr + cur * hslab;
 
-    // 12a. A^T in the caller's column order (side stream)
-    if (a->d_W1) {
-        stage_begin(h, 12, ss);
-        ++h->launches;
-        transpose_launch(h->A.ptr, K1, M, nullptr, nullptr, M, K1, nullptr, h->At.ptr, ldt, c.C, kk,
-                         c.k_order == VLPROJ_ORDER_CHANNEL_OUTER ? 1 : 0, ss, 1);
-        VLP_CUDA(cudaGetLastError());
-    }
-
-    // 12b. dW1 = dP_1^T A and db1 (side stream, after dP_1)
+    // 12. dW1 = dP_1^T A and db1 (side stream, after dP_1): dP_1 and A read where they
+    //     lie (MN-major); dW1's columns come out in the kernel's position-outer K order and
+    //     go back to the caller's channel-outer order by one small pass
     if (want_l1) VLP_CUDA(cudaStreamWaitEvent(ss, h->join2, 0));
     if (a->d_W1) {
+        stage_begin(h, 12, ss);
+        const bool unpermute = c.k_order == VLPROJ_ORDER_CHANNEL_OUTER && kk > 1;
         if (encode_bf16_mn(&tmA2, dP1, M, c.N1, vlp::BM / 64) ||
-            encode_b_kb64(&tmB2, &tmB2h, h->At.ptr, K1, ldt, pick_bn(K1)))
+            encode_b_mn(&tmB2, &tmB2h, h->A.ptr, M, K1, pick_bn(K1)))
             return VLPROJ_ERR_CUDA;
         GemmParams q = gemm_params(h, c.N1, K1, M);
-        q.a_mn = 1;
-        q.b_kb64 = 1;
-        q.outf = a->d_W1;
+        q.a_mn = q.b_mn = 1;
+        q.outf = unpermute ? h->dW1p.ptr : a->d_W1;
         ++h->launches;
         rc = launch_gemm_bn<vlp::A_TILE, vlp::EPI_F32>(h, pick_bn(K1), h->pairs, tmA2, tmB2, tmB2h, q, ss);
         if (rc) return rc;
+        if (unpermute) {
+            ++h->launches;
+            vlp::vlp_unpermute_cols_kernel<<<dim3(static_cast<unsigned>(c.C / 64), static_cast<unsigned>(c.N1)), 64, 0,
+                                             ss>>>(h->dW1p.ptr, a->d_W1, c.C, kk);
+            VLP_CUDA(cudaGetLastError());
+        }
         stage_end(h, 12, ss);
     }
     if (a->d_b1) {
