@@ -91,12 +91,16 @@ SMALL = {
     "k3_no_ln": lambda: custom("k3_no_ln", 41, 3, 64, 192, 128, 2, 2, 200),
     "tiled_2x1": lambda: custom("tiled_2x1", 42, 2, 64, 128, 128, 2, 2, 260, tiled=True, tw=2, th=1),
     "fp32_no_ln": lambda: custom("fp32_no_ln", 43, 2, 64, 128, 96, 2, 1, 300, feat_fp32=True),
+    # regular grids (k | h, k | w), bf16, no LayerNorm, N2 not a multiple of 64: 5 images
+    # of 320 tokens, a ragged last tile
+    "regular_k3": lambda: custom("regular_k3", 44, 3, 64, 256, 160, 5, 5, 320),
 }
 GRIDS = {
     "ragged_ln_bf16": [[20, 30], [17, 9], [32, 32]],
     "k3_no_ln": [[10, 11], [7, 3]],
     "tiled_2x1": [[9, 9]] * 3 + [[7, 5]] * 3,
     "fp32_no_ln": [[15, 13], [4, 4]],
+    "regular_k3": [[30, 96]] * 5,
 }
 
 
@@ -131,9 +135,10 @@ def test_backward_position_outer_weights():
     assert_grads_close(got, oracle_grads(case, d_f64), "position-outer")
 
 
-def test_backward_is_deterministic_and_tile_shape_independent():
-    wl = SMALL["ragged_ln_bf16"]()
-    case = make_case(wl, GRIDS["ragged_ln_bf16"])
+@pytest.mark.parametrize("name", ["ragged_ln_bf16", "regular_k3"])
+def test_backward_is_deterministic_and_tile_shape_independent(name):
+    wl = SMALL[name]()
+    case = make_case(wl, GRIDS[name])
     proj = make_projector(case)
     dev = DeviceInputs(case)
     _, d_dev, _ = dev_dout(case)
