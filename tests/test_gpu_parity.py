@@ -44,6 +44,10 @@ SMALL = {
     # regular k = 3 grid with w' = 32: M = 800, a ragged last tile (the 5D box path)
     "regular_k3": (custom("regular_k3", 109, 3, 128, 256, 256, 5, 5, 256), [[15, 96]] * 5, "head",
                    vp.ORDER_CHANNEL_OUTER),
+    # same-shape odd grids (TMA im2col) with N1 = 1024: 256 x 512 pair tiles, M = 588 (a
+    # ragged third tile), two N-tiles
+    "wide_im2col": (custom("wide_im2col", 120, 2, 64, 1024, 256, 3, 3, 200), [[27, 27]] * 3, "head",
+                    vp.ORDER_CHANNEL_OUTER),
 }
 
 
@@ -74,7 +78,7 @@ def test_small_case_all_rows(name, mode):
 
 
 @pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
-@pytest.mark.parametrize("name", ["ragged_k3_ln", "tiled_head_odd", "fp32_noln", "many_images", "regular_k3"])
+@pytest.mark.parametrize("name", ["ragged_k3_ln", "tiled_head_odd", "fp32_noln", "many_images", "regular_k3", "wide_im2col"])
 def test_hidden_stage(name, mode):
     """Stage parity of H = bf16(GELU(A W1^T + b1)) for every merged token."""
     wl, hw, gvp, order = SMALL[name]

@@ -120,7 +120,10 @@ struct GemmLayout {
     static constexpr int RING_OFFSET = MISC_OFFSET + 16;          // tile indices of the dynamic order
     static constexpr int BYTES = RING_OFFSET + 4 * SCHED_SLOTS;
     static constexpr int SMEM_ALLOC = BYTES + 1024;      // room to align the base to 1024 B
-    static constexpr uint32_t TMEM_COLS = 2 * BN;        // two accumulators
+    // two accumulators (one tile's epilogue overlaps the next tile's MMAs), or one for
+    // 256 x 512 tiles, whose accumulator spans all 512 TMEM columns
+    static constexpr int NUM_ACC = 2 * BN <= 512 ? 2 : 1;
+    static constexpr uint32_t TMEM_COLS = NUM_ACC * BN;
 };
 
 // Statistics bytes per stage in A_TGATHER_LN: (mean, rstd) of each of the 128 rows.
@@ -353,7 +356,10 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     constexpr bool kLN = kAMode == A_TGATHER_LN;           // ... and normalise it in place
     constexpr bool kFused = kAMode == A_FUSED;             // warps 8-11 produce A, TMA tiles read it
     static_assert(!(kPair && kGatherThreads), "the 64-thread cp.async gather runs on single CTAs");
-    static_assert(!kPair || BN == 256, "CTA pairs run 256 x 256 tiles");
+    static_assert(!kPair || BN == 256 || BN == 512, "CTA pairs run 256 x 256 or 256 x 512 tiles");
+    static_assert(kPair || BN <= 256, "single CTAs run 128 x 128 or 128 x 256 tiles");
+    // 256 x 512 tiles (GEMM1 fed by TMA im2col): two N = 256 MMAs per K step share the A
+    // stage, so each im2col load feeds twice the FLOPs; each CTA stages 2 x 128 B rows
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
@@ -507,8 +513,15 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                                                         ch[q].w, static_cast<uint16_t>(dx), static_cast<uint16_t>(dy));
                             }
                         }
-                        if (p.b_mn) tma_load_3d_pair(sb, &tmB, bar, 0, kb * BK, b_row / 64);
-                        else tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
+                        if constexpr (BN == 512) {
+                            // this CTA's 128 rows of each 256-column half of the tile
+                            tma_load_2d_pair(sb, &tmB, bar, kb * BK, n_blk * BN + static_cast<int>(rank) * 128);
+                            tma_load_2d_pair(sb + 128 * 128, &tmB, bar, kb * BK, n_blk * BN + 256 + static_cast<int>(rank) * 128);
+                        } else if (p.b_mn) {
+                            tma_load_3d_pair(sb, &tmB, bar, 0, kb * BK, b_row / 64);
+                        } else {
+                            tma_load_2d_pair(sb, &tmB, bar, kb * BK, b_row);
+                        }
                     } else {
                         mbar_arrive_expect_tx(&full_tma[stage], expect);
                         if (kAMode == A_TILE || kFused) {
@@ -570,7 +583,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (the pair leader's lane 0)
         if (lane == 0 && leader) {
-            const uint32_t idesc = idesc_bf16_f32(BM * kCtas, BN) | (p.a_mn ? IDESC_A_MN : 0u) |
+            constexpr int MMA_N = BN > 256 ? 256 : BN;           // N of one MMA instruction
+            const uint32_t idesc = idesc_bf16_f32(BM * kCtas, MMA_N) | (p.a_mn ? IDESC_A_MN : 0u) |
                                    (p.b_mn ? IDESC_B_MN : 0u);
             // a 16-deep K slice: 32 bytes further along a K-major row, 2 KB (two 8-row
             // atoms) further down an MN-major strip
@@ -604,10 +618,13 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                         // the start address (16-byte units) is the descriptor's low field
                         const uint64_t dak = da + static_cast<uint64_t>((kk * a_step) >> 4);
                         const uint64_t dbk = db + static_cast<uint64_t>((kk * b_step) >> 4);
-                        if constexpr (kPair)
+                        if constexpr (kPair) {
                             tc_mma_f16_pair(d_tmem, dak, dbk, idesc, (kb | kk) != 0);
-                        else
+                            if constexpr (BN == 512)          // second half: B rows 16 KB on, columns 256 on
+                                tc_mma_f16_pair(d_tmem + 256, dak, dbk + ((128 * 128) >> 4), idesc, (kb | kk) != 0);
+                        } else {
                             tc_mma_f16(d_tmem, dak, dbk, idesc, (kb | kk) != 0);
+                        }
                     }
                     if constexpr (kPair) tc_commit_pair(&empty[stage], 0x3);
                     else tc_commit(&empty[stage]);
@@ -616,7 +633,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                 if (!ok) break;
                 if constexpr (kPair) tc_commit_pair(&tmem_full[acc], 0x3);
                 else tc_commit(&tmem_full[acc]);
-                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+                if (++acc == L::NUM_ACC) { acc = 0; acc_phase ^= 1; }
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -1111,7 +1128,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                 if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&tmem_empty[acc]), 0));
                 else mbar_arrive(&tmem_empty[acc]);
             }
-            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            if (++acc == L::NUM_ACC) { acc = 0; acc_phase ^= 1; }
         }
         if (!ok) {
             *abort_flag = 1;

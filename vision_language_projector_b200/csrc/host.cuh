@@ -533,7 +533,7 @@ int launch_gemm_bn(vlproj_handle* h, int bn, bool pair, const CUtensorMap& ta, c
                    const CUtensorMap& tb_half, GemmParams p, cudaStream_t s, const CUtensorMap& tc = no_map(),
                    const CUtensorMap& tc2 = no_map()) {
     const int num_sms = h->num_sms;
-    const int ctas = (A != vlp::A_CPASYNC && pair && bn == 256) ? 2 : 1;
+    const int ctas = (A != vlp::A_CPASYNC && pair && bn >= 256) ? 2 : 1;
     const int64_t tiles = ((static_cast<int64_t>(p.M) + vlp::BM * ctas - 1) / (vlp::BM * ctas)) * ((p.N + bn - 1) / bn);
     const int64_t kblocks = (static_cast<int64_t>(p.K) + vlp::BK - 1) / vlp::BK;
     const bool dyn = h->tile_order == VLPROJ_TILE_ORDER_DYNAMIC ||
@@ -541,10 +541,13 @@ int launch_gemm_bn(vlproj_handle* h, int bn, bool pair, const CUtensorMap& ta, c
                       (A != vlp::A_TILE ||
                        tiles * kblocks >= static_cast<int64_t>(kDynamicMinWaves) * 64 * (num_sms / ctas)));
     p.tile_queue = (dyn && h->tqueue) ? h->tqueue + 2 * (h->tq_next++ % kTileQueues) : nullptr;
-    if constexpr (A != vlp::A_CPASYNC) {
-        if (pair && bn == 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tc2, p, num_sms, s);
+    if constexpr (A == vlp::A_IM2COL && E == vlp::EPI_GELU) {
+        if (pair && bn == 512) return launch_gemm<512, A, E, 2>(ta, tb_half, tc, tc2, p, num_sms, s);
     }
-    if (bn == 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tc2, p, num_sms, s);
+    if constexpr (A != vlp::A_CPASYNC) {
+        if (pair && bn >= 256) return launch_gemm<256, A, E, 2>(ta, tb_half, tc, tc2, p, num_sms, s);
+    }
+    if (bn >= 256) return launch_gemm<256, A, E, 1>(ta, tb, tc, tc2, p, num_sms, s);
     return launch_gemm<128, A, E, 1>(ta, tb, tc, tc2, p, num_sms, s);
 }
 

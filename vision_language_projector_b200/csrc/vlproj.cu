@@ -195,9 +195,9 @@ int run_merge_gemm1(vlproj_handle* h, const Plan& pl, const void* features, cons
     else if (pl.box5)
         rc = launch_gemm_bn<vlp::A_BOX5, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
                                                         s, tmC);
-    else if (im2col)
-        rc = launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(h, pick_bn(c.N1), h->pairs, tmA, h->tmW1, h->tmW1h, p,
-                                                          s, tmC);
+    else if (im2col)      // 256 x 512 pair tiles where N1 allows: each im2col load feeds two MMAs
+        rc = launch_gemm_bn<vlp::A_IM2COL, vlp::EPI_GELU>(h, c.N1 % 512 == 0 ? 512 : pick_bn(c.N1), h->pairs, tmA,
+                                                          h->tmW1, h->tmW1h, p, s, tmC);
     else
         rc = launch_gemm_bn<vlp::A_CPASYNC, vlp::EPI_GELU>(h, pick_bn(c.N1), false, tmA, h->tmW1, h->tmW1h, p,
                                                            s, tmC);
