@@ -129,8 +129,11 @@ struct GemmLayout {
 // Statistics bytes per stage in A_TGATHER_LN: (mean, rstd) of each of the 128 rows.
 __host__ __device__ constexpr int a_aux_bytes(int amode) { return amode == A_TGATHER_LN ? BM * 8 : 0; }
 __host__ __device__ constexpr bool a_thread_gather(int amode) { return amode == A_TGATHER || amode == A_TGATHER_LN; }
-__host__ __device__ constexpr int gemm_threads(int amode) {
-    return (a_thread_gather(amode) || amode == A_FUSED) ? GEMM_THREADS_TG : GEMM_THREADS;
+// Epilogue warp groups: 256 x 512 tiles drain their one accumulator with two groups of
+// four warps (columns 0-255 and 256-511), since no other tile's MMAs hide that drain.
+__host__ __device__ constexpr int epi_groups(int bn) { return bn == 512 ? 2 : 1; }
+__host__ __device__ constexpr int gemm_threads(int amode, int bn = 256) {
+    return (a_thread_gather(amode) || amode == A_FUSED || epi_groups(bn) == 2) ? GEMM_THREADS_TG : GEMM_THREADS;
 }
 constexpr int FUSED_BLOCK = 256;        // A_FUSED readiness granularity: rows per block (one pair tile)
 
@@ -344,11 +347,12 @@ __device__ __forceinline__ void write_row_block(const uint32_t (&packed)[16], ui
 }
 
 template <int BN, int kAMode, int kEpi, int kCtas>
-__global__ void __launch_bounds__(gemm_threads(kAMode), 1)
+__global__ void __launch_bounds__(gemm_threads(kAMode, BN), 1)
     vlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                     const GemmParams p) {
-    using L = GemmLayout<BN, kCtas, epi_stage_bytes(kEpi), a_aux_bytes(kAMode)>;
+    using L = GemmLayout<BN, kCtas, epi_stage_bytes(kEpi) * epi_groups(BN), a_aux_bytes(kAMode)>;
+    constexpr int kEpiGroups = epi_groups(BN);
     constexpr int S = L::STAGES;
     constexpr bool kPair = kCtas == 2;
     constexpr bool kGatherThreads = kAMode == A_CPASYNC;
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     // readers of each ring slot: the second CTA's TMA producer, the MMA issuer, the relay
     // threads, the cp.async gather warps, the thread-gather warps, the epilogue warps
     constexpr uint32_t sched_readers = (kPair ? 1 : 0) + 1 + ((kTG && !kLN) ? kCtas : 0) + (kGatherThreads ? 2 : 0) +
-                                       (kTG ? 4 * kCtas : 0) + 4 * kCtas;
+                                       (kTG ? 4 * kCtas : 0) + 4 * kEpiGroups * kCtas;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFFSET);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFFSET + 4);
 
@@ -397,7 +401,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tmem_full[a], 1);
-            mbar_init(&tmem_empty[a], 4 * kCtas);               // every epilogue warp of the pair
+            mbar_init(&tmem_empty[a], 4 * kEpiGroups * kCtas);  // every epilogue warp of the pair
         }
         mbar_init(drain, 1);
         for (int j = 0; j < SCHED_SLOTS; ++j) {
@@ -878,7 +882,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
             }
             cp_async_wait_all();
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 8 && kEpiGroups == 1) {
         // ------------------------------------------------ A producers (A_FUSED, warps 8-11)
         // Each warp takes two items at a time from the kernel-wide counter, in (256-row
         // block, tap, row) order, so the blocks become ready in the order the tiles need
@@ -942,7 +946,8 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
     } else {
         // ------------------------------------------------ epilogue (warps 4..7 of each CTA)
         const int ew = warp & 3;                      // TMEM lanes 32*ew .. 32*ew+31
-        uint8_t* ebuf = smem + L::EPI_OFFSET + ew * epi_blocks(kEpi) * EPI_BLOCK_BYTES;   // this warp's blocks
+        const int eg = kEpiGroups == 2 ? (warp >> 3) : 0;   // column group (warps 8-11: the second)
+        uint8_t* ebuf = smem + L::EPI_OFFSET + (eg * 4 + ew) * epi_blocks(kEpi) * EPI_BLOCK_BYTES;   // this warp's blocks
         int ehalf = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -976,8 +981,9 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                 if (row_ok) fold = __ldg(&p.gmeta[m]);
             }
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(acc * BN);
+            constexpr int kChunks = BN / 32 / kEpiGroups;      // this warp's 32-column chunks
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = eg * kChunks; c < (eg + 1) * kChunks; ++c) {
                 const int n0 = n_blk * BN + c * 32;
                 if (n0 >= p.N) break;                  // uniform across the warp
                 uint32_t v[32];
@@ -1068,7 +1074,7 @@ __global__ void __launch_bounds__(gemm_threads(kAMode), 1)
                         *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
                             make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
                     }
-                    if (half == 1 || c + 1 == BN / 32 || n0 + 32 >= p.N) {
+                    if (half == 1 || c + 1 == (eg + 1) * kChunks || n0 + 32 >= p.N) {
                         __syncwarp();
                         const int nb = n0 - half * 32;               // first column of the block
                         const int q = lane & 7;

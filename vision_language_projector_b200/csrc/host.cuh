@@ -399,13 +399,13 @@ inline int raster_group(int N, int K, int BN, int64_t budget = 0, int units = 74
 template <int BN, int A, int E, int CTAS>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tc2,
                 GemmParams p, int num_sms, cudaStream_t s) {
-    using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E), vlp::a_aux_bytes(A)>;
+    using L = GemmLayout<BN, CTAS, vlp::epi_stage_bytes(E) * vlp::epi_groups(BN), vlp::a_aux_bytes(A)>;
     auto kernel = vlp::vlp_gemm_kernel<BN, A, E, CTAS>;
     if (p.group_n <= 0) p.group_n = raster_group(p.N, p.K, BN, p.l2_budget, num_sms / CTAS);
     VLP_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC));
     const int tiles = ((p.M + vlp::BM * CTAS - 1) / (vlp::BM * CTAS)) * ((p.N + BN - 1) / BN);
     cudaLaunchConfig_t cfg{};
-    cfg.blockDim = dim3(vlp::gemm_threads(A));
+    cfg.blockDim = dim3(vlp::gemm_threads(A, BN));
     cfg.dynamicSmemBytes = L::SMEM_ALLOC;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
