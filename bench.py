@@ -100,11 +100,25 @@ def peak_clock_mhz(peaks: dict, sustained: bool):
     return None
 
 
+def code_only(text: str) -> str:
+    """The source without // comments, trailing blanks and empty lines: an edit of the
+    comments alone keeps the stored DRAM counters valid."""
+    out = []
+    for line in text.splitlines():
+        i = line.find("//")
+        if i >= 0 and line.count('"', 0, i) % 2 == 0:
+            line = line[:i]
+        line = line.rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

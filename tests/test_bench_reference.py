@@ -51,3 +51,16 @@ def test_images_override_scales_the_sequences():
     wl = bench.pick_workload(argparse.Namespace(workload="moonvit", images=4))
     assert (wl.n_images, wl.B) == (4, 4)
     assert bench.pick_workload(argparse.Namespace(workload="vl2", images=0)) is W.WORKLOADS["vl2"]
+
+
+def test_code_only_ignores_comments_and_blank_lines():
+    """The stored DRAM counters stay keyed to the kernels' code: comment edits keep the
+    key, code edits change it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int x = 1;  // one\n\n// a note\nint y = 2;\n"
+    b = "int x = 1;  // the first\n// another note\nint y = 2;   \n\n"
+    c = "int x = 1;\nint y = 3;\n"
+    assert bench.code_only(a) == bench.code_only(b) == "int x = 1;\nint y = 2;"
+    assert bench.code_only(c) != bench.code_only(a)
+    assert bench.code_only('printf("//");') == 'printf("//");'

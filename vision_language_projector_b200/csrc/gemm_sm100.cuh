@@ -17,27 +17,29 @@
 //       out[dest[m], n] = bf16( sum_q H[m, q] W2[n, q] + b2[n] )
 //       the epilogue writes each row straight into its placeholder row.
 //   Backward epilogues (A_TILE, no scatter):
-//       EPI_BWD_H   P = acc + b1: G = bf16(GELU'(P)) row-major and H^T = bf16(GELU(P))
-//                   transposed, so H^T can be a K-major operand of the W2 gradient
-//       EPI_DGELU   dP = bf16(acc * G), row-major and transposed (dP^T)
-//   bf16 outputs with plain rows (GEMM1's H, the backward's G, H^T, dP, dP^T) leave the
-//   epilogue as 32 x 32 blocks through shared memory and TMA tile stores.
+//       EPI_BWD_H   P = acc + b1: G = bf16(GELU'(P)) and H = bf16(GELU(P)), row-major
+//       EPI_DGELU   dP = bf16(acc * G), row-major
+//   The weight gradients (K = tokens) read dY, H, dP and A row-major as MN-major operands.
+//   bf16 outputs with plain rows (GEMM1's H, the backward's G, H, dP) leave the epilogue
+//   as 32 x 32 blocks through shared memory and TMA tile stores.
 //       EPI_F32     acc as fp32, row-major (weight and input gradients)
 //       EPI_BF16    acc as bf16 through TMA stores (the LayerNorm backward's dA)
 //       EPI_FOLD_F32  acc as fp32, folded back onto the patches: column p*C + c of
 //                   merged token m goes to channel c of the patch at position p of its
 //                   k x k neighbourhood (gmeta), so dA never goes to memory
 //
-// One persistent CTA per SM walks output tiles of BM x BN in banded order (see
-// tile_coords: the CTAs running together share A tiles and an L2-sized band of B).
-// Roles, by warp:
+// One persistent CTA (or CTA pair) per SM (pair of SMs) walks output tiles in banded
+// order (see tile_coords: the CTAs running together share A tiles and an L2-sized band
+// of B), statically or from a device counter (TileSeq). Roles, by warp:
 //   warp 0      TMA producer (B; A in the TMA modes)
 //   warp 1      TMEM allocator and the single MMA-issuing thread
 //   warps 2-3   A gather producers in A_CPASYNC mode (64 threads)
 //   warps 4-7   epilogue: TMEM -> registers -> bias (+GELU) -> bf16 -> global
+//   warps 8-11  thread-gather / fused-producer modes, or the second epilogue group of
+//               256 x 512 tiles
 // Shared memory holds a STAGES-deep ring of (A, B) K-blocks of 64 bf16 (128 B
-// rows, 128-byte swizzle); TMEM holds two BM x BN fp32 accumulators so the
-// epilogue of one tile overlaps the MMAs of the next.
+// rows, 128-byte swizzle); TMEM holds two accumulators so the epilogue of one tile
+// overlaps the MMAs of the next (one, over all 512 columns, for 256 x 512 tiles).
 //
 // Every wait is bounded (GemmParams::wait_ns). When one runs out, the kernel
 // latches VLPROJ_ERR_TIMEOUT, every role unwinds, outstanding copies and MMAs
