@@ -122,6 +122,8 @@ struct GemmLayout {
     static constexpr int RING_OFFSET = MISC_OFFSET + 16;          // tile indices of the dynamic order
     static constexpr int BYTES = RING_OFFSET + 4 * SCHED_SLOTS;
     static constexpr int SMEM_ALLOC = BYTES + 1024;      // room to align the base to 1024 B
+    static_assert(SMEM_ALLOC <= 232448, "a CTA may use at most 227 KB of shared memory");
+    static_assert(STAGES >= 2, "at least two stages in the ring");
     // two accumulators (one tile's epilogue overlaps the next tile's MMAs), or one for
     // 256 x 512 tiles, whose accumulator spans all 512 TMEM columns
     static constexpr int NUM_ACC = 2 * BN <= 512 ? 2 : 1;
